@@ -1,0 +1,140 @@
+"""Seeded synthetic Q/K/V for the S2O prefill path.
+
+This module is the only code shared by the CPU oracle's tests and the CUDA path's tests and
+benchmark: it produces input bytes and nothing else (none of the method's arithmetic lives here).
+
+The pages evaluate on Llama-3.1-8B / Qwen3-8B activations over long-context datasets that are not
+available; these inputs stand in for them with the same attention shapes (32 query heads, 8 KV
+heads, d = 128) and with the stripe patterns the S2O card's Summary says real attention maps are
+made of (vertical stripes on a few key positions, a diagonal).
+
+Recipe (each (tensor, batch, head) slab has its own counter-free numpy stream, so the bytes do not
+depend on how many threads draw them):
+
+1. Q, K, V ~ N(0, 1) float32; slab (t, beta, head) drawn from
+   ``Generator(PCG64(SeedSequence(seed, spawn_key=(t, beta, head))))`` with t = 0, 1, 2 for Q, K, V.
+2. For each (beta, g): from ``SeedSequence(seed, spawn_key=(3, beta, g))`` draw a direction
+   u_g ~ N(0, I_d) (float64, then normalised) and ``round(stripe_frac * N)`` distinct key positions
+   (or ``stripe_count`` when given); those keys get ``+ amp * u_g`` and every query of the heads of
+   group g gets ``+ q_shift * u_g``.
+3. If ``diag`` is non-zero: ``q[h, i] += diag * k[g(h), i]`` using the final K (the literal
+   diagonal reading of "diagonal band for local window 512").
+4. Round to bf16, nearest-even.
+"""
+from __future__ import annotations
+
+import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "workload"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    seq_len: int
+    head_dim: int
+    segment_len: int
+    block_size: int
+    tau: float
+    seed: int
+    amp: float = 4.0
+    stripe_frac: float = 0.01
+    stripe_count: int | None = None
+    q_shift: float = 1.0
+    diag: float = 0.5
+    query_perm: int = 1
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+    @property
+    def dense_causal_flops(self) -> float:
+        """4·d·N(N+1)/2 per query head: QKᵀ and PV over the causal triangle."""
+        n = self.seq_len
+        return 4.0 * self.head_dim * n * (n + 1) / 2 * self.n_q_heads * self.batch
+
+
+WORKLOADS = {
+    # 1 head, d = 64, N = 1024; 8 planted stripe keys at amplitude 3, all queries +1·u.
+    "tiny": Workload("tiny", 1, 1, 1, 1024, 64, 256, 64, 0.01, 0, amp=3.0,
+                     stripe_count=8, diag=0.0),
+    "llama-32k": Workload("llama-32k", 1, 32, 8, 32768, 128, 2048, 128, 0.01, 1),
+    "llama-128k": Workload("llama-128k", 1, 32, 8, 131072, 128, 2048, 128, 0.01, 2),
+    "qwen-128k": Workload("qwen-128k", 1, 32, 8, 131072, 128, 2048, 128, 0.01, 3),
+}
+
+
+def workload(name: str, **overrides) -> Workload:
+    w = WORKLOADS[name]
+    return w.replace(**overrides) if overrides else w
+
+
+def layer_workload(layer: int) -> Workload:
+    """Layer l of the 32-layer stack: stripe density 0.5 % + 2.5 %·l/31, seed 1000 + l."""
+    frac = 0.005 + 0.025 * layer / 31.0
+    return WORKLOADS["llama-128k"].replace(name=f"stack-layer{layer}", stripe_frac=frac,
+                                           seed=1000 + layer)
+
+
+def _stream(seed: int, *key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=key)))
+
+
+def make_inputs(w: Workload, threads: int | None = None, keep_fp32: bool = False):
+    """Return ``(q, k, v)`` as contiguous CPU bf16 tensors in BHND layout.
+
+    With ``keep_fp32`` also returns the float32 arrays before rounding (used by the tiny case's
+    own Eq. 1 check).
+    """
+    B, Hq, Hkv, N, d = w.batch, w.n_q_heads, w.n_kv_heads, w.seq_len, w.head_dim
+    G = Hq // Hkv
+    threads = threads or min(32, os.cpu_count() or 1)
+    q = np.empty((B, Hq, N, d), np.float32)
+    k = np.empty((B, Hkv, N, d), np.float32)
+    v = np.empty((B, Hkv, N, d), np.float32)
+
+    jobs = [(0, b, h) for b in range(B) for h in range(Hq)]
+    jobs += [(t, b, h) for t in (1, 2) for b in range(B) for h in range(Hkv)]
+    dst = {0: q, 1: k, 2: v}
+
+    def fill(job):
+        t, b, h = job
+        dst[t][b, h] = _stream(w.seed, t, b, h).standard_normal((N, d), dtype=np.float32)
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(fill, jobs))
+
+    n_stripe = w.stripe_count if w.stripe_count is not None else int(round(w.stripe_frac * N))
+    for b in range(B):
+        for g in range(Hkv):
+            rng = _stream(w.seed, 3, b, g)
+            u = rng.standard_normal(d)
+            u = (u / np.linalg.norm(u)).astype(np.float32)
+            pos = rng.choice(N, size=n_stripe, replace=False)
+            k[b, g, pos, :] += np.float32(w.amp) * u
+            q[b, g * G:(g + 1) * G] += np.float32(w.q_shift) * u
+
+    if w.diag:
+        def diag(job):
+            b, h = job
+            q[b, h] += np.float32(w.diag) * k[b, h // G]
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(diag, [(b, h) for b in range(B) for h in range(Hq)]))
+
+    out = tuple(torch.from_numpy(x).to(torch.bfloat16).contiguous() for x in (q, k, v))
+    if keep_fp32:
+        return out + ((q, k, v),)
+    return out
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """The raw bf16 bit patterns of a CPU bf16 tensor as a uint16 numpy array (no copy)."""
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)

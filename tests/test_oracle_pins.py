@@ -1,0 +1,330 @@
+"""Pins for the CPU oracle: what the pages and the mathematics fix, checked on the CPU.
+
+Each test ties the oracle to something other than itself: a hand-worked case, a library routine
+that the method reduces to in a special case (torch's causal scaled-dot-product attention at
+τ = 0, per-segment causal attention at τ > 1), invariants the pages state (tensors are never moved,
+so permutations leave the output unchanged; blocks are visited in importance order and the loop
+stops at τ, so the selected sets are nested), libm for exp64, and float64 re-derivations of every
+pooled quantity. A dropped term, a wrong sign or index, or a transposed operand anywhere in the
+oracle fails at least one of them.
+"""
+import json
+import math
+import os
+from decimal import Decimal, getcontext
+
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_case.json")
+
+SMALL_GQA = gen.Workload("small-gqa", batch=2, n_q_heads=4, n_kv_heads=2, seq_len=512,
+                         head_dim=64, segment_len=128, block_size=64, tau=0.05, seed=7,
+                         amp=4.0, stripe_count=12, diag=0.5)
+
+
+def _hand():
+    with open(GOLDEN) as f:
+        g = json.load(f)
+    c = g["config"]
+    q = torch.tensor(g["q"], dtype=torch.bfloat16).reshape(1, 1, 8, 4)
+    k = torch.tensor(g["k"], dtype=torch.bfloat16).reshape(1, 1, 8, 4)
+    v = torch.arange(32, dtype=torch.float32).reshape(1, 1, 8, 4).to(torch.bfloat16)
+    return g, c, q, k, v
+
+
+def _cfg(c, tau, query_perm=1):
+    return oracle.Config(c["batch"], c["n_q_heads"], c["n_kv_heads"], c["seq_len"],
+                         c["head_dim"], c["segment_len"], c["block_size"], tau, query_perm)
+
+
+def _sdpa_causal(q, k, v, G):
+    """torch's causal SDPA in float64 (K/V heads shared by G query heads)."""
+    q64, k64, v64 = (x.to(torch.float64) for x in (q, k, v))
+    k64 = k64.repeat_interleave(G, dim=1)
+    v64 = v64.repeat_interleave(G, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(q64, k64, v64, is_causal=True)
+
+
+def _sdpa_segment_local(q, k, v, G, S):
+    outs = []
+    for s0 in range(0, q.shape[2], S):
+        sl = slice(s0, s0 + S)
+        outs.append(_sdpa_causal(q[:, :, sl], k[:, :, sl], v[:, :, sl], G))
+    return torch.cat(outs, dim=2)
+
+
+# ----------------------------------------------------------------------------- hand case
+
+def test_hand_case_intermediates():
+    g, c, q, k, _ = _hand()
+    idx = oracle.build_indices(_cfg(c, 0.3), q, k, debug=True)
+    for name in ("qbar", "kbar_all", "kappa", "kbar_top", "u", "rho", "Qbar", "Kbar", "r"):
+        np.testing.assert_array_equal(idx[name].reshape(-1), np.asarray(g[name], np.float32)
+                                      .reshape(-1), err_msg=name)
+    np.testing.assert_array_equal(idx["perm_k"][0, 0], g["perm_k"])
+    np.testing.assert_array_equal(idx["perm_q"][0, 0], g["perm_q"])
+    np.testing.assert_array_equal(idx["n"][0, 0], g["n"])
+    np.testing.assert_array_equal(idx["local_tiles"][0, 0], g["local_tiles"])
+
+
+def test_hand_case_probabilities_closed_form():
+    g, c, q, k, _ = _hand()
+    p = oracle.build_indices(_cfg(c, 0.3), q, k, debug=True)["p"][0, 0]
+    z2 = 1 + math.exp(-0.25) + 2 * math.exp(-0.625)
+    z3 = 2 + 2 * math.exp(-0.25)
+    want = np.array([[0, 0, 0, 0], [0, 0, 0, 0],
+                     [1 / z2, math.exp(-0.25) / z2, 2 * math.exp(-0.625) / z2, 0],
+                     [1 / z3, 1 / z3, 2 * math.exp(-0.25) / z3, 0]])
+    np.testing.assert_allclose(p, want, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("tau", ["0.0", "0.28", "0.3", "0.4", "0.5"])
+def test_hand_case_selection_and_pairs(tau):
+    g, c, q, k, v = _hand()
+    cfg = _cfg(c, float(tau))
+    idx = oracle.build_indices(cfg, q, k)
+    want = g["selection"][tau]
+    for b, sel in enumerate(want["sel"]):
+        assert idx["sel_cnt"][0, 0, b] == len(sel)
+        np.testing.assert_array_equal(idx["sel_blk"][0, 0, b, :len(sel)], sel)
+        assert (idx["sel_blk"][0, 0, b, len(sel):] == -1).all()
+    assert oracle.pair_count(cfg, idx) == want["pairs"]
+    _, pairs = oracle.attention(cfg, q, k, v, idx)
+    assert pairs == want["pairs"]
+
+
+def test_hand_case_key_sets():
+    """At τ = 0.3 row i attends exactly to the hand-derived key set: compare with SDPA over it."""
+    g, c, q, k, v = _hand()
+    cfg = _cfg(c, 0.3)
+    idx = oracle.build_indices(cfg, q, k)
+    rows = np.array([4, 5, 6, 7])
+    out, _ = oracle.attention(cfg, q, k, v, idx, rows=rows)
+    for x, i in enumerate(rows):
+        keys = g["key_sets_tau_0.3"][str(i)]
+        mask = torch.zeros(1, 8, dtype=torch.bool)
+        mask[0, keys] = True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[0, 0, i:i + 1].double(), k[0, 0].double(), v[0, 0].double(), attn_mask=mask)
+        np.testing.assert_allclose(out[x], ref[0].numpy(), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- exp64 / constants
+
+def test_exp64_constants_from_high_precision():
+    getcontext().prec = 60
+    ln2 = Decimal(2).ln()
+    inv = 1 / ln2
+
+    def nearest(x):
+        return float(x)  # Decimal -> float is correctly rounded
+
+    assert nearest(inv).hex() == "0x1.71547652b82fep+0"
+    hi = nearest(ln2)
+    assert hi.hex() == "0x1.62e42fefa39efp-1"
+    assert nearest(ln2 - Decimal(hi)).hex() == "0x1.abc9e3b39803fp-56"
+
+
+def test_score_scale_constants():
+    getcontext().prec = 60
+    for d, want in ((64, "0x1.0000000000000p-3"), (128, "0x1.6a09e60000000p-4")):
+        exact = 1 / Decimal(d).sqrt()
+        f32 = np.float32(float(exact))  # float(Decimal) then float32: double rounding is safe here
+        assert float(f32).hex() == want
+        assert float(np.float32(oracle.score_scale(d))).hex() == want
+        # nearest-to-exact check without double rounding: neighbours are farther away
+        lo, hi = np.nextafter(f32, np.float32(0)), np.nextafter(f32, np.float32(1))
+        err = abs(Decimal(float(f32)) - exact)
+        assert err <= abs(Decimal(float(lo)) - exact) and err <= abs(Decimal(float(hi)) - exact)
+
+
+def test_exp64_within_two_ulp_of_libm():
+    xs = np.concatenate([-np.linspace(0, 700, 20001), -np.geomspace(1e-300, 1, 2001),
+                         [-0.0, -0.5 * math.log(2), -math.log(2), -699.999]])
+    worst = 0.0
+    for x in xs:
+        got, ref = oracle.exp64(float(x)), math.exp(float(x))
+        worst = max(worst, abs(got - ref) / math.ulp(ref))
+    assert worst <= 2.0, worst
+    assert oracle.exp64(-700.5) == 0.0
+    assert oracle.exp64(0.0) == 1.0
+
+
+# ----------------------------------------------------------------------------- special cases
+
+@pytest.mark.parametrize("w", [gen.workload("tiny"), SMALL_GQA], ids=["tiny", "small-gqa"])
+def test_tau_zero_is_dense_causal_attention(w):
+    """τ = 0 keeps every candidate block, so the key set is [0, i]: Eq. 1 exactly."""
+    q, k, v = gen.make_inputs(w)
+    cfg = oracle.config(w, tau=0.0)
+    idx = oracle.build_indices(cfg, q, k)
+    out, pairs = oracle.attention(cfg, q, k, v, idx)
+    ref = _sdpa_causal(q, k, v, w.n_q_heads // w.n_kv_heads).reshape(-1, w.head_dim)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-10)
+    N = w.seq_len
+    assert pairs == w.batch * w.n_q_heads * N * (N + 1) // 2
+    np.testing.assert_allclose(oracle.dense_causal(cfg, q, k, v), ref.numpy(), rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("w", [gen.workload("tiny"), SMALL_GQA], ids=["tiny", "small-gqa"])
+def test_tau_above_one_is_local_window_only(w):
+    """τ > 1 selects nothing: each query sees only its own segment causally."""
+    q, k, v = gen.make_inputs(w)
+    cfg = oracle.config(w, tau=1.5)
+    idx = oracle.build_indices(cfg, q, k)
+    assert (idx["sel_cnt"] == 0).all()
+    out, _ = oracle.attention(cfg, q, k, v, idx)
+    ref = _sdpa_segment_local(q, k, v, w.n_q_heads // w.n_kv_heads, w.segment_len)
+    np.testing.assert_allclose(out, ref.reshape(-1, w.head_dim).numpy(), rtol=0, atol=1e-10)
+
+
+def test_permutation_invariance_with_full_selection():
+    """Arbitrary key and segment-local query orderings with every block selected give Eq. 1:
+    the orderings only relabel addresses, the tensors are never moved."""
+    w = SMALL_GQA
+    q, k, v = gen.make_inputs(w)
+    cfg = oracle.config(w)
+    rng = np.random.default_rng(11)
+    B, Hq, N = w.batch, w.n_q_heads, w.seq_len
+    nB, S = N // w.block_size, w.segment_len
+    perm_k = np.stack([np.stack([rng.permutation(N) for _ in range(Hq)]) for _ in range(B)])
+    perm_q = np.empty_like(perm_k)
+    for b in range(B):
+        for h in range(Hq):
+            for s0 in range(0, N, S):
+                perm_q[b, h, s0:s0 + S] = s0 + rng.permutation(S)
+    sel_blk = np.broadcast_to(rng.permutation(nB).astype(np.int32), (B, Hq, nB, nB)).copy()
+    idx = dict(perm_q=perm_q.astype(np.int32), perm_k=perm_k.astype(np.int32),
+               sel_cnt=np.full((B, Hq, nB), nB, np.int32), sel_blk=sel_blk)
+    out, _ = oracle.attention(cfg, q, k, v, idx)
+    ref = _sdpa_causal(q, k, v, w.n_q_heads // w.n_kv_heads).reshape(-1, w.head_dim)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-10)
+
+
+def test_segment_zero_is_dense_for_any_tau():
+    w = SMALL_GQA
+    q, k, v = gen.make_inputs(w)
+    ref = _sdpa_causal(q, k, v, w.n_q_heads // w.n_kv_heads)
+    S = w.segment_len
+    for tau in (0.0, 0.05, 0.5, 2.0):
+        cfg = oracle.config(w, tau=tau)
+        idx = oracle.build_indices(cfg, q, k)
+        rows = np.array([(bh * w.seq_len + i) for bh in range(w.batch * w.n_q_heads)
+                         for i in range(S)])
+        out, _ = oracle.attention(cfg, q, k, v, idx, rows=rows)
+        np.testing.assert_allclose(out, ref[:, :, :S].reshape(-1, w.head_dim).numpy(), rtol=0,
+                                   atol=1e-10)
+
+
+# ----------------------------------------------------------------------------- invariants
+
+def test_selection_nested_in_tau_and_sparsity_monotone():
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    taus = [0.0, 0.001, 0.01, 0.02, 0.05, 0.1, 0.3, 1.0, 1.5]
+    prev_sets, prev_pairs = None, None
+    for tau in taus:
+        cfg = oracle.config(w, tau=tau)
+        idx = oracle.build_indices(cfg, q, k)
+        sets = [set(idx["sel_blk"][b, h, x, :idx["sel_cnt"][b, h, x]].tolist())
+                for b in range(w.batch) for h in range(w.n_q_heads)
+                for x in range(w.seq_len // w.block_size)]
+        pairs = oracle.pair_count(cfg, idx)
+        if prev_sets is not None:
+            assert all(s <= p for s, p in zip(sets, prev_sets))
+            assert pairs <= prev_pairs
+        prev_sets, prev_pairs = sets, pairs
+
+
+def test_probabilities_and_selection_rule():
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    cfg = oracle.config(w)
+    idx = oracle.build_indices(cfg, q, k, debug=True)
+    S, Bk, nB = w.segment_len, w.block_size, w.seq_len // w.block_size
+    for b in range(w.batch):
+        for h in range(w.n_q_heads):
+            for x in range(nB):
+                s = x * Bk // S
+                cand = idx["n"][b, h, s] > 0
+                p = idx["p"][b, h, x]
+                cnt = idx["sel_cnt"][b, h, x]
+                if s == 0:
+                    assert not cand.any() and cnt == 0
+                    continue
+                assert abs(p[cand].sum() - 1.0) < 1e-12
+                assert (p[~cand] == 0).all()
+                chosen = np.nonzero(cand & (p >= np.float64(np.float32(w.tau))))[0]
+                order = sorted(chosen, key=lambda c: (-p[c], c))
+                np.testing.assert_array_equal(idx["sel_blk"][b, h, x, :cnt], order)
+
+
+def test_index_arrays_are_sorted_permutations():
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    idx = oracle.build_indices(oracle.config(w), q, k, debug=True)
+    N, S, Bk = w.seq_len, w.segment_len, w.block_size
+    for b in range(w.batch):
+        for h in range(w.n_q_heads):
+            pk, pq = idx["perm_k"][b, h], idx["perm_q"][b, h]
+            assert sorted(pk.tolist()) == list(range(N))
+            ks = idx["kappa"][b, h][pk]
+            assert (np.diff(ks) <= 0).all()
+            ties = np.nonzero(np.diff(ks) == 0)[0]
+            assert (pk[ties] < pk[ties + 1]).all()
+            for s0 in range(0, N, S):
+                seg = pq[s0:s0 + S]
+                assert sorted(seg.tolist()) == list(range(s0, s0 + S))
+                rs = idx["rho"][b, h][seg]
+                assert (np.diff(rs) <= 0).all()
+                t = np.nonzero(np.diff(rs) == 0)[0]
+                assert (seg[t] < seg[t + 1]).all()
+            for x in range(N // Bk):
+                s0 = (x * Bk // S) * S
+                assert idx["local_tiles"][b, h, x] == (pq[x * Bk:(x + 1) * Bk].max() - s0) // Bk + 1
+
+
+def test_query_perm_off_is_identity_and_triangle():
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    idx = oracle.build_indices(oracle.config(w, query_perm=0), q, k)
+    N, S, Bk = w.seq_len, w.segment_len, w.block_size
+    np.testing.assert_array_equal(idx["perm_q"], np.broadcast_to(np.arange(N), idx["perm_q"].shape))
+    x = np.arange(N // Bk)
+    np.testing.assert_array_equal(idx["local_tiles"][0, 0], x - (x * Bk // S) * (S // Bk) + 1)
+
+
+def test_float64_rederivation_of_pooled_quantities():
+    """Every pooled quantity against an independent float64 numpy computation (GQA mapping,
+    operand order, signs and the 1/sqrt(d) scale); n and local tiles exactly."""
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    idx = oracle.build_indices(oracle.config(w), q, k, debug=True)
+    Q, K = q.double().numpy(), k.double().numpy()
+    G, N, S, Bk, d = w.n_q_heads // w.n_kv_heads, w.seq_len, w.segment_len, w.block_size, w.head_dim
+    nB = N // Bk
+    tol = dict(rtol=1e-5, atol=1e-5)
+    for b in range(w.batch):
+        for h in range(w.n_q_heads):
+            Kg = K[b, h // G]
+            qbar = Q[b, h].mean(0)
+            np.testing.assert_allclose(idx["qbar"][b, h], qbar, **tol)
+            np.testing.assert_allclose(idx["kbar_all"][b, h // G], Kg.mean(0), **tol)
+            np.testing.assert_allclose(idx["kappa"][b, h], Kg @ qbar, **tol)
+            pk, pq = idx["perm_k"][b, h], idx["perm_q"][b, h]
+            u = Kg[pk[:Bk]].mean(0) - Kg.mean(0)
+            np.testing.assert_allclose(idx["u"][b, h], u, **tol)
+            np.testing.assert_allclose(idx["rho"][b, h], Q[b, h] @ u, **tol)
+            Qbar = Q[b, h][pq].reshape(nB, Bk, d).mean(1)
+            Kbar = Kg[pk].reshape(nB, Bk, d).mean(1)
+            np.testing.assert_allclose(idx["Qbar"][b, h], Qbar, **tol)
+            np.testing.assert_allclose(idx["Kbar"][b, h], Kbar, **tol)
+            np.testing.assert_allclose(idx["r"][b, h], Qbar @ Kbar.T / math.sqrt(d), **tol)
+            seg_of_key = pk.reshape(nB, Bk) // S
+            n = np.stack([(seg_of_key < s).sum(1) for s in range(N // S)])
+            np.testing.assert_array_equal(idx["n"][b, h], n)
