@@ -1,0 +1,344 @@
+"""Benchmark of the S2O prefill hot path on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path — index build (stripe pooling, both orderings, block
+scores, early-stop lists) then the fused gather-attention — over one synthetic Llama-3.1-8B-shaped
+128K layer (32 query / 8 KV heads, d = 128, S = 2048, B = 128, τ = 0.01), inputs resident in HBM.
+Q alone is 1.07 GB, larger than the 126 MB L2, so no flush is needed between steps.
+
+Metric (the pages' headline): sparse prefill attention time and effective TFLOP/s at 128K, with
+sparsity and MSE, against the bf16 peak. ``value`` is the effective (dense-causal-equivalent)
+TFLOP/s of the whole job: N GPUs × 4·d·N(N+1)/2·Hq FLOPs ÷ the slowest rank's step time.
+
+Multi-GPU (``torchrun``): every rank runs its own independent layer (heads and problems shard
+with no exchange), so scaling is weak and no data-path collective is used; NCCL carries only the
+barrier and the max-over-ranks timing.
+
+``--impl reference`` times the CPU oracle (the only reference arm this project has) on a bounded
+sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+METRIC = "sparse prefill attention ms & effective TFLOPS @128K (sparsity, MSE) vs bf16 peak"
+UNIT = "TFLOP/s (dense-causal-equivalent)"
+WORKLOAD = "llama-128k"
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p.get("bf16_tflops", 1590.0), p.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                maxes.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sms)), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, world, local
+    return None, 0, 1, 0
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(w, q, k, v, max_rows=2048, seed=0):
+    """The oracle as it stands on a bounded sample: one KV group (G query heads) — its index build
+    in full and the attention of `max_rows` random query rows per head — extrapolated to the whole
+    layer. Returns (seconds for the full layer, description, threads)."""
+    import oracle
+    G = w.n_q_heads // w.n_kv_heads
+    sub = w.replace(n_q_heads=G, n_kv_heads=1)
+    qs, ks, vs = q[:, :G].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous()
+    cfg = oracle.config(sub)
+    threads = oracle.threads()
+    t0 = time.perf_counter()
+    idx = oracle.build_indices(cfg, qs, ks, n_threads=threads)
+    t_idx = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    rows = np.sort(np.concatenate([h * w.seq_len + rng.choice(w.seq_len, max_rows, replace=False)
+                                   for h in range(G)]))
+    t0 = time.perf_counter()
+    oracle.attention(cfg, qs, ks, vs, idx, rows=rows, n_threads=threads)
+    t_attn = time.perf_counter() - t0
+    groups = w.n_kv_heads * w.batch
+    full = groups * (t_idx + t_attn * (w.seq_len / max_rows))
+    desc = (f"index build of 1 KV group ({G} query heads) in full ({t_idx:.2f} s) + attention of "
+            f"{max_rows} random rows per head ({t_attn:.2f} s), extrapolated x{groups} groups and "
+            f"x{w.seq_len / max_rows:.0f} rows")
+    return full, desc, threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = gen.workload(args.workload, tau=args.tau)
+    q, k, v = gen.make_inputs(w)
+    times, desc, threads = [], "", 0
+    for i in range(args.warmup + args.steps):
+        full, desc, threads = cpu_oracle_sample(w, q, k, v, max_rows=args.ref_rows, seed=i)
+        if i >= args.warmup:
+            times.append(full)
+    sec = float(np.median(times))
+    value = w.dense_causal_flops / sec / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
+                   "n_kv_heads": w.n_kv_heads, "seq_len": w.seq_len, "head_dim": w.head_dim,
+                   "segment_len": w.segment_len, "block_size": w.block_size, "tau": w.tau},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_s2o(args):
+    import long_context_sparse_stripe_b200 as s2o
+
+    dist, rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = gen.workload(args.workload, tau=args.tau)
+    # Each rank runs its own independent layer (weak scaling).
+    q, k, v = gen.make_inputs(w.replace(seed=w.seed + 100 * rank))
+    cfg = s2o.Config.of(w)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    o = torch.empty_like(qd)
+    idx = s2o.alloc_indices(cfg, dev)
+    ws = s2o.alloc_workspace(cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx, out=o)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if s2o.check_device_status(dev) != 0:
+        raise RuntimeError("device timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = s2o.kernel_launch_count()
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = s2o.kernel_launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    status = s2o.check_device_status(dev)
+    total_ms = start.elapsed_time(end)
+    index_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms_step = max_over_ranks(dist, total_ms / args.steps, dev)
+    attn_ms_max = max_over_ranks(dist, attn_ms, dev)
+
+    stats = s2o.index_stats(cfg, idx, ws)
+    tile_flops = 4.0 * w.block_size * w.block_size * w.head_dim
+    exec_flops = stats.executed_tiles * tile_flops
+    peak, hbm_peak, peak_kind = measured_peaks()
+
+    # Dense causal baseline on the same inputs, and the MSE of the S2O output against it.
+    od = torch.empty_like(qd)
+    s2o.dense_causal_prefill(cfg, qd, kd, vd, out=od)
+    torch.cuda.synchronize(dev)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(args.dense_steps):
+        s2o.dense_causal_prefill(cfg, qd, kd, vd, out=od)
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = d0.elapsed_time(d1) / args.dense_steps
+    mse = float(((o.float() - od.float()) ** 2).mean().item())
+    del od
+
+    # End to end through the public call with host buffers: pinned H2D of Q/K/V, the prefill,
+    # D2H of O, every step.
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        s2o.attention_prefill(cfg, qd, kd, vd, out=o, idx=idx, ws=ws)
+        oh.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.e2e_steps, dev)
+
+    flops_all = w.dense_causal_flops * world
+    line = None
+    if rank == 0:
+        achieved = exec_flops / (attn_ms_max * 1e-3) / 1e12
+        line = {
+            "metric": METRIC,
+            "value": flops_all / (ms_step * 1e-3) / 1e12,
+            "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
+                       "n_kv_heads": w.n_kv_heads, "seq_len": w.seq_len, "head_dim": w.head_dim,
+                       "segment_len": w.segment_len, "block_size": w.block_size, "tau": w.tau,
+                       "query_perm": w.query_perm, "parallelism": f"independent layer per GPU x{world}",
+                       "l2": "inputs larger than L2 (Q is 1.07 GB); no flush"},
+            "s2o_ms": ms_step, "index_ms": index_ms, "attention_ms": attn_ms,
+            "index_fraction_of_attention": index_ms / attn_ms,
+            "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms_step,
+            "pair_sparsity": stats.pair_sparsity,
+            "tile_density": stats.executed_tiles * w.block_size ** 2 * 1.0 / stats.causal_pairs,
+            "executed_tiles": stats.executed_tiles, "local_tiles": stats.local_tiles,
+            "selected_tiles": stats.selected_tiles, "mse_vs_dense": mse,
+            "exec_tflops": achieved,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "kernel": "s2o_attention_kernel<128,128>",
+                         "peak_source": f"{peak_kind} bf16 (burst)"},
+            "e2e": {"value": flops_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "device_status": s2o.STATUS.get(status, status),
+        }
+    if dist is not None:
+        dist.barrier()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        full, desc, threads = cpu_oracle_sample(w, q, k, v, max_rows=args.ref_rows)
+        line["cpu_baseline"] = {"value": w.dense_causal_flops / full / 1e12, "unit": UNIT,
+                                "cores": threads, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="s2o", choices=["s2o", "reference"])
+    ap.add_argument("--tau", type=float, default=0.01)
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(gen.WORKLOADS),
+                    help="bench lines use the default; smaller workloads serve profiling")
+    ap.add_argument("--dense-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-rows", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "s2o":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_s2o(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

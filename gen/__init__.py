@@ -8,8 +8,8 @@ available; these inputs stand in for them with the same attention shapes (32 que
 heads, d = 128) and with the stripe patterns the S2O card's Summary says real attention maps are
 made of (vertical stripes on a few key positions, a diagonal).
 
-Recipe (each (tensor, batch, head) slab has its own counter-free numpy stream, so the bytes do not
-depend on how many threads draw them):
+Recipe (each (tensor, batch, head) slab has its own numpy stream, so the bytes do not depend on
+how many threads draw them):
 
 1. Q, K, V ~ N(0, 1) float32; slab (t, beta, head) drawn from
    ``Generator(PCG64(SeedSequence(seed, spawn_key=(t, beta, head))))`` with t = 0, 1, 2 for Q, K, V.
@@ -88,6 +88,13 @@ def _stream(seed: int, *key: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=key)))
 
 
+def _to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even (inputs are finite)."""
+    b = x.view(np.uint32)
+    return ((b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)) \
+        .astype(np.uint16)
+
+
 def make_inputs(w: Workload, threads: int | None = None, keep_fp32: bool = False):
     """Return ``(q, k, v)`` as contiguous CPU bf16 tensors in BHND layout.
 
@@ -97,41 +104,45 @@ def make_inputs(w: Workload, threads: int | None = None, keep_fp32: bool = False
     B, Hq, Hkv, N, d = w.batch, w.n_q_heads, w.n_kv_heads, w.seq_len, w.head_dim
     G = Hq // Hkv
     threads = threads or min(32, os.cpu_count() or 1)
-    q = np.empty((B, Hq, N, d), np.float32)
-    k = np.empty((B, Hkv, N, d), np.float32)
-    v = np.empty((B, Hkv, N, d), np.float32)
+    n_stripe = w.stripe_count if w.stripe_count is not None else int(round(w.stripe_frac * N))
+    kf = np.empty((B, Hkv, N, d), np.float32)
+    qb = np.empty((B, Hq, N, d), np.uint16)
+    kb = np.empty((B, Hkv, N, d), np.uint16)
+    vb = np.empty((B, Hkv, N, d), np.uint16)
+    qf = np.empty((B, Hq, N, d), np.float32) if keep_fp32 else None
+    vf = np.empty((B, Hkv, N, d), np.float32) if keep_fp32 else None
+    u = np.empty((B, Hkv, d), np.float32)
 
-    jobs = [(0, b, h) for b in range(B) for h in range(Hq)]
-    jobs += [(t, b, h) for t in (1, 2) for b in range(B) for h in range(Hkv)]
-    dst = {0: q, 1: k, 2: v}
+    def kv_job(job):
+        b, g = job
+        _stream(w.seed, 1, b, g).standard_normal(out=kf[b, g], dtype=np.float32)
+        rng = _stream(w.seed, 3, b, g)
+        ug = rng.standard_normal(d)
+        u[b, g] = (ug / np.linalg.norm(ug)).astype(np.float32)
+        pos = rng.choice(N, size=n_stripe, replace=False)
+        kf[b, g, pos, :] += np.float32(w.amp) * u[b, g]
+        kb[b, g] = _to_bf16_bits(kf[b, g])
+        vslab = np.empty((N, d), np.float32) if vf is None else vf[b, g]
+        _stream(w.seed, 2, b, g).standard_normal(out=vslab, dtype=np.float32)
+        vb[b, g] = _to_bf16_bits(vslab)
 
-    def fill(job):
-        t, b, h = job
-        dst[t][b, h] = _stream(w.seed, t, b, h).standard_normal((N, d), dtype=np.float32)
+    def q_job(job):
+        b, h = job
+        g = h // G
+        slab = np.empty((N, d), np.float32) if qf is None else qf[b, h]
+        _stream(w.seed, 0, b, h).standard_normal(out=slab, dtype=np.float32)
+        slab += np.float32(w.q_shift) * u[b, g]
+        if w.diag:
+            slab += np.float32(w.diag) * kf[b, g]
+        qb[b, h] = _to_bf16_bits(slab)
 
     with ThreadPoolExecutor(threads) as ex:
-        list(ex.map(fill, jobs))
+        list(ex.map(kv_job, [(b, g) for b in range(B) for g in range(Hkv)]))
+        list(ex.map(q_job, [(b, h) for b in range(B) for h in range(Hq)]))
 
-    n_stripe = w.stripe_count if w.stripe_count is not None else int(round(w.stripe_frac * N))
-    for b in range(B):
-        for g in range(Hkv):
-            rng = _stream(w.seed, 3, b, g)
-            u = rng.standard_normal(d)
-            u = (u / np.linalg.norm(u)).astype(np.float32)
-            pos = rng.choice(N, size=n_stripe, replace=False)
-            k[b, g, pos, :] += np.float32(w.amp) * u
-            q[b, g * G:(g + 1) * G] += np.float32(w.q_shift) * u
-
-    if w.diag:
-        def diag(job):
-            b, h = job
-            q[b, h] += np.float32(w.diag) * k[b, h // G]
-        with ThreadPoolExecutor(threads) as ex:
-            list(ex.map(diag, [(b, h) for b in range(B) for h in range(Hq)]))
-
-    out = tuple(torch.from_numpy(x).to(torch.bfloat16).contiguous() for x in (q, k, v))
+    out = tuple(torch.from_numpy(x).view(torch.bfloat16) for x in (qb, kb, vb))
     if keep_fp32:
-        return out + ((q, k, v),)
+        return out + ((qf, kf, vf),)
     return out
 
 

@@ -1,0 +1,168 @@
+/*
+ * s2o.h — C ABI of libs2o: permuted, importance-ordered, early-stopped block-sparse causal
+ * attention prefill (S2O) on one NVIDIA B200 (sm_100a).
+ *
+ * What the library computes is defined step by step in the project's definition file; each entry
+ * point below names the passages of the pages it implements:
+ *   [S2O]  "S2O: Early Stopping for Sparse Attention via Online Permutation" (research card),
+ *          Summary ¶2 and Key points.
+ *   [PBS]  "Sparser Block-Sparse Attention via Token Permutation" (ICML poster), lay summary.
+ *   [AB]   "AB-Sparse", Eq. (1) and the Figure 2 workflow text.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are bf16, contiguous, BHND: Q and O [batch, Hq, N, d]; K and V [batch, Hkv, N, d].
+ *    Query head h reads key/value head h / (Hq/Hkv).
+ *  - Every pointer except `cfg`, size outputs and `s2o_stats*` is a DEVICE pointer owned by the
+ *    caller, 16-byte aligned. The library never allocates device memory: scratch comes from the
+ *    caller's workspace `ws` (size from s2o_workspace_size).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Launching calls are
+ *    asynchronous on it; argument errors are returned before anything is enqueued, and device
+ *    faults surface at the caller's next synchronisation (CUDA convention).
+ *  - Supported shapes: d ∈ {64, 128}; B ∈ {64, 128}; Hq % Hkv == 0; N % S == 0; S % B == 0;
+ *    N/B ≤ 2048; batch·Hq·N < 2^31; 0 ≤ tau (finite). tau > 1 is legal and selects no permuted block (local window only).
+ *    Anything else returns S2O_ERR_UNSUPPORTED.
+ *  - Calls on different streams must not share a workspace.
+ */
+#ifndef S2O_H
+#define S2O_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *s2o_stream; /* a cudaStream_t */
+
+typedef enum {
+  S2O_OK = 0,
+  S2O_ERR_INVALID_ARGUMENT = 1,    /* null/misaligned pointer, negative or NaN tau, ...    */
+  S2O_ERR_UNSUPPORTED = 2,         /* shape outside the supported set above              */
+  S2O_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below s2o_workspace_size                  */
+  S2O_ERR_INVALID_INDICES = 4,     /* s2o_validate_indices found a bad index array       */
+  S2O_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed               */
+  S2O_ERR_DEVICE_TIMEOUT = 6       /* a kernel gave up a bounded wait (see below)        */
+} s2o_status;
+
+/* One attention layer. `query_perm` = 1 builds the segment-local query ordering; 0 keeps the
+ * identity (the "Q perm" ablation of [S2O, Key points]). */
+typedef struct {
+  int batch, n_q_heads, n_kv_heads, seq_len, head_dim, segment_len, block_size;
+  float tau;
+  int query_perm;
+} s2o_config;
+
+/* Caller-owned index arrays (device, int32). nB = N / B.
+ *  perm_q      [batch, Hq, N]      original query index at each permuted slot; slots
+ *                                  [sS, (s+1)S) hold a permutation of segment s.
+ *  perm_k      [batch, Hq, N]      original key index at each rank (one ordering per query head).
+ *  sel_cnt     [batch, Hq, nB]     number of selected permuted key blocks of each query block.
+ *  sel_blk     [batch, Hq, nB, nB] selected key-block ids (blocks of perm_k), most important
+ *                                  first; entries at and after sel_cnt are not written.
+ *  local_tiles [batch, Hq, nB]     original-order key tiles of the query block's own segment that
+ *                                  the kernel runs (1 ≤ lt ≤ S/B). */
+typedef struct {
+  int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
+} s2o_indices;
+
+/* Work and sparsity counts of one index set (host struct, filled by s2o_index_stats). */
+typedef struct {
+  uint64_t local_tiles;    /* Σ_b lt_b                                                  */
+  uint64_t selected_tiles; /* Σ_b cnt_b                                                 */
+  uint64_t pairs;          /* Σ_i |K_i|: (query, key) pairs attended                   */
+  uint64_t causal_pairs;   /* batch·Hq·N(N+1)/2: pairs of dense causal attention          */
+} s2o_stats;
+
+/* Device pointers into a workspace after s2o_build_indices: the intermediate values of the
+ * index build (fp32 unless noted), for inspection and tests. Valid until the workspace is reused.
+ *  qbar [b,Hq,d]; kbar_all [b,Hkv,d]; kbar_top, u [b,Hq,d]; kappa, rho [b,Hq,N];
+ *  Qbar, Kbar [b,Hq,nB,d]; r [b,Hq,nB,nB]; n [b,Hq,nSeg,nB] (int32). */
+typedef struct {
+  float *qbar, *kbar_all, *kbar_top, *u, *kappa, *rho, *Qbar, *Kbar, *r;
+  int32_t *n;
+} s2o_workspace_view;
+
+/* Human-readable name of a status. Never NULL. */
+const char *s2o_status_string(s2o_status status);
+
+/* Bytes of scratch that s2o_build_indices / s2o_attention_prefill / s2o_validate_indices need
+ * for `cfg`, written to *bytes. Host only; no device work. */
+s2o_status s2o_workspace_size(const s2o_config *cfg, size_t *bytes);
+
+/* Element counts of the five index arrays of `cfg`, in s2o_indices field order. Host only. */
+s2o_status s2o_index_sizes(const s2o_config *cfg, size_t counts[5]);
+
+/* Steps 1–2 of the method ([S2O, Summary ¶2]: stripe-level mean pooling, the global key/value
+ * ordering, the segment-local query ordering, block scores and the early stop at tau) for every
+ * (batch, query head): writes the index arrays of `out`. Bit-exact with the definition: same
+ * inputs give the same indices on every run. q, k: device bf16 as above. */
+s2o_status s2o_build_indices(const s2o_config *cfg, const void *q, const void *k,
+                             const s2o_indices *out, void *ws, size_t ws_bytes,
+                             s2o_stream stream);
+
+/* Pointers to the intermediate values held in `ws` (see s2o_workspace_view). Host only. */
+s2o_status s2o_workspace_views(const s2o_config *cfg, void *ws, size_t ws_bytes,
+                               s2o_workspace_view *view);
+
+/* The whole hot path ([S2O, Summary ¶2]): s2o_build_indices into `idx`, then the fused
+ * gather-attention over local tiles and selected permuted blocks; O [batch, Hq, N, d] bf16 is
+ * written at original positions. */
+s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const void *k,
+                                 const void *v, void *o, const s2o_indices *idx, void *ws,
+                                 size_t ws_bytes, s2o_stream stream);
+
+/* Steps 3–4 only, on caller-supplied index arrays ([S2O, Summary ¶2]: the kernel fetches the
+ * scattered rows into shared memory by index and runs the blocks in list order; causality is
+ * enforced on original positions). Memory-safe for any index contents (out-of-range values are
+ * clamped and out-of-range output rows skipped), but the result is only defined for index arrays
+ * that s2o_validate_indices accepts. */
+s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void *q,
+                                              const void *k, const void *v,
+                                              const s2o_indices *idx, void *o,
+                                              s2o_stream stream);
+
+/* In-repo dense causal attention baseline, Eq. (1) of [AB], on the same kernel machinery
+ * (contiguous tiles, no index arrays). cfg->segment_len, tau and query_perm are ignored. */
+s2o_status s2o_dense_causal_prefill(const s2o_config *cfg, const void *q, const void *k,
+                                    const void *v, void *o, s2o_stream stream);
+
+/* Checks that perm_q is a segment-local permutation, perm_k a permutation of [0, N), every
+ * sel_cnt in [0, nB], every listed block id in [0, nB) and unique within its list, and every
+ * local_tiles value in [1, S/B] and covering its block's last query. Uses `ws`; SYNCHRONISES
+ * `stream`. Returns S2O_OK or S2O_ERR_INVALID_INDICES. */
+s2o_status s2o_validate_indices(const s2o_config *cfg, const s2o_indices *idx, void *ws,
+                                size_t ws_bytes, s2o_stream stream);
+
+/* Work and sparsity counts of an index set (definition: pair sparsity = 1 − pairs /
+ * causal_pairs). Uses `ws`; SYNCHRONISES `stream`; writes the host struct *stats. */
+s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *ws,
+                           size_t ws_bytes, s2o_stats *stats, s2o_stream stream);
+
+/* Every wait inside the attention kernel (on a TMA copy, a tensor-core commit or a peer warp) is
+ * bounded by this many nanoseconds of GPU time (default 2e9). When a wait runs out, the kernel
+ * records it, drains its own copies and tensor-core work, frees its tensor memory and returns.
+ * Affects launches made after the call; not thread-safe against concurrent launches. */
+void s2o_set_wait_limit_ns(uint64_t ns);
+
+/* Number of kernel launches the library has made in this process so far (all threads and
+ * devices), for launch accounting. Host only. */
+uint64_t s2o_kernel_launch_count(void);
+
+/* Synchronises `stream`, then reports and clears the device error record: S2O_ERR_DEVICE_TIMEOUT
+ * if a bounded wait ran out since the last check, S2O_ERR_CUDA if the stream holds an error,
+ * else S2O_OK. */
+s2o_status s2o_check_device_status(s2o_stream stream);
+
+/* Diagnostic: evaluates the library's exp64 — the binary64 exponential behind the block weights of
+ * the early stop (a Cody–Waite reduction by ln 2 and a degree-13 Taylor polynomial, defined in
+ * the project's definition file; the pages give no normalisation, see [S2O, Summary ¶2]) — on n
+ * device doubles x (each ≤ 0), writing device doubles y. Asynchronous on `stream`. */
+s2o_status s2o_exp64_eval(const double *x, double *y, int n, s2o_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2O_H */

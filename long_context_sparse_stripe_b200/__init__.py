@@ -1,0 +1,334 @@
+"""Python binding of libs2o: S2O permuted, importance-ordered, early-stopped block-sparse causal
+attention prefill on one B200.
+
+The binding only marshals arguments: it checks tensor shapes, dtypes and devices, allocates
+outputs and the workspace with PyTorch (device memory and streams are PyTorch's job), and passes
+raw device pointers and the current CUDA stream to the C ABI declared in ``include/s2o.h``. Every
+step of the method runs in the library's CUDA kernels; there is no CPU or PyTorch fallback — if
+``libs2o.so`` cannot be loaded, importing this package raises.
+
+Sources: "S2O: Early Stopping for Sparse Attention via Online Permutation" (Summary ¶2) for the
+method, "AB-Sparse" Eq. (1) for the dense baseline.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "Config", "Indices", "Stats", "S2OError", "workspace_size", "index_sizes", "alloc_indices",
+    "alloc_workspace", "build_indices", "attention_prefill", "attention_prefill_with_indices",
+    "dense_causal_prefill", "validate_indices", "index_stats", "workspace_views",
+    "set_wait_limit_ns", "check_device_status", "exp64_eval", "library_path",
+    "kernel_launch_count",
+]
+
+STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
+          3: "S2O_ERR_WORKSPACE_TOO_SMALL", 4: "S2O_ERR_INVALID_INDICES", 5: "S2O_ERR_CUDA",
+          6: "S2O_ERR_DEVICE_TIMEOUT"}
+
+
+class S2OError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("seq_len", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("segment_len", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("tau", ctypes.c_float),
+                ("query_perm", ctypes.c_int)]
+
+
+class _Indices(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("perm_q", "perm_k", "sel_cnt", "sel_blk", "local_tiles")]
+
+
+class _Stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in
+                ("local_tiles", "selected_tiles", "pairs", "causal_pairs")]
+
+
+class _View(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("qbar", "kbar_all", "kbar_top", "u", "kappa", "rho", "Qbar", "Kbar", "r", "n")]
+
+
+@dataclasses.dataclass(frozen=True)
+class Config:
+    """One attention layer (the fields of ``s2o_config``)."""
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    seq_len: int
+    head_dim: int
+    segment_len: int
+    block_size: int
+    tau: float
+    query_perm: int = 1
+
+    @classmethod
+    def of(cls, obj, **overrides) -> "Config":
+        f = {k.name: getattr(obj, k.name) for k in dataclasses.fields(cls)}
+        f.update(overrides)
+        return cls(**f)
+
+    def _c(self) -> _Config:
+        return _Config(self.batch, self.n_q_heads, self.n_kv_heads, self.seq_len, self.head_dim,
+                       self.segment_len, self.block_size, float(self.tau), self.query_perm)
+
+    @property
+    def n_blocks(self) -> int:
+        return self.seq_len // self.block_size
+
+
+@dataclasses.dataclass
+class Indices:
+    """Index arrays on the device (int32), shapes as in ``s2o_indices``."""
+    perm_q: torch.Tensor
+    perm_k: torch.Tensor
+    sel_cnt: torch.Tensor
+    sel_blk: torch.Tensor
+    local_tiles: torch.Tensor
+
+    def tensors(self):
+        # Not dataclasses.astuple: that deep-copies its fields, and the library must see these
+        # exact tensors.
+        return (self.perm_q, self.perm_k, self.sel_cnt, self.sel_blk, self.local_tiles)
+
+    def _c(self) -> _Indices:
+        for t in self.tensors():
+            if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError("index arrays must be contiguous int32 CUDA tensors")
+        return _Indices(*(t.data_ptr() for t in self.tensors()))
+
+
+@dataclasses.dataclass(frozen=True)
+class Stats:
+    local_tiles: int
+    selected_tiles: int
+    pairs: int
+    causal_pairs: int
+
+    @property
+    def pair_sparsity(self) -> float:
+        return 1.0 - self.pairs / self.causal_pairs
+
+    @property
+    def executed_tiles(self) -> int:
+        return self.local_tiles + self.selected_tiles
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        vp, st, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        C, I = ctypes.POINTER(_Config), ctypes.POINTER(_Indices)
+        sig = {
+            "s2o_workspace_size": [C, ctypes.POINTER(sz)],
+            "s2o_index_sizes": [C, ctypes.POINTER(sz * 5)],
+            "s2o_build_indices": [C, vp, vp, I, vp, sz, vp],
+            "s2o_workspace_views": [C, vp, sz, ctypes.POINTER(_View)],
+            "s2o_attention_prefill": [C, vp, vp, vp, vp, I, vp, sz, vp],
+            "s2o_attention_prefill_with_indices": [C, vp, vp, vp, I, vp, vp],
+            "s2o_dense_causal_prefill": [C, vp, vp, vp, vp, vp],
+            "s2o_validate_indices": [C, I, vp, sz, vp],
+            "s2o_index_stats": [C, I, vp, sz, ctypes.POINTER(_Stats), vp],
+            "s2o_check_device_status": [vp],
+            "s2o_exp64_eval": [vp, vp, ctypes.c_int, vp],
+        }
+        for name, args in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = st
+        lib.s2o_kernel_launch_count.argtypes = []
+        lib.s2o_kernel_launch_count.restype = ctypes.c_uint64
+        lib.s2o_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.s2o_set_wait_limit_ns.restype = None
+        lib.s2o_status_string.argtypes = [st]
+        lib.s2o_status_string.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise S2OError(status, where)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _bf16(t: torch.Tensor, shape, name: str):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _qkv(cfg: Config, q, k, v=None):
+    _bf16(q, (cfg.batch, cfg.n_q_heads, cfg.seq_len, cfg.head_dim), "q")
+    _bf16(k, (cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim), "k")
+    if v is not None:
+        _bf16(v, (cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim), "v")
+
+
+def workspace_size(cfg: Config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_load().s2o_workspace_size(ctypes.byref(cfg._c()), ctypes.byref(n)),
+           "s2o_workspace_size")
+    return n.value
+
+
+def index_sizes(cfg: Config):
+    arr = (ctypes.c_size_t * 5)()
+    _check(_load().s2o_index_sizes(ctypes.byref(cfg._c()), ctypes.byref(arr)), "s2o_index_sizes")
+    return list(arr)
+
+
+def alloc_workspace(cfg: Config, device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def alloc_indices(cfg: Config, device="cuda") -> Indices:
+    B, H, N, nB = cfg.batch, cfg.n_q_heads, cfg.seq_len, cfg.n_blocks
+    e = lambda *s: torch.empty(s, dtype=torch.int32, device=device)  # noqa: E731
+    return Indices(e(B, H, N), e(B, H, N), e(B, H, nB), e(B, H, nB, nB), e(B, H, nB))
+
+
+def build_indices(cfg: Config, q, k, out: Indices | None = None,
+                  ws: torch.Tensor | None = None) -> Indices:
+    _qkv(cfg, q, k)
+    out = out or alloc_indices(cfg, q.device)
+    ws = ws if ws is not None else alloc_workspace(cfg, q.device)
+    idx = out._c()
+    _check(_load().s2o_build_indices(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
+                                     ctypes.byref(idx), ws.data_ptr(), ws.numel(),
+                                     _stream(q.device)), "s2o_build_indices")
+    return out
+
+
+def workspace_views(cfg: Config, ws: torch.Tensor) -> dict:
+    """Intermediate values of the last index build held in ``ws`` (views, no copy)."""
+    view = _View()
+    _check(_load().s2o_workspace_views(ctypes.byref(cfg._c()), ws.data_ptr(), ws.numel(),
+                                       ctypes.byref(view)), "s2o_workspace_views")
+    B, Hq, Hkv, N, d = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim
+    nB, nSeg = cfg.n_blocks, cfg.seq_len // cfg.segment_len
+    shapes = dict(qbar=(B, Hq, d), kbar_all=(B, Hkv, d), kbar_top=(B, Hq, d), u=(B, Hq, d),
+                  kappa=(B, Hq, N), rho=(B, Hq, N), Qbar=(B, Hq, nB, d), Kbar=(B, Hq, nB, d),
+                  r=(B, Hq, nB, nB), n=(B, Hq, nSeg, nB))
+    base = ws.data_ptr()
+    out = {}
+    for name, shape in shapes.items():
+        off = getattr(view, name) - base
+        count = 1
+        for s in shape:
+            count *= s
+        dt = torch.int32 if name == "n" else torch.float32
+        out[name] = ws[off:off + 4 * count].view(dt).view(shape)
+    return out
+
+
+def attention_prefill(cfg: Config, q, k, v, out: torch.Tensor | None = None,
+                      idx: Indices | None = None, ws: torch.Tensor | None = None):
+    """The whole S2O hot path: index build then gather-attention. Returns (O, indices)."""
+    _qkv(cfg, q, k, v)
+    o = out if out is not None else torch.empty_like(q)
+    _bf16(o, q.shape, "out")
+    idx = idx or alloc_indices(cfg, q.device)
+    ws = ws if ws is not None else alloc_workspace(cfg, q.device)
+    ci = idx._c()
+    _check(_load().s2o_attention_prefill(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
+                                         v.data_ptr(), o.data_ptr(), ctypes.byref(ci),
+                                         ws.data_ptr(), ws.numel(), _stream(q.device)),
+           "s2o_attention_prefill")
+    return o, idx
+
+
+def attention_prefill_with_indices(cfg: Config, q, k, v, idx: Indices,
+                                   out: torch.Tensor | None = None) -> torch.Tensor:
+    _qkv(cfg, q, k, v)
+    o = out if out is not None else torch.empty_like(q)
+    _bf16(o, q.shape, "out")
+    ci = idx._c()
+    _check(_load().s2o_attention_prefill_with_indices(ctypes.byref(cfg._c()), q.data_ptr(),
+                                                      k.data_ptr(), v.data_ptr(),
+                                                      ctypes.byref(ci), o.data_ptr(),
+                                                      _stream(q.device)),
+           "s2o_attention_prefill_with_indices")
+    return o
+
+
+def dense_causal_prefill(cfg: Config, q, k, v, out: torch.Tensor | None = None) -> torch.Tensor:
+    _qkv(cfg, q, k, v)
+    o = out if out is not None else torch.empty_like(q)
+    _bf16(o, q.shape, "out")
+    _check(_load().s2o_dense_causal_prefill(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
+                                            v.data_ptr(), o.data_ptr(), _stream(q.device)),
+           "s2o_dense_causal_prefill")
+    return o
+
+
+def validate_indices(cfg: Config, idx: Indices, ws: torch.Tensor | None = None) -> bool:
+    """True when the index arrays are valid (synchronises the current stream)."""
+    dev = idx.perm_q.device
+    ws = ws if ws is not None else alloc_workspace(cfg, dev)
+    ci = idx._c()
+    st = _load().s2o_validate_indices(ctypes.byref(cfg._c()), ctypes.byref(ci), ws.data_ptr(),
+                                      ws.numel(), _stream(dev))
+    if st == 4:
+        return False
+    _check(st, "s2o_validate_indices")
+    return True
+
+
+def index_stats(cfg: Config, idx: Indices, ws: torch.Tensor | None = None) -> Stats:
+    dev = idx.perm_q.device
+    ws = ws if ws is not None else alloc_workspace(cfg, dev)
+    ci = idx._c()
+    s = _Stats()
+    _check(_load().s2o_index_stats(ctypes.byref(cfg._c()), ctypes.byref(ci), ws.data_ptr(),
+                                   ws.numel(), ctypes.byref(s), _stream(dev)), "s2o_index_stats")
+    return Stats(s.local_tiles, s.selected_tiles, s.pairs, s.causal_pairs)
+
+
+def kernel_launch_count() -> int:
+    """Kernel launches made by libs2o in this process so far."""
+    return int(_load().s2o_kernel_launch_count())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _load().s2o_set_wait_limit_ns(int(ns))
+
+
+def check_device_status(device="cuda") -> int:
+    """Synchronises and returns the library status (0 = S2O_OK, 6 = a bounded wait ran out)."""
+    return _load().s2o_check_device_status(_stream(torch.device(device)))
+
+
+def exp64_eval(x: torch.Tensor) -> torch.Tensor:
+    if x.dtype != torch.float64 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float64 CUDA tensor")
+    y = torch.empty_like(x)
+    _check(_load().s2o_exp64_eval(x.data_ptr(), y.data_ptr(), x.numel(), _stream(x.device)),
+           "s2o_exp64_eval")
+    return y

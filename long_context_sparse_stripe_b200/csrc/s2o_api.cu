@@ -1,0 +1,277 @@
+// Host side of the libs2o C ABI: argument checks, workspace layout and launches. Every check
+// runs before anything is enqueued, so a returned error means no device work was started.
+#include <atomic>
+#include <cmath>
+
+#include "s2o_internal.h"
+
+namespace s2o {
+
+namespace {
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<unsigned long long> g_launches{0};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+s2o_status check_config(const s2o_config *c) {
+  if (!c) return S2O_ERR_INVALID_ARGUMENT;
+  if (!(c->tau >= 0.0f) || std::isinf(c->tau)) return S2O_ERR_INVALID_ARGUMENT;
+  if (c->batch <= 0 || c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->seq_len <= 0 ||
+      c->segment_len <= 0)
+    return S2O_ERR_INVALID_ARGUMENT;
+  if (c->query_perm != 0 && c->query_perm != 1) return S2O_ERR_INVALID_ARGUMENT;
+  if (c->head_dim != 64 && c->head_dim != 128) return S2O_ERR_UNSUPPORTED;
+  if (c->block_size != 64 && c->block_size != 128) return S2O_ERR_UNSUPPORTED;
+  if (c->n_q_heads % c->n_kv_heads) return S2O_ERR_UNSUPPORTED;
+  if (c->segment_len % c->block_size || c->seq_len % c->segment_len) return S2O_ERR_UNSUPPORTED;
+  // The block scheduler keeps one warp's weights per query block: at most 2048 key blocks.
+  if (c->seq_len / c->block_size > 2048) return S2O_ERR_UNSUPPORTED;
+  // Flattened row coordinates of the TMA maps are 32-bit.
+  if ((long long)c->batch * c->n_q_heads * c->seq_len >= (1ll << 31)) return S2O_ERR_UNSUPPORTED;
+  return S2O_OK;
+}
+
+s2o_status check_dense_config(const s2o_config *c) {
+  if (!c) return S2O_ERR_INVALID_ARGUMENT;
+  s2o_config x = *c;
+  x.segment_len = x.seq_len;
+  x.tau = 0.f;
+  x.query_perm = 1;
+  return check_config(&x);
+}
+
+bool indices_ok(const s2o_indices *idx) {
+  return idx && idx->perm_q && idx->perm_k && idx->sel_cnt && idx->sel_blk && idx->local_tiles &&
+         aligned16(idx->perm_q) && aligned16(idx->perm_k) && aligned16(idx->sel_cnt) &&
+         aligned16(idx->sel_blk) && aligned16(idx->local_tiles);
+}
+
+s2o_status from_cuda(cudaError_t e) { return e == cudaSuccess ? S2O_OK : S2O_ERR_CUDA; }
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+unsigned long long launch_count() { return g_launches.load(std::memory_order_relaxed); }
+
+Dims dims_of(const s2o_config &c) {
+  Dims d;
+  d.batch = c.batch;
+  d.Hq = c.n_q_heads;
+  d.Hkv = c.n_kv_heads;
+  d.G = c.n_q_heads / c.n_kv_heads;
+  d.N = c.seq_len;
+  d.D = c.head_dim;
+  d.S = c.segment_len;
+  d.B = c.block_size;
+  d.nB = c.seq_len / c.block_size;
+  d.nSeg = c.seq_len / c.segment_len;
+  return d;
+}
+
+WsLayout ws_layout(const Dims &d) {
+  WsLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const size_t bhq = (size_t)d.bhq(), bhkv = (size_t)d.bhkv();
+  L.qchunk = take(bhq * d.nB * d.D * 4);
+  L.kchunk = take(bhkv * d.nB * d.D * 4);
+  L.qbar = take(bhq * d.D * 4);
+  L.kbar_all = take(bhkv * d.D * 4);
+  L.kbar_top = take(bhq * d.D * 4);
+  L.u = take(bhq * d.D * 4);
+  L.kappa = take(bhq * d.N * 4);
+  L.rho = take(bhq * d.N * 4);
+  L.keys0 = take(bhq * d.N * 8);
+  L.keys1 = take(bhq * d.N * 8);
+  L.Qbar = take(bhq * d.nB * d.D * 4);
+  L.Kbar = take(bhq * d.nB * d.D * 4);
+  L.r = take(bhq * d.nB * d.nB * 4);
+  L.ncount = take(bhq * d.nSeg * d.nB * 4);
+  L.flags = take(64);
+  L.total = off;
+  return L;
+}
+
+}  // namespace s2o
+
+using namespace s2o;
+
+extern "C" {
+
+const char *s2o_status_string(s2o_status st) {
+  switch (st) {
+    case S2O_OK: return "S2O_OK";
+    case S2O_ERR_INVALID_ARGUMENT: return "S2O_ERR_INVALID_ARGUMENT";
+    case S2O_ERR_UNSUPPORTED: return "S2O_ERR_UNSUPPORTED";
+    case S2O_ERR_WORKSPACE_TOO_SMALL: return "S2O_ERR_WORKSPACE_TOO_SMALL";
+    case S2O_ERR_INVALID_INDICES: return "S2O_ERR_INVALID_INDICES";
+    case S2O_ERR_CUDA: return "S2O_ERR_CUDA";
+    case S2O_ERR_DEVICE_TIMEOUT: return "S2O_ERR_DEVICE_TIMEOUT";
+  }
+  return "S2O_ERR_UNKNOWN";
+}
+
+s2o_status s2o_workspace_size(const s2o_config *cfg, size_t *bytes) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!bytes) return S2O_ERR_INVALID_ARGUMENT;
+  *bytes = ws_layout(dims_of(*cfg)).total;
+  return S2O_OK;
+}
+
+s2o_status s2o_index_sizes(const s2o_config *cfg, size_t counts[5]) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!counts) return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  counts[0] = (size_t)d.bhq() * d.N;
+  counts[1] = (size_t)d.bhq() * d.N;
+  counts[2] = (size_t)d.bhq() * d.nB;
+  counts[3] = (size_t)d.bhq() * d.nB * d.nB;
+  counts[4] = (size_t)d.bhq() * d.nB;
+  return S2O_OK;
+}
+
+s2o_status s2o_build_indices(const s2o_config *cfg, const void *q, const void *k,
+                             const s2o_indices *out, void *ws, size_t ws_bytes,
+                             s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!q || !k || !ws || !aligned16(q) || !aligned16(k) || !aligned16(ws) || !indices_ok(out))
+    return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  if (ws_bytes < ws_layout(d).total) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(launch_build_indices(d, *cfg, static_cast<const uint16_t *>(q),
+                                        static_cast<const uint16_t *>(k), *out,
+                                        static_cast<char *>(ws), (cudaStream_t)stream));
+}
+
+s2o_status s2o_workspace_views(const s2o_config *cfg, void *ws, size_t ws_bytes,
+                               s2o_workspace_view *view) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!ws || !view) return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  const WsLayout L = ws_layout(d);
+  if (ws_bytes < L.total) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  char *b = static_cast<char *>(ws);
+  view->qbar = reinterpret_cast<float *>(b + L.qbar);
+  view->kbar_all = reinterpret_cast<float *>(b + L.kbar_all);
+  view->kbar_top = reinterpret_cast<float *>(b + L.kbar_top);
+  view->u = reinterpret_cast<float *>(b + L.u);
+  view->kappa = reinterpret_cast<float *>(b + L.kappa);
+  view->rho = reinterpret_cast<float *>(b + L.rho);
+  view->Qbar = reinterpret_cast<float *>(b + L.Qbar);
+  view->Kbar = reinterpret_cast<float *>(b + L.Kbar);
+  view->r = reinterpret_cast<float *>(b + L.r);
+  view->n = reinterpret_cast<int32_t *>(b + L.ncount);
+  return S2O_OK;
+}
+
+s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void *q,
+                                              const void *k, const void *v,
+                                              const s2o_indices *idx, void *o,
+                                              s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !indices_ok(idx))
+    return S2O_ERR_INVALID_ARGUMENT;
+  AttnArgs a{q, k, v, o, idx->perm_q, idx->perm_k, idx->sel_cnt, idx->sel_blk, idx->local_tiles,
+             false};
+  return from_cuda(launch_attention(dims_of(*cfg), a, g_wait_limit_ns.load(),
+                                    (cudaStream_t)stream));
+}
+
+s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const void *k,
+                                 const void *v, void *o, const s2o_indices *idx, void *ws,
+                                 size_t ws_bytes, s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!v || !o || !aligned16(v) || !aligned16(o)) return S2O_ERR_INVALID_ARGUMENT;
+  st = s2o_build_indices(cfg, q, k, idx, ws, ws_bytes, stream);
+  if (st != S2O_OK) return st;
+  return s2o_attention_prefill_with_indices(cfg, q, k, v, idx, o, stream);
+}
+
+s2o_status s2o_dense_causal_prefill(const s2o_config *cfg, const void *q, const void *k,
+                                    const void *v, void *o, s2o_stream stream) {
+  s2o_status st = check_dense_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return S2O_ERR_INVALID_ARGUMENT;
+  s2o_config c = *cfg;
+  c.segment_len = c.seq_len;
+  AttnArgs a{q, k, v, o, nullptr, nullptr, nullptr, nullptr, nullptr, true};
+  return from_cuda(launch_attention(dims_of(c), a, g_wait_limit_ns.load(), (cudaStream_t)stream));
+}
+
+s2o_status s2o_validate_indices(const s2o_config *cfg, const s2o_indices *idx, void *ws,
+                                size_t ws_bytes, s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!ws || !aligned16(ws) || !indices_ok(idx)) return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  const WsLayout L = ws_layout(d);
+  if (ws_bytes < L.total) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  char *b = static_cast<char *>(ws);
+  uint32_t *flag = reinterpret_cast<uint32_t *>(b + L.flags);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_validate(d, *idx, b, flag, s);
+  if (e != cudaSuccess) return S2O_ERR_CUDA;
+  uint32_t host_flag = 0;
+  if (cudaMemcpyAsync(&host_flag, flag, sizeof(host_flag), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return S2O_ERR_CUDA;
+  return host_flag ? S2O_ERR_INVALID_INDICES : S2O_OK;
+}
+
+s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *ws,
+                           size_t ws_bytes, s2o_stats *stats, s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!ws || !aligned16(ws) || !stats || !indices_ok(idx)) return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  const WsLayout L = ws_layout(d);
+  if (ws_bytes < L.total) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  unsigned long long *acc = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) +
+                                                                   L.flags);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_stats(d, *idx, acc, s) != cudaSuccess) return S2O_ERR_CUDA;
+  unsigned long long h[3] = {0, 0, 0};
+  if (cudaMemcpyAsync(h, acc, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return S2O_ERR_CUDA;
+  stats->local_tiles = h[0];
+  stats->selected_tiles = h[1];
+  stats->pairs = h[2];
+  stats->causal_pairs = (uint64_t)d.bhq() * (uint64_t)d.N * (uint64_t)(d.N + 1) / 2;
+  return S2O_OK;
+}
+
+void s2o_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+uint64_t s2o_kernel_launch_count(void) { return launch_count(); }
+
+s2o_status s2o_check_device_status(s2o_stream stream) {
+  unsigned int err = 0;
+  cudaError_t e = read_and_clear_device_error(&err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return S2O_ERR_CUDA;
+  return err ? S2O_ERR_DEVICE_TIMEOUT : S2O_OK;
+}
+
+// Diagnostic: the library's exp64 (used for block weights) on n device doubles, so that tests
+// can compare it bit for bit with an independent implementation.
+s2o_status s2o_exp64_eval(const double *x, double *y, int n, s2o_stream stream) {
+  if (!x || !y || n < 0) return S2O_ERR_INVALID_ARGUMENT;
+  if (n == 0) return S2O_OK;
+  return from_cuda(launch_exp64_probe(x, y, n, (cudaStream_t)stream));
+}
+
+}  // extern "C"

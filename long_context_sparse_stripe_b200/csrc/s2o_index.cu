@@ -1,0 +1,798 @@
+// Index construction of S2O on sm_100a: stripe mean pooling, the global key/value ordering, the
+// segment-local query ordering, block scores and the importance-ordered early stop.
+//
+// Sources: "S2O: Early Stopping for Sparse Attention via Online Permutation" (research card),
+// Summary ¶2 (stripe-level mean pooling; a segment-local query ordering and a global key/value
+// ordering kept as index arrays; blocks processed from most to least important, stopping once a
+// block's score falls under τ) and "AB-Sparse", Figure 2 workflow text (block score r = q·cᵀ
+// against mean-pooled centroids). The formulas where the pages are silent are this project's
+// readings, fixed in its definition file.
+//
+// Every floating-point step below is an explicitly rounded IEEE operation (__fadd_rn, __fmaf_rn,
+// __fdiv_rn, __dadd_rn, __ddiv_rn, ...) in the order the definition fixes, so the index arrays are
+// bit-exact and reproducible. These kernels are bandwidth- or latency-bound; none is a dense
+// contraction worth tensor cores (the block-score product needs a fixed fp32 FMA order).
+#include <algorithm>
+#include <climits>
+
+#include "s2o_internal.h"
+
+namespace s2o {
+namespace {
+
+constexpr int kWarp = 32;
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+__device__ __forceinline__ float bf16_at(const uint16_t *p) {
+  return __uint_as_float((uint32_t)__ldg(p) << 16);
+}
+
+// Sort key of an fp32 score: monotone in the value, −0 folded onto +0, NaN below everything.
+__device__ __forceinline__ uint32_t sort_key(float x) {
+  uint32_t b = __float_as_uint(x);
+  if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;
+  if ((b & 0x7fffffffu) == 0u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Ascending order of this word = descending score, ties to the lower index (a stable
+// descending sort). Indices are below 2^31, so no word equals the all-ones padding value.
+__device__ __forceinline__ unsigned long long order_word(float score, uint32_t idx) {
+  return ((unsigned long long)(~sort_key(score)) << 32) | idx;
+}
+
+// exp64: Cody–Waite reduction by ln 2 with a two-part constant, then the degree-13 Taylor
+// polynomial of e^t by Horner's rule with fused multiply-adds, then an exact scaling by 2^k.
+// Written for this project from the mathematics; defined for x <= 0 (all block-weight arguments).
+__device__ double exp64(double x) {
+  if (x < -700.0) return 0.0;
+  const double kInvLn2 = 0x1.71547652b82fep+0;  // nearest binary64 to 1/ln 2
+  const double kLn2Hi = 0x1.62e42fefa39efp-1;   // nearest binary64 to ln 2
+  const double kLn2Lo = 0x1.abc9e3b39803fp-56;  // nearest binary64 to ln 2 − kLn2Hi
+  // 1/j! for j = 0..13, each the correctly rounded quotient (j! is exact in binary64).
+  const double c[14] = {1.0 / 1.0,         1.0 / 1.0,          1.0 / 2.0,
+                        1.0 / 6.0,         1.0 / 24.0,         1.0 / 120.0,
+                        1.0 / 720.0,       1.0 / 5040.0,       1.0 / 40320.0,
+                        1.0 / 362880.0,    1.0 / 3628800.0,    1.0 / 39916800.0,
+                        1.0 / 479001600.0, 1.0 / 6227020800.0};
+  const double k = rint(__dmul_rn(x, kInvLn2));
+  double t = __fma_rn(-k, kLn2Hi, x);
+  t = __fma_rn(-k, kLn2Lo, t);
+  double p = c[13];
+#pragma unroll
+  for (int j = 12; j >= 0; --j) p = __fma_rn(p, t, c[j]);
+  // k in [-1010, 0]: 2^k is a normal binary64 number, so the product is exact.
+  const double two_k = __longlong_as_double((long long)((int)k + 1023) << 52);
+  return __dmul_rn(p, two_k);
+}
+
+// ------------------------------------------------------------------ pooling (step 1a)
+
+// Chunk sums of the MEAN rule: one thread per (chunk of B rows, two columns), rows summed
+// sequentially from +0 in row order.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_pool_chunks(const uint16_t *__restrict__ src, float *__restrict__ out, int B,
+                  long long n_chunks) {
+  constexpr int P = D / 2;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long chunk = tid / P;
+  const int t = (int)(tid % P) * 2;
+  if (chunk >= n_chunks) return;
+  const uint32_t *p = reinterpret_cast<const uint32_t *>(src + (size_t)chunk * B * D + t);
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+  for (int e = 0; e < B; ++e) {
+    const uint32_t v = __ldg(p + (size_t)e * P);
+    a0 = __fadd_rn(a0, bf16_lo(v));
+    a1 = __fadd_rn(a1, bf16_hi(v));
+  }
+  *reinterpret_cast<float2 *>(out + (size_t)chunk * D + t) = make_float2(a0, a1);
+}
+
+// Chunk sums added sequentially in chunk order, then divided by the list length.
+__global__ void k_pool_finish(const float *__restrict__ chunks, float *__restrict__ out,
+                              int n_chunks, int D, float len, long long n_out) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= n_out) return;
+  const long long head = tid / D;
+  const int t = (int)(tid % D);
+  const float *p = chunks + (size_t)head * n_chunks * D + t;
+  float acc = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < n_chunks; ++c) acc = __fadd_rn(acc, __ldg(p + (size_t)c * D));
+  out[tid] = __fdiv_rn(acc, len);
+}
+
+// kappa_j = DOT(qbar_h, k_j) for 64 keys of one KV head and all G query heads of its group.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_kappa(const uint16_t *__restrict__ k, const float *__restrict__ qbar,
+            float *__restrict__ kappa, int N, int Hq, int Hkv, int G) {
+  extern __shared__ float smem[];
+  float *ks = smem;                 // [64][D + 1]
+  float *qb = smem + 64 * (D + 1);  // [G][D]
+  const long long kh = blockIdx.y;
+  const int j0 = blockIdx.x * 64;
+  const long long beta = kh / Hkv;
+  const int g = (int)(kh % Hkv);
+  const uint16_t *rows = k + ((size_t)kh * N + j0) * D;
+  for (int x = threadIdx.x; x < 64 * D / 2; x += blockDim.x) {
+    const int r = x / (D / 2), c2 = (x % (D / 2)) * 2;
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(rows + (size_t)r * D + c2));
+    ks[r * (D + 1) + c2] = bf16_lo(v);
+    ks[r * (D + 1) + c2 + 1] = bf16_hi(v);
+  }
+  const size_t qh0 = (size_t)beta * Hq + (size_t)g * G;
+  for (int x = threadIdx.x; x < G * D; x += blockDim.x) qb[x] = qbar[qh0 * D + x];
+  __syncthreads();
+  const int j = threadIdx.x % 64;
+  for (int hi = threadIdx.x / 64; hi < G; hi += blockDim.x / 64) {
+    const float *a = qb + hi * D;
+    const float *b = ks + j * (D + 1);
+    float acc = 0.f;
+#pragma unroll 16
+    for (int t = 0; t < D; ++t) acc = __fmaf_rn(a[t], b[t], acc);
+    kappa[(qh0 + hi) * N + j0 + j] = acc;
+  }
+}
+
+// kbar_top = MEAN of the B top-ranked keys (rank order); u = kbar_top − kbar_all.
+__global__ void k_kbar_top(const uint16_t *__restrict__ k, const int32_t *__restrict__ perm_k,
+                           const float *__restrict__ kbar_all, float *__restrict__ kbar_top,
+                           float *__restrict__ u, int N, int D, int B, int Hq, int Hkv, int G) {
+  const long long qh = blockIdx.x;
+  const long long kh = (qh / Hq) * Hkv + (qh % Hq) / G;
+  const int t = threadIdx.x;
+  float acc = 0.f;
+  for (int e = 0; e < B; ++e) {
+    const int j = __ldg(perm_k + qh * N + e);
+    acc = __fadd_rn(acc, bf16_at(k + ((size_t)kh * N + j) * D + t));
+  }
+  const float top = __fdiv_rn(acc, (float)B);
+  kbar_top[qh * D + t] = top;
+  u[qh * D + t] = __fsub_rn(top, kbar_all[kh * D + t]);
+}
+
+// rho_i = DOT(q_i, u_h) for 128 query rows of one head.
+template <int D>
+__global__ void __launch_bounds__(128)
+    k_rho(const uint16_t *__restrict__ q, const float *__restrict__ u, float *__restrict__ rho,
+          int N) {
+  extern __shared__ float smem[];
+  float *qs = smem;                  // [128][D + 1]
+  float *us = smem + 128 * (D + 1);  // [D]
+  const long long qh = blockIdx.y;
+  const int i0 = blockIdx.x * 128;
+  const int n_rows = min(128, N - i0);
+  const uint16_t *rows = q + ((size_t)qh * N + i0) * D;
+  for (int x = threadIdx.x; x < n_rows * D / 2; x += blockDim.x) {
+    const int r = x / (D / 2), c2 = (x % (D / 2)) * 2;
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(rows + (size_t)r * D + c2));
+    qs[r * (D + 1) + c2] = bf16_lo(v);
+    qs[r * (D + 1) + c2 + 1] = bf16_hi(v);
+  }
+  for (int x = threadIdx.x; x < D; x += blockDim.x) us[x] = u[qh * D + x];
+  __syncthreads();
+  if ((int)threadIdx.x >= n_rows) return;
+  const float *a = qs + threadIdx.x * (D + 1);
+  float acc = 0.f;
+#pragma unroll 16
+  for (int t = 0; t < D; ++t) acc = __fmaf_rn(a[t], us[t], acc);
+  rho[qh * N + i0 + threadIdx.x] = acc;
+}
+
+// ------------------------------------------------------------------ ordering (step 2)
+
+__global__ void k_make_keys(const float *__restrict__ score, unsigned long long *__restrict__ keys,
+                            int N, long long total) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < total) keys[x] = order_word(score[x], (uint32_t)(x % N));
+}
+
+// Sorts each tile of TILE consecutive words of a run in shared memory (bitonic network); the
+// last tile of a run is padded with all-ones words, which sort last.
+template <int TILE>
+__global__ void __launch_bounds__(1024)
+    k_tile_sort(unsigned long long *__restrict__ keys, long long run_len, int tiles_per_run) {
+  __shared__ unsigned long long s[TILE];
+  const long long run = blockIdx.x / tiles_per_run;
+  const long long tile0 = (long long)(blockIdx.x % tiles_per_run) * TILE;
+  const long long begin = run * run_len + tile0;
+  const int n = (int)min((long long)TILE, run_len - tile0);
+  for (int i = threadIdx.x; i < TILE; i += blockDim.x) s[i] = i < n ? keys[begin + i] : ~0ull;
+  __syncthreads();
+  for (int k = 2; k <= TILE; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < TILE; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = s[i], b = s[ixj];
+          if ((a > b) == ((i & k) == 0)) {
+            s[i] = b;
+            s[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[begin + i] = s[i];
+}
+
+__device__ __forceinline__ long long count_less(const unsigned long long *a, long long n,
+                                                unsigned long long key) {
+  long long lo = 0, hi = n;
+  while (lo < hi) {
+    const long long mid = (lo + hi) >> 1;
+    if (a[mid] < key)
+      lo = mid + 1;
+    else
+      hi = mid;
+  }
+  return lo;
+}
+
+// One merge pass: sorted neighbours of `width` words inside each run become sorted pairs. Words
+// are unique, so an element's output slot is its own offset plus the number of smaller words in
+// the other half.
+__global__ void k_merge_pass(const unsigned long long *__restrict__ src,
+                             unsigned long long *__restrict__ dst, long long run_len,
+                             long long width, long long total) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= total) return;
+  const long long run = x / run_len, off = x % run_len;
+  const long long pair0 = off - off % (2 * width);
+  const long long left_n = min(width, run_len - pair0);
+  const long long right_n = max(0LL, min(width, run_len - pair0 - width));
+  const unsigned long long *base = src + run * run_len + pair0;
+  const unsigned long long key = src[x];
+  const long long in_pair = off - pair0;
+  long long pos;
+  if (in_pair < width)
+    pos = in_pair + count_less(base + width, right_n, key);
+  else
+    pos = (in_pair - width) + count_less(base, left_n, key);
+  dst[run * run_len + pair0 + pos] = key;
+}
+
+__global__ void k_extract_perm(const unsigned long long *__restrict__ keys,
+                               int32_t *__restrict__ perm, long long total) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < total) perm[x] = (int32_t)(keys[x] & 0xffffffffull);
+}
+
+__global__ void k_identity_perm(int32_t *__restrict__ perm, int N, long long total) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < total) perm[x] = (int32_t)(x % N);
+}
+
+// ------------------------------------------------------------------ blocks and scores
+
+// Block means over permuted blocks: out[(qh·nB + blk)] = MEAN(rows perm[blk·B .. blk·B+B-1]) of
+// source head src_head(qh) (the query head itself, or its KV head when kv_map is set).
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_block_means(const uint16_t *__restrict__ src, const int32_t *__restrict__ perm,
+                  float *__restrict__ out, int N, int B, int nB, long long n_blocks, int Hq,
+                  int Hkv, int G, int kv_map) {
+  constexpr int P = D / 2;
+  constexpr int PER = 256 / P;
+  const long long blk = (long long)blockIdx.x * PER + threadIdx.x / P;
+  const int t = (threadIdx.x % P) * 2;
+  if (blk >= n_blocks) return;
+  const long long qh = blk / nB;
+  const int b = (int)(blk % nB);
+  const long long sh = kv_map ? (qh / Hq) * Hkv + (qh % Hq) / G : qh;
+  const int32_t *pp = perm + qh * N + (size_t)b * B;
+  const uint16_t *base = src + (size_t)sh * N * D + t;
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+  for (int e = 0; e < B; ++e) {
+    const int row = __ldg(pp + e);
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(base + (size_t)row * D));
+    a0 = __fadd_rn(a0, bf16_lo(v));
+    a1 = __fadd_rn(a1, bf16_hi(v));
+  }
+  const float len = (float)B;
+  *reinterpret_cast<float2 *>(out + (size_t)blk * D + t) =
+      make_float2(__fdiv_rn(a0, len), __fdiv_rn(a1, len));
+}
+
+// n[qh][s][c] = number of keys of permuted key block c whose original index is below s·S.
+__global__ void __launch_bounds__(256)
+    k_ncount(const int32_t *__restrict__ perm_k, int32_t *__restrict__ n, int N, int B, int S,
+             int nB, int nSeg) {
+  extern __shared__ int seg_of[];  // [32][B + 1]
+  const long long qh = blockIdx.y;
+  const int c0 = blockIdx.x * 32;
+  for (int x = threadIdx.x; x < 32 * B; x += blockDim.x) {
+    const int cl = x / B, e = x % B, c = c0 + cl;
+    seg_of[cl * (B + 1) + e] = c < nB ? __ldg(perm_k + qh * N + (size_t)c * B + e) / S : INT_MAX;
+  }
+  __syncthreads();
+  const int cl = threadIdx.x % 32, c = c0 + cl;
+  if (c >= nB) return;
+  const int *mine = seg_of + cl * (B + 1);
+  for (int s = threadIdx.x / 32; s < nSeg; s += blockDim.x / 32) {
+    int cnt = 0;
+    for (int e = 0; e < B; ++e) cnt += mine[e] < s;
+    n[((size_t)qh * nSeg + s) * nB + c] = cnt;
+  }
+}
+
+// r[qh][b][c] = DOT(Qbar_b, Kbar_c) × σ_d: a register-tiled fp32 product whose accumulators
+// each run the definition's sequential FMA chain over t = 0..D-1.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_block_scores(const float *__restrict__ Qbar, const float *__restrict__ Kbar,
+                   float *__restrict__ r, int nB, float sigma) {
+  __shared__ __align__(16) float As[32][128 + 4];
+  __shared__ __align__(16) float Bs[32][128 + 4];
+  const long long qh = blockIdx.z;
+  const int b0 = blockIdx.y * 128, c0 = blockIdx.x * 128;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  const float *A = Qbar + (size_t)qh * nB * D;
+  const float *Bm = Kbar + (size_t)qh * nB * D;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int t0 = 0; t0 < D; t0 += 32) {
+    for (int x = threadIdx.x; x < 128 * 32; x += 256) {
+      const int row = x / 32, tt = x % 32;
+      As[tt][row] = b0 + row < nB ? A[(size_t)(b0 + row) * D + t0 + tt] : 0.f;
+      Bs[tt][row] = c0 + row < nB ? Bm[(size_t)(c0 + row) * D + t0 + tt] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int tt = 0; tt < 32; ++tt) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[tt][tr * 8]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[tt][tr * 8 + 4]);
+      const float4 v0 = *reinterpret_cast<const float4 *>(&Bs[tt][tc * 8]);
+      const float4 v1 = *reinterpret_cast<const float4 *>(&Bs[tt][tc * 8 + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(a[i], v[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = b0 + tr * 8 + i;
+    if (b >= nB) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + tc * 8 + j;
+      if (c < nB) r[((size_t)qh * nB + b) * nB + c] = __fmul_rn(acc[i][j], sigma);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ scheduling (step 4 order)
+
+__device__ __forceinline__ bool goes_before(double pa, int ca, double pb, int cb) {
+  return pa > pb || (pa == pb && ca < cb);
+}
+
+// One warp per query block: local tile count, normalised block scores p over the candidate
+// blocks, selection p >= τ, and the list sorted by (p descending, block ascending).
+__global__ void __launch_bounds__(128)
+    k_schedule(const float *__restrict__ r, const int32_t *__restrict__ ncount,
+               const int32_t *__restrict__ perm_q, int32_t *__restrict__ sel_cnt,
+               int32_t *__restrict__ sel_blk, int32_t *__restrict__ local_tiles, int N, int B,
+               int S, int nB, int nSeg, int P2, double tau, long long n_qblocks) {
+  extern __shared__ unsigned char smem_raw[];
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const long long qb = (long long)blockIdx.x * (blockDim.x / kWarp) + warp;
+  if (qb >= n_qblocks) return;
+  const size_t per_warp = ((size_t)nB * 8 + (size_t)P2 * 12 + 15) & ~(size_t)15;
+  double *w = reinterpret_cast<double *>(smem_raw + per_warp * warp);
+  double *lp = w + nB;
+  int *lc = reinterpret_cast<int *>(lp + P2);
+
+  const long long qh = qb / nB;
+  const int b = (int)(qb % nB);
+  const int s = (int)((long long)b * B / S);
+  const unsigned full = 0xffffffffu;
+
+  int mx = -1;
+  for (int e = lane; e < B; e += kWarp) mx = max(mx, __ldg(perm_q + qh * N + (size_t)b * B + e));
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(full, mx, o));
+  if (lane == 0) local_tiles[qb] = (mx - s * S) / B + 1;
+
+  const float *rr = r + (size_t)qb * nB;
+  const int32_t *nn = ncount + ((size_t)qh * nSeg + s) * nB;
+
+  // M = max block score over the candidates (blocks with a visible key).
+  float M = 0.f;
+  bool any = false;
+  for (int c = lane; c < nB; c += kWarp) {
+    if (__ldg(nn + c) > 0) {
+      const float x = __ldg(rr + c);
+      M = any ? fmaxf(M, x) : x;
+      any = true;
+    }
+  }
+  const unsigned have = __ballot_sync(full, any);
+  if (have == 0) {
+    if (lane == 0) sel_cnt[qb] = 0;
+    return;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    const float other = __shfl_xor_sync(full, M, o);
+    const bool other_any = __shfl_xor_sync(full, any ? 1 : 0, o) != 0;
+    if (other_any) M = any ? fmaxf(M, other) : other;
+    any = any || other_any;
+  }
+
+  // Weights w_c and their sum Z: chunks of 32 consecutive blocks (chunk k is summed by lane
+  // k mod 32 sequentially), then the chunk sums in chunk order.
+  const int n_chunks = (nB + 31) / 32;
+  double part0 = 0.0, part1 = 0.0;  // this lane's chunks k = lane and k = lane + 32
+  for (int k = lane; k < n_chunks; k += kWarp) {
+    double part = 0.0;
+    const int c_end = min(nB, 32 * k + 32);
+    for (int c = 32 * k; c < c_end; ++c) {
+      const int nv = __ldg(nn + c);
+      const double wc =
+          nv > 0 ? __dmul_rn((double)nv, exp64(__dsub_rn((double)__ldg(rr + c), (double)M)))
+                 : 0.0;
+      w[c] = wc;
+      part = __dadd_rn(part, wc);
+    }
+    if (k < kWarp)
+      part0 = part;
+    else
+      part1 = part;
+  }
+  double Z = 0.0;
+  for (int k = 0; k < n_chunks; ++k) {
+    const double v = __shfl_sync(full, k < kWarp ? part0 : part1, k % kWarp);
+    Z = __dadd_rn(Z, v);
+  }
+  __syncwarp();
+
+  // Selection p_c = w_c / Z >= τ, compacted through a warp prefix count.
+  int mine = 0;
+  for (int k = lane; k < n_chunks; k += kWarp) {
+    const int c_end = min(nB, 32 * k + 32);
+    for (int c = 32 * k; c < c_end; ++c)
+      if (__ldg(nn + c) > 0 && __ddiv_rn(w[c], Z) >= tau) ++mine;
+  }
+  int incl = mine;
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const int v = __shfl_up_sync(full, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int cnt = __shfl_sync(full, incl, kWarp - 1);
+  int slot = incl - mine;
+  for (int k = lane; k < n_chunks; k += kWarp) {
+    const int c_end = min(nB, 32 * k + 32);
+    for (int c = 32 * k; c < c_end; ++c) {
+      if (__ldg(nn + c) > 0) {
+        const double p = __ddiv_rn(w[c], Z);
+        if (p >= tau) {
+          lp[slot] = p;
+          lc[slot] = c;
+          ++slot;
+        }
+      }
+    }
+  }
+  int P = 1;
+  while (P < cnt) P <<= 1;
+  for (int e = cnt + lane; e < P; e += kWarp) {
+    lp[e] = -1.0;
+    lc[e] = INT_MAX;
+  }
+  __syncwarp();
+  // Bitonic network over P entries, order "goes_before".
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = lane; i < P; i += kWarp) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const bool up = (i & k) == 0;
+          const bool after = goes_before(lp[ixj], lc[ixj], lp[i], lc[i]);
+          if (after == up) {
+            const double tp = lp[i];
+            const int tcb = lc[i];
+            lp[i] = lp[ixj];
+            lc[i] = lc[ixj];
+            lp[ixj] = tp;
+            lc[ixj] = tcb;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+  int32_t *dst = sel_blk + (size_t)qb * nB;
+  for (int e = lane; e < cnt; e += kWarp) dst[e] = lc[e];
+  if (lane == 0) sel_cnt[qb] = cnt;
+}
+
+// ------------------------------------------------------------------ validation and stats
+
+__global__ void k_validate_perms(const int32_t *__restrict__ perm_q,
+                                 const int32_t *__restrict__ perm_k,
+                                 unsigned *__restrict__ seen_q, unsigned *__restrict__ seen_k,
+                                 int N, int S, long long total, unsigned *__restrict__ flag) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= total) return;
+  const long long qh = x / N;
+  const int slot = (int)(x % N);
+  const int s0 = (slot / S) * S;
+  const int iq = perm_q[x], ik = perm_k[x];
+  if (iq < s0 || iq >= s0 + S) {
+    atomicOr(flag, 1u);
+  } else {
+    const long long bit = qh * N + iq;
+    if (atomicOr(seen_q + bit / 32, 1u << (bit % 32)) & (1u << (bit % 32))) atomicOr(flag, 2u);
+  }
+  if (ik < 0 || ik >= N) {
+    atomicOr(flag, 4u);
+  } else {
+    const long long bit = qh * N + ik;
+    if (atomicOr(seen_k + bit / 32, 1u << (bit % 32)) & (1u << (bit % 32))) atomicOr(flag, 8u);
+  }
+}
+
+// One warp per query block: list length, block ids in range and unique, local tile count in
+// range and covering the block's last query (when perm_q is in range).
+__global__ void __launch_bounds__(128)
+    k_validate_lists(const int32_t *__restrict__ perm_q, const int32_t *__restrict__ sel_cnt,
+                     const int32_t *__restrict__ sel_blk, const int32_t *__restrict__ local_tiles,
+                     int N, int B, int S, int nB, long long n_qblocks, unsigned *__restrict__ flag) {
+  extern __shared__ unsigned bits[];  // per warp: (nB + 31) / 32 words
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const long long qb = (long long)blockIdx.x * (blockDim.x / kWarp) + warp;
+  if (qb >= n_qblocks) return;
+  const int words = (nB + 31) / 32;
+  unsigned *mine = bits + warp * words;
+  for (int e = lane; e < words; e += kWarp) mine[e] = 0u;
+  __syncwarp();
+  const long long qh = qb / nB;
+  const int b = (int)(qb % nB);
+  const int s0 = (int)((long long)b * B / S) * S;
+  const int cnt = sel_cnt[qb];
+  if (cnt < 0 || cnt > nB) {
+    if (lane == 0) atomicOr(flag, 16u);
+  } else {
+    for (int e = lane; e < cnt; e += kWarp) {
+      const int c = sel_blk[qb * nB + e];
+      if (c < 0 || c >= nB) {
+        atomicOr(flag, 32u);
+      } else if (atomicOr(mine + c / 32, 1u << (c % 32)) & (1u << (c % 32))) {
+        atomicOr(flag, 64u);
+      }
+    }
+  }
+  int mx = -1;
+  for (int e = lane; e < B; e += kWarp) mx = max(mx, perm_q[qh * N + (size_t)b * B + e]);
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) {
+    const int lt = local_tiles[qb];
+    if (lt < 1 || lt > S / B) atomicOr(flag, 128u);
+    if (mx >= s0 && mx < s0 + S && lt < (mx - s0) / B + 1) atomicOr(flag, 256u);
+  }
+}
+
+// acc[0] += Σ lt, acc[1] += Σ cnt, acc[2] += Σ_i |K_i| (local keys plus visible keys of the
+// listed blocks), one warp per query block.
+__global__ void __launch_bounds__(128)
+    k_stats(const int32_t *__restrict__ perm_q, const int32_t *__restrict__ perm_k,
+            const int32_t *__restrict__ sel_cnt, const int32_t *__restrict__ sel_blk,
+            const int32_t *__restrict__ local_tiles, int N, int B, int S, int nB,
+            long long n_qblocks, unsigned long long *__restrict__ acc) {
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const long long qb = (long long)blockIdx.x * (blockDim.x / kWarp) + warp;
+  if (qb >= n_qblocks) return;
+  const long long qh = qb / nB;
+  const int b = (int)(qb % nB);
+  const int s0 = (int)((long long)b * B / S) * S;
+  const int cnt = min(max(sel_cnt[qb], 0), nB);
+  unsigned long long local_pairs = 0, visible = 0;
+  for (int e = lane; e < B; e += kWarp) local_pairs += perm_q[qh * N + (size_t)b * B + e] - s0 + 1;
+  for (int x = 0; x < cnt; ++x) {
+    const int c = min(max(sel_blk[qb * nB + x], 0), nB - 1);
+    for (int e = lane; e < B; e += kWarp) visible += perm_k[qh * N + (size_t)c * B + e] < s0;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    local_pairs += __shfl_xor_sync(0xffffffffu, local_pairs, o);
+    visible += __shfl_xor_sync(0xffffffffu, visible, o);
+  }
+  if (lane == 0) {
+    atomicAdd(acc + 0, (unsigned long long)local_tiles[qb]);
+    atomicAdd(acc + 1, (unsigned long long)cnt);
+    atomicAdd(acc + 2, local_pairs + visible * (unsigned long long)B);
+  }
+}
+
+__global__ void k_exp64_probe(const double *x, double *y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp64(x[i]);
+}
+
+inline unsigned blocks_for(long long n, int per) { return (unsigned)((n + per - 1) / per); }
+
+cudaError_t sort_runs(unsigned long long *a, unsigned long long *b, long long total,
+                      long long run_len, int32_t *perm_out, cudaStream_t st) {
+  // Tile size: the smallest of 1024 / 2048 / 4096 that covers a run, capped at 4096.
+  const int tile = run_len <= 1024 ? 1024 : run_len <= 2048 ? 2048 : 4096;
+  const int tiles_per_run = (int)((run_len + tile - 1) / tile);
+  const unsigned grid = (unsigned)((total / run_len) * tiles_per_run);
+  if (tile == 1024)
+    k_tile_sort<1024><<<grid, 512, 0, st>>>(a, run_len, tiles_per_run);
+  else if (tile == 2048)
+    k_tile_sort<2048><<<grid, 1024, 0, st>>>(a, run_len, tiles_per_run);
+  else
+    k_tile_sort<4096><<<grid, 1024, 0, st>>>(a, run_len, tiles_per_run);
+    note_launch();
+  unsigned long long *src = a, *dst = b;
+  for (long long width = tile; width < run_len; width *= 2) {
+    k_merge_pass<<<blocks_for(total, 256), 256, 0, st>>>(src, dst, run_len, width, total);
+    note_launch();
+    unsigned long long *t = src;
+    src = dst;
+    dst = t;
+  }
+  k_extract_perm<<<blocks_for(total, 256), 256, 0, st>>>(src, perm_out, total);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, const uint16_t *k,
+                    const s2o_indices &out, char *ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(d);
+  float *qchunk = reinterpret_cast<float *>(ws + L.qchunk);
+  float *kchunk = reinterpret_cast<float *>(ws + L.kchunk);
+  float *qbar = reinterpret_cast<float *>(ws + L.qbar);
+  float *kbar_all = reinterpret_cast<float *>(ws + L.kbar_all);
+  float *kbar_top = reinterpret_cast<float *>(ws + L.kbar_top);
+  float *u = reinterpret_cast<float *>(ws + L.u);
+  float *kappa = reinterpret_cast<float *>(ws + L.kappa);
+  float *rho = reinterpret_cast<float *>(ws + L.rho);
+  unsigned long long *keys0 = reinterpret_cast<unsigned long long *>(ws + L.keys0);
+  unsigned long long *keys1 = reinterpret_cast<unsigned long long *>(ws + L.keys1);
+  float *Qbar = reinterpret_cast<float *>(ws + L.Qbar);
+  float *Kbar = reinterpret_cast<float *>(ws + L.Kbar);
+  float *r = reinterpret_cast<float *>(ws + L.r);
+  int32_t *ncount = reinterpret_cast<int32_t *>(ws + L.ncount);
+
+  const long long bhq = d.bhq(), bhkv = d.bhkv();
+  const long long nq = bhq * d.N, nkv_rows = bhkv * d.N;
+  cudaError_t e;
+
+  // Step 1a: mean query per query head, mean key per KV head, kappa.
+  k_pool_chunks<D><<<blocks_for(nq / d.B * (D / 2), 256), 256, 0, st>>>(q, qchunk, d.B, nq / d.B);
+  note_launch();
+  k_pool_chunks<D><<<blocks_for(nkv_rows / d.B * (D / 2), 256), 256, 0, st>>>(k, kchunk, d.B,
+                                                                               nkv_rows / d.B);
+  note_launch();
+  k_pool_finish<<<blocks_for(bhq * D, 256), 256, 0, st>>>(qchunk, qbar, d.nB, D, (float)d.N,
+                                                          bhq * D);
+  note_launch();
+  k_pool_finish<<<blocks_for(bhkv * D, 256), 256, 0, st>>>(kchunk, kbar_all, d.nB, D, (float)d.N,
+                                                           bhkv * D);
+  note_launch();
+  const size_t kappa_smem = (64 * (D + 1) + (size_t)d.G * D) * sizeof(float);
+  if ((e = cudaFuncSetAttribute(k_kappa<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kappa_smem)) != cudaSuccess)
+    return e;
+  k_kappa<D><<<dim3(d.N / 64, (unsigned)bhkv), 256, kappa_smem, st>>>(k, qbar, kappa, d.N, d.Hq,
+                                                                       d.Hkv, d.G);
+  note_launch();
+  // Step 2a: global key/value ordering.
+  k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(kappa, keys0, d.N, nq);
+  note_launch();
+  if ((e = sort_runs(keys0, keys1, nq, d.N, out.perm_k, st)) != cudaSuccess) return e;
+  // Step 1b: query scores against the top stripe block.
+  k_kbar_top<<<(unsigned)bhq, D, 0, st>>>(k, out.perm_k, kbar_all, kbar_top, u, d.N, D, d.B, d.Hq,
+                                          d.Hkv, d.G);
+  note_launch();
+  const size_t rho_smem = (128 * (D + 1) + D) * sizeof(float);
+  if ((e = cudaFuncSetAttribute(k_rho<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)rho_smem)) != cudaSuccess)
+    return e;
+  k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, rho_smem, st>>>(q, u, rho, d.N);
+  note_launch();
+  // Step 2b: segment-local query ordering.
+  if (cfg.query_perm) {
+    k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(rho, keys0, d.N, nq);
+    note_launch();
+    if ((e = sort_runs(keys0, keys1, nq, d.S, out.perm_q, st)) != cudaSuccess) return e;
+  } else {
+    k_identity_perm<<<blocks_for(nq, 256), 256, 0, st>>>(out.perm_q, d.N, nq);
+    note_launch();
+  }
+  // Block means, visibility counts, block scores.
+  const long long nblk = bhq * d.nB;
+  constexpr int PER = 256 / (D / 2);
+  k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
+                                                          nblk, d.Hq, d.Hkv, d.G, 0);
+  note_launch();
+  k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(k, out.perm_k, Kbar, d.N, d.B, d.nB,
+                                                          nblk, d.Hq, d.Hkv, d.G, 1);
+  note_launch();
+  const size_t nc_smem = (size_t)32 * (d.B + 1) * sizeof(int);
+  k_ncount<<<dim3((d.nB + 31) / 32, (unsigned)bhq), 256, nc_smem, st>>>(out.perm_k, ncount, d.N,
+                                                                        d.B, d.S, d.nB, d.nSeg);
+  note_launch();
+  const float sigma = D == 64 ? 0x1p-3f : 0x1.6a09e6p-4f;  // nearest fp32 to 1/sqrt(D)
+  const unsigned tiles = (unsigned)((d.nB + 127) / 128);
+  k_block_scores<D><<<dim3(tiles, tiles, (unsigned)bhq), 256, 0, st>>>(Qbar, Kbar, r, d.nB, sigma);
+  note_launch();
+  // Scheduling.
+  int P2 = 1;
+  while (P2 < d.nB) P2 <<= 1;
+  const size_t per_warp = ((size_t)d.nB * 8 + (size_t)P2 * 12 + 15) & ~(size_t)15;
+  const int warps = (int)std::max<size_t>(1, std::min<size_t>(4, (200u << 10) / per_warp));
+  const size_t sched_smem = per_warp * warps;
+  if ((e = cudaFuncSetAttribute(k_schedule, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sched_smem)) != cudaSuccess)
+    return e;
+  k_schedule<<<blocks_for(nblk, warps), warps * kWarp, sched_smem, st>>>(
+      r, ncount, out.perm_q, out.sel_cnt, out.sel_blk, out.local_tiles, d.N, d.B, d.S, d.nB,
+      d.nSeg, P2, (double)cfg.tau, nblk);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_build_indices(const Dims &d, const s2o_config &cfg, const uint16_t *q,
+                                 const uint16_t *k, const s2o_indices &out, char *ws,
+                                 cudaStream_t st) {
+  return d.D == 64 ? build_d<64>(d, cfg, q, k, out, ws, st) : build_d<128>(d, cfg, q, k, out, ws, st);
+}
+
+cudaError_t launch_validate(const Dims &d, const s2o_indices &idx, char *ws, uint32_t *flag_dev,
+                            cudaStream_t st) {
+  const WsLayout L = ws_layout(d);
+  const long long total = d.bhq() * d.N;
+  const size_t words = (size_t)((total + 31) / 32);
+  unsigned *seen_q = reinterpret_cast<unsigned *>(ws + L.keys0);
+  unsigned *seen_k = seen_q + words;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(seen_q, 0, 2 * words * sizeof(unsigned), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(flag_dev, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+  k_validate_perms<<<blocks_for(total, 256), 256, 0, st>>>(idx.perm_q, idx.perm_k, seen_q, seen_k,
+                                                           d.N, d.S, total, flag_dev);
+  note_launch();
+  const long long nblk = d.bhq() * d.nB;
+  const size_t smem = (size_t)4 * ((d.nB + 31) / 32) * sizeof(unsigned);
+  k_validate_lists<<<blocks_for(nblk, 4), 128, smem, st>>>(idx.perm_q, idx.sel_cnt, idx.sel_blk,
+                                                           idx.local_tiles, d.N, d.B, d.S, d.nB,
+                                                           nblk, flag_dev);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats(const Dims &d, const s2o_indices &idx, unsigned long long *acc_dev,
+                         cudaStream_t st) {
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(acc_dev, 0, 3 * sizeof(unsigned long long), st)) != cudaSuccess)
+    return e;
+  const long long nblk = d.bhq() * d.nB;
+  k_stats<<<blocks_for(nblk, 4), 128, 0, st>>>(idx.perm_q, idx.perm_k, idx.sel_cnt, idx.sel_blk,
+                                               idx.local_tiles, d.N, d.B, d.S, d.nB, nblk,
+                                               acc_dev);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_exp64_probe(const double *x, double *y, int n, cudaStream_t st) {
+  k_exp64_probe<<<blocks_for(n, 256), 256, 0, st>>>(x, y, n);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace s2o

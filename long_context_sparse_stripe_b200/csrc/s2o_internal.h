@@ -1,0 +1,56 @@
+// Internal declarations shared by the host API and the kernels of libs2o.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "s2o.h"
+
+namespace s2o {
+
+// Derived sizes of one configuration.
+struct Dims {
+  int batch, Hq, Hkv, G, N, D, S, B, nB, nSeg;
+  long long bhq() const { return (long long)batch * Hq; }
+  long long bhkv() const { return (long long)batch * Hkv; }
+};
+
+Dims dims_of(const s2o_config &c);
+
+// Byte offsets of the scratch arrays inside a workspace (256-byte aligned).
+struct WsLayout {
+  size_t qchunk, kchunk, qbar, kbar_all, kbar_top, u, kappa, rho, keys0, keys1, Qbar, Kbar, r,
+      ncount, flags, total;
+};
+
+WsLayout ws_layout(const Dims &d);
+
+// Index build (s2o_index.cu). All launches on `st`; returns the first launch error.
+cudaError_t launch_build_indices(const Dims &d, const s2o_config &cfg, const uint16_t *q,
+                                 const uint16_t *k, const s2o_indices &out, char *ws,
+                                 cudaStream_t st);
+cudaError_t launch_validate(const Dims &d, const s2o_indices &idx, char *ws, uint32_t *flag_dev,
+                            cudaStream_t st);
+cudaError_t launch_stats(const Dims &d, const s2o_indices &idx, unsigned long long *acc_dev,
+                         cudaStream_t st);
+cudaError_t launch_exp64_probe(const double *x, double *y, int n, cudaStream_t st);
+
+// Attention (s2o_attn.cu).
+struct AttnArgs {
+  const void *q, *k, *v;
+  void *o;
+  const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
+  bool dense;
+};
+cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
+                             cudaStream_t st);
+
+// Host-side count of kernel launches made by the library (all threads, all devices).
+void note_launch();
+unsigned long long launch_count();
+
+// Device error record (bit 0: a bounded wait ran out).
+cudaError_t read_and_clear_device_error(unsigned int *out, cudaStream_t st);
+
+}  // namespace s2o

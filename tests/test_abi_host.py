@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every function that
+``include/s2o.h`` declares, sizes its buffers as documented and rejects bad arguments before
+enqueueing any device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_sparse_stripe_b200 as s2o
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "s2o.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(s2o_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = s2o._load()
+    names = declared_functions()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_library_is_the_in_tree_build():
+    path = s2o.library_path()
+    assert os.path.isfile(path)
+    assert os.path.dirname(path) == os.path.dirname(os.path.abspath(s2o.__file__))
+
+
+def test_status_strings():
+    lib = s2o._load()
+    for code, name in s2o.STATUS.items():
+        assert lib.s2o_status_string(code).decode() == name
+    assert lib.s2o_status_string(99).decode() == "S2O_ERR_UNKNOWN"
+
+
+LLAMA_128K = s2o.Config(1, 32, 8, 131072, 128, 2048, 128, 0.01)
+
+
+def test_index_sizes_and_workspace_are_documented_shapes():
+    cfg = LLAMA_128K
+    nB = 1024
+    assert s2o.index_sizes(cfg) == [32 * 131072, 32 * 131072, 32 * nB, 32 * nB * nB, 32 * nB]
+    ws = s2o.workspace_size(cfg)
+    # kappa/rho/keys (2 x 8-byte) per query slot, Qbar/Kbar/chunks, block scores and counts
+    lower = 32 * 131072 * (4 + 4 + 16) + 32 * nB * nB * 4 + 32 * 64 * nB * 4
+    assert lower <= ws <= lower + 96 * 2**20
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 96, 2), ("block_size", 32, 2), ("n_kv_heads", 3, 2), ("segment_len", 192, 2),
+    ("seq_len", 131072 + 2048 * 0 + 64, 2), ("tau", -0.1, 1), ("tau", float("nan"), 1),
+    ("tau", float("inf"), 1), ("batch", 0, 1), ("query_perm", 2, 1),
+])
+def test_bad_config_rejected(field, value, code):
+    cfg = s2o.Config(**{**LLAMA_128K.__dict__, field: value})
+    n = ctypes.c_size_t(0)
+    assert s2o._load().s2o_workspace_size(ctypes.byref(cfg._c()), ctypes.byref(n)) == code
+
+
+def test_tau_above_one_is_legal():
+    cfg = s2o.Config(**{**LLAMA_128K.__dict__, "tau": 1.5})
+    assert s2o.workspace_size(cfg) > 0
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch():
+    lib = s2o._load()
+    c = LLAMA_128K._c()
+    idx = s2o._Indices(0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+    # null q
+    assert lib.s2o_build_indices(ctypes.byref(c), None, 0x1000, ctypes.byref(idx), 0x1000,
+                                 1 << 40, None) == 1
+    # misaligned k
+    assert lib.s2o_build_indices(ctypes.byref(c), 0x1000, 0x1008, ctypes.byref(idx), 0x1000,
+                                 1 << 40, None) == 1
+    # null index array
+    bad = s2o._Indices(0x1000, 0, 0x3000, 0x4000, 0x5000)
+    assert lib.s2o_build_indices(ctypes.byref(c), 0x1000, 0x1000, ctypes.byref(bad), 0x1000,
+                                 1 << 40, None) == 1
+    assert lib.s2o_attention_prefill_with_indices(ctypes.byref(c), 0x1000, 0x1000, None,
+                                                  ctypes.byref(idx), 0x1000, None) == 1
+    assert lib.s2o_dense_causal_prefill(ctypes.byref(c), 0x1000, 0x1000, 0x1000, None, None) == 1
+    assert lib.s2o_exp64_eval(None, None, 4, None) == 1
+
+
+def test_workspace_too_small_rejected_before_launch():
+    lib = s2o._load()
+    c = LLAMA_128K._c()
+    idx = s2o._Indices(0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+    need = s2o.workspace_size(LLAMA_128K)
+    assert lib.s2o_build_indices(ctypes.byref(c), 0x1000, 0x1000, ctypes.byref(idx), 0x1000,
+                                 need - 1, None) == 3
+    assert lib.s2o_attention_prefill(ctypes.byref(c), 0x1000, 0x1000, 0x1000, 0x1000,
+                                     ctypes.byref(idx), 0x1000, need - 1, None) == 3
+    assert lib.s2o_validate_indices(ctypes.byref(c), ctypes.byref(idx), 0x1000, need - 1,
+                                    None) == 3
+    st = s2o._Stats()
+    assert lib.s2o_index_stats(ctypes.byref(c), ctypes.byref(idx), 0x1000, need - 1,
+                               ctypes.byref(st), None) == 3
+
+
+def test_workspace_views_are_inside_the_workspace():
+    cfg = LLAMA_128K
+    need = s2o.workspace_size(cfg)
+    view = s2o._View()
+    base = 1 << 32
+    assert s2o._load().s2o_workspace_views(ctypes.byref(cfg._c()), base, need,
+                                           ctypes.byref(view)) == 0
+    ptrs = [getattr(view, f) for f, _ in s2o._View._fields_]
+    assert all(base <= p < base + need for p in ptrs)
+    assert len(set(ptrs)) == len(ptrs)

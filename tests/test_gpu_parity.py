@@ -1,0 +1,257 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on the same seeded inputs.
+
+Index arrays and every intermediate value of the index build must be bit-exact; attention
+outputs must be within max-abs 2e-2 and mean-abs 1e-3 of the oracle's binary64 result when run
+on the oracle's own indices (bf16 tensor-core products with fp32 accumulation against binary64).
+"""
+import numpy as np
+import pytest
+import torch
+
+import gen
+import long_context_sparse_stripe_b200 as s2o
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS = 2e-2, 1e-3
+
+W_A = gen.Workload("a-d128-b128", batch=1, n_q_heads=4, n_kv_heads=2, seq_len=4096, head_dim=128,
+                   segment_len=1024, block_size=128, tau=0.01, seed=5)
+# Ragged: N is not a power of two (the key sort's last merge pairs 8192 with 4096 words) and S is
+# not a multiple of the 2048-word segment sort tile; two batch elements.
+W_B = gen.Workload("b-ragged", batch=2, n_q_heads=4, n_kv_heads=2, seq_len=12288, head_dim=128,
+                   segment_len=1536, block_size=128, tau=0.01, seed=6)
+W_C = gen.Workload("c-d64-b128", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=2048, head_dim=64,
+                   segment_len=512, block_size=128, tau=0.02, seed=8)
+W_D = gen.Workload("d-d128-b64", batch=1, n_q_heads=2, n_kv_heads=2, seq_len=2048, head_dim=128,
+                   segment_len=512, block_size=64, tau=0.02, seed=9)
+W_TINY = gen.workload("tiny")
+
+INDEX_NAMES = ("perm_q", "perm_k", "sel_cnt", "local_tiles")
+VIEW_NAMES = ("qbar", "kbar_all", "kbar_top", "u", "kappa", "rho", "Qbar", "Kbar", "r", "n")
+
+_inputs_cache = {}
+
+
+def inputs(w):
+    key = (w.name, w.seed, w.seq_len, w.batch)
+    if key not in _inputs_cache:
+        _inputs_cache.clear()
+        _inputs_cache[key] = gen.make_inputs(w)
+    return _inputs_cache[key]
+
+
+def to_dev(*ts):
+    return [t.cuda() for t in ts]
+
+
+def gpu_indices(w, q, k):
+    cfg = s2o.Config.of(w)
+    ws = s2o.alloc_workspace(cfg)
+    idx = s2o.build_indices(cfg, q, k, ws=ws)
+    torch.cuda.synchronize()
+    return cfg, idx, ws
+
+
+def assert_indices_equal(idx, ref, nB):
+    for name in INDEX_NAMES:
+        got = getattr(idx, name).cpu().numpy()
+        np.testing.assert_array_equal(got, ref[name], err_msg=name)
+    cnt = ref["sel_cnt"]
+    sel = idx.sel_blk.cpu().numpy()
+    mask = np.arange(nB)[None, None, None, :] < cnt[..., None]
+    np.testing.assert_array_equal(np.where(mask, sel, -1), ref["sel_blk"], err_msg="sel_blk")
+
+
+def oracle_indices_on_device(ref):
+    return s2o.Indices(*(torch.from_numpy(np.ascontiguousarray(ref[n])).cuda()
+                         for n in ("perm_q", "perm_k", "sel_cnt", "sel_blk", "local_tiles")))
+
+
+def assert_close(got_bf16, want_f64):
+    got = got_bf16.float().cpu().numpy().astype(np.float64).reshape(want_f64.shape)
+    err = np.abs(got - want_f64)
+    assert err.max() <= MAX_ABS, f"max abs error {err.max():.3g}"
+    assert err.mean() <= MEAN_ABS, f"mean abs error {err.mean():.3g}"
+
+
+# ----------------------------------------------------------------------------- exp64
+
+def test_exp64_bit_exact_with_oracle():
+    xs = np.concatenate([-np.linspace(0, 720, 40001), -np.geomspace(1e-300, 50, 4001),
+                         [0.0, -0.0, -699.9999, -700.0, -700.0000001]])
+    got = s2o.exp64_eval(torch.from_numpy(xs).cuda()).cpu().numpy()
+    want = np.array([oracle.exp64(x) for x in xs])
+    np.testing.assert_array_equal(got.view(np.uint64), want.view(np.uint64))
+
+
+# ----------------------------------------------------------------------------- index build
+
+@pytest.mark.parametrize("w", [
+    W_TINY, W_TINY.replace(tau=0.0), W_TINY.replace(tau=0.07), W_TINY.replace(tau=0.2),
+    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D,
+], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
+def test_indices_and_intermediates_bit_exact(w):
+    q, k, _ = inputs(w)
+    ref = oracle.build_indices(oracle.config(w), q, k, debug=True)
+    cfg, idx, ws = gpu_indices(w, *to_dev(q, k))
+    assert_indices_equal(idx, ref, cfg.n_blocks)
+    views = s2o.workspace_views(cfg, ws)
+    for name in VIEW_NAMES:
+        got = views[name].cpu().numpy()
+        want = ref[name]
+        np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32), err_msg=name)
+
+
+def test_index_build_is_deterministic():
+    q, k, _ = inputs(W_B)
+    qd, kd = to_dev(q, k)
+    _, a, _ = gpu_indices(W_B, qd, kd)
+    _, b, _ = gpu_indices(W_B, qd, kd)
+    for name in ("perm_q", "perm_k", "sel_cnt", "local_tiles"):
+        assert torch.equal(getattr(a, name), getattr(b, name))
+
+
+# ----------------------------------------------------------------------------- attention
+
+@pytest.mark.parametrize("w", [W_TINY, W_TINY.replace(tau=0.07), W_TINY.replace(tau=1.5), W_A,
+                               W_A.replace(query_perm=0), W_C, W_D],
+                         ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
+def test_attention_on_oracle_indices(w):
+    q, k, v = inputs(w)
+    cfg = oracle.config(w)
+    ref = oracle.build_indices(cfg, q, k)
+    want, _ = oracle.attention(cfg, q, k, v, ref)
+    qd, kd, vd = to_dev(q, k, v)
+    o = s2o.attention_prefill_with_indices(s2o.Config.of(w), qd, kd, vd,
+                                           oracle_indices_on_device(ref))
+    torch.cuda.synchronize()
+    assert s2o.check_device_status() == 0
+    assert_close(o, want)
+
+
+def test_full_path_ragged_sampled_rows():
+    w = W_B
+    q, k, v = inputs(w)
+    cfg = oracle.config(w)
+    ref = oracle.build_indices(cfg, q, k)
+    qd, kd, vd = to_dev(q, k, v)
+    o, idx = s2o.attention_prefill(s2o.Config.of(w), qd, kd, vd)
+    torch.cuda.synchronize()
+    assert_indices_equal(idx, ref, w.seq_len // w.block_size)
+    rng = np.random.default_rng(0)
+    total = w.batch * w.n_q_heads * w.seq_len
+    # every segment's first and last rows plus a random sample
+    edge = [(bh * w.seq_len + s0 + e) for bh in range(w.batch * w.n_q_heads)
+            for s0 in range(0, w.seq_len, w.segment_len) for e in (0, w.segment_len - 1)]
+    rows = np.unique(np.concatenate([rng.choice(total, 3000, replace=False), edge]))
+    want, _ = oracle.attention(cfg, q, k, v, ref, rows=rows)
+    got = o.reshape(-1, w.head_dim)[torch.from_numpy(rows).cuda()]
+    assert_close(got, want)
+
+
+@pytest.mark.parametrize("w", [W_TINY, W_A, W_C, W_D], ids=lambda w: w.name)
+def test_dense_causal_kernel(w):
+    q, k, v = inputs(w)
+    want = oracle.dense_causal(oracle.config(w), q, k, v)
+    qd, kd, vd = to_dev(q, k, v)
+    o = s2o.dense_causal_prefill(s2o.Config.of(w), qd, kd, vd)
+    torch.cuda.synchronize()
+    assert_close(o, want)
+
+
+def test_tau_zero_matches_dense_causal():
+    w = W_A.replace(tau=0.0)
+    q, k, v = inputs(w)
+    want = oracle.dense_causal(oracle.config(w), q, k, v)
+    qd, kd, vd = to_dev(q, k, v)
+    o, _ = s2o.attention_prefill(s2o.Config.of(w), qd, kd, vd)
+    torch.cuda.synchronize()
+    assert_close(o, want)
+
+
+def test_permutation_invariance_full_selection():
+    """Arbitrary orderings with every block listed: the output is dense causal attention."""
+    w = W_A
+    q, k, v = inputs(w)
+    B, H, N = w.batch, w.n_q_heads, w.seq_len
+    nB, S = N // w.block_size, w.segment_len
+    rng = np.random.default_rng(3)
+    perm_k = np.stack([np.stack([rng.permutation(N) for _ in range(H)]) for _ in range(B)])
+    perm_q = np.empty_like(perm_k)
+    for b in range(B):
+        for h in range(H):
+            for s0 in range(0, N, S):
+                perm_q[b, h, s0:s0 + S] = s0 + rng.permutation(S)
+    blk = perm_q.reshape(B, H, nB, w.block_size)
+    lt = (blk.max(-1) - (np.arange(nB) * w.block_size // S * S)) // w.block_size + 1
+    ref = dict(perm_q=perm_q.astype(np.int32), perm_k=perm_k.astype(np.int32),
+               sel_cnt=np.full((B, H, nB), nB, np.int32),
+               sel_blk=np.broadcast_to(rng.permutation(nB).astype(np.int32), (B, H, nB, nB)),
+               local_tiles=lt.astype(np.int32))
+    want = oracle.dense_causal(oracle.config(w), q, k, v)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w)
+    idx = oracle_indices_on_device(ref)
+    assert s2o.validate_indices(cfg, idx)
+    o = s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx)
+    torch.cuda.synchronize()
+    assert_close(o, want)
+
+
+# ----------------------------------------------------------------------------- validation/stats
+
+def test_validate_indices_accepts_and_rejects():
+    w = W_A
+    q, k, _ = inputs(w)
+    cfg, idx, ws = gpu_indices(w, *to_dev(q, k))
+    assert s2o.validate_indices(cfg, idx, ws)
+    nB = cfg.n_blocks
+
+    def corrupted(fn):
+        c = s2o.Indices(*(t.clone() for t in (idx.perm_q, idx.perm_k, idx.sel_cnt, idx.sel_blk,
+                                              idx.local_tiles)))
+        fn(c)
+        return c
+
+    bad = [
+        corrupted(lambda c: c.perm_k[0, 1, :2].copy_(torch.tensor([5, 5]))),      # duplicate
+        corrupted(lambda c: c.perm_k[0, 0, 7].fill_(w.seq_len)),                   # range
+        corrupted(lambda c: c.perm_q[0, 2, 3].fill_(w.segment_len + 3)),           # other segment
+        corrupted(lambda c: c.sel_cnt[0, 0, nB - 1].fill_(nB + 1)),                # count
+        corrupted(lambda c: (c.sel_cnt[0, 3, nB - 2].fill_(2),
+                             c.sel_blk[0, 3, nB - 2, :2].copy_(torch.tensor([4, 4])))),
+        corrupted(lambda c: (c.sel_cnt[0, 3, nB - 2].fill_(1),
+                             c.sel_blk[0, 3, nB - 2, :1].fill_(-1))),
+        corrupted(lambda c: c.local_tiles[0, 1, 9].fill_(0)),
+        corrupted(lambda c: c.local_tiles[0, 1, 9].fill_(w.segment_len // w.block_size + 1)),
+    ]
+    for i, c in enumerate(bad):
+        assert not s2o.validate_indices(cfg, c, ws), i
+
+
+@pytest.mark.parametrize("w", [W_TINY.replace(tau=0.07), W_A, W_B], ids=lambda w: w.name)
+def test_index_stats_match_oracle(w):
+    q, k, _ = inputs(w)
+    ref = oracle.build_indices(oracle.config(w), q, k)
+    cfg, idx, ws = gpu_indices(w, *to_dev(q, k))
+    st = s2o.index_stats(cfg, idx, ws)
+    assert st.pairs == oracle.pair_count(oracle.config(w), ref)
+    assert st.local_tiles == int(ref["local_tiles"].sum())
+    assert st.selected_tiles == int(ref["sel_cnt"].sum())
+    N = w.seq_len
+    assert st.causal_pairs == w.batch * w.n_q_heads * N * (N + 1) // 2
+
+
+def test_sparsity_monotone_in_tau_on_gpu():
+    w = W_B
+    q, k, _ = inputs(w)
+    qd, kd = to_dev(q, k)
+    prev = None
+    for tau in (0.0, 0.002, 0.005, 0.01, 0.02, 0.05, 2.0):
+        cfg, idx, ws = gpu_indices(w.replace(tau=tau), qd, kd)
+        pairs = s2o.index_stats(cfg, idx, ws).pairs
+        if prev is not None:
+            assert pairs <= prev
+        prev = pairs
