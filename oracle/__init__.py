@@ -56,11 +56,11 @@ class _Debug(ctypes.Structure):
                  "p")]
 
 
-def _load():
+def _load(path: str | None = None):
     global _lib
     with _lock:
-        if _lib is None:
-            lib = ctypes.CDLL(build())
+        if _lib is None or path is not None:
+            lib = ctypes.CDLL(path or build())
             vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
             lib.oracle_build_indices.argtypes = [ctypes.POINTER(Config), vp, vp, vp, vp, vp, vp,
                                                  vp, ctypes.POINTER(_Debug), i32]
@@ -77,8 +77,28 @@ def _load():
             lib.oracle_score_scale.restype = ctypes.c_float
             lib.oracle_exp64.argtypes = [ctypes.c_double]
             lib.oracle_exp64.restype = ctypes.c_double
+            if path is not None:
+                return lib
             _lib = lib
     return _lib
+
+
+class use_library:
+    """Context manager that points this module at another build of the oracle source (used by
+    the mutation tests, which compile deliberately broken copies and check the pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _load()
+        _lib = _load(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
 
 
 def config(w, **overrides) -> Config:

@@ -1,0 +1,84 @@
+"""The pins have teeth: each test plants one plausible mistake in a copy of the oracle's source
+(a dropped term, a wrong sign, an off-by-one, a transposed operand, a reversed tie-break), builds
+it on the CPU and checks that the pin suite in test_oracle_pins.py rejects it. The real oracle is
+never modified."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "s2o_oracle.c")
+
+MUTATIONS = {
+    "u-sign": ("u[t] = kbar_top[t] - kbar_all[t];", "u[t] = kbar_all[t] - kbar_top[t];"),
+    "drop-score-scale": ("Kbar + (size_t)c * d, d) * sigma;", "Kbar + (size_t)c * d, d);"),
+    "visible-count-le": ("if (perm_k[c * B + e] < s * S) ++cntv;",
+                         "if (perm_k[c * B + e] <= s * S) ++cntv;"),
+    "tie-break-reversed": ("return (a->idx > b->idx) - (a->idx < b->idx);",
+                           "return (a->idx < b->idx) - (a->idx > b->idx);"),
+    "local-window-off-by-one": ("for (int j = s0; j <= i; ++j) keys[nk++] = j;",
+                                "for (int j = s0; j < i; ++j) keys[nk++] = j;"),
+    "gqa-mapping": ("G = Hq / Hkv, g = h / G;", "G = Hq / Hkv, g = h % Hkv;"),
+    "no-normalisation": ("double p = any ? w[c] / Z : 0.0;", "double p = any ? w[c] : 0.0;"),
+    "transposed-block-score": (
+        "dot_f32(Qbar + (size_t)b * d, Kbar + (size_t)c * d, d) * sigma;",
+        "dot_f32(Qbar + (size_t)c * d, Kbar + (size_t)b * d, d) * sigma;"),
+    "kappa-from-mean-key": ("kappa[j] = dot_f32_bf16(qbar, K + (size_t)j * d, d);",
+                            "kappa[j] = dot_f32_bf16(kbar_all, K + (size_t)j * d, d);"),
+    "dropped-visibility-weight": (
+        "w[c] = ns[c] > 0 ? (double)ns[c] * oracle_exp64((double)rb[c] - (double)M) : 0.0;",
+        "w[c] = ns[c] > 0 ? oracle_exp64((double)rb[c] - (double)M) : 0.0;"),
+}
+
+# The pins that run against each mutant (all CPU, seconds each).
+PIN_TESTS = [
+    pins.test_hand_case_intermediates,
+    pins.test_hand_case_probabilities_closed_form,
+    lambda: [pins.test_hand_case_selection_and_pairs(t) for t in ("0.0", "0.28", "0.3", "0.4")],
+    pins.test_hand_case_key_sets,
+    lambda: [pins.test_tau_zero_is_dense_causal_attention(w)
+             for w in (pins.gen.workload("tiny"), pins.SMALL_GQA)],
+    lambda: [pins.test_tau_above_one_is_local_window_only(w)
+             for w in (pins.gen.workload("tiny"), pins.SMALL_GQA)],
+    pins.test_index_arrays_are_sorted_permutations,
+    pins.test_probabilities_and_selection_rule,
+    pins.test_float64_rederivation_of_pooled_quantities,
+]
+
+
+def build_mutant(tmp_path, name):
+    old, new = MUTATIONS[name]
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    src = tmp_path / f"{name}.c"
+    src.write_text(text.replace(old, new))
+    lib = tmp_path / f"{name}.so"
+    subprocess.run(["gcc", *oracle.CFLAGS, "-o", str(lib), str(src), "-lm"], check=True)
+    return str(lib)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_reject_planted_mistake(tmp_path, name):
+    lib = build_mutant(tmp_path, name)
+    caught = []
+    with oracle.use_library(lib):
+        for pin in PIN_TESTS:
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                caught.append(getattr(pin, "__name__", "lambda"))
+    assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    src = tmp_path / "same.c"
+    shutil.copy(SRC, src)
+    lib = tmp_path / "same.so"
+    subprocess.run(["gcc", *oracle.CFLAGS, "-o", str(lib), str(src), "-lm"], check=True)
+    with oracle.use_library(str(lib)):
+        for pin in PIN_TESTS:
+            pin()
