@@ -48,40 +48,59 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs.
+
+    The sampler is started and confirmed running before the region opens; only samples whose
+    arrival time falls inside [mark_start, mark_end] are kept."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+    def __init__(self, gpu_index: int, period_ms: int = 20):
+        self.gpu, self.period = gpu_index, period_ms
+        self.proc, self.samples, self.t0, self.t1 = None, [], None, None
+
+    def _reader(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.samples.append((time.perf_counter(), ln))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.period)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        threading.Thread(target=self._reader, daemon=True).start()
+        deadline = time.perf_counter() + 5.0
+        while not self.samples and time.perf_counter() < deadline:
+            time.sleep(0.01)
         return self
 
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
         sms, maxes, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for t, ln in list(self.samples):
+            if self.t0 is None or self.t1 is None or not (self.t0 <= t <= self.t1):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -216,11 +235,13 @@ def run_s2o(args):
     torch.cuda.synchronize(dev)
     launches0 = s2o.kernel_launch_count()
     with ClockSampler(local) as clocks:
+        clocks.mark_start()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         end.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.mark_end()
     launches = s2o.kernel_launch_count() - launches0
     if dist is not None:
         dist.barrier()
@@ -322,7 +343,7 @@ def run_s2o(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="s2o", choices=["s2o", "reference"])
     ap.add_argument("--tau", type=float, default=0.01)
