@@ -155,6 +155,28 @@ uint64_t s2o_kernel_launch_count(void);
  * else S2O_OK. */
 s2o_status s2o_check_device_status(s2o_stream stream);
 
+/* Size of the device scratch array behind s2o_build_indices_static (48 MiB: enough for a
+ * 32-query-head, 8-KV-head, 32K-token layer with d = 128 and B = 128). */
+#define S2O_STATIC_WORKSPACE_BYTES (48u << 20)
+
+/* s2o_build_indices for callers that cannot allocate device memory (an operator embedded in a
+ * host framework that only hands over its inputs and outputs, a serving path that must not call
+ * cudaMalloc after start-up). No counterpart on the pages: it is the same index build as
+ * s2o_build_indices, but its scratch is a fixed array inside the library
+ * (S2O_STATIC_WORKSPACE_BYTES per GPU, held from library load until process exit) instead of a
+ * caller workspace. The caller still owns and passes q, k and the index arrays.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *  - Configurations whose s2o_workspace_size exceeds S2O_STATIC_WORKSPACE_BYTES are rejected with
+ *    S2O_ERR_WORKSPACE_TOO_SMALL before any device work.
+ *  - The first call on each device (with that device current) looks up the array's device address
+ *    with cudaGetSymbolAddress; make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents behind; calls whose GPU
+ *    work overlaps (different streams, or different host threads) race on it and must be
+ *    serialised by the caller. s2o_workspace_views does not apply to it.
+ * Arguments, layouts, results and the other errors are those of s2o_build_indices. */
+s2o_status s2o_build_indices_static(const s2o_config *cfg, const void *q, const void *k,
+                                    const s2o_indices *out, s2o_stream stream);
+
 /* Diagnostic: evaluates the library's exp64 — the binary64 exponential behind the block weights of
  * the early stop (a Cody–Waite reduction by ln 2 and a degree-13 Taylor polynomial, defined in
  * the project's definition file; the pages give no normalisation, see [S2O, Summary ¶2]) — on n

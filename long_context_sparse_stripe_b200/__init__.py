@@ -25,7 +25,7 @@ __all__ = [
     "alloc_workspace", "build_indices", "attention_prefill", "attention_prefill_with_indices",
     "dense_causal_prefill", "validate_indices", "index_stats", "workspace_views",
     "set_wait_limit_ns", "check_device_status", "exp64_eval", "library_path",
-    "kernel_launch_count",
+    "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
 ]
 
 STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
@@ -145,6 +145,7 @@ def _load():
             "s2o_workspace_size": [C, ctypes.POINTER(sz)],
             "s2o_index_sizes": [C, ctypes.POINTER(sz * 5)],
             "s2o_build_indices": [C, vp, vp, I, vp, sz, vp],
+            "s2o_build_indices_static": [C, vp, vp, I, vp],
             "s2o_workspace_views": [C, vp, sz, ctypes.POINTER(_View)],
             "s2o_attention_prefill": [C, vp, vp, vp, vp, I, vp, sz, vp],
             "s2o_attention_prefill_with_indices": [C, vp, vp, vp, I, vp, vp],
@@ -223,6 +224,22 @@ def build_indices(cfg: Config, q, k, out: Indices | None = None,
     _check(_load().s2o_build_indices(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
                                      ctypes.byref(idx), ws.data_ptr(), ws.numel(),
                                      _stream(q.device)), "s2o_build_indices")
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 48 << 20  # S2O_STATIC_WORKSPACE_BYTES in include/s2o.h
+
+
+def build_indices_static(cfg: Config, q, k, out: Indices) -> Indices:
+    """The index build for callers that cannot allocate device memory: the library's fixed
+    scratch array (``STATIC_WORKSPACE_BYTES`` per GPU) replaces the caller workspace. ``out`` must
+    be preallocated. Calls whose GPU work overlaps share that array and race; the first call on a
+    device does a one-time address lookup and should come before any stream capture."""
+    _qkv(cfg, q, k)
+    idx = out._c()
+    _check(_load().s2o_build_indices_static(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
+                                            ctypes.byref(idx), _stream(q.device)),
+           "s2o_build_indices_static")
     return out
 
 

@@ -20,6 +20,7 @@ SOURCES = {
     "s2o_api.cu": ["-O3"],
     "s2o_index.cu": ["-O3", "--fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true"],
     "s2o_attn.cu": ["-O3"],
+    "s2o_static_ws.cu": ["-O3"],
 }
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
