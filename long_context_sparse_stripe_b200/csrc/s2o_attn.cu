@@ -582,21 +582,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!((mw[cc / 32] >> (cc % 32)) & 1u)) s[cc] = __float_as_uint(-INFINITY);
         }
       }
-      float mt = -INFINITY;
+      // Row max and (below) row sum with 8 independent partial results: no 128-long dependency
+      // chain on a single accumulator.
+      float mp[8];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mt = fmaxf(mt, __uint_as_float(s[c]));
+      for (int x = 0; x < 8; ++x) mp[x] = __uint_as_float(s[x]);
+#pragma unroll
+      for (int c = 8; c < BN; ++c) mp[c % 8] = fmaxf(mp[c % 8], __uint_as_float(s[c]));
+      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float m_new = fmaxf(m_run, mt * sl2);
       const bool rescale = m_new > m_run + 8.0f;
       float m_use = rescale ? m_new : m_run;
       if (m_use == -INFINITY) m_use = 0.f;
       const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
-      float rs = 0.f;
+      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
         const float pv = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
-        rs += pv;
+        sp[c % 8] += pv;
         s[c] = __float_as_uint(pv);
       }
+      const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
       if (j > 0) {
         if (!__all_sync(full, mbar_wait(bar(kPVDone), (j - 1) & 1, lim))) {
           ok = false;

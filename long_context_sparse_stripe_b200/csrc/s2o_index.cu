@@ -14,6 +14,7 @@
 // contraction worth tensor cores (the block-score product needs a fixed fp32 FMA order).
 #include <algorithm>
 #include <climits>
+#include <cmath>
 
 #include "s2o_internal.h"
 
@@ -26,6 +27,40 @@ __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 __device__ __forceinline__ float bf16_at(const uint16_t *p) {
   return __uint_as_float((uint32_t)__ldg(p) << 16);
+}
+
+// DOT(row, vec) of a bf16 row (D values, 16-byte aligned) against an fp32 vector: the
+// definition's sequential FMA chain over t = 0..D-1. The whole row is loaded first (D/8 16-byte
+// loads in flight per thread).
+template <int D>
+__device__ __forceinline__ float dot_row(const uint16_t *row, const float *vec) {
+  uint4 v[D / 8];
+  const uint4 *p = reinterpret_cast<const uint4 *>(row);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) v[c] = __ldg(p + c);
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      acc = __fmaf_rn(bf16_lo(w[x]), vec[c * 8 + 2 * x], acc);
+      acc = __fmaf_rn(bf16_hi(w[x]), vec[c * 8 + 2 * x + 1], acc);
+    }
+  }
+  return acc;
+}
+
+// Two independent IEEE fp32 fused multiply-adds in one instruction: acc.{x,y} = fma(a.{x,y},
+// b.{x,y}, acc.{x,y}), each rounded on its own (same results as two fmaf calls).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 acc) {
+  unsigned long long r;
+  const unsigned long long A = ((unsigned long long)__float_as_uint(a.y) << 32) | __float_as_uint(a.x);
+  const unsigned long long B = ((unsigned long long)__float_as_uint(b.y) << 32) | __float_as_uint(b.x);
+  const unsigned long long C =
+      ((unsigned long long)__float_as_uint(acc.y) << 32) | __float_as_uint(acc.x);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(A), "l"(B), "l"(C));
+  return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
 }
 
 // Sort key of an fp32 score: monotone in the value, −0 folded onto +0, NaN below everything.
@@ -91,50 +126,62 @@ __global__ void __launch_bounds__(256)
   *reinterpret_cast<float2 *>(out + (size_t)chunk * D + t) = make_float2(a0, a1);
 }
 
-// Chunk sums added sequentially in chunk order, then divided by the list length.
-__global__ void k_pool_finish(const float *__restrict__ chunks, float *__restrict__ out,
-                              int n_chunks, int D, float len, long long n_out) {
-  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (tid >= n_out) return;
-  const long long head = tid / D;
-  const int t = (int)(tid % D);
-  const float *p = chunks + (size_t)head * n_chunks * D + t;
+// Chunk sums added sequentially in chunk order, then divided by the list length. One CTA per
+// head, one thread per column; chunk sums are staged through shared memory 128 chunks at a time
+// so that many loads are in flight.
+template <int D>
+__global__ void __launch_bounds__(D)
+    k_pool_finish(const float *__restrict__ chunks, float *__restrict__ out, int n_chunks,
+                  float len) {
+  constexpr int kStage = 128;
+  extern __shared__ float stage[];  // [kStage][D]
+  const long long head = blockIdx.x;
+  const int t = threadIdx.x;
+  const float *base = chunks + (size_t)head * n_chunks * D;
   float acc = 0.f;
-#pragma unroll 8
-  for (int c = 0; c < n_chunks; ++c) acc = __fadd_rn(acc, __ldg(p + (size_t)c * D));
-  out[tid] = __fdiv_rn(acc, len);
+  for (int c0 = 0; c0 < n_chunks; c0 += kStage) {
+    const int n = min(kStage, n_chunks - c0);
+    for (int x = t; x < n * D; x += D) stage[x] = __ldg(base + (size_t)c0 * D + x);
+    __syncthreads();
+    for (int c = 0; c < n; ++c) acc = __fadd_rn(acc, stage[c * D + t]);
+    __syncthreads();
+  }
+  out[head * D + t] = __fdiv_rn(acc, len);
 }
 
-// kappa_j = DOT(qbar_h, k_j) for 64 keys of one KV head and all G query heads of its group.
+// kappa_j = DOT(qbar_h, k_j): one thread per key row of a KV head, for all G query heads of
+// its group (the row is loaded once).
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
     k_kappa(const uint16_t *__restrict__ k, const float *__restrict__ qbar,
             float *__restrict__ kappa, int N, int Hq, int Hkv, int G) {
-  extern __shared__ float smem[];
-  float *ks = smem;                 // [64][D + 1]
-  float *qb = smem + 64 * (D + 1);  // [G][D]
+  extern __shared__ float qb[];  // [G][D]
   const long long kh = blockIdx.y;
-  const int j0 = blockIdx.x * 64;
+  const int j = blockIdx.x * 128 + threadIdx.x;
   const long long beta = kh / Hkv;
   const int g = (int)(kh % Hkv);
-  const uint16_t *rows = k + ((size_t)kh * N + j0) * D;
-  for (int x = threadIdx.x; x < 64 * D / 2; x += blockDim.x) {
-    const int r = x / (D / 2), c2 = (x % (D / 2)) * 2;
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(rows + (size_t)r * D + c2));
-    ks[r * (D + 1) + c2] = bf16_lo(v);
-    ks[r * (D + 1) + c2 + 1] = bf16_hi(v);
-  }
   const size_t qh0 = (size_t)beta * Hq + (size_t)g * G;
   for (int x = threadIdx.x; x < G * D; x += blockDim.x) qb[x] = qbar[qh0 * D + x];
   __syncthreads();
-  const int j = threadIdx.x % 64;
-  for (int hi = threadIdx.x / 64; hi < G; hi += blockDim.x / 64) {
+  if (j >= N) return;
+  const uint16_t *row = k + ((size_t)kh * N + j) * D;
+  uint4 v[D / 8];
+  const uint4 *p = reinterpret_cast<const uint4 *>(row);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) v[c] = __ldg(p + c);
+  for (int hi = 0; hi < G; ++hi) {
     const float *a = qb + hi * D;
-    const float *b = ks + j * (D + 1);
     float acc = 0.f;
-#pragma unroll 16
-    for (int t = 0; t < D; ++t) acc = __fmaf_rn(a[t], b[t], acc);
-    kappa[(qh0 + hi) * N + j0 + j] = acc;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        acc = __fmaf_rn(a[c * 8 + 2 * x], bf16_lo(w[x]), acc);
+        acc = __fmaf_rn(a[c * 8 + 2 * x + 1], bf16_hi(w[x]), acc);
+      }
+    }
+    kappa[(qh0 + hi) * N + j] = acc;
   }
 }
 
@@ -155,32 +202,18 @@ __global__ void k_kbar_top(const uint16_t *__restrict__ k, const int32_t *__rest
   u[qh * D + t] = __fsub_rn(top, kbar_all[kh * D + t]);
 }
 
-// rho_i = DOT(q_i, u_h) for 128 query rows of one head.
+// rho_i = DOT(q_i, u_h), one thread per query row (used when segments exceed the fused kernel's
+// shared-memory sort).
 template <int D>
 __global__ void __launch_bounds__(128)
     k_rho(const uint16_t *__restrict__ q, const float *__restrict__ u, float *__restrict__ rho,
           int N) {
-  extern __shared__ float smem[];
-  float *qs = smem;                  // [128][D + 1]
-  float *us = smem + 128 * (D + 1);  // [D]
+  __shared__ float us[D];
   const long long qh = blockIdx.y;
-  const int i0 = blockIdx.x * 128;
-  const int n_rows = min(128, N - i0);
-  const uint16_t *rows = q + ((size_t)qh * N + i0) * D;
-  for (int x = threadIdx.x; x < n_rows * D / 2; x += blockDim.x) {
-    const int r = x / (D / 2), c2 = (x % (D / 2)) * 2;
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(rows + (size_t)r * D + c2));
-    qs[r * (D + 1) + c2] = bf16_lo(v);
-    qs[r * (D + 1) + c2 + 1] = bf16_hi(v);
-  }
+  const int i = blockIdx.x * 128 + threadIdx.x;
   for (int x = threadIdx.x; x < D; x += blockDim.x) us[x] = u[qh * D + x];
   __syncthreads();
-  if ((int)threadIdx.x >= n_rows) return;
-  const float *a = qs + threadIdx.x * (D + 1);
-  float acc = 0.f;
-#pragma unroll 16
-  for (int t = 0; t < D; ++t) acc = __fmaf_rn(a[t], us[t], acc);
-  rho[qh * N + i0 + threadIdx.x] = acc;
+  if (i < N) rho[qh * N + i] = dot_row<D>(q + ((size_t)qh * N + i) * D, us);
 }
 
 // ------------------------------------------------------------------ ordering (step 2)
@@ -191,21 +224,11 @@ __global__ void k_make_keys(const float *__restrict__ score, unsigned long long 
   if (x < total) keys[x] = order_word(score[x], (uint32_t)(x % N));
 }
 
-// Sorts each tile of TILE consecutive words of a run in shared memory (bitonic network); the
-// last tile of a run is padded with all-ones words, which sort last.
-template <int TILE>
-__global__ void __launch_bounds__(1024)
-    k_tile_sort(unsigned long long *__restrict__ keys, long long run_len, int tiles_per_run) {
-  __shared__ unsigned long long s[TILE];
-  const long long run = blockIdx.x / tiles_per_run;
-  const long long tile0 = (long long)(blockIdx.x % tiles_per_run) * TILE;
-  const long long begin = run * run_len + tile0;
-  const int n = (int)min((long long)TILE, run_len - tile0);
-  for (int i = threadIdx.x; i < TILE; i += blockDim.x) s[i] = i < n ? keys[begin + i] : ~0ull;
-  __syncthreads();
-  for (int k = 2; k <= TILE; k <<= 1) {
+// Ascending bitonic sort of n (a power of two) words in shared memory by the whole CTA.
+__device__ __forceinline__ void bitonic_sort_smem(unsigned long long *s, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < TILE; i += blockDim.x) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const unsigned long long a = s[i], b = s[ixj];
@@ -218,43 +241,58 @@ __global__ void __launch_bounds__(1024)
       __syncthreads();
     }
   }
+}
+
+// Sorts each tile of TILE consecutive words of a run in shared memory; the last tile of a run is
+// padded with all-ones words, which sort last.
+template <int TILE>
+__global__ void __launch_bounds__(1024)
+    k_tile_sort(unsigned long long *__restrict__ keys, long long run_len, int tiles_per_run) {
+  __shared__ unsigned long long s[TILE];
+  const long long run = blockIdx.x / tiles_per_run;
+  const long long tile0 = (long long)(blockIdx.x % tiles_per_run) * TILE;
+  const long long begin = run * run_len + tile0;
+  const int n = (int)min((long long)TILE, run_len - tile0);
+  for (int i = threadIdx.x; i < TILE; i += blockDim.x) s[i] = i < n ? keys[begin + i] : ~0ull;
+  __syncthreads();
+  bitonic_sort_smem(s, TILE);
   for (int i = threadIdx.x; i < n; i += blockDim.x) keys[begin + i] = s[i];
 }
 
-__device__ __forceinline__ long long count_less(const unsigned long long *a, long long n,
-                                                unsigned long long key) {
-  long long lo = 0, hi = n;
+// One merge pass: sorted neighbours of `width` words inside each run become sorted pairs. Each
+// thread writes kItems consecutive outputs: it finds where its first output splits the two inputs
+// by a binary search along the merge diagonal, then merges sequentially. Words are unique.
+constexpr int kMergeItems = 8;
+
+__global__ void k_merge_pass(const unsigned long long *__restrict__ src,
+                             unsigned long long *__restrict__ dst, long long run_len,
+                             long long width, long long total) {
+  const long long g = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * kMergeItems;
+  if (g >= total) return;
+  const long long run = g / run_len, off = g % run_len;
+  const long long pair0 = off - off % (2 * width);
+  const long long left_n = min(width, run_len - pair0);
+  const long long right_n = max(0LL, min(width, run_len - pair0 - width));
+  const unsigned long long *A = src + run * run_len + pair0;
+  const unsigned long long *Bv = A + left_n;
+  const long long o = off - pair0;
+  long long lo = max(0LL, o - right_n), hi = min(o, left_n);
   while (lo < hi) {
     const long long mid = (lo + hi) >> 1;
-    if (a[mid] < key)
+    if (A[mid] < Bv[o - 1 - mid])
       lo = mid + 1;
     else
       hi = mid;
   }
-  return lo;
-}
-
-// One merge pass: sorted neighbours of `width` words inside each run become sorted pairs. Words
-// are unique, so an element's output slot is its own offset plus the number of smaller words in
-// the other half.
-__global__ void k_merge_pass(const unsigned long long *__restrict__ src,
-                             unsigned long long *__restrict__ dst, long long run_len,
-                             long long width, long long total) {
-  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x >= total) return;
-  const long long run = x / run_len, off = x % run_len;
-  const long long pair0 = off - off % (2 * width);
-  const long long left_n = min(width, run_len - pair0);
-  const long long right_n = max(0LL, min(width, run_len - pair0 - width));
-  const unsigned long long *base = src + run * run_len + pair0;
-  const unsigned long long key = src[x];
-  const long long in_pair = off - pair0;
-  long long pos;
-  if (in_pair < width)
-    pos = in_pair + count_less(base + width, right_n, key);
-  else
-    pos = (in_pair - width) + count_less(base, left_n, key);
-  dst[run * run_len + pair0 + pos] = key;
+  long long i = lo, j = o - lo;
+  unsigned long long *out = dst + run * run_len + pair0 + o;
+  const int n = (int)min((long long)kMergeItems, left_n + right_n - o);
+  for (int x = 0; x < n; ++x) {
+    if (i < left_n && (j >= right_n || A[i] < Bv[j]))
+      out[x] = A[i++];
+    else
+      out[x] = Bv[j++];
+  }
 }
 
 __global__ void k_extract_perm(const unsigned long long *__restrict__ keys,
@@ -266,6 +304,58 @@ __global__ void k_extract_perm(const unsigned long long *__restrict__ keys,
 __global__ void k_identity_perm(int32_t *__restrict__ perm, int N, long long total) {
   const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (x < total) perm[x] = (int32_t)(x % N);
+}
+
+// Segment-local query ordering fused with its input and outputs, one CTA per (query head,
+// segment) for segments of at most TILE queries: rho_i = DOT(q_i, u) for the segment's rows, a
+// sort of their order words in shared memory (skipped when the query ordering is off), perm_q,
+// and the block means Qbar of the segment's query blocks (the rows were just read, so the
+// gathered re-read mostly hits L2).
+template <int D, int TILE>
+__global__ void __launch_bounds__(512)
+    k_segment_order(const uint16_t *__restrict__ q, const float *__restrict__ u,
+                    float *__restrict__ rho, int32_t *__restrict__ perm_q,
+                    float *__restrict__ Qbar, int N, int S, int B, int nB, int query_perm) {
+  __shared__ unsigned long long keys[TILE];
+  __shared__ float us[D];
+  const long long qh = blockIdx.y;
+  const int s0 = blockIdx.x * S;
+  for (int x = threadIdx.x; x < D; x += blockDim.x) us[x] = u[qh * D + x];
+  __syncthreads();
+  const uint16_t *Qh = q + (size_t)qh * N * D;
+  for (int r = threadIdx.x; r < TILE; r += blockDim.x) {
+    if (r < S) {
+      const int i = s0 + r;
+      const float v = dot_row<D>(Qh + (size_t)i * D, us);
+      rho[qh * N + i] = v;
+      keys[r] = query_perm ? order_word(v, (uint32_t)i) : (unsigned long long)i;
+    } else {
+      keys[r] = ~0ull;
+    }
+  }
+  __syncthreads();
+  if (query_perm) bitonic_sort_smem(keys, TILE);
+  for (int r = threadIdx.x; r < S; r += blockDim.x)
+    perm_q[qh * N + s0 + r] = (int32_t)(keys[r] & 0xffffffffull);
+  const int nbl = S / B;
+  const int items = nbl * (D / 4);
+  const float len = (float)B;
+  for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    const int bl = it / (D / 4), t = (it % (D / 4)) * 4;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+    for (int e = 0; e < B; ++e) {
+      const int row = (int)(keys[bl * B + e] & 0xffffffffull);
+      const uint2 v = __ldg(reinterpret_cast<const uint2 *>(Qh + (size_t)row * D + t));
+      a0 = __fadd_rn(a0, bf16_lo(v.x));
+      a1 = __fadd_rn(a1, bf16_hi(v.x));
+      a2 = __fadd_rn(a2, bf16_lo(v.y));
+      a3 = __fadd_rn(a3, bf16_hi(v.y));
+    }
+    float *dst = Qbar + ((size_t)qh * nB + (size_t)(s0 / B) + bl) * D + t;
+    *reinterpret_cast<float4 *>(dst) =
+        make_float4(__fdiv_rn(a0, len), __fdiv_rn(a1, len), __fdiv_rn(a2, len), __fdiv_rn(a3, len));
+  }
 }
 
 // ------------------------------------------------------------------ blocks and scores
@@ -335,11 +425,11 @@ __global__ void __launch_bounds__(256)
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   const float *A = Qbar + (size_t)qh * nB * D;
   const float *Bm = Kbar + (size_t)qh * nB * D;
-  float acc[8][8];
+  float2 acc[8][4];  // acc[i][jj] holds columns 2jj and 2jj+1
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
   for (int t0 = 0; t0 < D; t0 += 32) {
     for (int x = threadIdx.x; x < 128 * 32; x += 256) {
       const int row = x / 32, tt = x % 32;
@@ -354,11 +444,12 @@ __global__ void __launch_bounds__(256)
       const float4 v0 = *reinterpret_cast<const float4 *>(&Bs[tt][tc * 8]);
       const float4 v1 = *reinterpret_cast<const float4 *>(&Bs[tt][tc * 8 + 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      const float2 v[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w),
+                           make_float2(v1.x, v1.y), make_float2(v1.z, v1.w)};
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(a[i], v[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma2(make_float2(a[i], a[i]), v[j], acc[i][j]);
     }
     __syncthreads();
   }
@@ -369,7 +460,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int c = c0 + tc * 8 + j;
-      if (c < nB) r[((size_t)qh * nB + b) * nB + c] = __fmul_rn(acc[i][j], sigma);
+      const float x = (j & 1) ? acc[i][j >> 1].y : acc[i][j >> 1].x;
+      if (c < nB) r[((size_t)qh * nB + b) * nB + c] = __fmul_rn(x, sigma);
     }
   }
 }
@@ -382,19 +474,24 @@ __device__ __forceinline__ bool goes_before(double pa, int ca, double pb, int cb
 
 // One warp per query block: local tile count, normalised block scores p over the candidate
 // blocks, selection p >= τ, and the list sorted by (p descending, block ascending).
+// Shared memory per warp: the weights (nB doubles, one pad slot per 32 so that a lane walking its
+// own chunk hits distinct banks) and the selected list (cap2 entries; cap2 bounds the list
+// length: at most floor(1/τ) + 1 blocks can reach p >= τ since the p sum to one).
 __global__ void __launch_bounds__(128)
     k_schedule(const float *__restrict__ r, const int32_t *__restrict__ ncount,
                const int32_t *__restrict__ perm_q, int32_t *__restrict__ sel_cnt,
                int32_t *__restrict__ sel_blk, int32_t *__restrict__ local_tiles, int N, int B,
-               int S, int nB, int nSeg, int P2, double tau, long long n_qblocks) {
+               int S, int nB, int nSeg, int cap2, double tau, long long n_qblocks) {
   extern __shared__ unsigned char smem_raw[];
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const long long qb = (long long)blockIdx.x * (blockDim.x / kWarp) + warp;
   if (qb >= n_qblocks) return;
-  const size_t per_warp = ((size_t)nB * 8 + (size_t)P2 * 12 + 15) & ~(size_t)15;
+  const int wslots = nB + (nB + 31) / 32;
+  const size_t per_warp = ((size_t)wslots * 8 + (size_t)cap2 * 12 + 15) & ~(size_t)15;
   double *w = reinterpret_cast<double *>(smem_raw + per_warp * warp);
-  double *lp = w + nB;
-  int *lc = reinterpret_cast<int *>(lp + P2);
+  double *lp = w + wslots;
+  int *lc = reinterpret_cast<int *>(lp + cap2);
+  auto wi = [](int c) { return c + (c >> 5); };
 
   const long long qh = qb / nB;
   const int b = (int)(qb % nB);
@@ -419,8 +516,7 @@ __global__ void __launch_bounds__(128)
       any = true;
     }
   }
-  const unsigned have = __ballot_sync(full, any);
-  if (have == 0) {
+  if (__ballot_sync(full, any) == 0) {
     if (lane == 0) sel_cnt[qb] = 0;
     return;
   }
@@ -431,21 +527,21 @@ __global__ void __launch_bounds__(128)
     any = any || other_any;
   }
 
-  // Weights w_c and their sum Z: chunks of 32 consecutive blocks (chunk k is summed by lane
-  // k mod 32 sequentially), then the chunk sums in chunk order.
+  // Weights (independent per block, computed lane-strided), then Z: chunks of 32 consecutive
+  // blocks, chunk k summed sequentially by lane k mod 32, then the chunk sums in chunk order.
+#pragma unroll 4
+  for (int c = lane; c < nB; c += kWarp) {
+    const int nv = __ldg(nn + c);
+    w[wi(c)] = nv > 0 ? __dmul_rn((double)nv, exp64(__dsub_rn((double)__ldg(rr + c), (double)M)))
+                      : 0.0;
+  }
+  __syncwarp();
   const int n_chunks = (nB + 31) / 32;
   double part0 = 0.0, part1 = 0.0;  // this lane's chunks k = lane and k = lane + 32
   for (int k = lane; k < n_chunks; k += kWarp) {
     double part = 0.0;
     const int c_end = min(nB, 32 * k + 32);
-    for (int c = 32 * k; c < c_end; ++c) {
-      const int nv = __ldg(nn + c);
-      const double wc =
-          nv > 0 ? __dmul_rn((double)nv, exp64(__dsub_rn((double)__ldg(rr + c), (double)M)))
-                 : 0.0;
-      w[c] = wc;
-      part = __dadd_rn(part, wc);
-    }
+    for (int c = 32 * k; c < c_end; ++c) part = __dadd_rn(part, w[wi(c)]);
     if (k < kWarp)
       part0 = part;
     else
@@ -456,35 +552,31 @@ __global__ void __launch_bounds__(128)
     const double v = __shfl_sync(full, k < kWarp ? part0 : part1, k % kWarp);
     Z = __dadd_rn(Z, v);
   }
-  __syncwarp();
 
-  // Selection p_c = w_c / Z >= τ, compacted through a warp prefix count.
-  int mine = 0;
-  for (int k = lane; k < n_chunks; k += kWarp) {
-    const int c_end = min(nB, 32 * k + 32);
-    for (int c = 32 * k; c < c_end; ++c)
-      if (__ldg(nn + c) > 0 && __ddiv_rn(w[c], Z) >= tau) ++mine;
-  }
-  int incl = mine;
-  for (int o = 1; o < kWarp; o <<= 1) {
-    const int v = __shfl_up_sync(full, incl, o);
-    if (lane >= o) incl += v;
-  }
-  const int cnt = __shfl_sync(full, incl, kWarp - 1);
-  int slot = incl - mine;
-  for (int k = lane; k < n_chunks; k += kWarp) {
-    const int c_end = min(nB, 32 * k + 32);
-    for (int c = 32 * k; c < c_end; ++c) {
-      if (__ldg(nn + c) > 0) {
-        const double p = __ddiv_rn(w[c], Z);
-        if (p >= tau) {
-          lp[slot] = p;
-          lc[slot] = c;
-          ++slot;
-        }
+  // Selection p_c = w_c / Z >= τ. A weight below (τ·Z)(1 − 2^-48) gives p < τ whatever the
+  // rounding, so its division is skipped; every other candidate's p is computed exactly.
+  const double t_lo = __dmul_rn(__dmul_rn(tau, Z), 1.0 - 0x1p-48);
+  int cnt = 0;
+  for (int c0 = 0; c0 < nB; c0 += kWarp) {
+    const int c = c0 + lane;
+    bool sel = false;
+    double p = 0.0;
+    if (c < nB && __ldg(nn + c) > 0) {
+      const double wc = w[wi(c)];
+      if (tau == 0.0 || !(wc < t_lo)) {
+        p = __ddiv_rn(wc, Z);
+        sel = p >= tau;
       }
     }
+    const unsigned m = __ballot_sync(full, sel);
+    const int slot = cnt + __popc(m & ((1u << lane) - 1u));
+    if (sel && slot < cap2) {
+      lp[slot] = p;
+      lc[slot] = c;
+    }
+    cnt += __popc(m);
   }
+  cnt = min(cnt, cap2);
   int P = 1;
   while (P < cnt) P <<= 1;
   for (int e = cnt + lane; e < P; e += kWarp) {
@@ -637,7 +729,8 @@ cudaError_t sort_runs(unsigned long long *a, unsigned long long *b, long long to
     note_launch();
   unsigned long long *src = a, *dst = b;
   for (long long width = tile; width < run_len; width *= 2) {
-    k_merge_pass<<<blocks_for(total, 256), 256, 0, st>>>(src, dst, run_len, width, total);
+    k_merge_pass<<<blocks_for((total + kMergeItems - 1) / kMergeItems, 256), 256, 0, st>>>(
+        src, dst, run_len, width, total);
     note_launch();
     unsigned long long *t = src;
     src = dst;
@@ -677,18 +770,20 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   k_pool_chunks<D><<<blocks_for(nkv_rows / d.B * (D / 2), 256), 256, 0, st>>>(k, kchunk, d.B,
                                                                                nkv_rows / d.B);
   note_launch();
-  k_pool_finish<<<blocks_for(bhq * D, 256), 256, 0, st>>>(qchunk, qbar, d.nB, D, (float)d.N,
-                                                          bhq * D);
+  const size_t fin_smem = (size_t)128 * D * sizeof(float);
+  if ((e = cudaFuncSetAttribute(k_pool_finish<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fin_smem)) != cudaSuccess)
+    return e;
+  k_pool_finish<D><<<(unsigned)bhq, D, fin_smem, st>>>(qchunk, qbar, d.nB, (float)d.N);
   note_launch();
-  k_pool_finish<<<blocks_for(bhkv * D, 256), 256, 0, st>>>(kchunk, kbar_all, d.nB, D, (float)d.N,
-                                                           bhkv * D);
+  k_pool_finish<D><<<(unsigned)bhkv, D, fin_smem, st>>>(kchunk, kbar_all, d.nB, (float)d.N);
   note_launch();
-  const size_t kappa_smem = (64 * (D + 1) + (size_t)d.G * D) * sizeof(float);
+  const size_t kappa_smem = (size_t)d.G * D * sizeof(float);
   if ((e = cudaFuncSetAttribute(k_kappa<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kappa_smem)) != cudaSuccess)
     return e;
-  k_kappa<D><<<dim3(d.N / 64, (unsigned)bhkv), 256, kappa_smem, st>>>(k, qbar, kappa, d.N, d.Hq,
-                                                                       d.Hkv, d.G);
+  k_kappa<D><<<dim3((d.N + 127) / 128, (unsigned)bhkv), 128, kappa_smem, st>>>(k, qbar, kappa, d.N,
+                                                                              d.Hq, d.Hkv, d.G);
   note_launch();
   // Step 2a: global key/value ordering.
   k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(kappa, keys0, d.N, nq);
@@ -698,27 +793,40 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   k_kbar_top<<<(unsigned)bhq, D, 0, st>>>(k, out.perm_k, kbar_all, kbar_top, u, d.N, D, d.B, d.Hq,
                                           d.Hkv, d.G);
   note_launch();
-  const size_t rho_smem = (128 * (D + 1) + D) * sizeof(float);
-  if ((e = cudaFuncSetAttribute(k_rho<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)rho_smem)) != cudaSuccess)
-    return e;
-  k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, rho_smem, st>>>(q, u, rho, d.N);
-  note_launch();
-  // Step 2b: segment-local query ordering.
-  if (cfg.query_perm) {
-    k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(rho, keys0, d.N, nq);
-    note_launch();
-    if ((e = sort_runs(keys0, keys1, nq, d.S, out.perm_q, st)) != cudaSuccess) return e;
-  } else {
-    k_identity_perm<<<blocks_for(nq, 256), 256, 0, st>>>(out.perm_q, d.N, nq);
-    note_launch();
-  }
-  // Block means, visibility counts, block scores.
+  // Step 2b: segment-local query ordering, with rho and the query block means.
   const long long nblk = bhq * d.nB;
   constexpr int PER = 256 / (D / 2);
-  k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
-                                                          nblk, d.Hq, d.Hkv, d.G, 0);
+  const int qp = cfg.query_perm ? 1 : 0;
+  const dim3 seg_grid((unsigned)d.nSeg, (unsigned)bhq);
+  if (d.S <= 512) {
+    k_segment_order<D, 512><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
+                                                      d.nB, qp);
+  } else if (d.S <= 1024) {
+    k_segment_order<D, 1024><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
+                                                       d.nB, qp);
+  } else if (d.S <= 2048) {
+    k_segment_order<D, 2048><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
+                                                       d.nB, qp);
+  } else if (d.S <= 4096) {
+    k_segment_order<D, 4096><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
+                                                       d.nB, qp);
+  } else {
+    // Segments longer than the shared-memory sort: rho, a sort of each segment, block means.
+    k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
+    note_launch();
+    if (qp) {
+      k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(rho, keys0, d.N, nq);
+      note_launch();
+      if ((e = sort_runs(keys0, keys1, nq, d.S, out.perm_q, st)) != cudaSuccess) return e;
+    } else {
+      k_identity_perm<<<blocks_for(nq, 256), 256, 0, st>>>(out.perm_q, d.N, nq);
+      note_launch();
+    }
+    k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
+                                                            nblk, d.Hq, d.Hkv, d.G, 0);
+  }
   note_launch();
+  // Key block means, visibility counts, block scores.
   k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(k, out.perm_k, Kbar, d.N, d.B, d.nB,
                                                           nblk, d.Hq, d.Hkv, d.G, 1);
   note_launch();
@@ -730,10 +838,16 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   const unsigned tiles = (unsigned)((d.nB + 127) / 128);
   k_block_scores<D><<<dim3(tiles, tiles, (unsigned)bhq), 256, 0, st>>>(Qbar, Kbar, r, d.nB, sigma);
   note_launch();
-  // Scheduling.
-  int P2 = 1;
-  while (P2 < d.nB) P2 <<= 1;
-  const size_t per_warp = ((size_t)d.nB * 8 + (size_t)P2 * 12 + 15) & ~(size_t)15;
+  // Scheduling. The selected list of a query block holds at most floor(1/τ) + 1 entries.
+  int cap = d.nB;
+  if (cfg.tau > 0.f) {
+    const double bound = std::floor(1.0 / (double)cfg.tau) + 2.0;
+    if (bound < (double)cap) cap = (int)bound;
+  }
+  int cap2 = 1;
+  while (cap2 < cap) cap2 <<= 1;
+  const size_t per_warp =
+      ((size_t)(d.nB + (d.nB + 31) / 32) * 8 + (size_t)cap2 * 12 + 15) & ~(size_t)15;
   const int warps = (int)std::max<size_t>(1, std::min<size_t>(4, (200u << 10) / per_warp));
   const size_t sched_smem = per_warp * warps;
   if ((e = cudaFuncSetAttribute(k_schedule, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -741,7 +855,7 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
     return e;
   k_schedule<<<blocks_for(nblk, warps), warps * kWarp, sched_smem, st>>>(
       r, ncount, out.perm_q, out.sel_cnt, out.sel_blk, out.local_tiles, d.N, d.B, d.S, d.nB,
-      d.nSeg, P2, (double)cfg.tau, nblk);
+      d.nSeg, cap2, (double)cfg.tau, nblk);
   note_launch();
   return cudaGetLastError();
 }
