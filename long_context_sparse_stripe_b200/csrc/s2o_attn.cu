@@ -7,24 +7,36 @@
 // itself is Eq. (1) of "AB-Sparse" restricted to the selected key set, computed flash-style with
 // an online softmax (the normaliser of Milakov & Gimelshein, cited by the S2O paper).
 //
-// One CTA owns one (batch, query head, query block) work item: 128 query rows (the block's B rows
-// gathered by perm_q; rows B..127 are zero when B = 64). It runs lt local tiles (contiguous keys of
-// the block's own segment, mask key <= query) and then the cnt selected key blocks (keys gathered
-// by perm_k, mask key < segment start). Warp roles (256 threads):
-//   warp 0  K producer: Q once, then K tiles into a 3-deep ring (TMA tile loads for contiguous
-//           tiles, TMA tile::gather4 for gathered rows; 128-byte swizzle).
-//   warp 1  MMA issuer: owns TMEM; S = Q·Kᵀ into one of two TMEM S buffers, O += P·V into TMEM.
-//   warp 2  V producer: V tiles into a 2-deep ring.
-//   warp 3  idle.
-//   warps 4-7 softmax: thread r owns query row r (TMEM lane r): masks, online max/sum in the exp2
-//           domain, conditional rescale of O (only when the running max grows by more than 2^8),
-//           P as bf16 into a 128B-swizzled shared tile, and the final O/ℓ store at original rows.
-// Every wait is bounded (globaltimer); on a timeout the kernel records it, drains its own TMA
-// copies and tensor-core work, frees TMEM and exits.
+// Work decomposition. A unit is one (batch, query head, query block): 128 query rows (the block's
+// B rows gathered by perm_q; rows B..127 are zero when B = 64) that run lt local tiles (contiguous
+// keys of the block's own segment, mask key <= query) and then the cnt selected key blocks (keys
+// gathered by perm_k, mask key < segment start). Units are ordered (batch, KV head, segment,
+// block, query head of the group), so consecutive units usually read the same local key tiles. A
+// work item is two consecutive units, Q0 and Q1, with one stream of key/value tiles: the local
+// tiles once for both when they share them, then the two selected lists interleaved. The grid is
+// persistent (one CTA per SM, work items strided by the grid size).
+//
+// Warp roles (352 threads):
+//   warp 0      K/V producer: K and V tiles of the stream into two rings (TMA tile loads for
+//               contiguous tiles, TMA tile::gather4 for gathered rows; 128-byte swizzle).
+//   warp 1      MMA issuer: owns TMEM (512 columns: S0, S1, O0, O1). S_x = Q_x·Kᵀ, then
+//               O_x += P_x·V with P_x read from TMEM (bf16 pairs written over S_x). The two query
+//               tiles ping-pong: while one softmax group works on S0, the tensor core runs Q1's
+//               products.
+//   warp 2      Q producer: Q0 and Q1 of the next work item as soon as the last Q·Kᵀ of the
+//               current one has finished.
+//   warps 3-6   softmax of Q0, warps 7-10 softmax of Q1: the thread of TMEM lane r owns query row
+//               r (a warp reaches the lane quarter warp % 4):
+//               masks on original positions, online max/sum in the exp2 domain, conditional
+//               rescale of O (only when the running max grows by more than 2^8, exact in real
+//               arithmetic), P as bf16 into TMEM, and the final O/ℓ store at the original rows.
+// Every wait is bounded (globaltimer); on a timeout the kernel records it in a device error word,
+// drains its own TMA copies and tensor-core work, frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "s2o_internal.h"
 
@@ -34,8 +46,8 @@ __device__ unsigned int g_device_error;
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kM = 128;  // query rows per CTA (UMMA M)
+constexpr int kThreads = 352;
+constexpr int kM = 128;  // query rows per tile (UMMA M)
 constexpr uint64_t kDrainNs = 2000000000ull;
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -199,41 +211,51 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, int a_mn, int b_
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+// D (TMEM) = A·B (+ D): A read from TMEM (128 lanes, bf16 pairs along K), B from shared memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ layout
 
 template <int D, int BN>
 struct Layout {
-  static constexpr int KST = 3, VST = 2;
   static constexpr uint32_t ATOM_Q = kM * 128;  // bytes of one 64-column atom of a 128-row tile
   static constexpr uint32_t ATOM_KV = BN * 128;
   static constexpr uint32_t Q_BYTES = kM * D * 2;
   static constexpr uint32_t KV_BYTES = BN * D * 2;
-  static constexpr uint32_t P_BYTES = kM * BN * 2;
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int KST = KV_BYTES >= 32768 ? 3 : 4;  // K ring depth
+  static constexpr int VST = KV_BYTES >= 32768 ? 2 : 4;  // V ring depth
+  static constexpr uint32_t OFF_Q = 0;                   // Q0, then Q1
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr uint32_t OFF_P = OFF_V + VST * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr uint32_t SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
-  static constexpr uint32_t COLS_NEEDED = 2 * BN + D;
-  static constexpr uint32_t TMEM_COLS = COLS_NEEDED <= 256 ? 256 : 512;
-  static constexpr uint32_t S_COL = 0, O_COL = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL = 0;    // S_x at S_COL + 128·x (P_x over its first BN/2 columns)
+  static constexpr uint32_t O_COL = 256;  // O_x at O_COL + D·x
 };
 
-// Barrier slots (8 bytes each) inside the barrier area.
+// Barrier slots (8 bytes each) inside the barrier area; rings use up to four slots.
 enum Bar {
-  kQFull = 0,
-  kKFull = 1,    // 3
-  kKEmpty = 4,   // 3
-  kVFull = 7,    // 2
-  kVEmpty = 9,   // 2
-  kSFull = 11,   // 2
-  kSFree = 13,   // 2
-  kPFull = 15,
-  kPVDone = 16,
-  kDrain = 17,
-  kNumBars = 18
+  kQFull = 0,    // 2: Q_x landed (TMA transaction count)
+  kQEmpty = 2,   // 2: the last Q_x·Kᵀ of a work item finished
+  kKFull = 4,    // 4
+  kKEmpty = 8,   // 4
+  kVFull = 12,   // 4
+  kVEmpty = 16,  // 4
+  kSFull = 20,   // 2: S_x = Q_x·Kᵀ finished (and every earlier product of the CTA)
+  kPFull = 22,   // 2: P_x written to TMEM and O_x rescaled (128 arrivals)
+  kOFull = 24,   // 2: the last O_x += P_x·V of a work item finished
+  kDrain = 26,
+  kNumBars = 27
 };
 
 struct Params {
@@ -241,59 +263,232 @@ struct Params {
   uint16_t *o;
   int N, S, nB, nSeg, Hq, Hkv, G;
   int dense;
+  long long n_units, n_items;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
 };
 
-struct Work {
+struct Unit {
   long long qh, kh;  // flat (batch, query head) and (batch, kv head)
-  int b, s, lt, cnt;
+  int b, seg0, lt, cnt;
   const int32_t *sel;  // the query block's selected list (sel_blk row)
 };
 
-// Work item order: S2O groups the CTAs of one (batch, KV head, segment) together so that the
-// segment's K/V tiles and the group's gathered rows stay in L2; the dense baseline runs the
-// longest query blocks first.
+// Unit order: S2O keeps the units of one (batch, KV head, segment) together, query heads of the
+// group fastest, so that the segment's K/V tiles stay in L2 and paired units share local tiles;
+// the dense baseline runs the longest query blocks first.
 template <int BN>
-__device__ __forceinline__ Work decode_work(const Params &p) {
-  Work w;
-  long long item = blockIdx.x;
-  const int hi = (int)(item % p.G);
-  item /= p.G;
+__device__ __forceinline__ Unit decode_unit(const Params &p, long long u) {
+  Unit r;
+  const int hi = (int)(u % p.G);
+  u /= p.G;
   const int per_seg = p.S / BN;
-  int b, g;
-  long long beta;
+  int b;
   if (p.dense) {
-    b = p.nB - 1 - (int)(item % p.nB);
-    item /= p.nB;
+    b = p.nB - 1 - (int)(u % p.nB);
+    u /= p.nB;
   } else {
-    const int bl = (int)(item % per_seg);
-    item /= per_seg;
-    const int s = (int)(item % p.nSeg);
-    item /= p.nSeg;
+    const int bl = (int)(u % per_seg);
+    u /= per_seg;
+    const int s = (int)(u % p.nSeg);
+    u /= p.nSeg;
     b = s * per_seg + bl;
   }
-  g = (int)(item % p.Hkv);
-  beta = item / p.Hkv;
-  w.qh = beta * p.Hq + (long long)g * p.G + hi;
-  w.kh = beta * p.Hkv + g;
-  w.b = b;
-  w.s = (int)((long long)b * BN / p.S);
+  const int g = (int)(u % p.Hkv);
+  const long long beta = u / p.Hkv;
+  r.qh = beta * p.Hq + (long long)g * p.G + hi;
+  r.kh = beta * p.Hkv + g;
+  r.b = b;
+  r.seg0 = (int)((long long)b * BN / p.S) * p.S;
   if (p.dense) {
-    w.lt = b + 1;
-    w.cnt = 0;
-    w.sel = nullptr;
+    r.lt = b + 1;
+    r.cnt = 0;
+    r.sel = nullptr;
   } else {
-    const long long qb = w.qh * p.nB + b;
-    w.lt = min(max(__ldg(p.local_tiles + qb), 1), per_seg);
-    w.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
-    w.sel = p.sel_blk + qb * p.nB;
+    const long long qb = r.qh * p.nB + b;
+    r.lt = min(max(__ldg(p.local_tiles + qb), 1), per_seg);
+    r.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
+    r.sel = p.sel_blk + qb * p.nB;
   }
-  return w;
+  return r;
 }
 
-__device__ __forceinline__ int selected_block(const Work &w, const Params &p, int j) {
-  return min(max(__ldg(w.sel + (j - w.lt)), 0), p.nB - 1);
+struct Pair {
+  Unit u0, u1;
+  int valid1;  // the second unit exists (the last work item may hold one)
+  int shared;  // both units read the same local key tiles
+  int L;       // local items of the stream
+  int total;   // stream length
+};
+
+template <int BN>
+__device__ __forceinline__ Pair decode_pair(const Params &p, long long w) {
+  Pair P;
+  P.u0 = decode_unit<BN>(p, 2 * w);
+  P.valid1 = 2 * w + 1 < p.n_units;
+  if (P.valid1) {
+    P.u1 = decode_unit<BN>(p, 2 * w + 1);
+  } else {
+    P.u1 = P.u0;
+    P.u1.lt = 0;
+    P.u1.cnt = 0;
+  }
+  P.shared = P.valid1 && P.u0.kh == P.u1.kh && P.u0.seg0 == P.u1.seg0;
+  P.L = P.shared ? max(P.u0.lt, P.u1.lt) : P.u0.lt + P.u1.lt;
+  P.total = P.L + P.u0.cnt + P.u1.cnt;
+  return P;
+}
+
+// Position j of a two-way interleaving of a items of unit 0 and b items of unit 1 (alternating
+// while both have items left): the unit x and its item index.
+__device__ __forceinline__ void interleave(int a, int b, int j, int &x, int &idx) {
+  const int m = min(a, b);
+  if (j < 2 * m) {
+    x = j & 1;
+    idx = j >> 1;
+  } else {
+    x = a > b ? 0 : 1;
+    idx = m + (j - 2 * m);
+  }
+}
+
+// Stream item j: which units use it (bit x), the unit whose indices locate its rows, whether it is
+// a local tile, and the tile index (local) or the position in that unit's selected list.
+struct Item {
+  int users, x, local, t;
+};
+
+__device__ __forceinline__ Item item_at(const Pair &P, int j) {
+  Item it;
+  if (j >= P.total) {
+    it.users = 0;
+    it.x = 0;
+    it.local = 0;
+    it.t = 0;
+    return it;
+  }
+  if (j < P.L) {
+    it.local = 1;
+    if (P.shared) {
+      it.users = (j < P.u0.lt ? 1 : 0) | (j < P.u1.lt ? 2 : 0);
+      it.x = (it.users & 1) ? 0 : 1;
+      it.t = j;
+    } else {
+      interleave(P.u0.lt, P.u1.lt, j, it.x, it.t);
+      it.users = 1 << it.x;
+    }
+  } else {
+    it.local = 0;
+    interleave(P.u0.cnt, P.u1.cnt, j - P.L, it.x, it.t);
+    it.users = 1 << it.x;
+  }
+  return it;
+}
+
+// The units that use stream item j (bit x for unit x; 0 past the end).
+__device__ __forceinline__ int users_at(const Pair &P, int j) {
+  if (j >= P.total) return 0;
+  int x, idx;
+  if (j < P.L) {
+    if (P.shared) return (j < P.u0.lt ? 1 : 0) | (j < P.u1.lt ? 2 : 0);
+    interleave(P.u0.lt, P.u1.lt, j, x, idx);
+  } else {
+    interleave(P.u0.cnt, P.u1.cnt, j - P.L, x, idx);
+  }
+  return 1 << x;
+}
+
+// Loads the K or V rows of stream item `it` into one ring stage (all 32 lanes of the warp call it;
+// the transaction count has been set). Contiguous local tiles: one TMA tile load per 64-column
+// atom; gathered rows: tile::gather4, four rows per lane.
+template <int D, int BN>
+__device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap *tm_tile,
+                                        const CUtensorMap *tm_row, const Params &p,
+                                        const Pair &P, const Item &it, uint32_t bar, int lane) {
+  using L = Layout<D, BN>;
+  const Unit &u = it.x ? P.u1 : P.u0;
+  const int row0 = (int)(u.kh * p.N);
+  if (it.local) {
+    if (lane == 0)
+      for (int a = 0; a < D / 64; ++a)
+        tma_load_tile(dst + a * L::ATOM_KV, tm_tile, a * 64, row0 + u.seg0 + it.t * BN, bar);
+  } else if (lane < BN / 4) {
+    const int c = min(max(__ldg(u.sel + it.t), 0), p.nB - 1);
+    const int4 r4 =
+        __ldg(reinterpret_cast<const int4 *>(p.perm_k + u.qh * p.N + (size_t)c * BN) + lane);
+    const int hi = p.N - 1;
+    const int y0 = row0 + min(max(r4.x, 0), hi), y1 = row0 + min(max(r4.y, 0), hi),
+              y2 = row0 + min(max(r4.z, 0), hi), y3 = row0 + min(max(r4.w, 0), hi);
+    for (int a = 0; a < D / 64; ++a)
+      tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, tm_row, a * 64, y0, y1, y2, y3, bar);
+  }
+}
+
+// Waits (lane 0, bounded) and broadcasts the outcome to the warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar_addr, uint32_t parity, uint64_t lim,
+                                          int lane) {
+  bool got = true;
+  if (lane == 0) got = mbar_wait(bar_addr, parity, lim);
+  return __shfl_sync(0xffffffffu, got, 0);
+}
+
+// Lane 0 waits (bounded) for the last fill of each stage of a ring of `stages` slots that has
+// received `filled` fills in total.
+__device__ __forceinline__ void drain_ring(uint32_t full0, int stages, long long filled) {
+  for (int st = 0; st < stages; ++st) {
+    if (filled <= st) continue;
+    const long long last = st + ((filled - 1 - st) / stages) * stages;
+    mbar_wait(full0 + 8u * (uint32_t)st, (uint32_t)((last / stages) & 1), kDrainNs);
+  }
+}
+
+// Eight tcgen05.mma (kind::f16) into one accumulator, issued back to back from registers: A and B
+// shared-memory descriptors per K step; the first product accumulates only if `acc0` is set.
+__device__ __forceinline__ void mma8_ss(uint32_t d, uint32_t idesc, const uint64_t (&a)[8],
+                                        const uint64_t (&b)[8], uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t"
+      "setp.ne.b32 p0, %18, 0;\n\t"
+      "setp.eq.b32 p1, %0, %0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %1, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %17, %1, p1;\n\t}\n" ::"r"(d),
+      "r"(idesc), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]),
+      "l"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]),
+      "l"(b[7]), "r"(acc0)
+      : "memory");
+}
+
+// As mma8_ss with A read from TMEM (eight column addresses).
+__device__ __forceinline__ void mma8_ts(uint32_t d, uint32_t idesc, const uint32_t (&a)[8],
+                                        const uint64_t (&b)[8], uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t"
+      "setp.ne.b32 p0, %18, 0;\n\t"
+      "setp.eq.b32 p1, %0, %0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %1, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %17, %1, p1;\n\t}\n" ::"r"(d),
+      "r"(idesc), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]),
+      "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]),
+      "l"(b[7]), "r"(acc0)
+      : "memory");
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -312,17 +507,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::OFF_Q, sK = sbase + L::OFF_K, sV = sbase + L::OFF_V,
-                 sP = sbase + L::OFF_P, sBar = sbase + L::OFF_BAR;
+                 sBar = sbase + L::OFF_BAR;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_BAR + kNumBars * 8);
   auto bar = [&](int i) { return sBar + 8u * (uint32_t)i; };
-
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const Work w = decode_work<BN>(p);
-  const int T = w.lt + w.cnt;
-  const int seg0 = w.s * p.S;  // first original position of the block's segment
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(kQFull), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(kQFull + x), 1);
+      mbar_init(bar(kQEmpty + x), 1);
+      mbar_init(bar(kSFull + x), 1);
+      mbar_init(bar(kPFull + x), 128);
+      mbar_init(bar(kOFull + x), 1);
+    }
     for (int i = 0; i < L::KST; ++i) {
       mbar_init(bar(kKFull + i), 1);
       mbar_init(bar(kKEmpty + i), 1);
@@ -331,12 +528,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kVFull + i), 1);
       mbar_init(bar(kVEmpty + i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kSFull + i), 1);
-      mbar_init(bar(kSFree + i), 128);
-    }
-    mbar_init(bar(kPFull), 128);
-    mbar_init(bar(kPVDone), 1);
     mbar_init(bar(kDrain), 1);
     fence_barrier_init();
   }
@@ -347,12 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (BN < kM && warp >= 4) {
-    // Rows BN..127 of the Q tile are padding: zero them (the TMA writes rows 0..BN-1).
-    const int row = threadIdx.x - 128;
+  if (BN < kM && warp >= 3) {
+    // Rows BN..127 of both Q tiles are padding: zero them once (TMA writes rows 0..BN-1 only).
+    const int x = (warp - 3) >> 2, row = (warp & 3) * 32 + lane;
     if (row >= BN) {
       for (int a = 0; a < D / 64; ++a) {
-        uint4 *dst = reinterpret_cast<uint4 *>(smem + L::OFF_Q + a * L::ATOM_Q + row * 128);
+        uint4 *dst = reinterpret_cast<uint4 *>(smem + L::OFF_Q + x * L::Q_BYTES + a * L::ATOM_Q +
+                                               row * 128);
         for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
       }
     }
@@ -362,313 +554,377 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
   const uint64_t lim = p.limit_ns;
   bool ok = true;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- K producer (+ Q)
-    int issued = 0;
-    if (lane == 0) mbar_expect_tx(bar(kQFull), BN * D * 2);
-    __syncwarp();
-    const int q_row0 = (int)(w.qh * p.N);
-    if (p.dense || p.perm_q == nullptr) {
-      if (lane == 0)
-        for (int a = 0; a < D / 64; ++a)
-          tma_load_tile(sQ + a * L::ATOM_Q, &tm_q_tile, a * 64, q_row0 + w.b * BN, bar(kQFull));
-    } else if (lane < BN / 4) {
-      const int4 r4 = __ldg(reinterpret_cast<const int4 *>(p.perm_q + w.qh * p.N +
-                                                          (size_t)w.b * BN) + lane);
-      const int hiq = p.N - 1;
-      const int y0 = q_row0 + min(max(r4.x, 0), hiq), y1 = q_row0 + min(max(r4.y, 0), hiq),
-                y2 = q_row0 + min(max(r4.z, 0), hiq), y3 = q_row0 + min(max(r4.w, 0), hiq);
-      for (int a = 0; a < D / 64; ++a)
-        tma_gather4(sQ + a * L::ATOM_Q + lane * 4 * 128, &tm_q_row, a * 64, y0, y1, y2, y3,
-                    bar(kQFull));
-    }
-    const int kv_row0 = (int)(w.kh * p.N);
-    for (int j = 0; j < T; ++j) {
-      const int st = j % L::KST;
-      if (j >= L::KST) {
-        bool got = true;
-        if (lane == 0) got = mbar_wait(bar(kKEmpty + st), ((j / L::KST) - 1) & 1, lim);
-        if (!__shfl_sync(0xffffffffu, got, 0)) {
+    // ---------------------------------------------------------------- K / V producer
+    long long kj = 0;  // stream items issued so far (all work items of this CTA)
+    for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+      const Pair P = decode_pair<BN>(p, w);
+      for (int j = 0; j < P.total; ++j) {
+        const Item it = item_at(P, j);
+        const int ks = (int)(kj % L::KST), vs = (int)(kj % L::VST);
+        if (kj >= L::KST &&
+            !warp_wait(bar(kKEmpty + ks), (uint32_t)(((kj / L::KST) - 1) & 1), lim, lane)) {
           ok = false;
           break;
         }
+        if (lane == 0) mbar_expect_tx(bar(kKFull + ks), L::KV_BYTES);
+        __syncwarp();
+        load_kv<D, BN>(sK + ks * L::KV_BYTES, &tm_k_tile, &tm_k_row, p, P, it, bar(kKFull + ks),
+                       lane);
+        if (kj >= L::VST &&
+            !warp_wait(bar(kVEmpty + vs), (uint32_t)(((kj / L::VST) - 1) & 1), lim, lane)) {
+          // K of this item is in flight: count it for the drain below.
+          drain_ring(bar(kKFull), L::KST, kj + 1);
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_expect_tx(bar(kVFull + vs), L::KV_BYTES);
+        __syncwarp();
+        load_kv<D, BN>(sV + vs * L::KV_BYTES, &tm_v_tile, &tm_v_row, p, P, it, bar(kVFull + vs),
+                       lane);
+        ++kj;
       }
-      if (lane == 0) mbar_expect_tx(bar(kKFull + st), L::KV_BYTES);
-      __syncwarp();
-      const uint32_t dst = sK + st * L::KV_BYTES;
-      if (j < w.lt) {
-        if (lane == 0)
-          for (int a = 0; a < D / 64; ++a)
-            tma_load_tile(dst + a * L::ATOM_KV, &tm_k_tile, a * 64, kv_row0 + seg0 + j * BN,
-                          bar(kKFull + st));
-      } else if (lane < BN / 4) {
-        const int c = selected_block(w, p, j);
-        const int4 r4 = __ldg(reinterpret_cast<const int4 *>(p.perm_k + w.qh * p.N +
-                                                            (size_t)c * BN) + lane);
-        const int hik = p.N - 1;
-        const int y0 = kv_row0 + min(max(r4.x, 0), hik), y1 = kv_row0 + min(max(r4.y, 0), hik),
-                  y2 = kv_row0 + min(max(r4.z, 0), hik), y3 = kv_row0 + min(max(r4.w, 0), hik);
-        for (int a = 0; a < D / 64; ++a)
-          tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, &tm_k_row, a * 64, y0, y1, y2, y3,
-                      bar(kKFull + st));
-      }
-      issued = j + 1;
     }
-    // Drain: the last copy issued into each slot must have landed before the CTA exits.
+    // Drain: the last copy issued into each stage must have landed before the CTA exits.
     if (lane == 0) {
-      mbar_wait(bar(kQFull), 0, kDrainNs);
-      for (int st = 0; st < L::KST; ++st) {
-        int last = -1;
-        for (int j = st; j < issued; j += L::KST) last = j;
-        if (last >= 0) mbar_wait(bar(kKFull + st), (last / L::KST) & 1, kDrainNs);
-      }
+      drain_ring(bar(kKFull), L::KST, kj);
+      drain_ring(bar(kVFull), L::VST, kj);
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ---------------------------------------------------------------- V producer
-    int issued = 0;
-    const int kv_row0 = (int)(w.kh * p.N);
-    for (int j = 0; j < T; ++j) {
-      const int st = j % L::VST;
-      if (j >= L::VST) {
-        bool got = true;
-        if (lane == 0) got = mbar_wait(bar(kVEmpty + st), ((j / L::VST) - 1) & 1, lim);
-        if (!__shfl_sync(0xffffffffu, got, 0)) {
+    // ---------------------------------------------------------------- Q producer
+    long long qn[2] = {0, 0};
+    for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+      const Pair P = decode_pair<BN>(p, w);
+      for (int x = 0; ok && x < 1 + P.valid1; ++x) {
+        if (qn[x] >= 1 &&
+            !warp_wait(bar(kQEmpty + x), (uint32_t)((qn[x] - 1) & 1), lim, lane)) {
           ok = false;
           break;
         }
-      }
-      if (lane == 0) mbar_expect_tx(bar(kVFull + st), L::KV_BYTES);
-      __syncwarp();
-      const uint32_t dst = sV + st * L::KV_BYTES;
-      if (j < w.lt) {
-        if (lane == 0)
+        if (lane == 0) mbar_expect_tx(bar(kQFull + x), BN * D * 2);
+        __syncwarp();
+        const Unit &u = x ? P.u1 : P.u0;
+        const uint32_t dst = sQ + x * L::Q_BYTES;
+        const int q_row0 = (int)(u.qh * p.N);
+        if (p.dense || p.perm_q == nullptr) {
+          if (lane == 0)
+            for (int a = 0; a < D / 64; ++a)
+              tma_load_tile(dst + a * L::ATOM_Q, &tm_q_tile, a * 64, q_row0 + u.b * BN,
+                            bar(kQFull + x));
+        } else if (lane < BN / 4) {
+          const int4 r4 = __ldg(reinterpret_cast<const int4 *>(p.perm_q + u.qh * p.N +
+                                                              (size_t)u.b * BN) + lane);
+          const int hi = p.N - 1;
+          const int y0 = q_row0 + min(max(r4.x, 0), hi), y1 = q_row0 + min(max(r4.y, 0), hi),
+                    y2 = q_row0 + min(max(r4.z, 0), hi), y3 = q_row0 + min(max(r4.w, 0), hi);
           for (int a = 0; a < D / 64; ++a)
-            tma_load_tile(dst + a * L::ATOM_KV, &tm_v_tile, a * 64, kv_row0 + seg0 + j * BN,
-                          bar(kVFull + st));
-      } else if (lane < BN / 4) {
-        const int c = selected_block(w, p, j);
-        const int4 r4 = __ldg(reinterpret_cast<const int4 *>(p.perm_k + w.qh * p.N +
-                                                            (size_t)c * BN) + lane);
-        const int hik = p.N - 1;
-        const int y0 = kv_row0 + min(max(r4.x, 0), hik), y1 = kv_row0 + min(max(r4.y, 0), hik),
-                  y2 = kv_row0 + min(max(r4.z, 0), hik), y3 = kv_row0 + min(max(r4.w, 0), hik);
-        for (int a = 0; a < D / 64; ++a)
-          tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, &tm_v_row, a * 64, y0, y1, y2, y3,
-                      bar(kVFull + st));
-      }
-      issued = j + 1;
-    }
-    if (lane == 0) {
-      for (int st = 0; st < L::VST; ++st) {
-        int last = -1;
-        for (int j = st; j < issued; j += L::VST) last = j;
-        if (last >= 0) mbar_wait(bar(kVFull + st), (last / L::VST) & 1, kDrainNs);
+            tma_gather4(dst + a * L::ATOM_Q + lane * 4 * 128, &tm_q_row, a * 64, y0, y1, y2, y3,
+                        bar(kQFull + x));
+        }
+        ++qn[x];
       }
     }
+    if (lane == 0)
+      for (int x = 0; x < 2; ++x)
+        if (qn[x] > 0) mbar_wait(bar(kQFull + x), (uint32_t)((qn[x] - 1) & 1), kDrainNs);
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // One thread issues every tensor-core operation. Its loop is kept short (32-bit counters,
+    // descriptors advanced by constant offsets): it shares a scheduler with two softmax warps
+    // that issue back to back, and each of its instructions delays the next product.
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16(kM, BN, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16(kM, D, 0, 1);
-      auto issue_qk = [&](int j) -> bool {
-        const int st = j % L::KST;
-        if (!mbar_wait(bar(kKFull + st), (j / L::KST) & 1, lim)) return false;
-        if (j >= 2 && !mbar_wait(bar(kSFree + (j & 1)), ((j >> 1) - 1) & 1, lim)) return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + L::S_COL + (uint32_t)(j & 1) * BN;
-        const uint32_t kst = sK + st * L::KV_BYTES;
+      static_assert((L::VST & (L::VST - 1)) == 0, "V ring depth must be a power of two");
+      // Descriptor start addresses are 16-byte units in bits 0-13; every operand address stays
+      // below 2^18 bytes, so constant offsets are added to the descriptor directly.
+      const uint64_t qdesc0 = sw128_desc(sQ, 16), kdesc0 = sw128_desc(sK, 16),
+                     vdesc0 = sw128_desc(sV, L::ATOM_KV);
+      // Per K step: Q descriptors of both tiles, the K offset inside a stage, P columns in TMEM.
+      constexpr uint64_t kOffK[8] = {0, 2, 4, 6, L::ATOM_KV >> 4, (L::ATOM_KV >> 4) + 2,
+                                     (L::ATOM_KV >> 4) + 4, (L::ATOM_KV >> 4) + 6};
+      constexpr uint64_t kOffQ[8] = {0, 2, 4, 6, L::ATOM_Q >> 4, (L::ATOM_Q >> 4) + 2,
+                                     (L::ATOM_Q >> 4) + 4, (L::ATOM_Q >> 4) + 6};
+      uint64_t qa[2][8];
+      uint32_t ptm[2][8];
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sw128_desc(sQ + (kk / 4) * L::ATOM_Q + (kk % 4) * 32, 16);
-          const uint64_t bd = sw128_desc(kst + (kk / 4) * L::ATOM_KV + (kk % 4) * 32, 16);
-          tc_mma(d_tmem, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(kKEmpty + st));
-        tc_commit(bar(kSFull + (j & 1)));
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % L::VST;
-        if (!mbar_wait(bar(kVFull + st), (j / L::VST) & 1, lim)) return false;
-        if (!mbar_wait(bar(kPFull), j & 1, lim)) return false;
-        tc_fence_after();
-        const uint32_t vst = sV + st * L::KV_BYTES;
+      for (int x = 0; x < 2; ++x)
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = sw128_desc(sP + (kk / 4) * L::ATOM_Q + (kk % 4) * 32, 16);
-          const uint64_t bd = sw128_desc(vst + kk * 16 * 128, L::ATOM_KV);
-          tc_mma(tmem + L::O_COL, a, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          qa[x][kk] = qdesc0 + (uint64_t)(x * (L::Q_BYTES >> 4)) + kOffQ[kk % (D / 16)];
+          ptm[x][kk] = tmem + L::S_COL + 128u * x + 8u * (kk % (BN / 16));
         }
-        tc_commit(bar(kVEmpty + st));
-        tc_commit(bar(kPVDone));
-        return true;
-      };
-      ok = mbar_wait(bar(kQFull), 0, lim);
-      if (ok) ok = issue_qk(0);
-      if (ok && T > 1) ok = issue_qk(1);
-      for (int j = 0; ok && j < T; ++j) {
-        ok = issue_pv(j);
-        if (ok && j + 2 < T) ok = issue_qk(j + 2);
+      uint32_t k_st = 0, k_ph = 0;  // K ring stage and phase of the next stream item
+      uint32_t v_base = 0;          // stream items of this CTA's earlier work items
+      uint32_t q_ph[2] = {0, 0}, p_ph[2] = {0, 0};
+      for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+        const Pair P = decode_pair<BN>(p, w);
+        if (!mbar_wait(bar(kQFull + 0), q_ph[0], lim) ||
+            (P.valid1 && !mbar_wait(bar(kQFull + 1), q_ph[1], lim))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int n_of[2] = {P.u0.lt + P.u0.cnt, P.u1.lt + P.u1.cnt};
+        int pend[2] = {-1, -1}, qk[2] = {0, 0};
+        uint32_t acc[2] = {0u, 0u};
+        uint32_t vleft = 0;  // 2 bits per V stage: products still to issue on its tile
+        // O_x += P_x·V for stream item jj (P_x bf16 pairs in TMEM, V in its ring stage). The V
+        // stage is released once every unit using the tile has issued its product.
+        auto issue_pv = [&](auto xc, int jj) -> bool {
+          constexpr int x = decltype(xc)::value;
+          const uint32_t vi = v_base + (uint32_t)jj;
+          const uint32_t vs = vi & (L::VST - 1);
+          if (!mbar_wait(bar(kVFull + vs), (vi / L::VST) & 1u, lim)) return false;
+          if (!mbar_wait(bar(kPFull + x), p_ph[x], lim)) return false;
+          p_ph[x] ^= 1u;
+          tc_fence_after();
+          const uint64_t vd = vdesc0 + vs * (L::KV_BYTES >> 4);
+          uint64_t b[8];
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) b[kk] = vd + (uint64_t)((kk % (BN / 16)) * (16 * 128 / 16));
+          if (BN == 128) {
+            mma8_ts(tmem + L::O_COL + (uint32_t)(D * x), kIdescPV, ptm[x], b, acc[x]);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              tc_mma_ts(tmem + L::O_COL + (uint32_t)(D * x), ptm[x][kk], b[kk], kIdescPV,
+                        acc[x] | (kk > 0 ? 1u : 0u));
+          }
+          acc[x] = 1u;
+          const uint32_t left = ((vleft >> (2 * vs)) & 3u) - 1u;
+          vleft = (vleft & ~(3u << (2 * vs))) | ((left & 3u) << (2 * vs));
+          if (left == 0) tc_commit(bar(kVEmpty + vs));
+          return true;
+        };
+        auto issue_qk = [&](auto xc, const uint64_t (&kb)[8]) {
+          constexpr int x = decltype(xc)::value;
+          const uint32_t d_tmem = tmem + L::S_COL + 128u * x;
+          if (D == 128) {
+            mma8_ss(d_tmem, kIdescQK, qa[x], kb, 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              tc_mma(d_tmem, qa[x][kk], kb[kk], kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(kSFull + x));
+        };
+        // One unit's step at stream item j: its pending product goes first (P_x lives in S_x's
+        // columns), or now if the unit skips the next item (its V tile must leave the ring).
+        auto step = [&](auto xc, int j, int users, int nusers, const uint64_t (&kb)[8]) -> bool {
+          constexpr int x = decltype(xc)::value;
+          const bool use = (users >> x) & 1;
+          if (pend[x] >= 0 && (use || !((nusers >> x) & 1))) {
+            if (!issue_pv(xc, pend[x])) return false;
+            pend[x] = -1;
+          }
+          if (use) {
+            issue_qk(xc, kb);
+            pend[x] = j;
+            if (++qk[x] == n_of[x]) tc_commit(bar(kQEmpty + x));
+          }
+          return true;
+        };
+        int users = users_at(P, 0);
+        for (int j = 0; j < P.total; ++j) {
+          const int nusers = users_at(P, j + 1);
+          if (!mbar_wait(bar(kKFull + k_st), k_ph, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = kdesc0 + k_st * (L::KV_BYTES >> 4);
+          uint64_t kb[8];
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) kb[kk] = kd + kOffK[kk % (D / 16)];
+          if (!step(std::integral_constant<int, 0>{}, j, users, nusers, kb) ||
+              !step(std::integral_constant<int, 1>{}, j, users, nusers, kb)) {
+            ok = false;
+            break;
+          }
+          tc_commit(bar(kKEmpty + k_st));
+          const uint32_t vs = (v_base + (uint32_t)j) & (L::VST - 1);
+          vleft = (vleft & ~(3u << (2 * vs))) | ((uint32_t)__popc(users) << (2 * vs));
+          if (++k_st == (uint32_t)L::KST) {
+            k_st = 0;
+            k_ph ^= 1u;
+          }
+          users = nusers;
+        }
+        if (ok && pend[0] >= 0) ok = issue_pv(std::integral_constant<int, 0>{}, pend[0]);
+        if (ok && pend[1] >= 0) ok = issue_pv(std::integral_constant<int, 1>{}, pend[1]);
+        if (!ok) break;
+        tc_commit(bar(kOFull + 0));
+        q_ph[0] ^= 1u;
+        if (P.valid1) {
+          tc_commit(bar(kOFull + 1));
+          q_ph[1] ^= 1u;
+        }
+        v_base += (uint32_t)P.total;
       }
       // Drain: every tensor-core operation issued above completes before TMEM is freed.
       tc_commit(bar(kDrain));
       mbar_wait(bar(kDrain), 0, kDrainNs);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int quad = warp - 4;
+    const int x = (warp - 3) >> 2;  // query tile of this warp's group
+    const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t s_addr = trow + L::S_COL + 128u * (uint32_t)x;
+    const uint32_t o_addr = trow + L::O_COL + (uint32_t)(D * x);
     const unsigned full = 0xffffffffu;
-    // Original position of this row's query (padding rows: the segment's last position).
-    int i_orig = seg0 + p.S - 1;
-    bool store_row = false;
-    if (row < BN) {
-      const int v = (p.dense || p.perm_q == nullptr)
-                        ? w.b * BN + row
-                        : __ldg(p.perm_q + w.qh * p.N + (size_t)w.b * BN + row);
-      store_row = v >= seg0 && v < seg0 + p.S;
-      i_orig = store_row ? v : seg0;
-    }
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    uint32_t s[BN];
-    for (int j = 0; j < T; ++j) {
-      const int buf = j & 1;
-      // Warp-uniform outcome: the tcgen05.ld below is a warp-collective instruction.
-      if (!__all_sync(full, mbar_wait(bar(kSFull + buf), (j >> 1) & 1, lim))) {
-        ok = false;
-        break;
+    long long sn = 0, on = 0;  // S_x tiles and work items consumed
+    for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+      const Pair P = decode_pair<BN>(p, w);
+      if (x == 1 && !P.valid1) continue;
+      const Unit u = x ? P.u1 : P.u0;
+      const int seg0 = u.seg0;
+      // Original position of this row's query (padding rows: the segment's last position).
+      int i_orig = seg0 + p.S - 1;
+      bool store_row = false;
+      if (row < BN) {
+        const int v = (p.dense || p.perm_q == nullptr)
+                          ? u.b * BN + row
+                          : __ldg(p.perm_q + u.qh * p.N + (size_t)u.b * BN + row);
+        store_row = v >= seg0 && v < seg0 + p.S;
+        i_orig = store_row ? v : seg0;
       }
-      tc_fence_after();
-#pragma unroll
-      for (int c0 = 0; c0 < BN / 32; ++c0) {
-        uint32_t(&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[c0 * 32]);
-        tmem_ld32(trow + L::S_COL + buf * BN + c0 * 32, chunk);
-        tmem_wait_ld(chunk);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(kSFree + buf));
-
-      // Masks on original positions.
-      if (j < w.lt) {
-        const int limit = i_orig - (seg0 + j * BN);  // keys col <= limit are causal
-        if (__any_sync(full, limit < BN - 1)) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c > limit) s[c] = __float_as_uint(-INFINITY);
-        }
-      } else {
-        const int c = selected_block(w, p, j);
-        const int32_t *keys = p.perm_k + w.qh * p.N + (size_t)c * BN;
-        uint32_t mw[BN / 32];
-        bool all = true;
-#pragma unroll
-        for (int x = 0; x < BN / 32; ++x) {
-          const int key = __ldg(keys + x * 32 + lane);
-          mw[x] = __ballot_sync(full, key >= 0 && key < seg0);
-          all = all && mw[x] == full;
-        }
-        if (!all) {
-#pragma unroll
-          for (int cc = 0; cc < BN; ++cc)
-            if (!((mw[cc / 32] >> (cc % 32)) & 1u)) s[cc] = __float_as_uint(-INFINITY);
-        }
-      }
-      // Row max and (below) row sum with 8 independent partial results: no 128-long dependency
-      // chain on a single accumulator.
-      float mp[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) mp[x] = __uint_as_float(s[x]);
-#pragma unroll
-      for (int c = 8; c < BN; ++c) mp[c % 8] = fmaxf(mp[c % 8], __uint_as_float(s[c]));
-      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const float m_new = fmaxf(m_run, mt * sl2);
-      const bool rescale = m_new > m_run + 8.0f;
-      float m_use = rescale ? m_new : m_run;
-      if (m_use == -INFINITY) m_use = 0.f;
-      const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
-      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        const float pv = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
-        sp[c % 8] += pv;
-        s[c] = __float_as_uint(pv);
-      }
-      const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-      if (j > 0) {
-        if (!__all_sync(full, mbar_wait(bar(kPVDone), (j - 1) & 1, lim))) {
+      float m_run = -INFINITY, l_run = 0.f;
+      const int n_items = u.lt + u.cnt;
+      for (int n = 0; n < n_items; ++n) {
+        // Warp-uniform outcome: the tcgen05.ld below is a warp-collective instruction.
+        if (!__all_sync(full, mbar_wait(bar(kSFull + x), (uint32_t)(sn & 1), lim))) {
           ok = false;
           break;
         }
+        ++sn;
         tc_fence_after();
-        if (__any_sync(full, rescale)) {
+        uint32_t s[BN];
+#pragma unroll
+        for (int c0 = 0; c0 < BN / 32; ++c0)
+          tmem_ld32(s_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c0 * 32]));
+#pragma unroll
+        for (int c0 = 0; c0 < BN / 32; ++c0)
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&s[c0 * 32]));
+
+        // Masks on original positions.
+        if (n < u.lt) {
+          const int limit = i_orig - (seg0 + n * BN);  // keys col <= limit are causal
+          if (__any_sync(full, limit < BN - 1)) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              if (c > limit) s[c] = __float_as_uint(-INFINITY);
+          }
+        } else {
+          const int c = min(max(__ldg(u.sel + (n - u.lt)), 0), p.nB - 1);
+          const int32_t *keys = p.perm_k + u.qh * p.N + (size_t)c * BN;
+          uint32_t mw[BN / 32];
+          bool all = true;
+#pragma unroll
+          for (int q = 0; q < BN / 32; ++q) {
+            const int key = __ldg(keys + q * 32 + lane);
+            mw[q] = __ballot_sync(full, key >= 0 && key < seg0);
+            all = all && mw[q] == full;
+          }
+          if (!all) {
+#pragma unroll
+            for (int cc = 0; cc < BN; ++cc)
+              if (!((mw[cc / 32] >> (cc % 32)) & 1u)) s[cc] = __float_as_uint(-INFINITY);
+          }
+        }
+        // Row max with 8 independent partial results (no 128-long dependency chain), three inputs
+        // per instruction.
+        float mp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mp[q] = __uint_as_float(s[q]);
+#pragma unroll
+        for (int c = 8; c < BN; c += 16)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            mp[q] = max3f(mp[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
+        const float mt = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]),
+                               fmaxf(mp[6], mp[7]));
+        const float m_new = fmaxf(m_run, mt * sl2);
+        const bool rescale = m_new > m_run + 8.0f;
+        float m_use = rescale ? m_new : m_run;
+        if (m_use == -INFINITY) m_use = 0.f;
+        const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
+        // P = 2^(s·log2(e)/√d − m) as bf16 pairs, written over the first BN/2 columns of S_x.
+        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
+          sp[c % 8] += p0;
+          sp[(c + 1) % 8] += p1;
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
+        const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+#pragma unroll
+        for (int c0 = 0; c0 < BN / 64; ++c0)
+          tmem_st32(s_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0 * 32]));
+        // O_x holds the products of earlier tiles (S_x's completion covers them): rescale it when
+        // the running max moved.
+        if (n > 0 && __any_sync(full, rescale)) {
 #pragma unroll
           for (int c0 = 0; c0 < D / 32; ++c0) {
             uint32_t o[32];
-            tmem_ld32(trow + L::O_COL + c0 * 32, o);
+            tmem_ld32(o_addr + c0 * 32, o);
             tmem_wait_ld(o);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(trow + L::O_COL + c0 * 32, o);
+            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+            tmem_st32(o_addr + c0 * 32, o);
           }
-          tmem_wait_st();
         }
+        tmem_wait_st();
+        l_run = l_run * alpha + rs;
+        m_run = m_use;
+        tc_fence_before();
+        mbar_arrive(bar(kPFull + x));
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_use;
-      // P (bf16) into the K-major 128B-swizzled A tile: row `row`, 16-byte chunk ch of the
-      // 64-column atom ch / 8 lands at physical chunk (ch % 8) ^ (row % 8).
-      unsigned char *prow = smem + L::OFF_P + row * 128;
-#pragma unroll
-      for (int ch = 0; ch < BN / 8; ++ch) {
-        uint4 v;
-        v.x = pack_bf16(__uint_as_float(s[ch * 8 + 0]), __uint_as_float(s[ch * 8 + 1]));
-        v.y = pack_bf16(__uint_as_float(s[ch * 8 + 2]), __uint_as_float(s[ch * 8 + 3]));
-        v.z = pack_bf16(__uint_as_float(s[ch * 8 + 4]), __uint_as_float(s[ch * 8 + 5]));
-        v.w = pack_bf16(__uint_as_float(s[ch * 8 + 6]), __uint_as_float(s[ch * 8 + 7]));
-        *reinterpret_cast<uint4 *>(prow + (ch / 8) * L::ATOM_Q + (((ch % 8) ^ (row % 8)) * 16)) =
-            v;
+      if (!ok) break;
+      // Epilogue: O/ℓ as bf16 at the query's original row.
+      if (!__all_sync(full, mbar_wait(bar(kOFull + x), (uint32_t)(on & 1), lim))) {
+        ok = false;
+        break;
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(kPFull));
-    }
-    if (ok && __all_sync(full, mbar_wait(bar(kPVDone), (T - 1) & 1, lim))) {
+      ++on;
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      uint16_t *orow = p.o + ((size_t)w.qh * p.N + i_orig) * D;
+      uint16_t *orow = p.o + ((size_t)u.qh * p.N + i_orig) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D / 32; ++c0) {
         uint32_t o[32];
-        tmem_ld32(trow + L::O_COL + c0 * 32, o);
+        tmem_ld32(o_addr + c0 * 32, o);
         tmem_wait_ld(o);
         if (store_row) {
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
+          for (int q = 0; q < 4; ++q) {
             uint4 v;
-            v.x = pack_bf16(__uint_as_float(o[x * 8 + 0]) * inv_l,
-                            __uint_as_float(o[x * 8 + 1]) * inv_l);
-            v.y = pack_bf16(__uint_as_float(o[x * 8 + 2]) * inv_l,
-                            __uint_as_float(o[x * 8 + 3]) * inv_l);
-            v.z = pack_bf16(__uint_as_float(o[x * 8 + 4]) * inv_l,
-                            __uint_as_float(o[x * 8 + 5]) * inv_l);
-            v.w = pack_bf16(__uint_as_float(o[x * 8 + 6]) * inv_l,
-                            __uint_as_float(o[x * 8 + 7]) * inv_l);
-            *reinterpret_cast<uint4 *>(orow + c0 * 32 + x * 8) = v;
+            v.x = pack_bf16(__uint_as_float(o[q * 8 + 0]) * inv_l,
+                            __uint_as_float(o[q * 8 + 1]) * inv_l);
+            v.y = pack_bf16(__uint_as_float(o[q * 8 + 2]) * inv_l,
+                            __uint_as_float(o[q * 8 + 3]) * inv_l);
+            v.z = pack_bf16(__uint_as_float(o[q * 8 + 4]) * inv_l,
+                            __uint_as_float(o[q * 8 + 5]) * inv_l);
+            v.w = pack_bf16(__uint_as_float(o[q * 8 + 6]) * inv_l,
+                            __uint_as_float(o[q * 8 + 7]) * inv_l);
+            *reinterpret_cast<uint4 *>(orow + c0 * 32 + q * 8) = v;
           }
         }
       }
+      tc_fence_before();
     }
-    tc_fence_before();
   }
 
   __syncthreads();
@@ -711,10 +967,24 @@ bool make_map(CUtensorMap *m, const void *base, long long rows, int D, int box_r
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
 template <int D, int BN>
 cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaStream_t st) {
   using L = Layout<D, BN>;
   static_assert(L::SMEM <= 232448, "shared memory budget");
+  static_assert(kNumBars * 8 + 4 <= (int)L::BAR_BYTES, "barrier area");
   CUtensorMap tq, tqr, tk, tkr, tv, tvr;
   const long long q_rows = d.bhq() * d.N, kv_rows = d.bhkv() * d.N;
   if (!make_map(&tq, a.q, q_rows, D, BN) || !make_map(&tqr, a.q, q_rows, D, 1) ||
@@ -739,10 +1009,13 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
   p.Hkv = d.Hkv;
   p.G = d.G;
   p.dense = a.dense ? 1 : 0;
+  p.n_units = d.bhq() * d.nB;
+  p.n_items = (p.n_units + 1) / 2;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   p.limit_ns = limit_ns;
-  const unsigned grid = (unsigned)(d.bhq() * d.nB);
-  s2o_attention_kernel<D, BN><<<grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv, tvr, p);
+  const long long grid = p.n_items < sm_count() ? p.n_items : sm_count();
+  s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv, tvr,
+                                                                         p);
   note_launch();
   return cudaGetLastError();
 }
