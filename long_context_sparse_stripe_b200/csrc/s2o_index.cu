@@ -15,6 +15,7 @@
 #include <algorithm>
 #include <climits>
 #include <cmath>
+#include <type_traits>
 
 #include "s2o_internal.h"
 
@@ -51,6 +52,27 @@ __device__ __forceinline__ float dot_row(const uint16_t *row, const float *vec) 
   return acc;
 }
 
+// DOT(row, vec) for a row already in registers (D bf16 values as D/8 16-byte words) against an
+// fp32 vector in shared memory read four values at a time: the same sequential FMA chain over
+// t = 0..D-1.
+template <int D>
+__device__ __forceinline__ float dot_regs(const uint4 (&v)[D / 8], const float4 *vec4) {
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const float4 a = vec4[2 * c], b = vec4[2 * c + 1];
+    acc = __fmaf_rn(bf16_lo(v[c].x), a.x, acc);
+    acc = __fmaf_rn(bf16_hi(v[c].x), a.y, acc);
+    acc = __fmaf_rn(bf16_lo(v[c].y), a.z, acc);
+    acc = __fmaf_rn(bf16_hi(v[c].y), a.w, acc);
+    acc = __fmaf_rn(bf16_lo(v[c].z), b.x, acc);
+    acc = __fmaf_rn(bf16_hi(v[c].z), b.y, acc);
+    acc = __fmaf_rn(bf16_lo(v[c].w), b.z, acc);
+    acc = __fmaf_rn(bf16_hi(v[c].w), b.w, acc);
+  }
+  return acc;
+}
+
 // Two independent IEEE fp32 fused multiply-adds in one instruction: acc.{x,y} = fma(a.{x,y},
 // b.{x,y}, acc.{x,y}), each rounded on its own (same results as two fmaf calls).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 acc) {
@@ -80,26 +102,35 @@ __device__ __forceinline__ unsigned long long order_word(float score, uint32_t i
 // exp64: Cody–Waite reduction by ln 2 with a two-part constant, then the degree-13 Taylor
 // polynomial of e^t by Horner's rule with fused multiply-adds, then an exact scaling by 2^k.
 // Written for this project from the mathematics; defined for x <= 0 (all block-weight arguments).
-__device__ double exp64(double x) {
+// k = rint(x/ln 2) is taken by adding and subtracting 1.5·2^52 (round half to even, as rint),
+// which also leaves k in the low word of the sum: no conversion instruction is needed.
+__device__ __forceinline__ double exp64(double x) {
   if (x < -700.0) return 0.0;
   const double kInvLn2 = 0x1.71547652b82fep+0;  // nearest binary64 to 1/ln 2
   const double kLn2Hi = 0x1.62e42fefa39efp-1;   // nearest binary64 to ln 2
   const double kLn2Lo = 0x1.abc9e3b39803fp-56;  // nearest binary64 to ln 2 − kLn2Hi
+  const double kRound = 0x1.8p52;
   // 1/j! for j = 0..13, each the correctly rounded quotient (j! is exact in binary64).
   const double c[14] = {1.0 / 1.0,         1.0 / 1.0,          1.0 / 2.0,
                         1.0 / 6.0,         1.0 / 24.0,         1.0 / 120.0,
                         1.0 / 720.0,       1.0 / 5040.0,       1.0 / 40320.0,
                         1.0 / 362880.0,    1.0 / 3628800.0,    1.0 / 39916800.0,
                         1.0 / 479001600.0, 1.0 / 6227020800.0};
-  const double k = rint(__dmul_rn(x, kInvLn2));
+  const double y = __dadd_rn(__dmul_rn(x, kInvLn2), kRound);
+  const double k = __dsub_rn(y, kRound);
   double t = __fma_rn(-k, kLn2Hi, x);
   t = __fma_rn(-k, kLn2Lo, t);
   double p = c[13];
 #pragma unroll
   for (int j = 12; j >= 0; --j) p = __fma_rn(p, t, c[j]);
   // k in [-1010, 0]: 2^k is a normal binary64 number, so the product is exact.
-  const double two_k = __longlong_as_double((long long)((int)k + 1023) << 52);
-  return __dmul_rn(p, two_k);
+  const int ki = __double2loint(y);
+  return __dmul_rn(p, __hiloint2double((ki + 1023) << 20, 0));
+}
+
+// An integer 0 <= n < 2^31 as binary64, exactly, without a conversion instruction.
+__device__ __forceinline__ double int_to_double(int n) {
+  return __dsub_rn(__hiloint2double(0x43300000, n), 0x1p52);
 }
 
 // ------------------------------------------------------------------ pooling (step 1a)
@@ -127,61 +158,83 @@ __global__ void __launch_bounds__(256)
 }
 
 // Chunk sums added sequentially in chunk order, then divided by the list length. One CTA per
-// head, one thread per column; chunk sums are staged through shared memory 128 chunks at a time
-// so that many loads are in flight.
+// (head, 32 columns): all threads stage up to 1024 chunk sums at once in shared memory (many loads
+// in flight), then one warp adds them in chunk order.
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(256)
     k_pool_finish(const float *__restrict__ chunks, float *__restrict__ out, int n_chunks,
                   float len) {
-  constexpr int kStage = 128;
-  extern __shared__ float stage[];  // [kStage][D]
-  const long long head = blockIdx.x;
-  const int t = threadIdx.x;
-  const float *base = chunks + (size_t)head * n_chunks * D;
+  constexpr int kStage = 1024;
+  extern __shared__ float4 stage4[];  // [kStage][32]
+  float *stage = reinterpret_cast<float *>(stage4);
+  const long long head = blockIdx.y;
+  const int col0 = blockIdx.x * 32;
+  const float *base = chunks + (size_t)head * n_chunks * D + col0;
   float acc = 0.f;
   for (int c0 = 0; c0 < n_chunks; c0 += kStage) {
     const int n = min(kStage, n_chunks - c0);
-    for (int x = t; x < n * D; x += D) stage[x] = __ldg(base + (size_t)c0 * D + x);
+    for (int x = threadIdx.x; x < n * 8; x += blockDim.x)
+      stage4[x] = __ldg(reinterpret_cast<const float4 *>(base + (size_t)(c0 + x / 8) * D) + x % 8);
     __syncthreads();
-    for (int c = 0; c < n; ++c) acc = __fadd_rn(acc, stage[c * D + t]);
+    if (threadIdx.x < 32) {
+      int c = 0;
+      for (; c + 8 <= n; c += 8) {
+        float v[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) v[x] = stage[(c + x) * 32 + threadIdx.x];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc = __fadd_rn(acc, v[x]);
+      }
+      for (; c < n; ++c) acc = __fadd_rn(acc, stage[c * 32 + threadIdx.x]);
+    }
     __syncthreads();
   }
-  out[head * D + t] = __fdiv_rn(acc, len);
+  if (threadIdx.x < 32) out[head * D + col0 + threadIdx.x] = __fdiv_rn(acc, len);
 }
 
-// kappa_j = DOT(qbar_h, k_j): one thread per key row of a KV head, for all G query heads of
-// its group (the row is loaded once).
+// One pass over K, one CTA per chunk of B key rows of a KV head:
+//   kappa_j = DOT(qbar_h, k_j) for the G query heads of the group (one thread per key row, the row
+//   in registers, qbar read four values at a time from shared memory), and
+//   the chunk sum of the MEAN rule for kbar_all (the rows staged in shared memory, one thread per
+//   two columns adding the rows in order).
 template <int D>
 __global__ void __launch_bounds__(128)
-    k_kappa(const uint16_t *__restrict__ k, const float *__restrict__ qbar,
-            float *__restrict__ kappa, int N, int Hq, int Hkv, int G) {
-  extern __shared__ float qb[];  // [G][D]
+    k_kpass(const uint16_t *__restrict__ k, const float *__restrict__ qbar,
+            float *__restrict__ kappa, float *__restrict__ kchunk, int N, int B, int Hq, int Hkv,
+            int G) {
+  extern __shared__ float4 sm4[];
+  float *qb = reinterpret_cast<float *>(sm4);                     // [G][D]
+  uint4 *rows = reinterpret_cast<uint4 *>(sm4 + (size_t)G * D / 4);  // [B][D/8]
   const long long kh = blockIdx.y;
-  const int j = blockIdx.x * 128 + threadIdx.x;
+  const int chunk = blockIdx.x, r = threadIdx.x;
   const long long beta = kh / Hkv;
   const int g = (int)(kh % Hkv);
   const size_t qh0 = (size_t)beta * Hq + (size_t)g * G;
   for (int x = threadIdx.x; x < G * D; x += blockDim.x) qb[x] = qbar[qh0 * D + x];
-  __syncthreads();
-  if (j >= N) return;
-  const uint16_t *row = k + ((size_t)kh * N + j) * D;
+  const int j = chunk * B + r;
   uint4 v[D / 8];
-  const uint4 *p = reinterpret_cast<const uint4 *>(row);
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) v[c] = __ldg(p + c);
-  for (int hi = 0; hi < G; ++hi) {
-    const float *a = qb + hi * D;
-    float acc = 0.f;
+  if (r < B) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(k + ((size_t)kh * N + j) * D);
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
-      const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        acc = __fmaf_rn(a[c * 8 + 2 * x], bf16_lo(w[x]), acc);
-        acc = __fmaf_rn(a[c * 8 + 2 * x + 1], bf16_hi(w[x]), acc);
-      }
+      v[c] = __ldg(src + c);
+      rows[r * (D / 8) + c] = v[c];
     }
-    kappa[(qh0 + hi) * N + j] = acc;
+  }
+  __syncthreads();
+  if (r < B)
+    for (int hi = 0; hi < G; ++hi)
+      kappa[(qh0 + hi) * N + j] = dot_regs<D>(v, sm4 + (size_t)hi * D / 4);
+  if (r < D / 2) {
+    const uint32_t *rw = reinterpret_cast<const uint32_t *>(rows);
+    float a0 = 0.f, a1 = 0.f;
+    for (int e = 0; e < B; ++e) {
+      const uint32_t w = rw[e * (D / 2) + r];
+      a0 = __fadd_rn(a0, bf16_lo(w));
+      a1 = __fadd_rn(a1, bf16_hi(w));
+    }
+    *reinterpret_cast<float2 *>(kchunk + ((size_t)kh * (N / B) + chunk) * D + 2 * r) =
+        make_float2(a0, a1);
   }
 }
 
@@ -202,18 +255,23 @@ __global__ void k_kbar_top(const uint16_t *__restrict__ k, const int32_t *__rest
   u[qh * D + t] = __fsub_rn(top, kbar_all[kh * D + t]);
 }
 
-// rho_i = DOT(q_i, u_h), one thread per query row (used when segments exceed the fused kernel's
-// shared-memory sort).
+// rho_i = DOT(q_i, u_h), one thread per query row (the row in registers, u read four values at a
+// time from shared memory).
 template <int D>
 __global__ void __launch_bounds__(128)
     k_rho(const uint16_t *__restrict__ q, const float *__restrict__ u, float *__restrict__ rho,
           int N) {
-  __shared__ float us[D];
+  __shared__ float4 us4[D / 4];
   const long long qh = blockIdx.y;
   const int i = blockIdx.x * 128 + threadIdx.x;
-  for (int x = threadIdx.x; x < D; x += blockDim.x) us[x] = u[qh * D + x];
+  if (threadIdx.x < D / 4) us4[threadIdx.x] = reinterpret_cast<const float4 *>(u + qh * D)[threadIdx.x];
   __syncthreads();
-  if (i < N) rho[qh * N + i] = dot_row<D>(q + ((size_t)qh * N + i) * D, us);
+  if (i >= N) return;
+  uint4 v[D / 8];
+  const uint4 *src = reinterpret_cast<const uint4 *>(q + ((size_t)qh * N + i) * D);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) v[c] = __ldg(src + c);
+  rho[qh * N + i] = dot_regs<D>(v, us4);
 }
 
 // ------------------------------------------------------------------ ordering (step 2)
@@ -224,29 +282,81 @@ __global__ void k_make_keys(const float *__restrict__ score, unsigned long long 
   if (x < total) keys[x] = order_word(score[x], (uint32_t)(x % N));
 }
 
-// Ascending bitonic sort of n (a power of two) words in shared memory by the whole CTA.
-__device__ __forceinline__ void bitonic_sort_smem(unsigned long long *s, int n) {
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = s[i], b = s[ixj];
-          if ((a > b) == ((i & k) == 0)) {
-            s[i] = b;
-            s[ixj] = a;
-          }
+// One compare-exchange stage of a bitonic network on the 128 words a warp holds in registers
+// (word i of lane l is element base + 4l + i): partners closer than four elements sit in the
+// same lane, the others are exchanged through shuffles.
+__device__ __forceinline__ void warp_stage64(unsigned long long (&k)[4], int base, int lane,
+                                             int size, int stride) {
+  if (stride >= 4) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = base + 4 * lane + i;
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, k[i], stride >> 2);
+      // The lower element of a pair keeps the minimum in ascending runs, the maximum in
+      // descending ones; the upper element the other.
+      const bool keep_min = ((e & size) == 0) == ((e & stride) == 0);
+      const bool less = k[i] < other;
+      k[i] = (keep_min == less) ? k[i] : other;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = i ^ stride;
+      if (j > i) {
+        const bool up = ((base + 4 * lane + i) & size) == 0;
+        const unsigned long long lo = k[i] < k[j] ? k[i] : k[j];
+        const unsigned long long hi = k[i] < k[j] ? k[j] : k[i];
+        k[i] = up ? lo : hi;
+        k[j] = up ? hi : lo;
+      }
+    }
+  }
+}
+
+// Ascending bitonic sort of the 128·(blockDim.x/32) distinct words in shared memory: runs of up
+// to 128 words and every stage of stride below 128 run in registers (each warp owns 128
+// consecutive words), only the stages of larger stride go through shared memory.
+__device__ __forceinline__ void block_sort64(unsigned long long *s) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, n = blockDim.x * 4;
+  const int base = warp * 128;
+  unsigned long long k[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) k[i] = s[base + 4 * lane + i];
+#pragma unroll
+  for (int size = 2; size <= 128; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) warp_stage64(k, base, lane, size, stride);
+  for (int size = 256; size <= n; size <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[base + 4 * lane + i] = k[i];
+    __syncthreads();
+    for (int stride = size >> 1; stride >= 128; stride >>= 1) {
+      for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
+        const int lo = ((i / stride) * 2 * stride) + (i % stride), hi = lo + stride;
+        const unsigned long long a = s[lo], b = s[hi];
+        const bool up = (lo & size) == 0;
+        if ((a > b) == up) {
+          s[lo] = b;
+          s[hi] = a;
         }
       }
       __syncthreads();
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) k[i] = s[base + 4 * lane + i];
+#pragma unroll
+    for (int stride = 64; stride > 0; stride >>= 1) warp_stage64(k, base, lane, size, stride);
   }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) s[base + 4 * lane + i] = k[i];
+  __syncthreads();
 }
 
 // Sorts each tile of TILE consecutive words of a run in shared memory; the last tile of a run is
 // padded with all-ones words, which sort last.
 template <int TILE>
-__global__ void __launch_bounds__(1024)
+__global__ void __launch_bounds__(TILE / 4)
     k_tile_sort(unsigned long long *__restrict__ keys, long long run_len, int tiles_per_run) {
   __shared__ unsigned long long s[TILE];
   const long long run = blockIdx.x / tiles_per_run;
@@ -255,7 +365,7 @@ __global__ void __launch_bounds__(1024)
   const int n = (int)min((long long)TILE, run_len - tile0);
   for (int i = threadIdx.x; i < TILE; i += blockDim.x) s[i] = i < n ? keys[begin + i] : ~0ull;
   __syncthreads();
-  bitonic_sort_smem(s, TILE);
+  block_sort64(s);
   for (int i = threadIdx.x; i < n; i += blockDim.x) keys[begin + i] = s[i];
 }
 
@@ -306,88 +416,81 @@ __global__ void k_identity_perm(int32_t *__restrict__ perm, int N, long long tot
   if (x < total) perm[x] = (int32_t)(x % N);
 }
 
-// Segment-local query ordering fused with its input and outputs, one CTA per (query head,
-// segment) for segments of at most TILE queries: rho_i = DOT(q_i, u) for the segment's rows, a
-// sort of their order words in shared memory (skipped when the query ordering is off), perm_q,
-// and the block means Qbar of the segment's query blocks (the rows were just read, so the
-// gathered re-read mostly hits L2).
-template <int D, int TILE>
-__global__ void __launch_bounds__(512)
-    k_segment_order(const uint16_t *__restrict__ q, const float *__restrict__ u,
-                    float *__restrict__ rho, int32_t *__restrict__ perm_q,
-                    float *__restrict__ Qbar, int N, int S, int B, int nB, int query_perm) {
+// Segment-local query ordering, one CTA per (query head, segment) of at most TILE queries: the
+// order words of the segment's rho values sorted in shared memory (the identity when the query
+// ordering is off), written out as perm_q.
+template <int TILE>
+__global__ void __launch_bounds__(TILE / 4)
+    k_segment_sort(const float *__restrict__ rho, int32_t *__restrict__ perm_q, int N, int S,
+                   int query_perm) {
   __shared__ unsigned long long keys[TILE];
-  __shared__ float us[D];
   const long long qh = blockIdx.y;
   const int s0 = blockIdx.x * S;
-  for (int x = threadIdx.x; x < D; x += blockDim.x) us[x] = u[qh * D + x];
-  __syncthreads();
-  const uint16_t *Qh = q + (size_t)qh * N * D;
   for (int r = threadIdx.x; r < TILE; r += blockDim.x) {
-    if (r < S) {
-      const int i = s0 + r;
-      const float v = dot_row<D>(Qh + (size_t)i * D, us);
-      rho[qh * N + i] = v;
-      keys[r] = query_perm ? order_word(v, (uint32_t)i) : (unsigned long long)i;
-    } else {
-      keys[r] = ~0ull;
-    }
+    const int i = s0 + r;
+    keys[r] = r >= S ? ~0ull
+                     : query_perm ? order_word(__ldg(rho + qh * N + i), (uint32_t)i)
+                                  : (unsigned long long)i;
   }
   __syncthreads();
-  if (query_perm) bitonic_sort_smem(keys, TILE);
+  if (query_perm) block_sort64(keys);
   for (int r = threadIdx.x; r < S; r += blockDim.x)
     perm_q[qh * N + s0 + r] = (int32_t)(keys[r] & 0xffffffffull);
-  const int nbl = S / B;
-  const int items = nbl * (D / 4);
-  const float len = (float)B;
-  for (int it = threadIdx.x; it < items; it += blockDim.x) {
-    const int bl = it / (D / 4), t = (it % (D / 4)) * 4;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-    for (int e = 0; e < B; ++e) {
-      const int row = (int)(keys[bl * B + e] & 0xffffffffull);
-      const uint2 v = __ldg(reinterpret_cast<const uint2 *>(Qh + (size_t)row * D + t));
-      a0 = __fadd_rn(a0, bf16_lo(v.x));
-      a1 = __fadd_rn(a1, bf16_hi(v.x));
-      a2 = __fadd_rn(a2, bf16_lo(v.y));
-      a3 = __fadd_rn(a3, bf16_hi(v.y));
-    }
-    float *dst = Qbar + ((size_t)qh * nB + (size_t)(s0 / B) + bl) * D + t;
-    *reinterpret_cast<float4 *>(dst) =
-        make_float4(__fdiv_rn(a0, len), __fdiv_rn(a1, len), __fdiv_rn(a2, len), __fdiv_rn(a3, len));
-  }
 }
 
 // ------------------------------------------------------------------ blocks and scores
 
 // Block means over permuted blocks: out[(qh·nB + blk)] = MEAN(rows perm[blk·B .. blk·B+B-1]) of
-// source head src_head(qh) (the query head itself, or its KV head when kv_map is set).
+// source head src_head(qh) (the query head itself, or its KV head when kv_map is set). One warp
+// per block, D/32 columns per lane, the rows added in list order; row loads go out 16 at a time.
 template <int D>
 __global__ void __launch_bounds__(256)
     k_block_means(const uint16_t *__restrict__ src, const int32_t *__restrict__ perm,
                   float *__restrict__ out, int N, int B, int nB, long long n_blocks, int Hq,
                   int Hkv, int G, int kv_map) {
-  constexpr int P = D / 2;
-  constexpr int PER = 256 / P;
-  const long long blk = (long long)blockIdx.x * PER + threadIdx.x / P;
-  const int t = (threadIdx.x % P) * 2;
+  constexpr int CPL = D / 32;  // columns per lane (4 or 2)
+  using Vec = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
+  const long long blk = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
   if (blk >= n_blocks) return;
   const long long qh = blk / nB;
   const int b = (int)(blk % nB);
   const long long sh = kv_map ? (qh / Hq) * Hkv + (qh % Hq) / G : qh;
   const int32_t *pp = perm + qh * N + (size_t)b * B;
-  const uint16_t *base = src + (size_t)sh * N * D + t;
-  float a0 = 0.f, a1 = 0.f;
-#pragma unroll 4
-  for (int e = 0; e < B; ++e) {
-    const int row = __ldg(pp + e);
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(base + (size_t)row * D));
-    a0 = __fadd_rn(a0, bf16_lo(v));
-    a1 = __fadd_rn(a1, bf16_hi(v));
+  const Vec *base = reinterpret_cast<const Vec *>(src + (size_t)sh * N * D) + lane;
+  float acc[CPL];
+#pragma unroll
+  for (int x = 0; x < CPL; ++x) acc[x] = 0.f;
+  for (int e0 = 0; e0 < B; e0 += 32) {
+    const int my_row = min(max(__ldg(pp + e0 + lane), 0), N - 1);
+#pragma unroll
+    for (int h = 0; h < 32; h += 16) {
+      Vec v[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int row = __shfl_sync(0xffffffffu, my_row, h + e);
+        v[e] = __ldg(base + (size_t)row * (D / CPL));
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if constexpr (CPL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2 *>(&v[e]);
+          acc[0] = __fadd_rn(acc[0], bf16_lo(w.x));
+          acc[1] = __fadd_rn(acc[1], bf16_hi(w.x));
+          acc[2] = __fadd_rn(acc[2], bf16_lo(w.y));
+          acc[3] = __fadd_rn(acc[3], bf16_hi(w.y));
+        } else {
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(&v[e]);
+          acc[0] = __fadd_rn(acc[0], bf16_lo(w));
+          acc[1] = __fadd_rn(acc[1], bf16_hi(w));
+        }
+      }
+    }
   }
   const float len = (float)B;
-  *reinterpret_cast<float2 *>(out + (size_t)blk * D + t) =
-      make_float2(__fdiv_rn(a0, len), __fdiv_rn(a1, len));
+  float *dst = out + (size_t)blk * D + lane * CPL;
+#pragma unroll
+  for (int x = 0; x < CPL; ++x) dst[x] = __fdiv_rn(acc[x], len);
 }
 
 // n[qh][s][c] = number of keys of permuted key block c whose original index is below s·S.
@@ -413,9 +516,12 @@ __global__ void __launch_bounds__(256)
 }
 
 // r[qh][b][c] = DOT(Qbar_b, Kbar_c) × σ_d: a register-tiled fp32 product whose accumulators
-// each run the definition's sequential FMA chain over t = 0..D-1.
+// each run the definition's sequential FMA chain over t = 0..D-1. A 128×128 tile per CTA, 8×8
+// accumulators per thread (paired FMAs); the operands go through shared memory transposed, 32
+// values of t at a time, and the next 32 are loaded into registers while the current ones are
+// consumed.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
     k_block_scores(const float *__restrict__ Qbar, const float *__restrict__ Kbar,
                    float *__restrict__ r, int nB, float sigma) {
   __shared__ __align__(16) float As[32][128 + 4];
@@ -425,19 +531,44 @@ __global__ void __launch_bounds__(256)
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   const float *A = Qbar + (size_t)qh * nB * D;
   const float *Bm = Kbar + (size_t)qh * nB * D;
+  // Loader mapping: 4 float4 per matrix per thread: row = x / 8, t = (x % 8) * 4.
+  float4 pa[4], pb[4];
+  auto fetch = [&](int t0) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int x = threadIdx.x + k * 256, row = x / 8, t = (x % 8) * 4;
+      pa[k] = b0 + row < nB ? __ldg(reinterpret_cast<const float4 *>(A + (size_t)(b0 + row) * D + t0 + t))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      pb[k] = c0 + row < nB ? __ldg(reinterpret_cast<const float4 *>(Bm + (size_t)(c0 + row) * D + t0 + t))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto stash = [&]() {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int x = threadIdx.x + k * 256, row = x / 8, t = (x % 8) * 4;
+      As[t + 0][row] = pa[k].x;
+      As[t + 1][row] = pa[k].y;
+      As[t + 2][row] = pa[k].z;
+      As[t + 3][row] = pa[k].w;
+      Bs[t + 0][row] = pb[k].x;
+      Bs[t + 1][row] = pb[k].y;
+      Bs[t + 2][row] = pb[k].z;
+      Bs[t + 3][row] = pb[k].w;
+    }
+  };
   float2 acc[8][4];  // acc[i][jj] holds columns 2jj and 2jj+1
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
+  fetch(0);
   for (int t0 = 0; t0 < D; t0 += 32) {
-    for (int x = threadIdx.x; x < 128 * 32; x += 256) {
-      const int row = x / 32, tt = x % 32;
-      As[tt][row] = b0 + row < nB ? A[(size_t)(b0 + row) * D + t0 + tt] : 0.f;
-      Bs[tt][row] = c0 + row < nB ? Bm[(size_t)(c0 + row) * D + t0 + tt] : 0.f;
-    }
+    __syncthreads();  // the previous chunk has been consumed
+    stash();
     __syncthreads();
-#pragma unroll 4
+    if (t0 + 32 < D) fetch(t0 + 32);
+#pragma unroll 8
     for (int tt = 0; tt < 32; ++tt) {
       const float4 a0 = *reinterpret_cast<const float4 *>(&As[tt][tr * 8]);
       const float4 a1 = *reinterpret_cast<const float4 *>(&As[tt][tr * 8 + 4]);
@@ -451,17 +582,25 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fma2(make_float2(a[i], a[i]), v[j], acc[i][j]);
     }
-    __syncthreads();
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int b = b0 + tr * 8 + i;
     if (b >= nB) continue;
+    float *dst = r + ((size_t)qh * nB + b) * nB + c0 + tc * 8;
+    if (c0 + tc * 8 + 8 <= nB) {
+      reinterpret_cast<float4 *>(dst)[0] =
+          make_float4(__fmul_rn(acc[i][0].x, sigma), __fmul_rn(acc[i][0].y, sigma),
+                      __fmul_rn(acc[i][1].x, sigma), __fmul_rn(acc[i][1].y, sigma));
+      reinterpret_cast<float4 *>(dst)[1] =
+          make_float4(__fmul_rn(acc[i][2].x, sigma), __fmul_rn(acc[i][2].y, sigma),
+                      __fmul_rn(acc[i][3].x, sigma), __fmul_rn(acc[i][3].y, sigma));
+    } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = c0 + tc * 8 + j;
-      const float x = (j & 1) ? acc[i][j >> 1].y : acc[i][j >> 1].x;
-      if (c < nB) r[((size_t)qh * nB + b) * nB + c] = __fmul_rn(x, sigma);
+      for (int j = 0; j < 8; ++j) {
+        const float x = (j & 1) ? acc[i][j >> 1].y : acc[i][j >> 1].x;
+        if (c0 + tc * 8 + j < nB) dst[j] = __fmul_rn(x, sigma);
+      }
     }
   }
 }
@@ -527,12 +666,13 @@ __global__ void __launch_bounds__(128)
     any = any || other_any;
   }
 
+  const double Md = (double)M;
   // Weights (independent per block, computed lane-strided), then Z: chunks of 32 consecutive
   // blocks, chunk k summed sequentially by lane k mod 32, then the chunk sums in chunk order.
 #pragma unroll 4
   for (int c = lane; c < nB; c += kWarp) {
     const int nv = __ldg(nn + c);
-    w[wi(c)] = nv > 0 ? __dmul_rn((double)nv, exp64(__dsub_rn((double)__ldg(rr + c), (double)M)))
+    w[wi(c)] = nv > 0 ? __dmul_rn(int_to_double(nv), exp64(__dsub_rn((double)__ldg(rr + c), Md)))
                       : 0.0;
   }
   __syncwarp();
@@ -721,12 +861,12 @@ cudaError_t sort_runs(unsigned long long *a, unsigned long long *b, long long to
   const int tiles_per_run = (int)((run_len + tile - 1) / tile);
   const unsigned grid = (unsigned)((total / run_len) * tiles_per_run);
   if (tile == 1024)
-    k_tile_sort<1024><<<grid, 512, 0, st>>>(a, run_len, tiles_per_run);
+    k_tile_sort<1024><<<grid, 256, 0, st>>>(a, run_len, tiles_per_run);
   else if (tile == 2048)
-    k_tile_sort<2048><<<grid, 1024, 0, st>>>(a, run_len, tiles_per_run);
+    k_tile_sort<2048><<<grid, 512, 0, st>>>(a, run_len, tiles_per_run);
   else
     k_tile_sort<4096><<<grid, 1024, 0, st>>>(a, run_len, tiles_per_run);
-    note_launch();
+  note_launch();
   unsigned long long *src = a, *dst = b;
   for (long long width = tile; width < run_len; width *= 2) {
     k_merge_pass<<<blocks_for((total + kMergeItems - 1) / kMergeItems, 256), 256, 0, st>>>(
@@ -761,29 +901,28 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   int32_t *ncount = reinterpret_cast<int32_t *>(ws + L.ncount);
 
   const long long bhq = d.bhq(), bhkv = d.bhkv();
-  const long long nq = bhq * d.N, nkv_rows = bhkv * d.N;
+  const long long nq = bhq * d.N;
   cudaError_t e;
 
-  // Step 1a: mean query per query head, mean key per KV head, kappa.
+  // Step 1a: mean query per query head; one pass over K for kappa and the mean key per KV head.
   k_pool_chunks<D><<<blocks_for(nq / d.B * (D / 2), 256), 256, 0, st>>>(q, qchunk, d.B, nq / d.B);
   note_launch();
-  k_pool_chunks<D><<<blocks_for(nkv_rows / d.B * (D / 2), 256), 256, 0, st>>>(k, kchunk, d.B,
-                                                                               nkv_rows / d.B);
-  note_launch();
-  const size_t fin_smem = (size_t)128 * D * sizeof(float);
+  const size_t fin_smem = (size_t)1024 * 32 * sizeof(float);
   if ((e = cudaFuncSetAttribute(k_pool_finish<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)fin_smem)) != cudaSuccess)
     return e;
-  k_pool_finish<D><<<(unsigned)bhq, D, fin_smem, st>>>(qchunk, qbar, d.nB, (float)d.N);
+  k_pool_finish<D><<<dim3(D / 32, (unsigned)bhq), 256, fin_smem, st>>>(qchunk, qbar, d.nB,
+                                                                       (float)d.N);
   note_launch();
-  k_pool_finish<D><<<(unsigned)bhkv, D, fin_smem, st>>>(kchunk, kbar_all, d.nB, (float)d.N);
-  note_launch();
-  const size_t kappa_smem = (size_t)d.G * D * sizeof(float);
-  if ((e = cudaFuncSetAttribute(k_kappa<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kappa_smem)) != cudaSuccess)
+  const size_t kpass_smem = (size_t)d.G * D * sizeof(float) + (size_t)d.B * D * 2;
+  if ((e = cudaFuncSetAttribute(k_kpass<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kpass_smem)) != cudaSuccess)
     return e;
-  k_kappa<D><<<dim3((d.N + 127) / 128, (unsigned)bhkv), 128, kappa_smem, st>>>(k, qbar, kappa, d.N,
-                                                                              d.Hq, d.Hkv, d.G);
+  k_kpass<D><<<dim3((unsigned)d.nB, (unsigned)bhkv), 128, kpass_smem, st>>>(
+      k, qbar, kappa, kchunk, d.N, d.B, d.Hq, d.Hkv, d.G);
+  note_launch();
+  k_pool_finish<D><<<dim3(D / 32, (unsigned)bhkv), 256, fin_smem, st>>>(kchunk, kbar_all, d.nB,
+                                                                         (float)d.N);
   note_launch();
   // Step 2a: global key/value ordering.
   k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(kappa, keys0, d.N, nq);
@@ -793,42 +932,37 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   k_kbar_top<<<(unsigned)bhq, D, 0, st>>>(k, out.perm_k, kbar_all, kbar_top, u, d.N, D, d.B, d.Hq,
                                           d.Hkv, d.G);
   note_launch();
-  // Step 2b: segment-local query ordering, with rho and the query block means.
+  // Step 2b: query scores, segment-local query ordering, query block means.
   const long long nblk = bhq * d.nB;
-  constexpr int PER = 256 / (D / 2);
   const int qp = cfg.query_perm ? 1 : 0;
+  k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
+  note_launch();
   const dim3 seg_grid((unsigned)d.nSeg, (unsigned)bhq);
-  if (d.S <= 512) {
-    k_segment_order<D, 512><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
-                                                      d.nB, qp);
-  } else if (d.S <= 1024) {
-    k_segment_order<D, 1024><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
-                                                       d.nB, qp);
-  } else if (d.S <= 2048) {
-    k_segment_order<D, 2048><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
-                                                       d.nB, qp);
-  } else if (d.S <= 4096) {
-    k_segment_order<D, 4096><<<seg_grid, 512, 0, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
-                                                       d.nB, qp);
-  } else {
-    // Segments longer than the shared-memory sort: rho, a sort of each segment, block means.
-    k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
+  if (d.S <= 4096) {
+    if (d.S <= 512)
+      k_segment_sort<512><<<seg_grid, 128, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
+    else if (d.S <= 1024)
+      k_segment_sort<1024><<<seg_grid, 256, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
+    else if (d.S <= 2048)
+      k_segment_sort<2048><<<seg_grid, 512, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
+    else
+      k_segment_sort<4096><<<seg_grid, 1024, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
     note_launch();
-    if (qp) {
-      k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(rho, keys0, d.N, nq);
-      note_launch();
-      if ((e = sort_runs(keys0, keys1, nq, d.S, out.perm_q, st)) != cudaSuccess) return e;
-    } else {
-      k_identity_perm<<<blocks_for(nq, 256), 256, 0, st>>>(out.perm_q, d.N, nq);
-      note_launch();
-    }
-    k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
-                                                            nblk, d.Hq, d.Hkv, d.G, 0);
+  } else if (qp) {
+    // Segments longer than the shared-memory sort: merge sort of the order words per segment.
+    k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(rho, keys0, d.N, nq);
+    note_launch();
+    if ((e = sort_runs(keys0, keys1, nq, d.S, out.perm_q, st)) != cudaSuccess) return e;
+  } else {
+    k_identity_perm<<<blocks_for(nq, 256), 256, 0, st>>>(out.perm_q, d.N, nq);
+    note_launch();
   }
+  k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
+                                                        nblk, d.Hq, d.Hkv, d.G, 0);
   note_launch();
   // Key block means, visibility counts, block scores.
-  k_block_means<D><<<blocks_for(nblk, PER), 256, 0, st>>>(k, out.perm_k, Kbar, d.N, d.B, d.nB,
-                                                          nblk, d.Hq, d.Hkv, d.G, 1);
+  k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(k, out.perm_k, Kbar, d.N, d.B, d.nB, nblk,
+                                                        d.Hq, d.Hkv, d.G, 1);
   note_launch();
   const size_t nc_smem = (size_t)32 * (d.B + 1) * sizeof(int);
   k_ncount<<<dim3((d.nB + 31) / 32, (unsigned)bhq), 256, nc_smem, st>>>(out.perm_k, ncount, d.N,
