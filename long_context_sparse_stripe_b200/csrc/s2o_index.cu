@@ -85,6 +85,19 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 acc) {
   return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
 }
 
+// 16-byte asynchronous copy global -> shared (cached in L2 only), and the wait for all of this
+// thread's copies. A CTA stages contiguous rows this way with no registers held per load, so many
+// loads are in flight.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Sort key of an fp32 score: monotone in the value, −0 folded onto +0, NaN below everything.
 __device__ __forceinline__ uint32_t sort_key(float x) {
   uint32_t b = __float_as_uint(x);
@@ -192,44 +205,59 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x < 32) out[head * D + col0 + threadIdx.x] = __fdiv_rn(acc, len);
 }
 
-// One pass over K, one CTA per chunk of B key rows of a KV head:
-//   kappa_j = DOT(qbar_h, k_j) for the G query heads of the group (one thread per key row, the row
-//   in registers, qbar read four values at a time from shared memory), and
-//   the chunk sum of the MEAN rule for kbar_all (the rows staged in shared memory, one thread per
+// One pass over K, one CTA per chunk of B key rows of a KV head. The chunk's rows (contiguous in
+// memory) are staged in shared memory with coalesced asynchronous copies (rows padded by 16 bytes,
+// so that per-row reads are free of bank conflicts), then:
+//   kappa_j = DOT(qbar_h, k_j) for the G query heads of the group (one thread per key row, qbar
+//   read four values at a time), and the chunk sum of the MEAN rule for kbar_all (one thread per
 //   two columns adding the rows in order).
 template <int D>
 __global__ void __launch_bounds__(128)
     k_kpass(const uint16_t *__restrict__ k, const float *__restrict__ qbar,
             float *__restrict__ kappa, float *__restrict__ kchunk, int N, int B, int Hq, int Hkv,
             int G) {
+  constexpr int RS = D * 2 + 16;  // staged row stride in bytes
   extern __shared__ float4 sm4[];
-  float *qb = reinterpret_cast<float *>(sm4);                     // [G][D]
-  uint4 *rows = reinterpret_cast<uint4 *>(sm4 + (size_t)G * D / 4);  // [B][D/8]
+  float *qb = reinterpret_cast<float *>(sm4);                                     // [G][D]
+  unsigned char *rows = reinterpret_cast<unsigned char *>(sm4 + (size_t)G * D / 4);  // [B][RS]
   const long long kh = blockIdx.y;
   const int chunk = blockIdx.x, r = threadIdx.x;
   const long long beta = kh / Hkv;
   const int g = (int)(kh % Hkv);
   const size_t qh0 = (size_t)beta * Hq + (size_t)g * G;
+  const unsigned char *src =
+      reinterpret_cast<const unsigned char *>(k + ((size_t)kh * N + (size_t)chunk * B) * D);
+  for (int x = threadIdx.x; x < B * (D / 8); x += blockDim.x)
+    cp_async16(rows + (x / (D / 8)) * RS + (x % (D / 8)) * 16, src + (size_t)x * 16);
   for (int x = threadIdx.x; x < G * D; x += blockDim.x) qb[x] = qbar[qh0 * D + x];
+  cp_async_wait_all();
+  __syncthreads();
   const int j = chunk * B + r;
-  uint4 v[D / 8];
   if (r < B) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(k + ((size_t)kh * N + j) * D);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      v[c] = __ldg(src + c);
-      rows[r * (D / 8) + c] = v[c];
+    const uint4 *row = reinterpret_cast<const uint4 *>(rows + r * RS);
+    for (int hi = 0; hi < G; ++hi) {
+      const float4 *qv = sm4 + (size_t)hi * D / 4;
+      float acc = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = row[c];
+        const float4 a = qv[2 * c], b = qv[2 * c + 1];
+        acc = __fmaf_rn(bf16_lo(v.x), a.x, acc);
+        acc = __fmaf_rn(bf16_hi(v.x), a.y, acc);
+        acc = __fmaf_rn(bf16_lo(v.y), a.z, acc);
+        acc = __fmaf_rn(bf16_hi(v.y), a.w, acc);
+        acc = __fmaf_rn(bf16_lo(v.z), b.x, acc);
+        acc = __fmaf_rn(bf16_hi(v.z), b.y, acc);
+        acc = __fmaf_rn(bf16_lo(v.w), b.z, acc);
+        acc = __fmaf_rn(bf16_hi(v.w), b.w, acc);
+      }
+      kappa[(qh0 + hi) * N + j] = acc;
     }
   }
-  __syncthreads();
-  if (r < B)
-    for (int hi = 0; hi < G; ++hi)
-      kappa[(qh0 + hi) * N + j] = dot_regs<D>(v, sm4 + (size_t)hi * D / 4);
   if (r < D / 2) {
-    const uint32_t *rw = reinterpret_cast<const uint32_t *>(rows);
     float a0 = 0.f, a1 = 0.f;
     for (int e = 0; e < B; ++e) {
-      const uint32_t w = rw[e * (D / 2) + r];
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(rows + e * RS + r * 4);
       a0 = __fadd_rn(a0, bf16_lo(w));
       a1 = __fadd_rn(a1, bf16_hi(w));
     }
@@ -255,23 +283,32 @@ __global__ void k_kbar_top(const uint16_t *__restrict__ k, const int32_t *__rest
   u[qh * D + t] = __fsub_rn(top, kbar_all[kh * D + t]);
 }
 
-// rho_i = DOT(q_i, u_h), one thread per query row (the row in registers, u read four values at a
-// time from shared memory).
+// rho_i = DOT(q_i, u_h), one thread per query row. A CTA's 128 rows (contiguous) are staged in
+// shared memory with coalesced asynchronous copies (rows padded by 16 bytes), then each thread
+// reads its row and runs the chain with u read four values at a time.
 template <int D>
 __global__ void __launch_bounds__(128)
     k_rho(const uint16_t *__restrict__ q, const float *__restrict__ u, float *__restrict__ rho,
           int N) {
+  constexpr int RS = D * 2 + 16;
+  __shared__ __align__(16) unsigned char rows[128 * RS];
   __shared__ float4 us4[D / 4];
   const long long qh = blockIdx.y;
-  const int i = blockIdx.x * 128 + threadIdx.x;
+  const int i0 = blockIdx.x * 128;
+  const int nrows = min(128, N - i0);
+  const unsigned char *src =
+      reinterpret_cast<const unsigned char *>(q + ((size_t)qh * N + i0) * D);
+  for (int x = threadIdx.x; x < nrows * (D / 8); x += blockDim.x)
+    cp_async16(rows + (x / (D / 8)) * RS + (x % (D / 8)) * 16, src + (size_t)x * 16);
   if (threadIdx.x < D / 4) us4[threadIdx.x] = reinterpret_cast<const float4 *>(u + qh * D)[threadIdx.x];
+  cp_async_wait_all();
   __syncthreads();
-  if (i >= N) return;
+  if (threadIdx.x >= nrows) return;
   uint4 v[D / 8];
-  const uint4 *src = reinterpret_cast<const uint4 *>(q + ((size_t)qh * N + i) * D);
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) v[c] = __ldg(src + c);
-  rho[qh * N + i] = dot_regs<D>(v, us4);
+  for (int c = 0; c < D / 8; ++c)
+    v[c] = *reinterpret_cast<const uint4 *>(rows + threadIdx.x * RS + c * 16);
+  rho[qh * N + i0 + threadIdx.x] = dot_regs<D>(v, us4);
 }
 
 // ------------------------------------------------------------------ ordering (step 2)
@@ -645,15 +682,26 @@ __global__ void __launch_bounds__(128)
   const float *rr = r + (size_t)qb * nB;
   const int32_t *nn = ncount + ((size_t)qh * nSeg + s) * nB;
 
-  // M = max block score over the candidates (blocks with a visible key).
+  // M = max block score over the candidates (blocks with a visible key). A lane's blocks are
+  // c = lane + 32k; their counts and scores are loaded 16 at a time.
+  constexpr int kBatch = 16;
   float M = 0.f;
   bool any = false;
-  for (int c = lane; c < nB; c += kWarp) {
-    if (__ldg(nn + c) > 0) {
-      const float x = __ldg(rr + c);
-      M = any ? fmaxf(M, x) : x;
-      any = true;
+  for (int c0 = 0; c0 < nB; c0 += kBatch * kWarp) {
+    int nv[kBatch];
+    float rv[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int c = c0 + k * kWarp + lane;
+      nv[k] = c < nB ? __ldg(nn + c) : 0;
+      rv[k] = c < nB ? __ldg(rr + c) : 0.f;
     }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k)
+      if (nv[k] > 0) {
+        M = any ? fmaxf(M, rv[k]) : rv[k];
+        any = true;
+      }
   }
   if (__ballot_sync(full, any) == 0) {
     if (lane == 0) sel_cnt[qb] = 0;
@@ -667,13 +715,26 @@ __global__ void __launch_bounds__(128)
   }
 
   const double Md = (double)M;
-  // Weights (independent per block, computed lane-strided), then Z: chunks of 32 consecutive
-  // blocks, chunk k summed sequentially by lane k mod 32, then the chunk sums in chunk order.
-#pragma unroll 4
-  for (int c = lane; c < nB; c += kWarp) {
-    const int nv = __ldg(nn + c);
-    w[wi(c)] = nv > 0 ? __dmul_rn(int_to_double(nv), exp64(__dsub_rn((double)__ldg(rr + c), Md)))
-                      : 0.0;
+  // Weights (independent per block, computed lane-strided; -1 marks a block that is not a
+  // candidate), then Z: chunks of 32 consecutive blocks, chunk k summed sequentially by lane
+  // k mod 32 (a non-candidate adds +0), then the chunk sums in chunk order.
+  for (int c0 = 0; c0 < nB; c0 += kBatch * kWarp) {
+    int nv[kBatch];
+    float rv[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int c = c0 + k * kWarp + lane;
+      nv[k] = c < nB ? __ldg(nn + c) : 0;
+      rv[k] = c < nB ? __ldg(rr + c) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int c = c0 + k * kWarp + lane;
+      if (c < nB)
+        w[wi(c)] = nv[k] > 0
+                       ? __dmul_rn(int_to_double(nv[k]), exp64(__dsub_rn((double)rv[k], Md)))
+                       : -1.0;
+    }
   }
   __syncwarp();
   const int n_chunks = (nB + 31) / 32;
@@ -681,7 +742,10 @@ __global__ void __launch_bounds__(128)
   for (int k = lane; k < n_chunks; k += kWarp) {
     double part = 0.0;
     const int c_end = min(nB, 32 * k + 32);
-    for (int c = 32 * k; c < c_end; ++c) part = __dadd_rn(part, w[wi(c)]);
+    for (int c = 32 * k; c < c_end; ++c) {
+      const double wc = w[wi(c)];
+      part = __dadd_rn(part, wc < 0.0 ? 0.0 : wc);
+    }
     if (k < kWarp)
       part0 = part;
     else
@@ -701,12 +765,10 @@ __global__ void __launch_bounds__(128)
     const int c = c0 + lane;
     bool sel = false;
     double p = 0.0;
-    if (c < nB && __ldg(nn + c) > 0) {
-      const double wc = w[wi(c)];
-      if (tau == 0.0 || !(wc < t_lo)) {
-        p = __ddiv_rn(wc, Z);
-        sel = p >= tau;
-      }
+    const double wc = c < nB ? w[wi(c)] : -1.0;
+    if (wc >= 0.0 && (tau == 0.0 || !(wc < t_lo))) {
+      p = __ddiv_rn(wc, Z);
+      sel = p >= tau;
     }
     const unsigned m = __ballot_sync(full, sel);
     const int slot = cnt + __popc(m & ((1u << lane) - 1u));
@@ -914,7 +976,7 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   k_pool_finish<D><<<dim3(D / 32, (unsigned)bhq), 256, fin_smem, st>>>(qchunk, qbar, d.nB,
                                                                        (float)d.N);
   note_launch();
-  const size_t kpass_smem = (size_t)d.G * D * sizeof(float) + (size_t)d.B * D * 2;
+  const size_t kpass_smem = (size_t)d.G * D * sizeof(float) + (size_t)d.B * (D * 2 + 16);
   if ((e = cudaFuncSetAttribute(k_kpass<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kpass_smem)) != cudaSuccess)
     return e;
