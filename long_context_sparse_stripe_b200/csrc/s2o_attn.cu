@@ -48,6 +48,7 @@ namespace {
 
 constexpr int kThreads = 352;
 constexpr int kM = 128;  // query rows per tile (UMMA M)
+constexpr int kList = 256;  // units per work-list window
 constexpr uint64_t kDrainNs = 2000000000ull;
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -237,7 +238,8 @@ struct Layout {
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
-  static constexpr uint32_t SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t OFF_LIST = OFF_BAR + BAR_BYTES;  // work list: kList units + count
+  static constexpr uint32_t SMEM = OFF_LIST + kList * 4 + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;    // S_x at S_COL + 128·x (P_x over its first BN/2 columns)
   static constexpr uint32_t O_COL = 256;  // O_x at O_COL + D·x
@@ -258,11 +260,19 @@ enum Bar {
   kNumBars = 27
 };
 
+// Unit sets of a launch.
+enum Mode {
+  kPermuted = 0,  // query blocks of perm_q: local tiles then the selected list
+  kDense = 1,     // dense causal attention (Eq. 1): original-order blocks, all earlier keys
+  kLocal = 2      // the dense local window only: original-order blocks, keys of their segment
+};
+
 struct Params {
   const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
   uint16_t *o;
   int N, S, nB, nSeg, Hq, Hkv, G;
-  int dense;
+  int mode;
+  int skip_empty;  // permuted mode: only blocks with a non-empty selected list
   long long n_units, n_items;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
@@ -274,9 +284,9 @@ struct Unit {
   const int32_t *sel;  // the query block's selected list (sel_blk row)
 };
 
-// Unit order: S2O keeps the units of one (batch, KV head, segment) together, query heads of the
-// group fastest, so that the segment's K/V tiles stay in L2 and paired units share local tiles;
-// the dense baseline runs the longest query blocks first.
+// Unit order: the permuted and local modes keep the units of one (batch, KV head, segment)
+// together, query heads of the group fastest, so that the segment's K/V tiles stay in L2 and
+// paired units share local tiles; the dense baseline runs the longest query blocks first.
 template <int BN>
 __device__ __forceinline__ Unit decode_unit(const Params &p, long long u) {
   Unit r;
@@ -284,7 +294,7 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, long long u) {
   u /= p.G;
   const int per_seg = p.S / BN;
   int b;
-  if (p.dense) {
+  if (p.mode == kDense) {
     b = p.nB - 1 - (int)(u % p.nB);
     u /= p.nB;
   } else {
@@ -300,8 +310,8 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, long long u) {
   r.kh = beta * p.Hkv + g;
   r.b = b;
   r.seg0 = (int)((long long)b * BN / p.S) * p.S;
-  if (p.dense) {
-    r.lt = b + 1;
+  if (p.mode != kPermuted) {
+    r.lt = b - r.seg0 / BN + 1;  // the causal triangle of the block's segment (or sequence)
     r.cnt = 0;
     r.sel = nullptr;
   } else {
@@ -321,13 +331,15 @@ struct Pair {
   int total;   // stream length
 };
 
+// Work item i of the current window: units list[2i] and list[2i+1] (the second may be absent).
 template <int BN>
-__device__ __forceinline__ Pair decode_pair(const Params &p, long long w) {
+__device__ __forceinline__ Pair decode_pair(const Params &p, const uint32_t *list, int n_list,
+                                            int i) {
   Pair P;
-  P.u0 = decode_unit<BN>(p, 2 * w);
-  P.valid1 = 2 * w + 1 < p.n_units;
+  P.u0 = decode_unit<BN>(p, list[2 * i]);
+  P.valid1 = 2 * i + 1 < n_list;
   if (P.valid1) {
-    P.u1 = decode_unit<BN>(p, 2 * w + 1);
+    P.u1 = decode_unit<BN>(p, list[2 * i + 1]);
   } else {
     P.u1 = P.u0;
     P.u1.lt = 0;
@@ -485,10 +497,53 @@ __device__ __forceinline__ void mma8_ts(uint32_t d, uint32_t idesc, const uint32
       : "memory");
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// Fills the work list for window k0 of this CTA's share (warp 0; returns the entry count, or -1
+// past the end of the share). Without skipping, the share is the work items w = blockIdx.x +
+// k·gridDim.x, each contributing its units 2w and 2w+1 (adjacent units, which usually share
+// local tiles); with skip_empty it is the units u = blockIdx.x + k·gridDim.x whose selected list
+// is not empty, paired in list order.
+template <int BN>
+__device__ int build_list(const Params &p, long long k0, uint32_t *list, int lane) {
+  const long long span = p.skip_empty ? kList : kList / 2;
+  const long long first = blockIdx.x + k0 * gridDim.x;
+  if (first >= (p.skip_empty ? p.n_units : p.n_items)) return -1;
+  int n = 0;
+  for (long long k = k0; k < k0 + span; k += 32) {
+    const long long pos = blockIdx.x + (k + lane) * gridDim.x;
+    if (p.skip_empty) {
+      bool keep = false;
+      if (pos < p.n_units) {
+        const Unit un = decode_unit<BN>(p, pos);
+        keep = un.cnt > 0;
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) list[n + __popc(m & ((1u << lane) - 1u))] = (uint32_t)pos;
+      n += __popc(m);
+    } else {
+      const bool keep = pos < p.n_items;
+      const bool two = 2 * pos + 1 < p.n_units;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      const unsigned m2 = __ballot_sync(0xffffffffu, keep && two);
+      // Only the last item of all can hold a single unit, so lower lanes hold two each.
+      if (keep) {
+        const int at = n + 2 * __popc(m & ((1u << lane) - 1u));
+        list[at] = (uint32_t)(2 * pos);
+        if (two) list[at + 1] = (uint32_t)(2 * pos + 1);
+      }
+      n += __popc(m) + __popc(m2);
+    }
+  }
+  return n;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -556,12 +611,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint64_t lim = p.limit_ns;
   bool ok = true;
+  // Work comes in windows of this CTA's share: warp 0 fills the work list between two CTA-wide
+  // barriers and every role then walks the window's items (a role that gave up a bounded wait
+  // keeps meeting the barriers without working).
+  uint32_t *list = reinterpret_cast<uint32_t *>(smem + L::OFF_LIST);
+  volatile int *list_n = reinterpret_cast<volatile int *>(smem + L::OFF_LIST + kList * 4);
+  auto for_each_window = [&](auto &&body) {
+    for (long long k0 = 0;; k0 += p.skip_empty ? kList : kList / 2) {
+      named_bar_sync(1, kThreads);
+      if (warp == 0) {
+        const int n = build_list<BN>(p, k0, list, lane);
+        if (lane == 0) *list_n = n;
+        __syncwarp();
+      }
+      named_bar_sync(1, kThreads);
+      const int n_list = *list_n;
+      if (n_list < 0) break;
+      body(n_list);
+    }
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- K / V producer
     long long kj = 0;  // stream items issued so far (all work items of this CTA)
-    for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
-      const Pair P = decode_pair<BN>(p, w);
+    for_each_window([&](int n_list) {
+    for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
+      const Pair P = decode_pair<BN>(p, list, n_list, wi);
       for (int j = 0; j < P.total; ++j) {
         const Item it = item_at(P, j);
         const int ks = (int)(kj % L::KST), vs = (int)(kj % L::VST);
@@ -588,6 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++kj;
       }
     }
+    });
     // Drain: the last copy issued into each stage must have landed before the CTA exits.
     if (lane == 0) {
       drain_ring(bar(kKFull), L::KST, kj);
@@ -597,8 +673,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ---------------------------------------------------------------- Q producer
     long long qn[2] = {0, 0};
-    for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
-      const Pair P = decode_pair<BN>(p, w);
+    for_each_window([&](int n_list) {
+    for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
+      const Pair P = decode_pair<BN>(p, list, n_list, wi);
       for (int x = 0; ok && x < 1 + P.valid1; ++x) {
         if (qn[x] >= 1 &&
             !warp_wait(bar(kQEmpty + x), (uint32_t)((qn[x] - 1) & 1), lim, lane)) {
@@ -610,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit &u = x ? P.u1 : P.u0;
         const uint32_t dst = sQ + x * L::Q_BYTES;
         const int q_row0 = (int)(u.qh * p.N);
-        if (p.dense || p.perm_q == nullptr) {
+        if (p.mode != kPermuted || p.perm_q == nullptr) {
           if (lane == 0)
             for (int a = 0; a < D / 64; ++a)
               tma_load_tile(dst + a * L::ATOM_Q, &tm_q_tile, a * 64, q_row0 + u.b * BN,
@@ -628,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++qn[x];
       }
     }
+    });
     if (lane == 0)
       for (int x = 0; x < 2; ++x)
         if (qn[x] > 0) mbar_wait(bar(kQFull + x), (uint32_t)((qn[x] - 1) & 1), kDrainNs);
@@ -637,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One thread issues every tensor-core operation. Its loop is kept short (32-bit counters,
     // descriptors advanced by constant offsets): it shares a scheduler with two softmax warps
     // that issue back to back, and each of its instructions delays the next product.
-    if (lane == 0) {
+    {
       constexpr uint32_t kIdescQK = idesc_bf16(kM, BN, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16(kM, D, 0, 1);
       static_assert((L::VST & (L::VST - 1)) == 0, "V ring depth must be a power of two");
@@ -662,8 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t k_st = 0, k_ph = 0;  // K ring stage and phase of the next stream item
       uint32_t v_base = 0;          // stream items of this CTA's earlier work items
       uint32_t q_ph[2] = {0, 0}, p_ph[2] = {0, 0};
-      for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
-        const Pair P = decode_pair<BN>(p, w);
+      for_each_window([&](int n_list) {
+      if (lane == 0)
+      for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
+        const Pair P = decode_pair<BN>(p, list, n_list, wi);
         if (!mbar_wait(bar(kQFull + 0), q_ph[0], lim) ||
             (P.valid1 && !mbar_wait(bar(kQFull + 1), q_ph[1], lim))) {
           ok = false;
@@ -767,9 +847,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         v_base += (uint32_t)P.total;
       }
+      __syncwarp();
+      });
       // Drain: every tensor-core operation issued above completes before TMEM is freed.
-      tc_commit(bar(kDrain));
-      mbar_wait(bar(kDrain), 0, kDrainNs);
+      if (lane == 0) {
+        tc_commit(bar(kDrain));
+        mbar_wait(bar(kDrain), 0, kDrainNs);
+      }
     }
     __syncwarp();
   } else {
@@ -783,8 +867,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const unsigned full = 0xffffffffu;
     const float sl2 = p.scale_log2;
     long long sn = 0, on = 0;  // S_x tiles and work items consumed
-    for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
-      const Pair P = decode_pair<BN>(p, w);
+    for_each_window([&](int n_list) {
+    for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
+      const Pair P = decode_pair<BN>(p, list, n_list, wi);
       if (x == 1 && !P.valid1) continue;
       const Unit u = x ? P.u1 : P.u0;
       const int seg0 = u.seg0;
@@ -792,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int i_orig = seg0 + p.S - 1;
       bool store_row = false;
       if (row < BN) {
-        const int v = (p.dense || p.perm_q == nullptr)
+        const int v = (p.mode != kPermuted || p.perm_q == nullptr)
                           ? u.b * BN + row
                           : __ldg(p.perm_q + u.qh * p.N + (size_t)u.b * BN + row);
         store_row = v >= seg0 && v < seg0 + p.S;
@@ -925,6 +1010,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
     }
+    });
   }
 
   __syncthreads();
@@ -1002,22 +1088,33 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
   p.local_tiles = a.local_tiles;
   p.o = static_cast<uint16_t *>(a.o);
   p.N = d.N;
-  p.S = a.dense ? d.N : d.S;
   p.nB = d.nB;
-  p.nSeg = a.dense ? 1 : d.nSeg;
   p.Hq = d.Hq;
   p.Hkv = d.Hkv;
   p.G = d.G;
-  p.dense = a.dense ? 1 : 0;
   p.n_units = d.bhq() * d.nB;
   p.n_items = (p.n_units + 1) / 2;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   p.limit_ns = limit_ns;
-  const long long grid = p.n_items < sm_count() ? p.n_items : sm_count();
-  s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv, tvr,
-                                                                         p);
-  note_launch();
-  return cudaGetLastError();
+  auto launch = [&](int mode, int skip_empty) -> cudaError_t {
+    p.mode = mode;
+    p.skip_empty = skip_empty;
+    p.S = mode == kDense ? d.N : d.S;
+    p.nSeg = mode == kDense ? 1 : d.nSeg;
+    const long long work = skip_empty ? p.n_units : p.n_items;
+    const long long grid = work < sm_count() ? work : sm_count();
+    s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv,
+                                                                           tvr, p);
+    note_launch();
+    return cudaGetLastError();
+  };
+  if (a.dense) return launch(kDense, 0);
+  // S2O: every row first gets the dense local window of its segment, computed in original order
+  // (causal triangles, masks on diagonal tiles only); then the query blocks whose selected list is
+  // not empty are recomputed in full (local tiles and selected blocks, permuted order) and
+  // overwrite their rows. Each row's result is the attention over its key set either way.
+  if ((e = launch(kLocal, 0)) != cudaSuccess) return e;
+  return launch(kPermuted, 1);
 }
 
 }  // namespace

@@ -617,7 +617,10 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma2(make_float2(a[i], a[i]), v[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j].x = __fmaf_rn(a[i], v[j].x, acc[i][j].x);
+          acc[i][j].y = __fmaf_rn(a[i], v[j].y, acc[i][j].y);
+        }
     }
   }
 #pragma unroll
