@@ -254,7 +254,15 @@ def run_s2o(args):
 
     stats = s2o.index_stats(cfg, idx, ws)
     tile_flops = 4.0 * w.block_size * w.block_size * w.head_dim
-    exec_flops = stats.executed_tiles * tile_flops
+    # Tiles the attention kernel executes: the local pass runs every segment's causal triangle in
+    # original order; the permuted pass reruns the query blocks with a non-empty selected list
+    # (their local tiles plus the selected blocks).
+    per_seg = w.segment_len // w.block_size
+    local_pass = w.batch * w.n_q_heads * (w.seq_len // w.segment_len) * per_seg * (per_seg + 1) // 2
+    busy = idx.sel_cnt > 0
+    permuted_pass = int((idx.local_tiles[busy].long() + idx.sel_cnt[busy].long()).sum().item())
+    kernel_tiles = local_pass + permuted_pass
+    exec_flops = kernel_tiles * tile_flops
     peak, hbm_peak, peak_kind = measured_peaks()
 
     # Dense causal baseline on the same inputs, and the MSE of the S2O output against it.
@@ -315,11 +323,13 @@ def run_s2o(args):
             "pair_sparsity": stats.pair_sparsity,
             "tile_density": stats.executed_tiles * w.block_size ** 2 * 1.0 / stats.causal_pairs,
             "executed_tiles": stats.executed_tiles, "local_tiles": stats.local_tiles,
-            "selected_tiles": stats.selected_tiles, "mse_vs_dense": mse,
+            "selected_tiles": stats.selected_tiles,
+            "kernel_tiles": {"local_pass": local_pass, "permuted_pass": permuted_pass},
+            "mse_vs_dense": mse,
             "exec_tflops": achieved,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                         "kernel": "s2o_attention_kernel<128,128>",
+                         "kernel": "s2o_attention_kernel<128,128> (local + permuted pass)",
                          "peak_source": f"{peak_kind} bf16 (burst)"},
             "e2e": {"value": flops_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
