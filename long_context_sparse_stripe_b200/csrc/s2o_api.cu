@@ -1,5 +1,6 @@
 // Host side of the libs2o C ABI: argument checks, workspace layout and launches. Every check
 // runs before anything is enqueued, so a returned error means no device work was started.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -88,6 +89,9 @@ WsLayout ws_layout(const Dims &d) {
   L.rho = take(bhq * d.N * 4);
   L.keys0 = take(bhq * d.N * 8);
   L.keys1 = take(bhq * d.N * 8);
+  // Radix digit counts: 256 per tile of 4096 elements of each sorted run (runs of N or of S).
+  const size_t tiles_n = (size_t)(d.N + 4095) / 4096, tiles_s = (size_t)(d.S + 4095) / 4096;
+  L.radix = take(bhq * 256 * std::max(tiles_n, tiles_s * (size_t)d.nSeg) * 4);
   L.Qbar = take(bhq * d.nB * d.D * 4);
   L.Kbar = take(bhq * d.nB * d.D * 4);
   L.r = take(bhq * d.nB * d.nB * 4);

@@ -73,18 +73,6 @@ __device__ __forceinline__ float dot_regs(const uint4 (&v)[D / 8], const float4 
   return acc;
 }
 
-// Two independent IEEE fp32 fused multiply-adds in one instruction: acc.{x,y} = fma(a.{x,y},
-// b.{x,y}, acc.{x,y}), each rounded on its own (same results as two fmaf calls).
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 acc) {
-  unsigned long long r;
-  const unsigned long long A = ((unsigned long long)__float_as_uint(a.y) << 32) | __float_as_uint(a.x);
-  const unsigned long long B = ((unsigned long long)__float_as_uint(b.y) << 32) | __float_as_uint(b.x);
-  const unsigned long long C =
-      ((unsigned long long)__float_as_uint(acc.y) << 32) | __float_as_uint(acc.x);
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(A), "l"(B), "l"(C));
-  return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
-}
-
 // 16-byte asynchronous copy global -> shared (cached in L2 only), and the wait for all of this
 // thread's copies. A CTA stages contiguous rows this way with no registers held per load, so many
 // loads are in flight.
@@ -104,12 +92,6 @@ __device__ __forceinline__ uint32_t sort_key(float x) {
   if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;
   if ((b & 0x7fffffffu) == 0u) b = 0u;
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-// Ascending order of this word = descending score, ties to the lower index (a stable
-// descending sort). Indices are below 2^31, so no word equals the all-ones padding value.
-__device__ __forceinline__ unsigned long long order_word(float score, uint32_t idx) {
-  return ((unsigned long long)(~sort_key(score)) << 32) | idx;
 }
 
 // exp64: Cody–Waite reduction by ln 2 with a two-part constant, then the degree-13 Taylor
@@ -313,166 +295,269 @@ __global__ void __launch_bounds__(128)
 
 // ------------------------------------------------------------------ ordering (step 2)
 
-__global__ void k_make_keys(const float *__restrict__ score, unsigned long long *__restrict__ keys,
-                            int N, long long total) {
-  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x < total) keys[x] = order_word(score[x], (uint32_t)(x % N));
-}
+// ------------------------------------------------------------------ stable radix sorting
+//
+// Orderings are stable least-significant-digit radix sorts of 32-bit keys, 8 bits per pass, with
+// the original index as the value: key = ~(sort key), so ascending keys are descending scores and
+// equal keys keep index order (the lower index first), exactly the ordering the definition fixes.
 
-// One compare-exchange stage of a bitonic network on the 128 words a warp holds in registers
-// (word i of lane l is element base + 4l + i): partners closer than four elements sit in the
-// same lane, the others are exchanged through shuffles.
-__device__ __forceinline__ void warp_stage64(unsigned long long (&k)[4], int base, int lane,
-                                             int size, int stride) {
-  if (stride >= 4) {
+__device__ __forceinline__ uint32_t desc_key(float score) { return ~sort_key(score); }
+
+// Lanes of the warp holding the same 8-bit digit (eight ballots).
+__device__ __forceinline__ unsigned match_digit(uint32_t d) {
+  unsigned peers = 0xffffffffu;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = base + 4 * lane + i;
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, k[i], stride >> 2);
-      // The lower element of a pair keeps the minimum in ascending runs, the maximum in
-      // descending ones; the upper element the other.
-      const bool keep_min = ((e & size) == 0) == ((e & stride) == 0);
-      const bool less = k[i] < other;
-      k[i] = (keep_min == less) ? k[i] : other;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = i ^ stride;
-      if (j > i) {
-        const bool up = ((base + 4 * lane + i) & size) == 0;
-        const unsigned long long lo = k[i] < k[j] ? k[i] : k[j];
-        const unsigned long long hi = k[i] < k[j] ? k[j] : k[i];
-        k[i] = up ? lo : hi;
-        k[j] = up ? hi : lo;
-      }
-    }
+  for (int b = 0; b < 8; ++b) {
+    const unsigned bb = __ballot_sync(0xffffffffu, (d >> b) & 1u);
+    peers &= ((d >> b) & 1u) ? bb : ~bb;
   }
+  return peers;
 }
 
-// Ascending bitonic sort of the 128·(blockDim.x/32) distinct words in shared memory: runs of up
-// to 128 words and every stage of stride below 128 run in registers (each warp owns 128
-// consecutive words), only the stages of larger stride go through shared memory.
-__device__ __forceinline__ void block_sort64(unsigned long long *s) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, n = blockDim.x * 4;
-  const int base = warp * 128;
-  unsigned long long k[4];
+// One counting pass inside a CTA: the destination, in stable order by digit, of R elements per
+// lane (element r of lane l of warp w is w·32R + r·32 + l). Scratch: hist[warps·256],
+// dbase[256]. Also returns, in dbase, each digit's first destination.
+template <int R>
+__device__ __forceinline__ void radix_ranks(const uint32_t (&digit)[R], int (&dest)[R],
+                                            int *hist, int *dbase) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
+  const unsigned full = 0xffffffffu, below = (1u << lane) - 1u;
+  int *wh = hist + warp * 256;
+  for (int d = lane; d < 256; d += 32) wh[d] = 0;
+  __syncwarp();
+  int rank[R];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) k[i] = s[base + 4 * lane + i];
-#pragma unroll
-  for (int size = 2; size <= 128; size <<= 1)
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) warp_stage64(k, base, lane, size, stride);
-  for (int size = 256; size <= n; size <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s[base + 4 * lane + i] = k[i];
-    __syncthreads();
-    for (int stride = size >> 1; stride >= 128; stride >>= 1) {
-      for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
-        const int lo = ((i / stride) * 2 * stride) + (i % stride), hi = lo + stride;
-        const unsigned long long a = s[lo], b = s[hi];
-        const bool up = (lo & size) == 0;
-        if ((a > b) == up) {
-          s[lo] = b;
-          s[hi] = a;
-        }
-      }
-      __syncthreads();
+  for (int r = 0; r < R; ++r) {
+    const unsigned peers = match_digit(digit[r]);
+    rank[r] = wh[digit[r]] + __popc(peers & below);
+    __syncwarp();
+    if (lane == __ffs(peers) - 1) wh[digit[r]] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // Per digit: exclusive prefix over the warps (in place) and the digit's total.
+  for (int d = threadIdx.x; d < 256; d += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int c = hist[w * 256 + d];
+      hist[w * 256 + d] = run;
+      run += c;
     }
+    dbase[d] = run;
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the 256 digit totals, 8 per lane
+    int v[8], sum = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) k[i] = s[base + 4 * lane + i];
+    for (int i = 0; i < 8; ++i) {
+      v[i] = dbase[lane * 8 + i];
+      sum += v[i];
+    }
+    int incl = sum;
 #pragma unroll
-    for (int stride = 64; stride > 0; stride >>= 1) warp_stage64(k, base, lane, size, stride);
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      dbase[lane * 8 + i] = run;
+      run += v[i];
+    }
   }
   __syncthreads();
 #pragma unroll
-  for (int i = 0; i < 4; ++i) s[base + 4 * lane + i] = k[i];
-  __syncthreads();
+  for (int r = 0; r < R; ++r) dest[r] = dbase[digit[r]] + wh[digit[r]] + rank[r];
 }
 
-// Sorts each tile of TILE consecutive words of a run in shared memory; the last tile of a run is
-// padded with all-ones words, which sort last.
-template <int TILE>
-__global__ void __launch_bounds__(TILE / 4)
-    k_tile_sort(unsigned long long *__restrict__ keys, long long run_len, int tiles_per_run) {
-  __shared__ unsigned long long s[TILE];
-  const long long run = blockIdx.x / tiles_per_run;
-  const long long tile0 = (long long)(blockIdx.x % tiles_per_run) * TILE;
-  const long long begin = run * run_len + tile0;
-  const int n = (int)min((long long)TILE, run_len - tile0);
-  for (int i = threadIdx.x; i < TILE; i += blockDim.x) s[i] = i < n ? keys[begin + i] : ~0ull;
-  __syncthreads();
-  block_sort64(s);
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[begin + i] = s[i];
-}
-
-// One merge pass: sorted neighbours of `width` words inside each run become sorted pairs. Each
-// thread writes kItems consecutive outputs: it finds where its first output splits the two inputs
-// by a binary search along the merge diagonal, then merges sequentially. Words are unique.
-constexpr int kMergeItems = 8;
-
-__global__ void k_merge_pass(const unsigned long long *__restrict__ src,
-                             unsigned long long *__restrict__ dst, long long run_len,
-                             long long width, long long total) {
-  const long long g = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * kMergeItems;
-  if (g >= total) return;
-  const long long run = g / run_len, off = g % run_len;
-  const long long pair0 = off - off % (2 * width);
-  const long long left_n = min(width, run_len - pair0);
-  const long long right_n = max(0LL, min(width, run_len - pair0 - width));
-  const unsigned long long *A = src + run * run_len + pair0;
-  const unsigned long long *Bv = A + left_n;
-  const long long o = off - pair0;
-  long long lo = max(0LL, o - right_n), hi = min(o, left_n);
-  while (lo < hi) {
-    const long long mid = (lo + hi) >> 1;
-    if (A[mid] < Bv[o - 1 - mid])
-      lo = mid + 1;
-    else
-      hi = mid;
-  }
-  long long i = lo, j = o - lo;
-  unsigned long long *out = dst + run * run_len + pair0 + o;
-  const int n = (int)min((long long)kMergeItems, left_n + right_n - o);
-  for (int x = 0; x < n; ++x) {
-    if (i < left_n && (j >= right_n || A[i] < Bv[j]))
-      out[x] = A[i++];
-    else
-      out[x] = Bv[j++];
-  }
-}
-
-__global__ void k_extract_perm(const unsigned long long *__restrict__ keys,
-                               int32_t *__restrict__ perm, long long total) {
-  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x < total) perm[x] = (int32_t)(keys[x] & 0xffffffffull);
-}
-
-__global__ void k_identity_perm(int32_t *__restrict__ perm, int N, long long total) {
-  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x < total) perm[x] = (int32_t)(x % N);
-}
-
-// Segment-local query ordering, one CTA per (query head, segment) of at most TILE queries: the
-// order words of the segment's rho values sorted in shared memory (the identity when the query
-// ordering is off), written out as perm_q.
-template <int TILE>
-__global__ void __launch_bounds__(TILE / 4)
+// Segment-local query ordering, one CTA per (query head, segment) of at most 32·R·(blockDim/32)
+// queries: four counting passes over the keys of the segment's rho values in shared memory, then
+// perm_q (the identity when the query ordering is off).
+template <int R>
+__global__ void __launch_bounds__(512)
     k_segment_sort(const float *__restrict__ rho, int32_t *__restrict__ perm_q, int N, int S,
                    int query_perm) {
-  __shared__ unsigned long long keys[TILE];
+  extern __shared__ int sm_i[];
+  const int n = blockDim.x * R;
+  uint32_t *skey = reinterpret_cast<uint32_t *>(sm_i);  // [n]
+  uint32_t *sval = skey + n;                            // [n]
+  int *hist = reinterpret_cast<int *>(sval + n);        // [warps·256]
+  int *dbase = hist + (blockDim.x / 32) * 256;          // [256]
   const long long qh = blockIdx.y;
   const int s0 = blockIdx.x * S;
-  for (int r = threadIdx.x; r < TILE; r += blockDim.x) {
-    const int i = s0 + r;
-    keys[r] = r >= S ? ~0ull
-                     : query_perm ? order_word(__ldg(rho + qh * N + i), (uint32_t)i)
-                                  : (unsigned long long)i;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (!query_perm) {
+    for (int r = threadIdx.x; r < S; r += blockDim.x) perm_q[qh * N + s0 + r] = s0 + r;
+    return;
+  }
+  uint32_t key[R], val[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = warp * 32 * R + r * 32 + lane;
+    key[r] = e < S ? desc_key(__ldg(rho + qh * N + s0 + e)) : 0xffffffffu;
+    val[r] = (uint32_t)e;
+  }
+  for (int pass = 0; pass < 4; ++pass) {
+    uint32_t dig[R];
+    int dest[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) dig[r] = (key[r] >> (8 * pass)) & 255u;
+    radix_ranks<R>(dig, dest, hist, dbase);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      skey[dest[r]] = key[r];
+      sval[dest[r]] = val[r];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = warp * 32 * R + r * 32 + lane;
+      key[r] = skey[e];
+      val[r] = sval[e];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = warp * 32 * R + r * 32 + lane;
+    if (e < S) perm_q[qh * N + s0 + e] = s0 + (int32_t)val[r];
+  }
+  (void)n;
+}
+
+// Multi-CTA stable radix sort of runs of run_len elements (one run per query head), tiles of
+// kRadixTile elements: per pass a digit count per tile, then a scatter per tile that derives its
+// offsets from the run's counts.
+constexpr int kRadixR = 8, kRadixThreads = 512, kRadixTile = kRadixR * kRadixThreads;
+
+// Element e of a tile, for thread (warp, lane) and round r.
+__device__ __forceinline__ int radix_elem(int r) {
+  return (threadIdx.x / 32) * 32 * kRadixR + r * 32 + threadIdx.x % 32;
+}
+
+// Keys and values of pass 0 come from the scores: key = desc_key(score), value = the index in
+// the run (idx0 = index of the tile's first element).
+__device__ __forceinline__ void radix_load(const float *score, const uint32_t *keys,
+                                           const uint32_t *vals, long long base, int idx0, int n,
+                                           uint32_t (&key)[kRadixR], uint32_t (&val)[kRadixR]) {
+#pragma unroll
+  for (int r = 0; r < kRadixR; ++r) {
+    const int e = radix_elem(r);
+    if (e < n) {
+      key[r] = score ? desc_key(__ldg(score + base + e)) : __ldg(keys + base + e);
+      val[r] = score ? (uint32_t)(idx0 + e) : __ldg(vals + base + e);
+    } else {
+      key[r] = 0xffffffffu;
+      val[r] = 0u;
+    }
+  }
+}
+
+// counts[(run·256 + digit)·tiles + tile] for one pass.
+__global__ void __launch_bounds__(kRadixThreads)
+    k_radix_count(const float *__restrict__ score, const uint32_t *__restrict__ keys,
+                  long long run_len, int tiles, int shift, int *__restrict__ counts) {
+  __shared__ int h[256];
+  const long long run = blockIdx.x / tiles;
+  const int tile = blockIdx.x % tiles;
+  const long long base = run * run_len + (long long)tile * kRadixTile;
+  const int n = (int)min((long long)kRadixTile, run_len - (long long)tile * kRadixTile);
+  for (int d = threadIdx.x; d < 256; d += blockDim.x) h[d] = 0;
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const uint32_t k = score ? desc_key(__ldg(score + base + e)) : __ldg(keys + base + e);
+    atomicAdd(&h[(k >> shift) & 255u], 1);
   }
   __syncthreads();
-  if (query_perm) block_sort64(keys);
-  for (int r = threadIdx.x; r < S; r += blockDim.x)
-    perm_q[qh * N + s0 + r] = (int32_t)(keys[r] & 0xffffffffull);
+  for (int d = threadIdx.x; d < 256; d += blockDim.x)
+    counts[(run * 256 + d) * tiles + tile] = h[d];
+}
+
+// Scatter of one pass: each tile ranks its elements by digit (stable), groups them in shared
+// memory and writes each digit's run to its offset. The last pass writes only the values, as the
+// permutation.
+__global__ void __launch_bounds__(kRadixThreads)
+    k_radix_scatter(const float *__restrict__ score, const uint32_t *__restrict__ keys_in,
+                    const uint32_t *__restrict__ vals_in, uint32_t *__restrict__ keys_out,
+                    uint32_t *__restrict__ vals_out, int32_t *__restrict__ perm_out,
+                    long long run_len, int tiles, int shift, const int *__restrict__ offsets) {  // raw digit counts of the pass
+  extern __shared__ int sm_r[];
+  uint32_t *skey = reinterpret_cast<uint32_t *>(sm_r);   // [tile]
+  uint32_t *sval = skey + kRadixTile;                     // [tile]
+  int *hist = reinterpret_cast<int *>(sval + kRadixTile);  // [warps·256]
+  int *dbase = hist + (kRadixThreads / 32) * 256;          // [256]
+  int *goff = dbase + 256;                                 // [256]
+  const long long run = blockIdx.x / tiles;
+  const int tile = blockIdx.x % tiles;
+  const long long base = run * run_len + (long long)tile * kRadixTile;
+  const int n = (int)min((long long)kRadixTile, run_len - (long long)tile * kRadixTile);
+  // This tile's output offset per digit, from the run's raw counts: the digits before it over
+  // the whole run, plus the same digit in the tiles before this one.
+  if (threadIdx.x < 256) {
+    const int d = threadIdx.x;
+    const int *c = offsets + (run * 256 + d) * tiles;
+    int before = 0, total = 0;
+    for (int t0 = 0; t0 < tiles; t0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = t0 + k < tiles ? __ldg(c + t0 + k) : 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        before += t0 + k < tile ? v[k] : 0;
+        total += v[k];
+      }
+    }
+    goff[d] = before;
+    dbase[d] = total;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // exclusive scan of the digit totals, 8 per lane
+    const int lane = threadIdx.x;
+    int v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = dbase[lane * 8 + i];
+      sum += v[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int run_sum = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      goff[lane * 8 + i] += run_sum;
+      run_sum += v[i];
+    }
+  }
+  __syncthreads();
+  uint32_t key[kRadixR], val[kRadixR], dig[kRadixR];
+  int dest[kRadixR];
+  radix_load(score, keys_in, vals_in, base, tile * kRadixTile, n, key, val);
+#pragma unroll
+  for (int r = 0; r < kRadixR; ++r) dig[r] = (key[r] >> shift) & 255u;
+  radix_ranks<kRadixR>(dig, dest, hist, dbase);
+#pragma unroll
+  for (int r = 0; r < kRadixR; ++r) {
+    skey[dest[r]] = key[r];
+    sval[dest[r]] = val[r];
+  }
+  __syncthreads();
+  const long long out0 = run * run_len;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t k = skey[i];
+    const int d = (int)((k >> shift) & 255u);
+    const long long o = out0 + goff[d] + (i - dbase[d]);
+    if (perm_out)
+      perm_out[o] = (int32_t)sval[i];
+    else {
+      keys_out[o] = k;
+      vals_out[o] = sval[i];
+    }
+  }
 }
 
 // ------------------------------------------------------------------ blocks and scores
@@ -919,30 +1004,33 @@ __global__ void k_exp64_probe(const double *x, double *y, int n) {
 
 inline unsigned blocks_for(long long n, int per) { return (unsigned)((n + per - 1) / per); }
 
-cudaError_t sort_runs(unsigned long long *a, unsigned long long *b, long long total,
-                      long long run_len, int32_t *perm_out, cudaStream_t st) {
-  // Tile size: the smallest of 1024 / 2048 / 4096 that covers a run, capped at 4096.
-  const int tile = run_len <= 1024 ? 1024 : run_len <= 2048 ? 2048 : 4096;
-  const int tiles_per_run = (int)((run_len + tile - 1) / tile);
-  const unsigned grid = (unsigned)((total / run_len) * tiles_per_run);
-  if (tile == 1024)
-    k_tile_sort<1024><<<grid, 256, 0, st>>>(a, run_len, tiles_per_run);
-  else if (tile == 2048)
-    k_tile_sort<2048><<<grid, 512, 0, st>>>(a, run_len, tiles_per_run);
-  else
-    k_tile_sort<4096><<<grid, 1024, 0, st>>>(a, run_len, tiles_per_run);
-  note_launch();
-  unsigned long long *src = a, *dst = b;
-  for (long long width = tile; width < run_len; width *= 2) {
-    k_merge_pass<<<blocks_for((total + kMergeItems - 1) / kMergeItems, 256), 256, 0, st>>>(
-        src, dst, run_len, width, total);
+// Stable radix sort of runs of run_len scores each (descending, ties to the lower index), the
+// permutation written to perm_out. Keys and values ping-pong between (k0, v0) and (k1, v1).
+cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint32_t *k1,
+                            uint32_t *v1, int *counts, long long total, long long run_len,
+                            int32_t *perm_out, cudaStream_t st) {
+  const int tiles = (int)((run_len + kRadixTile - 1) / kRadixTile);
+  const long long runs = total / run_len;
+  const unsigned grid = (unsigned)(runs * tiles);
+  const size_t smem = (size_t)2 * kRadixTile * 4 + (size_t)(kRadixThreads / 32) * 256 * 4 + 512 * 4;
+  cudaError_t e = cudaFuncSetAttribute(k_radix_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const uint32_t *kin = nullptr, *vin = nullptr;
+  uint32_t *kout = k0, *vout = v0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const float *sc = pass == 0 ? score : nullptr;
+    k_radix_count<<<grid, kRadixThreads, 0, st>>>(sc, kin, run_len, tiles, 8 * pass, counts);
     note_launch();
-    unsigned long long *t = src;
-    src = dst;
-    dst = t;
+    k_radix_scatter<<<grid, kRadixThreads, smem, st>>>(sc, kin, vin, kout, vout,
+                                                       pass == 3 ? perm_out : nullptr, run_len,
+                                                       tiles, 8 * pass, counts);
+    note_launch();
+    kin = kout;
+    vin = vout;
+    kout = kout == k0 ? k1 : k0;
+    vout = vout == v0 ? v1 : v0;
   }
-  k_extract_perm<<<blocks_for(total, 256), 256, 0, st>>>(src, perm_out, total);
-  note_launch();
   return cudaGetLastError();
 }
 
@@ -958,8 +1046,10 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   float *u = reinterpret_cast<float *>(ws + L.u);
   float *kappa = reinterpret_cast<float *>(ws + L.kappa);
   float *rho = reinterpret_cast<float *>(ws + L.rho);
-  unsigned long long *keys0 = reinterpret_cast<unsigned long long *>(ws + L.keys0);
-  unsigned long long *keys1 = reinterpret_cast<unsigned long long *>(ws + L.keys1);
+  // Radix sort buffers: keys and values of two ping-pong copies, digit counts.
+  uint32_t *rk0 = reinterpret_cast<uint32_t *>(ws + L.keys0), *rv0 = rk0 + d.bhq() * d.N;
+  uint32_t *rk1 = reinterpret_cast<uint32_t *>(ws + L.keys1), *rv1 = rk1 + d.bhq() * d.N;
+  int *rcount = reinterpret_cast<int *>(ws + L.radix);
   float *Qbar = reinterpret_cast<float *>(ws + L.Qbar);
   float *Kbar = reinterpret_cast<float *>(ws + L.Kbar);
   float *r = reinterpret_cast<float *>(ws + L.r);
@@ -990,9 +1080,9 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
                                                                          (float)d.N);
   note_launch();
   // Step 2a: global key/value ordering.
-  k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(kappa, keys0, d.N, nq);
-  note_launch();
-  if ((e = sort_runs(keys0, keys1, nq, d.N, out.perm_k, st)) != cudaSuccess) return e;
+  if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, nq, d.N, out.perm_k, st)) !=
+      cudaSuccess)
+    return e;
   // Step 1b: query scores against the top stripe block.
   k_kbar_top<<<(unsigned)bhq, D, 0, st>>>(k, out.perm_k, kbar_all, kbar_top, u, d.N, D, d.B, d.Hq,
                                           d.Hkv, d.G);
@@ -1003,24 +1093,26 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
   note_launch();
   const dim3 seg_grid((unsigned)d.nSeg, (unsigned)bhq);
-  if (d.S <= 4096) {
-    if (d.S <= 512)
-      k_segment_sort<512><<<seg_grid, 128, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
-    else if (d.S <= 1024)
-      k_segment_sort<1024><<<seg_grid, 256, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
-    else if (d.S <= 2048)
-      k_segment_sort<2048><<<seg_grid, 512, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
-    else
-      k_segment_sort<4096><<<seg_grid, 1024, 0, st>>>(rho, out.perm_q, d.N, d.S, qp);
+  if (d.S <= 4096 || !qp) {
+    auto seg = [&](auto kernel, int R) -> cudaError_t {
+      const size_t smem = (size_t)2 * 512 * R * 4 + 16 * 256 * 4 + 256 * 4;
+      cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+      if (err != cudaSuccess) return err;
+      kernel<<<seg_grid, 512, smem, st>>>(rho, out.perm_q, d.N, d.S, qp);
+      return cudaSuccess;
+    };
+    if ((e = d.S <= 512    ? seg(k_segment_sort<1>, 1)
+             : d.S <= 1024 ? seg(k_segment_sort<2>, 2)
+             : d.S <= 2048 ? seg(k_segment_sort<4>, 4)
+                           : seg(k_segment_sort<8>, 8)) != cudaSuccess)
+      return e;
     note_launch();
-  } else if (qp) {
-    // Segments longer than the shared-memory sort: merge sort of the order words per segment.
-    k_make_keys<<<blocks_for(nq, 256), 256, 0, st>>>(rho, keys0, d.N, nq);
-    note_launch();
-    if ((e = sort_runs(keys0, keys1, nq, d.S, out.perm_q, st)) != cudaSuccess) return e;
   } else {
-    k_identity_perm<<<blocks_for(nq, 256), 256, 0, st>>>(out.perm_q, d.N, nq);
-    note_launch();
+    // Segments longer than one CTA's sort: the multi-CTA radix sort over runs of S.
+    if ((e = radix_sort_runs(rho, rk0, rv0, rk1, rv1, rcount, nq, d.S, out.perm_q, st)) !=
+        cudaSuccess)
+      return e;
   }
   k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
                                                         nblk, d.Hq, d.Hkv, d.G, 0);

@@ -20,7 +20,7 @@ Dims dims_of(const s2o_config &c);
 
 // Byte offsets of the scratch arrays inside a workspace (256-byte aligned).
 struct WsLayout {
-  size_t qchunk, kchunk, qbar, kbar_all, kbar_top, u, kappa, rho, keys0, keys1, Qbar, Kbar, r,
+  size_t qchunk, kchunk, qbar, kbar_all, kbar_top, u, kappa, rho, keys0, keys1, radix, Qbar, Kbar, r,
       ncount, flags, total;
 };
 
