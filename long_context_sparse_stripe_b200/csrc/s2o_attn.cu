@@ -522,9 +522,19 @@ __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lan
     const long long pos = blockIdx.x + (k + lane) * gridDim.x;
     if (p.skip_empty) {
       bool keep = false;
-      if (pos < p.n_units) {
-        const Unit un = decode_unit<BN>(p, pos);
-        keep = un.cnt > 0;
+      if (pos < p.n_units && p.sel_cnt) {
+        // The unit's (query head, block) in permuted-mode order, then its list length.
+        long long u = pos;
+        const int hi = (int)(u % p.G);
+        u /= p.G;
+        const int per_seg = p.S / BN;
+        const int bl = (int)(u % per_seg);
+        u /= per_seg;
+        const int sg = (int)(u % p.nSeg);
+        u /= p.nSeg;
+        const int g = (int)(u % p.Hkv);
+        const long long qh = (u / p.Hkv) * p.Hq + (long long)g * p.G + hi;
+        keep = __ldg(p.sel_cnt + qh * p.nB + sg * per_seg + bl) > 0;
       }
       const unsigned m = __ballot_sync(0xffffffffu, keep);
       if (keep) list[n + __popc(m & ((1u << lane) - 1u))] = (uint32_t)pos;
