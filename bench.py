@@ -369,6 +369,96 @@ def run_s2o(args):
     return 0
 
 
+def run_sweep(args):
+    """Per-configuration report (not the headline line): the llama-32k layer, the llama-128k layer
+    at three thresholds, the qwen-128k ablations (threshold, segment length, query permutation off)
+    and the 32-layer stack. One JSON line per configuration on stdout."""
+    import long_context_sparse_stripe_b200 as s2o
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak = measured_peaks()[0]
+    cache = {}
+
+    def events():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def measure(w, reps=5, dense=True):
+        key = (w.name, w.seed, w.seq_len, w.stripe_frac)
+        if key not in cache:
+            cache.clear()
+            cache[key] = tuple(t.to(dev) for t in gen.make_inputs(w))
+        qd, kd, vd = cache[key]
+        cfg = s2o.Config.of(w)
+        idx, ws, o = s2o.alloc_indices(cfg, dev), s2o.alloc_workspace(cfg, dev), torch.empty_like(qd)
+        for _ in range(2):
+            s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
+            s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx, out=o)
+        a0, a1 = events()
+        b0, b1 = events()
+        a0.record()
+        for _ in range(reps):
+            s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
+        a1.record()
+        b0.record()
+        for _ in range(reps):
+            s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx, out=o)
+        b1.record()
+        torch.cuda.synchronize()
+        index_ms, attn_ms = a0.elapsed_time(a1) / reps, b0.elapsed_time(b1) / reps
+        stats = s2o.index_stats(cfg, idx, ws)
+        per_seg = w.segment_len // w.block_size
+        local_pass = w.batch * w.n_q_heads * (w.seq_len // w.segment_len) * per_seg * (per_seg + 1) // 2
+        busy = idx.sel_cnt > 0
+        permuted_pass = int((idx.local_tiles[busy].long() + idx.sel_cnt[busy].long()).sum().item())
+        tile_flops = 4.0 * w.block_size ** 2 * w.head_dim
+        row = {"workload": w.name, "tau": w.tau, "segment_len": w.segment_len,
+               "query_perm": w.query_perm, "stripe_frac": w.stripe_frac,
+               "pair_sparsity": stats.pair_sparsity,
+               "tile_density": stats.executed_tiles * w.block_size ** 2 / stats.causal_pairs,
+               "selected_tiles": stats.selected_tiles,
+               "kernel_tiles": {"local_pass": local_pass, "permuted_pass": permuted_pass},
+               "index_ms": index_ms, "attention_ms": attn_ms,
+               "index_fraction_of_attention": index_ms / attn_ms,
+               "exec_tflops": (local_pass + permuted_pass) * tile_flops / (attn_ms * 1e-3) / 1e12,
+               "effective_tflops": w.dense_causal_flops / ((index_ms + attn_ms) * 1e-3) / 1e12}
+        row["exec_frac_of_peak"] = row["exec_tflops"] / peak
+        if dense:
+            od = torch.empty_like(qd)
+            s2o.dense_causal_prefill(cfg, qd, kd, vd, out=od)
+            d0, d1 = events()
+            d0.record()
+            s2o.dense_causal_prefill(cfg, qd, kd, vd, out=od)
+            d1.record()
+            torch.cuda.synchronize()
+            row["dense_ms"] = d0.elapsed_time(d1)
+            row["mse_vs_dense"] = float(((o.float() - od.float()) ** 2).mean().item())
+            del od
+        if s2o.check_device_status(dev) != 0:
+            raise RuntimeError("device timeout")
+        return row
+
+    configs = [gen.workload("llama-32k")]
+    configs += [gen.workload("llama-128k", tau=t) for t in (0.005, 0.01, 0.02)]
+    qwen = gen.workload("qwen-128k")
+    configs += [qwen.replace(tau=t) for t in (0.001, 0.005, 0.01, 0.02)]
+    configs += [qwen.replace(segment_len=s) for s in (1024, 4096)]
+    configs += [qwen.replace(query_perm=0)]
+    for w in configs:
+        print(json.dumps({"config": measure(w)}), flush=True)
+    stack = [measure(gen.layer_workload(l), reps=2, dense=(l % 8 == 7)) for l in range(32)]
+    tot_i = sum(r["index_ms"] for r in stack)
+    tot_a = sum(r["attention_ms"] for r in stack)
+    print(json.dumps({"stack32": {
+        "layers": 32, "index_ms_total": tot_i, "attention_ms_total": tot_a,
+        "index_fraction_of_attention": tot_i / tot_a,
+        "pair_sparsity_mean": float(np.mean([r["pair_sparsity"] for r in stack])),
+        "mse_vs_dense_layers_7_15_23_31": [r["mse_vs_dense"] for r in stack if "mse_vs_dense" in r],
+        "effective_tflops": sum(gen.layer_workload(l).dense_causal_flops for l in range(32))
+        / ((tot_i + tot_a) * 1e-3) / 1e12}}), flush=True)
+    return 0
+
+
 def run_profile_target(args):
     """A short fixed sequence for profiler captures (not a bench line): one index build, then
     `--steps` attention calls (each a local pass and a permuted pass) and one dense-baseline call."""
@@ -376,6 +466,9 @@ def run_profile_target(args):
 
     torch.cuda.set_device(0)
     w = gen.workload(args.workload, tau=args.tau)
+    if args.heads:
+        hq, hkv = (int(x) for x in args.heads.split(","))
+        w = w.replace(n_q_heads=hq, n_kv_heads=hkv)
     q, k, v = (t.cuda() for t in gen.make_inputs(w))
     cfg = s2o.Config.of(w)
     idx = s2o.build_indices(cfg, q, k)
@@ -402,6 +495,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-rows", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", default="",
+                    help="profile target only: 'Hq,Hkv' (the first KV groups of the workload)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="per-configuration report (one JSON line per configuration)")
     ap.add_argument("--profile-target", action="store_true",
                     help="run a short fixed call sequence for profiler captures; print nothing")
     args = ap.parse_args()
@@ -409,6 +506,8 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.profile_target:
         return run_profile_target(args)
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_s2o(args)

@@ -7,18 +7,28 @@
 // itself is Eq. (1) of "AB-Sparse" restricted to the selected key set, computed flash-style with
 // an online softmax (the normaliser of Milakov & Gimelshein, cited by the S2O paper).
 //
-// Work decomposition. A unit is one (batch, query head, query block): 128 query rows (the block's
-// B rows gathered by perm_q; rows B..127 are zero when B = 64) that run lt local tiles (contiguous
-// keys of the block's own segment, mask key <= query) and then the cnt selected key blocks (keys
-// gathered by perm_k, mask key < segment start). Units are ordered (batch, KV head, segment,
-// block, query head of the group), so consecutive units usually read the same local key tiles. A
-// work item is two consecutive units, Q0 and Q1, with one stream of key/value tiles: the local
-// tiles once for both when they share them, then the two selected lists interleaved. The grid is
-// persistent (one CTA per SM, work items strided by the grid size).
+// Work decomposition. A unit is one (batch, query head, query block) of 128 query rows (rows
+// B..127 are zero when B = 64). S2O runs in two launches of the same kernel:
+//   local pass     every original-order query block runs the causal triangle of its own segment
+//                  (the dense local window; masks on the diagonal tile only) and writes its rows;
+//   permuted pass  only the query blocks whose selected list is not empty, rows gathered by
+//                  perm_q: lt local tiles (contiguous keys of the block's segment, mask key <=
+//                  query on original positions), then the cnt selected key blocks (keys gathered
+//                  by perm_k, mask key < segment start); it overwrites their rows.
+// Each row ends with the attention over exactly its key set. The dense baseline is a third mode
+// (original-order blocks over all earlier keys). Units are ordered (batch, KV head, segment,
+// block, query head of the group) — the dense mode longest blocks first — so consecutive units
+// usually read the same local key tiles. A work item is two units, Q0 and Q1, with one stream of
+// key/value tiles: the local tiles once for both when they share them, then the two selected
+// lists interleaved. The grid is persistent (one CTA per SM); each CTA walks windows of a work
+// list that warp 0 fills between two CTA-wide barriers (the permuted pass lists only units with
+// selected blocks).
 //
-// Warp roles (352 threads):
-//   warp 0      K/V producer: K and V tiles of the stream into two rings (TMA tile loads for
-//               contiguous tiles, TMA tile::gather4 for gathered rows; 128-byte swizzle).
+// Warp roles (384 threads):
+//   warps 0, 11 K and V producers: K (warp 0) and V (warp 11) tiles of the stream into two rings
+//               (TMA tile loads for contiguous tiles, TMA tile::gather4 for gathered rows; 128-byte
+//               swizzle). Gathers are issued from two warps because one warp's stream of gather4
+//               instructions limits the permuted pass when lists are long.
 //   warp 1      MMA issuer: owns TMEM (512 columns: S0, S1, O0, O1). S_x = Q_x·Kᵀ, then
 //               O_x += P_x·V with P_x read from TMEM (bf16 pairs written over S_x). The two query
 //               tiles ping-pong: while one softmax group works on S0, the tensor core runs Q1's
@@ -46,7 +56,7 @@ __device__ unsigned int g_device_error;
 
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kM = 128;  // query rows per tile (UMMA M)
 constexpr int kList = 256;  // units per work-list window
 constexpr uint64_t kDrainNs = 2000000000ull;
@@ -410,29 +420,42 @@ __device__ __forceinline__ int users_at(const Pair &P, int j) {
   return 1 << x;
 }
 
+// The selected block of a unit's list position (clamped), or -1 past the list.
+__device__ __forceinline__ int sel_block(const Params &p, const Unit &u, int t) {
+  return t < u.cnt ? min(max(__ldg(u.sel + t), 0), p.nB - 1) : -1;
+}
+
+// This lane's four gathered key rows of permuted block c of unit u (flattened row indices,
+// clamped into the KV head); lanes >= B/4 and c < 0 give zeros.
+template <int BN>
+__device__ __forceinline__ int4 block_rows(const Params &p, const Unit &u, int c, int lane) {
+  if (c < 0 || lane >= BN / 4) return make_int4(0, 0, 0, 0);
+  const int4 r4 =
+      __ldg(reinterpret_cast<const int4 *>(p.perm_k + u.qh * p.N + (size_t)c * BN) + lane);
+  const int row0 = (int)(u.kh * p.N), hi = p.N - 1;
+  return make_int4(row0 + min(max(r4.x, 0), hi), row0 + min(max(r4.y, 0), hi),
+                   row0 + min(max(r4.z, 0), hi), row0 + min(max(r4.w, 0), hi));
+}
+
 // Loads the K or V rows of stream item `it` into one ring stage (all 32 lanes of the warp call it;
 // the transaction count has been set). Contiguous local tiles: one TMA tile load per 64-column
-// atom; gathered rows: tile::gather4, four rows per lane.
+// atom; gathered rows (prepared by block_rows): tile::gather4, four rows per lane.
 template <int D, int BN>
 __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap *tm_tile,
                                         const CUtensorMap *tm_row, const Params &p,
-                                        const Pair &P, const Item &it, uint32_t bar, int lane) {
+                                        const Pair &P, const Item &it, int4 rows, uint32_t bar,
+                                        int lane) {
   using L = Layout<D, BN>;
   const Unit &u = it.x ? P.u1 : P.u0;
-  const int row0 = (int)(u.kh * p.N);
   if (it.local) {
     if (lane == 0)
       for (int a = 0; a < D / 64; ++a)
-        tma_load_tile(dst + a * L::ATOM_KV, tm_tile, a * 64, row0 + u.seg0 + it.t * BN, bar);
+        tma_load_tile(dst + a * L::ATOM_KV, tm_tile, a * 64,
+                      (int)(u.kh * p.N) + u.seg0 + it.t * BN, bar);
   } else if (lane < BN / 4) {
-    const int c = min(max(__ldg(u.sel + it.t), 0), p.nB - 1);
-    const int4 r4 =
-        __ldg(reinterpret_cast<const int4 *>(p.perm_k + u.qh * p.N + (size_t)c * BN) + lane);
-    const int hi = p.N - 1;
-    const int y0 = row0 + min(max(r4.x, 0), hi), y1 = row0 + min(max(r4.y, 0), hi),
-              y2 = row0 + min(max(r4.z, 0), hi), y3 = row0 + min(max(r4.w, 0), hi);
     for (int a = 0; a < D / 64; ++a)
-      tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, tm_row, a * 64, y0, y1, y2, y3, bar);
+      tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, tm_row, a * 64, rows.x, rows.y, rows.z,
+                  rows.w, bar);
   }
 }
 
@@ -603,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (BN < kM && warp >= 3) {
+  if (BN < kM && warp >= 3 && warp < 11) {
     // Rows BN..127 of both Q tiles are padding: zero them once (TMA writes rows 0..BN-1 only).
     const int x = (warp - 3) >> 2, row = (warp & 3) * 32 + lane;
     if (row >= BN) {
@@ -641,44 +664,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- K / V producer
+  if (warp == 0 || warp == kThreads / 32 - 1) {
+    // ---------------------------------------------------------------- K and V producers
+    // Warp 0 loads K, the last warp V; both walk the same stream.
+    const bool is_k = warp == 0;
+    const int stages = is_k ? L::KST : L::VST;
+    const uint32_t ring = is_k ? sK : sV;
+    const int full0 = is_k ? kKFull : kVFull, empty0 = is_k ? kKEmpty : kVEmpty;
+    const CUtensorMap *tm_tile = is_k ? &tm_k_tile : &tm_v_tile;
+    const CUtensorMap *tm_row = is_k ? &tm_k_row : &tm_v_row;
     long long kj = 0;  // stream items issued so far (all work items of this CTA)
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
       const Pair P = decode_pair<BN>(p, list, n_list, wi);
+      // Gathered rows are looked up ahead: the rows of item j+1 and the block of item j+2 are
+      // requested before item j waits for its ring stage, so the dependent index loads are off
+      // the critical path.
+      auto block_of = [&](int j) -> int {
+        if (j >= P.total) return -1;
+        const Item t = item_at(P, j);
+        return t.local ? -1 : sel_block(p, t.x ? P.u1 : P.u0, t.t);
+      };
+      auto rows_of = [&](int j, int c) -> int4 {
+        if (j >= P.total || c < 0) return make_int4(0, 0, 0, 0);
+        const Item t = item_at(P, j);
+        return block_rows<BN>(p, t.x ? P.u1 : P.u0, c, lane);
+      };
+      int4 rows = rows_of(0, block_of(0));
+      int c_next = block_of(1);
       for (int j = 0; j < P.total; ++j) {
         const Item it = item_at(P, j);
-        const int ks = (int)(kj % L::KST), vs = (int)(kj % L::VST);
-        if (kj >= L::KST &&
-            !warp_wait(bar(kKEmpty + ks), (uint32_t)(((kj / L::KST) - 1) & 1), lim, lane)) {
+        const int4 rows_next = rows_of(j + 1, c_next);
+        c_next = block_of(j + 2);
+        const int st = (int)(kj % stages);
+        if (kj >= stages &&
+            !warp_wait(bar(empty0 + st), (uint32_t)(((kj / stages) - 1) & 1), lim, lane)) {
           ok = false;
           break;
         }
-        if (lane == 0) mbar_expect_tx(bar(kKFull + ks), L::KV_BYTES);
+        if (lane == 0) mbar_expect_tx(bar(full0 + st), L::KV_BYTES);
         __syncwarp();
-        load_kv<D, BN>(sK + ks * L::KV_BYTES, &tm_k_tile, &tm_k_row, p, P, it, bar(kKFull + ks),
+        load_kv<D, BN>(ring + st * L::KV_BYTES, tm_tile, tm_row, p, P, it, rows, bar(full0 + st),
                        lane);
-        if (kj >= L::VST &&
-            !warp_wait(bar(kVEmpty + vs), (uint32_t)(((kj / L::VST) - 1) & 1), lim, lane)) {
-          // K of this item is in flight: count it for the drain below.
-          drain_ring(bar(kKFull), L::KST, kj + 1);
-          ok = false;
-          break;
-        }
-        if (lane == 0) mbar_expect_tx(bar(kVFull + vs), L::KV_BYTES);
-        __syncwarp();
-        load_kv<D, BN>(sV + vs * L::KV_BYTES, &tm_v_tile, &tm_v_row, p, P, it, bar(kVFull + vs),
-                       lane);
+        rows = rows_next;
         ++kj;
       }
     }
     });
     // Drain: the last copy issued into each stage must have landed before the CTA exits.
-    if (lane == 0) {
-      drain_ring(bar(kKFull), L::KST, kj);
-      drain_ring(bar(kVFull), L::VST, kj);
-    }
+    if (lane == 0) drain_ring(bar(full0), stages, kj);
     __syncwarp();
   } else if (warp == 2) {
     // ---------------------------------------------------------------- Q producer
@@ -895,7 +929,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float m_run = -INFINITY, l_run = 0.f;
       const int n_items = u.lt + u.cnt;
+      // Keys of a selected block (for its mask) are requested before the wait for its S, the
+      // block id one tile earlier.
+      auto blk = [&](int n) { return n >= u.lt && n < n_items ? sel_block(p, u, n - u.lt) : -1; };
+      int c_cur = blk(0), c_next = blk(1);
       for (int n = 0; n < n_items; ++n) {
+        int keys[BN / 32];
+#pragma unroll
+        for (int q = 0; q < BN / 32; ++q)
+          keys[q] = c_cur < 0 ? 0 : __ldg(p.perm_k + u.qh * p.N + (size_t)c_cur * BN + q * 32 + lane);
+        c_cur = c_next;
+        c_next = blk(n + 2);
         // Warp-uniform outcome: the tcgen05.ld below is a warp-collective instruction.
         if (!__all_sync(full, mbar_wait(bar(kSFull + x), (uint32_t)(sn & 1), lim))) {
           ok = false;
@@ -920,14 +964,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c > limit) s[c] = __float_as_uint(-INFINITY);
           }
         } else {
-          const int c = min(max(__ldg(u.sel + (n - u.lt)), 0), p.nB - 1);
-          const int32_t *keys = p.perm_k + u.qh * p.N + (size_t)c * BN;
           uint32_t mw[BN / 32];
           bool all = true;
 #pragma unroll
           for (int q = 0; q < BN / 32; ++q) {
-            const int key = __ldg(keys + q * 32 + lane);
-            mw[q] = __ballot_sync(full, key >= 0 && key < seg0);
+            mw[q] = __ballot_sync(full, keys[q] >= 0 && keys[q] < seg0);
             all = all && mw[q] == full;
           }
           if (!all) {
