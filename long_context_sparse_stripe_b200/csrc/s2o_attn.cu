@@ -283,6 +283,7 @@ struct Params {
   int N, S, nB, nSeg, Hq, Hkv, G;
   int mode;
   int skip_empty;  // permuted mode: only blocks with a non-empty selected list
+  int o_v8;        // O is 32-byte aligned: rows are written with 32-byte stores
   long long n_units, n_items;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
@@ -518,6 +519,13 @@ __device__ __forceinline__ void mma8_ts(uint32_t d, uint32_t idesc, const uint32
       "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]),
       "l"(b[7]), "r"(acc0)
       : "memory");
+}
+
+// 32-byte global store of eight 32-bit words (one full sector).
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
@@ -1038,24 +1046,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       uint16_t *orow = p.o + ((size_t)u.qh * p.N + i_orig) * D;
+      // The whole row of O from TMEM (one wait), then 32-byte stores (full sectors).
+      uint32_t o[D];
 #pragma unroll
-      for (int c0 = 0; c0 < D / 32; ++c0) {
-        uint32_t o[32];
-        tmem_ld32(o_addr + c0 * 32, o);
-        tmem_wait_ld(o);
-        if (store_row) {
+      for (int c0 = 0; c0 < D / 32; ++c0)
+        tmem_ld32(o_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16(__uint_as_float(o[q * 8 + 0]) * inv_l,
-                            __uint_as_float(o[q * 8 + 1]) * inv_l);
-            v.y = pack_bf16(__uint_as_float(o[q * 8 + 2]) * inv_l,
-                            __uint_as_float(o[q * 8 + 3]) * inv_l);
-            v.z = pack_bf16(__uint_as_float(o[q * 8 + 4]) * inv_l,
-                            __uint_as_float(o[q * 8 + 5]) * inv_l);
-            v.w = pack_bf16(__uint_as_float(o[q * 8 + 6]) * inv_l,
-                            __uint_as_float(o[q * 8 + 7]) * inv_l);
-            *reinterpret_cast<uint4 *>(orow + c0 * 32 + q * 8) = v;
+      for (int c0 = 0; c0 < D / 32; ++c0) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
+      if (store_row) {
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t w[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            w[q] = pack_bf16(__uint_as_float(o[c * 16 + 2 * q]) * inv_l,
+                             __uint_as_float(o[c * 16 + 2 * q + 1]) * inv_l);
+          if (p.o_v8) {
+            st_global_v8(orow + c * 16, w);
+          } else {
+            reinterpret_cast<uint4 *>(orow + c * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<uint4 *>(orow + c * 16)[1] = make_uint4(w[4], w[5], w[6], w[7]);
           }
         }
       }
@@ -1138,6 +1148,7 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
   p.sel_blk = a.sel_blk;
   p.local_tiles = a.local_tiles;
   p.o = static_cast<uint16_t *>(a.o);
+  p.o_v8 = (reinterpret_cast<uintptr_t>(a.o) & 31u) == 0 ? 1 : 0;
   p.N = d.N;
   p.nB = d.nB;
   p.Hq = d.Hq;
