@@ -241,12 +241,14 @@ struct Layout {
   static constexpr uint32_t ATOM_KV = BN * 128;
   static constexpr uint32_t Q_BYTES = kM * D * 2;
   static constexpr uint32_t KV_BYTES = BN * D * 2;
-  static constexpr int KST = KV_BYTES >= 32768 ? 3 : 4;  // K ring depth
+  static constexpr int KST = KV_BYTES >= 32768 ? 2 : 4;  // K ring depth
   static constexpr int VST = KV_BYTES >= 32768 ? 2 : 4;  // V ring depth
   static constexpr uint32_t OFF_Q = 0;                   // Q0, then Q1
   static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
+  // Output staging: one 64-column atom of a 128-row tile per softmax group (TMA tile stores).
+  static constexpr uint32_t OFF_OST = OFF_V + VST * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_OST + 2 * ATOM_Q;
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr uint32_t OFF_LIST = OFF_BAR + BAR_BYTES;  // work list: kList units + count
   static constexpr uint32_t SMEM = OFF_LIST + kList * 4 + 16 + 1024;  // + alignment slack
@@ -521,6 +523,25 @@ __device__ __forceinline__ void mma8_ts(uint32_t d, uint32_t idesc, const uint32
       : "memory");
 }
 
+// TMA tile store shared -> global (bulk async-group of the issuing thread), its commit, and the
+// waits for the group's source reads / full completion.
+__device__ __forceinline__ void tma_store_tile(const CUtensorMap *tm, int x, int y, uint32_t src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // 32-byte global store of eight 32-bit words (one full sector).
 __device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&w)[8]) {
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]),
@@ -596,7 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_k_tile,
                          const __grid_constant__ CUtensorMap tm_k_row,
                          const __grid_constant__ CUtensorMap tm_v_tile,
-                         const __grid_constant__ CUtensorMap tm_v_row, const Params p) {
+                         const __grid_constant__ CUtensorMap tm_v_row,
+                         const __grid_constant__ CUtensorMap tm_o_tile, const Params p) {
   using L = Layout<D, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -1053,7 +1075,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(o_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
 #pragma unroll
       for (int c0 = 0; c0 < D / 32; ++c0) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
-      if (store_row) {
+      if (p.mode != kPermuted) {
+        // Contiguous rows: each 64-column atom is staged in shared memory (128-byte swizzle) and
+        // written with one TMA tile store; the group's first thread issues the stores and, before
+        // its stage is overwritten, waits until the previous store has read it.
+        const bool leader = quad == 0 && lane == 0;
+        const uint32_t ost = sbase + L::OFF_OST + (uint32_t)x * L::ATOM_Q;
+        unsigned char *ostp = smem + L::OFF_OST + x * L::ATOM_Q + row * 128;
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a) {
+          if (leader) bulk_wait_read();
+          named_bar_sync(2 + x, 128);
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int c = a * 64 + ch * 8;
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+            v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
+            v.z = pack_bf16(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
+            v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
+            *reinterpret_cast<uint4 *>(ostp + ((ch ^ (row & 7)) * 16)) = v;
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(2 + x, 128);
+          if (leader) {
+            tma_store_tile(&tm_o_tile, a * 64, (int)(u.qh * p.N) + u.b * BN, ost);
+            bulk_commit();
+          }
+        }
+      } else if (store_row) {
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t w[8];
@@ -1072,6 +1122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
     }
     });
+    // The output stores of this group's stage complete before the CTA exits.
+    if (quad == 0 && lane == 0) bulk_wait_all();
   }
 
   __syncthreads();
@@ -1132,11 +1184,12 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
   using L = Layout<D, BN>;
   static_assert(L::SMEM <= 232448, "shared memory budget");
   static_assert(kNumBars * 8 + 4 <= (int)L::BAR_BYTES, "barrier area");
-  CUtensorMap tq, tqr, tk, tkr, tv, tvr;
+  CUtensorMap tq, tqr, tk, tkr, tv, tvr, to;
   const long long q_rows = d.bhq() * d.N, kv_rows = d.bhkv() * d.N;
   if (!make_map(&tq, a.q, q_rows, D, BN) || !make_map(&tqr, a.q, q_rows, D, 1) ||
       !make_map(&tk, a.k, kv_rows, D, BN) || !make_map(&tkr, a.k, kv_rows, D, 1) ||
-      !make_map(&tv, a.v, kv_rows, D, BN) || !make_map(&tvr, a.v, kv_rows, D, 1))
+      !make_map(&tv, a.v, kv_rows, D, BN) || !make_map(&tvr, a.v, kv_rows, D, 1) ||
+      !make_map(&to, a.o, q_rows, D, BN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
@@ -1166,7 +1219,7 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
     const long long work = skip_empty ? p.n_units : p.n_items;
     const long long grid = work < sm_count() ? work : sm_count();
     s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv,
-                                                                           tvr, p);
+                                                                           tvr, to, p);
     note_launch();
     return cudaGetLastError();
   };
