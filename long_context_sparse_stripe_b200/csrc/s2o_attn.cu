@@ -266,7 +266,7 @@ enum Bar {
   kVFull = 12,   // 4
   kVEmpty = 16,  // 4
   kSFull = 20,   // 2: S_x = Q_x·Kᵀ finished (and every earlier product of the CTA)
-  kPFull = 22,   // 2: P_x written to TMEM and O_x rescaled (128 arrivals)
+  kPFull = 22,   // 2: P_x written to TMEM and O_x rescaled (one arrival per softmax warp)
   kOFull = 24,   // 2: the last O_x += P_x·V of a work item finished
   kDrain = 26,
   kNumBars = 27
@@ -279,6 +279,30 @@ enum Mode {
   kLocal = 2      // the dense local window only: original-order blocks, keys of their segment
 };
 
+// Division of n < 2^31 by a fixed divisor d ≥ 1 as a multiply-high and a shift (division by
+// invariant integers using multiplication, Granlund and Montgomery): with L = ⌈log2 d⌉, p = 31 + L
+// and m = ⌈2^p / d⌉ (m < 2^32), m = (2^p + e)/d with 0 ≤ e < d ≤ 2^L, so n·e < 2^p and
+// ⌊n·m / 2^p⌋ = ⌊n/d⌋. d = 1 is passed through.
+struct FastDiv {
+  uint32_t d, m, s;  // divisor, multiplier, p − 32 (d > 1)
+  void init(int divisor) {
+    d = (uint32_t)divisor;
+    int L = 0;
+    while ((1ull << L) < d) ++L;
+    m = d > 1 ? (uint32_t)(((1ull << (31 + L)) + d - 1) / d) : 0u;
+    s = d > 1 ? (uint32_t)(L - 1) : 0u;
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    return d > 1 ? __umulhi(n, m) >> s : n;
+  }
+  // Quotient, and n − q·d into r.
+  __device__ __forceinline__ uint32_t divmod(uint32_t n, uint32_t &r) const {
+    const uint32_t q = div(n);
+    r = n - q * d;
+    return q;
+  }
+};
+
 struct Params {
   const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
   uint16_t *o;
@@ -289,6 +313,7 @@ struct Params {
   long long n_units, n_items;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
+  FastDiv div_G, div_seg, div_nB, div_nSeg, div_Hkv;  // unit-id decoding (S/B blocks a segment)
 };
 
 struct Unit {
@@ -301,35 +326,38 @@ struct Unit {
 // together, query heads of the group fastest, so that the segment's K/V tiles stay in L2 and
 // paired units share local tiles; the dense baseline runs the longest query blocks first.
 template <int BN>
-__device__ __forceinline__ Unit decode_unit(const Params &p, long long u) {
+__device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
+  // Unit ids are below 2^31 (the host checks): divisions by multiply-high.
   Unit r;
-  const int hi = (int)(u % p.G);
-  u /= p.G;
-  const int per_seg = p.S / BN;
-  int b;
+  uint32_t rem;
+  u = p.div_G.divmod(u, rem);
+  const int hi = (int)rem;
+  int b, bl;  // block, and its index inside the segment
   if (p.mode == kDense) {
-    b = p.nB - 1 - (int)(u % p.nB);
-    u /= p.nB;
+    u = p.div_nB.divmod(u, rem);
+    b = p.nB - 1 - (int)rem;
+    bl = b;
+    r.seg0 = 0;
   } else {
-    const int bl = (int)(u % per_seg);
-    u /= per_seg;
-    const int s = (int)(u % p.nSeg);
-    u /= p.nSeg;
-    b = s * per_seg + bl;
+    u = p.div_seg.divmod(u, rem);
+    bl = (int)rem;
+    u = p.div_nSeg.divmod(u, rem);
+    b = (int)rem * (int)p.div_seg.d + bl;
+    r.seg0 = (int)rem * p.S;
   }
-  const int g = (int)(u % p.Hkv);
-  const long long beta = u / p.Hkv;
+  const uint32_t beta_u = p.div_Hkv.divmod(u, rem);
+  const int g = (int)rem;
+  const long long beta = beta_u;
   r.qh = beta * p.Hq + (long long)g * p.G + hi;
   r.kh = beta * p.Hkv + g;
   r.b = b;
-  r.seg0 = (int)((long long)b * BN / p.S) * p.S;
   if (p.mode != kPermuted) {
-    r.lt = b - r.seg0 / BN + 1;  // the causal triangle of the block's segment (or sequence)
+    r.lt = bl + 1;  // the causal triangle of the block's segment (or sequence)
     r.cnt = 0;
     r.sel = nullptr;
   } else {
     const long long qb = r.qh * p.nB + b;
-    r.lt = min(max(__ldg(p.local_tiles + qb), 1), per_seg);
+    r.lt = min(max(__ldg(p.local_tiles + qb), 1), (int)p.div_seg.d);
     r.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
     r.sel = p.sel_blk + qb * p.nB;
   }
@@ -635,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kQFull + x), 1);
       mbar_init(bar(kQEmpty + x), 1);
       mbar_init(bar(kSFull + x), 1);
-      mbar_init(bar(kPFull + x), 128);
+      mbar_init(bar(kPFull + x), 4);  // one arrival per softmax warp
       mbar_init(bar(kOFull + x), 1);
     }
     for (int i = 0; i < L::KST; ++i) {
@@ -815,24 +843,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t v_base = 0;          // stream items of this CTA's earlier work items
       uint32_t q_ph[2] = {0, 0}, p_ph[2] = {0, 0};
       for_each_window([&](int n_list) {
-      if (lane == 0)
-      for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-        const Pair P = decode_pair<BN>(p, list, n_list, wi);
-        if (!mbar_wait(bar(kQFull + 0), q_ph[0], lim) ||
-            (P.valid1 && !mbar_wait(bar(kQFull + 1), q_ph[1], lim))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int n_of[2] = {P.u0.lt + P.u0.cnt, P.u1.lt + P.u1.cnt};
-        int pend[2] = {-1, -1}, qk[2] = {0, 0};
+        // Each tile x has at most one product O_x += P_x·V still to issue (its P_x lives in
+        // S_x's columns): the one of stream item pend[x]. A unit's last product is issued at tile
+        // x's next step, which may belong to the next work item, so the tensor core goes on to
+        // the next unit's first Q_x·Kᵀ without draining; O_x is committed right after it. The
+        // window's last products are issued at its end.
+        constexpr uint32_t kNone = 0xffffffffu;
+        uint32_t pend[2] = {kNone, kNone};
+        bool pend_last[2] = {false, false};
         uint32_t acc[2] = {0u, 0u};
         uint32_t vleft = 0;  // 2 bits per V stage: products still to issue on its tile
-        // O_x += P_x·V for stream item jj (P_x bf16 pairs in TMEM, V in its ring stage). The V
-        // stage is released once every unit using the tile has issued its product.
-        auto issue_pv = [&](auto xc, int jj) -> bool {
+        // The V stage is released once every unit using the tile has issued its product.
+        auto issue_pv = [&](auto xc) -> bool {
           constexpr int x = decltype(xc)::value;
-          const uint32_t vi = v_base + (uint32_t)jj;
+          const uint32_t vi = pend[x];
           const uint32_t vs = vi & (L::VST - 1);
           if (!mbar_wait(bar(kVFull + vs), (vi / L::VST) & 1u, lim)) return false;
           if (!mbar_wait(bar(kPFull + x), p_ph[x], lim)) return false;
@@ -841,7 +865,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t vd = vdesc0 + vs * (L::KV_BYTES >> 4);
           uint64_t b[8];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) b[kk] = vd + (uint64_t)((kk % (BN / 16)) * (16 * 128 / 16));
+          for (int kk = 0; kk < 8; ++kk)
+            b[kk] = vd + (uint64_t)((kk % (BN / 16)) * (16 * 128 / 16));
           if (BN == 128) {
             mma8_ts(tmem + L::O_COL + (uint32_t)(D * x), kIdescPV, ptm[x], b, acc[x]);
           } else {
@@ -854,6 +879,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t left = ((vleft >> (2 * vs)) & 3u) - 1u;
           vleft = (vleft & ~(3u << (2 * vs))) | ((left & 3u) << (2 * vs));
           if (left == 0) tc_commit(bar(kVEmpty + vs));
+          if (pend_last[x]) {
+            tc_commit(bar(kOFull + x));
+            acc[x] = 0u;
+          }
+          pend[x] = kNone;
           return true;
         };
         auto issue_qk = [&](auto xc, const uint64_t (&kb)[8]) {
@@ -868,19 +898,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(kSFull + x));
         };
-        // One unit's step at stream item j: its pending product goes first (P_x lives in S_x's
-        // columns), or now if the unit skips the next item (its V tile must leave the ring).
+      if (lane == 0) {
+      for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
+        const Pair P = decode_pair<BN>(p, list, n_list, wi);
+        const int n_of[2] = {P.u0.lt + P.u0.cnt, P.u1.lt + P.u1.cnt};
+        int qk[2] = {0, 0};
+        // One unit's step at stream item j: its pending product goes first, or now if the unit
+        // skips the next item (its V tile must leave the ring); a unit's first Q_x·Kᵀ waits for
+        // its Q_x tile.
         auto step = [&](auto xc, int j, int users, int nusers, const uint64_t (&kb)[8]) -> bool {
           constexpr int x = decltype(xc)::value;
           const bool use = (users >> x) & 1;
-          if (pend[x] >= 0 && (use || !((nusers >> x) & 1))) {
-            if (!issue_pv(xc, pend[x])) return false;
-            pend[x] = -1;
-          }
+          if (pend[x] != kNone && (use || !((nusers >> x) & 1)) && !issue_pv(xc)) return false;
           if (use) {
+            if (qk[x] == 0) {
+              if (!mbar_wait(bar(kQFull + x), q_ph[x], lim)) return false;
+              q_ph[x] ^= 1u;
+              tc_fence_after();
+            }
             issue_qk(xc, kb);
-            pend[x] = j;
-            if (++qk[x] == n_of[x]) tc_commit(bar(kQEmpty + x));
+            pend[x] = v_base + (uint32_t)j;
+            pend_last[x] = ++qk[x] == n_of[x];
+            if (pend_last[x]) tc_commit(bar(kQEmpty + x));
           }
           return true;
         };
@@ -910,16 +949,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           users = nusers;
         }
-        if (ok && pend[0] >= 0) ok = issue_pv(std::integral_constant<int, 0>{}, pend[0]);
-        if (ok && pend[1] >= 0) ok = issue_pv(std::integral_constant<int, 1>{}, pend[1]);
-        if (!ok) break;
-        tc_commit(bar(kOFull + 0));
-        q_ph[0] ^= 1u;
-        if (P.valid1) {
-          tc_commit(bar(kOFull + 1));
-          q_ph[1] ^= 1u;
-        }
         v_base += (uint32_t)P.total;
+      }
+      // The window's last products: every role meets the next window barrier only after its
+      // units are complete.
+      if (ok && pend[0] != kNone) ok = issue_pv(std::integral_constant<int, 0>{});
+      if (ok && pend[1] != kNone) ok = issue_pv(std::integral_constant<int, 1>{});
       }
       __syncwarp();
       });
@@ -1055,8 +1090,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         l_run = l_run * alpha + rs;
         m_run = m_use;
+        // One arrival per warp (after the warp's tensor-memory stores): arrivals on one barrier
+        // are serialised, so 128 of them would delay the product by hundreds of cycles.
         tc_fence_before();
-        mbar_arrive(bar(kPFull + x));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kPFull + x));
       }
       if (!ok) break;
       // Epilogue: O/ℓ as bf16 at the query's original row.
@@ -1208,14 +1246,20 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
   p.Hkv = d.Hkv;
   p.G = d.G;
   p.n_units = d.bhq() * d.nB;
+  if (p.n_units > 0x7fffffffLL) return cudaErrorInvalidValue;  // unit ids are 32-bit
   p.n_items = (p.n_units + 1) / 2;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   p.limit_ns = limit_ns;
+  p.div_G.init(d.G);
+  p.div_nB.init(d.nB);
+  p.div_Hkv.init(d.Hkv);
   auto launch = [&](int mode, int skip_empty) -> cudaError_t {
     p.mode = mode;
     p.skip_empty = skip_empty;
     p.S = mode == kDense ? d.N : d.S;
     p.nSeg = mode == kDense ? 1 : d.nSeg;
+    p.div_seg.init(p.S / BN);
+    p.div_nSeg.init(p.nSeg);
     const long long work = skip_empty ? p.n_units : p.n_items;
     const long long grid = work < sm_count() ? work : sm_count();
     s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv,
