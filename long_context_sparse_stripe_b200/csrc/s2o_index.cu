@@ -1034,6 +1034,30 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
   return cudaGetLastError();
 }
 
+// A second stream of the calling thread on the current device, for kernels that are independent
+// of the caller's stream between a fork and a join (both by events, so the pair is also valid
+// inside stream capture). Created on first use, kept for the thread's lifetime.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
+};
+
+cudaError_t side_stream(SideStream **out) {
+  thread_local SideStream cache[16];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+  SideStream &ss = cache[dev];
+  if (!ss.s) {
+    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.fork_ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.join_ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
 template <int D>
 cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, const uint16_t *k,
                     const s2o_indices &out, char *ws, cudaStream_t st) {
@@ -1083,12 +1107,39 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, nq, d.N, out.perm_k, st)) !=
       cudaSuccess)
     return e;
+  // Key side of step 2c (block means K̄ and visibility counts): they depend only on perm_k and
+  // run on a side stream next to the query-side kernels, joined before the block scores.
+  const long long nblk = bhq * d.nB;
+  SideStream *side = nullptr;
+  if ((e = side_stream(&side)) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(side->fork_ev, st)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(side->s, side->fork_ev, 0)) != cudaSuccess) return e;
+  k_block_means<D><<<blocks_for(nblk, 8), 256, 0, side->s>>>(k, out.perm_k, Kbar, d.N, d.B, d.nB,
+                                                             nblk, d.Hq, d.Hkv, d.G, 1);
+  note_launch();
+  const size_t nc_smem = (size_t)32 * (d.B + 1) * sizeof(int);
+  k_ncount<<<dim3((d.nB + 31) / 32, (unsigned)bhq), 256, nc_smem, side->s>>>(
+      out.perm_k, ncount, d.N, d.B, d.S, d.nB, d.nSeg);
+  note_launch();
+  if ((e = cudaEventRecord(side->join_ev, side->s)) != cudaSuccess) return e;
+  // The caller's stream waits for the side stream on every path out of this function.
+  struct Join {
+    cudaStream_t st;
+    cudaEvent_t ev;
+    bool pending = true;
+    cudaError_t now() {
+      pending = false;
+      return cudaStreamWaitEvent(st, ev, 0);
+    }
+    ~Join() {
+      if (pending) cudaStreamWaitEvent(st, ev, 0);
+    }
+  } join{st, side->join_ev};
   // Step 1b: query scores against the top stripe block.
   k_kbar_top<<<(unsigned)bhq, D, 0, st>>>(k, out.perm_k, kbar_all, kbar_top, u, d.N, D, d.B, d.Hq,
                                           d.Hkv, d.G);
   note_launch();
   // Step 2b: query scores, segment-local query ordering, query block means.
-  const long long nblk = bhq * d.nB;
   const int qp = cfg.query_perm ? 1 : 0;
   k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
   note_launch();
@@ -1117,14 +1168,8 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
                                                         nblk, d.Hq, d.Hkv, d.G, 0);
   note_launch();
-  // Key block means, visibility counts, block scores.
-  k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(k, out.perm_k, Kbar, d.N, d.B, d.nB, nblk,
-                                                        d.Hq, d.Hkv, d.G, 1);
-  note_launch();
-  const size_t nc_smem = (size_t)32 * (d.B + 1) * sizeof(int);
-  k_ncount<<<dim3((d.nB + 31) / 32, (unsigned)bhq), 256, nc_smem, st>>>(out.perm_k, ncount, d.N,
-                                                                        d.B, d.S, d.nB, d.nSeg);
-  note_launch();
+  // Block scores (after the key side joins).
+  if ((e = join.now()) != cudaSuccess) return e;
   const float sigma = D == 64 ? 0x1p-3f : 0x1.6a09e6p-4f;  // nearest fp32 to 1/sqrt(D)
   const unsigned tiles = (unsigned)((d.nB + 127) / 128);
   k_block_scores<D><<<dim3(tiles, tiles, (unsigned)bhq), 256, 0, st>>>(Qbar, Kbar, r, d.nB, sigma);
