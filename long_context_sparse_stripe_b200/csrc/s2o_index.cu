@@ -99,8 +99,10 @@ __device__ __forceinline__ uint32_t sort_key(float x) {
 // Written for this project from the mathematics; defined for x <= 0 (all block-weight arguments).
 // k = rint(x/ln 2) is taken by adding and subtracting 1.5·2^52 (round half to even, as rint),
 // which also leaves k in the low word of the sum: no conversion instruction is needed.
-__device__ __forceinline__ double exp64(double x) {
-  if (x < -700.0) return 0.0;
+__device__ __forceinline__ double exp64(double x_in) {
+  // Branch-free: arguments below -700 (results that underflow) run the same steps on -700 and are
+  // replaced by 0 at the end, so that independent calls interleave.
+  const double x = x_in < -700.0 ? -700.0 : x_in;
   const double kInvLn2 = 0x1.71547652b82fep+0;  // nearest binary64 to 1/ln 2
   const double kLn2Hi = 0x1.62e42fefa39efp-1;   // nearest binary64 to ln 2
   const double kLn2Lo = 0x1.abc9e3b39803fp-56;  // nearest binary64 to ln 2 − kLn2Hi
@@ -120,7 +122,8 @@ __device__ __forceinline__ double exp64(double x) {
   for (int j = 12; j >= 0; --j) p = __fma_rn(p, t, c[j]);
   // k in [-1010, 0]: 2^k is a normal binary64 number, so the product is exact.
   const int ki = __double2loint(y);
-  return __dmul_rn(p, __hiloint2double((ki + 1023) << 20, 0));
+  const double e = __dmul_rn(p, __hiloint2double((ki + 1023) << 20, 0));
+  return x_in < -700.0 ? 0.0 : e;
 }
 
 // An integer 0 <= n < 2^31 as binary64, exactly, without a conversion instruction.
@@ -815,13 +818,14 @@ __global__ void __launch_bounds__(128)
       nv[k] = c < nB ? __ldg(nn + c) : 0;
       rv[k] = c < nB ? __ldg(rr + c) : 0.f;
     }
+    double wv[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k)
+      wv[k] = __dmul_rn(int_to_double(max(nv[k], 0)), exp64(__dsub_rn((double)rv[k], Md)));
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
       const int c = c0 + k * kWarp + lane;
-      if (c < nB)
-        w[wi(c)] = nv[k] > 0
-                       ? __dmul_rn(int_to_double(nv[k]), exp64(__dsub_rn((double)rv[k], Md)))
-                       : -1.0;
+      if (c < nB) w[wi(c)] = nv[k] > 0 ? wv[k] : -1.0;
     }
   }
   __syncwarp();
