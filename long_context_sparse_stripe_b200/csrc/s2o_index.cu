@@ -320,10 +320,10 @@ __device__ __forceinline__ unsigned match_digit(uint32_t d) {
 // One counting pass inside a CTA: the destination, in stable order by digit, of R elements per
 // lane (element r of lane l of warp w is w·32R + r·32 + l). Scratch: hist[warps·256],
 // dbase[256]. Also returns, in dbase, each digit's first destination.
-template <int R>
+template <int R, int NW>
 __device__ __forceinline__ void radix_ranks(const uint32_t (&digit)[R], int (&dest)[R],
                                             int *hist, int *dbase) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const unsigned full = 0xffffffffu, below = (1u << lane) - 1u;
   int *wh = hist + warp * 256;
   for (int d = lane; d < 256; d += 32) wh[d] = 0;
@@ -338,13 +338,17 @@ __device__ __forceinline__ void radix_ranks(const uint32_t (&digit)[R], int (&de
     __syncwarp();
   }
   __syncthreads();
-  // Per digit: exclusive prefix over the warps (in place) and the digit's total.
+  // Per digit: exclusive prefix over the NW warps (in place) and the digit's total; the NW
+  // counts are loaded together.
   for (int d = threadIdx.x; d < 256; d += blockDim.x) {
+    int c[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) c[w] = hist[w * 256 + d];
     int run = 0;
-    for (int w = 0; w < nwarps; ++w) {
-      const int c = hist[w * 256 + d];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
       hist[w * 256 + d] = run;
-      run += c;
+      run += c[w];
     }
     dbase[d] = run;
   }
@@ -406,7 +410,7 @@ __global__ void __launch_bounds__(512)
     int dest[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) dig[r] = (key[r] >> (8 * pass)) & 255u;
-    radix_ranks<R>(dig, dest, hist, dbase);
+    radix_ranks<R, 16>(dig, dest, hist, dbase);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       skey[dest[r]] = key[r];
@@ -477,6 +481,47 @@ __global__ void __launch_bounds__(kRadixThreads)
     counts[(run * 256 + d) * tiles + tile] = h[d];
 }
 
+// Output offsets of one pass, in place over the counts: for run, digit d and tile t, the number of
+// elements of the run with a smaller digit plus those with digit d in tiles before t. One CTA of
+// 256 threads per run (thread = digit).
+__global__ void __launch_bounds__(256) k_radix_offsets(int *__restrict__ counts, int tiles) {
+  __shared__ int tot[256];
+  const long long run = blockIdx.x;
+  const int d = threadIdx.x;
+  int *c = counts + (run * 256 + d) * tiles;
+  int sum = 0;
+  for (int t = 0; t < tiles; ++t) sum += c[t];
+  tot[d] = sum;
+  __syncthreads();
+  if (d < 32) {  // exclusive scan of the 256 digit totals, 8 per lane
+    int v[8], s8 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = tot[d * 8 + i];
+      s8 += v[i];
+    }
+    int incl = s8;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (d >= o) incl += t;
+    }
+    int run_sum = incl - s8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      tot[d * 8 + i] = run_sum;
+      run_sum += v[i];
+    }
+  }
+  __syncthreads();
+  int off = tot[d];
+  for (int t = 0; t < tiles; ++t) {
+    const int x = c[t];
+    c[t] = off;
+    off += x;
+  }
+}
+
 // Scatter of one pass: each tile ranks its elements by digit (stable), groups them in shared
 // memory and writes each digit's run to its offset. The last pass writes only the values, as the
 // permutation.
@@ -484,7 +529,7 @@ __global__ void __launch_bounds__(kRadixThreads)
     k_radix_scatter(const float *__restrict__ score, const uint32_t *__restrict__ keys_in,
                     const uint32_t *__restrict__ vals_in, uint32_t *__restrict__ keys_out,
                     uint32_t *__restrict__ vals_out, int32_t *__restrict__ perm_out,
-                    long long run_len, int tiles, int shift, const int *__restrict__ offsets) {  // raw digit counts of the pass
+                    long long run_len, int tiles, int shift, const int *__restrict__ offsets) {
   extern __shared__ int sm_r[];
   uint32_t *skey = reinterpret_cast<uint32_t *>(sm_r);   // [tile]
   uint32_t *sval = skey + kRadixTile;                     // [tile]
@@ -495,54 +540,15 @@ __global__ void __launch_bounds__(kRadixThreads)
   const int tile = blockIdx.x % tiles;
   const long long base = run * run_len + (long long)tile * kRadixTile;
   const int n = (int)min((long long)kRadixTile, run_len - (long long)tile * kRadixTile);
-  // This tile's output offset per digit, from the run's raw counts: the digits before it over
-  // the whole run, plus the same digit in the tiles before this one.
-  if (threadIdx.x < 256) {
-    const int d = threadIdx.x;
-    const int *c = offsets + (run * 256 + d) * tiles;
-    int before = 0, total = 0;
-    for (int t0 = 0; t0 < tiles; t0 += 8) {
-      int v[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = t0 + k < tiles ? __ldg(c + t0 + k) : 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        before += t0 + k < tile ? v[k] : 0;
-        total += v[k];
-      }
-    }
-    goff[d] = before;
-    dbase[d] = total;
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {  // exclusive scan of the digit totals, 8 per lane
-    const int lane = threadIdx.x;
-    int v[8], sum = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = dbase[lane * 8 + i];
-      sum += v[i];
-    }
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    int run_sum = incl - sum;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      goff[lane * 8 + i] += run_sum;
-      run_sum += v[i];
-    }
-  }
+  // This tile's output offset per digit (prefixed by k_radix_offsets).
+  if (threadIdx.x < 256) goff[threadIdx.x] = __ldg(offsets + (run * 256 + threadIdx.x) * tiles + tile);
   __syncthreads();
   uint32_t key[kRadixR], val[kRadixR], dig[kRadixR];
   int dest[kRadixR];
   radix_load(score, keys_in, vals_in, base, tile * kRadixTile, n, key, val);
 #pragma unroll
   for (int r = 0; r < kRadixR; ++r) dig[r] = (key[r] >> shift) & 255u;
-  radix_ranks<kRadixR>(dig, dest, hist, dbase);
+  radix_ranks<kRadixR, kRadixThreads / 32>(dig, dest, hist, dbase);
 #pragma unroll
   for (int r = 0; r < kRadixR; ++r) {
     skey[dest[r]] = key[r];
@@ -646,7 +652,7 @@ __global__ void __launch_bounds__(256)
 // values of t at a time, and the next 32 are loaded into registers while the current ones are
 // consumed.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
     k_block_scores(const float *__restrict__ Qbar, const float *__restrict__ Kbar,
                    float *__restrict__ r, int nB, float sigma) {
   __shared__ __align__(16) float As[32][128 + 4];
@@ -687,12 +693,11 @@ __global__ void __launch_bounds__(256, 1)
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
-  fetch(0);
   for (int t0 = 0; t0 < D; t0 += 32) {
+    fetch(t0);
     __syncthreads();  // the previous chunk has been consumed
     stash();
     __syncthreads();
-    if (t0 + 32 < D) fetch(t0 + 32);
 #pragma unroll 8
     for (int tt = 0; tt < 32; ++tt) {
       const float4 a0 = *reinterpret_cast<const float4 *>(&As[tt][tr * 8]);
@@ -1025,6 +1030,8 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
   for (int pass = 0; pass < 4; ++pass) {
     const float *sc = pass == 0 ? score : nullptr;
     k_radix_count<<<grid, kRadixThreads, 0, st>>>(sc, kin, run_len, tiles, 8 * pass, counts);
+    note_launch();
+    k_radix_offsets<<<(unsigned)runs, 256, 0, st>>>(counts, tiles);
     note_launch();
     k_radix_scatter<<<grid, kRadixThreads, smem, st>>>(sc, kin, vin, kout, vout,
                                                        pass == 3 ? perm_out : nullptr, run_len,
