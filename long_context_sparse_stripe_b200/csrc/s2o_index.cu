@@ -490,7 +490,13 @@ __global__ void __launch_bounds__(256) k_radix_offsets(int *__restrict__ counts,
   const int d = threadIdx.x;
   int *c = counts + (run * 256 + d) * tiles;
   int sum = 0;
-  for (int t = 0; t < tiles; ++t) sum += c[t];
+  for (int t0 = 0; t0 < tiles; t0 += 8) {  // eight loads in flight
+    int v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = t0 + k < tiles ? c[t0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sum += v[k];
+  }
   tot[d] = sum;
   __syncthreads();
   if (d < 32) {  // exclusive scan of the 256 digit totals, 8 per lane
@@ -515,10 +521,15 @@ __global__ void __launch_bounds__(256) k_radix_offsets(int *__restrict__ counts,
   }
   __syncthreads();
   int off = tot[d];
-  for (int t = 0; t < tiles; ++t) {
-    const int x = c[t];
-    c[t] = off;
-    off += x;
+  for (int t0 = 0; t0 < tiles; t0 += 8) {
+    int v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = t0 + k < tiles ? c[t0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (t0 + k < tiles) c[t0 + k] = off;
+      off += v[k];
+    }
   }
 }
 
