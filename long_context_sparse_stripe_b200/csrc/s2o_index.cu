@@ -219,24 +219,38 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   const int j = chunk * B + r;
   if (r < B) {
+    // Up to four query heads at a time: their chains interleave (each still runs over t in
+    // order) and the row is read once per group of heads.
     const uint4 *row = reinterpret_cast<const uint4 *>(rows + r * RS);
-    for (int hi = 0; hi < G; ++hi) {
-      const float4 *qv = sm4 + (size_t)hi * D / 4;
-      float acc = 0.f;
-#pragma unroll 4
+    for (int h0 = 0; h0 < G; h0 += 4) {
+      const int nh = min(4, G - h0);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
       for (int c = 0; c < D / 8; ++c) {
         const uint4 v = row[c];
-        const float4 a = qv[2 * c], b = qv[2 * c + 1];
-        acc = __fmaf_rn(bf16_lo(v.x), a.x, acc);
-        acc = __fmaf_rn(bf16_hi(v.x), a.y, acc);
-        acc = __fmaf_rn(bf16_lo(v.y), a.z, acc);
-        acc = __fmaf_rn(bf16_hi(v.y), a.w, acc);
-        acc = __fmaf_rn(bf16_lo(v.z), b.x, acc);
-        acc = __fmaf_rn(bf16_hi(v.z), b.y, acc);
-        acc = __fmaf_rn(bf16_lo(v.w), b.z, acc);
-        acc = __fmaf_rn(bf16_hi(v.w), b.w, acc);
+        const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                            bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          if (hh < nh) {
+            const float4 *qv = sm4 + (size_t)(h0 + hh) * D / 4;
+            const float4 a = qv[2 * c], b = qv[2 * c + 1];
+            float t = acc[hh];
+            t = __fmaf_rn(x[0], a.x, t);
+            t = __fmaf_rn(x[1], a.y, t);
+            t = __fmaf_rn(x[2], a.z, t);
+            t = __fmaf_rn(x[3], a.w, t);
+            t = __fmaf_rn(x[4], b.x, t);
+            t = __fmaf_rn(x[5], b.y, t);
+            t = __fmaf_rn(x[6], b.z, t);
+            t = __fmaf_rn(x[7], b.w, t);
+            acc[hh] = t;
+          }
+        }
       }
-      kappa[(qh0 + hi) * N + j] = acc;
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh)
+        if (hh < nh) kappa[(qh0 + h0 + hh) * N + j] = acc[hh];
     }
   }
   if (r < D / 2) {
