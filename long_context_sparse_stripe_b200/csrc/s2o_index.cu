@@ -554,7 +554,8 @@ __global__ void __launch_bounds__(kRadixThreads)
     k_radix_scatter(const float *__restrict__ score, const uint32_t *__restrict__ keys_in,
                     const uint32_t *__restrict__ vals_in, uint32_t *__restrict__ keys_out,
                     uint32_t *__restrict__ vals_out, int32_t *__restrict__ perm_out,
-                    long long run_len, int tiles, int shift, const int *__restrict__ offsets) {
+                    long long run_len, long long head_len, int tiles, int shift,
+                    const int *__restrict__ offsets) {
   extern __shared__ int sm_r[];
   uint32_t *skey = reinterpret_cast<uint32_t *>(sm_r);   // [tile]
   uint32_t *sval = skey + kRadixTile;                     // [tile]
@@ -585,8 +586,8 @@ __global__ void __launch_bounds__(kRadixThreads)
     const uint32_t k = skey[i];
     const int d = (int)((k >> shift) & 255u);
     const long long o = out0 + goff[d] + (i - dbase[d]);
-    if (perm_out)
-      perm_out[o] = (int32_t)sval[i];
+    if (perm_out)  // positions within the head: a run's first element sits at run·run_len mod N
+      perm_out[o] = (int32_t)((run * run_len) % head_len + sval[i]);
     else {
       keys_out[o] = k;
       vals_out[o] = sval[i];
@@ -1039,10 +1040,12 @@ __global__ void k_exp64_probe(const double *x, double *y, int n) {
 inline unsigned blocks_for(long long n, int per) { return (unsigned)((n + per - 1) / per); }
 
 // Stable radix sort of runs of run_len scores each (descending, ties to the lower index), the
-// permutation written to perm_out. Keys and values ping-pong between (k0, v0) and (k1, v1).
+// permutation written to perm_out as positions within a head of head_len elements (a run of
+// segment length S starts at its segment's first position). Keys and values ping-pong between
+// (k0, v0) and (k1, v1).
 cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint32_t *k1,
                             uint32_t *v1, int *counts, long long total, long long run_len,
-                            int32_t *perm_out, cudaStream_t st) {
+                            long long head_len, int32_t *perm_out, cudaStream_t st) {
   const int tiles = (int)((run_len + kRadixTile - 1) / kRadixTile);
   const long long runs = total / run_len;
   const unsigned grid = (unsigned)(runs * tiles);
@@ -1060,6 +1063,7 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
     note_launch();
     k_radix_scatter<<<grid, kRadixThreads, smem, st>>>(sc, kin, vin, kout, vout,
                                                        pass == 3 ? perm_out : nullptr, run_len,
+                                                       head_len,
                                                        tiles, 8 * pass, counts);
     note_launch();
     kin = kout;
@@ -1140,7 +1144,7 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
                                                                          (float)d.N);
   note_launch();
   // Step 2a: global key/value ordering.
-  if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, nq, d.N, out.perm_k, st)) !=
+  if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, nq, d.N, d.N, out.perm_k, st)) !=
       cudaSuccess)
     return e;
   // Key side of step 2c (block means K̄ and visibility counts): they depend only on perm_k and
@@ -1197,7 +1201,7 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
     note_launch();
   } else {
     // Segments longer than one CTA's sort: the multi-CTA radix sort over runs of S.
-    if ((e = radix_sort_runs(rho, rk0, rv0, rk1, rv1, rcount, nq, d.S, out.perm_q, st)) !=
+    if ((e = radix_sort_runs(rho, rk0, rv0, rk1, rv1, rcount, nq, d.S, d.N, out.perm_q, st)) !=
         cudaSuccess)
       return e;
   }

@@ -26,6 +26,10 @@ W_C = gen.Workload("c-d64-b128", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=204
                    segment_len=512, block_size=128, tau=0.02, seed=8)
 W_D = gen.Workload("d-d128-b64", batch=1, n_q_heads=2, n_kv_heads=2, seq_len=2048, head_dim=128,
                    segment_len=512, block_size=64, tau=0.02, seed=9)
+# Segments longer than one CTA's sort (S > 4096): the query ordering takes the multi-CTA radix
+# sort, and the key ordering then runs before the query-side kernels instead of next to them.
+W_E = gen.Workload("e-long-segments", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=16384,
+                   head_dim=64, segment_len=8192, block_size=128, tau=0.01, seed=10)
 W_TINY = gen.workload("tiny")
 
 INDEX_NAMES = ("perm_q", "perm_k", "sel_cnt", "local_tiles")
@@ -90,7 +94,7 @@ def test_exp64_bit_exact_with_oracle():
 
 @pytest.mark.parametrize("w", [
     W_TINY, W_TINY.replace(tau=0.0), W_TINY.replace(tau=0.07), W_TINY.replace(tau=0.2),
-    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D,
+    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E,
 ], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
 def test_indices_and_intermediates_bit_exact(w):
     q, k, _ = inputs(w)
