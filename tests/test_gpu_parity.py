@@ -30,6 +30,13 @@ W_D = gen.Workload("d-d128-b64", batch=1, n_q_heads=2, n_kv_heads=2, seq_len=204
 # sort, and the key ordering then runs before the query-side kernels instead of next to them.
 W_E = gen.Workload("e-long-segments", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=16384,
                    head_dim=64, segment_len=8192, block_size=128, tau=0.01, seed=10)
+# Ragged everywhere: a key run of 1.5 radix tiles, 96 blocks (not a multiple of the 32-block
+# chunks of the schedule or of the 128-block score tiles), 3072-query segments.
+W_F = gen.Workload("f-ragged-tiles", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=6144,
+                   head_dim=64, segment_len=3072, block_size=64, tau=0.01, seed=11)
+# One segment spanning the whole sequence (the local window is the causal triangle of all keys).
+W_G = gen.Workload("g-one-segment", batch=1, n_q_heads=2, n_kv_heads=2, seq_len=4096,
+                   head_dim=128, segment_len=4096, block_size=128, tau=0.01, seed=12)
 W_TINY = gen.workload("tiny")
 
 INDEX_NAMES = ("perm_q", "perm_k", "sel_cnt", "local_tiles")
@@ -94,7 +101,7 @@ def test_exp64_bit_exact_with_oracle():
 
 @pytest.mark.parametrize("w", [
     W_TINY, W_TINY.replace(tau=0.0), W_TINY.replace(tau=0.07), W_TINY.replace(tau=0.2),
-    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E,
+    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E, W_F, W_G,
 ], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
 def test_indices_and_intermediates_bit_exact(w):
     q, k, _ = inputs(w)
@@ -120,7 +127,7 @@ def test_index_build_is_deterministic():
 # ----------------------------------------------------------------------------- attention
 
 @pytest.mark.parametrize("w", [W_TINY, W_TINY.replace(tau=0.07), W_TINY.replace(tau=1.5), W_A,
-                               W_A.replace(query_perm=0), W_C, W_D],
+                               W_A.replace(query_perm=0), W_C, W_D, W_F, W_G],
                          ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
 def test_attention_on_oracle_indices(w):
     q, k, v = inputs(w)
