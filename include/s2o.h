@@ -146,6 +146,12 @@ s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *
  * Affects launches made after the call; not thread-safe against concurrent launches. */
 void s2o_set_wait_limit_ns(uint64_t ns);
 
+/* Caps the persistent attention grid at `max_ctas` CTAs (0, the default: one CTA per SM). A smaller
+ * grid gives each CTA more work items and more work-list windows, which lets small inputs exercise
+ * the window turnover; results do not depend on the grid. Affects launches made after the call;
+ * not thread-safe against concurrent launches. Negative values are treated as 0. */
+void s2o_set_attention_max_ctas(int max_ctas);
+
 /* Number of kernel launches the library has made in this process so far (all threads and
  * devices), for launch accounting. Host only. */
 uint64_t s2o_kernel_launch_count(void);

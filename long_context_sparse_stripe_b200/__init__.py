@@ -24,7 +24,7 @@ __all__ = [
     "Config", "Indices", "Stats", "S2OError", "workspace_size", "index_sizes", "alloc_indices",
     "alloc_workspace", "build_indices", "attention_prefill", "attention_prefill_with_indices",
     "dense_causal_prefill", "validate_indices", "index_stats", "workspace_views",
-    "set_wait_limit_ns", "check_device_status", "exp64_eval", "library_path",
+    "set_wait_limit_ns", "set_attention_max_ctas", "check_device_status", "exp64_eval", "library_path",
     "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
 ]
 
@@ -163,6 +163,8 @@ def _load():
         lib.s2o_kernel_launch_count.restype = ctypes.c_uint64
         lib.s2o_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         lib.s2o_set_wait_limit_ns.restype = None
+        lib.s2o_set_attention_max_ctas.argtypes = [ctypes.c_int]
+        lib.s2o_set_attention_max_ctas.restype = None
         lib.s2o_status_string.argtypes = [st]
         lib.s2o_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -335,6 +337,11 @@ def kernel_launch_count() -> int:
 
 def set_wait_limit_ns(ns: int) -> None:
     _load().s2o_set_wait_limit_ns(int(ns))
+
+
+def set_attention_max_ctas(max_ctas: int) -> None:
+    """Caps the persistent attention grid (0 = one CTA per SM); results do not depend on it."""
+    _load().s2o_set_attention_max_ctas(int(max_ctas))
 
 
 def check_device_status(device="cuda") -> int:

@@ -10,6 +10,7 @@ namespace s2o {
 
 namespace {
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_attention_max_ctas{0};
 std::atomic<unsigned long long> g_launches{0};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -189,6 +190,7 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
   AttnArgs a{q, k, v, o, idx->perm_q, idx->perm_k, idx->sel_cnt, idx->sel_blk, idx->local_tiles,
              false};
   return from_cuda(launch_attention(dims_of(*cfg), a, g_wait_limit_ns.load(),
+                                    g_attention_max_ctas.load(),
                                     (cudaStream_t)stream));
 }
 
@@ -212,7 +214,8 @@ s2o_status s2o_dense_causal_prefill(const s2o_config *cfg, const void *q, const 
   s2o_config c = *cfg;
   c.segment_len = c.seq_len;
   AttnArgs a{q, k, v, o, nullptr, nullptr, nullptr, nullptr, nullptr, true};
-  return from_cuda(launch_attention(dims_of(c), a, g_wait_limit_ns.load(), (cudaStream_t)stream));
+  return from_cuda(launch_attention(dims_of(c), a, g_wait_limit_ns.load(),
+                                    g_attention_max_ctas.load(), (cudaStream_t)stream));
 }
 
 s2o_status s2o_validate_indices(const s2o_config *cfg, const s2o_indices *idx, void *ws,
@@ -260,6 +263,10 @@ s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *
 }
 
 void s2o_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+void s2o_set_attention_max_ctas(int max_ctas) {
+  g_attention_max_ctas.store(max_ctas > 0 ? max_ctas : 0);
+}
 
 uint64_t s2o_kernel_launch_count(void) { return launch_count(); }
 

@@ -1218,7 +1218,8 @@ int sm_count() {
 }
 
 template <int D, int BN>
-cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaStream_t st) {
+cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int max_ctas,
+                     cudaStream_t st) {
   using L = Layout<D, BN>;
   static_assert(L::SMEM <= 232448, "shared memory budget");
   static_assert(kNumBars * 8 + 4 <= (int)L::BAR_BYTES, "barrier area");
@@ -1261,7 +1262,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
     p.div_seg.init(p.S / BN);
     p.div_nSeg.init(p.nSeg);
     const long long work = skip_empty ? p.n_units : p.n_items;
-    const long long grid = work < sm_count() ? work : sm_count();
+    const long long cap = max_ctas > 0 && max_ctas < sm_count() ? max_ctas : sm_count();
+    const long long grid = work < cap ? work : cap;
     s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv,
                                                                            tvr, to, p);
     note_launch();
@@ -1279,11 +1281,11 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, cudaSt
 }  // namespace
 
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
-                             cudaStream_t st) {
-  if (d.D == 128 && d.B == 128) return launch_t<128, 128>(d, a, wait_limit_ns, st);
-  if (d.D == 128 && d.B == 64) return launch_t<128, 64>(d, a, wait_limit_ns, st);
-  if (d.D == 64 && d.B == 128) return launch_t<64, 128>(d, a, wait_limit_ns, st);
-  return launch_t<64, 64>(d, a, wait_limit_ns, st);
+                             int max_ctas, cudaStream_t st) {
+  if (d.D == 128 && d.B == 128) return launch_t<128, 128>(d, a, wait_limit_ns, max_ctas, st);
+  if (d.D == 128 && d.B == 64) return launch_t<128, 64>(d, a, wait_limit_ns, max_ctas, st);
+  if (d.D == 64 && d.B == 128) return launch_t<64, 128>(d, a, wait_limit_ns, max_ctas, st);
+  return launch_t<64, 64>(d, a, wait_limit_ns, max_ctas, st);
 }
 
 cudaError_t read_and_clear_device_error(unsigned int *out, cudaStream_t st) {

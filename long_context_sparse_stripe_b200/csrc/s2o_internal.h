@@ -44,7 +44,7 @@ struct AttnArgs {
   bool dense;
 };
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
-                             cudaStream_t st);
+                             int max_ctas, cudaStream_t st);
 
 // Host-side count of kernel launches made by the library (all threads, all devices).
 void note_launch();

@@ -266,3 +266,28 @@ def test_sparsity_monotone_in_tau_on_gpu():
         if prev is not None:
             assert pairs <= prev
         prev = pairs
+
+
+def test_attention_independent_of_grid_and_windows():
+    """A grid of one, two or five CTAs makes every CTA walk several work-list windows (the work
+    list holds 128 work items): the local, permuted and dense passes give the same bits as the
+    full grid, and the selected blocks of the ragged case reach the permuted pass."""
+    w = W_B
+    q, k, v = inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w)
+    idx = s2o.build_indices(cfg, qd, kd)
+    assert int(idx.sel_cnt.sum()) > 0
+    base = s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx)
+    dense = s2o.dense_causal_prefill(cfg, qd, kd, vd)
+    try:
+        for n in (1, 2, 5):
+            s2o.set_attention_max_ctas(n)
+            o = s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx)
+            d = s2o.dense_causal_prefill(cfg, qd, kd, vd)
+            torch.cuda.synchronize()
+            assert s2o.check_device_status() == 0
+            assert torch.equal(o, base), f"grid of {n}: S2O output differs"
+            assert torch.equal(d, dense), f"grid of {n}: dense output differs"
+    finally:
+        s2o.set_attention_max_ctas(0)
