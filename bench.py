@@ -136,18 +136,34 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE / MASTER_*): the process
+    group for the barriers and the max-over-ranks times; None when the job has one rank. The
+    tests drive the same code with the gloo backend on the host."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timedelta(seconds=60))
         return dist, rank, world, local
     return None, 0, 1, 0
+
+
+def layer_seed(w, rank: int) -> int:
+    """Seed of the independent layer rank `rank` runs (weak scaling: one layer per GPU)."""
+    return w.seed + 100 * rank
+
+
+def whole_job_value(flops_per_layer: float, world: int, ms_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's layer over the slowest rank's step time."""
+    return flops_per_layer * world / (ms_step * 1e-3) / 1e12
 
 
 def max_over_ranks(dist, x: float, device) -> float:
@@ -222,7 +238,7 @@ def run_s2o(args):
     torch.cuda.set_device(dev)
     w = gen.workload(args.workload, tau=args.tau)
     # Each rank runs its own independent layer (weak scaling).
-    q, k, v = gen.make_inputs(w.replace(seed=w.seed + 100 * rank))
+    q, k, v = gen.make_inputs(w.replace(seed=layer_seed(w, rank)))
     cfg = s2o.Config.of(w)
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     o = torch.empty_like(qd)
@@ -318,13 +334,12 @@ def run_s2o(args):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.e2e_steps, dev)
 
-    flops_all = w.dense_causal_flops * world
     line = None
     if rank == 0:
         achieved = exec_flops / (attn_ms_max * 1e-3) / 1e12
         line = {
             "metric": METRIC,
-            "value": flops_all / (ms_step * 1e-3) / 1e12,
+            "value": whole_job_value(w.dense_causal_flops, world, ms_step),
             "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
@@ -350,7 +365,7 @@ def run_s2o(args):
                          "traffic": attention_traffic(args.workload),
                          "kernel": "s2o_attention_kernel<128,128> (local + permuted pass)",
                          "peak_source": f"{peak_kind} bf16 (burst)"},
-            "e2e": {"value": flops_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+            "e2e": {"value": whole_job_value(w.dense_causal_flops, world, e2e_ms), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks.summary(),
