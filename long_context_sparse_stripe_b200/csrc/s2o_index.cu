@@ -272,10 +272,17 @@ __global__ void k_kbar_top(const uint16_t *__restrict__ k, const int32_t *__rest
   const long long qh = blockIdx.x;
   const long long kh = (qh / Hq) * Hkv + (qh % Hq) / G;
   const int t = threadIdx.x;
+  // Rows in rank order, sixteen loads in flight, added sequentially.
   float acc = 0.f;
-  for (int e = 0; e < B; ++e) {
-    const int j = __ldg(perm_k + qh * N + e);
-    acc = __fadd_rn(acc, bf16_at(k + ((size_t)kh * N + j) * D + t));
+  for (int e0 = 0; e0 < B; e0 += 16) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int j = __ldg(perm_k + qh * N + e0 + i);
+      v[i] = bf16_at(k + ((size_t)kh * N + j) * D + t);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc = __fadd_rn(acc, v[i]);
   }
   const float top = __fdiv_rn(acc, (float)B);
   kbar_top[qh * D + t] = top;
