@@ -91,6 +91,27 @@ def test_llama_128k_tau_sweep(tau):
     check_layer(gen.workload("llama-128k", tau=tau), groups=(0,) if tau != 0.01 else (0, 7))
 
 
+def test_dense_kernel_full_size_sampled_rows():
+    """The in-repo dense baseline (the bench's MSE reference and speed baseline) at 128K against
+    Eq. 1 on sampled rows: the first and last row of every head and random rows."""
+    w = gen.workload("llama-128k")
+    q, k, v = inputs(w)
+    cfg = s2o.Config.of(w)
+    o = s2o.dense_causal_prefill(cfg, *(t.cuda() for t in (q, k, v)))
+    torch.cuda.synchronize()
+    assert s2o.check_device_status() == 0
+    rng = np.random.default_rng(3)
+    total = w.n_q_heads * w.seq_len
+    heads = np.arange(w.n_q_heads) * w.seq_len
+    rows = np.unique(np.concatenate([heads, heads + w.seq_len - 1,
+                                     rng.choice(total, 192, replace=False)]))
+    want = oracle.dense_causal(oracle.config(w), q, k, v, rows=rows)
+    got = o.reshape(-1, w.head_dim)[torch.from_numpy(rows).cuda()]
+    err = np.abs(got.float().cpu().numpy().astype(np.float64) - want)
+    assert err.max() <= MAX_ABS, f"max abs error {err.max():.3g}"
+    assert err.mean() <= MEAN_ABS, f"mean abs error {err.mean():.3g}"
+
+
 @pytest.mark.parametrize("variant", ["tau0.001", "S1024", "S4096", "qperm-off"])
 def test_qwen_128k_ablation(variant):
     w = gen.workload("qwen-128k")
