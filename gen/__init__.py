@@ -51,6 +51,7 @@ class Workload:
     q_shift: float = 1.0
     diag: float = 0.5
     query_perm: int = 1
+    shared_key_order: int = 0
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

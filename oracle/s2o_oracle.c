@@ -36,6 +36,7 @@ typedef struct {
   int batch, n_q_heads, n_kv_heads, seq_len, head_dim, segment_len, block_size;
   float tau;
   int query_perm; /* 1: segment-local query ordering (default); 0: identity (Q-perm ablation) */
+  int shared_key_order; /* 0: one key ordering per query head (default); 1: per KV head */
 } oracle_config;
 
 /* Optional intermediate values, all per (batch, query head) unless noted; any pointer may be
@@ -196,10 +197,27 @@ static int build_head(const oracle_config *cfg, const uint16_t *q_all, const uin
     return ORACLE_ERR_NOMEM;
   for (int i = 0; i < N; ++i) ident[i] = i;
 
-  /* Step 1a — vertical-stripe pooling: mean query, mean key, kappa_j = qbar·k_j. */
+  /* Step 1a — vertical-stripe pooling: mean query, mean key, kappa_j = qbar·k_j. With a
+   * shared key ordering kappa uses the group's pooled query: the G heads' mean queries added in
+   * head order, divided by G. */
   list_mean(Q, d, ident, N, B, qbar);
   list_mean(K, d, ident, N, B, kbar_all);
-  for (int j = 0; j < N; ++j) kappa[j] = dot_f32_bf16(qbar, K + (size_t)j * d, d);
+  if (cfg->shared_key_order) {
+    float *qsum = malloc((size_t)d * sizeof(float));
+    float *qh_bar = malloc((size_t)d * sizeof(float));
+    if (!qsum || !qh_bar) return ORACLE_ERR_NOMEM;
+    for (int t = 0; t < d; ++t) qsum[t] = 0.0f;
+    for (int hh = g * G; hh < (g + 1) * G; ++hh) {
+      list_mean(q_all + ((size_t)bi * Hq + hh) * N * d, d, ident, N, B, qh_bar);
+      for (int t = 0; t < d; ++t) qsum[t] = qsum[t] + qh_bar[t];
+    }
+    for (int t = 0; t < d; ++t) qsum[t] = qsum[t] / (float)G;
+    for (int j = 0; j < N; ++j) kappa[j] = dot_f32_bf16(qsum, K + (size_t)j * d, d);
+    free(qsum);
+    free(qh_bar);
+  } else {
+    for (int j = 0; j < N; ++j) kappa[j] = dot_f32_bf16(qbar, K + (size_t)j * d, d);
+  }
 
   /* Step 2a — global key/value ordering: stable descending sort of kappa. */
   for (int j = 0; j < N; ++j) {

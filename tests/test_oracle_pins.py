@@ -328,3 +328,43 @@ def test_float64_rederivation_of_pooled_quantities():
             seg_of_key = pk.reshape(nB, Bk) // S
             n = np.stack([(seg_of_key < s).sum(1) for s in range(N // S)])
             np.testing.assert_array_equal(idx["n"][b, h], n)
+
+
+def test_shared_key_order_variant():
+    """The labelled variant with one key ordering per KV head: the group's kappa is the float64
+    product of K_g with the mean of the group's mean queries; every query head of a group carries
+    that ordering (a sorted permutation of kappa, ties to the lower index) and reads its k̄_top and
+    K̄ from it; it differs from the per-head ordering when G > 1, and equals it when G = 1."""
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    idx = oracle.build_indices(oracle.config(w, shared_key_order=1), q, k, debug=True)
+    base = oracle.build_indices(oracle.config(w), q, k)
+    Q, K = q.double().numpy(), k.double().numpy()
+    G, N, Bk, d = w.n_q_heads // w.n_kv_heads, w.seq_len, w.block_size, w.head_dim
+    nB = N // Bk
+    tol = dict(rtol=1e-5, atol=1e-5)
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            heads = range(g * G, (g + 1) * G)
+            qg = np.mean([Q[b, h].mean(0) for h in heads], axis=0)
+            Kg = K[b, g]
+            pk = idx["perm_k"][b, g * G]
+            assert sorted(pk.tolist()) == list(range(N))
+            for h in heads:
+                np.testing.assert_allclose(idx["kappa"][b, h], Kg @ qg, **tol)
+                np.testing.assert_array_equal(idx["perm_k"][b, h], pk)
+                u = Kg[pk[:Bk]].mean(0) - Kg.mean(0)
+                np.testing.assert_allclose(idx["u"][b, h], u, **tol)
+                np.testing.assert_allclose(idx["Kbar"][b, h],
+                                           Kg[pk].reshape(nB, Bk, d).mean(1), **tol)
+            ks = idx["kappa"][b, g * G][pk]
+            assert (np.diff(ks) <= 0).all()
+            ties = np.nonzero(np.diff(ks) == 0)[0]
+            assert (pk[ties] < pk[ties + 1]).all()
+    assert not np.array_equal(idx["perm_k"], base["perm_k"])
+    w1 = SMALL_GQA.replace(name="small-mha", n_q_heads=2, n_kv_heads=2)
+    q1, k1, _ = gen.make_inputs(w1)
+    a = oracle.build_indices(oracle.config(w1, shared_key_order=1), q1, k1)
+    c = oracle.build_indices(oracle.config(w1), q1, k1)
+    for name in ("perm_q", "perm_k", "sel_cnt", "sel_blk", "local_tiles"):
+        np.testing.assert_array_equal(a[name], c[name], err_msg=name)
