@@ -47,11 +47,15 @@ typedef enum {
 } s2o_status;
 
 /* One attention layer. `query_perm` = 1 builds the segment-local query ordering; 0 keeps the
- * identity (the "Q perm" ablation of [S2O, Key points]). */
+ * identity (the "Q perm" ablation of [S2O, Key points]). `shared_key_order` = 0 (the default)
+ * builds one key ordering per query head; 1 builds one per KV head, ranked by the group's pooled
+ * query, and writes it to the perm_k row of each of the group's query heads (a labelled variant:
+ * the pages say "for each head" without saying which kind of head). */
 typedef struct {
   int batch, n_q_heads, n_kv_heads, seq_len, head_dim, segment_len, block_size;
   float tau;
   int query_perm;
+  int shared_key_order;
 } s2o_config;
 
 /* Caller-owned index arrays (device, int32). nB = N / B.

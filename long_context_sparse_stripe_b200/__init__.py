@@ -44,7 +44,7 @@ class _Config(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int), ("seq_len", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("segment_len", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("tau", ctypes.c_float),
-                ("query_perm", ctypes.c_int)]
+                ("query_perm", ctypes.c_int), ("shared_key_order", ctypes.c_int)]
 
 
 class _Indices(ctypes.Structure):
@@ -74,6 +74,7 @@ class Config:
     block_size: int
     tau: float
     query_perm: int = 1
+    shared_key_order: int = 0
 
     @classmethod
     def of(cls, obj, **overrides) -> "Config":
@@ -83,7 +84,8 @@ class Config:
 
     def _c(self) -> _Config:
         return _Config(self.batch, self.n_q_heads, self.n_kv_heads, self.seq_len, self.head_dim,
-                       self.segment_len, self.block_size, float(self.tau), self.query_perm)
+                       self.segment_len, self.block_size, float(self.tau), self.query_perm,
+                       self.shared_key_order)
 
     @property
     def n_blocks(self) -> int:

@@ -200,7 +200,7 @@ template <int D>
 __global__ void __launch_bounds__(128)
     k_kpass(const uint16_t *__restrict__ k, const float *__restrict__ qbar,
             float *__restrict__ kappa, float *__restrict__ kchunk, int N, int B, int Hq, int Hkv,
-            int G) {
+            int G, int shared_order) {
   constexpr int RS = D * 2 + 16;  // staged row stride in bytes
   extern __shared__ float4 sm4[];
   float *qb = reinterpret_cast<float *>(sm4);                                     // [G][D]
@@ -217,13 +217,24 @@ __global__ void __launch_bounds__(128)
   for (int x = threadIdx.x; x < G * D; x += blockDim.x) qb[x] = qbar[qh0 * D + x];
   cp_async_wait_all();
   __syncthreads();
+  if (shared_order) {
+    // One ordering per KV head: the group's pooled query (the G mean queries added in head
+    // order, divided by G) replaces the first head's; column t is read and written by thread t.
+    for (int t = threadIdx.x; t < D; t += blockDim.x) {
+      float acc = qb[t];
+      for (int hi = 1; hi < G; ++hi) acc = __fadd_rn(acc, qb[hi * D + t]);
+      qb[t] = __fdiv_rn(acc, (float)G);
+    }
+    __syncthreads();
+  }
+  const int n_heads = shared_order ? 1 : G;
   const int j = chunk * B + r;
   if (r < B) {
     // Up to four query heads at a time: their chains interleave (each still runs over t in
     // order) and the row is read once per group of heads.
     const uint4 *row = reinterpret_cast<const uint4 *>(rows + r * RS);
-    for (int h0 = 0; h0 < G; h0 += 4) {
-      const int nh = min(4, G - h0);
+    for (int h0 = 0; h0 < n_heads; h0 += 4) {
+      const int nh = min(4, n_heads - h0);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 2
       for (int c = 0; c < D / 8; ++c) {
@@ -251,6 +262,8 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int hh = 0; hh < 4; ++hh)
         if (hh < nh) kappa[(qh0 + h0 + hh) * N + j] = acc[hh];
+      if (shared_order)  // the group's score, in every query head's row
+        for (int hi = 1; hi < G; ++hi) kappa[(qh0 + hi) * N + j] = acc[0];
     }
   }
   if (r < D / 2) {
@@ -454,6 +467,17 @@ __global__ void __launch_bounds__(512)
   (void)n;
 }
 
+// Copies the first row of each group of G rows (row_len int32, a multiple of 4, 16-byte aligned
+// rows) to the group's other G - 1 rows. Grid: (any, groups).
+__global__ void k_replicate_group_rows(int32_t *__restrict__ a, long long row_len, int G) {
+  int32_t *grp = a + (long long)blockIdx.y * G * row_len;
+  for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < row_len / 4;
+       x += (long long)gridDim.x * blockDim.x) {
+    const int4 v = reinterpret_cast<const int4 *>(grp)[x];
+    for (int hi = 1; hi < G; ++hi) reinterpret_cast<int4 *>(grp + hi * row_len)[x] = v;
+  }
+}
+
 // Multi-CTA stable radix sort of runs of run_len elements (one run per query head), tiles of
 // kRadixTile elements: per pass a digit count per tile, then a scatter per tile that derives its
 // offsets from the run's counts.
@@ -464,16 +488,18 @@ __device__ __forceinline__ int radix_elem(int r) {
   return (threadIdx.x / 32) * 32 * kRadixR + r * 32 + threadIdx.x % 32;
 }
 
-// Keys and values of pass 0 come from the scores: key = desc_key(score), value = the index in
-// the run (idx0 = index of the tile's first element).
+// Keys and values of pass 0 come from the scores (read at score_base): key = desc_key(score),
+// value = the index in the run (idx0 = index of the tile's first element); later passes read the
+// keys and values at base.
 __device__ __forceinline__ void radix_load(const float *score, const uint32_t *keys,
-                                           const uint32_t *vals, long long base, int idx0, int n,
+                                           const uint32_t *vals, long long score_base,
+                                           long long base, int idx0, int n,
                                            uint32_t (&key)[kRadixR], uint32_t (&val)[kRadixR]) {
 #pragma unroll
   for (int r = 0; r < kRadixR; ++r) {
     const int e = radix_elem(r);
     if (e < n) {
-      key[r] = score ? desc_key(__ldg(score + base + e)) : __ldg(keys + base + e);
+      key[r] = score ? desc_key(__ldg(score + score_base + e)) : __ldg(keys + base + e);
       val[r] = score ? (uint32_t)(idx0 + e) : __ldg(vals + base + e);
     } else {
       key[r] = 0xffffffffu;
@@ -485,11 +511,12 @@ __device__ __forceinline__ void radix_load(const float *score, const uint32_t *k
 // counts[(run·256 + digit)·tiles + tile] for one pass.
 __global__ void __launch_bounds__(kRadixThreads)
     k_radix_count(const float *__restrict__ score, const uint32_t *__restrict__ keys,
-                  long long run_len, int tiles, int shift, int *__restrict__ counts) {
+                  long long run_len, long long score_stride, int tiles, int shift,
+                  int *__restrict__ counts) {
   __shared__ int h[256];
   const long long run = blockIdx.x / tiles;
   const int tile = blockIdx.x % tiles;
-  const long long base = run * run_len + (long long)tile * kRadixTile;
+  const long long base = (score ? run * score_stride : run * run_len) + (long long)tile * kRadixTile;
   const int n = (int)min((long long)kRadixTile, run_len - (long long)tile * kRadixTile);
   for (int d = threadIdx.x; d < 256; d += blockDim.x) h[d] = 0;
   __syncthreads();
@@ -561,7 +588,8 @@ __global__ void __launch_bounds__(kRadixThreads)
     k_radix_scatter(const float *__restrict__ score, const uint32_t *__restrict__ keys_in,
                     const uint32_t *__restrict__ vals_in, uint32_t *__restrict__ keys_out,
                     uint32_t *__restrict__ vals_out, int32_t *__restrict__ perm_out,
-                    long long run_len, long long head_len, int tiles, int shift,
+                    long long run_len, long long head_len, long long score_stride,
+                    long long perm_stride, int tiles, int shift,
                     const int *__restrict__ offsets) {
   extern __shared__ int sm_r[];
   uint32_t *skey = reinterpret_cast<uint32_t *>(sm_r);   // [tile]
@@ -578,7 +606,8 @@ __global__ void __launch_bounds__(kRadixThreads)
   __syncthreads();
   uint32_t key[kRadixR], val[kRadixR], dig[kRadixR];
   int dest[kRadixR];
-  radix_load(score, keys_in, vals_in, base, tile * kRadixTile, n, key, val);
+  radix_load(score, keys_in, vals_in, run * score_stride + (long long)tile * kRadixTile, base,
+             tile * kRadixTile, n, key, val);
 #pragma unroll
   for (int r = 0; r < kRadixR; ++r) dig[r] = (key[r] >> shift) & 255u;
   radix_ranks<kRadixR, kRadixThreads / 32>(dig, dest, hist, dbase);
@@ -592,12 +621,12 @@ __global__ void __launch_bounds__(kRadixThreads)
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const uint32_t k = skey[i];
     const int d = (int)((k >> shift) & 255u);
-    const long long o = out0 + goff[d] + (i - dbase[d]);
+    const long long at = goff[d] + (i - dbase[d]);
     if (perm_out)  // positions within the head: a run's first element sits at run·run_len mod N
-      perm_out[o] = (int32_t)((run * run_len) % head_len + sval[i]);
+      perm_out[run * perm_stride + at] = (int32_t)((run * run_len) % head_len + sval[i]);
     else {
-      keys_out[o] = k;
-      vals_out[o] = sval[i];
+      keys_out[out0 + at] = k;
+      vals_out[out0 + at] = sval[i];
     }
   }
 }
@@ -1048,11 +1077,15 @@ inline unsigned blocks_for(long long n, int per) { return (unsigned)((n + per - 
 
 // Stable radix sort of runs of run_len scores each (descending, ties to the lower index), the
 // permutation written to perm_out as positions within a head of head_len elements (a run of
-// segment length S starts at its segment's first position). Keys and values ping-pong between
-// (k0, v0) and (k1, v1).
+// segment length S starts at its segment's first position). Run r's scores start at
+// score + r·score_stride and its permutation at perm_out + r·perm_stride (both default to
+// run_len). Keys and values ping-pong between (k0, v0) and (k1, v1).
 cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint32_t *k1,
                             uint32_t *v1, int *counts, long long total, long long run_len,
-                            long long head_len, int32_t *perm_out, cudaStream_t st) {
+                            long long head_len, int32_t *perm_out, cudaStream_t st,
+                            long long score_stride = 0, long long perm_stride = 0) {
+  if (score_stride <= 0) score_stride = run_len;
+  if (perm_stride <= 0) perm_stride = run_len;
   const int tiles = (int)((run_len + kRadixTile - 1) / kRadixTile);
   const long long runs = total / run_len;
   const unsigned grid = (unsigned)(runs * tiles);
@@ -1064,13 +1097,14 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
   uint32_t *kout = k0, *vout = v0;
   for (int pass = 0; pass < 4; ++pass) {
     const float *sc = pass == 0 ? score : nullptr;
-    k_radix_count<<<grid, kRadixThreads, 0, st>>>(sc, kin, run_len, tiles, 8 * pass, counts);
+    k_radix_count<<<grid, kRadixThreads, 0, st>>>(sc, kin, run_len, score_stride, tiles,
+                                                  8 * pass, counts);
     note_launch();
     k_radix_offsets<<<(unsigned)runs, 256, 0, st>>>(counts, tiles);
     note_launch();
     k_radix_scatter<<<grid, kRadixThreads, smem, st>>>(sc, kin, vin, kout, vout,
                                                        pass == 3 ? perm_out : nullptr, run_len,
-                                                       head_len,
+                                                       head_len, score_stride, perm_stride,
                                                        tiles, 8 * pass, counts);
     note_launch();
     kin = kout;
@@ -1144,16 +1178,28 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   if ((e = cudaFuncSetAttribute(k_kpass<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kpass_smem)) != cudaSuccess)
     return e;
+  const int shared_order = cfg.shared_key_order && d.G > 1 ? 1 : 0;
   k_kpass<D><<<dim3((unsigned)d.nB, (unsigned)bhkv), 128, kpass_smem, st>>>(
-      k, qbar, kappa, kchunk, d.N, d.B, d.Hq, d.Hkv, d.G);
+      k, qbar, kappa, kchunk, d.N, d.B, d.Hq, d.Hkv, d.G, shared_order);
   note_launch();
   k_pool_finish<D><<<dim3(D / 32, (unsigned)bhkv), 256, fin_smem, st>>>(kchunk, kbar_all, d.nB,
                                                                          (float)d.N);
   note_launch();
   // Step 2a: global key/value ordering.
-  if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, nq, d.N, d.N, out.perm_k, st)) !=
-      cudaSuccess)
+  if (shared_order) {
+    // One ordering per KV head (sorted from the group's first query-head rows), copied to the
+    // other rows of the group.
+    const long long gstride = (long long)d.G * d.N;
+    if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, bhkv * d.N, d.N, d.N, out.perm_k,
+                             st, gstride, gstride)) != cudaSuccess)
+      return e;
+    const unsigned rep_x = std::min(blocks_for(d.N / 4, 256), 64u);
+    k_replicate_group_rows<<<dim3(rep_x, (unsigned)bhkv), 256, 0, st>>>(out.perm_k, d.N, d.G);
+    note_launch();
+  } else if ((e = radix_sort_runs(kappa, rk0, rv0, rk1, rv1, rcount, nq, d.N, d.N, out.perm_k,
+                                  st)) != cudaSuccess) {
     return e;
+  }
   // Key side of step 2c (block means K̄ and visibility counts): they depend only on perm_k and
   // run on a side stream next to the query-side kernels, joined before the block scores.
   const long long nblk = bhq * d.nB;

@@ -102,7 +102,9 @@ def test_exp64_bit_exact_with_oracle():
 @pytest.mark.parametrize("w", [
     W_TINY, W_TINY.replace(tau=0.0), W_TINY.replace(tau=0.07), W_TINY.replace(tau=0.2),
     W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E, W_F, W_G,
-], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
+    W_A.replace(shared_key_order=1), W_B.replace(shared_key_order=1),
+    W_E.replace(shared_key_order=1),
+], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}-sk{w.shared_key_order}")
 def test_indices_and_intermediates_bit_exact(w):
     q, k, _ = inputs(w)
     ref = oracle.build_indices(oracle.config(w), q, k, debug=True)
