@@ -428,7 +428,8 @@ def run_sweep(args):
         permuted_pass = int((idx.local_tiles[busy].long() + idx.sel_cnt[busy].long()).sum().item())
         tile_flops = 4.0 * w.block_size ** 2 * w.head_dim
         row = {"workload": w.name, "tau": w.tau, "segment_len": w.segment_len,
-               "query_perm": w.query_perm, "stripe_frac": w.stripe_frac,
+               "query_perm": w.query_perm, "shared_key_order": w.shared_key_order,
+               "stripe_frac": w.stripe_frac,
                "pair_sparsity": stats.pair_sparsity,
                "tile_density": stats.executed_tiles * w.block_size ** 2 / stats.causal_pairs,
                "selected_tiles": stats.selected_tiles,
@@ -459,6 +460,9 @@ def run_sweep(args):
     configs += [qwen.replace(tau=t) for t in (0.001, 0.005, 0.01, 0.02)]
     configs += [qwen.replace(segment_len=s) for s in (1024, 4096)]
     configs += [qwen.replace(query_perm=0)]
+    # Labelled variant beside the specified configurations: one key ordering per KV head.
+    configs += [gen.workload("llama-128k").replace(shared_key_order=1),
+                qwen.replace(tau=0.001, shared_key_order=1)]
     for w in configs:
         print(json.dumps({"config": measure(w)}), flush=True)
     stack = [measure(gen.layer_workload(l), reps=2, dense=(l % 8 == 7)) for l in range(32)]
