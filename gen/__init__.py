@@ -52,6 +52,7 @@ class Workload:
     diag: float = 0.5
     query_perm: int = 1
     shared_key_order: int = 0
+    int4_centroids: int = 0
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

@@ -47,7 +47,8 @@ class Config(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int), ("seq_len", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("segment_len", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("tau", ctypes.c_float),
-                ("query_perm", ctypes.c_int), ("shared_key_order", ctypes.c_int)]
+                ("query_perm", ctypes.c_int), ("shared_key_order", ctypes.c_int),
+                ("int4_centroids", ctypes.c_int)]
 
 
 class _Debug(ctypes.Structure):

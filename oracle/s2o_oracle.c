@@ -37,6 +37,7 @@ typedef struct {
   float tau;
   int query_perm; /* 1: segment-local query ordering (default); 0: identity (Q-perm ablation) */
   int shared_key_order; /* 0: one key ordering per query head (default); 1: per KV head */
+  int int4_centroids;   /* 0: fp32 block scores (default); 1: 4-bit key centroids, integer score */
 } oracle_config;
 
 /* Optional intermediate values, all per (batch, query head) unless noted; any pointer may be
@@ -248,9 +249,59 @@ static int build_head(const oracle_config *cfg, const uint16_t *q_all, const uin
     list_mean(K, d, perm_k + (size_t)b * B, B, B, Kbar + (size_t)b * d);
   }
   const float sigma = oracle_score_scale(d);
-  for (int b = 0; b < nB; ++b)
-    for (int c = 0; c < nB; ++c)
-      r[(size_t)b * nB + c] = dot_f32(Qbar + (size_t)b * d, Kbar + (size_t)c * d, d) * sigma;
+  if (!cfg->int4_centroids) {
+    for (int b = 0; b < nB; ++b)
+      for (int c = 0; c < nB; ++c)
+        r[(size_t)b * nB + c] = dot_f32(Qbar + (size_t)b * d, Kbar + (size_t)c * d, d) * sigma;
+  } else {
+    /* 4-bit key centroids per channel (asymmetric), 8-bit query centroids scaled by the key
+     * channel steps (symmetric per block), r from the exact integer product. */
+    float *step = malloc((size_t)d * sizeof(float));
+    float *lo = malloc((size_t)d * sizeof(float));
+    int *qk = malloc((size_t)nB * d * sizeof(int));
+    int *qa = malloc((size_t)d * sizeof(int));
+    float *a = malloc((size_t)d * sizeof(float));
+    if (!step || !lo || !qk || !qa || !a) return ORACLE_ERR_NOMEM;
+    for (int t = 0; t < d; ++t) {
+      float mn = Kbar[t], mx = Kbar[t];
+      for (int c = 1; c < nB; ++c) {
+        const float x = Kbar[(size_t)c * d + t];
+        if (x < mn) mn = x;
+        if (x > mx) mx = x;
+      }
+      float st = (mx - mn) / 15.0f;
+      if (st == 0.0f) st = 1.0f;
+      lo[t] = mn;
+      step[t] = st;
+      for (int c = 0; c < nB; ++c) {
+        float code = rintf((Kbar[(size_t)c * d + t] - mn) / st);
+        if (code < 0.0f) code = 0.0f;
+        if (code > 15.0f) code = 15.0f;
+        qk[(size_t)c * d + t] = (int)code;
+      }
+    }
+    for (int b = 0; b < nB; ++b) {
+      float m = 0.0f;
+      for (int t = 0; t < d; ++t) {
+        a[t] = Qbar[(size_t)b * d + t] * step[t];
+        if (fabsf(a[t]) > m) m = fabsf(a[t]);
+      }
+      float sq = m / 127.0f;
+      if (sq == 0.0f) sq = 1.0f;
+      for (int t = 0; t < d; ++t) {
+        float code = rintf(a[t] / sq);
+        if (code < -127.0f) code = -127.0f;
+        if (code > 127.0f) code = 127.0f;
+        qa[t] = (int)code;
+      }
+      for (int c = 0; c < nB; ++c) {
+        long long acc = 0;
+        for (int t = 0; t < d; ++t) acc += (long long)qa[t] * qk[(size_t)c * d + t];
+        r[(size_t)b * nB + c] = ((float)acc * sq) * sigma;
+      }
+    }
+    free(step); free(lo); free(qk); free(qa); free(a);
+  }
 
   /* Visibility counts n[s][c] = #keys of key block c before the start of segment s. */
   for (int s = 0; s < nSeg; ++s)

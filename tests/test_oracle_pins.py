@@ -368,3 +368,38 @@ def test_shared_key_order_variant():
     c = oracle.build_indices(oracle.config(w1), q1, k1)
     for name in ("perm_q", "perm_k", "sel_cnt", "sel_blk", "local_tiles"):
         np.testing.assert_array_equal(a[name], c[name], err_msg=name)
+
+
+def test_int4_centroid_variant():
+    """The labelled variant with 4-bit key centroids: its block scores against the exact float64
+    centroid product without the per-block constant (σ·Q̄_b·(K̄_c − lo)), within the quantisation
+    error bound (half a key step per channel, half a query step per code); everything before the
+    scores is the default's, and at τ = 0 both select every candidate."""
+    w = SMALL_GQA
+    q, k, _ = gen.make_inputs(w)
+    v = oracle.build_indices(oracle.config(w, int4_centroids=1), q, k, debug=True)
+    base = oracle.build_indices(oracle.config(w), q, k, debug=True)
+    for name in ("perm_q", "perm_k", "local_tiles"):
+        np.testing.assert_array_equal(v[name], base[name], err_msg=name)
+    np.testing.assert_array_equal(v["Qbar"], base["Qbar"])
+    np.testing.assert_array_equal(v["Kbar"], base["Kbar"])
+    d = w.head_dim
+    sigma = 1.0 / math.sqrt(d)
+    for b in range(w.batch):
+        for h in range(w.n_q_heads):
+            Qb = v["Qbar"][b, h].astype(np.float64)
+            Kb = v["Kbar"][b, h].astype(np.float64)
+            lo = Kb.min(0)
+            step = (Kb.max(0) - lo) / 15.0
+            step[step == 0] = 1.0
+            exact = sigma * (Qb @ (Kb - lo).T)
+            sq = np.abs(Qb * step).max(1) / 127.0
+            bound = sigma * (np.abs(Qb) @ (step / 2.0) + 15.0 * d * sq / 2.0)
+            err = np.abs(v["r"][b, h].astype(np.float64) - exact)
+            assert (err <= bound[:, None] * 1.01 + 1e-6).all(), float((err - bound[:, None]).max())
+            # The bound is not vacuous: the scores carry the centroid signal.
+            assert np.corrcoef(v["r"][b, h].ravel(), exact.ravel())[0, 1] > 0.9
+    v0 = oracle.build_indices(oracle.config(w, tau=0.0, int4_centroids=1), q, k)
+    b0 = oracle.build_indices(oracle.config(w, tau=0.0), q, k)
+    np.testing.assert_array_equal(v0["sel_cnt"], b0["sel_cnt"])
+    np.testing.assert_array_equal(np.sort(v0["sel_blk"], axis=-1), np.sort(b0["sel_blk"], axis=-1))
