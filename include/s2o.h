@@ -50,12 +50,15 @@ typedef enum {
  * identity (the "Q perm" ablation of [S2O, Key points]). `shared_key_order` = 0 (the default)
  * builds one key ordering per query head; 1 builds one per KV head, ranked by the group's pooled
  * query, and writes it to the perm_k row of each of the group's query heads (a labelled variant:
- * the pages say "for each head" without saying which kind of head). */
+ * the pages say "for each head" without saying which kind of head). `int4_centroids` = 1 scores
+ * blocks with 4-bit key centroids and an exact integer product (a labelled variant after
+ * [AB-Sparse, INT4 centroids]; 0, the default, is the fp32 centroid product). */
 typedef struct {
   int batch, n_q_heads, n_kv_heads, seq_len, head_dim, segment_len, block_size;
   float tau;
   int query_perm;
   int shared_key_order;
+  int int4_centroids;
 } s2o_config;
 
 /* Caller-owned index arrays (device, int32). nB = N / B.

@@ -44,7 +44,8 @@ class _Config(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int), ("seq_len", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("segment_len", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("tau", ctypes.c_float),
-                ("query_perm", ctypes.c_int), ("shared_key_order", ctypes.c_int)]
+                ("query_perm", ctypes.c_int), ("shared_key_order", ctypes.c_int),
+                ("int4_centroids", ctypes.c_int)]
 
 
 class _Indices(ctypes.Structure):
@@ -75,6 +76,7 @@ class Config:
     tau: float
     query_perm: int = 1
     shared_key_order: int = 0
+    int4_centroids: int = 0
 
     @classmethod
     def of(cls, obj, **overrides) -> "Config":
@@ -85,7 +87,7 @@ class Config:
     def _c(self) -> _Config:
         return _Config(self.batch, self.n_q_heads, self.n_kv_heads, self.seq_len, self.head_dim,
                        self.segment_len, self.block_size, float(self.tau), self.query_perm,
-                       self.shared_key_order)
+                       self.shared_key_order, self.int4_centroids)
 
     @property
     def n_blocks(self) -> int:

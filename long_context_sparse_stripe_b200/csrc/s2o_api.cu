@@ -25,6 +25,7 @@ s2o_status check_config(const s2o_config *c) {
     return S2O_ERR_INVALID_ARGUMENT;
   if (c->query_perm != 0 && c->query_perm != 1) return S2O_ERR_INVALID_ARGUMENT;
   if (c->shared_key_order != 0 && c->shared_key_order != 1) return S2O_ERR_INVALID_ARGUMENT;
+  if (c->int4_centroids != 0 && c->int4_centroids != 1) return S2O_ERR_INVALID_ARGUMENT;
   if (c->head_dim != 64 && c->head_dim != 128) return S2O_ERR_UNSUPPORTED;
   if (c->block_size != 64 && c->block_size != 128) return S2O_ERR_UNSUPPORTED;
   if (c->n_q_heads % c->n_kv_heads) return S2O_ERR_UNSUPPORTED;
@@ -43,6 +44,7 @@ s2o_status check_dense_config(const s2o_config *c) {
   x.tau = 0.f;
   x.query_perm = 1;
   x.shared_key_order = 0;
+  x.int4_centroids = 0;
   return check_config(&x);
 }
 

@@ -800,6 +800,139 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
+// ------------------------------------------------------------------ 4-bit key centroids (variant)
+
+// Key-centroid codes per query head and channel t: lo = min_c K̄, step = (max − lo)/15 (1 if 0),
+// code = clamp(rint((K̄ − lo)/step), 0, 15). One CTA per (query head, 32 channels): lane = channel,
+// the 32 warps split the blocks for the min/max (exact in any order) and write the codes.
+template <int D>
+__global__ void __launch_bounds__(1024)
+    k_kbar_codes(const float *__restrict__ Kbar, int8_t *__restrict__ kcode,
+                 float *__restrict__ kstep, int nB) {
+  __shared__ float smin[32][33], smax[32][33];
+  const long long qh = blockIdx.y;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const int t = blockIdx.x * 32 + lane;
+  const float *kb = Kbar + (size_t)qh * nB * D + t;
+  float mn = kb[0], mx = kb[0];
+  for (int c = warp; c < nB; c += 32) {
+    const float x = kb[(size_t)c * D];
+    mn = x < mn ? x : mn;
+    mx = x > mx ? x : mx;
+  }
+  smin[warp][lane] = mn;
+  smax[warp][lane] = mx;
+  __syncthreads();
+  mn = smin[0][lane];
+  mx = smax[0][lane];
+  for (int w = 1; w < 32; ++w) {
+    mn = smin[w][lane] < mn ? smin[w][lane] : mn;
+    mx = smax[w][lane] > mx ? smax[w][lane] : mx;
+  }
+  float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  if (step == 0.0f) step = 1.0f;
+  if (warp == 0) kstep[qh * D + t] = step;
+  for (int c = warp; c < nB; c += 32) {
+    const int code = __float2int_rn(__fdiv_rn(__fsub_rn(kb[(size_t)c * D], mn), step));
+    kcode[((size_t)qh * nB + c) * D + t] = (int8_t)min(max(code, 0), 15);
+  }
+}
+
+// Query-centroid codes per query block: a_t = Q̄_t × step_t, sq = max_t |a_t| / 127 (1 if 0),
+// code = clamp(rint(a_t / sq), −127, 127). One warp per block.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_qbar_codes(const float *__restrict__ Qbar, const float *__restrict__ kstep,
+                 int8_t *__restrict__ qcode, float *__restrict__ qstep, int nB,
+                 long long n_blocks) {
+  const long long blk = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (blk >= n_blocks) return;
+  const long long qh = blk / nB;
+  float a[D / 32], m = 0.0f;
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {
+    const int t = lane + 32 * k;
+    a[k] = __fmul_rn(Qbar[(size_t)blk * D + t], kstep[qh * D + t]);
+    m = fmaxf(m, fabsf(a[k]));
+  }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sq = __fdiv_rn(m, 127.0f);
+  if (sq == 0.0f) sq = 1.0f;
+  if (lane == 0) qstep[blk] = sq;
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {
+    const int code = __float2int_rn(__fdiv_rn(a[k], sq));
+    qcode[(size_t)blk * D + lane + 32 * k] = (int8_t)min(max(code, -127), 127);
+  }
+}
+
+// r[qh][b][c] = fp32(fp32(Σ_t qa_{b,t}·qK_{c,t}) × sq_b) × σ_d, the sum an exact integer (four
+// codes per dp4a). A 128×128 tile per CTA, 8×8 outputs per thread; the code words are staged
+// word-major (word w of every row of the tile contiguous) so that a thread reads its 8 rows' or
+// columns' words with two 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_block_scores_i8(const int8_t *__restrict__ qcode, const int8_t *__restrict__ kcode,
+                      const float *__restrict__ qstep, float *__restrict__ r, int nB,
+                      float sigma) {
+  constexpr int W = D / 4;  // 32-bit words per row
+  __shared__ __align__(16) int As[W][128];
+  __shared__ __align__(16) int Bs[W][128];
+  const long long qh = blockIdx.z;
+  const int b0 = blockIdx.y * 128, c0 = blockIdx.x * 128;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  const int *qa = reinterpret_cast<const int *>(qcode + (size_t)qh * nB * D);
+  const int *qk = reinterpret_cast<const int *>(kcode + (size_t)qh * nB * D);
+  for (int x = threadIdx.x; x < 128 * (W / 4); x += blockDim.x) {
+    const int row = x / (W / 4), w0 = (x % (W / 4)) * 4;
+    const int4 va = b0 + row < nB
+                        ? *reinterpret_cast<const int4 *>(qa + (size_t)(b0 + row) * W + w0)
+                        : make_int4(0, 0, 0, 0);
+    const int4 vb = c0 + row < nB
+                        ? *reinterpret_cast<const int4 *>(qk + (size_t)(c0 + row) * W + w0)
+                        : make_int4(0, 0, 0, 0);
+    As[w0][row] = va.x;
+    As[w0 + 1][row] = va.y;
+    As[w0 + 2][row] = va.z;
+    As[w0 + 3][row] = va.w;
+    Bs[w0][row] = vb.x;
+    Bs[w0 + 1][row] = vb.y;
+    Bs[w0 + 2][row] = vb.z;
+    Bs[w0 + 3][row] = vb.w;
+  }
+  __syncthreads();
+  int acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0;
+#pragma unroll 4
+  for (int w = 0; w < W; ++w) {
+    const int4 a0 = *reinterpret_cast<const int4 *>(&As[w][tr * 8]);
+    const int4 a1 = *reinterpret_cast<const int4 *>(&As[w][tr * 8 + 4]);
+    const int4 v0 = *reinterpret_cast<const int4 *>(&Bs[w][tc * 8]);
+    const int4 v1 = *reinterpret_cast<const int4 *>(&Bs[w][tc * 8 + 4]);
+    const int a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const int v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = __dp4a(a[i], v[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = b0 + tr * 8 + i;
+    if (b >= nB) continue;
+    const float sq = qstep[(size_t)qh * nB + b];
+    float *dst = r + ((size_t)qh * nB + b) * nB + c0 + tc * 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (c0 + tc * 8 + j < nB)
+        dst[j] = __fmul_rn(__fmul_rn(__int2float_rn(acc[i][j]), sq), sigma);
+  }
+}
+
 // ------------------------------------------------------------------ scheduling (step 4 order)
 
 __device__ __forceinline__ bool goes_before(double pa, int ca, double pb, int cb) {
@@ -1265,8 +1398,24 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   if ((e = join.now()) != cudaSuccess) return e;
   const float sigma = D == 64 ? 0x1p-3f : 0x1.6a09e6p-4f;  // nearest fp32 to 1/sqrt(D)
   const unsigned tiles = (unsigned)((d.nB + 127) / 128);
-  k_block_scores<D><<<dim3(tiles, tiles, (unsigned)bhq), 256, 0, st>>>(Qbar, Kbar, r, d.nB, sigma);
-  note_launch();
+  if (cfg.int4_centroids) {
+    // Codes in the radix key buffer (free once the orderings are built).
+    int8_t *kcode = reinterpret_cast<int8_t *>(rk0);
+    int8_t *qcode = kcode + (size_t)bhq * d.nB * D;
+    float *kstep = reinterpret_cast<float *>(qcode + (size_t)bhq * d.nB * D);
+    float *qstep = kstep + (size_t)bhq * D;
+    k_kbar_codes<D><<<dim3(D / 32, (unsigned)bhq), 1024, 0, st>>>(Kbar, kcode, kstep, d.nB);
+    note_launch();
+    k_qbar_codes<D><<<blocks_for(nblk, 8), 256, 0, st>>>(Qbar, kstep, qcode, qstep, d.nB, nblk);
+    note_launch();
+    k_block_scores_i8<D><<<dim3(tiles, tiles, (unsigned)bhq), 256, 0, st>>>(qcode, kcode, qstep,
+                                                                             r, d.nB, sigma);
+    note_launch();
+  } else {
+    k_block_scores<D><<<dim3(tiles, tiles, (unsigned)bhq), 256, 0, st>>>(Qbar, Kbar, r, d.nB,
+                                                                         sigma);
+    note_launch();
+  }
   // Scheduling. The selected list of a query block holds at most floor(1/τ) + 1 entries.
   int cap = d.nB;
   if (cfg.tau > 0.f) {

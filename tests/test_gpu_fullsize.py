@@ -112,12 +112,14 @@ def test_dense_kernel_full_size_sampled_rows():
     assert err.mean() <= MEAN_ABS, f"mean abs error {err.mean():.3g}"
 
 
-@pytest.mark.parametrize("variant", ["tau0.001", "S1024", "S4096", "qperm-off", "shared-keys"])
+@pytest.mark.parametrize("variant", ["tau0.001", "S1024", "S4096", "qperm-off", "shared-keys",
+                                     "int4-centroids"])
 def test_qwen_128k_ablation(variant):
     w = gen.workload("qwen-128k")
     w = {"tau0.001": w.replace(tau=0.001), "S1024": w.replace(segment_len=1024),
          "S4096": w.replace(segment_len=4096), "qperm-off": w.replace(query_perm=0),
-         "shared-keys": w.replace(shared_key_order=1)}[variant]
+         "shared-keys": w.replace(shared_key_order=1),
+         "int4-centroids": w.replace(int4_centroids=1)}[variant]
     selected = check_layer(w, groups=(3,))
     if variant == "tau0.001":
         assert selected > 0  # the permuted pass does real work at this threshold

@@ -104,7 +104,10 @@ def test_exp64_bit_exact_with_oracle():
     W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E, W_F, W_G,
     W_A.replace(shared_key_order=1), W_B.replace(shared_key_order=1),
     W_E.replace(shared_key_order=1),
-], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}-sk{w.shared_key_order}")
+    W_TINY.replace(int4_centroids=1), W_A.replace(int4_centroids=1), W_C.replace(int4_centroids=1),
+    W_F.replace(int4_centroids=1), W_B.replace(shared_key_order=1, int4_centroids=1),
+], ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}-sk{w.shared_key_order}"
+                 f"-i4{w.int4_centroids}")
 def test_indices_and_intermediates_bit_exact(w):
     q, k, _ = inputs(w)
     ref = oracle.build_indices(oracle.config(w), q, k, debug=True)
