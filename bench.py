@@ -429,6 +429,7 @@ def run_sweep(args):
         tile_flops = 4.0 * w.block_size ** 2 * w.head_dim
         row = {"workload": w.name, "tau": w.tau, "segment_len": w.segment_len,
                "query_perm": w.query_perm, "shared_key_order": w.shared_key_order,
+               "int4_centroids": w.int4_centroids,
                "stripe_frac": w.stripe_frac,
                "pair_sparsity": stats.pair_sparsity,
                "tile_density": stats.executed_tiles * w.block_size ** 2 / stats.causal_pairs,
@@ -463,6 +464,9 @@ def run_sweep(args):
     # Labelled variant beside the specified configurations: one key ordering per KV head.
     configs += [gen.workload("llama-128k").replace(shared_key_order=1),
                 qwen.replace(tau=0.001, shared_key_order=1)]
+    # Labelled variant: 4-bit key centroids for the block scores (alone and with the above).
+    configs += [gen.workload("llama-128k").replace(int4_centroids=1),
+                gen.workload("llama-128k").replace(shared_key_order=1, int4_centroids=1)]
     for w in configs:
         print(json.dumps({"config": measure(w)}), flush=True)
     stack = [measure(gen.layer_workload(l), reps=2, dense=(l % 8 == 7)) for l in range(32)]
