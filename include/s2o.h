@@ -64,7 +64,9 @@ typedef struct {
 /* Caller-owned index arrays (device, int32). nB = N / B.
  *  perm_q      [batch, Hq, N]      original query index at each permuted slot; slots
  *                                  [sS, (s+1)S) hold a permutation of segment s.
- *  perm_k      [batch, Hq, N]      original key index at each rank (one ordering per query head).
+ *  perm_k      [batch, Hq, N]      original key index at each rank (one ordering per query head;
+ *                                  with shared_key_order, each head of a KV group holds the
+ *                                  group's ordering).
  *  sel_cnt     [batch, Hq, nB]     number of selected permuted key blocks of each query block.
  *  sel_blk     [batch, Hq, nB, nB] selected key-block ids (blocks of perm_k), most important
  *                                  first; entries at and after sel_cnt are not written.
@@ -104,7 +106,10 @@ s2o_status s2o_index_sizes(const s2o_config *cfg, size_t counts[5]);
 /* Steps 1–2 of the method ([S2O, Summary ¶2]: stripe-level mean pooling, the global key/value
  * ordering, the segment-local query ordering, block scores and the early stop at tau) for every
  * (batch, query head): writes the index arrays of `out`. Bit-exact with the definition: same
- * inputs give the same indices on every run. q, k: device bf16 as above. */
+ * inputs give the same indices on every run. q, k: device bf16 as above. The key-side kernels
+ * run on a second stream of the calling thread (created on first use, kept for the thread's
+ * lifetime), forked from and joined back to `stream` with events, so the call stays ordered on
+ * `stream` and can be captured in a CUDA graph. */
 s2o_status s2o_build_indices(const s2o_config *cfg, const void *q, const void *k,
                              const s2o_indices *out, void *ws, size_t ws_bytes,
                              s2o_stream stream);
