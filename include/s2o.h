@@ -109,7 +109,7 @@ s2o_status s2o_index_sizes(const s2o_config *cfg, size_t counts[5]);
  * inputs give the same indices on every run. q, k: device bf16 as above. The key-side kernels
  * run on a second stream of the calling thread (created on first use, kept for the thread's
  * lifetime), forked from and joined back to `stream` with events, so the call stays ordered on
- * `stream` and can be captured in a CUDA graph. */
+ * `stream`. */
 s2o_status s2o_build_indices(const s2o_config *cfg, const void *q, const void *k,
                              const s2o_indices *out, void *ws, size_t ws_bytes,
                              s2o_stream stream);

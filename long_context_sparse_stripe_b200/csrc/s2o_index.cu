@@ -1249,8 +1249,8 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
 }
 
 // A second stream of the calling thread on the current device, for kernels that are independent
-// of the caller's stream between a fork and a join (both by events, so the pair is also valid
-// inside stream capture). Created on first use, kept for the thread's lifetime.
+// of the caller's stream between a fork and a join (both by events). Created on first use, kept
+// for the thread's lifetime.
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
