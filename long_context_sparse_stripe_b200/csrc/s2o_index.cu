@@ -939,149 +939,187 @@ __device__ __forceinline__ bool goes_before(double pa, int ca, double pb, int cb
   return pa > pb || (pa == pb && ca < cb);
 }
 
-// One warp per query block: local tile count, normalised block scores p over the candidate
-// blocks, selection p >= τ, and the list sorted by (p descending, block ascending).
-// Shared memory per warp: the weights (nB doubles, one pad slot per 32 so that a lane walking its
-// own chunk hits distinct banks) and the selected list (cap2 entries; cap2 bounds the list
-// length: at most floor(1/τ) + 1 blocks can reach p >= τ since the p sum to one).
+// a[i] for a register array and a run-time index, by a tree of selects (no local memory).
+__device__ __forceinline__ double pick32(const double (&a)[32], int i) {
+  double l1[16], l2[8], l3[4], l4[2];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) l1[j] = (i & 1) ? a[2 * j + 1] : a[2 * j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) l2[j] = (i & 2) ? l1[2 * j + 1] : l1[2 * j];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) l3[j] = (i & 4) ? l2[2 * j + 1] : l2[2 * j];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) l4[j] = (i & 8) ? l3[2 * j + 1] : l3[2 * j];
+  return (i & 16) ? l4[1] : l4[0];
+}
+
+// Block scheduling: for each query block the local tile count, the normalised block scores p
+// over its candidate blocks, the selection p >= τ, and the selected list sorted by
+// (p descending, block ascending).
+// A group of GL lanes (a power of two; 32/GL query blocks per warp) serves one query block. Lane l
+// of the group owns the chunks k = l + GL·h (h < CPL) of 32 consecutive blocks: it sums a chunk's
+// weights sequentially in block order, keeping them in registers until the selection (they are
+// recomputed when it owns two chunks), and Z adds the chunk sums in chunk order. Shared memory per
+// query block holds only the selected list (cap2 entries; cap2 bounds the list length: at most
+// floor(1/τ) + 1 blocks can reach p >= τ since the p sum to one).
+template <int CPL>
 __global__ void __launch_bounds__(128)
     k_schedule(const float *__restrict__ r, const int32_t *__restrict__ ncount,
                const int32_t *__restrict__ perm_q, int32_t *__restrict__ sel_cnt,
                int32_t *__restrict__ sel_blk, int32_t *__restrict__ local_tiles, int N, int B,
-               int S, int nB, int nSeg, int cap2, double tau, long long n_qblocks) {
+               int S, int nB, int nSeg, int cap2, int GL, double tau, long long n_qblocks) {
   extern __shared__ unsigned char smem_raw[];
-  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
-  const long long qb = (long long)blockIdx.x * (blockDim.x / kWarp) + warp;
-  if (qb >= n_qblocks) return;
-  const int wslots = nB + (nB + 31) / 32;
-  const size_t per_warp = ((size_t)wslots * 8 + (size_t)cap2 * 12 + 15) & ~(size_t)15;
-  double *w = reinterpret_cast<double *>(smem_raw + per_warp * warp);
-  double *lp = w + wslots;
+  const int lane = threadIdx.x % kWarp, li = lane & (GL - 1), gi = threadIdx.x / GL;
+  const long long per_cta = blockDim.x / GL;
+  const long long qb = (long long)blockIdx.x * per_cta + gi;
+  // A warp whose first query block is past the end has nothing to do; inside a warp every lane
+  // takes part in the shuffles, and a group past the end works on block 0 and writes nothing.
+  if ((long long)blockIdx.x * per_cta + (threadIdx.x & ~(kWarp - 1)) / GL >= n_qblocks) return;
+  const bool real = qb < n_qblocks;
+  const long long q0 = real ? qb : 0;
+  const size_t per_q = ((size_t)cap2 * 12 + 15) & ~(size_t)15;
+  double *lp = reinterpret_cast<double *>(smem_raw + per_q * gi);
   int *lc = reinterpret_cast<int *>(lp + cap2);
-  auto wi = [](int c) { return c + (c >> 5); };
-
-  const long long qh = qb / nB;
-  const int b = (int)(qb % nB);
-  const int s = (int)((long long)b * B / S);
   const unsigned full = 0xffffffffu;
 
+  const long long qh = q0 / nB;
+  const int b = (int)(q0 % nB);
+  const int s = (int)((long long)b * B / S);
+
   int mx = -1;
-  for (int e = lane; e < B; e += kWarp) mx = max(mx, __ldg(perm_q + qh * N + (size_t)b * B + e));
-  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(full, mx, o));
-  if (lane == 0) local_tiles[qb] = (mx - s * S) / B + 1;
+  for (int e = li; e < B; e += GL) mx = max(mx, __ldg(perm_q + qh * N + (size_t)b * B + e));
+  for (int o = GL / 2; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(full, mx, o, GL));
+  if (real && li == 0) local_tiles[qb] = (mx - s * S) / B + 1;
 
-  const float *rr = r + (size_t)qb * nB;
+  const float *rr = r + (size_t)q0 * nB;
   const int32_t *nn = ncount + ((size_t)qh * nSeg + s) * nB;
+  // Rows start 16-byte aligned when nB is a multiple of 4 (the arrays themselves are).
+  const bool vec = (nB & 3) == 0;
+  const int n_chunks = (nB + 31) / 32;
+  int nv[32];
+  float rv[32];
+  // Counts and scores of this lane's chunk h (zeros past nB).
+  auto load_chunk = [&](int h) {
+    const int c0 = 32 * (li + GL * h);
+    if (vec && c0 + 32 <= nB) {
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const int4 n4 = __ldg(reinterpret_cast<const int4 *>(nn + c0) + v);
+        const float4 r4 = __ldg(reinterpret_cast<const float4 *>(rr + c0) + v);
+        nv[4 * v] = n4.x, nv[4 * v + 1] = n4.y, nv[4 * v + 2] = n4.z, nv[4 * v + 3] = n4.w;
+        rv[4 * v] = r4.x, rv[4 * v + 1] = r4.y, rv[4 * v + 2] = r4.z, rv[4 * v + 3] = r4.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int c = c0 + i;
+        nv[i] = c < nB ? __ldg(nn + c) : 0;
+        rv[i] = c < nB ? __ldg(rr + c) : 0.f;
+      }
+    }
+  };
 
-  // M = max block score over the candidates (blocks with a visible key). A lane's blocks are
-  // c = lane + 32k; their counts and scores are loaded 16 at a time.
-  constexpr int kBatch = 16;
+  // M = max block score over the candidates (blocks with a visible key). A query block with no
+  // candidate runs the steps below with no weights and ends with an empty list.
   float M = 0.f;
   bool any = false;
-  for (int c0 = 0; c0 < nB; c0 += kBatch * kWarp) {
-    int nv[kBatch];
-    float rv[kBatch];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int c = c0 + k * kWarp + lane;
-      nv[k] = c < nB ? __ldg(nn + c) : 0;
-      rv[k] = c < nB ? __ldg(rr + c) : 0.f;
-    }
+  for (int h = 0; h < CPL; ++h) {
+    load_chunk(h);
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k)
-      if (nv[k] > 0) {
-        M = any ? fmaxf(M, rv[k]) : rv[k];
+    for (int i = 0; i < 32; ++i)
+      if (nv[i] > 0) {
+        M = any ? fmaxf(M, rv[i]) : rv[i];
         any = true;
       }
   }
-  if (__ballot_sync(full, any) == 0) {
-    if (lane == 0) sel_cnt[qb] = 0;
-    return;
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    const float other = __shfl_xor_sync(full, M, o);
-    const bool other_any = __shfl_xor_sync(full, any ? 1 : 0, o) != 0;
+  for (int o = GL / 2; o > 0; o >>= 1) {
+    const float other = __shfl_xor_sync(full, M, o, GL);
+    const bool other_any = __shfl_xor_sync(full, any ? 1 : 0, o, GL) != 0;
     if (other_any) M = any ? fmaxf(M, other) : other;
     any = any || other_any;
   }
-
   const double Md = (double)M;
-  // Weights (independent per block, computed lane-strided; -1 marks a block that is not a
-  // candidate), then Z: chunks of 32 consecutive blocks, chunk k summed sequentially by lane
-  // k mod 32 (a non-candidate adds +0), then the chunk sums in chunk order.
-  for (int c0 = 0; c0 < nB; c0 += kBatch * kWarp) {
-    int nv[kBatch];
-    float rv[kBatch];
+
+  // Weights of the loaded chunk (-1 marks a block that is not a candidate).
+  double wk[32];
+  auto weights = [&]() {
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int c = c0 + k * kWarp + lane;
-      nv[k] = c < nB ? __ldg(nn + c) : 0;
-      rv[k] = c < nB ? __ldg(rr + c) : 0.f;
+    for (int i = 0; i < 32; ++i) {
+      const double e =
+          __dmul_rn(int_to_double(max(nv[i], 0)), exp64(__dsub_rn((double)rv[i], Md)));
+      wk[i] = nv[i] > 0 ? e : -1.0;
     }
-    double wv[kBatch];
+  };
+  // Z: each chunk summed sequentially from +0 in block order (a non-candidate adds +0), then the
+  // chunk sums in chunk order.
+  double part[CPL];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k)
-      wv[k] = __dmul_rn(int_to_double(max(nv[k], 0)), exp64(__dsub_rn((double)rv[k], Md)));
+  for (int h = 0; h < CPL; ++h) {
+    if (CPL > 1) load_chunk(h);
+    weights();
+    double acc = 0.0;
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int c = c0 + k * kWarp + lane;
-      if (c < nB) w[wi(c)] = nv[k] > 0 ? wv[k] : -1.0;
+    for (int i = 0; i < 32; ++i) acc = __dadd_rn(acc, wk[i] < 0.0 ? 0.0 : wk[i]);
+    part[h] = acc;
+  }
+  double Z = 0.0;
+#pragma unroll
+  for (int h = 0; h < CPL; ++h)
+    for (int k = 0; k < GL && GL * h + k < n_chunks; ++k)
+      Z = __dadd_rn(Z, __shfl_sync(full, part[h], k, GL));
+
+  // Selection p_c = w_c / Z >= τ. A weight below (τ·Z)(1 − 2^-48) gives p < τ whatever the
+  // rounding, so its division is skipped; every other candidate's p is computed exactly. The
+  // selected blocks go to the list in block order (the lanes of a group own consecutive chunks),
+  // their p computed again when written.
+  const double t_lo = __dmul_rn(__dmul_rn(tau, Z), 1.0 - 0x1p-48);
+  int cnt = 0;
+#pragma unroll
+  for (int h = 0; h < CPL; ++h) {
+    if (CPL > 1) {
+      load_chunk(h);
+      weights();
+    }
+    unsigned near = 0, mine = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (wk[i] >= 0.0 && (tau == 0.0 || !(wk[i] < t_lo))) near |= 1u << i;
+    for (unsigned m = near; m; m &= m - 1) {
+      const int i = __ffs(m) - 1;
+      if (__ddiv_rn(pick32(wk, i), Z) >= tau) mine |= 1u << i;
+    }
+    const int n_mine = __popc(mine);
+    int incl = n_mine;
+    for (int o = 1; o < GL; o <<= 1) {
+      const int t = __shfl_up_sync(full, incl, o, GL);
+      if (li >= o) incl += t;
+    }
+    int slot = cnt + incl - n_mine;
+    cnt += __shfl_sync(full, incl, GL - 1, GL);
+    for (unsigned m = mine; m; m &= m - 1, ++slot) {
+      const int i = __ffs(m) - 1;
+      if (slot < cap2) {
+        lp[slot] = __ddiv_rn(pick32(wk, i), Z);
+        lc[slot] = 32 * (li + GL * h) + i;
+      }
     }
   }
   __syncwarp();
-  const int n_chunks = (nB + 31) / 32;
-  double part0 = 0.0, part1 = 0.0;  // this lane's chunks k = lane and k = lane + 32
-  for (int k = lane; k < n_chunks; k += kWarp) {
-    double part = 0.0;
-    const int c_end = min(nB, 32 * k + 32);
-    for (int c = 32 * k; c < c_end; ++c) {
-      const double wc = w[wi(c)];
-      part = __dadd_rn(part, wc < 0.0 ? 0.0 : wc);
-    }
-    if (k < kWarp)
-      part0 = part;
-    else
-      part1 = part;
-  }
-  double Z = 0.0;
-  for (int k = 0; k < n_chunks; ++k) {
-    const double v = __shfl_sync(full, k < kWarp ? part0 : part1, k % kWarp);
-    Z = __dadd_rn(Z, v);
-  }
-
-  // Selection p_c = w_c / Z >= τ. A weight below (τ·Z)(1 − 2^-48) gives p < τ whatever the
-  // rounding, so its division is skipped; every other candidate's p is computed exactly.
-  const double t_lo = __dmul_rn(__dmul_rn(tau, Z), 1.0 - 0x1p-48);
-  int cnt = 0;
-  for (int c0 = 0; c0 < nB; c0 += kWarp) {
-    const int c = c0 + lane;
-    bool sel = false;
-    double p = 0.0;
-    const double wc = c < nB ? w[wi(c)] : -1.0;
-    if (wc >= 0.0 && (tau == 0.0 || !(wc < t_lo))) {
-      p = __ddiv_rn(wc, Z);
-      sel = p >= tau;
-    }
-    const unsigned m = __ballot_sync(full, sel);
-    const int slot = cnt + __popc(m & ((1u << lane) - 1u));
-    if (sel && slot < cap2) {
-      lp[slot] = p;
-      lc[slot] = c;
-    }
-    cnt += __popc(m);
-  }
   cnt = min(cnt, cap2);
-  int P = 1;
-  while (P < cnt) P <<= 1;
-  for (int e = cnt + lane; e < P; e += kWarp) {
+  // Bitonic network over the warp's largest power of two Pw >= every group's count (lists padded
+  // with entries that go after every block), order "goes_before".
+  int Pw = 1;
+  while (Pw < cnt) Pw <<= 1;
+  for (int o = 16; o > 0; o >>= 1) Pw = max(Pw, __shfl_xor_sync(full, Pw, o));
+  for (int e = cnt + li; e < Pw; e += GL) {
     lp[e] = -1.0;
     lc[e] = INT_MAX;
   }
   __syncwarp();
-  // Bitonic network over P entries, order "goes_before".
-  for (int k = 2; k <= P; k <<= 1) {
+  for (int k = 2; k <= Pw; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = lane; i < P; i += kWarp) {
+      for (int i = li; i < Pw; i += GL) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const bool up = (i & k) == 0;
@@ -1099,9 +1137,11 @@ __global__ void __launch_bounds__(128)
       __syncwarp();
     }
   }
-  int32_t *dst = sel_blk + (size_t)qb * nB;
-  for (int e = lane; e < cnt; e += kWarp) dst[e] = lc[e];
-  if (lane == 0) sel_cnt[qb] = cnt;
+  if (real) {
+    int32_t *dst = sel_blk + (size_t)qb * nB;
+    for (int e = li; e < cnt; e += GL) dst[e] = lc[e];
+    if (li == 0) sel_cnt[qb] = cnt;
+  }
 }
 
 // ------------------------------------------------------------------ validation and stats
@@ -1424,16 +1464,21 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   }
   int cap2 = 1;
   while (cap2 < cap) cap2 <<= 1;
-  const size_t per_warp =
-      ((size_t)(d.nB + (d.nB + 31) / 32) * 8 + (size_t)cap2 * 12 + 15) & ~(size_t)15;
-  const int warps = (int)std::max<size_t>(1, std::min<size_t>(4, (200u << 10) / per_warp));
-  const size_t sched_smem = per_warp * warps;
-  if ((e = cudaFuncSetAttribute(k_schedule, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // Lanes per query block: the chunks of 32 blocks rounded up to a power of two, at most 32 (two
+  // chunks per lane beyond 1024 blocks; check_config caps nB at 2048).
+  const int n_chunks = (d.nB + 31) / 32;
+  int GL = 1;
+  while (GL < n_chunks && GL < 32) GL <<= 1;
+  const size_t per_q = ((size_t)cap2 * 12 + 15) & ~(size_t)15;
+  const int sched_threads = 128;
+  const size_t sched_smem = per_q * (size_t)(sched_threads / GL);
+  auto sched = n_chunks <= 32 ? k_schedule<1> : k_schedule<2>;
+  if ((e = cudaFuncSetAttribute(sched, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)sched_smem)) != cudaSuccess)
     return e;
-  k_schedule<<<blocks_for(nblk, warps), warps * kWarp, sched_smem, st>>>(
+  sched<<<blocks_for(nblk, sched_threads / GL), sched_threads, sched_smem, st>>>(
       r, ncount, out.perm_q, out.sel_cnt, out.sel_blk, out.local_tiles, d.N, d.B, d.S, d.nB,
-      d.nSeg, cap2, (double)cfg.tau, nblk);
+      d.nSeg, cap2, GL, (double)cfg.tau, nblk);
   note_launch();
   return cudaGetLastError();
 }
