@@ -482,6 +482,7 @@ __global__ void k_replicate_group_rows(int32_t *__restrict__ a, long long row_le
 // kRadixTile elements: per pass a digit count per tile, then a scatter per tile that derives its
 // offsets from the run's counts.
 constexpr int kRadixR = 8, kRadixThreads = 512, kRadixTile = kRadixR * kRadixThreads;
+static_assert(kRadixThreads == 2 * 256, "the scatter reads each digit's counts with two threads");
 
 // Element e of a tile, for thread (warp, lane) and round r.
 __device__ __forceinline__ int radix_elem(int r) {
@@ -529,85 +530,96 @@ __global__ void __launch_bounds__(kRadixThreads)
     counts[(run * 256 + d) * tiles + tile] = h[d];
 }
 
-// Output offsets of one pass, in place over the counts: for run, digit d and tile t, the number of
-// elements of the run with a smaller digit plus those with digit d in tiles before t. One CTA of
-// 256 threads per run (thread = digit).
-__global__ void __launch_bounds__(256) k_radix_offsets(int *__restrict__ counts, int tiles) {
-  __shared__ int tot[256];
-  const long long run = blockIdx.x;
-  const int d = threadIdx.x;
-  int *c = counts + (run * 256 + d) * tiles;
-  int sum = 0;
-  for (int t0 = 0; t0 < tiles; t0 += 8) {  // eight loads in flight
-    int v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = t0 + k < tiles ? c[t0 + k] : 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) sum += v[k];
-  }
-  tot[d] = sum;
-  __syncthreads();
-  if (d < 32) {  // exclusive scan of the 256 digit totals, 8 per lane
-    int v[8], s8 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = tot[d * 8 + i];
-      s8 += v[i];
-    }
-    int incl = s8;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (d >= o) incl += t;
-    }
-    int run_sum = incl - s8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      tot[d * 8 + i] = run_sum;
-      run_sum += v[i];
-    }
-  }
-  __syncthreads();
-  int off = tot[d];
-  for (int t0 = 0; t0 < tiles; t0 += 8) {
-    int v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = t0 + k < tiles ? c[t0 + k] : 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (t0 + k < tiles) c[t0 + k] = off;
-      off += v[k];
-    }
-  }
-}
-
-// Scatter of one pass: each tile ranks its elements by digit (stable), groups them in shared
-// memory and writes each digit's run to its offset. The last pass writes only the values, as the
-// permutation.
+// Scatter of one pass: each tile derives its output offset per digit from the per-tile counts
+// (the run's elements with a smaller digit plus those with the same digit in earlier tiles), ranks
+// its elements by digit (stable), groups them in shared memory and writes each digit's run to its
+// offset. The last pass writes only the values, as the permutation.
 __global__ void __launch_bounds__(kRadixThreads)
     k_radix_scatter(const float *__restrict__ score, const uint32_t *__restrict__ keys_in,
                     const uint32_t *__restrict__ vals_in, uint32_t *__restrict__ keys_out,
                     uint32_t *__restrict__ vals_out, int32_t *__restrict__ perm_out,
                     long long run_len, long long head_len, long long score_stride,
                     long long perm_stride, int tiles, int shift,
-                    const int *__restrict__ offsets) {
+                    const int *__restrict__ counts) {
   extern __shared__ int sm_r[];
   uint32_t *skey = reinterpret_cast<uint32_t *>(sm_r);   // [tile]
   uint32_t *sval = skey + kRadixTile;                     // [tile]
   int *hist = reinterpret_cast<int *>(sval + kRadixTile);  // [warps·256]
   int *dbase = hist + (kRadixThreads / 32) * 256;          // [256]
   int *goff = dbase + 256;                                 // [256]
+  int *dtot = goff + 256;                                  // [256]
   const long long run = blockIdx.x / tiles;
   const int tile = blockIdx.x % tiles;
   const long long base = run * run_len + (long long)tile * kRadixTile;
   const int n = (int)min((long long)kRadixTile, run_len - (long long)tile * kRadixTile);
-  // This tile's output offset per digit (prefixed by k_radix_offsets).
-  if (threadIdx.x < 256) goff[threadIdx.x] = __ldg(offsets + (run * 256 + threadIdx.x) * tiles + tile);
-  __syncthreads();
   uint32_t key[kRadixR], val[kRadixR], dig[kRadixR];
   int dest[kRadixR];
   radix_load(score, keys_in, vals_in, run * score_stride + (long long)tile * kRadixTile, base,
              tile * kRadixTile, n, key, val);
+  // Per digit d (threads 2d and 2d + 1, half of the tiles each): the run's total and the count in
+  // tiles before this one; then the exclusive scan of the 256 totals.
+  const unsigned full = 0xffffffffu;
+  {
+    const int d = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int *c = counts + (run * 256 + d) * tiles;
+    int tot = 0, pre = 0;
+    if ((tiles & 7) == 0 && tiles <= 64) {  // 16-byte aligned halves of at most 32 counts
+      const int per = tiles / 2, t0 = half * per;
+      const int4 *c4 = reinterpret_cast<const int4 *>(c + t0);
+      int4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (4 * k < per) v[k] = __ldg(c4 + k);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (4 * k < per) {
+          const int t = t0 + 4 * k;
+          tot += v[k].x + v[k].y + v[k].z + v[k].w;
+          pre += (t < tile ? v[k].x : 0) + (t + 1 < tile ? v[k].y : 0) +
+                 (t + 2 < tile ? v[k].z : 0) + (t + 3 < tile ? v[k].w : 0);
+        }
+    } else {
+      for (int t0 = half; t0 < tiles; t0 += 16) {  // eight loads in flight
+        int v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = t0 + 2 * k < tiles ? __ldg(c + t0 + 2 * k) : 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          tot += v[k];
+          pre += t0 + 2 * k < tile ? v[k] : 0;
+        }
+      }
+    }
+    tot += __shfl_xor_sync(full, tot, 1);
+    pre += __shfl_xor_sync(full, pre, 1);
+    if (!half) {
+      goff[d] = pre;
+      dtot[d] = tot;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int v[8], s8 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = dtot[lane * 8 + i];
+      s8 += v[i];
+    }
+    int incl = s8;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int run_sum = incl - s8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      goff[lane * 8 + i] += run_sum;
+      run_sum += v[i];
+    }
+  }
+  // (radix_ranks synchronises the CTA before goff is read.)
 #pragma unroll
   for (int r = 0; r < kRadixR; ++r) dig[r] = (key[r] >> shift) & 255u;
   radix_ranks<kRadixR, kRadixThreads / 32>(dig, dest, hist, dbase);
@@ -1262,7 +1274,7 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
   const int tiles = (int)((run_len + kRadixTile - 1) / kRadixTile);
   const long long runs = total / run_len;
   const unsigned grid = (unsigned)(runs * tiles);
-  const size_t smem = (size_t)2 * kRadixTile * 4 + (size_t)(kRadixThreads / 32) * 256 * 4 + 512 * 4;
+  const size_t smem = (size_t)2 * kRadixTile * 4 + (size_t)(kRadixThreads / 32) * 256 * 4 + 768 * 4;
   cudaError_t e = cudaFuncSetAttribute(k_radix_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -1272,8 +1284,6 @@ cudaError_t radix_sort_runs(const float *score, uint32_t *k0, uint32_t *v0, uint
     const float *sc = pass == 0 ? score : nullptr;
     k_radix_count<<<grid, kRadixThreads, 0, st>>>(sc, kin, run_len, score_stride, tiles,
                                                   8 * pass, counts);
-    note_launch();
-    k_radix_offsets<<<(unsigned)runs, 256, 0, st>>>(counts, tiles);
     note_launch();
     k_radix_scatter<<<grid, kRadixThreads, smem, st>>>(sc, kin, vin, kout, vout,
                                                        pass == 3 ? perm_out : nullptr, run_len,
