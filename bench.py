@@ -243,7 +243,8 @@ def run_s2o(args):
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     o = torch.empty_like(qd)
     idx = s2o.alloc_indices(cfg, dev)
-    ws = s2o.alloc_workspace(cfg, dev)
+    # With room for the permuted copy of K and V, which the library makes when it pays.
+    ws = s2o.alloc_prefill_workspace(cfg, dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -252,7 +253,7 @@ def run_s2o(args):
         s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
         if ev is not None:
             ev[1].record(stream)
-        s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx, out=o)
+        s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws, out=o)
         if ev is not None:
             ev[2].record(stream)
 
@@ -405,10 +406,11 @@ def run_sweep(args):
             cache[key] = tuple(t.to(dev) for t in gen.make_inputs(w))
         qd, kd, vd = cache[key]
         cfg = s2o.Config.of(w)
-        idx, ws, o = s2o.alloc_indices(cfg, dev), s2o.alloc_workspace(cfg, dev), torch.empty_like(qd)
+        idx, o = s2o.alloc_indices(cfg, dev), torch.empty_like(qd)
+        ws = s2o.alloc_prefill_workspace(cfg, dev)
         for _ in range(2):
             s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
-            s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx, out=o)
+            s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws, out=o)
         a0, a1 = events()
         b0, b1 = events()
         a0.record()
@@ -417,7 +419,7 @@ def run_sweep(args):
         a1.record()
         b0.record()
         for _ in range(reps):
-            s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx, out=o)
+            s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws, out=o)
         b1.record()
         torch.cuda.synchronize()
         index_ms, attn_ms = a0.elapsed_time(a1) / reps, b0.elapsed_time(b1) / reps

@@ -120,7 +120,8 @@ s2o_status s2o_workspace_views(const s2o_config *cfg, void *ws, size_t ws_bytes,
 
 /* The whole hot path ([S2O, Summary ¶2]): s2o_build_indices into `idx`, then the fused
  * gather-attention over local tiles and selected permuted blocks; O [batch, Hq, N, d] bf16 is
- * written at original positions. */
+ * written at original positions. With ws_bytes >= s2o_prefill_workspace_size the permuted copy of
+ * K and V may be used (see s2o_set_permuted_copy); s2o_workspace_size bytes suffice without it. */
 s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const void *k,
                                  const void *v, void *o, const s2o_indices *idx, void *ws,
                                  size_t ws_bytes, s2o_stream stream);
@@ -134,6 +135,33 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
                                               const void *k, const void *v,
                                               const s2o_indices *idx, void *o,
                                               s2o_stream stream);
+
+/* Bytes of scratch with which s2o_attention_prefill and s2o_attention_prefill_with_indices_ws may
+ * also make the permuted copy of K and V (see s2o_set_permuted_copy): s2o_workspace_size, a
+ * 256-byte flag area, and the copy itself, 2 · copy_heads · N · d bf16 values with copy_heads =
+ * batch · n_q_heads (batch · n_kv_heads for s2o_attention_prefill with shared_key_order = 1).
+ * Written to *bytes. Host only; no device work. */
+s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes);
+
+/* As s2o_attention_prefill_with_indices, with a workspace: when ws_bytes is at least
+ * s2o_prefill_workspace_size (with shared_key_order treated as 0) and the permuted copy is on,
+ * a device-side decision may copy K and V into each query head's key order first, and the
+ * permuted pass then loads every selected block as one contiguous tile instead of gathering its
+ * rows. The output is bit for bit the same as without the copy. With a smaller workspace this is
+ * s2o_attention_prefill_with_indices. ws: device, 16-byte aligned, owned by the caller. */
+s2o_status s2o_attention_prefill_with_indices_ws(const s2o_config *cfg, const void *q,
+                                                 const void *k, const void *v,
+                                                 const s2o_indices *idx, void *o, void *ws,
+                                                 size_t ws_bytes, s2o_stream stream);
+
+/* The permuted copy ([S2O, Summary ¶2] gathers the scattered rows by index; when most blocks are
+ * selected, permuting K and V once in memory makes each selected block contiguous, so it loads
+ * as one tile). mode 0: never; 1 (the default): when the selected blocks of the call outnumber
+ * twice the blocks the copy writes (copying a block costs about one gather of it), decided on the
+ * device without synchronising; 2: always (for tests). Only calls given a workspace of
+ * s2o_prefill_workspace_size bytes make it. Affects calls made after it; not thread-safe against
+ * concurrent calls. Other values are treated as 1. */
+void s2o_set_permuted_copy(int mode);
 
 /* In-repo dense causal attention baseline, Eq. (1) of [AB], on the same kernel machinery
  * (contiguous tiles, no index arrays). cfg->segment_len, tau and query_perm are ignored. */
@@ -196,8 +224,8 @@ s2o_status s2o_build_indices_static(const s2o_config *cfg, const void *q, const 
                                     const s2o_indices *out, s2o_stream stream);
 
 /* Diagnostic: evaluates the library's exp64 — the binary64 exponential behind the block weights of
- * the early stop (a Cody–Waite reduction by ln 2 and a degree-13 Taylor polynomial, defined in
- * the project's definition file; the pages give no normalisation, see [S2O, Summary ¶2]) — on n
+ * the early stop (a Cody–Waite reduction by ln 2 and a degree-13 Taylor polynomial written for
+ * this library; the pages give no normalisation, see [S2O, Summary ¶2]) — on n
  * device doubles x (each ≤ 0), writing device doubles y. Asynchronous on `stream`. */
 s2o_status s2o_exp64_eval(const double *x, double *y, int n, s2o_stream stream);
 

@@ -26,6 +26,8 @@ __all__ = [
     "dense_causal_prefill", "validate_indices", "index_stats", "workspace_views",
     "set_wait_limit_ns", "set_attention_max_ctas", "check_device_status", "exp64_eval", "library_path",
     "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
+    "prefill_workspace_size", "alloc_prefill_workspace", "attention_prefill_with_indices_ws",
+    "set_permuted_copy",
 ]
 
 STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
@@ -147,12 +149,14 @@ def _load():
         C, I = ctypes.POINTER(_Config), ctypes.POINTER(_Indices)
         sig = {
             "s2o_workspace_size": [C, ctypes.POINTER(sz)],
+            "s2o_prefill_workspace_size": [C, ctypes.POINTER(sz)],
             "s2o_index_sizes": [C, ctypes.POINTER(sz * 5)],
             "s2o_build_indices": [C, vp, vp, I, vp, sz, vp],
             "s2o_build_indices_static": [C, vp, vp, I, vp],
             "s2o_workspace_views": [C, vp, sz, ctypes.POINTER(_View)],
             "s2o_attention_prefill": [C, vp, vp, vp, vp, I, vp, sz, vp],
             "s2o_attention_prefill_with_indices": [C, vp, vp, vp, I, vp, vp],
+            "s2o_attention_prefill_with_indices_ws": [C, vp, vp, vp, I, vp, vp, sz, vp],
             "s2o_dense_causal_prefill": [C, vp, vp, vp, vp, vp],
             "s2o_validate_indices": [C, I, vp, sz, vp],
             "s2o_index_stats": [C, I, vp, sz, ctypes.POINTER(_Stats), vp],
@@ -169,6 +173,8 @@ def _load():
         lib.s2o_set_wait_limit_ns.restype = None
         lib.s2o_set_attention_max_ctas.argtypes = [ctypes.c_int]
         lib.s2o_set_attention_max_ctas.restype = None
+        lib.s2o_set_permuted_copy.argtypes = [ctypes.c_int]
+        lib.s2o_set_permuted_copy.restype = None
         lib.s2o_status_string.argtypes = [st]
         lib.s2o_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -213,6 +219,18 @@ def index_sizes(cfg: Config):
 
 def alloc_workspace(cfg: Config, device="cuda") -> torch.Tensor:
     return torch.empty(workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def prefill_workspace_size(cfg: Config) -> int:
+    """Workspace bytes with which the prefill may also use the permuted copy of K and V."""
+    n = ctypes.c_size_t(0)
+    _check(_load().s2o_prefill_workspace_size(ctypes.byref(cfg._c()), ctypes.byref(n)),
+           "s2o_prefill_workspace_size")
+    return n.value
+
+
+def alloc_prefill_workspace(cfg: Config, device="cuda") -> torch.Tensor:
+    return torch.empty(prefill_workspace_size(cfg), dtype=torch.uint8, device=device)
 
 
 def alloc_indices(cfg: Config, device="cuda") -> Indices:
@@ -278,7 +296,7 @@ def attention_prefill(cfg: Config, q, k, v, out: torch.Tensor | None = None,
     o = out if out is not None else torch.empty_like(q)
     _bf16(o, q.shape, "out")
     idx = idx or alloc_indices(cfg, q.device)
-    ws = ws if ws is not None else alloc_workspace(cfg, q.device)
+    ws = ws if ws is not None else alloc_prefill_workspace(cfg, q.device)
     ci = idx._c()
     _check(_load().s2o_attention_prefill(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
                                          v.data_ptr(), o.data_ptr(), ctypes.byref(ci),
@@ -298,6 +316,25 @@ def attention_prefill_with_indices(cfg: Config, q, k, v, idx: Indices,
                                                       ctypes.byref(ci), o.data_ptr(),
                                                       _stream(q.device)),
            "s2o_attention_prefill_with_indices")
+    return o
+
+
+def attention_prefill_with_indices_ws(cfg: Config, q, k, v, idx: Indices, ws: torch.Tensor,
+                                      out: torch.Tensor | None = None) -> torch.Tensor:
+    """Steps 3-4 on given indices with a workspace (the permuted copy needs
+    ``prefill_workspace_size`` bytes)."""
+    _qkv(cfg, q, k, v)
+    o = out if out is not None else torch.empty_like(q)
+    _bf16(o, q.shape, "out")
+    if ws.dtype != torch.uint8 or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous uint8 CUDA tensor")
+    ci = idx._c()
+    _check(_load().s2o_attention_prefill_with_indices_ws(ctypes.byref(cfg._c()), q.data_ptr(),
+                                                         k.data_ptr(), v.data_ptr(),
+                                                         ctypes.byref(ci), o.data_ptr(),
+                                                         ws.data_ptr(), ws.numel(),
+                                                         _stream(q.device)),
+           "s2o_attention_prefill_with_indices_ws")
     return o
 
 
@@ -341,6 +378,11 @@ def kernel_launch_count() -> int:
 
 def set_wait_limit_ns(ns: int) -> None:
     _load().s2o_set_wait_limit_ns(int(ns))
+
+
+def set_permuted_copy(mode: int) -> None:
+    """Permuted copy of K/V for the permuted pass: 0 never, 1 when it pays (default), 2 always."""
+    _load().s2o_set_permuted_copy(int(mode))
 
 
 def set_attention_max_ctas(max_ctas: int) -> None:

@@ -11,6 +11,7 @@ namespace s2o {
 namespace {
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_attention_max_ctas{0};
+std::atomic<int> g_permuted_copy{1};
 std::atomic<unsigned long long> g_launches{0};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -55,6 +56,35 @@ bool indices_ok(const s2o_indices *idx) {
 }
 
 s2o_status from_cuda(cudaError_t e) { return e == cudaSuccess ? S2O_OK : S2O_ERR_CUDA; }
+
+// Bytes of one of the permuted copies (K or V) for `heads` copy heads, 256-byte aligned.
+size_t copy_bytes(const Dims &d, long long heads) {
+  return align256((size_t)heads * (size_t)d.N * (size_t)d.D * 2);
+}
+constexpr size_t kFlagArea = 256;
+
+// Steps 3-4 with the optional permuted copy (copy heads: KV heads when per_kv, else query heads);
+// the copy is used when the workspace holds it and the mode allows it.
+s2o_status attention_ws(const s2o_config &c, const void *q, const void *k, const void *v,
+                        const s2o_indices &idx, void *o, void *ws, size_t ws_bytes, bool per_kv,
+                        cudaStream_t st) {
+  const Dims d = dims_of(c);
+  AttnArgs a{q, k, v, o, idx.perm_q, idx.perm_k, idx.sel_cnt, idx.sel_blk, idx.local_tiles, false};
+  const int mode = g_permuted_copy.load();
+  const size_t base = ws_layout(d).total, cb = copy_bytes(d, per_kv ? d.bhkv() : d.bhq());
+  if (mode != 0 && ws && ws_bytes >= base + kFlagArea + 2 * cb) {
+    char *b = static_cast<char *>(ws);
+    uint32_t *flag = reinterpret_cast<uint32_t *>(b + base);
+    a.kp = b + base + kFlagArea;
+    a.vp = b + base + kFlagArea + cb;
+    a.copy_flag = flag;
+    a.copy_per_kv = per_kv;
+    const cudaError_t e = launch_permuted_copy(d, a, mode, flag, st);
+    if (e != cudaSuccess) return S2O_ERR_CUDA;
+  }
+  return from_cuda(launch_attention(d, a, g_wait_limit_ns.load(), g_attention_max_ctas.load(),
+                                    st));
+}
 }  // namespace
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -198,6 +228,19 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
                                     (cudaStream_t)stream));
 }
 
+s2o_status s2o_attention_prefill_with_indices_ws(const s2o_config *cfg, const void *q,
+                                                 const void *k, const void *v,
+                                                 const s2o_indices *idx, void *o, void *ws,
+                                                 size_t ws_bytes, s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !indices_ok(idx) || (ws && !aligned16(ws)))
+    return S2O_ERR_INVALID_ARGUMENT;
+  // Caller-supplied indices: one copy per query head, each in that head's own key order.
+  return attention_ws(*cfg, q, k, v, *idx, o, ws, ws_bytes, false, (cudaStream_t)stream);
+}
+
 s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const void *k,
                                  const void *v, void *o, const s2o_indices *idx, void *ws,
                                  size_t ws_bytes, s2o_stream stream) {
@@ -206,7 +249,9 @@ s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const voi
   if (!v || !o || !aligned16(v) || !aligned16(o)) return S2O_ERR_INVALID_ARGUMENT;
   st = s2o_build_indices(cfg, q, k, idx, ws, ws_bytes, stream);
   if (st != S2O_OK) return st;
-  return s2o_attention_prefill_with_indices(cfg, q, k, v, idx, o, stream);
+  // The indices were built here: with one key ordering per KV head the copy is made per KV head.
+  return attention_ws(*cfg, q, k, v, *idx, o, ws, ws_bytes, cfg->shared_key_order != 0,
+                      (cudaStream_t)stream);
 }
 
 s2o_status s2o_dense_causal_prefill(const s2o_config *cfg, const void *q, const void *k,
@@ -267,6 +312,17 @@ s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *
 }
 
 void s2o_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!bytes) return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  *bytes = ws_layout(d).total + kFlagArea + 2 * copy_bytes(d, d.bhq());
+  return S2O_OK;
+}
+
+void s2o_set_permuted_copy(int mode) { g_permuted_copy.store(mode == 0 || mode == 2 ? mode : 1); }
 
 void s2o_set_attention_max_ctas(int max_ctas) {
   g_attention_max_ctas.store(max_ctas > 0 ? max_ctas : 0);

@@ -314,6 +314,8 @@ struct Params {
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
   FastDiv div_G, div_seg, div_nB, div_nSeg, div_Hkv;  // unit-id decoding (S/B blocks a segment)
+  const uint32_t *copy_flag;  // permuted copy of K/V in use when non-null and set
+  int copy_per_kv;            // copy rows per KV head (else per query head)
 };
 
 struct Unit {
@@ -473,9 +475,9 @@ __device__ __forceinline__ int4 block_rows(const Params &p, const Unit &u, int c
 // atom; gathered rows (prepared by block_rows): tile::gather4, four rows per lane.
 template <int D, int BN>
 __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap *tm_tile,
-                                        const CUtensorMap *tm_row, const Params &p,
-                                        const Pair &P, const Item &it, int4 rows, uint32_t bar,
-                                        int lane) {
+                                        const CUtensorMap *tm_row, const CUtensorMap *tm_copy,
+                                        const Params &p, const Pair &P, const Item &it, int4 rows,
+                                        int c, bool use_copy, uint32_t bar, int lane) {
   using L = Layout<D, BN>;
   const Unit &u = it.x ? P.u1 : P.u0;
   if (it.local) {
@@ -483,6 +485,13 @@ __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap *tm_tile
       for (int a = 0; a < D / 64; ++a)
         tma_load_tile(dst + a * L::ATOM_KV, tm_tile, a * 64,
                       (int)(u.kh * p.N) + u.seg0 + it.t * BN, bar);
+  } else if (use_copy) {
+    // Selected block c of the permuted copy: contiguous rows c·B.. of the unit's copy head.
+    if (lane == 0) {
+      const long long h = p.copy_per_kv ? u.kh : u.qh;
+      for (int a = 0; a < D / 64; ++a)
+        tma_load_tile(dst + a * L::ATOM_KV, tm_copy, a * 64, (int)(h * p.N) + c * BN, bar);
+    }
   } else if (lane < BN / 4) {
     for (int a = 0; a < D / 64; ++a)
       tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, tm_row, a * 64, rows.x, rows.y, rows.z,
@@ -646,7 +655,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_k_row,
                          const __grid_constant__ CUtensorMap tm_v_tile,
                          const __grid_constant__ CUtensorMap tm_v_row,
-                         const __grid_constant__ CUtensorMap tm_o_tile, const Params p) {
+                         const __grid_constant__ CUtensorMap tm_o_tile,
+                         const __grid_constant__ CUtensorMap tm_kp_tile,
+                         const __grid_constant__ CUtensorMap tm_vp_tile, const Params p) {
   using L = Layout<D, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -731,6 +742,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int full0 = is_k ? kKFull : kVFull, empty0 = is_k ? kKEmpty : kVEmpty;
     const CUtensorMap *tm_tile = is_k ? &tm_k_tile : &tm_v_tile;
     const CUtensorMap *tm_row = is_k ? &tm_k_row : &tm_v_row;
+    const CUtensorMap *tm_copy = is_k ? &tm_kp_tile : &tm_vp_tile;
+    // Selected blocks come from the permuted copy when the launch has one and its flag is set.
+    const bool use_copy = p.copy_flag != nullptr && __ldg(p.copy_flag) != 0u;
     long long kj = 0;  // stream items issued so far (all work items of this CTA)
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
@@ -744,15 +758,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         return t.local ? -1 : sel_block(p, t.x ? P.u1 : P.u0, t.t);
       };
       auto rows_of = [&](int j, int c) -> int4 {
-        if (j >= P.total || c < 0) return make_int4(0, 0, 0, 0);
+        if (j >= P.total || c < 0 || use_copy) return make_int4(0, 0, 0, 0);
         const Item t = item_at(P, j);
         return block_rows<BN>(p, t.x ? P.u1 : P.u0, c, lane);
       };
-      int4 rows = rows_of(0, block_of(0));
+      int c_cur = block_of(0);
+      int4 rows = rows_of(0, c_cur);
       int c_next = block_of(1);
       for (int j = 0; j < P.total; ++j) {
         const Item it = item_at(P, j);
         const int4 rows_next = rows_of(j + 1, c_next);
+        const int c_this = c_cur;
+        c_cur = c_next;
         c_next = block_of(j + 2);
         const int st = (int)(kj % stages);
         if (kj >= stages &&
@@ -762,8 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) mbar_expect_tx(bar(full0 + st), L::KV_BYTES);
         __syncwarp();
-        load_kv<D, BN>(ring + st * L::KV_BYTES, tm_tile, tm_row, p, P, it, rows, bar(full0 + st),
-                       lane);
+        load_kv<D, BN>(ring + st * L::KV_BYTES, tm_tile, tm_row, tm_copy, p, P, it, rows, c_this,
+                       use_copy, bar(full0 + st), lane);
         rows = rows_next;
         ++kj;
       }
@@ -1189,6 +1206,62 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// ------------------------------------------------------------------ permuted copy of K and V
+
+// Whether the permuted pass uses the permuted copy: always (mode 2), or (mode 1) when the
+// selected blocks of all query blocks outnumber twice the blocks the copy writes; copying a
+// block costs about one gather of it, and each selected block then loads as a contiguous tile.
+// One CTA.
+__global__ void __launch_bounds__(1024)
+    k_copy_decide(const int32_t *__restrict__ sel_cnt, long long n_units, int nB, int mode,
+                  long long copy_blocks, uint32_t *__restrict__ flag) {
+  __shared__ unsigned long long part[32];
+  unsigned long long sum = 0;
+  for (long long i = threadIdx.x; i < n_units; i += blockDim.x)
+    sum += (unsigned long long)min(max(__ldg(sel_cnt + i), 0), nB);
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (threadIdx.x % 32 == 0) part[threadIdx.x / 32] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long total = 0;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) total += part[w];
+    *flag = (mode == 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks)) ? 1u : 0u;
+  }
+}
+
+// kp[h·N + rank] = K row perm_k[hq(h)][rank] of h's KV head, and the same for V (h a query head,
+// or a KV head whose first query head's ordering is used). 16-byte pieces, grid-stride; nothing
+// when the flag is clear.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_permute_kv(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                 const int32_t *__restrict__ perm_k, uint4 *__restrict__ kp,
+                 uint4 *__restrict__ vp, long long copy_rows, int N, int Hq, int Hkv, int G,
+                 int per_kv, const uint32_t *__restrict__ flag) {
+  if (__ldg(flag) == 0u) return;
+  constexpr int PIECES = D * 2 / 16;  // 16-byte pieces per row
+  const long long n = copy_rows * PIECES;
+  for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < n;
+       x += (long long)gridDim.x * blockDim.x) {
+    const long long row = x / PIECES;
+    const int piece = (int)(x % PIECES);
+    const long long h = row / N;
+    const int rank = (int)(row % N);
+    // (batch, head) of the copy row, its KV head, and the query head whose ordering it follows.
+    const int heads = per_kv ? Hkv : Hq;
+    const long long beta = h / heads;
+    const int hh = (int)(h % heads);
+    const long long kh = beta * Hkv + (per_kv ? hh : hh / G);
+    const long long qh = beta * Hq + (per_kv ? hh * G : hh);
+    const int j = min(max(__ldg(perm_k + qh * N + rank), 0), N - 1);
+    const long long src = (kh * N + j) * PIECES + piece;
+    kp[x] = __ldg(k + src);
+    vp[x] = __ldg(v + src);
+  }
+}
+
+
+
 // 2-D bf16 tensor map over a [rows, D] row-major matrix, box {64 columns, box_rows}, 128-byte
 // swizzle (one 64-column atom per box row is exactly one 128-byte swizzle span).
 bool make_map(CUtensorMap *m, const void *base, long long rows, int D, int box_rows) {
@@ -1223,13 +1296,23 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   using L = Layout<D, BN>;
   static_assert(L::SMEM <= 232448, "shared memory budget");
   static_assert(kNumBars * 8 + 4 <= (int)L::BAR_BYTES, "barrier area");
-  CUtensorMap tq, tqr, tk, tkr, tv, tvr, to;
+  CUtensorMap tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp;
   const long long q_rows = d.bhq() * d.N, kv_rows = d.bhkv() * d.N;
   if (!make_map(&tq, a.q, q_rows, D, BN) || !make_map(&tqr, a.q, q_rows, D, 1) ||
       !make_map(&tk, a.k, kv_rows, D, BN) || !make_map(&tkr, a.k, kv_rows, D, 1) ||
       !make_map(&tv, a.v, kv_rows, D, BN) || !make_map(&tvr, a.v, kv_rows, D, 1) ||
       !make_map(&to, a.o, q_rows, D, BN))
     return cudaErrorInvalidValue;
+  // The permuted copy's maps (without a copy they repeat K's and V's and are never used).
+  const bool copy = a.copy_flag != nullptr && a.kp != nullptr && a.vp != nullptr;
+  const long long copy_rows = (a.copy_per_kv ? d.bhkv() : d.bhq()) * d.N;
+  if (copy) {
+    if (!make_map(&tkp, a.kp, copy_rows, D, BN) || !make_map(&tvp, a.vp, copy_rows, D, BN))
+      return cudaErrorInvalidValue;
+  } else {
+    tkp = tk;
+    tvp = tv;
+  }
   cudaError_t e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
   if (e != cudaSuccess) return e;
@@ -1254,6 +1337,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   p.div_G.init(d.G);
   p.div_nB.init(d.nB);
   p.div_Hkv.init(d.Hkv);
+  p.copy_flag = copy ? a.copy_flag : nullptr;
+  p.copy_per_kv = a.copy_per_kv ? 1 : 0;
   auto launch = [&](int mode, int skip_empty) -> cudaError_t {
     p.mode = mode;
     p.skip_empty = skip_empty;
@@ -1264,8 +1349,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
     const long long work = skip_empty ? p.n_units : p.n_items;
     const long long cap = max_ctas > 0 && max_ctas < sm_count() ? max_ctas : sm_count();
     const long long grid = work < cap ? work : cap;
-    s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(tq, tqr, tk, tkr, tv,
-                                                                           tvr, to, p);
+    s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+        tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
     note_launch();
     return cudaGetLastError();
   };
@@ -1279,6 +1364,27 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
 }
 
 }  // namespace
+
+cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
+                                 cudaStream_t st) {
+  if (!a.kp || !a.vp || !flag || !a.sel_cnt || !a.perm_k) return cudaErrorInvalidValue;
+  const long long copy_rows = (a.copy_per_kv ? d.bhkv() : d.bhq()) * d.N;
+  k_copy_decide<<<1, 1024, 0, st>>>(a.sel_cnt, d.bhq() * d.nB, d.nB, mode, copy_rows / d.B, flag);
+  note_launch();
+  const unsigned grid = (unsigned)sm_count() * 8u;
+  if (d.D == 128)
+    k_permute_kv<128><<<grid, 256, 0, st>>>(
+        static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.perm_k,
+        static_cast<uint4 *>(const_cast<void *>(a.kp)), static_cast<uint4 *>(const_cast<void *>(a.vp)),
+        copy_rows, d.N, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0, flag);
+  else
+    k_permute_kv<64><<<grid, 256, 0, st>>>(
+        static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.perm_k,
+        static_cast<uint4 *>(const_cast<void *>(a.kp)), static_cast<uint4 *>(const_cast<void *>(a.vp)),
+        copy_rows, d.N, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0, flag);
+  note_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
                              int max_ctas, cudaStream_t st) {

@@ -42,9 +42,22 @@ struct AttnArgs {
   void *o;
   const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
   bool dense;
+  // Optional permuted copy of K and V: row rank of copy head h at h·N + rank holds the key/value
+  // row perm_k[head][rank]. The permuted pass loads its selected blocks from it (tile loads
+  // instead of row gathers) when *copy_flag is non-zero; copy_flag == nullptr means no copy.
+  // Copy heads are query heads, or KV heads when copy_per_kv is set (one key ordering per KV
+  // head).
+  const void *kp = nullptr, *vp = nullptr;
+  const uint32_t *copy_flag = nullptr;
+  bool copy_per_kv = false;
 };
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
                              int max_ctas, cudaStream_t st);
+// The permuted copy for the permuted pass: a decision kernel sets *flag when `mode` is 2, or when
+// it is 1 and the selected blocks outnumber twice the copied blocks; the copy kernel then fills
+// a.kp and a.vp (nothing when the flag is clear).
+cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
+                                 cudaStream_t st);
 
 // Host-side count of kernel launches made by the library (all threads, all devices).
 void note_launch();

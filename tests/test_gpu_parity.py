@@ -296,3 +296,80 @@ def test_attention_independent_of_grid_and_windows():
             assert torch.equal(d, dense), f"grid of {n}: dense output differs"
     finally:
         s2o.set_attention_max_ctas(0)
+
+
+# ----------------------------------------------------------------------------- permuted copy
+
+def _copy_flag(cfg, ws):
+    at = s2o.workspace_size(cfg)
+    return int(ws[at:at + 4].cpu().numpy().view(np.uint32)[0])
+
+
+@pytest.mark.parametrize("w", [W_A.replace(tau=0.0), W_C.replace(tau=0.0), W_D.replace(tau=0.0),
+                               W_F.replace(tau=0.0)], ids=lambda w: w.name)
+def test_permuted_copy_matches_gathers_and_oracle(w):
+    """Selected blocks loaded as tiles of the permuted copy of K and V give exactly the bits of
+    the row gathers (on the oracle's indices), and the oracle's result."""
+    q, k, v = inputs(w)
+    ocfg = oracle.config(w)
+    ref = oracle.build_indices(ocfg, q, k)
+    want, _ = oracle.attention(ocfg, q, k, v, ref)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w)
+    idx = oracle_indices_on_device(ref)
+    ws = s2o.alloc_prefill_workspace(cfg)
+    outs = {}
+    try:
+        for mode in (0, 2):
+            s2o.set_permuted_copy(mode)
+            outs[mode] = s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws)
+            torch.cuda.synchronize()
+            if mode == 2:
+                assert _copy_flag(cfg, ws) == 1
+    finally:
+        s2o.set_permuted_copy(1)
+    assert s2o.check_device_status() == 0
+    assert torch.equal(outs[0], outs[2])
+    assert_close(outs[2], want)
+
+
+def test_permuted_copy_decision():
+    """Mode 1 copies only when the selected blocks outnumber twice the copied blocks: with every
+    block selected (τ = 0) it copies, with none (τ > 1) it does not; a workspace of
+    s2o_workspace_size bytes never copies and gives the same output."""
+    for w, expect in ((W_A.replace(tau=0.0), 1), (W_A.replace(tau=1.5), 0)):
+        q, k, v = to_dev(*inputs(w))
+        cfg = s2o.Config.of(w)
+        idx = s2o.build_indices(cfg, q, k)
+        ws = s2o.alloc_prefill_workspace(cfg)
+        ws[s2o.workspace_size(cfg):s2o.workspace_size(cfg) + 4].fill_(7)
+        o = s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, ws)
+        torch.cuda.synchronize()
+        assert _copy_flag(cfg, ws) == expect, w.name
+        small = s2o.alloc_workspace(cfg)
+        o_small = s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, small)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_small)
+
+
+def test_permuted_copy_per_kv_head_under_shared_key_order():
+    """The whole path with one key ordering per KV head copies K and V once per KV head; the
+    output equals the gather path's bit for bit and the indices stay the oracle's."""
+    w = W_B.replace(tau=0.001, shared_key_order=1)
+    q, k, v = inputs(w)
+    ref = oracle.build_indices(oracle.config(w), q, k)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w)
+    ws = s2o.alloc_prefill_workspace(cfg)
+    outs = {}
+    try:
+        for mode in (0, 2):
+            s2o.set_permuted_copy(mode)
+            outs[mode], idx = s2o.attention_prefill(cfg, qd, kd, vd, ws=ws)
+            torch.cuda.synchronize()
+    finally:
+        s2o.set_permuted_copy(1)
+    assert s2o.check_device_status() == 0
+    assert int(idx.sel_cnt.sum()) > 0
+    assert_indices_equal(idx, ref, cfg.n_blocks)
+    assert torch.equal(outs[0], outs[2])
