@@ -138,17 +138,20 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
 
 /* Bytes of scratch with which s2o_attention_prefill and s2o_attention_prefill_with_indices_ws may
  * also make the permuted copy of K and V (see s2o_set_permuted_copy): s2o_workspace_size, a
- * 256-byte flag area, and the copy itself, 2 · copy_heads · N · d bf16 values with copy_heads =
- * batch · n_q_heads (batch · n_kv_heads for s2o_attention_prefill with shared_key_order = 1).
- * Written to *bytes. Host only; no device work. */
+ * 256-byte flag area, the copy itself (2 · copy_heads · N · d bf16 values with copy_heads =
+ * batch · n_q_heads; s2o_attention_prefill with shared_key_order = 1 uses only batch · n_kv_heads
+ * copy heads), and the block bitmaps and block-ordered lists of the selected blocks
+ * (batch · n_q_heads · nB · (ceil(nB/32) + 1 + nB) int32 values). Written to *bytes. Host only;
+ * no device work. */
 s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes);
 
 /* As s2o_attention_prefill_with_indices, with a workspace: when ws_bytes is at least
- * s2o_prefill_workspace_size (with shared_key_order treated as 0) and the permuted copy is on,
- * a device-side decision may copy K and V into each query head's key order first, and the
- * permuted pass then loads every selected block as one contiguous tile instead of gathering its
- * rows. The output is bit for bit the same as without the copy. With a smaller workspace this is
- * s2o_attention_prefill_with_indices. ws: device, 16-byte aligned, owned by the caller. */
+ * s2o_prefill_workspace_size and the permuted copy is on, a device-side decision may copy K and V
+ * into each query head's key order first, and the permuted pass then loads every selected block
+ * as one contiguous tile instead of gathering its rows (and, for dense selections, runs bitmap
+ * streams; see s2o_set_permuted_copy). The copy alone leaves the output bit for bit unchanged.
+ * With a smaller workspace this is s2o_attention_prefill_with_indices. ws: device, 16-byte
+ * aligned, owned by the caller. */
 s2o_status s2o_attention_prefill_with_indices_ws(const s2o_config *cfg, const void *q,
                                                  const void *k, const void *v,
                                                  const s2o_indices *idx, void *o, void *ws,
@@ -156,10 +159,16 @@ s2o_status s2o_attention_prefill_with_indices_ws(const s2o_config *cfg, const vo
 
 /* The permuted copy ([S2O, Summary ¶2] gathers the scattered rows by index; when most blocks are
  * selected, permuting K and V once in memory makes each selected block contiguous, so it loads
- * as one tile). mode 0: never; 1 (the default): when the selected blocks of the call outnumber
- * twice the blocks the copy writes (copying a block costs about one gather of it), decided on the
- * device without synchronising; 2: always (for tests). Only calls given a workspace of
- * s2o_prefill_workspace_size bytes make it. Affects calls made after it; not thread-safe against
+ * as one tile). With it, when the selected blocks are dense, the permuted pass can also run them
+ * in block order from bitmaps of the lists, so that two query blocks of one query head and
+ * segment load each block they both selected once (bitmap streams; the output is the attention
+ * over the same key sets, its fp32 accumulation in another order).
+ * mode 0: never; 1 (the default): decided on the device without synchronising, the copy when the
+ * selected blocks of the call outnumber twice the blocks the copy writes (copying a block costs
+ * about one gather of it), bitmap streams when they also fill at least an eighth of all pairs of
+ * query block and key block; 2: always the copy, never bitmap streams (output bit for bit that of
+ * the gathers; for tests); 3: always both (for tests). Only calls given a workspace of
+ * s2o_prefill_workspace_size bytes use them. Affects calls made after it; not thread-safe against
  * concurrent calls. Other values are treated as 1. */
 void s2o_set_permuted_copy(int mode);
 

@@ -381,7 +381,8 @@ def set_wait_limit_ns(ns: int) -> None:
 
 
 def set_permuted_copy(mode: int) -> None:
-    """Permuted copy of K/V for the permuted pass: 0 never, 1 when it pays (default), 2 always."""
+    """Permuted copy of K/V for the permuted pass: 0 never, 1 when it pays (default), 2 always
+    (list order, bit-identical output), 3 always with bitmap streams (block order)."""
     _load().s2o_set_permuted_copy(int(mode))
 
 

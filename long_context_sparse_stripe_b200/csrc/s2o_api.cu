@@ -61,6 +61,14 @@ s2o_status from_cuda(cudaError_t e) { return e == cudaSuccess ? S2O_OK : S2O_ERR
 size_t copy_bytes(const Dims &d, long long heads) {
   return align256((size_t)heads * (size_t)d.N * (size_t)d.D * 2);
 }
+// Bytes of the block bitmaps and of their counts.
+size_t bits_bytes(const Dims &d) {
+  return align256((size_t)d.bhq() * (size_t)d.nB * (size_t)((d.nB + 31) / 32) * 4);
+}
+size_t bitcnt_bytes(const Dims &d) { return align256((size_t)d.bhq() * (size_t)d.nB * 4); }
+size_t ord_bytes(const Dims &d) {
+  return align256((size_t)d.bhq() * (size_t)d.nB * (size_t)d.nB * 4);
+}
 constexpr size_t kFlagArea = 256;
 
 // Steps 3-4 with the optional permuted copy (copy heads: KV heads when per_kv, else query heads);
@@ -72,11 +80,15 @@ s2o_status attention_ws(const s2o_config &c, const void *q, const void *k, const
   AttnArgs a{q, k, v, o, idx.perm_q, idx.perm_k, idx.sel_cnt, idx.sel_blk, idx.local_tiles, false};
   const int mode = g_permuted_copy.load();
   const size_t base = ws_layout(d).total, cb = copy_bytes(d, per_kv ? d.bhkv() : d.bhq());
-  if (mode != 0 && ws && ws_bytes >= base + kFlagArea + 2 * cb) {
+  const size_t bb = bits_bytes(d), nb = bitcnt_bytes(d), ob = ord_bytes(d);
+  if (mode != 0 && ws && ws_bytes >= base + kFlagArea + 2 * cb + bb + nb + ob) {
     char *b = static_cast<char *>(ws);
     uint32_t *flag = reinterpret_cast<uint32_t *>(b + base);
     a.kp = b + base + kFlagArea;
     a.vp = b + base + kFlagArea + cb;
+    a.sel_bits = reinterpret_cast<uint32_t *>(b + base + kFlagArea + 2 * cb);
+    a.sel_bitcnt = reinterpret_cast<int32_t *>(b + base + kFlagArea + 2 * cb + bb);
+    a.sel_ord = reinterpret_cast<int32_t *>(b + base + kFlagArea + 2 * cb + bb + nb);
     a.copy_flag = flag;
     a.copy_per_kv = per_kv;
     const cudaError_t e = launch_permuted_copy(d, a, mode, flag, st);
@@ -318,11 +330,14 @@ s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes) {
   if (st != S2O_OK) return st;
   if (!bytes) return S2O_ERR_INVALID_ARGUMENT;
   const Dims d = dims_of(*cfg);
-  *bytes = ws_layout(d).total + kFlagArea + 2 * copy_bytes(d, d.bhq());
+  *bytes = ws_layout(d).total + kFlagArea + 2 * copy_bytes(d, d.bhq()) + bits_bytes(d) +
+           bitcnt_bytes(d) + ord_bytes(d);
   return S2O_OK;
 }
 
-void s2o_set_permuted_copy(int mode) { g_permuted_copy.store(mode == 0 || mode == 2 ? mode : 1); }
+void s2o_set_permuted_copy(int mode) {
+  g_permuted_copy.store(mode == 0 || mode == 2 || mode == 3 ? mode : 1);
+}
 
 void s2o_set_attention_max_ctas(int max_ctas) {
   g_attention_max_ctas.store(max_ctas > 0 ? max_ctas : 0);

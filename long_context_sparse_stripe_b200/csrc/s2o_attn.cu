@@ -314,38 +314,57 @@ struct Params {
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
   FastDiv div_G, div_seg, div_nB, div_nSeg, div_Hkv;  // unit-id decoding (S/B blocks a segment)
-  const uint32_t *copy_flag;  // permuted copy of K/V in use when non-null and set
+  const uint32_t *copy_flag;  // bit 0: the permuted copy of K/V is in use; bit 1: block bitmaps
   int copy_per_kv;            // copy rows per KV head (else per query head)
+  const uint32_t *sel_bits;   // per query block, nwords words: bit c set when block c is selected
+  const int32_t *sel_bitcnt;  // per query block, the bitmap's population count
+  const int32_t *sel_ord;     // per query block (nB entries): its selected blocks in block order
+  int nwords;
 };
 
 struct Unit {
   long long qh, kh;  // flat (batch, query head) and (batch, kv head)
   int b, seg0, lt, cnt;
-  const int32_t *sel;  // the query block's selected list (sel_blk row)
+  const int32_t *sel;  // the query block's selected list (sel_blk row; in block order for bitmap
+                       // streams)
 };
 
-// Unit order: the permuted and local modes keep the units of one (batch, KV head, segment)
+// Unit order: the local and permuted modes keep the units of one (batch, KV head, segment)
 // together, query heads of the group fastest, so that the segment's K/V tiles stay in L2 and
-// paired units share local tiles; the dense baseline runs the longest query blocks first.
-template <int BN>
+// paired units share local tiles; the dense baseline runs the longest query blocks first. With
+// bitmap streams (BITS) the permuted mode instead runs the blocks of one (batch, query head,
+// segment) in a row, so that the two units of a pair position read one key ordering and can share
+// the selected blocks they have in common; their list lengths and block-ordered lists then come
+// from the bitmap kernel.
+template <int BN, bool BITS>
 __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
   // Unit ids are below 2^31 (the host checks): divisions by multiply-high.
   Unit r;
   uint32_t rem;
-  u = p.div_G.divmod(u, rem);
-  const int hi = (int)rem;
-  int b, bl;  // block, and its index inside the segment
-  if (p.mode == kDense) {
-    u = p.div_nB.divmod(u, rem);
-    b = p.nB - 1 - (int)rem;
-    bl = b;
-    r.seg0 = 0;
-  } else {
+  int hi, b, bl;  // query head of the group, block, and the block's index inside its segment
+  if (BITS && p.mode == kPermuted) {
     u = p.div_seg.divmod(u, rem);
     bl = (int)rem;
     u = p.div_nSeg.divmod(u, rem);
     b = (int)rem * (int)p.div_seg.d + bl;
     r.seg0 = (int)rem * p.S;
+    u = p.div_G.divmod(u, rem);
+    hi = (int)rem;
+  } else {
+    u = p.div_G.divmod(u, rem);
+    hi = (int)rem;
+    if (p.mode == kDense) {
+      u = p.div_nB.divmod(u, rem);
+      b = p.nB - 1 - (int)rem;
+      bl = b;
+      r.seg0 = 0;
+    } else {
+      u = p.div_seg.divmod(u, rem);
+      bl = (int)rem;
+      u = p.div_nSeg.divmod(u, rem);
+      b = (int)rem * (int)p.div_seg.d + bl;
+      r.seg0 = (int)rem * p.S;
+    }
   }
   const uint32_t beta_u = p.div_Hkv.divmod(u, rem);
   const int g = (int)rem;
@@ -360,8 +379,13 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
   } else {
     const long long qb = r.qh * p.nB + b;
     r.lt = min(max(__ldg(p.local_tiles + qb), 1), (int)p.div_seg.d);
-    r.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
-    r.sel = p.sel_blk + qb * p.nB;
+    if (BITS) {
+      r.cnt = __ldg(p.sel_bitcnt + qb);
+      r.sel = p.sel_ord + qb * p.nB;
+    } else {
+      r.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
+      r.sel = p.sel_blk + qb * p.nB;
+    }
   }
   return r;
 }
@@ -370,29 +394,93 @@ struct Pair {
   Unit u0, u1;
   int valid1;  // the second unit exists (the last work item may hold one)
   int shared;  // both units read the same local key tiles
+  int uni;     // stream over the union of both units' selected blocks (bitmap streams)
   int L;       // local items of the stream
   int total;   // stream length
 };
 
-// Work item i of the current window: units list[2i] and list[2i+1] (the second may be absent).
-template <int BN>
+// Work item i of the current window: units list[2i] and list[2i+1] (the second may be absent:
+// past the list's end, or kNoUnit). With bitmap streams (BITS), a pair that reads one key
+// ordering and one segment (the same query head, or the same KV head when the key ordering is per
+// KV head) walks the union of its two bitmaps: a block both units selected is loaded once for
+// both. Its stream length then needs the union's size (union_size).
+constexpr uint32_t kNoUnit = 0xffffffffu;
+template <int BN, bool BITS>
 __device__ __forceinline__ Pair decode_pair(const Params &p, const uint32_t *list, int n_list,
                                             int i) {
   Pair P;
-  P.u0 = decode_unit<BN>(p, list[2 * i]);
-  P.valid1 = 2 * i + 1 < n_list;
+  P.u0 = decode_unit<BN, BITS>(p, list[2 * i]);
+  P.valid1 = 2 * i + 1 < n_list && (!BITS || list[2 * i + 1] != kNoUnit);
   if (P.valid1) {
-    P.u1 = decode_unit<BN>(p, list[2 * i + 1]);
+    P.u1 = decode_unit<BN, BITS>(p, list[2 * i + 1]);
   } else {
     P.u1 = P.u0;
     P.u1.lt = 0;
     P.u1.cnt = 0;
   }
   P.shared = P.valid1 && P.u0.kh == P.u1.kh && P.u0.seg0 == P.u1.seg0;
+  P.uni = BITS && P.shared && (P.u0.qh == P.u1.qh || p.copy_per_kv);
   P.L = P.shared ? max(P.u0.lt, P.u1.lt) : P.u0.lt + P.u1.lt;
   P.total = P.L + P.u0.cnt + P.u1.cnt;
   return P;
 }
+
+// A unit's block bitmap (bitmap streams).
+__device__ __forceinline__ const uint32_t *unit_bits(const Params &p, const Unit &u) {
+  return p.sel_bits + (u.qh * p.nB + u.b) * p.nwords;
+}
+
+// Blocks selected by either unit of a union pair (serial; or, with all 32 lanes, one word each).
+__device__ __forceinline__ int union_size(const Params &p, const Pair &P) {
+  const uint32_t *b0 = unit_bits(p, P.u0), *b1 = unit_bits(p, P.u1);
+  int n = 0;
+  for (int w = 0; w < p.nwords; ++w) n += __popc(__ldg(b0 + w) | __ldg(b1 + w));
+  return n;
+}
+__device__ __forceinline__ int union_size_warp(const Params &p, const Pair &P, int lane) {
+  const uint32_t *b0 = unit_bits(p, P.u0), *b1 = unit_bits(p, P.u1);
+  int n = 0;
+  for (int w = lane; w < p.nwords; w += 32) n += __popc(__ldg(b0 + w) | __ldg(b1 + w));
+  for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+  return n;
+}
+
+// The union of two block bitmaps in block order, with the units that selected each block; the
+// next words are loaded one word ahead.
+struct UnionCursor {
+  const uint32_t *r0, *r1;
+  int nwords, w;
+  uint32_t m0, m1, n0, n1;
+  __device__ __forceinline__ void init(const uint32_t *a, const uint32_t *b, int n) {
+    r0 = a;
+    r1 = b;
+    nwords = n;
+    w = 0;
+    m0 = n > 0 ? __ldg(a) : 0u;
+    m1 = n > 0 ? __ldg(b) : 0u;
+    n0 = n > 1 ? __ldg(a + 1) : 0u;
+    n1 = n > 1 ? __ldg(b + 1) : 0u;
+  }
+  __device__ __forceinline__ int next(int &users) {
+    while ((m0 | m1) == 0) {
+      if (++w >= nwords) {
+        users = 0;
+        return -1;
+      }
+      m0 = n0;
+      m1 = n1;
+      n0 = w + 1 < nwords ? __ldg(r0 + w + 1) : 0u;
+      n1 = w + 1 < nwords ? __ldg(r1 + w + 1) : 0u;
+    }
+    const int i = __ffs(m0 | m1) - 1;
+    const uint32_t bit = 1u << i;
+    users = ((m0 & bit) ? 1 : 0) | ((m1 & bit) ? 2 : 0);
+    m0 &= ~bit;
+    m1 &= ~bit;
+    return 32 * w + i;
+  }
+};
+
 
 // Position j of a two-way interleaving of a items of unit 0 and b items of unit 1 (alternating
 // while both have items left): the unit x and its item index.
@@ -600,34 +688,58 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // past the end of the share). Without skipping, the share is the work items w = blockIdx.x +
 // k·gridDim.x, each contributing its units 2w and 2w+1 (adjacent units, which usually share
 // local tiles); with skip_empty it is the units u = blockIdx.x + k·gridDim.x whose selected list
-// is not empty, paired in list order.
-template <int BN>
+// is not empty, paired in list order. With bitmap streams (BITS; always skip_empty) the share is
+// again the work items w, each contributing those of its units 2w and 2w+1 whose list is not
+// empty (the second slot kNoUnit when only one is), so that a pair is two consecutive blocks of
+// one query head.
+template <int BN, bool BITS>
 __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lane) {
-  const long long span = p.skip_empty ? kList : kList / 2;
+  const bool by_unit = p.skip_empty && !BITS;
+  const long long span = by_unit ? kList : kList / 2;
   const long long first = blockIdx.x + k0 * gridDim.x;
-  if (first >= (p.skip_empty ? p.n_units : p.n_items)) return -1;
+  if (first >= (by_unit ? p.n_units : p.n_items)) return -1;
+  // Whether unit u (permuted-mode order) has a non-empty selected list.
+  auto busy = [&](long long u) -> bool {
+    if (u >= p.n_units || !p.sel_cnt) return false;
+    const int per_seg = p.S / BN;
+    int hi, bl, sg;
+    if (BITS) {
+      bl = (int)(u % per_seg);
+      u /= per_seg;
+      sg = (int)(u % p.nSeg);
+      u /= p.nSeg;
+      hi = (int)(u % p.G);
+      u /= p.G;
+    } else {
+      hi = (int)(u % p.G);
+      u /= p.G;
+      bl = (int)(u % per_seg);
+      u /= per_seg;
+      sg = (int)(u % p.nSeg);
+      u /= p.nSeg;
+    }
+    const int g = (int)(u % p.Hkv);
+    const long long qh = (u / p.Hkv) * p.Hq + (long long)g * p.G + hi;
+    return __ldg(p.sel_cnt + qh * p.nB + sg * per_seg + bl) > 0;
+  };
   int n = 0;
   for (long long k = k0; k < k0 + span; k += 32) {
     const long long pos = blockIdx.x + (k + lane) * gridDim.x;
-    if (p.skip_empty) {
-      bool keep = false;
-      if (pos < p.n_units && p.sel_cnt) {
-        // The unit's (query head, block) in permuted-mode order, then its list length.
-        long long u = pos;
-        const int hi = (int)(u % p.G);
-        u /= p.G;
-        const int per_seg = p.S / BN;
-        const int bl = (int)(u % per_seg);
-        u /= per_seg;
-        const int sg = (int)(u % p.nSeg);
-        u /= p.nSeg;
-        const int g = (int)(u % p.Hkv);
-        const long long qh = (u / p.Hkv) * p.Hq + (long long)g * p.G + hi;
-        keep = __ldg(p.sel_cnt + qh * p.nB + sg * per_seg + bl) > 0;
-      }
+    if (by_unit) {
+      const bool keep = busy(pos);
       const unsigned m = __ballot_sync(0xffffffffu, keep);
       if (keep) list[n + __popc(m & ((1u << lane) - 1u))] = (uint32_t)pos;
       n += __popc(m);
+    } else if (BITS) {
+      const bool b0 = pos < p.n_items && busy(2 * pos), b1 = pos < p.n_items && busy(2 * pos + 1);
+      const bool keep = b0 || b1;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int at = n + 2 * __popc(m & ((1u << lane) - 1u));
+        list[at] = (uint32_t)(b0 ? 2 * pos : 2 * pos + 1);
+        list[at + 1] = b0 && b1 ? (uint32_t)(2 * pos + 1) : kNoUnit;
+      }
+      n += 2 * __popc(m);
     } else {
       const bool keep = pos < p.n_items;
       const bool two = 2 * pos + 1 < p.n_units;
@@ -647,7 +759,10 @@ __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lan
 
 // ------------------------------------------------------------------ the kernel
 
-template <int D, int BN>
+// BITS: the permuted pass with bitmap streams. A launch given block bitmaps (sel_bits) runs only
+// if the decision flag chose bitmap streams (BITS) or did not (!BITS): the host launches both
+// and one returns at once.
+template <int D, int BN, bool BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     s2o_attention_kernel(const __grid_constant__ CUtensorMap tm_q_tile,
                          const __grid_constant__ CUtensorMap tm_q_row,
@@ -659,6 +774,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_kp_tile,
                          const __grid_constant__ CUtensorMap tm_vp_tile, const Params p) {
   using L = Layout<D, BN>;
+  if (p.mode == kPermuted && p.sel_bits != nullptr &&
+      ((__ldg(p.copy_flag) & 3u) == 3u) != BITS)
+    return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -713,16 +831,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint64_t lim = p.limit_ns;
   bool ok = true;
+  // Set before the launch by the permuted-copy decision: selected blocks come from the permuted
+  // copy (bit 0), in block order from the block bitmaps (bit 1, only with bit 0).
+  const bool use_copy = p.copy_flag != nullptr && (__ldg(p.copy_flag) & 1u) != 0u;
   // Work comes in windows of this CTA's share: warp 0 fills the work list between two CTA-wide
   // barriers and every role then walks the window's items (a role that gave up a bounded wait
   // keeps meeting the barriers without working).
   uint32_t *list = reinterpret_cast<uint32_t *>(smem + L::OFF_LIST);
   volatile int *list_n = reinterpret_cast<volatile int *>(smem + L::OFF_LIST + kList * 4);
   auto for_each_window = [&](auto &&body) {
-    for (long long k0 = 0;; k0 += p.skip_empty ? kList : kList / 2) {
+    for (long long k0 = 0;; k0 += p.skip_empty && !BITS ? kList : kList / 2) {
       named_bar_sync(1, kThreads);
       if (warp == 0) {
-        const int n = build_list<BN>(p, k0, list, lane);
+        const int n = build_list<BN, BITS>(p, k0, list, lane);
         if (lane == 0) *list_n = n;
         __syncwarp();
       }
@@ -743,12 +864,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CUtensorMap *tm_tile = is_k ? &tm_k_tile : &tm_v_tile;
     const CUtensorMap *tm_row = is_k ? &tm_k_row : &tm_v_row;
     const CUtensorMap *tm_copy = is_k ? &tm_kp_tile : &tm_vp_tile;
-    // Selected blocks come from the permuted copy when the launch has one and its flag is set.
-    const bool use_copy = p.copy_flag != nullptr && __ldg(p.copy_flag) != 0u;
     long long kj = 0;  // stream items issued so far (all work items of this CTA)
+    // One stream item into the next ring stage.
+    auto issue = [&](const Pair &P, const Item &it, int4 rows, int c) -> bool {
+      const int st = (int)(kj % stages);
+      if (kj >= stages &&
+          !warp_wait(bar(empty0 + st), (uint32_t)(((kj / stages) - 1) & 1), lim, lane))
+        return false;
+      if (lane == 0) mbar_expect_tx(bar(full0 + st), L::KV_BYTES);
+      __syncwarp();
+      load_kv<D, BN>(ring + st * L::KV_BYTES, tm_tile, tm_row, tm_copy, p, P, it, rows, c,
+                     use_copy, bar(full0 + st), lane);
+      ++kj;
+      return true;
+    };
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      const Pair P = decode_pair<BN>(p, list, n_list, wi);
+      Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
+      if (BITS && P.uni) {
+        // Union stream: local tiles, then each block either unit selected, once, from the
+        // permuted copy.
+        P.total = P.L + union_size_warp(p, P, lane);
+        UnionCursor uc;
+        uc.init(unit_bits(p, P.u0), unit_bits(p, P.u1), p.nwords);
+        for (int j = 0; ok && j < P.total; ++j) {
+          Item it;
+          int c = -1;
+          if (j < P.L) {
+            it = item_at(P, j);
+          } else {
+            c = uc.next(it.users);
+            it.x = 0;
+            it.local = 0;
+            it.t = 0;
+          }
+          ok = issue(P, it, make_int4(0, 0, 0, 0), c);
+        }
+        continue;
+      }
       // Gathered rows are looked up ahead: the rows of item j+1 and the block of item j+2 are
       // requested before item j waits for its ring stage, so the dependent index loads are off
       // the critical path.
@@ -771,18 +924,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_this = c_cur;
         c_cur = c_next;
         c_next = block_of(j + 2);
-        const int st = (int)(kj % stages);
-        if (kj >= stages &&
-            !warp_wait(bar(empty0 + st), (uint32_t)(((kj / stages) - 1) & 1), lim, lane)) {
+        if (!issue(P, it, rows, c_this)) {
           ok = false;
           break;
         }
-        if (lane == 0) mbar_expect_tx(bar(full0 + st), L::KV_BYTES);
-        __syncwarp();
-        load_kv<D, BN>(ring + st * L::KV_BYTES, tm_tile, tm_row, tm_copy, p, P, it, rows, c_this,
-                       use_copy, bar(full0 + st), lane);
         rows = rows_next;
-        ++kj;
       }
     }
     });
@@ -794,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long qn[2] = {0, 0};
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      const Pair P = decode_pair<BN>(p, list, n_list, wi);
+      const Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
       for (int x = 0; ok && x < 1 + P.valid1; ++x) {
         if (qn[x] >= 1 &&
             !warp_wait(bar(kQEmpty + x), (uint32_t)((qn[x] - 1) & 1), lim, lane)) {
@@ -917,7 +1063,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
       if (lane == 0) {
       for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-        const Pair P = decode_pair<BN>(p, list, n_list, wi);
+        Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
+        // A union stream's selected part is walked once, item by item, for its users.
+        UnionCursor uc;
+        if (BITS && P.uni) {
+          P.total = P.L + union_size(p, P);
+          uc.init(unit_bits(p, P.u0), unit_bits(p, P.u1), p.nwords);
+        }
+        auto users_seq = [&](int j) -> int {
+          if (!BITS || !P.uni || j < P.L || j >= P.total) return users_at(P, j);
+          int us;
+          uc.next(us);
+          return us;
+        };
         const int n_of[2] = {P.u0.lt + P.u0.cnt, P.u1.lt + P.u1.cnt};
         int qk[2] = {0, 0};
         // One unit's step at stream item j: its pending product goes first, or now if the unit
@@ -940,9 +1098,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           return true;
         };
-        int users = users_at(P, 0);
+        int users = users_seq(0);
         for (int j = 0; j < P.total; ++j) {
-          const int nusers = users_at(P, j + 1);
+          const int nusers = users_seq(j + 1);
           if (!mbar_wait(bar(kKFull + k_st), k_ph, lim)) {
             ok = false;
             break;
@@ -995,7 +1153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long sn = 0, on = 0;  // S_x tiles and work items consumed
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      const Pair P = decode_pair<BN>(p, list, n_list, wi);
+      const Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
       if (x == 1 && !P.valid1) continue;
       const Unit u = x ? P.u1 : P.u0;
       const int seg0 = u.seg0;
@@ -1208,10 +1366,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // ------------------------------------------------------------------ permuted copy of K and V
 
-// Whether the permuted pass uses the permuted copy: always (mode 2), or (mode 1) when the
-// selected blocks of all query blocks outnumber twice the blocks the copy writes; copying a
-// block costs about one gather of it, and each selected block then loads as a contiguous tile.
-// One CTA.
+// Whether the permuted pass uses the permuted copy (bit 0): always (modes 2 and 3), or (mode 1)
+// when the selected blocks of all query blocks outnumber twice the blocks the copy writes; copying
+// a block costs about one gather of it, and each selected block then loads as a contiguous tile.
+// Whether it also runs bitmap streams (bit 1): always in mode 3, or (mode 1, with the copy) when
+// the selected blocks fill at least an eighth of all pairs of query block and key block, so that
+// the bitmaps are dense enough to walk word by word. One CTA.
 __global__ void __launch_bounds__(1024)
     k_copy_decide(const int32_t *__restrict__ sel_cnt, long long n_units, int nB, int mode,
                   long long copy_blocks, uint32_t *__restrict__ flag) {
@@ -1225,8 +1385,55 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) {
     unsigned long long total = 0;
     for (int w = 0; w < (int)(blockDim.x / 32); ++w) total += part[w];
-    *flag = (mode == 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks)) ? 1u : 0u;
+    const bool copy =
+        mode >= 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks);
+    const bool dense = mode == 3 || (mode == 1 && copy &&
+                                     total >= (unsigned long long)n_units * (unsigned long long)nB / 8);
+    *flag = (copy ? 1u : 0u) | (dense ? 2u : 0u);
   }
+}
+
+// Block bitmaps of the selected lists (flag bit 1 only): one warp per query block sets bit c of
+// word c/32 for each listed block c (clamped into range), then writes the bitmap, its population
+// count and the selected blocks in block order (each lane the set bits of its words, after the
+// blocks of the words before them).
+__global__ void __launch_bounds__(256)
+    k_sel_bits(const int32_t *__restrict__ sel_cnt, const int32_t *__restrict__ sel_blk,
+               long long n_units, int nB, int nwords, const uint32_t *__restrict__ flag,
+               uint32_t *__restrict__ bits, int32_t *__restrict__ bitcnt,
+               int32_t *__restrict__ ord) {
+  if ((__ldg(flag) & 2u) == 0u) return;
+  __shared__ uint32_t sw[8][64];
+  const unsigned full = 0xffffffffu;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long long qb = (long long)blockIdx.x * 8 + warp;
+  if (qb >= n_units) return;
+  for (int w = lane; w < nwords; w += 32) sw[warp][w] = 0u;
+  __syncwarp();
+  const int cnt = min(max(__ldg(sel_cnt + qb), 0), nB);
+  const int32_t *row = sel_blk + qb * nB;
+  for (int e = lane; e < cnt; e += 32) {
+    const int c = min(max(__ldg(row + e), 0), nB - 1);
+    atomicOr(&sw[warp][c >> 5], 1u << (c & 31));
+  }
+  __syncwarp();
+  int32_t *ord_row = ord + qb * nB;
+  int run = 0;
+  for (int w0 = 0; w0 < nwords; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t v = w < nwords ? sw[warp][w] : 0u;
+    const int pc = __popc(v);
+    int incl = pc;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int at = run + incl - pc;
+    for (uint32_t m = v; m; m &= m - 1) ord_row[at++] = 32 * w + __ffs(m) - 1;
+    if (w < nwords) bits[qb * nwords + w] = v;
+    run += __shfl_sync(full, incl, 31);
+  }
+  if (lane == 0) bitcnt[qb] = run;
 }
 
 // kp[h·N + rank] = K row perm_k[hq(h)][rank] of h's KV head, and the same for V (h a query head,
@@ -1313,9 +1520,13 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
     tkp = tk;
     tvp = tv;
   }
-  cudaError_t e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN>,
+  cudaError_t e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
   if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM)) !=
+      cudaSuccess)
+    return e;
   Params p;
   p.perm_q = a.perm_q;
   p.perm_k = a.perm_k;
@@ -1339,28 +1550,39 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   p.div_Hkv.init(d.Hkv);
   p.copy_flag = copy ? a.copy_flag : nullptr;
   p.copy_per_kv = a.copy_per_kv ? 1 : 0;
-  auto launch = [&](int mode, int skip_empty) -> cudaError_t {
+  const bool bitmaps = copy && a.sel_bits && a.sel_bitcnt && a.sel_ord;
+  p.sel_bits = bitmaps ? a.sel_bits : nullptr;
+  p.sel_bitcnt = bitmaps ? a.sel_bitcnt : nullptr;
+  p.sel_ord = bitmaps ? a.sel_ord : nullptr;
+  p.nwords = (d.nB + 31) / 32;
+  auto launch = [&](int mode, int skip_empty, bool bits) -> cudaError_t {
     p.mode = mode;
     p.skip_empty = skip_empty;
     p.S = mode == kDense ? d.N : d.S;
     p.nSeg = mode == kDense ? 1 : d.nSeg;
     p.div_seg.init(p.S / BN);
     p.div_nSeg.init(p.nSeg);
-    const long long work = skip_empty ? p.n_units : p.n_items;
+    const long long work = skip_empty && !bits ? p.n_units : p.n_items;
     const long long cap = max_ctas > 0 && max_ctas < sm_count() ? max_ctas : sm_count();
     const long long grid = work < cap ? work : cap;
-    s2o_attention_kernel<D, BN><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
-        tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+    if (bits)
+      s2o_attention_kernel<D, BN, true><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+          tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+    else
+      s2o_attention_kernel<D, BN, false><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+          tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
     note_launch();
     return cudaGetLastError();
   };
-  if (a.dense) return launch(kDense, 0);
+  if (a.dense) return launch(kDense, 0, false);
   // S2O: every row first gets the dense local window of its segment, computed in original order
   // (causal triangles, masks on diagonal tiles only); then the query blocks whose selected list is
   // not empty are recomputed in full (local tiles and selected blocks, permuted order) and
-  // overwrite their rows. Each row's result is the attention over its key set either way.
-  if ((e = launch(kLocal, 0)) != cudaSuccess) return e;
-  return launch(kPermuted, 1);
+  // overwrite their rows. Each row's result is the attention over its key set either way. With
+  // block bitmaps the permuted pass is launched in both forms and the device flag picks one.
+  if ((e = launch(kLocal, 0, false)) != cudaSuccess) return e;
+  if ((e = launch(kPermuted, 1, false)) != cudaSuccess) return e;
+  return p.sel_bits != nullptr ? launch(kPermuted, 1, true) : cudaSuccess;
 }
 
 }  // namespace
@@ -1371,6 +1593,13 @@ cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uin
   const long long copy_rows = (a.copy_per_kv ? d.bhkv() : d.bhq()) * d.N;
   k_copy_decide<<<1, 1024, 0, st>>>(a.sel_cnt, d.bhq() * d.nB, d.nB, mode, copy_rows / d.B, flag);
   note_launch();
+  if (a.sel_bits && a.sel_bitcnt && a.sel_ord) {
+    const long long n_units = d.bhq() * d.nB;
+    k_sel_bits<<<(unsigned)((n_units + 7) / 8), 256, 0, st>>>(
+        a.sel_cnt, a.sel_blk, n_units, d.nB, (d.nB + 31) / 32, flag, a.sel_bits, a.sel_bitcnt,
+        const_cast<int32_t *>(a.sel_ord));
+    note_launch();
+  }
   const unsigned grid = (unsigned)sm_count() * 8u;
   if (d.D == 128)
     k_permute_kv<128><<<grid, 256, 0, st>>>(

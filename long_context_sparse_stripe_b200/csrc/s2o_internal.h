@@ -50,12 +50,21 @@ struct AttnArgs {
   const void *kp = nullptr, *vp = nullptr;
   const uint32_t *copy_flag = nullptr;
   bool copy_per_kv = false;
+  // Block bitmaps of the selected lists (ceil(nB/32) words per query block), their population
+  // counts and the selected blocks in block order (nB entries per query block), filled when the
+  // decision also sets the flag's bit 1; the permuted pass then runs the selected blocks in block
+  // order and shares the blocks two paired query blocks both selected.
+  uint32_t *sel_bits = nullptr;
+  int32_t *sel_bitcnt = nullptr;
+  const int32_t *sel_ord = nullptr;  // per query block: its selected blocks in block order
 };
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
                              int max_ctas, cudaStream_t st);
-// The permuted copy for the permuted pass: a decision kernel sets *flag when `mode` is 2, or when
-// it is 1 and the selected blocks outnumber twice the copied blocks; the copy kernel then fills
-// a.kp and a.vp (nothing when the flag is clear).
+// The permuted copy for the permuted pass: a decision kernel sets bit 0 of *flag when `mode` is 2
+// or 3, or when it is 1 and the selected blocks outnumber twice the copied blocks, and bit 1 (block
+// bitmaps) when `mode` is 3, or when it is 1, bit 0 is set and the selected blocks fill at least an
+// eighth of all (query block, key block) pairs; the copy kernel then fills a.kp and a.vp and the
+// bitmap kernel a.sel_bits, a.sel_bitcnt and a.sel_ord (each does nothing when its bit is clear).
 cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
                                  cudaStream_t st);
 

@@ -306,10 +306,12 @@ def _copy_flag(cfg, ws):
 
 
 @pytest.mark.parametrize("w", [W_A.replace(tau=0.0), W_C.replace(tau=0.0), W_D.replace(tau=0.0),
-                               W_F.replace(tau=0.0)], ids=lambda w: w.name)
+                               W_F.replace(tau=0.0), W_A.replace(tau=0.01)],
+                         ids=lambda w: f"{w.name}-tau{w.tau}")
 def test_permuted_copy_matches_gathers_and_oracle(w):
     """Selected blocks loaded as tiles of the permuted copy of K and V give exactly the bits of
-    the row gathers (on the oracle's indices), and the oracle's result."""
+    the row gathers (mode 2, on the oracle's indices); bitmap streams (mode 3: block order, the
+    blocks two paired query blocks share loaded once) give the oracle's result."""
     q, k, v = inputs(w)
     ocfg = oracle.config(w)
     ref = oracle.build_indices(ocfg, q, k)
@@ -320,24 +322,26 @@ def test_permuted_copy_matches_gathers_and_oracle(w):
     ws = s2o.alloc_prefill_workspace(cfg)
     outs = {}
     try:
-        for mode in (0, 2):
+        for mode, flag in ((0, None), (2, 1), (3, 3)):
             s2o.set_permuted_copy(mode)
             outs[mode] = s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws)
             torch.cuda.synchronize()
-            if mode == 2:
-                assert _copy_flag(cfg, ws) == 1
+            if flag is not None:
+                assert _copy_flag(cfg, ws) == flag
     finally:
         s2o.set_permuted_copy(1)
     assert s2o.check_device_status() == 0
     assert torch.equal(outs[0], outs[2])
     assert_close(outs[2], want)
+    assert_close(outs[3], want)
 
 
 def test_permuted_copy_decision():
-    """Mode 1 copies only when the selected blocks outnumber twice the copied blocks: with every
-    block selected (τ = 0) it copies, with none (τ > 1) it does not; a workspace of
-    s2o_workspace_size bytes never copies and gives the same output."""
-    for w, expect in ((W_A.replace(tau=0.0), 1), (W_A.replace(tau=1.5), 0)):
+    """Mode 1 copies only when the selected blocks outnumber twice the copied blocks, and runs
+    bitmap streams only when they also fill an eighth of the block pairs: with every block
+    selected (τ = 0) it does both, with none (τ > 1) neither; a workspace of s2o_workspace_size
+    bytes never copies and gives the same output."""
+    for w, expect in ((W_A.replace(tau=0.0), 3), (W_A.replace(tau=1.5), 0)):
         q, k, v = to_dev(*inputs(w))
         cfg = s2o.Config.of(w)
         idx = s2o.build_indices(cfg, q, k)
@@ -346,24 +350,27 @@ def test_permuted_copy_decision():
         o = s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, ws)
         torch.cuda.synchronize()
         assert _copy_flag(cfg, ws) == expect, w.name
-        small = s2o.alloc_workspace(cfg)
-        o_small = s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, small)
-        torch.cuda.synchronize()
-        assert torch.equal(o, o_small)
+        if expect == 0:
+            small = s2o.alloc_workspace(cfg)
+            o_small = s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, small)
+            torch.cuda.synchronize()
+            assert torch.equal(o, o_small)
 
 
 def test_permuted_copy_per_kv_head_under_shared_key_order():
-    """The whole path with one key ordering per KV head copies K and V once per KV head; the
-    output equals the gather path's bit for bit and the indices stay the oracle's."""
+    """The whole path with one key ordering per KV head copies K and V once per KV head: the copy
+    alone (mode 2) equals the gather path bit for bit, bitmap streams (mode 3) agree with it
+    within the parity tolerance on sampled rows, and the indices stay the oracle's."""
     w = W_B.replace(tau=0.001, shared_key_order=1)
     q, k, v = inputs(w)
-    ref = oracle.build_indices(oracle.config(w), q, k)
+    ocfg = oracle.config(w)
+    ref = oracle.build_indices(ocfg, q, k)
     qd, kd, vd = to_dev(q, k, v)
     cfg = s2o.Config.of(w)
     ws = s2o.alloc_prefill_workspace(cfg)
     outs = {}
     try:
-        for mode in (0, 2):
+        for mode in (0, 2, 3):
             s2o.set_permuted_copy(mode)
             outs[mode], idx = s2o.attention_prefill(cfg, qd, kd, vd, ws=ws)
             torch.cuda.synchronize()
@@ -373,3 +380,8 @@ def test_permuted_copy_per_kv_head_under_shared_key_order():
     assert int(idx.sel_cnt.sum()) > 0
     assert_indices_equal(idx, ref, cfg.n_blocks)
     assert torch.equal(outs[0], outs[2])
+    rng = np.random.default_rng(1)
+    rows = rng.choice(w.batch * w.n_q_heads * w.seq_len, 1500, replace=False)
+    want, _ = oracle.attention(ocfg, q, k, v, ref, rows=np.sort(rows))
+    got = outs[3].reshape(-1, w.head_dim)[torch.from_numpy(np.sort(rows)).cuda()]
+    assert_close(got, want)
