@@ -484,6 +484,68 @@ def run_sweep(args):
     return 0
 
 
+def run_layer(args):
+    """End-to-end-shaped prefill (not the headline line): one Llama-3.1-8B-shaped decoder layer
+    with random weights at the bench workload's attention shape, S2O attention against the dense
+    causal baseline, CUDA events. A 32-layer prefill is 32 such layers (embedding and output head
+    left out). One JSON line on stdout."""
+    import long_context_sparse_stripe_b200 as s2o
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = gen.workload(args.workload, tau=args.tau)
+    shape = gen.LAYER_8B
+    host = gen.make_layer(w, shape)
+    wts = {k: v.to(dev) for k, v in host.items()}
+    x0 = wts.pop("x")
+    cfg = s2o.Config.of(w)
+    H, I, rows = w.n_q_heads * w.head_dim, shape.intermediate, w.batch * w.seq_len
+    qkvw = (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim
+    gemm_flops = 2.0 * rows * (H * qkvw + H * H + H * 2 * I + I * H)
+    peak = measured_peaks()[0]
+    out = {}
+    for dense in (False, True):
+        ws = torch.empty(s2o.layer_workspace_size(cfg, shape, dense), dtype=torch.uint8,
+                         device=dev)
+        x = torch.empty_like(x0)
+        reps = 3
+        for _ in range(1):
+            x.copy_(x0)
+            s2o.layer_prefill(cfg, shape, wts, x, ws=ws, dense=dense)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # the copy that restores x each repetition is timed on its own and subtracted
+        c0.record()
+        for _ in range(reps):
+            x.copy_(x0)
+        c1.record()
+        e0.record()
+        for _ in range(reps):
+            x.copy_(x0)
+            s2o.layer_prefill(cfg, shape, wts, x, ws=ws, dense=dense)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = (e0.elapsed_time(e1) - c0.elapsed_time(c1)) / reps
+        out["dense" if dense else "s2o"] = ms
+        del ws
+        torch.cuda.empty_cache()
+    attn_dense = w.dense_causal_flops
+    line = {"layer": {
+        "workload": w.name, "tau": w.tau, "hidden": H, "intermediate": I,
+        "weights": "random N(0, 1/fan_in), seeded", "status": s2o.check_device_status(dev),
+        "s2o_layer_ms": out["s2o"], "dense_layer_ms": out["dense"],
+        "e2e_speedup_vs_dense_attention": out["dense"] / out["s2o"],
+        "projection_tflop_per_layer": gemm_flops / 1e12,
+        "dense_attention_tflop_per_layer": attn_dense / 1e12,
+        "dense_layer_tflops": (gemm_flops + attn_dense) / (out["dense"] * 1e-3) / 1e12,
+        "prefill_32_layers_ms": {"s2o": 32 * out["s2o"], "dense": 32 * out["dense"]},
+        "peak_bf16_tflops": peak,
+    }}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_profile_target(args):
     """A short fixed sequence for profiler captures (not a bench line): one index build, then
     `--steps` attention calls (each a local pass and a permuted pass) and one dense-baseline call."""
@@ -524,6 +586,8 @@ def main():
                     help="profile target only: 'Hq,Hkv' (the first KV groups of the workload)")
     ap.add_argument("--sweep", action="store_true",
                     help="per-configuration report (one JSON line per configuration)")
+    ap.add_argument("--layer", action="store_true",
+                    help="end-to-end-shaped decoder layer, S2O vs dense attention (one JSON line)")
     ap.add_argument("--profile-target", action="store_true",
                     help="run a short fixed call sequence for profiler captures; print nothing")
     args = ap.parse_args()
@@ -533,6 +597,8 @@ def main():
         return run_profile_target(args)
     if args.sweep:
         return run_sweep(args)
+    if args.layer:
+        return run_layer(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_s2o(args)

@@ -30,7 +30,7 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "workload"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "workload", "LayerShape", "LAYER_8B", "make_layer"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -151,3 +151,71 @@ def make_inputs(w: Workload, threads: int | None = None, keep_fp32: bool = False
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The raw bf16 bit patterns of a CPU bf16 tensor as a uint16 numpy array (no copy)."""
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------ decoder layer (random weights)
+
+@dataclasses.dataclass(frozen=True)
+class LayerShape:
+    """The non-attention sizes of a Llama-3.1-8B-shaped decoder layer (the attention shape comes
+    from the Workload: hidden = n_q_heads · head_dim)."""
+    intermediate: int = 14336
+    rms_eps: float = 1e-5
+    rope_theta: float = 500000.0
+    rope_factor: float = 8.0
+    rope_low_freq_factor: float = 1.0
+    rope_high_freq_factor: float = 4.0
+    rope_original_context: int = 8192
+
+    def replace(self, **kw) -> "LayerShape":
+        return dataclasses.replace(self, **kw)
+
+
+LAYER_8B = LayerShape()
+
+
+def make_layer(w: Workload, shape: LayerShape = LAYER_8B, seed: int | None = None,
+               threads: int | None = None) -> dict:
+    """Random weights and input rows of one decoder layer, as CPU bf16 tensors.
+
+    x [batch, N, H] ~ N(0, 1); each projection W [fan_in, fan_out] ~ N(0, 1/fan_in); norm gains
+    ~ N(1, 0.1²). Every tensor is drawn in 1024-row chunks, chunk c of tensor t from
+    ``SeedSequence(seed, spawn_key=(100 + t, c))`` (seed defaults to the workload's), then rounded
+    to bf16 (nearest-even).
+    """
+    seed = w.seed if seed is None else seed
+    threads = threads or min(32, os.cpu_count() or 1)
+    H = w.n_q_heads * w.head_dim
+    qkv = (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim
+    I = shape.intermediate
+    specs = [  # name, shape (rows, cols), mean, std
+        ("x", (w.batch * w.seq_len, H), 0.0, 1.0),
+        ("attn_norm", (1, H), 1.0, 0.1),
+        ("w_qkv", (H, qkv), 0.0, H ** -0.5),
+        ("w_o", (H, H), 0.0, H ** -0.5),
+        ("mlp_norm", (1, H), 1.0, 0.1),
+        ("w_gu", (H, 2 * I), 0.0, H ** -0.5),
+        ("w_down", (I, H), 0.0, I ** -0.5),
+    ]
+    out = {}
+    jobs = []
+    for t, (name, (rows, cols), mean, std) in enumerate(specs):
+        bits = np.empty((rows, cols), np.uint16)
+        out[name] = bits
+        for c, r0 in enumerate(range(0, rows, 1024)):
+            jobs.append((t, c, bits, r0, min(rows, r0 + 1024), cols, mean, std))
+
+    def job(j):
+        t, c, bits, r0, r1, cols, mean, std = j
+        x = _stream(seed, 100 + t, c).standard_normal((r1 - r0, cols), dtype=np.float32)
+        x *= np.float32(std)
+        x += np.float32(mean)
+        bits[r0:r1] = _to_bf16_bits(x)
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(job, jobs))
+    res = {k: torch.from_numpy(v).view(torch.bfloat16) for k, v in out.items()}
+    res["x"] = res["x"].reshape(w.batch, w.seq_len, H)
+    res["attn_norm"] = res["attn_norm"].reshape(H)
+    res["mlp_norm"] = res["mlp_norm"].reshape(H)
+    return res

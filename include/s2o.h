@@ -232,6 +232,46 @@ s2o_status s2o_check_device_status(s2o_stream stream);
 s2o_status s2o_build_indices_static(const s2o_config *cfg, const void *q, const void *k,
                                     const s2o_indices *out, s2o_stream stream);
 
+/* ---- Decoder layer around the attention (end-to-end-shaped prefill with random weights) ----
+ * The pages measure S2O inside Llama-3.1-8B ([S2O, Key points]: end-to-end speedup at 128K);
+ * without trained weights this runs one Llama-3-architecture decoder layer with the S2O prefill
+ * (or the dense causal baseline) as its attention: x += W_o·attn(RoPE(W_qkv·norm(x))), then
+ * x += W_down·(silu(gate)·up) with [gate | up] = W_gu·norm(x). bf16 storage between the steps,
+ * fp32 arithmetic; projections are cuBLAS GEMMs (bf16 in, fp32 accumulation), the rest this
+ * library's kernels. Heads and sizes come from the s2o_config (hidden H = n_q_heads·head_dim). */
+typedef struct {
+  int intermediate;            /* MLP width I (multiple of 8)                                   */
+  float rms_eps;               /* RMS norm epsilon (1e-5)                                       */
+  double rope_theta;           /* rotary base (500000)                                          */
+  double rope_factor;          /* Llama 3.1 frequency scaling: factor (8; 0 turns it off)       */
+  double rope_low_freq_factor; /* (1)                                                           */
+  double rope_high_freq_factor;/* (4)                                                           */
+  int rope_original_context;   /* (8192)                                                        */
+  int dense_attention;         /* 1: dense causal attention instead of S2O (the baseline)       */
+} s2o_layer_config;
+
+/* Device bf16 weights, row-major, used as x·W: attn_norm [H]; w_qkv [H, (Hq + 2·Hkv)·d] (q heads,
+ * then k, then v); w_o [Hq·d, H]; mlp_norm [H]; w_gu [H, 2·I] (gate columns, then up);
+ * w_down [I, H]. 16-byte aligned, owned by the caller. */
+typedef struct {
+  const void *attn_norm, *w_qkv, *w_o, *mlp_norm, *w_gu, *w_down;
+} s2o_layer_weights;
+
+/* Bytes of scratch for s2o_layer_prefill: the layer's activations, index arrays and the
+ * attention's prefill workspace (s2o_prefill_workspace_size; none for the dense baseline).
+ * Host only. */
+s2o_status s2o_layer_workspace_size(const s2o_config *cfg, const s2o_layer_config *lc,
+                                    size_t *bytes);
+
+/* One decoder layer in place on x [batch, N, H] bf16 (device, 16-byte aligned). The S2O path
+ * builds its indices (cfg: segment_len, block_size, tau, variants) and runs the gather-attention
+ * as s2o_attention_prefill does. Errors: S2O_ERR_INVALID_ARGUMENT / S2O_ERR_UNSUPPORTED for bad
+ * arguments (H or I not a multiple of 8), S2O_ERR_WORKSPACE_TOO_SMALL, S2O_ERR_CUDA (a CUDA or
+ * cuBLAS failure). Asynchronous on `stream`. */
+s2o_status s2o_layer_prefill(const s2o_config *cfg, const s2o_layer_config *lc,
+                             const s2o_layer_weights *w, void *x, void *ws, size_t ws_bytes,
+                             s2o_stream stream);
+
 /* Diagnostic: evaluates the library's exp64 — the binary64 exponential behind the block weights of
  * the early stop (a Cody–Waite reduction by ln 2 and a degree-13 Taylor polynomial written for
  * this library; the pages give no normalisation, see [S2O, Summary ¶2]) — on n

@@ -27,7 +27,7 @@ __all__ = [
     "set_wait_limit_ns", "set_attention_max_ctas", "check_device_status", "exp64_eval", "library_path",
     "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
     "prefill_workspace_size", "alloc_prefill_workspace", "attention_prefill_with_indices_ws",
-    "set_permuted_copy",
+    "set_permuted_copy", "layer_workspace_size", "layer_prefill",
 ]
 
 STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
@@ -136,6 +136,28 @@ class Stats:
 _lib = None
 
 
+class _LayerConfig(ctypes.Structure):
+    _fields_ = [("intermediate", ctypes.c_int), ("rms_eps", ctypes.c_float),
+                ("rope_theta", ctypes.c_double), ("rope_factor", ctypes.c_double),
+                ("rope_low_freq_factor", ctypes.c_double),
+                ("rope_high_freq_factor", ctypes.c_double),
+                ("rope_original_context", ctypes.c_int), ("dense_attention", ctypes.c_int)]
+
+
+_LAYER_WEIGHTS = ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gu", "w_down")
+
+
+class _LayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _LAYER_WEIGHTS]
+
+
+def _layer_config(shape, dense: bool) -> _LayerConfig:
+    """From any object with the decoder-layer fields (e.g. ``gen.LayerShape``)."""
+    return _LayerConfig(shape.intermediate, shape.rms_eps, shape.rope_theta, shape.rope_factor,
+                        shape.rope_low_freq_factor, shape.rope_high_freq_factor,
+                        shape.rope_original_context, 1 if dense else 0)
+
+
 def library_path() -> str:
     return _build.LIB
 
@@ -162,6 +184,9 @@ def _load():
             "s2o_index_stats": [C, I, vp, sz, ctypes.POINTER(_Stats), vp],
             "s2o_check_device_status": [vp],
             "s2o_exp64_eval": [vp, vp, ctypes.c_int, vp],
+            "s2o_layer_workspace_size": [C, ctypes.POINTER(_LayerConfig), ctypes.POINTER(sz)],
+            "s2o_layer_prefill": [C, ctypes.POINTER(_LayerConfig), ctypes.POINTER(_LayerWeights),
+                                  vp, vp, sz, vp],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -378,6 +403,37 @@ def kernel_launch_count() -> int:
 
 def set_wait_limit_ns(ns: int) -> None:
     _load().s2o_set_wait_limit_ns(int(ns))
+
+
+def layer_workspace_size(cfg: Config, shape, dense: bool = False) -> int:
+    """Workspace bytes of ``layer_prefill`` (``shape``: the decoder-layer sizes, e.g.
+    ``gen.LayerShape``)."""
+    n = ctypes.c_size_t(0)
+    lc = _layer_config(shape, dense)
+    _check(_load().s2o_layer_workspace_size(ctypes.byref(cfg._c()), ctypes.byref(lc),
+                                            ctypes.byref(n)), "s2o_layer_workspace_size")
+    return n.value
+
+
+def layer_prefill(cfg: Config, shape, weights: dict, x: torch.Tensor,
+                  ws: torch.Tensor | None = None, dense: bool = False) -> torch.Tensor:
+    """One decoder layer in place on x [batch, N, H] (bf16, CUDA): S2O attention, or the dense
+    causal baseline with ``dense``. ``weights``: bf16 CUDA tensors named as in s2o_layer_weights."""
+    H = cfg.n_q_heads * cfg.head_dim
+    _bf16(x, (cfg.batch, cfg.seq_len, H), "x")
+    I = shape.intermediate
+    shapes = {"attn_norm": (H,), "w_qkv": (H, (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim),
+              "w_o": (H, H), "mlp_norm": (H,), "w_gu": (H, 2 * I), "w_down": (I, H)}
+    for name, shp in shapes.items():
+        _bf16(weights[name], shp, name)
+    lc = _layer_config(shape, dense)
+    ws = ws if ws is not None else torch.empty(layer_workspace_size(cfg, shape, dense),
+                                               dtype=torch.uint8, device=x.device)
+    wts = _LayerWeights(*(weights[n].data_ptr() for n in _LAYER_WEIGHTS))
+    _check(_load().s2o_layer_prefill(ctypes.byref(cfg._c()), ctypes.byref(lc), ctypes.byref(wts),
+                                     x.data_ptr(), ws.data_ptr(), ws.numel(), _stream(x.device)),
+           "s2o_layer_prefill")
+    return x
 
 
 def set_permuted_copy(mode: int) -> None:

@@ -266,6 +266,61 @@ s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const voi
                       (cudaStream_t)stream);
 }
 
+s2o_status s2o_layer_workspace_size(const s2o_config *cfg, const s2o_layer_config *lc,
+                                    size_t *bytes) {
+  if (!cfg || !lc || !bytes) return S2O_ERR_INVALID_ARGUMENT;
+  s2o_status st = lc->dense_attention ? check_dense_config(cfg) : check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (lc->intermediate <= 0 || lc->intermediate % 8 || !(lc->rms_eps > 0.f))
+    return S2O_ERR_INVALID_ARGUMENT;
+  // The dense baseline ignores the S2O fields: size it as one segment.
+  s2o_config c = *cfg;
+  if (lc->dense_attention) c.segment_len = c.seq_len;
+  const Dims d = dims_of(c);
+  size_t attn = 0;
+  if (!lc->dense_attention && (st = s2o_prefill_workspace_size(cfg, &attn)) != S2O_OK) return st;
+  *bytes = layer_ws_layout(d, *lc).attn_ws + attn;
+  return S2O_OK;
+}
+
+s2o_status s2o_layer_prefill(const s2o_config *cfg, const s2o_layer_config *lc,
+                             const s2o_layer_weights *w, void *x, void *ws, size_t ws_bytes,
+                             s2o_stream stream) {
+  size_t need = 0;
+  s2o_status st = s2o_layer_workspace_size(cfg, lc, &need);
+  if (st != S2O_OK) return st;
+  if (!w || !x || !ws || !aligned16(x) || !aligned16(ws) || !w->attn_norm || !w->w_qkv ||
+      !w->w_o || !w->mlp_norm || !w->w_gu || !w->w_down || !aligned16(w->attn_norm) ||
+      !aligned16(w->w_qkv) || !aligned16(w->w_o) || !aligned16(w->mlp_norm) ||
+      !aligned16(w->w_gu) || !aligned16(w->w_down))
+    return S2O_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < need) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  s2o_config c1 = *cfg;
+  if (lc->dense_attention) c1.segment_len = c1.seq_len;
+  const Dims d = dims_of(c1);
+  const LayerWs L = layer_ws_layout(d, *lc);
+  char *b = static_cast<char *>(ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  bool blas_ok = true;
+  cudaError_t e = launch_layer_pre(d, *lc, *w, x, b, L, s, &blas_ok);
+  if (e != cudaSuccess || !blas_ok) return S2O_ERR_CUDA;
+  void *q = b + L.q, *k = b + L.k, *v = b + L.v, *o = b + L.o;
+  if (lc->dense_attention) {
+    AttnArgs a{q, k, v, o, nullptr, nullptr, nullptr, nullptr, nullptr, true};
+    e = launch_attention(d, a, g_wait_limit_ns.load(), g_attention_max_ctas.load(), s);
+    if (e != cudaSuccess) return S2O_ERR_CUDA;
+  } else {
+    s2o_indices idx{reinterpret_cast<int32_t *>(b + L.perm_q), reinterpret_cast<int32_t *>(b + L.perm_k),
+                    reinterpret_cast<int32_t *>(b + L.sel_cnt), reinterpret_cast<int32_t *>(b + L.sel_blk),
+                    reinterpret_cast<int32_t *>(b + L.local_tiles)};
+    st = s2o_attention_prefill(cfg, q, k, v, o, &idx, b + L.attn_ws, ws_bytes - L.attn_ws, stream);
+    if (st != S2O_OK) return st;
+  }
+  e = launch_layer_post(d, *lc, *w, x, b, L, s, &blas_ok);
+  if (e != cudaSuccess || !blas_ok) return S2O_ERR_CUDA;
+  return S2O_OK;
+}
+
 s2o_status s2o_dense_causal_prefill(const s2o_config *cfg, const void *q, const void *k,
                                     const void *v, void *o, s2o_stream stream) {
   s2o_status st = check_dense_config(cfg);

@@ -68,6 +68,21 @@ cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_lim
 cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
                                  cudaStream_t st);
 
+// Decoder layer (s2o_layer.cu): byte offsets of its buffers in the layer workspace (the attention's
+// own workspace starts at attn_ws), and the launches before and after the attention. A false
+// *blas_ok reports a cuBLAS failure (no later launch was made).
+struct LayerWs {
+  size_t h, qkv, q, k, v, o, o_rows, gu, a, freqs, cs, perm_q, perm_k, sel_cnt, sel_blk,
+      local_tiles, attn_ws;
+};
+LayerWs layer_ws_layout(const Dims &d, const s2o_layer_config &lc);
+cudaError_t launch_layer_pre(const Dims &d, const s2o_layer_config &lc,
+                             const s2o_layer_weights &w, const void *x, char *ws,
+                             const LayerWs &L, cudaStream_t st, bool *blas_ok);
+cudaError_t launch_layer_post(const Dims &d, const s2o_layer_config &lc,
+                              const s2o_layer_weights &w, void *x, char *ws, const LayerWs &L,
+                              cudaStream_t st, bool *blas_ok);
+
 // Host-side count of kernel launches made by the library (all threads, all devices).
 void note_launch();
 unsigned long long launch_count();
