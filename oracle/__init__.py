@@ -13,6 +13,9 @@ Parity status per function (what pins it to something other than itself lives in
   causal attention at τ > 1, and by permutation invariance.
 * ``dense_causal`` — pinned by torch's causal scaled-dot-product attention.
 * ``exp64`` — pinned by libm exp (≤ 2 ulp) and the constants by a 60-digit derivation.
+* ``layer.layer`` (the decoder layer around the attention, ``oracle/layer.py``) — pinned in
+  ``tests/test_layer_oracle_pins.py`` (bf16 rounding against torch, closed-form norms, rotary
+  invariants, the frequency scaling's regimes, the silu identity, zero projections = identity).
 """
 from __future__ import annotations
 
