@@ -23,6 +23,7 @@
 #include <cublas_v2.h>
 
 #include <cmath>
+#include <type_traits>
 #include <mutex>
 
 #include "s2o_internal.h"
@@ -90,12 +91,15 @@ __global__ void k_rope_table(const double *__restrict__ freqs, float2 *__restric
 
 // One warp per (row, head) of qkv [b·N, (Hq + 2·Hkv)·d]: q and k heads rotated by the table
 // (pairs t, t + d/2), v copied; written head-major to Q [b, Hq, N, d], K and V [b, Hkv, N, d].
+// Lane l takes the PER consecutive t = PER·l .. of each half (4-byte accesses for d = 128).
 template <int D>
 __global__ void __launch_bounds__(256)
     k_rope_split(const uint16_t *__restrict__ qkv, const float2 *__restrict__ cs,
                  uint16_t *__restrict__ Q, uint16_t *__restrict__ K, uint16_t *__restrict__ V,
                  int N, int Hq, int Hkv, long long rows) {
-  constexpr int HALF = D / 2, PER = HALF / 32;  // pairs per lane
+  constexpr int HALF = D / 2, PER = HALF / 32;
+  static_assert(PER == 1 || PER == 2, "d = 64 or 128");
+  using W = typename std::conditional<PER == 2, uint32_t, uint16_t>::type;
   const int heads = Hq + 2 * Hkv;
   const long long wid = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -112,20 +116,23 @@ __global__ void __launch_bounds__(256)
     dst = K + ((b * Hkv + (h - Hq)) * N + i) * D;
   else
     dst = V + ((b * Hkv + (h - Hq - Hkv)) * N + i) * D;
-  const bool rot = h < Hq + Hkv;
-#pragma unroll
-  for (int p = 0; p < PER; ++p) {
-    const int t = lane + 32 * p;
-    const float a = bf16_to_f(src[t]), bb = bf16_to_f(src[t + HALF]);
-    if (rot) {
-      const float2 r = __ldg(cs + (long long)i * HALF + t);
-      dst[t] = f_to_bf16(a * r.x - bb * r.y);
-      dst[t + HALF] = f_to_bf16(bb * r.x + a * r.y);
-    } else {
-      dst[t] = src[t];
-      dst[t + HALF] = src[t + HALF];
-    }
+  const int t0 = PER * lane;
+  const W lo = *reinterpret_cast<const W *>(src + t0), hi = *reinterpret_cast<const W *>(src + HALF + t0);
+  if (h >= Hq + Hkv) {
+    *reinterpret_cast<W *>(dst + t0) = lo;
+    *reinterpret_cast<W *>(dst + HALF + t0) = hi;
+    return;
   }
+  W olo = 0, ohi = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const float a = bf16_to_f((uint16_t)(lo >> (16 * e))), bb = bf16_to_f((uint16_t)(hi >> (16 * e)));
+    const float2 r = __ldg(cs + (long long)i * HALF + t0 + e);
+    olo |= (W)f_to_bf16(a * r.x - bb * r.y) << (16 * e);
+    ohi |= (W)f_to_bf16(bb * r.x + a * r.y) << (16 * e);
+  }
+  *reinterpret_cast<W *>(dst + t0) = olo;
+  *reinterpret_cast<W *>(dst + HALF + t0) = ohi;
 }
 
 // rows[b·N + i][h·d + c] = O[b][h][i][c], 16-byte pieces.
