@@ -89,50 +89,53 @@ __global__ void k_rope_table(const double *__restrict__ freqs, float2 *__restric
   cs[e] = make_float2((float)c, (float)s);
 }
 
-// One warp per (row, head) of qkv [b·N, (Hq + 2·Hkv)·d]: q and k heads rotated by the table
-// (pairs t, t + d/2), v copied; written head-major to Q [b, Hq, N, d], K and V [b, Hkv, N, d].
-// Lane l takes the PER consecutive t = PER·l .. of each half (4-byte accesses for d = 128).
+// One CTA per row of qkv [b·N, (Hq + 2·Hkv)·d], its warps taking the heads in turn: q and k
+// heads rotated by the table (pairs t, t + d/2), v copied; written head-major to
+// Q [b, Hq, N, d], K and V [b, Hkv, N, d]. Lane l takes the PER consecutive t = PER·l .. of each
+// half (4-byte accesses for d = 128).
 template <int D>
 __global__ void __launch_bounds__(256)
     k_rope_split(const uint16_t *__restrict__ qkv, const float2 *__restrict__ cs,
                  uint16_t *__restrict__ Q, uint16_t *__restrict__ K, uint16_t *__restrict__ V,
-                 int N, int Hq, int Hkv, long long rows) {
+                 int N, int Hq, int Hkv) {
   constexpr int HALF = D / 2, PER = HALF / 32;
   static_assert(PER == 1 || PER == 2, "d = 64 or 128");
   using W = typename std::conditional<PER == 2, uint32_t, uint16_t>::type;
   const int heads = Hq + 2 * Hkv;
-  const long long wid = (long long)blockIdx.x * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  if (wid >= rows * heads) return;
-  const long long row = wid / heads;
-  const int h = (int)(wid % heads);
-  const long long b = row / N;
-  const int i = (int)(row % N);
-  const uint16_t *src = qkv + row * (long long)heads * D + (long long)h * D;
-  uint16_t *dst;
-  if (h < Hq)
-    dst = Q + ((b * Hq + h) * N + i) * D;
-  else if (h < Hq + Hkv)
-    dst = K + ((b * Hkv + (h - Hq)) * N + i) * D;
-  else
-    dst = V + ((b * Hkv + (h - Hq - Hkv)) * N + i) * D;
-  const int t0 = PER * lane;
-  const W lo = *reinterpret_cast<const W *>(src + t0), hi = *reinterpret_cast<const W *>(src + HALF + t0);
-  if (h >= Hq + Hkv) {
-    *reinterpret_cast<W *>(dst + t0) = lo;
-    *reinterpret_cast<W *>(dst + HALF + t0) = hi;
-    return;
-  }
-  W olo = 0, ohi = 0;
+  const long long row = blockIdx.x;
+  const int b = (int)(blockIdx.x / (unsigned)N), i = (int)(blockIdx.x % (unsigned)N);
+  const int lane = threadIdx.x % 32, t0 = PER * lane;
+  const float2 *csr = cs + (long long)i * HALF + t0;
+  float2 r[PER];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    const float a = bf16_to_f((uint16_t)(lo >> (16 * e))), bb = bf16_to_f((uint16_t)(hi >> (16 * e)));
-    const float2 r = __ldg(cs + (long long)i * HALF + t0 + e);
-    olo |= (W)f_to_bf16(a * r.x - bb * r.y) << (16 * e);
-    ohi |= (W)f_to_bf16(bb * r.x + a * r.y) << (16 * e);
+  for (int e = 0; e < PER; ++e) r[e] = __ldg(csr + e);
+  for (int h = threadIdx.x / 32; h < heads; h += blockDim.x / 32) {
+    const uint16_t *src = qkv + (row * heads + h) * D;
+    uint16_t *dst;
+    if (h < Hq)
+      dst = Q + (((long long)b * Hq + h) * N + i) * D;
+    else if (h < Hq + Hkv)
+      dst = K + (((long long)b * Hkv + (h - Hq)) * N + i) * D;
+    else
+      dst = V + (((long long)b * Hkv + (h - Hq - Hkv)) * N + i) * D;
+    const W lo = *reinterpret_cast<const W *>(src + t0);
+    const W hi = *reinterpret_cast<const W *>(src + HALF + t0);
+    if (h >= Hq + Hkv) {
+      *reinterpret_cast<W *>(dst + t0) = lo;
+      *reinterpret_cast<W *>(dst + HALF + t0) = hi;
+      continue;
+    }
+    W olo = 0, ohi = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const float a = bf16_to_f((uint16_t)(lo >> (16 * e)));
+      const float bb = bf16_to_f((uint16_t)(hi >> (16 * e)));
+      olo |= (W)f_to_bf16(a * r[e].x - bb * r[e].y) << (16 * e);
+      ohi |= (W)f_to_bf16(bb * r[e].x + a * r[e].y) << (16 * e);
+    }
+    *reinterpret_cast<W *>(dst + t0) = olo;
+    *reinterpret_cast<W *>(dst + HALF + t0) = ohi;
   }
-  *reinterpret_cast<W *>(dst + t0) = olo;
-  *reinterpret_cast<W *>(dst + HALF + t0) = ohi;
 }
 
 // rows[b·N + i][h·d + c] = O[b][h][i][c], 16-byte pieces.
@@ -152,31 +155,31 @@ __global__ void __launch_bounds__(256)
   rows[x] = __ldg(O + ((b * Hq + h) * N + i) * P + c);
 }
 
-// a[row][j] = bf16(silu(gate) · up), gate = gu[row][j], up = gu[row][I + j]; 8 values a thread.
+// a[row][j] = bf16(silu(gate) · up), gate = gu[row][j], up = gu[row][I + j]; one CTA per row,
+// 8 values a thread per step.
 __global__ void __launch_bounds__(256)
-    k_silu_mul(const uint16_t *__restrict__ gu, uint16_t *__restrict__ a, int I,
-               long long n_groups) {
-  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x >= n_groups) return;
-  const int per_row = I / 8;
-  const long long row = x / per_row;
-  const int j = (int)(x % per_row) * 8;
-  const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gu + row * 2LL * I + j));
-  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(gu + row * 2LL * I + I + j));
-  const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
-  uint32_t o[4];
+    k_silu_mul(const uint16_t *__restrict__ gu, uint16_t *__restrict__ a, int I) {
+  const long long row = blockIdx.x;
+  const uint4 *g4 = reinterpret_cast<const uint4 *>(gu + row * 2LL * I);
+  const uint4 *u4 = reinterpret_cast<const uint4 *>(gu + row * 2LL * I + I);
+  uint4 *a4 = reinterpret_cast<uint4 *>(a + row * (long long)I);
+  for (int c = threadIdx.x; c < I / 8; c += blockDim.x) {
+    const uint4 g = __ldg(g4 + c), u = __ldg(u4 + c);
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float r[2];
+    for (int k = 0; k < 4; ++k) {
+      float r[2];
 #pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-      const float z = bf16_to_f((uint16_t)(gw[k] >> (16 * hlf)));
-      const float up = bf16_to_f((uint16_t)(uw[k] >> (16 * hlf)));
-      r[hlf] = z / (1.0f + expf(-z)) * up;
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const float z = bf16_to_f((uint16_t)(gw[k] >> (16 * hlf)));
+        const float up = bf16_to_f((uint16_t)(uw[k] >> (16 * hlf)));
+        r[hlf] = __fdividef(z, 1.0f + __expf(-z)) * up;
+      }
+      o[k] = (uint32_t)f_to_bf16(r[0]) | ((uint32_t)f_to_bf16(r[1]) << 16);
     }
-    o[k] = (uint32_t)f_to_bf16(r[0]) | ((uint32_t)f_to_bf16(r[1]) << 16);
+    a4[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  *reinterpret_cast<uint4 *>(a + row * (long long)I + j) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 unsigned grid_for(long long n, int per) { return (unsigned)((n + per - 1) / per); }
@@ -284,15 +287,14 @@ cudaError_t launch_layer_pre(const Dims &d, const s2o_layer_config &lc,
                                                      reinterpret_cast<float2 *>(ws + L.cs), d.N,
                                                      d.D / 2);
   note_launch();
-  const long long warps = rows * (d.Hq + 2 * d.Hkv);
   auto *qkv = reinterpret_cast<const uint16_t *>(ws + L.qkv);
   auto *cs = reinterpret_cast<const float2 *>(ws + L.cs);
   auto *Q = reinterpret_cast<uint16_t *>(ws + L.q), *K = reinterpret_cast<uint16_t *>(ws + L.k),
        *V = reinterpret_cast<uint16_t *>(ws + L.v);
   if (d.D == 128)
-    k_rope_split<128><<<grid_for(warps, 8), 256, 0, st>>>(qkv, cs, Q, K, V, d.N, d.Hq, d.Hkv, rows);
+    k_rope_split<128><<<(unsigned)rows, 256, 0, st>>>(qkv, cs, Q, K, V, d.N, d.Hq, d.Hkv);
   else
-    k_rope_split<64><<<grid_for(warps, 8), 256, 0, st>>>(qkv, cs, Q, K, V, d.N, d.Hq, d.Hkv, rows);
+    k_rope_split<64><<<(unsigned)rows, 256, 0, st>>>(qkv, cs, Q, K, V, d.N, d.Hq, d.Hkv);
   note_launch();
   return cudaGetLastError();
 }
@@ -331,10 +333,8 @@ cudaError_t launch_layer_post(const Dims &d, const s2o_layer_config &lc,
     *blas_ok = false;
     return cudaSuccess;
   }
-  const long long groups = rows * I / 8;
-  k_silu_mul<<<grid_for(groups, 256), 256, 0, st>>>(reinterpret_cast<const uint16_t *>(ws + L.gu),
-                                                    reinterpret_cast<uint16_t *>(ws + L.a),
-                                                    (int)I, groups);
+  k_silu_mul<<<(unsigned)rows, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(ws + L.gu),
+                                             reinterpret_cast<uint16_t *>(ws + L.a), (int)I);
   note_launch();
   if (!gemm(hd, ws + L.a, w.w_down, x, rows, H, I, true)) {
     *blas_ok = false;
