@@ -114,3 +114,68 @@ def test_workspace_views_are_inside_the_workspace():
     ptrs = [getattr(view, f) for f, _ in s2o._View._fields_]
     assert all(base <= p < base + need for p in ptrs)
     assert len(set(ptrs)) == len(ptrs)
+
+
+# ----------------------------------------------------------------------------- prefill + layer
+
+
+def test_prefill_workspace_holds_the_copy_and_the_bitmaps():
+    cfg = LLAMA_128K
+    base = s2o.workspace_size(cfg)
+    full = s2o.prefill_workspace_size(cfg)
+    nB = 1024
+    copy = 2 * 32 * 131072 * 128 * 2          # K and V in each query head's key order
+    bitmaps = 32 * nB * (nB // 32 + 1 + nB) * 4  # bitmaps, their counts, block-ordered lists
+    assert full - base >= copy + bitmaps
+    assert full - base <= copy + bitmaps + 4096
+
+
+def test_permuted_copy_modes_are_accepted():
+    lib = s2o._load()
+    for mode in (0, 1, 2, 3, 7, -1):
+        s2o.set_permuted_copy(mode)
+    s2o.set_permuted_copy(1)
+    assert lib is s2o._load()
+
+
+def _layer_size(cfg, shape, dense=False):
+    n = ctypes.c_size_t(0)
+    lc = s2o._layer_config(shape, dense)
+    return s2o._load().s2o_layer_workspace_size(ctypes.byref(cfg._c()), ctypes.byref(lc),
+                                                ctypes.byref(n)), n.value
+
+
+def test_layer_workspace_size_and_argument_checks():
+    import gen
+    shape = gen.LAYER_8B
+    st, s2o_bytes = _layer_size(LLAMA_128K, shape)
+    assert st == 0
+    st, dense_bytes = _layer_size(LLAMA_128K, shape, dense=True)
+    assert st == 0
+    rows, H, I = 131072, 4096, 14336
+    # activations: h, qkv, q, k, v, o, o_rows, gate|up, silu product (bf16)
+    acts = rows * 2 * (H + 6144 + H + 1024 + 1024 + H + H + 2 * I + I)
+    assert dense_bytes >= acts
+    # the S2O layer adds the attention's prefill workspace
+    assert s2o_bytes - dense_bytes >= s2o.prefill_workspace_size(LLAMA_128K) - 1024
+    assert _layer_size(LLAMA_128K, shape.replace(intermediate=100))[0] == 1   # not a multiple of 8
+    assert _layer_size(LLAMA_128K, shape.replace(rms_eps=0.0))[0] == 1
+    # the dense baseline ignores the segment length; S2O does not
+    bad_seg = s2o.Config(**{**LLAMA_128K.__dict__, "segment_len": 192})
+    assert _layer_size(bad_seg, shape)[0] == 2
+    assert _layer_size(bad_seg, shape, dense=True)[0] == 0
+
+
+def test_layer_prefill_rejects_null_weights_before_launch():
+    import gen
+    lib = s2o._load()
+    shape = gen.LAYER_8B
+    lc = s2o._layer_config(shape, False)
+    w = s2o._LayerWeights(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0)  # w_down missing
+    st = lib.s2o_layer_prefill(ctypes.byref(LLAMA_128K._c()), ctypes.byref(lc), ctypes.byref(w),
+                               0x10000, 0x20000, 1 << 40, None)
+    assert st == 1
+    w = s2o._LayerWeights(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    st = lib.s2o_layer_prefill(ctypes.byref(LLAMA_128K._c()), ctypes.byref(lc), ctypes.byref(w),
+                               0x10000, 0x20000, 1024, None)
+    assert st == 3  # workspace too small

@@ -113,3 +113,17 @@ def test_layer_s2o_at_tau_zero_matches_dense_attention():
     # bf16 on all but a few elements
     assert np.mean(a != b) < 0.01
     assert np.max(np.abs(a - b)) <= 2 ** -6 * max(1.0, np.max(np.abs(a)))
+
+
+def test_layer_inputs_are_seeded_and_thread_independent():
+    w = gen.Workload("layer-pin", 1, 2, 1, 2048, 64, 128, 64, 0.01, 5)
+    shape = SHAPE.replace(intermediate=256)
+    a = gen.make_layer(w, shape, threads=1)
+    b = gen.make_layer(w, shape, threads=7)
+    c = gen.make_layer(w, shape, seed=6, threads=3)
+    for name in a:
+        assert torch.equal(a[name].view(torch.int16), b[name].view(torch.int16)), name
+    assert not torch.equal(a["w_qkv"].view(torch.int16), c["w_qkv"].view(torch.int16))
+    # projection scale N(0, 1/fan_in), norm gains around 1
+    assert abs(float(a["w_gu"].float().std()) * math.sqrt(128) - 1) < 0.05
+    assert abs(float(a["attn_norm"].float().mean()) - 1) < 0.05
