@@ -24,7 +24,6 @@
 
 #include <cmath>
 #include <type_traits>
-#include <mutex>
 
 #include "s2o_internal.h"
 
