@@ -336,13 +336,14 @@ struct Unit {
 // segment) in a row, so that the two units of a pair position read one key ordering and can share
 // the selected blocks they have in common; their list lengths and block-ordered lists then come
 // from the bitmap kernel.
-template <int BN, bool BITS>
+template <int BN, int KIND>
 __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
+  constexpr bool BITS = KIND == 2, PERM = KIND != 0;
   // Unit ids are below 2^31 (the host checks): divisions by multiply-high.
   Unit r;
   uint32_t rem;
   int hi, b, bl;  // query head of the group, block, and the block's index inside its segment
-  if (BITS && p.mode == kPermuted) {
+  if (BITS) {
     u = p.div_seg.divmod(u, rem);
     bl = (int)rem;
     u = p.div_nSeg.divmod(u, rem);
@@ -353,7 +354,7 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
   } else {
     u = p.div_G.divmod(u, rem);
     hi = (int)rem;
-    if (p.mode == kDense) {
+    if (!PERM && p.mode == kDense) {
       u = p.div_nB.divmod(u, rem);
       b = p.nB - 1 - (int)rem;
       bl = b;
@@ -372,7 +373,7 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
   r.qh = beta * p.Hq + (long long)g * p.G + hi;
   r.kh = beta * p.Hkv + g;
   r.b = b;
-  if (p.mode != kPermuted) {
+  if (!PERM) {
     r.lt = bl + 1;  // the causal triangle of the block's segment (or sequence)
     r.cnt = 0;
     r.sel = nullptr;
@@ -405,14 +406,15 @@ struct Pair {
 // KV head) walks the union of its two bitmaps: a block both units selected is loaded once for
 // both. Its stream length then needs the union's size (union_size).
 constexpr uint32_t kNoUnit = 0xffffffffu;
-template <int BN, bool BITS>
+template <int BN, int KIND>
 __device__ __forceinline__ Pair decode_pair(const Params &p, const uint32_t *list, int n_list,
                                             int i) {
+  constexpr bool BITS = KIND == 2;
   Pair P;
-  P.u0 = decode_unit<BN, BITS>(p, list[2 * i]);
+  P.u0 = decode_unit<BN, KIND>(p, list[2 * i]);
   P.valid1 = 2 * i + 1 < n_list && (!BITS || list[2 * i + 1] != kNoUnit);
   if (P.valid1) {
-    P.u1 = decode_unit<BN, BITS>(p, list[2 * i + 1]);
+    P.u1 = decode_unit<BN, KIND>(p, list[2 * i + 1]);
   } else {
     P.u1 = P.u0;
     P.u1.lt = 0;
@@ -692,8 +694,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // again the work items w, each contributing those of its units 2w and 2w+1 whose list is not
 // empty (the second slot kNoUnit when only one is), so that a pair is two consecutive blocks of
 // one query head.
-template <int BN, bool BITS>
+template <int BN, int KIND>
 __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lane) {
+  constexpr bool BITS = KIND == 2;
   const bool by_unit = p.skip_empty && !BITS;
   const long long span = by_unit ? kList : kList / 2;
   const long long first = blockIdx.x + k0 * gridDim.x;
@@ -759,10 +762,11 @@ __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lan
 
 // ------------------------------------------------------------------ the kernel
 
-// BITS: the permuted pass with bitmap streams. A launch given block bitmaps (sel_bits) runs only
-// if the decision flag chose bitmap streams (BITS) or did not (!BITS): the host launches both
-// and one returns at once.
-template <int D, int BN, bool BITS>
+// KIND 0: the contiguous modes (local pass, dense baseline), compiled without the permuted
+// pass's code; 1: the permuted pass with list streams; 2: the permuted pass with bitmap streams.
+// A permuted launch given block bitmaps (sel_bits) runs only if the decision flag chose bitmap
+// streams (KIND 2) or did not (KIND 1): the host launches both and one returns at once.
+template <int D, int BN, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     s2o_attention_kernel(const __grid_constant__ CUtensorMap tm_q_tile,
                          const __grid_constant__ CUtensorMap tm_q_row,
@@ -774,9 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_kp_tile,
                          const __grid_constant__ CUtensorMap tm_vp_tile, const Params p) {
   using L = Layout<D, BN>;
-  if (p.mode == kPermuted && p.sel_bits != nullptr &&
-      ((__ldg(p.copy_flag) & 3u) == 3u) != BITS)
-    return;
+  constexpr bool BITS = KIND == 2, PERM = KIND != 0;
+  const uint32_t flagv = p.copy_flag != nullptr ? __ldg(p.copy_flag) : 0u;
+  if (PERM && p.sel_bits != nullptr && ((flagv & 3u) == 3u) != BITS) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -833,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = true;
   // Set before the launch by the permuted-copy decision: selected blocks come from the permuted
   // copy (bit 0), in block order from the block bitmaps (bit 1, only with bit 0).
-  const bool use_copy = p.copy_flag != nullptr && (__ldg(p.copy_flag) & 1u) != 0u;
+  const bool use_copy = PERM && (flagv & 1u) != 0u;
   // Work comes in windows of this CTA's share: warp 0 fills the work list between two CTA-wide
   // barriers and every role then walks the window's items (a role that gave up a bounded wait
   // keeps meeting the barriers without working).
@@ -843,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (long long k0 = 0;; k0 += p.skip_empty && !BITS ? kList : kList / 2) {
       named_bar_sync(1, kThreads);
       if (warp == 0) {
-        const int n = build_list<BN, BITS>(p, k0, list, lane);
+        const int n = build_list<BN, KIND>(p, k0, list, lane);
         if (lane == 0) *list_n = n;
         __syncwarp();
       }
@@ -880,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
+      Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
       if (BITS && P.uni) {
         // Union stream: local tiles, then each block either unit selected, once, from the
         // permuted copy.
@@ -900,6 +904,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ok = issue(P, it, make_int4(0, 0, 0, 0), c);
         }
+        continue;
+      }
+      if (!PERM) {
+        // Contiguous modes: local tiles only.
+        for (int j = 0; ok && j < P.total; ++j) ok = issue(P, item_at(P, j), make_int4(0, 0, 0, 0), -1);
         continue;
       }
       // Gathered rows are looked up ahead: the rows of item j+1 and the block of item j+2 are
@@ -940,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long qn[2] = {0, 0};
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      const Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
+      const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
       for (int x = 0; ok && x < 1 + P.valid1; ++x) {
         if (qn[x] >= 1 &&
             !warp_wait(bar(kQEmpty + x), (uint32_t)((qn[x] - 1) & 1), lim, lane)) {
@@ -952,7 +961,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit &u = x ? P.u1 : P.u0;
         const uint32_t dst = sQ + x * L::Q_BYTES;
         const int q_row0 = (int)(u.qh * p.N);
-        if (p.mode != kPermuted || p.perm_q == nullptr) {
+        if (!PERM || p.perm_q == nullptr) {
           if (lane == 0)
             for (int a = 0; a < D / 64; ++a)
               tma_load_tile(dst + a * L::ATOM_Q, &tm_q_tile, a * 64, q_row0 + u.b * BN,
@@ -1063,7 +1072,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
       if (lane == 0) {
       for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-        Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
+        Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
         // A union stream's selected part is walked once, item by item, for its users.
         UnionCursor uc;
         if (BITS && P.uni) {
@@ -1153,7 +1162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long sn = 0, on = 0;  // S_x tiles and work items consumed
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      const Pair P = decode_pair<BN, BITS>(p, list, n_list, wi);
+      const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
       if (x == 1 && !P.valid1) continue;
       const Unit u = x ? P.u1 : P.u0;
       const int seg0 = u.seg0;
@@ -1161,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int i_orig = seg0 + p.S - 1;
       bool store_row = false;
       if (row < BN) {
-        const int v = (p.mode != kPermuted || p.perm_q == nullptr)
+        const int v = (!PERM || p.perm_q == nullptr)
                           ? u.b * BN + row
                           : __ldg(p.perm_q + u.qh * p.N + (size_t)u.b * BN + row);
         store_row = v >= seg0 && v < seg0 + p.S;
@@ -1171,7 +1180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_items = u.lt + u.cnt;
       // Keys of a selected block (for its mask) are requested before the wait for its S, the
       // block id one tile earlier.
-      auto blk = [&](int n) { return n >= u.lt && n < n_items ? sel_block(p, u, n - u.lt) : -1; };
+      auto blk = [&](int n) {
+        return PERM && n >= u.lt && n < n_items ? sel_block(p, u, n - u.lt) : -1;
+      };
       int c_cur = blk(0), c_next = blk(1);
       for (int n = 0; n < n_items; ++n) {
         int keys[BN / 32];
@@ -1196,7 +1207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&s[c0 * 32]));
 
         // Masks on original positions.
-        if (n < u.lt) {
+        if (!PERM || n < u.lt) {
           const int limit = i_orig - (seg0 + n * BN);  // keys col <= limit are causal
           if (__any_sync(full, limit < BN - 1)) {
 #pragma unroll
@@ -1288,7 +1299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(o_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
 #pragma unroll
       for (int c0 = 0; c0 < D / 32; ++c0) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
-      if (p.mode != kPermuted) {
+      if (!PERM) {
         // Contiguous rows: each 64-column atom is staged in shared memory (128-byte swizzle) and
         // written with one TMA tile store; the group's first thread issues the stores and, before
         // its stage is overwritten, waits until the previous store has read it.
@@ -1389,6 +1400,9 @@ __global__ void __launch_bounds__(1024)
         mode >= 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks);
     const bool dense = mode == 3 || (mode == 1 && copy &&
                                      total >= (unsigned long long)n_units * (unsigned long long)nB / 8);
+    // Merging into the local rows (bit 2) when at least 1 % of the query blocks have a
+    // selection: below that the permuted pass is too small to repay the local pass's extra
+    // softmax-state stores.
     *flag = (copy ? 1u : 0u) | (dense ? 2u : 0u);
   }
 }
@@ -1438,14 +1452,14 @@ __global__ void __launch_bounds__(256)
 
 // kp[h·N + rank] = K row perm_k[hq(h)][rank] of h's KV head, and the same for V (h a query head,
 // or a KV head whose first query head's ordering is used). 16-byte pieces, grid-stride; nothing
-// when the flag is clear.
+// when the flag's copy bit is clear.
 template <int D>
 __global__ void __launch_bounds__(256)
     k_permute_kv(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                  const int32_t *__restrict__ perm_k, uint4 *__restrict__ kp,
                  uint4 *__restrict__ vp, long long copy_rows, int N, int Hq, int Hkv, int G,
                  int per_kv, const uint32_t *__restrict__ flag) {
-  if (__ldg(flag) == 0u) return;
+  if ((__ldg(flag) & 1u) == 0u) return;
   constexpr int PIECES = D * 2 / 16;  // 16-byte pieces per row
   const long long n = copy_rows * PIECES;
   for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < n;
@@ -1520,13 +1534,12 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
     tkp = tk;
     tvp = tv;
   }
-  cudaError_t e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(s2o_attention_kernel<D, BN, true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM)) !=
-      cudaSuccess)
-    return e;
+  cudaError_t e = cudaSuccess;
+  for (auto fn : {s2o_attention_kernel<D, BN, 0>, s2o_attention_kernel<D, BN, 1>,
+                  s2o_attention_kernel<D, BN, 2>})
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)L::SMEM)) != cudaSuccess)
+      return e;
   Params p;
   p.perm_q = a.perm_q;
   p.perm_k = a.perm_k;
@@ -1565,11 +1578,14 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
     const long long work = skip_empty && !bits ? p.n_units : p.n_items;
     const long long cap = max_ctas > 0 && max_ctas < sm_count() ? max_ctas : sm_count();
     const long long grid = work < cap ? work : cap;
-    if (bits)
-      s2o_attention_kernel<D, BN, true><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+    if (mode != kPermuted)
+      s2o_attention_kernel<D, BN, 0><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+          tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+    else if (bits)
+      s2o_attention_kernel<D, BN, 2><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
           tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
     else
-      s2o_attention_kernel<D, BN, false><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+      s2o_attention_kernel<D, BN, 1><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
           tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
     note_launch();
     return cudaGetLastError();
