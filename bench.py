@@ -42,8 +42,8 @@ WORKLOAD = "llama-128k"
 # summarised in profiles/s2o_attention_kernel_local-pass_llama-32k_full.md (dram__bytes_read.sum +
 # dram__bytes_write.sum on llama-32k, scaled by the tile count to llama-128k). Valid only for the
 # kernel source it was taken on: reported as null once s2o_attn.cu changes.
-ATTN_TRAFFIC = {"src_sha256_16": "f5f5195440509e7a", "workload": "llama-128k",
-                "bytes_per_launch": (405.440512e6 + 236.548608e6) * 4}
+ATTN_TRAFFIC = {"src_sha256_16": "0ecfe9d39aed6d8d", "workload": "llama-128k",
+                "bytes_per_launch": (405.164800e6 + 235.952384e6) * 4}
 
 
 def attention_traffic(workload):
