@@ -224,7 +224,11 @@ s2o_status s2o_check_device_status(s2o_stream stream);
  *  - Configurations whose s2o_workspace_size exceeds S2O_STATIC_WORKSPACE_BYTES are rejected with
  *    S2O_ERR_WORKSPACE_TOO_SMALL before any device work.
  *  - The first call on each device (with that device current) looks up the array's device address
- *    with cudaGetSymbolAddress; make that first call before any stream capture.
+ *    with cudaGetSymbolAddress and keeps it with the id of the device's context; a call that finds
+ *    another context on the device (after cudaDeviceReset, say) looks it up again. The first call
+ *    on each host thread also creates the library's side stream and its two events for that
+ *    device (as every index build does). Make those first calls before any stream capture or any
+ *    region that must not create CUDA resources.
  *  - Every call on a device shares the one array and leaves its contents behind; calls whose GPU
  *    work overlaps (different streams, or different host threads) race on it and must be
  *    serialised by the caller. s2o_workspace_views does not apply to it.

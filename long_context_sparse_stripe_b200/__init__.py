@@ -283,12 +283,15 @@ def build_indices_static(cfg: Config, q, k, out: Indices) -> Indices:
     """The index build for callers that cannot allocate device memory: the library's fixed
     scratch array (``STATIC_WORKSPACE_BYTES`` per GPU) replaces the caller workspace. ``out`` must
     be preallocated. Calls whose GPU work overlaps share that array and race; the first call on a
-    device does a one-time address lookup and should come before any stream capture."""
+    device (and on each host thread) does a one-time set-up and should come before any stream
+    capture. The call runs with q's device current, so it uses that device's array."""
     _qkv(cfg, q, k)
     idx = out._c()
-    _check(_load().s2o_build_indices_static(ctypes.byref(cfg._c()), q.data_ptr(), k.data_ptr(),
-                                            ctypes.byref(idx), _stream(q.device)),
-           "s2o_build_indices_static")
+    with torch.cuda.device(q.device):
+        _check(_load().s2o_build_indices_static(ctypes.byref(cfg._c()), q.data_ptr(),
+                                                k.data_ptr(), ctypes.byref(idx),
+                                                _stream(q.device)),
+               "s2o_build_indices_static")
     return out
 
 

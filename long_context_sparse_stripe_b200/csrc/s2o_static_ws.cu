@@ -11,7 +11,13 @@
 // S2O_STATIC_WORKSPACE_BYTES for it until the process exits. Host code cannot use the symbol's
 // name as a device address (on the host it names a stand-in object), so the first call on each
 // device looks up the real address with cudaGetSymbolAddress while that device is current, and
-// caches it per device.
+// caches it per device together with the unique id of the device's context at that time. A later
+// call on a device whose context has been replaced (cudaDeviceReset, or a primary context released
+// and created again) finds another id and looks the address up again, so a stale address from a
+// destroyed context is never used.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "s2o_internal.h"
@@ -25,19 +31,50 @@ __device__ __align__(256) unsigned char g_static_workspace[S2O_STATIC_WORKSPACE_
 
 std::mutex g_static_mutex;
 char *g_static_ptr[kMaxDevices] = {};
+unsigned long long g_static_ctx[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device (set-up on first use).
+// Unique id of the calling thread's current context (cuCtxGetId, through the runtime's driver
+// entry point query: no link against libcuda). 0 if it cannot be had.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_id || !get_cur || get_cur(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the static scratch on the current device: looked up on the first call with
+// the device current and again whenever the device's context has changed since.
 cudaError_t static_workspace(char **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // 0 when no context is current on this thread yet (the runtime binds the device's primary
+  // context on its first call that needs one): the lookup below then runs, and binds it.
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_static_mutex);
-  if (!g_static_ptr[dev]) {
+  if (!g_static_ptr[dev] || ctx == 0 || g_static_ctx[dev] != ctx) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess) return e;
     g_static_ptr[dev] = static_cast<char *>(p);
+    g_static_ctx[dev] = current_context_id();
   }
   *out = g_static_ptr[dev];
   return cudaSuccess;

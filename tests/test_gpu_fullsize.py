@@ -1,10 +1,12 @@
 """Parity at the benchmark configurations' full sizes, in the launch configuration bench.py times.
 
 The GPU runs the whole layer (all 32 query heads, every kernel as the bench launches it); the CPU
-oracle recomputes one or two KV groups (4 query heads each) of the same inputs — each head's
-indices depend only on its own queries and its group's keys — and a sample of output rows:
-every segment's first and last row of those heads plus random rows. Index arrays must be
-bit-exact, outputs within max-abs 2e-2 and mean-abs 1e-3 of the oracle's binary64 result.
+oracle recomputes every KV group (4 query heads each) of the same inputs — each head's indices
+depend only on its own queries and its group's keys — and a sample of output rows of each group:
+every segment's first and last row of its heads, rows of query blocks that selected permuted
+blocks, and random rows. Index arrays must be bit-exact for all heads, outputs within max-abs 2e-2
+and mean-abs 1e-3 of the oracle's binary64 result. The 32-layer stack checks every layer, one KV
+group per layer (group l mod 8 for layer l, so the eight groups are all covered).
 
 Inputs of one workload are generated once (about half a minute on the host for a 128K layer) and
 reused for its variants (τ, segment length, query permutation off), which is how the ablation
@@ -39,7 +41,7 @@ def group_slice(w, q, k, v, g):
             v[:, g:g + 1].contiguous())
 
 
-def check_layer(w, groups, n_random=384, seed=0):
+def check_layer(w, groups=None, n_random=384, seed=0):
     q, k, v = inputs(w)
     cfg = s2o.Config.of(w)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
@@ -50,6 +52,8 @@ def check_layer(w, groups, n_random=384, seed=0):
     nB = w.seq_len // w.block_size
     rng = np.random.default_rng(seed)
     selected = 0
+    if groups is None:
+        groups = range(w.n_kv_heads)
     for g in groups:
         sub, qs, ks, vs = group_slice(w, q, k, v, g)
         ocfg = oracle.config(sub)
@@ -83,12 +87,20 @@ def check_layer(w, groups, n_random=384, seed=0):
 
 
 def test_llama_32k():
-    check_layer(gen.workload("llama-32k"), groups=(0, 7))
+    check_layer(gen.workload("llama-32k"))
 
 
 @pytest.mark.parametrize("tau", [0.005, 0.01, 0.02])
 def test_llama_128k_tau_sweep(tau):
-    check_layer(gen.workload("llama-128k", tau=tau), groups=(0,) if tau != 0.01 else (0, 7))
+    check_layer(gen.workload("llama-128k", tau=tau))
+
+
+def test_llama_128k_strong_stripes():
+    """The labelled strong-stripe workload: dozens of selected blocks per query block, so the
+    permuted pass (and the permuted copy of K and V it takes at this density) does most of the
+    work."""
+    selected = check_layer(gen.workload("llama-128k-strong"), n_random=256)
+    assert selected > 100000
 
 
 def test_dense_kernel_full_size_sampled_rows():
@@ -120,10 +132,11 @@ def test_qwen_128k_ablation(variant):
          "S4096": w.replace(segment_len=4096), "qperm-off": w.replace(query_perm=0),
          "shared-keys": w.replace(shared_key_order=1),
          "int4-centroids": w.replace(int4_centroids=1)}[variant]
-    selected = check_layer(w, groups=(3,))
+    selected = check_layer(w, n_random=256 if variant == "tau0.001" else 384)
     if variant == "tau0.001":
         assert selected > 0  # the permuted pass does real work at this threshold
 
 
-def test_stack_layer_densest():
-    check_layer(gen.layer_workload(31), groups=(5,))
+@pytest.mark.parametrize("layer", range(32))
+def test_stack_layer(layer):
+    check_layer(gen.layer_workload(layer), groups=(layer % 8,), n_random=128, seed=layer)

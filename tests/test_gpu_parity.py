@@ -177,13 +177,20 @@ def test_dense_causal_kernel(w):
     assert_close(o, want)
 
 
-def test_tau_zero_matches_dense_causal():
-    w = W_A.replace(tau=0.0)
+@pytest.mark.parametrize("w", [W_TINY.replace(tau=0.0), W_A.replace(tau=0.0)],
+                         ids=["tiny", "a-d128-b128"])
+def test_tau_zero_matches_dense_causal(w):
+    """τ = 0 keeps every candidate block, so the whole path (index build, then both attention
+    passes) is dense causal attention, Eq. 1, on the same bf16 inputs (the tiny configuration's
+    exact dense check; its fp32 inputs are rounded to bf16 before both sides run)."""
     q, k, v = inputs(w)
     want = oracle.dense_causal(oracle.config(w), q, k, v)
     qd, kd, vd = to_dev(q, k, v)
-    o, _ = s2o.attention_prefill(s2o.Config.of(w), qd, kd, vd)
+    cfg = s2o.Config.of(w)
+    o, idx = s2o.attention_prefill(cfg, qd, kd, vd)
     torch.cuda.synchronize()
+    assert s2o.check_device_status() == 0
+    assert s2o.index_stats(cfg, idx).pair_sparsity == 0.0
     assert_close(o, want)
 
 

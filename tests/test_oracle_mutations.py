@@ -32,6 +32,15 @@ MUTATIONS = {
     "dropped-visibility-weight": (
         "w[c] = ns[c] > 0 ? (double)ns[c] * oracle_exp64((double)rb[c] - (double)M) : 0.0;",
         "w[c] = ns[c] > 0 ? oracle_exp64((double)rb[c] - (double)M) : 0.0;"),
+    # Pooled means summed in one pass instead of chunks of B list entries.
+    "one-chunk-sum": ("  float *total = calloc((size_t)d, sizeof(float));",
+                      "  chunk = len;\n  float *total = calloc((size_t)d, sizeof(float));"),
+    # The normaliser Z summed in one pass instead of 32-block chunks.
+    "one-chunk-normaliser": (
+        "for (int c0 = 0; c0 < nB; c0 += 32) {\n      double part = 0.0;\n"
+        "      for (int c = c0; c < c0 + 32 && c < nB; ++c)",
+        "for (int c0 = 0; c0 < nB; c0 += nB) {\n      double part = 0.0;\n"
+        "      for (int c = c0; c < c0 + nB && c < nB; ++c)"),
 }
 
 # The pins that run against each mutant (all CPU, seconds each).
@@ -47,6 +56,8 @@ PIN_TESTS = [
     pins.test_index_arrays_are_sorted_permutations,
     pins.test_probabilities_and_selection_rule,
     pins.test_float64_rederivation_of_pooled_quantities,
+    pins.test_sum_order_case_chunked_means,
+    pins.test_sum_order_case_normaliser_chunks,
 ]
 
 

@@ -403,3 +403,70 @@ def test_int4_centroid_variant():
     b0 = oracle.build_indices(oracle.config(w, tau=0.0), q, k)
     np.testing.assert_array_equal(v0["sel_cnt"], b0["sel_cnt"])
     np.testing.assert_array_equal(np.sort(v0["sel_blk"], axis=-1), np.sort(b0["sel_blk"], axis=-1))
+
+
+# ----------------------------------------------------------------------------- summation orders
+
+SUM_ORDER = os.path.join(os.path.dirname(__file__), "golden", "sum_order_case.json")
+
+
+def _sum_order_case():
+    """Inputs of the hand-derived summation-order case, built from the rules in its JSON."""
+    with open(SUM_ORDER) as f:
+        g = json.load(f)
+    c, inp = g["config"], g["inputs"]
+    N, d = c["seq_len"], c["head_dim"]
+    q = np.zeros((N, d), np.float32)
+    q[:N // 2] = inp["q_segment0_row"]
+    q[N // 2:] = inp["q_segment1_row"]
+    for i, val in inp["q_channel2_overrides"].items():
+        q[int(i), 2] = val
+    k = np.zeros((N, d), np.float32)
+    half = N // 2
+    for j in range(half):
+        v0 = inp["k_channel0"]["key0_and_key64"] if j == 0 else inp["k_channel0"]["other_keys"]
+        k[j, 0] = k[half + j, 0] = v0
+        k[j, 1] = k[half + j, 1] = 63 - j
+    for j, val in inp["k_channel3_overrides"].items():
+        k[int(j), 3] = val
+    to_bf16 = lambda a: torch.from_numpy(a).to(torch.bfloat16).reshape(1, 1, N, d)  # noqa: E731
+    qt, kt = to_bf16(q), to_bf16(k)
+    # Every input value is exact in bf16.
+    assert torch.equal(qt.float().reshape(N, d), torch.from_numpy(q))
+    assert torch.equal(kt.float().reshape(N, d), torch.from_numpy(k))
+    cfg = oracle.Config(c["batch"], c["n_q_heads"], c["n_kv_heads"], N, d, c["segment_len"],
+                        c["block_size"], c["tau"], 1)
+    return g, cfg, qt, kt
+
+
+def test_sum_order_case_chunked_means():
+    """D1's SUM: chunks of B list entries, then the chunk sums in order (hand-derived bits)."""
+    g, cfg, q, k = _sum_order_case()
+    idx = oracle.build_indices(cfg, q, k, debug=True)
+    e = g["expected"]
+    np.testing.assert_array_equal(idx["qbar"][0, 0],
+                                  np.array([float.fromhex(x) for x in e["qbar"]], np.float32))
+    assert idx["kbar_all"][0, 0, 0] == np.float32(float.fromhex(e["kbar_all_channel0"]))
+    assert idx["kbar_all"][0, 0, 3] == np.float32(float.fromhex(e["kbar_all_channel3"]))
+    half = cfg.seq_len // 2
+    want_perm = np.stack([np.arange(half), np.arange(half) + half], axis=1).reshape(-1)
+    np.testing.assert_array_equal(idx["perm_k"][0, 0], want_perm)
+
+
+def test_sum_order_case_normaliser_chunks():
+    """D7's Z: chunks of 32 consecutive blocks, then the chunk sums in order (hand-derived bits
+    of p for the one block that carries almost all the weight)."""
+    g, cfg, q, k = _sum_order_case()
+    idx = oracle.build_indices(cfg, q, k, debug=True)
+    e = g["expected"]
+    nB = cfg.seq_len // cfg.block_size
+    first = (cfg.seq_len // cfg.segment_len - 1) * (cfg.segment_len // cfg.block_size)
+    r = idx["r"][0, 0]
+    assert (r[first:, 0] == np.float32(float.fromhex(e["r_block0"]))).all()
+    assert (r[first:, 1:] == np.float32(float.fromhex(e["r_other_blocks"]))).all()
+    p0 = idx["p"][0, 0, first:, 0]
+    assert (p0 == float.fromhex(e["p_block0_for_segment1_query_blocks"])).all(), p0[:4]
+    assert (idx["sel_cnt"][0, 0, first:] == e["sel_cnt_segment1"]).all()
+    assert (idx["sel_blk"][0, 0, first:, 0] == e["sel_blk0_segment1"]).all()
+    assert (idx["sel_cnt"][0, 0, :first] == 0).all()
+    assert nB > 32  # the normaliser spans more than one 32-block chunk

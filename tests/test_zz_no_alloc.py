@@ -29,11 +29,20 @@ def assert_same_indices(a: s2o.Indices, b: s2o.Indices):
     np.testing.assert_array_equal(np.where(listed, sa, -1), np.where(listed, sb, -1))
 
 
+# The size the array is advertised for: a 32-query-head, 8-KV-head, 32K-token layer with d = 128
+# (its scratch reaches close to the end of the array).
+LLAMA_32K = gen.workload("llama-32k")
+
+
+def test_static_scratch_covers_the_advertised_layer():
+    assert s2o.workspace_size(s2o.Config.of(LLAMA_32K)) <= s2o.STATIC_WORKSPACE_BYTES
+
+
 @pytest.mark.gpu
 def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
-    # Two different layers back to back (the second call finds the first call's leftovers in the
-    # shared array), then the first layer again.
-    for w in (SMALL, MEDIUM, SMALL):
+    # Different layers back to back (each call finds the previous call's leftovers in the shared
+    # array), the largest one the array is sized for among them, then the first layer again.
+    for w in (SMALL, MEDIUM, LLAMA_32K, SMALL):
         cfg = s2o.Config.of(w)
         assert s2o.workspace_size(cfg) <= s2o.STATIC_WORKSPACE_BYTES
         q, k, _ = (t.cuda() for t in gen.make_inputs(w))
