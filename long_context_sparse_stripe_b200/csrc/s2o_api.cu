@@ -61,38 +61,70 @@ s2o_status from_cuda(cudaError_t e) { return e == cudaSuccess ? S2O_OK : S2O_ERR
 size_t copy_bytes(const Dims &d, long long heads) {
   return align256((size_t)heads * (size_t)d.N * (size_t)d.D * 2);
 }
-// Bytes of the block bitmaps and of their counts.
-size_t bits_bytes(const Dims &d) {
-  return align256((size_t)d.bhq() * (size_t)d.nB * (size_t)((d.nB + 31) / 32) * 4);
-}
-size_t bitcnt_bytes(const Dims &d) { return align256((size_t)d.bhq() * (size_t)d.nB * 4); }
-size_t ord_bytes(const Dims &d) {
-  return align256((size_t)d.bhq() * (size_t)d.nB * (size_t)d.nB * 4);
-}
 constexpr size_t kFlagArea = 256;
 
-// Steps 3-4 with the optional permuted copy (copy heads: KV heads when per_kv, else query heads);
-// the copy is used when the workspace holds it and the mode allows it.
+// Chunk words per pair of units in the packed streams: each unit's key blocks at most B/16 chunks
+// each (two units that do not share a copy head or a segment may list the same block), plus the
+// padding of three groups to whole tiles.
+long long chunk_cap(const Dims &d) { return 2ll * d.nB * (d.B / 16) + 3 * (d.B / 16); }
+long long n_pairs(const Dims &d) { return (d.bhq() * d.nB + 1) / 2; }
+
+// Layout of the attention's part of a prefill workspace, after the index build's part (`base`):
+// the decision flag, the per-row log2-sum-exps of the merge path, the permuted copies of K and V,
+// the key positions in block order and the visible counts, the packed streams' chunk lists and
+// per-pair tile counts. Sized for copy heads = query heads (the largest case).
+struct PrefillLayout {
+  size_t flag, lse, kp, vp, pos, vis, chunks, meta, total;
+};
+PrefillLayout prefill_layout(const Dims &d) {
+  PrefillLayout L;
+  size_t off = ws_layout(d).total;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const long long heads = d.bhq();
+  L.flag = take(kFlagArea);
+  L.lse = take((size_t)d.bhq() * d.N * 4);
+  L.kp = take(copy_bytes(d, heads));
+  L.vp = take(copy_bytes(d, heads));
+  L.pos = take((size_t)heads * d.N * 4);
+  L.vis = take((size_t)heads * d.nSeg * d.nB);
+  L.chunks = take((size_t)n_pairs(d) * (size_t)chunk_cap(d) * 4);
+  L.meta = take((size_t)n_pairs(d) * 16);
+  L.total = off;
+  return L;
+}
+
+// Steps 3-4. With a workspace of s2o_prefill_workspace_size bytes (and mode != 3) the merge path
+// runs, with packed streams from the permuted copy when the mode allows them (copy heads: KV heads
+// when per_kv, else query heads); otherwise the path without a workspace.
 s2o_status attention_ws(const s2o_config &c, const void *q, const void *k, const void *v,
                         const s2o_indices &idx, void *o, void *ws, size_t ws_bytes, bool per_kv,
                         cudaStream_t st) {
   const Dims d = dims_of(c);
   AttnArgs a{q, k, v, o, idx.perm_q, idx.perm_k, idx.sel_cnt, idx.sel_blk, idx.local_tiles, false};
   const int mode = g_permuted_copy.load();
-  const size_t base = ws_layout(d).total, cb = copy_bytes(d, per_kv ? d.bhkv() : d.bhq());
-  const size_t bb = bits_bytes(d), nb = bitcnt_bytes(d), ob = ord_bytes(d);
-  if (mode != 0 && ws && ws_bytes >= base + kFlagArea + 2 * cb + bb + nb + ob) {
+  const PrefillLayout L = prefill_layout(d);
+  if (mode != 3 && ws && ws_bytes >= L.total) {
     char *b = static_cast<char *>(ws);
-    uint32_t *flag = reinterpret_cast<uint32_t *>(b + base);
-    a.kp = b + base + kFlagArea;
-    a.vp = b + base + kFlagArea + cb;
-    a.sel_bits = reinterpret_cast<uint32_t *>(b + base + kFlagArea + 2 * cb);
-    a.sel_bitcnt = reinterpret_cast<int32_t *>(b + base + kFlagArea + 2 * cb + bb);
-    a.sel_ord = reinterpret_cast<int32_t *>(b + base + kFlagArea + 2 * cb + bb + nb);
-    a.copy_flag = flag;
-    a.copy_per_kv = per_kv;
-    const cudaError_t e = launch_permuted_copy(d, a, mode, flag, st);
-    if (e != cudaSuccess) return S2O_ERR_CUDA;
+    a.merge = true;
+    a.lse = reinterpret_cast<float *>(b + L.lse);
+    if (mode != 0) {
+      uint32_t *flag = reinterpret_cast<uint32_t *>(b + L.flag);
+      a.kp = b + L.kp;
+      a.vp = b + L.vp;
+      a.pos_sorted = reinterpret_cast<int32_t *>(b + L.pos);
+      a.vis = reinterpret_cast<uint8_t *>(b + L.vis);
+      a.chunks = reinterpret_cast<uint32_t *>(b + L.chunks);
+      a.pair_meta = reinterpret_cast<int4 *>(b + L.meta);
+      a.chunk_cap = chunk_cap(d);
+      a.copy_flag = flag;
+      a.copy_per_kv = per_kv;
+      const cudaError_t e = launch_permuted_copy(d, a, mode, flag, st);
+      if (e != cudaSuccess) return S2O_ERR_CUDA;
+    }
   }
   return from_cuda(launch_attention(d, a, g_wait_limit_ns.load(), g_attention_max_ctas.load(),
                                     st));
@@ -384,9 +416,7 @@ s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes) {
   s2o_status st = check_config(cfg);
   if (st != S2O_OK) return st;
   if (!bytes) return S2O_ERR_INVALID_ARGUMENT;
-  const Dims d = dims_of(*cfg);
-  *bytes = ws_layout(d).total + kFlagArea + 2 * copy_bytes(d, d.bhq()) + bits_bytes(d) +
-           bitcnt_bytes(d) + ord_bytes(d);
+  *bytes = prefill_layout(dims_of(*cfg)).total;
   return S2O_OK;
 }
 

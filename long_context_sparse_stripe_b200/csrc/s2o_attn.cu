@@ -49,6 +49,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -307,6 +308,16 @@ struct FastDiv {
   }
 };
 
+// Kernel instantiations (a launch's mode picks one):
+//   kKindContig  the contiguous modes: the dense local window (local pass) and the dense baseline;
+//   kKindList    the permuted pass over list streams: query blocks gathered by perm_q, selected
+//                blocks gathered row by row by perm_k, in list order (with or without the block's
+//                local tiles, see Params::sel_only);
+//   kKindPacked  the permuted pass over packed streams from the permuted copy of K and V (see
+//                below);
+//   kKindMerge   the local pass that also merges each row with the permuted pass's partial result.
+enum Kind { kKindContig = 0, kKindList = 1, kKindPacked = 2, kKindMerge = 3 };
+
 struct Params {
   const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
   uint16_t *o;
@@ -318,36 +329,47 @@ struct Params {
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned long long limit_ns;
   FastDiv div_G, div_seg, div_nB, div_nSeg, div_Hkv;  // unit-id decoding (S/B blocks a segment)
-  const uint32_t *copy_flag;  // bit 0: the permuted copy of K/V is in use; bit 1: block bitmaps
+  // Permuted pass: 1 when it runs only the selected blocks and leaves the local window to the
+  // local pass (merge path): it writes each row's partial result O_sel (bf16, at the row's place
+  // in O) and its log2-sum-exp into lse_out; 0 when it also reruns the block's local tiles and
+  // writes the final rows (the path without a workspace).
+  int sel_only;
+  float *lse_out;        // permuted pass, sel_only: [b, Hq, N] log2 Σ 2^(s·log2e/√d) per row
+  const float *lse_in;   // kKindMerge: the same array (−inf where no selected block ran)
+  const uint32_t *copy_flag;  // bit 0: the permuted copy is in use (packed streams)
   int copy_per_kv;            // copy rows per KV head (else per query head)
-  const uint32_t *sel_bits;   // per query block, nwords words: bit c set when block c is selected
-  const int32_t *sel_bitcnt;  // per query block, the bitmap's population count
-  const int32_t *sel_ord;     // per query block (nB entries): its selected blocks in block order
-  int nwords;
+  // Packed streams (kKindPacked): per pair of units, chunk words at chunks + pair·chunk_cap (see
+  // k_pack_pairs) and the tile counts {both, only unit 0, only unit 1, -} in pair_meta; pairs
+  // are two heads of one KV head at one block when pair_heads is set, else two consecutive blocks
+  // of one query head.
+  const uint32_t *chunks;
+  const int4 *pair_meta;
+  long long chunk_cap;
+  int pair_heads;
 };
 
 struct Unit {
   long long qh, kh;  // flat (batch, query head) and (batch, kv head)
   int b, seg0, lt, cnt;
-  const int32_t *sel;  // the query block's selected list (sel_blk row; in block order for bitmap
-                       // streams)
+  const int32_t *sel;  // the query block's selected list (sel_blk row)
 };
 
-// Unit order: the local and permuted modes keep the units of one (batch, KV head, segment)
-// together, query heads of the group fastest, so that the segment's K/V tiles stay in L2 and
-// paired units share local tiles; the dense baseline runs the longest query blocks first. With
-// bitmap streams (BITS) the permuted mode instead runs the blocks of one (batch, query head,
-// segment) in a row, so that the two units of a pair position read one key ordering and can share
-// the selected blocks they have in common; their list lengths and block-ordered lists then come
-// from the bitmap kernel.
+// Unit order. The contiguous modes and list streams keep the units of one (batch, KV head,
+// segment) together, query heads of the group fastest, so that the segment's K/V tiles stay in L2
+// and paired units share local tiles; the dense baseline runs the longest query blocks first.
+// Packed streams pair two units that read one copy head and one segment: with a copy per query
+// head the order is (batch, KV head, query head of the group, segment, block), blocks fastest, so
+// that a pair is two consecutive blocks of one query head; with a copy per KV head (pair_heads)
+// it is the list-stream order, so that a pair is two query heads of one KV head at one block.
 template <int BN, int KIND>
 __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
-  constexpr bool BITS = KIND == 2, PERM = KIND != 0;
+  constexpr bool PERM = KIND == kKindList || KIND == kKindPacked;
+  constexpr bool PACKED = KIND == kKindPacked;
   // Unit ids are below 2^31 (the host checks): divisions by multiply-high.
   Unit r;
   uint32_t rem;
   int hi, b, bl;  // query head of the group, block, and the block's index inside its segment
-  if (BITS) {
+  if (PACKED && !p.pair_heads) {
     u = p.div_seg.divmod(u, rem);
     bl = (int)rem;
     u = p.div_nSeg.divmod(u, rem);
@@ -381,42 +403,66 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
     r.lt = bl + 1;  // the causal triangle of the block's segment (or sequence)
     r.cnt = 0;
     r.sel = nullptr;
+  } else if (PACKED) {
+    r.lt = 0;
+    r.cnt = 0;  // set from the pair's tile counts
+    r.sel = nullptr;
   } else {
     const long long qb = r.qh * p.nB + b;
-    r.lt = min(max(__ldg(p.local_tiles + qb), 1), (int)p.div_seg.d);
-    if (BITS) {
-      r.cnt = __ldg(p.sel_bitcnt + qb);
-      r.sel = p.sel_ord + qb * p.nB;
-    } else {
-      r.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
-      r.sel = p.sel_blk + qb * p.nB;
-    }
+    r.lt = p.sel_only ? 0 : min(max(__ldg(p.local_tiles + qb), 1), (int)p.div_seg.d);
+    r.cnt = p.sel_cnt ? min(max(__ldg(p.sel_cnt + qb), 0), p.nB) : 0;
+    r.sel = p.sel_blk + qb * p.nB;
   }
   return r;
 }
 
 struct Pair {
   Unit u0, u1;
-  int valid1;  // the second unit exists (the last work item may hold one)
+  int valid1;  // the second unit exists and has work (the last work item may hold one)
+  int valid0;  // the first unit has work (always, except in a packed pair whose unit 0 has none)
   int shared;  // both units read the same local key tiles
-  int uni;     // stream over the union of both units' selected blocks (bitmap streams)
   int L;       // local items of the stream
   int total;   // stream length
+  // Packed streams: tiles both units use, then tiles of unit 0 only and of unit 1 only
+  // (interleaved), the pair's chunk list, and each unit's copy head.
+  int tb, t0, t1;
+  long long chunk0;
+  long long ch0, ch1;
 };
 
-// Work item i of the current window: units list[2i] and list[2i+1] (the second may be absent:
-// past the list's end, or kNoUnit). With bitmap streams (BITS), a pair that reads one key
-// ordering and one segment (the same query head, or the same KV head when the key ordering is per
-// KV head) walks the union of its two bitmaps: a block both units selected is loaded once for
-// both. Its stream length then needs the union's size (union_size).
+// Work item i of the current window. List streams and the contiguous modes: units list[2i] and
+// list[2i+1] (the second may be absent past the list's end). Packed streams: the pair index is
+// list[2i]; its units are 2·pair and 2·pair + 1.
 constexpr uint32_t kNoUnit = 0xffffffffu;
 template <int BN, int KIND>
 __device__ __forceinline__ Pair decode_pair(const Params &p, const uint32_t *list, int n_list,
                                             int i) {
-  constexpr bool BITS = KIND == 2;
+  constexpr bool PACKED = KIND == kKindPacked;
   Pair P;
+  if (PACKED) {
+    const uint32_t w = list[2 * i];
+    const int4 m = __ldg(p.pair_meta + w);
+    P.tb = m.x;
+    P.t0 = m.y;
+    P.t1 = m.z;
+    P.chunk0 = (long long)w * p.chunk_cap;
+    P.u0 = decode_unit<BN, KIND>(p, 2 * w);
+    const bool has1 = 2ll * w + 1 < p.n_units;
+    P.u1 = has1 ? decode_unit<BN, KIND>(p, 2 * w + 1) : P.u0;
+    P.u0.cnt = P.tb + P.t0;
+    P.u1.cnt = has1 ? P.tb + P.t1 : 0;
+    P.valid0 = P.u0.cnt > 0;
+    P.valid1 = P.u1.cnt > 0;
+    P.shared = 0;
+    P.L = 0;
+    P.total = P.tb + P.t0 + P.t1;
+    P.ch0 = (p.copy_per_kv ? P.u0.kh : P.u0.qh) * p.N;
+    P.ch1 = (p.copy_per_kv ? P.u1.kh : P.u1.qh) * p.N;
+    return P;
+  }
   P.u0 = decode_unit<BN, KIND>(p, list[2 * i]);
-  P.valid1 = 2 * i + 1 < n_list && (!BITS || list[2 * i + 1] != kNoUnit);
+  P.valid0 = 1;
+  P.valid1 = 2 * i + 1 < n_list;
   if (P.valid1) {
     P.u1 = decode_unit<BN, KIND>(p, list[2 * i + 1]);
   } else {
@@ -425,68 +471,13 @@ __device__ __forceinline__ Pair decode_pair(const Params &p, const uint32_t *lis
     P.u1.cnt = 0;
   }
   P.shared = P.valid1 && P.u0.kh == P.u1.kh && P.u0.seg0 == P.u1.seg0;
-  P.uni = BITS && P.shared && (P.u0.qh == P.u1.qh || p.copy_per_kv);
   P.L = P.shared ? max(P.u0.lt, P.u1.lt) : P.u0.lt + P.u1.lt;
   P.total = P.L + P.u0.cnt + P.u1.cnt;
+  P.tb = P.t0 = P.t1 = 0;
+  P.chunk0 = 0;
+  P.ch0 = P.ch1 = 0;
   return P;
 }
-
-// A unit's block bitmap (bitmap streams).
-__device__ __forceinline__ const uint32_t *unit_bits(const Params &p, const Unit &u) {
-  return p.sel_bits + (u.qh * p.nB + u.b) * p.nwords;
-}
-
-// Blocks selected by either unit of a union pair (serial; or, with all 32 lanes, one word each).
-__device__ __forceinline__ int union_size(const Params &p, const Pair &P) {
-  const uint32_t *b0 = unit_bits(p, P.u0), *b1 = unit_bits(p, P.u1);
-  int n = 0;
-  for (int w = 0; w < p.nwords; ++w) n += __popc(__ldg(b0 + w) | __ldg(b1 + w));
-  return n;
-}
-__device__ __forceinline__ int union_size_warp(const Params &p, const Pair &P, int lane) {
-  const uint32_t *b0 = unit_bits(p, P.u0), *b1 = unit_bits(p, P.u1);
-  int n = 0;
-  for (int w = lane; w < p.nwords; w += 32) n += __popc(__ldg(b0 + w) | __ldg(b1 + w));
-  for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-  return n;
-}
-
-// The union of two block bitmaps in block order, with the units that selected each block; the
-// next words are loaded one word ahead.
-struct UnionCursor {
-  const uint32_t *r0, *r1;
-  int nwords, w;
-  uint32_t m0, m1, n0, n1;
-  __device__ __forceinline__ void init(const uint32_t *a, const uint32_t *b, int n) {
-    r0 = a;
-    r1 = b;
-    nwords = n;
-    w = 0;
-    m0 = n > 0 ? __ldg(a) : 0u;
-    m1 = n > 0 ? __ldg(b) : 0u;
-    n0 = n > 1 ? __ldg(a + 1) : 0u;
-    n1 = n > 1 ? __ldg(b + 1) : 0u;
-  }
-  __device__ __forceinline__ int next(int &users) {
-    while ((m0 | m1) == 0) {
-      if (++w >= nwords) {
-        users = 0;
-        return -1;
-      }
-      m0 = n0;
-      m1 = n1;
-      n0 = w + 1 < nwords ? __ldg(r0 + w + 1) : 0u;
-      n1 = w + 1 < nwords ? __ldg(r1 + w + 1) : 0u;
-    }
-    const int i = __ffs(m0 | m1) - 1;
-    const uint32_t bit = 1u << i;
-    users = ((m0 & bit) ? 1 : 0) | ((m1 & bit) ? 2 : 0);
-    m0 &= ~bit;
-    m1 &= ~bit;
-    return 32 * w + i;
-  }
-};
-
 
 // Position j of a two-way interleaving of a items of unit 0 and b items of unit 1 (alternating
 // while both have items left): the unit x and its item index.
@@ -499,6 +490,36 @@ __device__ __forceinline__ void interleave(int a, int b, int j, int &x, int &idx
     x = a > b ? 0 : 1;
     idx = m + (j - 2 * m);
   }
+}
+
+// Packed stream item j: the units that use it (bit x for unit x), the tile's index in the pair's
+// chunk list, and the copy rows it is loaded from.
+struct PackedItem {
+  int users, tile;
+  long long ch;
+};
+__device__ __forceinline__ PackedItem packed_item(const Pair &P, int j) {
+  PackedItem it;
+  if (j >= P.total) {
+    it.users = 0;
+    it.tile = 0;
+    it.ch = P.ch0;
+  } else if (j < P.tb) {
+    it.users = 3;
+    it.tile = j;
+    it.ch = P.ch0;
+  } else {
+    int x, idx;
+    interleave(P.t0, P.t1, j - P.tb, x, idx);
+    it.users = 1 << x;
+    it.tile = P.tb + (x ? P.t0 : 0) + idx;
+    it.ch = x ? P.ch1 : P.ch0;
+  }
+  return it;
+}
+// The chunk-list tile of unit x's n-th packed tile.
+__device__ __forceinline__ int packed_unit_tile(const Pair &P, int x, int n) {
+  return n < P.tb ? n : P.tb + (x ? P.t0 : 0) + (n - P.tb);
 }
 
 // Stream item j: which units use it (bit x), the unit whose indices locate its rows, whether it is
@@ -535,7 +556,9 @@ __device__ __forceinline__ Item item_at(const Pair &P, int j) {
 }
 
 // The units that use stream item j (bit x for unit x; 0 past the end).
+template <int KIND>
 __device__ __forceinline__ int users_at(const Pair &P, int j) {
+  if (KIND == kKindPacked) return packed_item(P, j).users;
   if (j >= P.total) return 0;
   int x, idx;
   if (j < P.L) {
@@ -569,9 +592,9 @@ __device__ __forceinline__ int4 block_rows(const Params &p, const Unit &u, int c
 // atom; gathered rows (prepared by block_rows): tile::gather4, four rows per lane.
 template <int D, int BN>
 __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap *tm_tile,
-                                        const CUtensorMap *tm_row, const CUtensorMap *tm_copy,
-                                        const Params &p, const Pair &P, const Item &it, int4 rows,
-                                        int c, bool use_copy, uint32_t bar, int lane) {
+                                        const CUtensorMap *tm_row, const Params &p,
+                                        const Pair &P, const Item &it, int4 rows, uint32_t bar,
+                                        int lane) {
   using L = Layout<D, BN>;
   const Unit &u = it.x ? P.u1 : P.u0;
   if (it.local) {
@@ -579,17 +602,29 @@ __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap *tm_tile
       for (int a = 0; a < D / 64; ++a)
         tma_load_tile(dst + a * L::ATOM_KV, tm_tile, a * 64,
                       (int)(u.kh * p.N) + u.seg0 + it.t * BN, bar);
-  } else if (use_copy) {
-    // Selected block c of the permuted copy: contiguous rows c·B.. of the unit's copy head.
-    if (lane == 0) {
-      const long long h = p.copy_per_kv ? u.kh : u.qh;
-      for (int a = 0; a < D / 64; ++a)
-        tma_load_tile(dst + a * L::ATOM_KV, tm_copy, a * 64, (int)(h * p.N) + c * BN, bar);
-    }
   } else if (lane < BN / 4) {
     for (int a = 0; a < D / 64; ++a)
       tma_gather4(dst + a * L::ATOM_KV + lane * 4 * 128, tm_row, a * 64, rows.x, rows.y, rows.z,
                   rows.w, bar);
+  }
+}
+
+// Chunks of a packed tile: 16 rows of the permuted copy each (BN/16 per tile).
+constexpr int kChunkRows = 16;
+
+// Loads one packed tile (all 32 lanes call it; the transaction count has been set): lane c < BN/16
+// loads chunk c, the 16 copy rows its chunk word names (row16 = word >> 5, in units of 16 rows of
+// the copy head whose first row is `ch`), with one TMA tile load of a {64, 16} box per 64-column
+// atom into rows 16c..16c+15 of the stage. Chunks past a group's end name rows 0..15 of the copy
+// head and are masked by the softmax.
+template <int D, int BN>
+__device__ __forceinline__ void load_packed(uint32_t dst, const CUtensorMap *tm_copy16,
+                                            long long ch, uint32_t word, uint32_t bar, int lane) {
+  using L = Layout<D, BN>;
+  if (lane < BN / kChunkRows) {
+    const int row = (int)(ch + (long long)(word >> 5) * kChunkRows);
+    for (int a = 0; a < D / 64; ++a)
+      tma_load_tile(dst + a * L::ATOM_KV + lane * kChunkRows * 128, tm_copy16, a * 64, row, bar);
   }
 }
 
@@ -693,38 +728,26 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // Fills the work list for window k0 of this CTA's share (warp 0; returns the entry count, or -1
 // past the end of the share). Without skipping, the share is the work items w = blockIdx.x +
 // k·gridDim.x, each contributing its units 2w and 2w+1 (adjacent units, which usually share
-// local tiles); with skip_empty it is the units u = blockIdx.x + k·gridDim.x whose selected list
-// is not empty, paired in list order. With bitmap streams (BITS; always skip_empty) the share is
-// again the work items w, each contributing those of its units 2w and 2w+1 whose list is not
-// empty (the second slot kNoUnit when only one is), so that a pair is two consecutive blocks of
-// one query head.
+// local tiles); with skip_empty (list streams) it is the units u = blockIdx.x + k·gridDim.x whose
+// selected list is not empty, paired in list order. Packed streams: the share is the pairs
+// w = blockIdx.x + k·gridDim.x that have a tile, each pair index at an even list position.
 template <int BN, int KIND>
 __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lane) {
-  constexpr bool BITS = KIND == 2;
-  const bool by_unit = p.skip_empty && !BITS;
+  constexpr bool PACKED = KIND == kKindPacked;
+  const bool by_unit = p.skip_empty && !PACKED;
   const long long span = by_unit ? kList : kList / 2;
   const long long first = blockIdx.x + k0 * gridDim.x;
   if (first >= (by_unit ? p.n_units : p.n_items)) return -1;
-  // Whether unit u (permuted-mode order) has a non-empty selected list.
+  // Whether unit u (list-stream order) has a non-empty selected list.
   auto busy = [&](long long u) -> bool {
     if (u >= p.n_units || !p.sel_cnt) return false;
     const int per_seg = p.S / BN;
-    int hi, bl, sg;
-    if (BITS) {
-      bl = (int)(u % per_seg);
-      u /= per_seg;
-      sg = (int)(u % p.nSeg);
-      u /= p.nSeg;
-      hi = (int)(u % p.G);
-      u /= p.G;
-    } else {
-      hi = (int)(u % p.G);
-      u /= p.G;
-      bl = (int)(u % per_seg);
-      u /= per_seg;
-      sg = (int)(u % p.nSeg);
-      u /= p.nSeg;
-    }
+    const int hi = (int)(u % p.G);
+    u /= p.G;
+    const int bl = (int)(u % per_seg);
+    u /= per_seg;
+    const int sg = (int)(u % p.nSeg);
+    u /= p.nSeg;
     const int g = (int)(u % p.Hkv);
     const long long qh = (u / p.Hkv) * p.Hq + (long long)g * p.G + hi;
     return __ldg(p.sel_cnt + qh * p.nB + sg * per_seg + bl) > 0;
@@ -737,14 +760,17 @@ __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lan
       const unsigned m = __ballot_sync(0xffffffffu, keep);
       if (keep) list[n + __popc(m & ((1u << lane) - 1u))] = (uint32_t)pos;
       n += __popc(m);
-    } else if (BITS) {
-      const bool b0 = pos < p.n_items && busy(2 * pos), b1 = pos < p.n_items && busy(2 * pos + 1);
-      const bool keep = b0 || b1;
+    } else if (PACKED) {
+      bool keep = false;
+      if (pos < p.n_items) {
+        const int4 m = __ldg(p.pair_meta + pos);
+        keep = m.x + m.y + m.z > 0;
+      }
       const unsigned m = __ballot_sync(0xffffffffu, keep);
       if (keep) {
         const int at = n + 2 * __popc(m & ((1u << lane) - 1u));
-        list[at] = (uint32_t)(b0 ? 2 * pos : 2 * pos + 1);
-        list[at + 1] = b0 && b1 ? (uint32_t)(2 * pos + 1) : kNoUnit;
+        list[at] = (uint32_t)pos;
+        list[at + 1] = kNoUnit;
       }
       n += 2 * __popc(m);
     } else {
@@ -766,10 +792,10 @@ __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lan
 
 // ------------------------------------------------------------------ the kernel
 
-// KIND 0: the contiguous modes (local pass, dense baseline), compiled without the permuted
-// pass's code; 1: the permuted pass with list streams; 2: the permuted pass with bitmap streams.
-// A permuted launch given block bitmaps (sel_bits) runs only if the decision flag chose bitmap
-// streams (KIND 2) or did not (KIND 1): the host launches both and one returns at once.
+// One instantiation per Kind (see the Kind enum), so that the hot local pass carries none of the
+// permuted pass's code. A permuted launch that has a decision flag runs only when the flag chose
+// its form (packed streams when bit 0 is set, list streams when it is clear): the host launches
+// both and one returns at once.
 template <int D, int BN, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     s2o_attention_kernel(const __grid_constant__ CUtensorMap tm_q_tile,
@@ -779,12 +805,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_v_tile,
                          const __grid_constant__ CUtensorMap tm_v_row,
                          const __grid_constant__ CUtensorMap tm_o_tile,
-                         const __grid_constant__ CUtensorMap tm_kp_tile,
-                         const __grid_constant__ CUtensorMap tm_vp_tile, const Params p) {
+                         const __grid_constant__ CUtensorMap tm_kp16,
+                         const __grid_constant__ CUtensorMap tm_vp16, const Params p) {
   using L = Layout<D, BN>;
-  constexpr bool BITS = KIND == 2, PERM = KIND != 0;
+  constexpr bool PERM = KIND == kKindList || KIND == kKindPacked;
+  constexpr bool PACKED = KIND == kKindPacked;
+  constexpr bool MERGE = KIND == kKindMerge;
+  constexpr int CPT = BN / kChunkRows;  // chunks per packed tile
   const uint32_t flagv = p.copy_flag != nullptr ? __ldg(p.copy_flag) : 0u;
-  if (PERM && p.sel_bits != nullptr && ((flagv & 3u) == 3u) != BITS) return;
+  if (PERM && p.copy_flag != nullptr && ((flagv & 1u) != 0u) != PACKED) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -839,16 +868,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint64_t lim = p.limit_ns;
   bool ok = true;
-  // Set before the launch by the permuted-copy decision: selected blocks come from the permuted
-  // copy (bit 0), in block order from the block bitmaps (bit 1, only with bit 0).
-  const bool use_copy = PERM && (flagv & 1u) != 0u;
   // Work comes in windows of this CTA's share: warp 0 fills the work list between two CTA-wide
   // barriers and every role then walks the window's items (a role that gave up a bounded wait
   // keeps meeting the barriers without working).
   uint32_t *list = reinterpret_cast<uint32_t *>(smem + L::OFF_LIST);
   volatile int *list_n = reinterpret_cast<volatile int *>(smem + L::OFF_LIST + kList * 4);
   auto for_each_window = [&](auto &&body) {
-    for (long long k0 = 0;; k0 += p.skip_empty && !BITS ? kList : kList / 2) {
+    for (long long k0 = 0;; k0 += p.skip_empty && !PACKED ? kList : kList / 2) {
       named_bar_sync(1, kThreads);
       if (warp == 0) {
         const int n = build_list<BN, KIND>(p, k0, list, lane);
@@ -871,48 +897,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int full0 = is_k ? kKFull : kVFull, empty0 = is_k ? kKEmpty : kVEmpty;
     const CUtensorMap *tm_tile = is_k ? &tm_k_tile : &tm_v_tile;
     const CUtensorMap *tm_row = is_k ? &tm_k_row : &tm_v_row;
-    const CUtensorMap *tm_copy = is_k ? &tm_kp_tile : &tm_vp_tile;
+    const CUtensorMap *tm_copy16 = is_k ? &tm_kp16 : &tm_vp16;
     long long kj = 0;  // stream items issued so far (all work items of this CTA)
-    // One stream item into the next ring stage.
-    auto issue = [&](const Pair &P, const Item &it, int4 rows, int c) -> bool {
+    // Waits for the next ring stage and sets its transaction count; false if the wait ran out.
+    auto next_stage = [&](uint32_t &dst, uint32_t &fb) -> bool {
       const int st = (int)(kj % stages);
       if (kj >= stages &&
           !warp_wait(bar(empty0 + st), (uint32_t)(((kj / stages) - 1) & 1), lim, lane))
         return false;
       if (lane == 0) mbar_expect_tx(bar(full0 + st), L::KV_BYTES);
       __syncwarp();
-      load_kv<D, BN>(ring + st * L::KV_BYTES, tm_tile, tm_row, tm_copy, p, P, it, rows, c,
-                     use_copy, bar(full0 + st), lane);
+      dst = ring + st * L::KV_BYTES;
+      fb = bar(full0 + st);
       ++kj;
       return true;
     };
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-      Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
-      if (BITS && P.uni) {
-        // Union stream: local tiles, then each block either unit selected, once, from the
-        // permuted copy.
-        P.total = P.L + union_size_warp(p, P, lane);
-        UnionCursor uc;
-        uc.init(unit_bits(p, P.u0), unit_bits(p, P.u1), p.nwords);
+      const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
+      if (PACKED) {
+        // Packed tiles: this lane's chunk word of the next item is loaded before the wait for
+        // the current item's stage.
+        auto word_of = [&](int j) -> uint32_t {
+          if (j >= P.total || lane >= CPT) return 0u;
+          const PackedItem t = packed_item(P, j);
+          return __ldg(p.chunks + P.chunk0 + (long long)t.tile * CPT + lane);
+        };
+        uint32_t w_cur = word_of(0);
         for (int j = 0; ok && j < P.total; ++j) {
-          Item it;
-          int c = -1;
-          if (j < P.L) {
-            it = item_at(P, j);
-          } else {
-            c = uc.next(it.users);
-            it.x = 0;
-            it.local = 0;
-            it.t = 0;
+          const uint32_t w_next = word_of(j + 1);
+          uint32_t dst, fb;
+          if (!next_stage(dst, fb)) {
+            ok = false;
+            break;
           }
-          ok = issue(P, it, make_int4(0, 0, 0, 0), c);
+          load_packed<D, BN>(dst, tm_copy16, packed_item(P, j).ch, w_cur, fb, lane);
+          w_cur = w_next;
         }
         continue;
       }
       if (!PERM) {
         // Contiguous modes: local tiles only.
-        for (int j = 0; ok && j < P.total; ++j) ok = issue(P, item_at(P, j), make_int4(0, 0, 0, 0), -1);
+        for (int j = 0; ok && j < P.total; ++j) {
+          uint32_t dst, fb;
+          if (!next_stage(dst, fb)) {
+            ok = false;
+            break;
+          }
+          load_kv<D, BN>(dst, tm_tile, tm_row, p, P, item_at(P, j), make_int4(0, 0, 0, 0), fb,
+                         lane);
+        }
         continue;
       }
       // Gathered rows are looked up ahead: the rows of item j+1 and the block of item j+2 are
@@ -924,7 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return t.local ? -1 : sel_block(p, t.x ? P.u1 : P.u0, t.t);
       };
       auto rows_of = [&](int j, int c) -> int4 {
-        if (j >= P.total || c < 0 || use_copy) return make_int4(0, 0, 0, 0);
+        if (j >= P.total || c < 0) return make_int4(0, 0, 0, 0);
         const Item t = item_at(P, j);
         return block_rows<BN>(p, t.x ? P.u1 : P.u0, c, lane);
       };
@@ -934,13 +968,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < P.total; ++j) {
         const Item it = item_at(P, j);
         const int4 rows_next = rows_of(j + 1, c_next);
-        const int c_this = c_cur;
         c_cur = c_next;
         c_next = block_of(j + 2);
-        if (!issue(P, it, rows, c_this)) {
+        uint32_t dst, fb;
+        if (!next_stage(dst, fb)) {
           ok = false;
           break;
         }
+        load_kv<D, BN>(dst, tm_tile, tm_row, p, P, it, rows, fb, lane);
         rows = rows_next;
       }
     }
@@ -954,7 +989,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
       const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
-      for (int x = 0; ok && x < 1 + P.valid1; ++x) {
+      for (int x = 0; ok && x < 2; ++x) {
+        if (!(x ? P.valid1 : P.valid0)) continue;
         if (qn[x] >= 1 &&
             !warp_wait(bar(kQEmpty + x), (uint32_t)((qn[x] - 1) & 1), lim, lane)) {
           ok = false;
@@ -1076,20 +1112,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
       if (lane == 0) {
       for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
-        Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
-        // A union stream's selected part is walked once, item by item, for its users.
-        UnionCursor uc;
-        if (BITS && P.uni) {
-          P.total = P.L + union_size(p, P);
-          uc.init(unit_bits(p, P.u0), unit_bits(p, P.u1), p.nwords);
-        }
-        auto users_seq = [&](int j) -> int {
-          if (!BITS || !P.uni || j < P.L || j >= P.total) return users_at(P, j);
-          int us;
-          uc.next(us);
-          return us;
-        };
-        const int n_of[2] = {P.u0.lt + P.u0.cnt, P.u1.lt + P.u1.cnt};
+        const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
+        auto users_seq = [&](int j) -> int { return users_at<KIND>(P, j); };
+        const int n_of[2] = {P.u0.lt + P.u0.cnt, P.valid1 ? P.u1.lt + P.u1.cnt : 0};
         int qk[2] = {0, 0};
         // One unit's step at stream item j: its pending product goes first, or now if the unit
         // skips the next item (its V tile must leave the ring); a unit's first Q_x·Kᵀ waits for
@@ -1167,7 +1192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
       const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
-      if (x == 1 && !P.valid1) continue;
+      if (!(x ? P.valid1 : P.valid0)) continue;
       const Unit u = x ? P.u1 : P.u0;
       const int seg0 = u.seg0;
       // Original position of this row's query (padding rows: the segment's last position).
@@ -1185,16 +1210,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Keys of a selected block (for its mask) are requested before the wait for its S, the
       // block id one tile earlier.
       auto blk = [&](int n) {
-        return PERM && n >= u.lt && n < n_items ? sel_block(p, u, n - u.lt) : -1;
+        return PERM && !PACKED && n >= u.lt && n < n_items ? sel_block(p, u, n - u.lt) : -1;
       };
       int c_cur = blk(0), c_next = blk(1);
+      // MERGE: the partial result of the permuted pass for this row is requested early.
+      float lse_sel = -INFINITY;
+      if (MERGE && store_row) lse_sel = __ldg(p.lse_in + (size_t)u.qh * p.N + i_orig);
       for (int n = 0; n < n_items; ++n) {
+        // Per column group q (columns 32q..32q+31, this lane's column 32q + lane): the key's
+        // original position (list streams), or the word of the chunk holding the column (packed
+        // streams: chunk 2q + lane/16 of the tile).
         int keys[BN / 32];
+        if (PACKED) {
+          const long long cw0 = P.chunk0 + (long long)packed_unit_tile(P, x, n) * CPT + (lane >> 4);
 #pragma unroll
-        for (int q = 0; q < BN / 32; ++q)
-          keys[q] = c_cur < 0 ? 0 : __ldg(p.perm_k + u.qh * p.N + (size_t)c_cur * BN + q * 32 + lane);
-        c_cur = c_next;
-        c_next = blk(n + 2);
+          for (int q = 0; q < BN / 32; ++q) keys[q] = (int)__ldg(p.chunks + cw0 + 2 * q);
+        } else {
+#pragma unroll
+          for (int q = 0; q < BN / 32; ++q)
+            keys[q] = c_cur < 0 ? 0 : __ldg(p.perm_k + u.qh * p.N + (size_t)c_cur * BN + q * 32 + lane);
+          c_cur = c_next;
+          c_next = blk(n + 2);
+        }
         // Warp-uniform outcome: the tcgen05.ld below is a warp-collective instruction.
         if (!__all_sync(full, mbar_wait(bar(kSFull + x), (uint32_t)(sn & 1), lim))) {
           ok = false;
@@ -1219,11 +1256,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c > limit) s[c] = __float_as_uint(-INFINITY);
           }
         } else {
+          // Permuted tiles: keys before the segment (list streams), or the first v rows of each
+          // 16-row chunk, v in the chunk word's low five bits (packed streams).
           uint32_t mw[BN / 32];
           bool all = true;
 #pragma unroll
           for (int q = 0; q < BN / 32; ++q) {
-            mw[q] = __ballot_sync(full, keys[q] >= 0 && keys[q] < seg0);
+            const bool valid = PACKED ? (int)(lane & 15) < (keys[q] & 31)
+                                      : keys[q] >= 0 && keys[q] < seg0;
+            mw[q] = __ballot_sync(full, valid);
             all = all && mw[q] == full;
           }
           if (!all) {
@@ -1246,8 +1287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                fmaxf(mp[6], mp[7]));
         const float m_new = fmaxf(m_run, mt * sl2);
         const bool rescale = m_new > m_run + 8.0f;
-        float m_use = rescale ? m_new : m_run;
-        if (m_use == -INFINITY) m_use = 0.f;
+        const float m_keep = rescale ? m_new : m_run;
+        // A row whose columns are all masked so far has no maximum: its exponents use 0, and (in
+        // the permuted pass, where that can happen) its running maximum stays −inf.
+        const float m_use = m_keep == -INFINITY ? 0.f : m_keep;
         const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
         // P = 2^(s·log2(e)/√d − m) as bf16 pairs, written over the first BN/2 columns of S_x.
         float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1279,7 +1322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         l_run = l_run * alpha + rs;
-        m_run = m_use;
+        m_run = PERM ? m_keep : m_use;
         // One arrival per warp (after the warp's tensor-memory stores): arrivals on one barrier
         // are serialised, so 128 of them would delay the product by hundreds of cycles.
         tc_fence_before();
@@ -1296,6 +1339,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       uint16_t *orow = p.o + ((size_t)u.qh * p.N + i_orig) * D;
+      // MERGE: the row's final result combines this pass's O/ℓ with the permuted pass's partial
+      // result o_sel (bf16, at the row's place in O) by their log2-sum-exps:
+      // o = (2^lse_loc·O/ℓ + 2^lse_sel·o_sel) / (2^lse_loc + 2^lse_sel).
+      float so = inv_l, ss = 0.f;
+      if (MERGE && lse_sel > -INFINITY) {
+        const float ll = m_run + __log2f(l_run);
+        const float mm = fmaxf(ll, lse_sel);
+        const float wa = ex2(ll - mm), wb = ex2(lse_sel - mm);
+        const float inv = 1.f / (wa + wb);
+        so = wa * inv * inv_l;
+        ss = wb * inv;
+      }
+      if (PERM && p.sel_only) {
+        // Partial result of the selected blocks: its log2-sum-exp for the merge (−inf, and no
+        // row written, when no key of the row was visible).
+        if (store_row)
+          p.lse_out[(size_t)u.qh * p.N + i_orig] = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+        store_row = store_row && l_run > 0.f;
+      }
       // The whole row of O from TMEM (one wait), then 32-byte stores (full sectors).
       uint32_t o[D];
 #pragma unroll
@@ -1312,16 +1374,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned char *ostp = smem + L::OFF_OST + x * L::ATOM_Q + row * 128;
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) {
+          // MERGE: this atom of o_sel, read before the stage wait (its row is this thread's).
+          uint4 sel[8];
+          if (MERGE) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              sel[ch] = ss != 0.f ? __ldg(reinterpret_cast<const uint4 *>(orow + a * 64 + ch * 8))
+                                  : make_uint4(0, 0, 0, 0);
+          }
           if (leader) bulk_wait_read();
           named_bar_sync(2 + x, 128);
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const int c = a * 64 + ch * 8;
             uint4 v;
-            v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
-            v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
-            v.z = pack_bf16(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
-            v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
+            if (MERGE) {
+              auto mix = [&](int cc, uint32_t w2) {
+                const float lo = __uint_as_float(w2 << 16), hi = __uint_as_float(w2 & 0xffff0000u);
+                return pack_bf16(fmaf(__uint_as_float(o[cc]), so, lo * ss),
+                                 fmaf(__uint_as_float(o[cc + 1]), so, hi * ss));
+              };
+              v.x = mix(c + 0, sel[ch].x);
+              v.y = mix(c + 2, sel[ch].y);
+              v.z = mix(c + 4, sel[ch].z);
+              v.w = mix(c + 6, sel[ch].w);
+            } else {
+              v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+              v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
+              v.z = pack_bf16(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
+              v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
+            }
             *reinterpret_cast<uint4 *>(ostp + ((ch ^ (row & 7)) * 16)) = v;
           }
           fence_proxy_async_smem();
@@ -1381,12 +1463,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // ------------------------------------------------------------------ permuted copy of K and V
 
-// Whether the permuted pass uses the permuted copy (bit 0): always (modes 2 and 3), or (mode 1)
-// when the selected blocks of all query blocks outnumber twice the blocks the copy writes; copying
-// a block costs about one gather of it, and each selected block then loads as a contiguous tile.
-// Whether it also runs bitmap streams (bit 1): always in mode 3, or (mode 1, with the copy) when
-// the selected blocks fill at least an eighth of all pairs of query block and key block, so that
-// the bitmaps are dense enough to walk word by word. One CTA.
+// Whether the permuted pass runs packed streams from the permuted copy (bit 0 of *flag): always
+// (mode 2), or (mode 1) when the selected blocks of all query blocks outnumber twice the blocks
+// the copy writes (copying a block costs about one gather of it, and each selected block then
+// loads as contiguous chunks). One CTA.
 __global__ void __launch_bounds__(1024)
     k_copy_decide(const int32_t *__restrict__ sel_cnt, long long n_units, int nB, int mode,
                   long long copy_blocks, uint32_t *__restrict__ flag) {
@@ -1401,66 +1481,77 @@ __global__ void __launch_bounds__(1024)
     unsigned long long total = 0;
     for (int w = 0; w < (int)(blockDim.x / 32); ++w) total += part[w];
     const bool copy =
-        mode >= 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks);
-    const bool dense = mode == 3 || (mode == 1 && copy &&
-                                     total >= (unsigned long long)n_units * (unsigned long long)nB / 8);
-    // Merging into the local rows (bit 2) when at least 1 % of the query blocks have a
-    // selection: below that the permuted pass is too small to repay the local pass's extra
-    // softmax-state stores.
-    *flag = (copy ? 1u : 0u) | (dense ? 2u : 0u);
+        mode == 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks);
+    *flag = copy ? 1u : 0u;
   }
 }
 
-// Block bitmaps of the selected lists (flag bit 1 only): one warp per query block sets bit c of
-// word c/32 for each listed block c (clamped into range), then writes the bitmap, its population
-// count and the selected blocks in block order (each lane the set bits of its words, after the
-// blocks of the words before them).
+// The (batch, query head) of copy head h: the head itself, or the first query head of KV head h
+// when the copy is per KV head.
+__device__ __forceinline__ long long copy_query_head(long long h, int per_kv, int Hq, int Hkv,
+                                                     int G) {
+  return per_kv ? (h / Hkv) * Hq + (h % Hkv) * G : h;
+}
+
+// Key order inside each block of the permuted copy (bit 0 only): one warp per (copy head, key
+// block) sorts the block's B original positions ascending (ranks by (position, slot), so any
+// index contents give a permutation of the block's slots) into pos_sorted, and counts for every
+// segment s the block's keys before s·S into vis[h][s][c]. With the rows of a block in position
+// order, the keys of block c that a query of segment s may see (original position < s·S) are its
+// first vis[h][s][c] rows.
+template <int B>
 __global__ void __launch_bounds__(256)
-    k_sel_bits(const int32_t *__restrict__ sel_cnt, const int32_t *__restrict__ sel_blk,
-               long long n_units, int nB, int nwords, const uint32_t *__restrict__ flag,
-               uint32_t *__restrict__ bits, int32_t *__restrict__ bitcnt,
-               int32_t *__restrict__ ord) {
-  if ((__ldg(flag) & 2u) == 0u) return;
-  __shared__ uint32_t sw[8][64];
-  const unsigned full = 0xffffffffu;
+    k_block_sort(const int32_t *__restrict__ perm_k, int32_t *__restrict__ pos_sorted,
+                 uint8_t *__restrict__ vis, long long copy_heads, int N, int S, int nB, int nSeg,
+                 int Hq, int Hkv, int G, int per_kv, const uint32_t *__restrict__ flag) {
+  if ((__ldg(flag) & 1u) == 0u) return;
+  constexpr int E = B / 32;
+  __shared__ int sv[8][B];
+  __shared__ int ss[8][B];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const long long qb = (long long)blockIdx.x * 8 + warp;
-  if (qb >= n_units) return;
-  for (int w = lane; w < nwords; w += 32) sw[warp][w] = 0u;
-  __syncwarp();
-  const int cnt = min(max(__ldg(sel_cnt + qb), 0), nB);
-  const int32_t *row = sel_blk + qb * nB;
-  for (int e = lane; e < cnt; e += 32) {
-    const int c = min(max(__ldg(row + e), 0), nB - 1);
-    atomicOr(&sw[warp][c >> 5], 1u << (c & 31));
+  const long long gw = (long long)blockIdx.x * 8 + warp;
+  if (gw >= copy_heads * nB) return;
+  const long long h = gw / nB;
+  const int c = (int)(gw % nB);
+  const long long qh = copy_query_head(h, per_kv, Hq, Hkv, G);
+  const int32_t *src = perm_k + qh * N + (long long)c * B;
+  int x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    x[e] = min(max(__ldg(src + e * 32 + lane), 0), N - 1);
+    sv[warp][e * 32 + lane] = x[e];
   }
   __syncwarp();
-  int32_t *ord_row = ord + qb * nB;
-  int run = 0;
-  for (int w0 = 0; w0 < nwords; w0 += 32) {
-    const int w = w0 + lane;
-    const uint32_t v = w < nwords ? sw[warp][w] : 0u;
-    const int pc = __popc(v);
-    int incl = pc;
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(full, incl, o);
-      if (lane >= o) incl += t;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = e * 32 + lane;
+    int rank = 0;
+    for (int j = 0; j < B; ++j) {
+      const int y = sv[warp][j];
+      rank += (y < x[e] || (y == x[e] && j < i)) ? 1 : 0;
     }
-    int at = run + incl - pc;
-    for (uint32_t m = v; m; m &= m - 1) ord_row[at++] = 32 * w + __ffs(m) - 1;
-    if (w < nwords) bits[qb * nwords + w] = v;
-    run += __shfl_sync(full, incl, 31);
+    ss[warp][rank] = x[e];
+    pos_sorted[h * N + (long long)c * B + rank] = x[e];
   }
-  if (lane == 0) bitcnt[qb] = run;
+  __syncwarp();
+  for (int s = lane; s < nSeg; s += 32) {
+    const int bound = s * S;
+    int lo = 0, hi = B;  // first slot whose position is >= bound
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (ss[warp][mid] < bound) lo = mid + 1;
+      else hi = mid;
+    }
+    vis[((size_t)h * nSeg + s) * nB + c] = (uint8_t)lo;
+  }
 }
 
-// kp[h·N + rank] = K row perm_k[hq(h)][rank] of h's KV head, and the same for V (h a query head,
-// or a KV head whose first query head's ordering is used). 16-byte pieces, grid-stride; nothing
-// when the flag's copy bit is clear.
+// kp[h·N + rank] = K row pos_sorted[h·N + rank] of h's KV head, and the same for V (h a copy
+// head). 16-byte pieces, grid-stride; nothing when the flag's bit 0 is clear.
 template <int D>
 __global__ void __launch_bounds__(256)
     k_permute_kv(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
-                 const int32_t *__restrict__ perm_k, uint4 *__restrict__ kp,
+                 const int32_t *__restrict__ pos_sorted, uint4 *__restrict__ kp,
                  uint4 *__restrict__ vp, long long copy_rows, int N, int Hq, int Hkv, int G,
                  int per_kv, const uint32_t *__restrict__ flag) {
   if ((__ldg(flag) & 1u) == 0u) return;
@@ -1471,21 +1562,132 @@ __global__ void __launch_bounds__(256)
     const long long row = x / PIECES;
     const int piece = (int)(x % PIECES);
     const long long h = row / N;
-    const int rank = (int)(row % N);
-    // (batch, head) of the copy row, its KV head, and the query head whose ordering it follows.
-    const int heads = per_kv ? Hkv : Hq;
-    const long long beta = h / heads;
-    const int hh = (int)(h % heads);
-    const long long kh = beta * Hkv + (per_kv ? hh : hh / G);
-    const long long qh = beta * Hq + (per_kv ? hh * G : hh);
-    const int j = min(max(__ldg(perm_k + qh * N + rank), 0), N - 1);
+    // KV head of copy head h.
+    const long long kh = per_kv ? h : (h / Hq) * Hkv + (h % Hq) / G;
+    const int j = min(max(__ldg(pos_sorted + row), 0), N - 1);
     const long long src = (kh * N + j) * PIECES + piece;
     kp[x] = __ldg(k + src);
     vp[x] = __ldg(v + src);
   }
 }
 
+// Packed streams (bit 0 only): one warp per pair of units (units 2w and 2w+1 in packed order).
+// Each unit's selected list becomes a bitmap of key blocks in shared memory. When both units have
+// selections and read one copy head and one segment, the blocks both selected form the pair's
+// shared group and the rest each unit's own group; otherwise each unit's blocks are its own group.
+// Every group, in block order, is cut into chunks of 16 rows of the permuted copy: block c gives
+// ceil(n/16) chunks for its n visible keys (n = vis of the unit's copy head, segment and c), chunk
+// i covering rows 16i.. of the block, of which min(16, n − 16i) are visible. The chunk word is
+// (row16 << 5) | visible, row16 = c·B/16 + i the chunk's place in the copy head. Each group is
+// padded with empty chunks (row16 0, visible 0) to whole tiles of BN/16 chunks; the pair's list is
+// [shared group][unit 0's group][unit 1's group] from chunks + w·cap, and pair_meta[w] holds the
+// three tile counts. cap = 2·nB·B/16 + 3·B/16 holds two units' blocks with their padding.
+template <int BN>
+__global__ void __launch_bounds__(256)
+    k_pack_pairs(const int32_t *__restrict__ sel_cnt, const int32_t *__restrict__ sel_blk,
+                 const uint8_t *__restrict__ vis, uint32_t *__restrict__ chunks,
+                 int4 *__restrict__ pair_meta, long long cap, long long n_units, int nB, int S,
+                 int nSeg, int Hq, int Hkv, int G, int per_kv, int pair_heads,
+                 const uint32_t *__restrict__ flag) {
+  if ((__ldg(flag) & 1u) == 0u) return;
+  constexpr int CPT = BN / kChunkRows;
+  constexpr int kMaxWords = 64;  // nB <= 2048
+  __shared__ uint32_t sw[8][2][kMaxWords];
+  const unsigned full = 0xffffffffu;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long long w = (long long)blockIdx.x * 8 + warp;
+  const long long n_pairs = (n_units + 1) / 2;
+  if (w >= n_pairs) return;
+  const int nwords = (nB + 31) / 32, per_seg = S / BN;
+  long long qh[2], hc[2];
+  int sg[2], cnt[2];
+  for (int x = 0; x < 2; ++x) {
+    long long u = 2 * w + x;
+    const bool has = u < n_units;
+    if (!has) u = 2 * w;
+    int hi, bl, s;
+    if (!pair_heads) {
+      bl = (int)(u % per_seg);
+      u /= per_seg;
+      s = (int)(u % nSeg);
+      u /= nSeg;
+      hi = (int)(u % G);
+      u /= G;
+    } else {
+      hi = (int)(u % G);
+      u /= G;
+      bl = (int)(u % per_seg);
+      u /= per_seg;
+      s = (int)(u % nSeg);
+      u /= nSeg;
+    }
+    const int g = (int)(u % Hkv);
+    const long long beta = u / Hkv;
+    qh[x] = beta * Hq + (long long)g * G + hi;
+    hc[x] = per_kv ? beta * Hkv + g : qh[x];
+    sg[x] = s;
+    const long long qb = qh[x] * nB + (long long)s * per_seg + bl;
+    cnt[x] = has ? min(max(__ldg(sel_cnt + qb), 0), nB) : 0;
+    for (int i = lane; i < kMaxWords; i += 32) sw[warp][x][i] = 0u;
+    __syncwarp();
+    const int32_t *row = sel_blk + qb * nB;
+    for (int e = lane; e < cnt[x]; e += 32) {
+      const int c = min(max(__ldg(row + e), 0), nB - 1);
+      atomicOr(&sw[warp][x][c >> 5], 1u << (c & 31));
+    }
+    __syncwarp();
+  }
+  const bool shared = cnt[0] > 0 && cnt[1] > 0 && hc[0] == hc[1] && sg[0] == sg[1];
+  uint32_t *out = chunks + w * cap;
+  long long pos = 0;  // chunks written so far (warp-uniform)
+  int T[3];
+  for (int grp = 0; grp < 3; ++grp) {
+    const long long start = pos;
+    const int x = grp == 2 ? 1 : 0;
+    const uint8_t *vrow = vis + ((size_t)hc[x] * nSeg + sg[x]) * nB;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+      const int wd = w0 + lane;
+      uint32_t m = 0u;
+      if (wd < nwords) {
+        const uint32_t a = sw[warp][0][wd], b = sw[warp][1][wd];
+        m = grp == 0 ? (shared ? a & b : 0u) : grp == 1 ? (shared ? a & ~b : a)
+                                                       : (shared ? b & ~a : b);
+      }
+      int mine = 0;
+      for (uint32_t r = m; r; r &= r - 1) {
+        const int c = 32 * wd + __ffs(r) - 1;
+        mine += (__ldg(vrow + c) + kChunkRows - 1) / kChunkRows;
+      }
+      int incl = mine;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(full, incl, o);
+        if (lane >= o) incl += t;
+      }
+      long long at = pos + incl - mine;
+      for (uint32_t r = m; r; r &= r - 1) {
+        const int c = 32 * wd + __ffs(r) - 1;
+        const int n = __ldg(vrow + c);
+        for (int i = 0; i * kChunkRows < n; ++i) {
+          const uint32_t row16 = (uint32_t)c * (BN / kChunkRows) + (uint32_t)i;
+          out[at++] = (row16 << 5) | (uint32_t)min(kChunkRows, n - i * kChunkRows);
+        }
+      }
+      pos += __shfl_sync(full, incl, 31);
+    }
+    T[grp] = (int)((pos - start + CPT - 1) / CPT);
+    const long long end = start + (long long)T[grp] * CPT;
+    for (long long i = pos + lane; i < end; i += 32) out[i] = 0u;
+    pos = end;
+  }
+  if (lane == 0) pair_meta[w] = make_int4(T[0], T[1], T[2], 0);
+}
 
+// Rows without a partial result from the permuted pass: lse = −inf.
+__global__ void __launch_bounds__(256) k_fill_neg_inf(float *__restrict__ p, long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    p[i] = -INFINITY;
+}
 
 // 2-D bf16 tensor map over a [rows, D] row-major matrix, box {64 columns, box_rows}, 128-byte
 // swizzle (one 64-column atom per box row is exactly one 128-byte swizzle span).
@@ -1528,19 +1730,22 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
       !make_map(&tv, a.v, kv_rows, D, BN) || !make_map(&tvr, a.v, kv_rows, D, 1) ||
       !make_map(&to, a.o, q_rows, D, BN))
     return cudaErrorInvalidValue;
-  // The permuted copy's maps (without a copy they repeat K's and V's and are never used).
-  const bool copy = a.copy_flag != nullptr && a.kp != nullptr && a.vp != nullptr;
+  // The permuted copy's maps, 16-row boxes (without a copy they repeat K's and V's row maps and
+  // are never used).
+  const bool packed = a.merge && a.copy_flag != nullptr && a.kp != nullptr && a.vp != nullptr &&
+                      a.chunks != nullptr && a.pair_meta != nullptr;
   const long long copy_rows = (a.copy_per_kv ? d.bhkv() : d.bhq()) * d.N;
-  if (copy) {
-    if (!make_map(&tkp, a.kp, copy_rows, D, BN) || !make_map(&tvp, a.vp, copy_rows, D, BN))
+  if (packed) {
+    if (!make_map(&tkp, a.kp, copy_rows, D, kChunkRows) ||
+        !make_map(&tvp, a.vp, copy_rows, D, kChunkRows))
       return cudaErrorInvalidValue;
   } else {
-    tkp = tk;
-    tvp = tv;
+    tkp = tkr;
+    tvp = tvr;
   }
   cudaError_t e = cudaSuccess;
-  for (auto fn : {s2o_attention_kernel<D, BN, 0>, s2o_attention_kernel<D, BN, 1>,
-                  s2o_attention_kernel<D, BN, 2>})
+  for (auto fn : {s2o_attention_kernel<D, BN, kKindContig>, s2o_attention_kernel<D, BN, kKindList>,
+                  s2o_attention_kernel<D, BN, kKindPacked>, s2o_attention_kernel<D, BN, kKindMerge>})
     if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)L::SMEM)) != cudaSuccess)
       return e;
@@ -1565,72 +1770,120 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   p.div_G.init(d.G);
   p.div_nB.init(d.nB);
   p.div_Hkv.init(d.Hkv);
-  p.copy_flag = copy ? a.copy_flag : nullptr;
+  p.sel_only = 0;
+  p.lse_out = nullptr;
+  p.lse_in = nullptr;
+  p.copy_flag = a.merge ? a.copy_flag : nullptr;
   p.copy_per_kv = a.copy_per_kv ? 1 : 0;
-  const bool bitmaps = copy && a.sel_bits && a.sel_bitcnt && a.sel_ord;
-  p.sel_bits = bitmaps ? a.sel_bits : nullptr;
-  p.sel_bitcnt = bitmaps ? a.sel_bitcnt : nullptr;
-  p.sel_ord = bitmaps ? a.sel_ord : nullptr;
-  p.nwords = (d.nB + 31) / 32;
-  auto launch = [&](int mode, int skip_empty, bool bits) -> cudaError_t {
+  p.chunks = a.chunks;
+  p.pair_meta = a.pair_meta;
+  p.chunk_cap = a.chunk_cap;
+  p.pair_heads = a.copy_per_kv ? 1 : 0;
+  auto launch = [&](int mode, int skip_empty, int kind) -> cudaError_t {
     p.mode = mode;
     p.skip_empty = skip_empty;
     p.S = mode == kDense ? d.N : d.S;
     p.nSeg = mode == kDense ? 1 : d.nSeg;
     p.div_seg.init(p.S / BN);
     p.div_nSeg.init(p.nSeg);
-    const long long work = skip_empty && !bits ? p.n_units : p.n_items;
+    const long long work = skip_empty && kind == kKindList ? p.n_units : p.n_items;
     const long long cap = max_ctas > 0 && max_ctas < sm_count() ? max_ctas : sm_count();
     const long long grid = work < cap ? work : cap;
-    if (mode != kPermuted)
-      s2o_attention_kernel<D, BN, 0><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
-          tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
-    else if (bits)
-      s2o_attention_kernel<D, BN, 2><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
-          tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
-    else
-      s2o_attention_kernel<D, BN, 1><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
-          tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+    switch (kind) {
+      case kKindContig:
+        s2o_attention_kernel<D, BN, kKindContig><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+            tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+        break;
+      case kKindList:
+        s2o_attention_kernel<D, BN, kKindList><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+            tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+        break;
+      case kKindPacked:
+        s2o_attention_kernel<D, BN, kKindPacked><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+            tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+        break;
+      default:
+        s2o_attention_kernel<D, BN, kKindMerge><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+            tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+    }
     note_launch();
     return cudaGetLastError();
   };
-  if (a.dense) return launch(kDense, 0, false);
-  // S2O: every row first gets the dense local window of its segment, computed in original order
-  // (causal triangles, masks on diagonal tiles only); then the query blocks whose selected list is
-  // not empty are recomputed in full (local tiles and selected blocks, permuted order) and
-  // overwrite their rows. Each row's result is the attention over its key set either way. With
-  // block bitmaps the permuted pass is launched in both forms and the device flag picks one.
-  if ((e = launch(kLocal, 0, false)) != cudaSuccess) return e;
-  if ((e = launch(kPermuted, 1, false)) != cudaSuccess) return e;
-  return p.sel_bits != nullptr ? launch(kPermuted, 1, true) : cudaSuccess;
+  if (a.dense) return launch(kDense, 0, kKindContig);
+  if (!a.merge || a.lse == nullptr) {
+    // Without a workspace: every row first gets the dense local window of its segment, computed
+    // in original order (causal triangles, masks on diagonal tiles only); then the query blocks
+    // whose selected list is not empty are recomputed in full (local tiles and selected blocks,
+    // permuted order) and overwrite their rows. Each row's result is the attention over its key
+    // set either way.
+    if ((e = launch(kLocal, 0, kKindContig)) != cudaSuccess) return e;
+    return launch(kPermuted, 1, kKindList);
+  }
+  // Merge path: the permuted pass runs only the selected blocks and leaves each row's partial
+  // result and its log2-sum-exp (−inf for rows it does not reach); the local pass then computes
+  // the local window in original order and merges the two. The permuted pass is launched in both
+  // forms when the device-side decision may pick packed streams; one returns at once.
+  const long long n_rows = d.bhq() * d.N;
+  const unsigned fill_grid = (unsigned)std::min<long long>((n_rows + 255) / 256, 148ll * 16);
+  k_fill_neg_inf<<<fill_grid, 256, 0, st>>>(a.lse, n_rows);
+  note_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  p.sel_only = 1;
+  p.lse_out = a.lse;
+  if ((e = launch(kPermuted, 1, kKindList)) != cudaSuccess) return e;
+  if (packed && (e = launch(kPermuted, 1, kKindPacked)) != cudaSuccess) return e;
+  p.sel_only = 0;
+  p.lse_out = nullptr;
+  p.lse_in = a.lse;
+  return launch(kLocal, 0, kKindMerge);
 }
 
 }  // namespace
 
 cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
                                  cudaStream_t st) {
-  if (!a.kp || !a.vp || !flag || !a.sel_cnt || !a.perm_k) return cudaErrorInvalidValue;
-  const long long copy_rows = (a.copy_per_kv ? d.bhkv() : d.bhq()) * d.N;
-  k_copy_decide<<<1, 1024, 0, st>>>(a.sel_cnt, d.bhq() * d.nB, d.nB, mode, copy_rows / d.B, flag);
+  if (!a.kp || !a.vp || !flag || !a.sel_cnt || !a.perm_k || !a.pos_sorted || !a.vis ||
+      !a.chunks || !a.pair_meta)
+    return cudaErrorInvalidValue;
+  const long long copy_heads = a.copy_per_kv ? d.bhkv() : d.bhq();
+  const long long copy_rows = copy_heads * d.N;
+  const long long n_units = d.bhq() * d.nB;
+  k_copy_decide<<<1, 1024, 0, st>>>(a.sel_cnt, n_units, d.nB, mode, copy_rows / d.B, flag);
   note_launch();
-  if (a.sel_bits && a.sel_bitcnt && a.sel_ord) {
-    const long long n_units = d.bhq() * d.nB;
-    k_sel_bits<<<(unsigned)((n_units + 7) / 8), 256, 0, st>>>(
-        a.sel_cnt, a.sel_blk, n_units, d.nB, (d.nB + 31) / 32, flag, a.sel_bits, a.sel_bitcnt,
-        const_cast<int32_t *>(a.sel_ord));
-    note_launch();
-  }
+  const unsigned sort_grid = (unsigned)((copy_heads * d.nB + 7) / 8);
+  if (d.B == 128)
+    k_block_sort<128><<<sort_grid, 256, 0, st>>>(a.perm_k, a.pos_sorted, a.vis, copy_heads, d.N,
+                                                 d.S, d.nB, d.nSeg, d.Hq, d.Hkv, d.G,
+                                                 a.copy_per_kv ? 1 : 0, flag);
+  else
+    k_block_sort<64><<<sort_grid, 256, 0, st>>>(a.perm_k, a.pos_sorted, a.vis, copy_heads, d.N,
+                                                d.S, d.nB, d.nSeg, d.Hq, d.Hkv, d.G,
+                                                a.copy_per_kv ? 1 : 0, flag);
+  note_launch();
   const unsigned grid = (unsigned)sm_count() * 8u;
   if (d.D == 128)
     k_permute_kv<128><<<grid, 256, 0, st>>>(
-        static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.perm_k,
+        static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.pos_sorted,
         static_cast<uint4 *>(const_cast<void *>(a.kp)), static_cast<uint4 *>(const_cast<void *>(a.vp)),
         copy_rows, d.N, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0, flag);
   else
     k_permute_kv<64><<<grid, 256, 0, st>>>(
-        static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.perm_k,
+        static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.pos_sorted,
         static_cast<uint4 *>(const_cast<void *>(a.kp)), static_cast<uint4 *>(const_cast<void *>(a.vp)),
         copy_rows, d.N, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0, flag);
+  note_launch();
+  const long long n_pairs = (n_units + 1) / 2;
+  const unsigned pack_grid = (unsigned)((n_pairs + 7) / 8);
+  if (d.B == 128)
+    k_pack_pairs<128><<<pack_grid, 256, 0, st>>>(a.sel_cnt, a.sel_blk, a.vis, a.chunks,
+                                                 a.pair_meta, a.chunk_cap, n_units, d.nB, d.S,
+                                                 d.nSeg, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0,
+                                                 a.copy_per_kv ? 1 : 0, flag);
+  else
+    k_pack_pairs<64><<<pack_grid, 256, 0, st>>>(a.sel_cnt, a.sel_blk, a.vis, a.chunks,
+                                                a.pair_meta, a.chunk_cap, n_units, d.nB, d.S,
+                                                d.nSeg, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0,
+                                                a.copy_per_kv ? 1 : 0, flag);
   note_launch();
   return cudaGetLastError();
 }

@@ -42,29 +42,32 @@ struct AttnArgs {
   void *o;
   const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
   bool dense;
-  // Optional permuted copy of K and V: row rank of copy head h at h·N + rank holds the key/value
-  // row perm_k[head][rank]. The permuted pass loads its selected blocks from it (tile loads
-  // instead of row gathers) when *copy_flag is non-zero; copy_flag == nullptr means no copy.
-  // Copy heads are query heads, or KV heads when copy_per_kv is set (one key ordering per KV
-  // head).
+  // Merge path (a workspace of s2o_prefill_workspace_size bytes): the permuted pass runs only
+  // the selected blocks and writes each row's partial result and its log2-sum-exp into lse
+  // [bhq, N]; the local pass then merges. Without it (merge false) the permuted pass reruns each
+  // busy block's local tiles and overwrites its rows.
+  bool merge = false;
+  float *lse = nullptr;
+  // Optional permuted copy of K and V for packed streams: row rank of copy head h at h·N + rank
+  // holds the key/value row pos_sorted[h·N + rank], the keys of each block of perm_k in position
+  // order. Copy heads are query heads, or KV heads when copy_per_kv is set (one key ordering per
+  // KV head). Used when *copy_flag has bit 0 set; copy_flag == nullptr means no copy.
   const void *kp = nullptr, *vp = nullptr;
   const uint32_t *copy_flag = nullptr;
   bool copy_per_kv = false;
-  // Block bitmaps of the selected lists (ceil(nB/32) words per query block), their population
-  // counts and the selected blocks in block order (nB entries per query block), filled when the
-  // decision also sets the flag's bit 1; the permuted pass then runs the selected blocks in block
-  // order and shares the blocks two paired query blocks both selected.
-  uint32_t *sel_bits = nullptr;
-  int32_t *sel_bitcnt = nullptr;
-  const int32_t *sel_ord = nullptr;  // per query block: its selected blocks in block order
+  int32_t *pos_sorted = nullptr;  // [copy heads, N]
+  uint8_t *vis = nullptr;         // [copy heads, nSeg, nB] visible keys of each block per segment
+  uint32_t *chunks = nullptr;     // [pairs, chunk_cap] chunk words of the packed streams
+  int4 *pair_meta = nullptr;      // [pairs] tile counts {shared, unit 0 only, unit 1 only, -}
+  long long chunk_cap = 0;
 };
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
                              int max_ctas, cudaStream_t st);
-// The permuted copy for the permuted pass: a decision kernel sets bit 0 of *flag when `mode` is 2
-// or 3, or when it is 1 and the selected blocks outnumber twice the copied blocks, and bit 1 (block
-// bitmaps) when `mode` is 3, or when it is 1, bit 0 is set and the selected blocks fill at least an
-// eighth of all (query block, key block) pairs; the copy kernel then fills a.kp and a.vp and the
-// bitmap kernel a.sel_bits, a.sel_bitcnt and a.sel_ord (each does nothing when its bit is clear).
+// The permuted copy for packed streams: a decision kernel sets bit 0 of *flag when `mode` is 2, or
+// when it is 1 and the selected blocks outnumber twice the copied blocks; then (each doing nothing
+// when the bit is clear) the blocks of perm_k are put in position order (a.pos_sorted, a.vis), K
+// and V are copied in that order (a.kp, a.vp), and each pair of units gets its chunk list
+// (a.chunks, a.pair_meta).
 cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
                                  cudaStream_t st);
 

@@ -119,15 +119,19 @@ def test_workspace_views_are_inside_the_workspace():
 # ----------------------------------------------------------------------------- prefill + layer
 
 
-def test_prefill_workspace_holds_the_copy_and_the_bitmaps():
+def test_prefill_workspace_holds_the_merge_and_packed_stream_buffers():
     cfg = LLAMA_128K
     base = s2o.workspace_size(cfg)
     full = s2o.prefill_workspace_size(cfg)
-    nB = 1024
-    copy = 2 * 32 * 131072 * 128 * 2          # K and V in each query head's key order
-    bitmaps = 32 * nB * (nB // 32 + 1 + nB) * 4  # bitmaps, their counts, block-ordered lists
-    assert full - base >= copy + bitmaps
-    assert full - base <= copy + bitmaps + 4096
+    Hq, N, d, B, S = 32, 131072, 128, 128, 2048
+    nB, nSeg = N // B, N // S
+    lse = Hq * N * 4                          # per-row log2-sum-exps of the merge path
+    copy = 2 * Hq * N * d * 2                 # K and V in each query head's key order
+    positions = Hq * N * 4 + Hq * nSeg * nB   # block-ordered key positions, visible counts
+    pairs = Hq * nB // 2
+    chunks = pairs * (2 * nB * (B // 16) + 3 * (B // 16)) * 4 + pairs * 16  # chunk lists, counts
+    want = lse + copy + positions + chunks
+    assert want <= full - base <= want + 4096
 
 
 def test_permuted_copy_modes_are_accepted():

@@ -305,20 +305,48 @@ def test_attention_independent_of_grid_and_windows():
         s2o.set_attention_max_ctas(0)
 
 
-# ----------------------------------------------------------------------------- permuted copy
+# ----------------------------------------------------------------------------- merge path, packed streams
+
+# Strong stripes (dozens of selected blocks per query block) on shapes the oracle finishes in
+# seconds: d = 128 with B = 128, and d = 64 with B = 64 and 32 blocks per segment.
+W_S1 = gen.Workload("s1-strong-d128", batch=1, n_q_heads=4, n_kv_heads=1, seq_len=8192,
+                    head_dim=128, segment_len=1024, block_size=128, tau=0.01, seed=21, amp=16.0,
+                    stripe_frac=0.05, q_shift=4.0)
+W_S2 = gen.Workload("s2-strong-d64-b64", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=8192,
+                    head_dim=64, segment_len=2048, block_size=64, tau=0.01, seed=22, amp=12.0,
+                    stripe_frac=0.05, q_shift=4.0)
+# Ragged: two batch elements, 96 blocks, 1536-query segments (12 blocks), 3 query heads per KV head
+# (pairs of heads straddle KV heads under one key ordering per KV head).
+W_S3 = gen.Workload("s3-strong-ragged", batch=2, n_q_heads=6, n_kv_heads=2, seq_len=12288,
+                    head_dim=128, segment_len=1536, block_size=128, tau=0.005, seed=23, amp=16.0,
+                    stripe_frac=0.05, q_shift=4.0)
+
 
 def _copy_flag(cfg, ws):
     at = s2o.workspace_size(cfg)
     return int(ws[at:at + 4].cpu().numpy().view(np.uint32)[0])
 
 
+def _with_mode(mode, fn):
+    try:
+        s2o.set_permuted_copy(mode)
+        out = fn()
+        torch.cuda.synchronize()
+        return out
+    finally:
+        s2o.set_permuted_copy(1)
+
+
 @pytest.mark.parametrize("w", [W_A.replace(tau=0.0), W_C.replace(tau=0.0), W_D.replace(tau=0.0),
-                               W_F.replace(tau=0.0), W_A.replace(tau=0.01)],
-                         ids=lambda w: f"{w.name}-tau{w.tau}")
-def test_permuted_copy_matches_gathers_and_oracle(w):
-    """Selected blocks loaded as tiles of the permuted copy of K and V give exactly the bits of
-    the row gathers (mode 2, on the oracle's indices); bitmap streams (mode 3: block order, the
-    blocks two paired query blocks share loaded once) give the oracle's result."""
+                               W_F.replace(tau=0.0), W_A.replace(tau=0.01), W_S1, W_S2, W_S3,
+                               W_S3.replace(query_perm=0)],
+                         ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
+def test_merge_and_packed_paths_match_oracle(w):
+    """On the oracle's indices, every form of steps 3-4 gives the oracle's output: the merge path
+    with gathered selected blocks (mode 0), the merge path with packed streams from the permuted
+    copy (mode 2: only the visible keys of each block, in 16-row chunks, blocks two paired query
+    blocks both selected loaded once), and the path without a workspace (mode 3: the permuted pass
+    reruns the local tiles)."""
     q, k, v = inputs(w)
     ocfg = oracle.config(w)
     ref = oracle.build_indices(ocfg, q, k)
@@ -327,28 +355,20 @@ def test_permuted_copy_matches_gathers_and_oracle(w):
     cfg = s2o.Config.of(w)
     idx = oracle_indices_on_device(ref)
     ws = s2o.alloc_prefill_workspace(cfg)
-    outs = {}
-    try:
-        for mode, flag in ((0, None), (2, 1), (3, 3)):
-            s2o.set_permuted_copy(mode)
-            outs[mode] = s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws)
-            torch.cuda.synchronize()
-            if flag is not None:
-                assert _copy_flag(cfg, ws) == flag
-    finally:
-        s2o.set_permuted_copy(1)
-    assert s2o.check_device_status() == 0
-    assert torch.equal(outs[0], outs[2])
-    assert_close(outs[2], want)
-    assert_close(outs[3], want)
+    for mode, flag in ((0, None), (2, 1), (3, None)):
+        o = _with_mode(mode, lambda: s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx,
+                                                                           ws))
+        assert s2o.check_device_status() == 0, mode
+        if flag is not None:
+            assert _copy_flag(cfg, ws) == flag
+        assert_close(o, want)
 
 
 def test_permuted_copy_decision():
-    """Mode 1 copies only when the selected blocks outnumber twice the copied blocks, and runs
-    bitmap streams only when they also fill an eighth of the block pairs: with every block
-    selected (τ = 0) it does both, with none (τ > 1) neither; a workspace of s2o_workspace_size
-    bytes never copies and gives the same output."""
-    for w, expect in ((W_A.replace(tau=0.0), 3), (W_A.replace(tau=1.5), 0)):
+    """Mode 1 copies only when the selected blocks outnumber twice the copied blocks: with every
+    block selected (τ = 0) it does, with none (τ > 1) it does not; with no selection the merge path
+    gives the bits of the path without a workspace."""
+    for w, expect in ((W_A.replace(tau=0.0), 1), (W_A.replace(tau=1.5), 0)):
         q, k, v = to_dev(*inputs(w))
         cfg = s2o.Config.of(w)
         idx = s2o.build_indices(cfg, q, k)
@@ -364,31 +384,46 @@ def test_permuted_copy_decision():
             assert torch.equal(o, o_small)
 
 
-def test_permuted_copy_per_kv_head_under_shared_key_order():
-    """The whole path with one key ordering per KV head copies K and V once per KV head: the copy
-    alone (mode 2) equals the gather path bit for bit, bitmap streams (mode 3) agree with it
-    within the parity tolerance on sampled rows, and the indices stay the oracle's."""
-    w = W_B.replace(tau=0.001, shared_key_order=1)
+@pytest.mark.parametrize("w", [W_B.replace(tau=0.001), W_S3], ids=["b-ragged", "s3-strong"])
+def test_permuted_copy_per_kv_head_under_shared_key_order(w):
+    """The whole path with one key ordering per KV head copies K and V once per KV head and pairs
+    two query heads of a KV head at one block, so a block both selected is loaded once for both:
+    every mode agrees with the oracle on sampled rows, and the indices stay the oracle's."""
+    w = w.replace(shared_key_order=1)
     q, k, v = inputs(w)
     ocfg = oracle.config(w)
     ref = oracle.build_indices(ocfg, q, k)
     qd, kd, vd = to_dev(q, k, v)
     cfg = s2o.Config.of(w)
     ws = s2o.alloc_prefill_workspace(cfg)
-    outs = {}
-    try:
-        for mode in (0, 2, 3):
-            s2o.set_permuted_copy(mode)
-            outs[mode], idx = s2o.attention_prefill(cfg, qd, kd, vd, ws=ws)
-            torch.cuda.synchronize()
-    finally:
-        s2o.set_permuted_copy(1)
-    assert s2o.check_device_status() == 0
-    assert int(idx.sel_cnt.sum()) > 0
-    assert_indices_equal(idx, ref, cfg.n_blocks)
-    assert torch.equal(outs[0], outs[2])
     rng = np.random.default_rng(1)
-    rows = rng.choice(w.batch * w.n_q_heads * w.seq_len, 1500, replace=False)
-    want, _ = oracle.attention(ocfg, q, k, v, ref, rows=np.sort(rows))
-    got = outs[3].reshape(-1, w.head_dim)[torch.from_numpy(np.sort(rows)).cuda()]
-    assert_close(got, want)
+    rows = np.sort(rng.choice(w.batch * w.n_q_heads * w.seq_len, 1500, replace=False))
+    want, _ = oracle.attention(ocfg, q, k, v, ref, rows=rows)
+    for mode in (0, 2, 3):
+        o, idx = _with_mode(mode, lambda: s2o.attention_prefill(cfg, qd, kd, vd, ws=ws))
+        assert s2o.check_device_status() == 0
+        assert int(idx.sel_cnt.sum()) > 0
+        assert_indices_equal(idx, ref, cfg.n_blocks)
+        got = o.reshape(-1, w.head_dim)[torch.from_numpy(rows).cuda()]
+        assert_close(got, want)
+
+
+def test_packed_path_independent_of_grid_and_windows():
+    """Packed streams and the merge with a grid of one, two or five CTAs (several work-list windows
+    each) give the same bits as the full grid."""
+    w = W_S3
+    q, k, v = inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w)
+    idx = s2o.build_indices(cfg, qd, kd)
+    ws = s2o.alloc_prefill_workspace(cfg)
+    base = _with_mode(2, lambda: s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws))
+    try:
+        for n in (1, 2, 5):
+            s2o.set_attention_max_ctas(n)
+            o = _with_mode(2, lambda: s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx,
+                                                                            ws))
+            assert s2o.check_device_status() == 0
+            assert torch.equal(o, base), f"grid of {n}"
+    finally:
+        s2o.set_attention_max_ctas(0)
