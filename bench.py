@@ -201,12 +201,14 @@ def cpu_oracle_sample(w, q, k, v, max_rows=2048, seed=0):
     return full, desc, threads
 
 
-def workload_config(name, w, world):
+def workload_config(name, w, world, parallel="replica"):
     """The bench line's ``config`` (the same keys on both arms)."""
+    par = (f"one layer split by KV head over {world} GPUs" if parallel == "heads"
+           else f"independent layer per GPU x{world}")
     return {"workload": name, "batch": w.batch, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "seq_len": w.seq_len, "head_dim": w.head_dim,
             "segment_len": w.segment_len, "block_size": w.block_size, "tau": w.tau,
-            "query_perm": w.query_perm, "parallelism": f"independent layer per GPU x{world}",
+            "query_perm": w.query_perm, "parallelism": par,
             "l2": "inputs larger than L2 (Q is 1.07 GB); no flush"}
 
 
@@ -235,7 +237,7 @@ def run_reference(args):
         "sample_ms_per_step": float(np.median(walls)) * 1e3,
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(args.workload, w, args.gpus),
+        "config": workload_config(args.workload, w, args.gpus, args.parallel),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -251,9 +253,19 @@ def run_s2o(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = gen.workload(args.workload, tau=args.tau)
-    # Each rank runs its own independent layer (weak scaling).
-    q, k, v = gen.make_inputs(w.replace(seed=layer_seed(w, rank)))
-    cfg = s2o.Config.of(w)
+    if args.parallel == "heads":
+        # One layer split by KV head: this rank's KV heads g (g mod world = rank) with their
+        # query heads; no data-path collective (strong scaling).
+        from long_context_sparse_stripe_b200 import shard
+        q, k, v = shard.shard_inputs(*gen.make_inputs(w), rank, world)
+        wr = shard.shard_config(w, rank, world)
+        job_flops = w.dense_causal_flops
+    else:
+        # Each rank runs its own independent layer (weak scaling).
+        q, k, v = gen.make_inputs(w.replace(seed=layer_seed(w, rank)))
+        wr = w
+        job_flops = w.dense_causal_flops * world
+    cfg = s2o.Config.of(wr)
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     o = torch.empty_like(qd)
     idx = s2o.alloc_indices(cfg, dev)
@@ -303,14 +315,13 @@ def run_s2o(args):
 
     stats = s2o.index_stats(cfg, idx, ws)
     tile_flops = 4.0 * w.block_size * w.block_size * w.head_dim
-    # Tiles the attention kernel executes: the local pass runs every segment's causal triangle in
-    # original order; the permuted pass reruns the query blocks with a non-empty selected list
-    # (their local tiles plus the selected blocks).
-    per_seg = w.segment_len // w.block_size
-    local_pass = w.batch * w.n_q_heads * (w.seq_len // w.segment_len) * per_seg * (per_seg + 1) // 2
-    busy = idx.sel_cnt > 0
-    permuted_pass = int((idx.local_tiles[busy].long() + idx.sel_cnt[busy].long()).sum().item())
-    kernel_tiles = local_pass + permuted_pass
+    # Tile products the attention kernel executes (local pass: every segment's causal triangle in
+    # original order; permuted pass: the selected blocks, packed when most are selected), and the
+    # tiles of (query, key) pairs the method attends (pairs / B²).
+    work = s2o.attention_work(cfg, idx, ws)
+    local_pass, permuted_pass = work.local_pass_tiles, work.permuted_unit_tiles
+    kernel_tiles = work.unit_tiles
+    useful_tiles = stats.pairs / float(w.block_size ** 2)
     exec_flops = kernel_tiles * tile_flops
     peak, hbm_peak, peak_kind = measured_peaks()
 
@@ -348,19 +359,32 @@ def run_s2o(args):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.e2e_steps, dev)
+    gather_ms = None
+    if args.parallel == "heads" and dist is not None:
+        # Assembling the whole O on every GPU, if a caller wants it: one NCCL all-gather of the
+        # shards (not part of the step; the step's output stays sharded).
+        from long_context_sparse_stripe_b200 import shard
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        full_o = shard.gather_output(o, w.n_q_heads, w.n_kv_heads, rank, world, dist)
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        gather_ms = max_over_ranks(dist, g0.elapsed_time(g1), dev)
+        del full_o
 
     line = None
     if rank == 0:
         achieved = exec_flops / (attn_ms_max * 1e-3) / 1e12
         line = {
             "metric": METRIC,
-            "value": whole_job_value(w.dense_causal_flops, world, ms_step),
+            "value": whole_job_value(job_flops, 1, ms_step),
             "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True,
+            "scaling": "strong" if args.parallel == "heads" else "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(args.workload, w, world),
+            "config": workload_config(args.workload, w, world, args.parallel),
             "s2o_ms": ms_step, "index_ms": index_ms, "attention_ms": attn_ms,
             "index_fraction_of_attention": index_ms / attn_ms,
             "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms_step,
@@ -368,17 +392,22 @@ def run_s2o(args):
             "tile_density": stats.executed_tiles * w.block_size ** 2 * 1.0 / stats.causal_pairs,
             "executed_tiles": stats.executed_tiles, "local_tiles": stats.local_tiles,
             "selected_tiles": stats.selected_tiles,
-            "kernel_tiles": {"local_pass": local_pass, "permuted_pass": permuted_pass},
+            "kernel_tiles": {"local_pass": local_pass, "permuted_pass": permuted_pass,
+                             "permuted_loaded": work.permuted_loaded_tiles,
+                             "packed_streams": work.packed,
+                             "executed_over_attended": kernel_tiles / useful_tiles},
             "mse_vs_dense": mse,
             "exec_tflops": achieved,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
                          "traffic": attention_traffic(args.workload),
-                         "kernel": "s2o_attention_kernel<128,128> (local + permuted pass)",
+                         "kernel": "s2o_attention_kernel<128,128> (permuted pass + local pass "
+                                   "with merge)",
                          "peak_source": f"{peak_kind} bf16 (burst)"},
-            "e2e": {"value": whole_job_value(w.dense_causal_flops, world, e2e_ms), "unit": UNIT,
+            "e2e": {"value": whole_job_value(job_flops, 1, e2e_ms), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
+            "o_all_gather_ms": gather_ms,
             "clocks": clocks.summary(),
             "device_status": s2o.STATUS.get(status, status),
         }
@@ -434,11 +463,10 @@ def run_sweep(args):
         torch.cuda.synchronize()
         index_ms, attn_ms = a0.elapsed_time(a1) / reps, b0.elapsed_time(b1) / reps
         stats = s2o.index_stats(cfg, idx, ws)
-        per_seg = w.segment_len // w.block_size
-        local_pass = w.batch * w.n_q_heads * (w.seq_len // w.segment_len) * per_seg * (per_seg + 1) // 2
-        busy = idx.sel_cnt > 0
-        permuted_pass = int((idx.local_tiles[busy].long() + idx.sel_cnt[busy].long()).sum().item())
+        work = s2o.attention_work(cfg, idx, ws)
+        local_pass, permuted_pass = work.local_pass_tiles, work.permuted_unit_tiles
         tile_flops = 4.0 * w.block_size ** 2 * w.head_dim
+        useful = stats.pairs / float(w.block_size ** 2)
         row = {"workload": w.name, "tau": w.tau, "segment_len": w.segment_len,
                "query_perm": w.query_perm, "shared_key_order": w.shared_key_order,
                "int4_centroids": w.int4_centroids,
@@ -446,7 +474,10 @@ def run_sweep(args):
                "pair_sparsity": stats.pair_sparsity,
                "tile_density": stats.executed_tiles * w.block_size ** 2 / stats.causal_pairs,
                "selected_tiles": stats.selected_tiles,
-               "kernel_tiles": {"local_pass": local_pass, "permuted_pass": permuted_pass},
+               "kernel_tiles": {"local_pass": local_pass, "permuted_pass": permuted_pass,
+                                "permuted_loaded": work.permuted_loaded_tiles,
+                                "packed_streams": work.packed,
+                                "executed_over_attended": (local_pass + permuted_pass) / useful},
                "index_ms": index_ms, "attention_ms": attn_ms,
                "index_fraction_of_attention": index_ms / attn_ms,
                "exec_tflops": (local_pass + permuted_pass) * tile_flops / (attn_ms * 1e-3) / 1e12,
@@ -468,6 +499,9 @@ def run_sweep(args):
         return row
 
     configs = [gen.workload("llama-32k")]
+    # Labelled strong-stripe workload (beside the specified ones): the permuted pass at the
+    # selection density the pages report.
+    configs += [gen.workload("llama-128k-strong", tau=t) for t in (0.005, 0.01, 0.02)]
     configs += [gen.workload("llama-128k", tau=t) for t in (0.005, 0.01, 0.02)]
     qwen = gen.workload("qwen-128k")
     configs += [qwen.replace(tau=t) for t in (0.001, 0.005, 0.01, 0.02)]
@@ -479,8 +513,13 @@ def run_sweep(args):
     # Labelled variant: 4-bit key centroids for the block scores (alone and with the above).
     configs += [gen.workload("llama-128k").replace(int4_centroids=1),
                 gen.workload("llama-128k").replace(shared_key_order=1, int4_centroids=1)]
+    if args.sweep_filter:
+        keep = args.sweep_filter.split(",")
+        configs = [w for w in configs if any(f"{w.name}@{w.tau}".startswith(k) for k in keep)]
     for w in configs:
         print(json.dumps({"config": measure(w)}), flush=True)
+    if args.sweep_filter and "stack" not in args.sweep_filter.split(","):
+        return 0
     stack = [measure(gen.layer_workload(l), reps=2, dense=(l % 8 == 7)) for l in range(32)]
     tot_i = sum(r["index_ms"] for r in stack)
     tot_a = sum(r["attention_ms"] for r in stack)
@@ -589,6 +628,9 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="s2o", choices=["s2o", "reference"])
+    ap.add_argument("--parallel", default="replica", choices=["replica", "heads"],
+                    help="N > 1: an independent layer per GPU (replica, weak scaling) or one "
+                         "layer split by KV head (heads, strong scaling)")
     ap.add_argument("--tau", type=float, default=0.01)
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(gen.WORKLOADS),
                     help="bench lines use the default; smaller workloads serve profiling")
@@ -600,6 +642,8 @@ def main():
                     help="profile target only: 'Hq,Hkv' (the first KV groups of the workload)")
     ap.add_argument("--sweep", action="store_true",
                     help="per-configuration report (one JSON line per configuration)")
+    ap.add_argument("--sweep-filter", default="",
+                    help="sweep only: comma-separated 'workload@tau' prefixes (and 'stack')")
     ap.add_argument("--layer", action="store_true",
                     help="end-to-end-shaped decoder layer, S2O vs dense attention (one JSON line)")
     ap.add_argument("--profile-target", action="store_true",

@@ -120,8 +120,9 @@ s2o_status s2o_workspace_views(const s2o_config *cfg, void *ws, size_t ws_bytes,
 
 /* The whole hot path ([S2O, Summary ¶2]): s2o_build_indices into `idx`, then the fused
  * gather-attention over local tiles and selected permuted blocks; O [batch, Hq, N, d] bf16 is
- * written at original positions. With ws_bytes >= s2o_prefill_workspace_size the permuted copy of
- * K and V may be used (see s2o_set_permuted_copy); s2o_workspace_size bytes suffice without it. */
+ * written at original positions. With ws_bytes >= s2o_prefill_workspace_size it runs the merge
+ * path of s2o_attention_prefill_with_indices_ws (packed streams allowed; under shared_key_order
+ * one copy per KV head); s2o_workspace_size bytes suffice without it. */
 s2o_status s2o_attention_prefill(const s2o_config *cfg, const void *q, const void *k,
                                  const void *v, void *o, const s2o_indices *idx, void *ws,
                                  size_t ws_bytes, s2o_stream stream);
@@ -136,41 +137,62 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
                                               const s2o_indices *idx, void *o,
                                               s2o_stream stream);
 
-/* Bytes of scratch with which s2o_attention_prefill and s2o_attention_prefill_with_indices_ws may
- * also make the permuted copy of K and V (see s2o_set_permuted_copy): s2o_workspace_size, a
- * 256-byte flag area, the copy itself (2 · copy_heads · N · d bf16 values with copy_heads =
- * batch · n_q_heads; s2o_attention_prefill with shared_key_order = 1 uses only batch · n_kv_heads
- * copy heads), and the block bitmaps and block-ordered lists of the selected blocks
- * (batch · n_q_heads · nB · (ceil(nB/32) + 1 + nB) int32 values). Written to *bytes. Host only;
- * no device work. */
+/* Bytes of scratch with which s2o_attention_prefill and s2o_attention_prefill_with_indices_ws run
+ * the merge path and may use packed streams (see s2o_set_permuted_copy): s2o_workspace_size, a
+ * 256-byte flag area, one fp32 log2-sum-exp per query row (batch · n_q_heads · N), the permuted
+ * copy of K and V (2 · batch · n_q_heads · N · d bf16 values; one ordering per KV head uses a
+ * quarter of it under GQA of four), the key positions of each key block in position order
+ * (batch · n_q_heads · N int32) with their visible counts per segment (batch · n_q_heads · nSeg ·
+ * nB bytes), and the packed streams' chunk lists (per pair of query blocks 2·nB·B/16 + 3·B/16
+ * int32) and tile counts (16 bytes per pair). Written to *bytes. Host only; no device work. */
 s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes);
 
-/* As s2o_attention_prefill_with_indices, with a workspace: when ws_bytes is at least
- * s2o_prefill_workspace_size and the permuted copy is on, a device-side decision may copy K and V
- * into each query head's key order first, and the permuted pass then loads every selected block
- * as one contiguous tile instead of gathering its rows (and, for dense selections, runs bitmap
- * streams; see s2o_set_permuted_copy). The copy alone leaves the output bit for bit unchanged.
- * With a smaller workspace this is s2o_attention_prefill_with_indices. ws: device, 16-byte
- * aligned, owned by the caller. */
+/* As s2o_attention_prefill_with_indices, with a workspace. With ws_bytes >=
+ * s2o_prefill_workspace_size (the merge path) the permuted pass runs only the selected blocks of
+ * each busy query block and leaves each row's partial result and its log2-sum-exp; the local pass
+ * then computes the dense local window in original order and merges the two (the attention over
+ * the same key set, the fp32 accumulation split in two). When most blocks are selected, a
+ * device-side decision may copy K and V into each query head's key order first, each key block's
+ * rows in position order, and run packed streams (see s2o_set_permuted_copy). With a smaller
+ * workspace this is s2o_attention_prefill_with_indices. ws: device, 16-byte aligned, owned by the
+ * caller. */
 s2o_status s2o_attention_prefill_with_indices_ws(const s2o_config *cfg, const void *q,
                                                  const void *k, const void *v,
                                                  const s2o_indices *idx, void *o, void *ws,
                                                  size_t ws_bytes, s2o_stream stream);
 
-/* The permuted copy ([S2O, Summary ¶2] gathers the scattered rows by index; when most blocks are
- * selected, permuting K and V once in memory makes each selected block contiguous, so it loads
- * as one tile). With it, when the selected blocks are dense, the permuted pass can also run them
- * in block order from bitmaps of the lists, so that two query blocks of one query head and
- * segment load each block they both selected once (bitmap streams; the output is the attention
- * over the same key sets, its fp32 accumulation in another order).
- * mode 0: never; 1 (the default): decided on the device without synchronising, the copy when the
- * selected blocks of the call outnumber twice the blocks the copy writes (copying a block costs
- * about one gather of it), bitmap streams when they also fill at least an eighth of all pairs of
- * query block and key block; 2: always the copy, never bitmap streams (output bit for bit that of
- * the gathers; for tests); 3: always both (for tests). Only calls given a workspace of
- * s2o_prefill_workspace_size bytes use them. Affects calls made after it; not thread-safe against
- * concurrent calls. Other values are treated as 1. */
+/* Packed streams ([S2O, Summary ¶2] fetches the scattered tokens of the selected blocks into
+ * on-chip memory by index): with the permuted copy of K and V, whose key blocks hold their rows in
+ * position order, the keys of block c that a query of segment s may see (position < s·S) are the
+ * block's first rows; the permuted pass loads only those, in chunks of 16 rows packed into full
+ * tiles, and pairs two query blocks that read one copy head and one segment so that a block both
+ * selected is loaded once for both (two consecutive blocks of a query head; two query heads of a
+ * KV head at one block under shared_key_order). Only the accumulation order differs from the
+ * gathered form.
+ * mode 1 (the default): decided on the device without synchronising: the merge path when more
+ * than 1/25 of the query blocks have a selection (below that, rerunning their local tiles costs
+ * less than the merge), packed streams when the selected blocks of the call outnumber twice the
+ * blocks the copy writes (copying a block costs about one gather of it); 0: the merge path with
+ * gathered rows (list order), never packed; 2: always packed; 3: the path without a workspace
+ * even when one is given (0, 2 and 3 are for tests). Only calls given a workspace of
+ * s2o_prefill_workspace_size bytes use modes 0-2. Affects calls made after it; not thread-safe
+ * against concurrent calls. Other values are treated as 1. */
 void s2o_set_permuted_copy(int mode);
+
+/* Work of the attention's last call on `ws` (merge path only), for reports. */
+typedef struct {
+  uint64_t local_pass_tiles;      /* tile products of the local pass: every segment's triangle */
+  uint64_t permuted_unit_tiles;   /* tile products (query tile × key tile) of the permuted pass */
+  uint64_t permuted_loaded_tiles; /* key/value tiles the permuted pass loaded                  */
+  int packed;                     /* 1 when it ran packed streams                              */
+  int merged;                     /* 1 when it ran the merge path                              */
+} s2o_work_counts;
+
+/* Fills *out for the last s2o_attention_prefill / s2o_attention_prefill_with_indices_ws call that
+ * used `ws` (ws_bytes >= s2o_prefill_workspace_size) with the index arrays `idx`. Uses `ws`'s
+ * small scratch; SYNCHRONISES `stream`. */
+s2o_status s2o_attention_work(const s2o_config *cfg, const s2o_indices *idx, void *ws,
+                              size_t ws_bytes, s2o_work_counts *out, s2o_stream stream);
 
 /* In-repo dense causal attention baseline, Eq. (1) of [AB], on the same kernel machinery
  * (contiguous tiles, no index arrays). cfg->segment_len, tau and query_perm are ignored. */

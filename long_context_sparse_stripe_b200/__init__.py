@@ -27,7 +27,7 @@ __all__ = [
     "set_wait_limit_ns", "set_attention_max_ctas", "check_device_status", "exp64_eval", "library_path",
     "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
     "prefill_workspace_size", "alloc_prefill_workspace", "attention_prefill_with_indices_ws",
-    "set_permuted_copy", "layer_workspace_size", "layer_prefill",
+    "set_permuted_copy", "layer_workspace_size", "layer_prefill", "WorkCounts", "attention_work",
 ]
 
 STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
@@ -58,6 +58,12 @@ class _Indices(ctypes.Structure):
 class _Stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in
                 ("local_tiles", "selected_tiles", "pairs", "causal_pairs")]
+
+
+class _Work(ctypes.Structure):
+    _fields_ = [("local_pass_tiles", ctypes.c_uint64), ("permuted_unit_tiles", ctypes.c_uint64),
+                ("permuted_loaded_tiles", ctypes.c_uint64), ("packed", ctypes.c_int),
+                ("merged", ctypes.c_int)]
 
 
 class _View(ctypes.Structure):
@@ -182,6 +188,7 @@ def _load():
             "s2o_dense_causal_prefill": [C, vp, vp, vp, vp, vp],
             "s2o_validate_indices": [C, I, vp, sz, vp],
             "s2o_index_stats": [C, I, vp, sz, ctypes.POINTER(_Stats), vp],
+            "s2o_attention_work": [C, I, vp, sz, ctypes.POINTER(_Work), vp],
             "s2o_check_device_status": [vp],
             "s2o_exp64_eval": [vp, vp, ctypes.c_int, vp],
             "s2o_layer_workspace_size": [C, ctypes.POINTER(_LayerConfig), ctypes.POINTER(sz)],
@@ -399,6 +406,32 @@ def index_stats(cfg: Config, idx: Indices, ws: torch.Tensor | None = None) -> St
     return Stats(s.local_tiles, s.selected_tiles, s.pairs, s.causal_pairs)
 
 
+@dataclasses.dataclass(frozen=True)
+class WorkCounts:
+    """Tile work of the last attention call on a prefill workspace (``s2o_work_counts``)."""
+    local_pass_tiles: int
+    permuted_unit_tiles: int
+    permuted_loaded_tiles: int
+    packed: bool
+    merged: bool
+
+    @property
+    def unit_tiles(self) -> int:
+        return self.local_pass_tiles + self.permuted_unit_tiles
+
+
+def attention_work(cfg: Config, idx: Indices, ws: torch.Tensor) -> WorkCounts:
+    """Tile products and loads of the last attention call that used ``ws`` (synchronises)."""
+    dev = idx.perm_q.device
+    ci = idx._c()
+    w = _Work()
+    _check(_load().s2o_attention_work(ctypes.byref(cfg._c()), ctypes.byref(ci), ws.data_ptr(),
+                                      ws.numel(), ctypes.byref(w), _stream(dev)),
+           "s2o_attention_work")
+    return WorkCounts(w.local_pass_tiles, w.permuted_unit_tiles, w.permuted_loaded_tiles,
+                      bool(w.packed), bool(w.merged))
+
+
 def kernel_launch_count() -> int:
     """Kernel launches made by libs2o in this process so far."""
     return int(_load().s2o_kernel_launch_count())
@@ -440,8 +473,8 @@ def layer_prefill(cfg: Config, shape, weights: dict, x: torch.Tensor,
 
 
 def set_permuted_copy(mode: int) -> None:
-    """Permuted copy of K/V for the permuted pass: 0 never, 1 when it pays (default), 2 always
-    (list order, bit-identical output), 3 always with bitmap streams (block order)."""
+    """Packed streams from the permuted copy of K/V: 0 never (gathered rows), 1 when they pay
+    (default), 2 always; 3 runs the path without a workspace even when one is given."""
     _load().s2o_set_permuted_copy(int(mode))
 
 

@@ -97,9 +97,10 @@ PrefillLayout prefill_layout(const Dims &d) {
   return L;
 }
 
-// Steps 3-4. With a workspace of s2o_prefill_workspace_size bytes (and mode != 3) the merge path
-// runs, with packed streams from the permuted copy when the mode allows them (copy heads: KV heads
-// when per_kv, else query heads); otherwise the path without a workspace.
+// Steps 3-4. With a workspace of s2o_prefill_workspace_size bytes (and mode != 3) the device-side
+// decision picks the path (the merge path, with packed streams from the permuted copy when the mode
+// allows them; copy heads: KV heads when per_kv, else query heads); otherwise the path without a
+// workspace.
 s2o_status attention_ws(const s2o_config &c, const void *q, const void *k, const void *v,
                         const s2o_indices &idx, void *o, void *ws, size_t ws_bytes, bool per_kv,
                         cudaStream_t st) {
@@ -111,20 +112,17 @@ s2o_status attention_ws(const s2o_config &c, const void *q, const void *k, const
     char *b = static_cast<char *>(ws);
     a.merge = true;
     a.lse = reinterpret_cast<float *>(b + L.lse);
-    if (mode != 0) {
-      uint32_t *flag = reinterpret_cast<uint32_t *>(b + L.flag);
-      a.kp = b + L.kp;
-      a.vp = b + L.vp;
-      a.pos_sorted = reinterpret_cast<int32_t *>(b + L.pos);
-      a.vis = reinterpret_cast<uint8_t *>(b + L.vis);
-      a.chunks = reinterpret_cast<uint32_t *>(b + L.chunks);
-      a.pair_meta = reinterpret_cast<int4 *>(b + L.meta);
-      a.chunk_cap = chunk_cap(d);
-      a.copy_flag = flag;
-      a.copy_per_kv = per_kv;
-      const cudaError_t e = launch_permuted_copy(d, a, mode, flag, st);
-      if (e != cudaSuccess) return S2O_ERR_CUDA;
-    }
+    uint32_t *flag = reinterpret_cast<uint32_t *>(b + L.flag);
+    a.kp = b + L.kp;
+    a.vp = b + L.vp;
+    a.pos_sorted = reinterpret_cast<int32_t *>(b + L.pos);
+    a.vis = reinterpret_cast<uint8_t *>(b + L.vis);
+    a.chunks = reinterpret_cast<uint32_t *>(b + L.chunks);
+    a.pair_meta = reinterpret_cast<int4 *>(b + L.meta);
+    a.chunk_cap = chunk_cap(d);
+    a.copy_flag = flag;
+    a.copy_per_kv = per_kv;
+    if (launch_permuted_copy(d, a, mode, flag, st) != cudaSuccess) return S2O_ERR_CUDA;
   }
   return from_cuda(launch_attention(d, a, g_wait_limit_ns.load(), g_attention_max_ctas.load(),
                                     st));
@@ -417,6 +415,57 @@ s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes) {
   if (st != S2O_OK) return st;
   if (!bytes) return S2O_ERR_INVALID_ARGUMENT;
   *bytes = prefill_layout(dims_of(*cfg)).total;
+  return S2O_OK;
+}
+
+s2o_status s2o_attention_work(const s2o_config *cfg, const s2o_indices *idx, void *ws,
+                              size_t ws_bytes, s2o_work_counts *out, s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!ws || !aligned16(ws) || !out || !indices_ok(idx)) return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  const PrefillLayout L = prefill_layout(d);
+  if (ws_bytes < L.total) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  char *b = static_cast<char *>(ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  const long long per_seg = d.S / d.B;
+  out->local_pass_tiles = (uint64_t)(d.bhq() * d.nSeg * per_seg * (per_seg + 1) / 2);
+  // Selected blocks (the gathered form of the permuted pass runs each once per unit).
+  unsigned long long *acc = reinterpret_cast<unsigned long long *>(b + ws_layout(d).flags);
+  if (launch_stats(d, *idx, acc, s) != cudaSuccess) return S2O_ERR_CUDA;
+  unsigned long long h[3] = {0, 0, 0};
+  uint32_t flag = 0;
+  if (cudaMemcpyAsync(h, acc, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(&flag, b + L.flag, sizeof(flag), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return S2O_ERR_CUDA;
+  out->packed = (flag & 1u) ? 1 : 0;
+  out->merged = (flag & 2u) ? 1 : 0;
+  {
+    // Without packed streams: the selected blocks (merge path), or each busy block's local tiles
+    // and selected blocks (the path without the merge).
+    unsigned long long bt[2] = {0, 0};
+    if (cudaMemsetAsync(acc, 0, sizeof(bt), s) != cudaSuccess ||
+        launch_busy_tiles(d, idx->sel_cnt, idx->local_tiles, acc, s) != cudaSuccess ||
+        cudaMemcpyAsync(bt, acc, sizeof(bt), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return S2O_ERR_CUDA;
+    out->permuted_unit_tiles = out->merged ? bt[1] : bt[0];
+    out->permuted_loaded_tiles = out->permuted_unit_tiles;
+  }
+  if (out->packed) {
+    unsigned long long pk[2] = {0, 0};
+    if (cudaMemsetAsync(acc, 0, sizeof(pk), s) != cudaSuccess ||
+        launch_packed_counts(d, reinterpret_cast<const int4 *>(b + L.meta),
+                             reinterpret_cast<const uint32_t *>(b + L.flag), acc, s) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(pk, acc, sizeof(pk), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return S2O_ERR_CUDA;
+    out->permuted_loaded_tiles = pk[0];
+    out->permuted_unit_tiles = pk[1];
+  }
   return S2O_OK;
 }
 

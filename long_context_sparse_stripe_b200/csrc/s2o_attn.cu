@@ -274,7 +274,8 @@ enum Bar {
   kPFull = 22,   // 2: P_x written to TMEM and O_x rescaled (one arrival per softmax warp)
   kOFull = 24,   // 2: the last O_x += P_x·V of a work item finished
   kDrain = 26,
-  kNumBars = 27
+  kOSel = 27,    // 2: an atom of the permuted pass's partial rows landed in the output stage
+  kNumBars = 29
 };
 
 // Unit sets of a launch.
@@ -336,7 +337,10 @@ struct Params {
   int sel_only;
   float *lse_out;        // permuted pass, sel_only: [b, Hq, N] log2 Σ 2^(s·log2e/√d) per row
   const float *lse_in;   // kKindMerge: the same array (−inf where no selected block ran)
-  const uint32_t *copy_flag;  // bit 0: the permuted copy is in use (packed streams)
+  // Device-side decision word (see k_copy_decide): bit 0 packed streams from the permuted copy,
+  // bit 1 the merge path. A launch given it runs only when (word & run_mask) == run_value.
+  const uint32_t *copy_flag;
+  uint32_t run_mask, run_value;
   int copy_per_kv;            // copy rows per KV head (else per query head)
   // Packed streams (kKindPacked): per pair of units, chunk words at chunks + pair·chunk_cap (see
   // k_pack_pairs) and the tile counts {both, only unit 0, only unit 1, -} in pair_meta; pairs
@@ -718,6 +722,19 @@ __device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&w)[8]) 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Named barrier that also returns whether any participating thread passed `v`.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %3, 0;\n\t"
+      "bar.red.or.pred p, %1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(threads), "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
@@ -812,8 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool PACKED = KIND == kKindPacked;
   constexpr bool MERGE = KIND == kKindMerge;
   constexpr int CPT = BN / kChunkRows;  // chunks per packed tile
-  const uint32_t flagv = p.copy_flag != nullptr ? __ldg(p.copy_flag) : 0u;
-  if (PERM && p.copy_flag != nullptr && ((flagv & 1u) != 0u) != PACKED) return;
+  if (p.copy_flag != nullptr && (__ldg(p.copy_flag) & p.run_mask) != p.run_value) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -831,6 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kSFull + x), 1);
       mbar_init(bar(kPFull + x), 4);  // one arrival per softmax warp
       mbar_init(bar(kOFull + x), 1);
+      mbar_init(bar(kOSel + x), 1);
     }
     for (int i = 0; i < L::KST; ++i) {
       mbar_init(bar(kKFull + i), 1);
@@ -1189,10 +1206,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const unsigned full = 0xffffffffu;
     const float sl2 = p.scale_log2;
     long long sn = 0, on = 0;  // S_x tiles and work items consumed
+    long long osel_n = 0;      // partial-row atoms loaded into this group's output stage (MERGE)
     for_each_window([&](int n_list) {
     for (int wi = 0; ok && wi < (n_list + 1) / 2; ++wi) {
       const Pair P = decode_pair<BN, KIND>(p, list, n_list, wi);
-      if (!(x ? P.valid1 : P.valid0)) continue;
+      if (x == 1 ? !P.valid1 : (PACKED && !P.valid0)) continue;
       const Unit u = x ? P.u1 : P.u0;
       const int seg0 = u.seg0;
       // Original position of this row's query (padding rows: the segment's last position).
@@ -1358,13 +1376,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.lse_out[(size_t)u.qh * p.N + i_orig] = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
         store_row = store_row && l_run > 0.f;
       }
-      // The whole row of O from TMEM (one wait), then 32-byte stores (full sectors).
-      uint32_t o[D];
-#pragma unroll
-      for (int c0 = 0; c0 < D / 32; ++c0)
-        tmem_ld32(o_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
-#pragma unroll
-      for (int c0 = 0; c0 < D / 32; ++c0) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
       if (!PERM) {
         // Contiguous rows: each 64-column atom is staged in shared memory (128-byte swizzle) and
         // written with one TMA tile store; the group's first thread issues the stores and, before
@@ -1372,32 +1383,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool leader = quad == 0 && lane == 0;
         const uint32_t ost = sbase + L::OFF_OST + (uint32_t)x * L::ATOM_Q;
         unsigned char *ostp = smem + L::OFF_OST + x * L::ATOM_Q + row * 128;
+        // MERGE: when a row of the tile has a partial result, each atom of the tile's rows of O
+        // (the permuted pass's partial rows o_sel, at these original positions) is first loaded
+        // into the stage by TMA, and every thread merges its row in place.
+        const bool merge_tile = MERGE && named_bar_or(2 + x, 128, ss != 0.f);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) {
-          // MERGE: this atom of o_sel, read before the stage wait (its row is this thread's).
-          uint4 sel[8];
-          if (MERGE) {
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-              sel[ch] = ss != 0.f ? __ldg(reinterpret_cast<const uint4 *>(orow + a * 64 + ch * 8))
-                                  : make_uint4(0, 0, 0, 0);
-          }
+          // This atom's 64 columns of O from TMEM (one atom at a time keeps the live set small).
+          uint32_t o[64];
+          tmem_ld32(o_addr + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_ld32(o_addr + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[32]));
           if (leader) bulk_wait_read();
           named_bar_sync(2 + x, 128);
+          if (merge_tile) {
+            if (leader) {
+              mbar_expect_tx(bar(kOSel + x), (uint32_t)BN * 128u);  // BN rows of the atom
+              tma_load_tile(ost, &tm_o_tile, a * 64, (int)(u.qh * p.N) + u.b * BN, bar(kOSel + x));
+            }
+            mbar_wait(bar(kOSel + x), (uint32_t)(osel_n & 1), lim);
+            ++osel_n;
+          }
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
-            const int c = a * 64 + ch * 8;
+            const int c = ch * 8;
             uint4 v;
             if (MERGE) {
+              const uint4 sel = merge_tile ? *reinterpret_cast<const uint4 *>(ostp + ((ch ^ (row & 7)) * 16))
+                                           : make_uint4(0, 0, 0, 0);
               auto mix = [&](int cc, uint32_t w2) {
                 const float lo = __uint_as_float(w2 << 16), hi = __uint_as_float(w2 & 0xffff0000u);
                 return pack_bf16(fmaf(__uint_as_float(o[cc]), so, lo * ss),
                                  fmaf(__uint_as_float(o[cc + 1]), so, hi * ss));
               };
-              v.x = mix(c + 0, sel[ch].x);
-              v.y = mix(c + 2, sel[ch].y);
-              v.z = mix(c + 4, sel[ch].z);
-              v.w = mix(c + 6, sel[ch].w);
+              v.x = mix(c + 0, sel.x);
+              v.y = mix(c + 2, sel.y);
+              v.z = mix(c + 4, sel.z);
+              v.w = mix(c + 6, sel.w);
             } else {
               v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
               v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
@@ -1414,6 +1437,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if (store_row) {
+        // The whole row of O from TMEM (one wait), then 32-byte stores (full sectors).
+        uint32_t o[D];
+#pragma unroll
+        for (int c0 = 0; c0 < D / 32; ++c0)
+          tmem_ld32(o_addr + c0 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
+#pragma unroll
+        for (int c0 = 0; c0 < D / 32; ++c0) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t w[8];
@@ -1432,8 +1462,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
     }
     });
-    // The output stores of this group's stage complete before the CTA exits.
-    if (quad == 0 && lane == 0) bulk_wait_all();
+    // The output stores of this group's stage complete before the CTA exits (and the last
+    // partial-row load into it, should a wait for it have given up).
+    if (quad == 0 && lane == 0) {
+      bulk_wait_all();
+      if (MERGE && osel_n > 0) mbar_wait(bar(kOSel + x), (uint32_t)((osel_n - 1) & 1), kDrainNs);
+    }
   }
 
   __syncthreads();
@@ -1463,26 +1497,45 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // ------------------------------------------------------------------ permuted copy of K and V
 
-// Whether the permuted pass runs packed streams from the permuted copy (bit 0 of *flag): always
-// (mode 2), or (mode 1) when the selected blocks of all query blocks outnumber twice the blocks
-// the copy writes (copying a block costs about one gather of it, and each selected block then
-// loads as contiguous chunks). One CTA.
+// The path of a call with a workspace, decided on the device without synchronising (one CTA):
+//   bit 1 (merge path): the permuted pass runs only the selected blocks and the local pass merges
+//     its partial rows; otherwise the local pass runs alone and the permuted pass reruns each busy
+//     query block's local tiles. Rerunning costs about S/B tiles per busy block, the merge a
+//     fixed few per cent of the local pass: merge when more than 1/25 of the query blocks have a
+//     selection (mode 1), always (modes 0 and 2), never (mode 3 is decided on the host).
+//   bit 0 (packed streams, with bit 1): when the selected blocks outnumber twice the blocks the
+//     permuted copy writes (copying a block costs about one gather of it; mode 1), always
+//     (mode 2), never (mode 0).
 __global__ void __launch_bounds__(1024)
     k_copy_decide(const int32_t *__restrict__ sel_cnt, long long n_units, int nB, int mode,
                   long long copy_blocks, uint32_t *__restrict__ flag) {
-  __shared__ unsigned long long part[32];
-  unsigned long long sum = 0;
-  for (long long i = threadIdx.x; i < n_units; i += blockDim.x)
-    sum += (unsigned long long)min(max(__ldg(sel_cnt + i), 0), nB);
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (threadIdx.x % 32 == 0) part[threadIdx.x / 32] = sum;
+  __shared__ unsigned long long part[32], part_busy[32];
+  unsigned long long sum = 0, busy = 0;
+  for (long long i = threadIdx.x; i < n_units; i += blockDim.x) {
+    const int c = min(max(__ldg(sel_cnt + i), 0), nB);
+    sum += (unsigned long long)c;
+    busy += c > 0 ? 1ull : 0ull;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    busy += __shfl_xor_sync(0xffffffffu, busy, o);
+  }
+  if (threadIdx.x % 32 == 0) {
+    part[threadIdx.x / 32] = sum;
+    part_busy[threadIdx.x / 32] = busy;
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
-    unsigned long long total = 0;
-    for (int w = 0; w < (int)(blockDim.x / 32); ++w) total += part[w];
-    const bool copy =
+    unsigned long long total = 0, total_busy = 0;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
+      total += part[w];
+      total_busy += part_busy[w];
+    }
+    const bool packed =
         mode == 2 || (mode == 1 && total > 2ull * (unsigned long long)copy_blocks);
-    *flag = copy ? 1u : 0u;
+    const bool merge = mode == 0 || packed ||
+                       (mode == 1 && 25ull * total_busy > (unsigned long long)n_units);
+    *flag = (packed ? 1u : 0u) | (merge ? 2u : 0u);
   }
 }
 
@@ -1682,8 +1735,56 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) pair_meta[w] = make_int4(T[0], T[1], T[2], 0);
 }
 
-// Rows without a partial result from the permuted pass: lse = −inf.
-__global__ void __launch_bounds__(256) k_fill_neg_inf(float *__restrict__ p, long long n) {
+// Tile counts of the packed streams of the last call (bit 0 only): acc[0] += Σ tiles loaded
+// (shared + unit 0 + unit 1), acc[1] += Σ tile products (2·shared + unit 0 + unit 1).
+__global__ void __launch_bounds__(256)
+    k_packed_counts(const int4 *__restrict__ pair_meta, long long n_pairs,
+                    const uint32_t *__restrict__ flag, unsigned long long *__restrict__ acc) {
+  if ((__ldg(flag) & 1u) == 0u) return;
+  unsigned long long loaded = 0, products = 0;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_pairs;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int4 m = __ldg(pair_meta + i);
+    loaded += (unsigned long long)(m.x + m.y + m.z);
+    products += (unsigned long long)(2 * m.x + m.y + m.z);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    loaded += __shfl_xor_sync(0xffffffffu, loaded, o);
+    products += __shfl_xor_sync(0xffffffffu, products, o);
+  }
+  if (threadIdx.x % 32 == 0) {
+    atomicAdd(acc, loaded);
+    atomicAdd(acc + 1, products);
+  }
+}
+
+// Work of the permuted pass without packed streams: acc[0] += Σ over busy query blocks of
+// (local tiles + selected blocks) (the path without the merge reruns the local tiles),
+// acc[1] += Σ selected blocks (the merge path with gathered blocks).
+__global__ void __launch_bounds__(256)
+    k_busy_tiles(const int32_t *__restrict__ sel_cnt, const int32_t *__restrict__ local_tiles,
+                 long long n_units, int nB, int per_seg, unsigned long long *__restrict__ acc) {
+  unsigned long long rerun = 0, sel = 0;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_units;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c = min(max(__ldg(sel_cnt + i), 0), nB);
+    if (c > 0) rerun += (unsigned long long)(c + min(max(__ldg(local_tiles + i), 1), per_seg));
+    sel += (unsigned long long)c;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    rerun += __shfl_xor_sync(0xffffffffu, rerun, o);
+    sel += __shfl_xor_sync(0xffffffffu, sel, o);
+  }
+  if (threadIdx.x % 32 == 0) {
+    atomicAdd(acc, rerun);
+    atomicAdd(acc + 1, sel);
+  }
+}
+
+// Rows without a partial result from the permuted pass: lse = −inf (merge path only).
+__global__ void __launch_bounds__(256)
+    k_fill_neg_inf(float *__restrict__ p, long long n, const uint32_t *__restrict__ flag) {
+  if (flag != nullptr && (__ldg(flag) & 2u) == 0u) return;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x)
     p[i] = -INFINITY;
@@ -1773,7 +1874,6 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   p.sel_only = 0;
   p.lse_out = nullptr;
   p.lse_in = nullptr;
-  p.copy_flag = a.merge ? a.copy_flag : nullptr;
   p.copy_per_kv = a.copy_per_kv ? 1 : 0;
   p.chunks = a.chunks;
   p.pair_meta = a.pair_meta;
@@ -1809,33 +1909,49 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
     note_launch();
     return cudaGetLastError();
   };
+  p.copy_flag = nullptr;
+  p.run_mask = p.run_value = 0u;
   if (a.dense) return launch(kDense, 0, kKindContig);
-  if (!a.merge || a.lse == nullptr) {
-    // Without a workspace: every row first gets the dense local window of its segment, computed
-    // in original order (causal triangles, masks on diagonal tiles only); then the query blocks
-    // whose selected list is not empty are recomputed in full (local tiles and selected blocks,
-    // permuted order) and overwrite their rows. Each row's result is the attention over its key
-    // set either way.
-    if ((e = launch(kLocal, 0, kKindContig)) != cudaSuccess) return e;
+  // The path without a workspace: every row first gets the dense local window of its segment,
+  // computed in original order (causal triangles, masks on diagonal tiles only); then the query
+  // blocks whose selected list is not empty are recomputed in full (local tiles and selected
+  // blocks, permuted order) and overwrite their rows. Each row's result is the attention over its
+  // key set either way.
+  auto legacy = [&]() -> cudaError_t {
+    cudaError_t r = launch(kLocal, 0, kKindContig);
+    if (r != cudaSuccess) return r;
     return launch(kPermuted, 1, kKindList);
-  }
-  // Merge path: the permuted pass runs only the selected blocks and leaves each row's partial
-  // result and its log2-sum-exp (−inf for rows it does not reach); the local pass then computes
-  // the local window in original order and merges the two. The permuted pass is launched in both
-  // forms when the device-side decision may pick packed streams; one returns at once.
+  };
+  if (!a.merge || a.lse == nullptr) return legacy();
+  // With a workspace every path is launched and the device-side decision word lets one run (the
+  // others return at once). Merge path: the permuted pass runs only the selected blocks (gathered,
+  // or packed streams) and leaves each row's partial result and its log2-sum-exp (−inf for rows
+  // it does not reach); the local pass then computes the local window in original order and
+  // merges the two.
+  p.copy_flag = a.copy_flag;
   const long long n_rows = d.bhq() * d.N;
   const unsigned fill_grid = (unsigned)std::min<long long>((n_rows + 255) / 256, 148ll * 16);
-  k_fill_neg_inf<<<fill_grid, 256, 0, st>>>(a.lse, n_rows);
+  k_fill_neg_inf<<<fill_grid, 256, 0, st>>>(a.lse, n_rows, a.copy_flag);
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.sel_only = 1;
   p.lse_out = a.lse;
+  p.run_mask = 3u;  // merge path with gathered blocks
+  p.run_value = 2u;
   if ((e = launch(kPermuted, 1, kKindList)) != cudaSuccess) return e;
-  if (packed && (e = launch(kPermuted, 1, kKindPacked)) != cudaSuccess) return e;
+  if (packed) {
+    p.run_mask = p.run_value = 1u;  // packed streams
+    if ((e = launch(kPermuted, 1, kKindPacked)) != cudaSuccess) return e;
+  }
   p.sel_only = 0;
   p.lse_out = nullptr;
   p.lse_in = a.lse;
-  return launch(kLocal, 0, kKindMerge);
+  p.run_mask = p.run_value = 2u;  // the merging local pass
+  if ((e = launch(kLocal, 0, kKindMerge)) != cudaSuccess) return e;
+  p.lse_in = nullptr;
+  p.run_mask = 2u;  // the path without the merge
+  p.run_value = 0u;
+  return a.copy_flag != nullptr ? legacy() : cudaSuccess;
 }
 
 }  // namespace
@@ -1884,6 +2000,24 @@ cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uin
                                                 a.pair_meta, a.chunk_cap, n_units, d.nB, d.S,
                                                 d.nSeg, d.Hq, d.Hkv, d.G, a.copy_per_kv ? 1 : 0,
                                                 a.copy_per_kv ? 1 : 0, flag);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_packed_counts(const Dims &d, const int4 *pair_meta, const uint32_t *flag,
+                                 unsigned long long *acc, cudaStream_t st) {
+  const long long n_pairs = (d.bhq() * d.nB + 1) / 2;
+  const unsigned grid = (unsigned)std::min<long long>((n_pairs + 255) / 256, 148ll * 4);
+  k_packed_counts<<<grid, 256, 0, st>>>(pair_meta, n_pairs, flag, acc);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_busy_tiles(const Dims &d, const int32_t *sel_cnt, const int32_t *local_tiles,
+                              unsigned long long *acc, cudaStream_t st) {
+  const long long n_units = d.bhq() * d.nB;
+  const unsigned grid = (unsigned)std::min<long long>((n_units + 255) / 256, 148ll * 4);
+  k_busy_tiles<<<grid, 256, 0, st>>>(sel_cnt, local_tiles, n_units, d.nB, d.S / d.B, acc);
   note_launch();
   return cudaGetLastError();
 }

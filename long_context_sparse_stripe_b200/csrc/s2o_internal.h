@@ -63,13 +63,21 @@ struct AttnArgs {
 };
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
                              int max_ctas, cudaStream_t st);
-// The permuted copy for packed streams: a decision kernel sets bit 0 of *flag when `mode` is 2, or
-// when it is 1 and the selected blocks outnumber twice the copied blocks; then (each doing nothing
-// when the bit is clear) the blocks of perm_k are put in position order (a.pos_sorted, a.vis), K
-// and V are copied in that order (a.kp, a.vp), and each pair of units gets its chunk list
-// (a.chunks, a.pair_meta).
+// The path of a call with a workspace: a decision kernel writes *flag (bit 1 the merge path, bit 0
+// packed streams from the permuted copy; see k_copy_decide for the rules per mode); then (each
+// doing nothing when bit 0 is clear) the blocks of perm_k are put in position order (a.pos_sorted,
+// a.vis), K and V are copied in that order (a.kp, a.vp), and each pair of units gets its chunk
+// list (a.chunks, a.pair_meta).
 cudaError_t launch_permuted_copy(const Dims &d, const AttnArgs &a, int mode, uint32_t *flag,
                                  cudaStream_t st);
+// acc[0] += tiles the packed streams of the last call loaded, acc[1] += their tile products
+// (nothing when *flag's bit 0 is clear).
+cudaError_t launch_packed_counts(const Dims &d, const int4 *pair_meta, const uint32_t *flag,
+                                 unsigned long long *acc, cudaStream_t st);
+// acc[0] += Σ over query blocks with a selection of (local tiles + selected blocks), acc[1] += Σ
+// selected blocks.
+cudaError_t launch_busy_tiles(const Dims &d, const int32_t *sel_cnt, const int32_t *local_tiles,
+                              unsigned long long *acc, cudaStream_t st);
 
 // Decoder layer (s2o_layer.cu): byte offsets of its buffers in the layer workspace (the attention's
 // own workspace starts at attn_ws), and the launches before and after the attention. A false

@@ -183,3 +183,17 @@ def test_layer_prefill_rejects_null_weights_before_launch():
     st = lib.s2o_layer_prefill(ctypes.byref(LLAMA_128K._c()), ctypes.byref(lc), ctypes.byref(w),
                                0x10000, 0x20000, 1024, None)
     assert st == 3  # workspace too small
+
+
+def test_attention_work_rejects_bad_arguments_before_device_work():
+    cfg = LLAMA_128K
+    lib = s2o._load()
+    idx = s2o._Indices(0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+    out = s2o._Work()
+    small = s2o.prefill_workspace_size(cfg) - 1
+    assert lib.s2o_attention_work(ctypes.byref(cfg._c()), ctypes.byref(idx), 0x10000, small,
+                                  ctypes.byref(out), None) == 3
+    assert lib.s2o_attention_work(ctypes.byref(cfg._c()), ctypes.byref(idx), 0x10000, small + 1,
+                                  None, None) == 1
+    assert lib.s2o_attention_work(ctypes.byref(cfg._c()), None, 0x10000, small + 1,
+                                  ctypes.byref(out), None) == 1

@@ -355,7 +355,7 @@ def test_merge_and_packed_paths_match_oracle(w):
     cfg = s2o.Config.of(w)
     idx = oracle_indices_on_device(ref)
     ws = s2o.alloc_prefill_workspace(cfg)
-    for mode, flag in ((0, None), (2, 1), (3, None)):
+    for mode, flag in ((0, 2), (2, 3), (3, None)):
         o = _with_mode(mode, lambda: s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx,
                                                                            ws))
         assert s2o.check_device_status() == 0, mode
@@ -365,10 +365,10 @@ def test_merge_and_packed_paths_match_oracle(w):
 
 
 def test_permuted_copy_decision():
-    """Mode 1 copies only when the selected blocks outnumber twice the copied blocks: with every
-    block selected (τ = 0) it does, with none (τ > 1) it does not; with no selection the merge path
-    gives the bits of the path without a workspace."""
-    for w, expect in ((W_A.replace(tau=0.0), 1), (W_A.replace(tau=1.5), 0)):
+    """Mode 1 merges and packs when the selected blocks outnumber twice the copied blocks: with
+    every block selected (τ = 0) it does both; with none (τ > 1) neither, and the call then runs
+    the kernels of the path without a workspace (same bits)."""
+    for w, expect in ((W_A.replace(tau=0.0), 3), (W_A.replace(tau=1.5), 0)):
         q, k, v = to_dev(*inputs(w))
         cfg = s2o.Config.of(w)
         idx = s2o.build_indices(cfg, q, k)
@@ -427,3 +427,28 @@ def test_packed_path_independent_of_grid_and_windows():
             assert torch.equal(o, base), f"grid of {n}"
     finally:
         s2o.set_attention_max_ctas(0)
+
+
+def test_attention_work_counts():
+    """The work report: gathered selected blocks run once per unit (mode 0); packed streams run
+    about the attended pairs, and load each tile once even when both units of a pair use it."""
+    w = W_S1
+    q, k, v = to_dev(*inputs(w))
+    cfg = s2o.Config.of(w)
+    idx = s2o.build_indices(cfg, q, k)
+    ws = s2o.alloc_prefill_workspace(cfg)
+    st = s2o.index_stats(cfg, idx)
+    per_seg = w.segment_len // w.block_size
+    local = w.n_q_heads * (w.seq_len // w.segment_len) * per_seg * (per_seg + 1) // 2
+    _with_mode(0, lambda: s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, ws))
+    gathered = s2o.attention_work(cfg, idx, ws)
+    assert gathered.merged and not gathered.packed
+    assert gathered.local_pass_tiles == local
+    assert gathered.permuted_unit_tiles == gathered.permuted_loaded_tiles == st.selected_tiles
+    _with_mode(2, lambda: s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, ws))
+    packed = s2o.attention_work(cfg, idx, ws)
+    assert packed.packed and packed.merged and packed.local_pass_tiles == local
+    attended = st.pairs / w.block_size ** 2
+    assert packed.unit_tiles < 1.3 * attended
+    assert packed.permuted_unit_tiles < gathered.permuted_unit_tiles
+    assert packed.permuted_loaded_tiles < packed.permuted_unit_tiles
