@@ -42,8 +42,8 @@ WORKLOAD = "llama-128k"
 # that kernel (dram__bytes_read.sum + dram__bytes_write.sum on llama-32k, scaled by the tile count
 # to llama-128k). Valid only for the kernel source it was taken on: reported as null once
 # s2o_attn.cu changes.
-ATTN_TRAFFIC = {"src_sha256_16": "23494639118c092a", "workload": "llama-128k",
-                "bytes_per_launch": (405.164800e6 + 235.952384e6) * 4}
+ATTN_TRAFFIC = {"src_sha256_16": "75573d0d5e71199f", "workload": "llama-128k",
+                "bytes_per_launch": (405.674240e6 + 235.413504e6) * 4}
 
 
 def attention_traffic(workload):
@@ -597,7 +597,11 @@ def run_layer(args):
 
 def run_profile_target(args):
     """A short fixed sequence for profiler captures (not a bench line): one index build, then
-    `--steps` attention calls (each a local pass and a permuted pass) and one dense-baseline call."""
+    `--steps` attention calls and one dense-baseline call. Without `--ws-mode` each call is the
+    path without a workspace (the local pass, then the permuted pass); with it, a call with a
+    prefill workspace in that permuted-copy mode launches, in order, the merge path's permuted
+    pass (gathered), its packed form, the merging local pass, the plain local pass and the plain
+    permuted pass, of which the device-side decision lets one path run."""
     import long_context_sparse_stripe_b200 as s2o
 
     torch.cuda.set_device(0)
@@ -613,8 +617,15 @@ def run_profile_target(args):
     cfg = s2o.Config.of(w)
     idx = s2o.build_indices(cfg, q, k)
     o = torch.empty_like(q)
+    ws = None
+    if args.ws_mode >= 0:
+        s2o.set_permuted_copy(args.ws_mode)
+        ws = s2o.alloc_prefill_workspace(cfg)
     for _ in range(args.steps):
-        s2o.attention_prefill_with_indices(cfg, q, k, v, idx, out=o)
+        if ws is None:
+            s2o.attention_prefill_with_indices(cfg, q, k, v, idx, out=o)
+        else:
+            s2o.attention_prefill_with_indices_ws(cfg, q, k, v, idx, ws, out=o)
     s2o.dense_causal_prefill(cfg, q, k, v, out=o)
     torch.cuda.synchronize()
     if s2o.check_device_status() != 0:
@@ -638,6 +649,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-rows", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ws-mode", type=int, default=-1,
+                    help="profile target only: call with a prefill workspace in this mode")
     ap.add_argument("--heads", default="",
                     help="profile target only: 'Hq,Hkv' (the first KV groups of the workload)")
     ap.add_argument("--sweep", action="store_true",
