@@ -13,6 +13,10 @@ Parity status per function (what pins it to something other than itself lives in
   causal attention at τ > 1, and by permutation invariance.
 * ``dense_causal`` — pinned by torch's causal scaled-dot-product attention.
 * ``exp64`` — pinned by libm exp (≤ 2 ulp) and the constants by a 60-digit derivation.
+* ``online_stop`` (the measured-share early stop, a labelled variant) — pinned by a hand-worked
+  case (``tests/golden/online_stop_case.md``), by τ = 0 (nothing stops), by a brute-force
+  restatement from whole-row softmax probabilities on small random inputs, and by the rule's
+  consequences (stopping never adds a block; lists stay prefixes).
 * ``layer.layer`` (the decoder layer around the attention, ``oracle/layer.py``) — pinned in
   ``tests/test_layer_oracle_pins.py`` (bf16 rounding against torch, closed-form norms, rotary
   invariants, the frequency scaling's regimes, the silu identity, zero projections = identity).
@@ -75,6 +79,9 @@ def _load(path: str | None = None):
             lib.oracle_dense_causal.argtypes = [ctypes.POINTER(Config), vp, vp, vp, vp, i64, vp,
                                                 i32]
             lib.oracle_dense_causal.restype = i32
+            lib.oracle_online_stop.argtypes = [ctypes.POINTER(Config), vp, vp, vp, vp, vp, vp,
+                                               vp, vp, i32]
+            lib.oracle_online_stop.restype = i32
             lib.oracle_pair_count.argtypes = [ctypes.POINTER(Config), vp, vp, vp, vp]
             lib.oracle_pair_count.restype = i64
             lib.oracle_score_scale.argtypes = [ctypes.c_int]
@@ -190,6 +197,32 @@ def dense_causal(cfg: Config, q, k, v, rows: np.ndarray | None = None,
                                  n_rows, _ptr(out), n_threads or threads())
     if st != 0:
         raise ValueError(f"oracle_dense_causal: status {st}")
+    return out
+
+
+def online_stop(cfg: Config, q, k, idx: dict, n_threads: int | None = None):
+    """The measured-share early stop (labelled variant): ``(stop_cnt [b, Hq, nB] int32,
+    max_share [b, Hq, nB, nB] float64)`` — the listed blocks each query block keeps, and for every
+    listed block the largest share over the block's rows (zero past the list)."""
+    lib = _load()
+    q, k = _bits(q), _bits(k)
+    B, Hq, N = cfg.batch, cfg.n_q_heads, cfg.seq_len
+    nB = N // cfg.block_size
+    stop = np.empty((B, Hq, nB), np.int32)
+    share = np.zeros((B, Hq, nB, nB), np.float64)
+    arrs = [np.ascontiguousarray(idx[n], dtype=np.int32)
+            for n in ("perm_q", "perm_k", "sel_cnt", "sel_blk")]
+    st = lib.oracle_online_stop(ctypes.byref(cfg), _ptr(q), _ptr(k), *map(_ptr, arrs),
+                                _ptr(stop), _ptr(share), n_threads or threads())
+    if st != 0:
+        raise ValueError(f"oracle_online_stop: status {st}")
+    return stop, share
+
+
+def with_counts(idx: dict, counts) -> dict:
+    """The index arrays with sel_cnt replaced (the lists cut to the given lengths)."""
+    out = dict(idx)
+    out["sel_cnt"] = np.ascontiguousarray(counts, dtype=np.int32)
     return out
 
 

@@ -475,6 +475,101 @@ int oracle_attention(const oracle_config *cfg, const uint16_t *q, const uint16_t
   return ORACLE_OK;
 }
 
+/* ------------------------------------------------------------ online early stop (variant) */
+
+/* Measured-share early stop (a labelled variant; the definition's D13): for query block b (segment
+ * s) with listed blocks c_0..c_{cnt-1} in list order, row i's share of block k is
+ *   share_{i,k} = Σ_{j ∈ V_k} e^{z_ij} / Σ_{j ∈ L_i ∪ V_0 ∪ … ∪ V_k} e^{z_ij},
+ * L_i = the local keys [sS, i], V_k = the keys of block c_k before sS, z_ij = q_i·k_j/√d. The
+ * block's list stops after the first k whose largest share over the block's rows is below τ (block
+ * k itself is kept). Writes stop_cnt[qb] (the listed blocks kept) and max_share[qb·nB + k] for
+ * every listed k (binary64; libm exp; each row's exponents taken against the row's largest z over
+ * its whole list, which leaves every ratio unchanged). */
+int oracle_online_stop(const oracle_config *cfg, const uint16_t *q, const uint16_t *k,
+                       const int32_t *perm_q, const int32_t *perm_k, const int32_t *sel_cnt,
+                       const int32_t *sel_blk, int32_t *stop_cnt, double *max_share,
+                       int n_threads) {
+  if (!check_config(cfg)) return ORACLE_ERR_UNSUPPORTED;
+  const int N = cfg->seq_len, d = cfg->head_dim, S = cfg->segment_len, B = cfg->block_size;
+  const int nB = N / B, G = cfg->n_q_heads / cfg->n_kv_heads;
+  const int64_t n_qblocks = (int64_t)cfg->batch * cfg->n_q_heads * nB;
+  const double inv_sqrt_d = 1.0 / sqrt((double)d);
+  const double tau = (double)cfg->tau;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+  {
+    double *zl = malloc((size_t)S * sizeof(double));
+    double *zb = malloc((size_t)nB * B * sizeof(double));
+    double *ek = malloc((size_t)nB * sizeof(double));
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t qb = 0; qb < n_qblocks; ++qb) {
+      const size_t qh = (size_t)(qb / nB);
+      const int b = (int)(qb % nB);
+      const int s0 = (b * B / S) * S;
+      const size_t kh = (qh / cfg->n_q_heads) * cfg->n_kv_heads + (qh % cfg->n_q_heads) / G;
+      const uint16_t *K = k + kh * N * d;
+      const int32_t *pk = perm_k + qh * N;
+      const int32_t *list = sel_blk + (size_t)qb * nB;
+      const int cnt = sel_cnt[qb];
+      double *ms = max_share + (size_t)qb * nB;
+      for (int x = 0; x < cnt; ++x) ms[x] = 0.0;
+      for (int e = 0; e < B; ++e) {
+        const int i = perm_q[qh * N + (size_t)b * B + e];
+        const uint16_t *qi = q + (qh * N + i) * d;
+        double m = -INFINITY;
+        int nl = 0;
+        for (int j = s0; j <= i; ++j) {
+          const uint16_t *kj = K + (size_t)j * d;
+          double acc = 0.0;
+          for (int t = 0; t < d; ++t) acc += (double)bf16_to_f32(qi[t]) * (double)bf16_to_f32(kj[t]);
+          zl[nl] = acc * inv_sqrt_d;
+          if (zl[nl] > m) m = zl[nl];
+          ++nl;
+        }
+        for (int x = 0; x < cnt; ++x)
+          for (int y = 0; y < B; ++y) {
+            const int j = pk[list[x] * B + y];
+            double zz = -INFINITY;
+            if (j < s0) {
+              const uint16_t *kj = K + (size_t)j * d;
+              double acc = 0.0;
+              for (int t = 0; t < d; ++t)
+                acc += (double)bf16_to_f32(qi[t]) * (double)bf16_to_f32(kj[t]);
+              zz = acc * inv_sqrt_d;
+              if (zz > m) m = zz;
+            }
+            zb[(size_t)x * B + y] = zz;
+          }
+        double den = 0.0;
+        for (int a = 0; a < nl; ++a) den += exp(zl[a] - m);
+        for (int x = 0; x < cnt; ++x) {
+          double e_k = 0.0;
+          for (int y = 0; y < B; ++y) {
+            const double zz = zb[(size_t)x * B + y];
+            if (zz != -INFINITY) e_k += exp(zz - m);
+          }
+          ek[x] = e_k;
+        }
+        for (int x = 0; x < cnt; ++x) {
+          den += ek[x];
+          const double share = ek[x] / den;
+          if (share > ms[x]) ms[x] = share;
+        }
+      }
+      int kept = cnt;
+      for (int x = 0; x < cnt; ++x)
+        if (ms[x] < tau) {
+          kept = x + 1;
+          break;
+        }
+      stop_cnt[qb] = kept;
+    }
+    free(zl);
+    free(zb);
+    free(ek);
+  }
+  return ORACLE_OK;
+}
+
 /* Dense causal attention, Eq. (1) written out in binary64, for listed rows (NULL = all). */
 int oracle_dense_causal(const oracle_config *cfg, const uint16_t *q, const uint16_t *k,
                         const uint16_t *v, const int64_t *rows, int64_t n_rows, double *out,

@@ -32,6 +32,15 @@ MUTATIONS = {
     "dropped-visibility-weight": (
         "w[c] = ns[c] > 0 ? (double)ns[c] * oracle_exp64((double)rb[c] - (double)M) : 0.0;",
         "w[c] = ns[c] > 0 ? oracle_exp64((double)rb[c] - (double)M) : 0.0;"),
+    # Online early stop: the stopping block dropped instead of kept.
+    "online-stop-drops-block": ("          kept = x + 1;\n          break;",
+                                "          kept = x;\n          break;"),
+    # Online early stop: the share's denominator without the block itself.
+    "online-share-denominator": ("          den += ek[x];\n          const double share = ek[x] / den;",
+                                 "          const double share = ek[x] / den;\n          den += ek[x];"),
+    # Online early stop: the smallest share over the rows instead of the largest.
+    "online-min-over-rows": ("          if (share > ms[x]) ms[x] = share;",
+                             "          if (e == 0 || share < ms[x]) ms[x] = share;"),
     # Pooled means summed in one pass instead of chunks of B list entries.
     "one-chunk-sum": ("  float *total = calloc((size_t)d, sizeof(float));",
                       "  chunk = len;\n  float *total = calloc((size_t)d, sizeof(float));"),
@@ -58,6 +67,8 @@ PIN_TESTS = [
     pins.test_float64_rederivation_of_pooled_quantities,
     pins.test_sum_order_case_chunked_means,
     pins.test_sum_order_case_normaliser_chunks,
+    pins.test_online_stop_hand_case,
+    lambda: pins.test_online_stop_against_softmax_probabilities(0.03),
 ]
 
 

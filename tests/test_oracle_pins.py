@@ -470,3 +470,90 @@ def test_sum_order_case_normaliser_chunks():
     assert (idx["sel_blk"][0, 0, first:, 0] == e["sel_blk0_segment1"]).all()
     assert (idx["sel_cnt"][0, 0, :first] == 0).all()
     assert nB > 32  # the normaliser spans more than one 32-block chunk
+
+
+# ----------------------------------------------------------------------------- online early stop
+
+def test_online_stop_hand_case():
+    """The measured-share stop on the hand case with τ = 0.4 and given lists (closed forms derived
+    by hand in tests/golden/online_stop_case.md)."""
+    g, c, q, k, _ = _hand()
+    cfg = _cfg(c, 0.4)
+    idx = oracle.build_indices(cfg, q, k)
+    lists = {3: [1, 2, 0], 2: [2, 0, 1]}
+    sel_cnt = np.zeros((1, 1, 4), np.int32)
+    sel_blk = np.full((1, 1, 4, 4), -1, np.int32)
+    for b, lst in lists.items():
+        sel_cnt[0, 0, b] = len(lst)
+        sel_blk[0, 0, b, :len(lst)] = lst
+    idx = dict(idx, sel_cnt=sel_cnt, sel_blk=sel_blk)
+    stop, share = oracle.online_stop(cfg, q, k, idx)
+    e, r = math.e, math.exp(0.5)
+    want3 = [0.5, 2 / (2 * r + 2), e / (2 * r + 2 + e)]
+    want2 = [(r + 1) / (e + 4 + r), e * e / (e + 4 + e * e), e / (2 * e + 4 + e * e)]
+    np.testing.assert_allclose(share[0, 0, 3, :3], want3, rtol=1e-14)
+    np.testing.assert_allclose(share[0, 0, 2, :3], want2, rtol=1e-14)
+    np.testing.assert_array_equal(stop[0, 0], [0, 0, 1, 2])
+
+
+def test_online_stop_tau_zero_keeps_every_list():
+    w = SMALL_GQA.replace(tau=0.0)
+    cfg = oracle.config(w)
+    q, k, _ = gen.make_inputs(w)
+    idx = oracle.build_indices(cfg, q, k)
+    stop, _ = oracle.online_stop(cfg, q, k, idx)
+    np.testing.assert_array_equal(stop, idx["sel_cnt"])
+
+
+STOP_CASE = gen.Workload("online-stop", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=2048,
+                         head_dim=64, segment_len=256, block_size=64, tau=0.0, seed=13, amp=4.0,
+                         stripe_count=60, diag=0.5)
+
+
+@pytest.mark.parametrize("tau", [0.005, 0.03, 0.08])
+def test_online_stop_against_softmax_probabilities(tau):
+    """Brute force from another formulation: each row's softmax probabilities over its whole list
+    key set (torch, float64); a block's share is its probability mass over the mass of the keys up
+    to and including it. Lists: every candidate block (built at τ = 0), so that later blocks carry
+    little mass and the stop at τ cuts them. The stop keeps lists as prefixes and never lengthens
+    them."""
+    w = STOP_CASE
+    q, k, _ = gen.make_inputs(w)
+    idx = oracle.build_indices(oracle.config(w), q, k)
+    cfg = oracle.config(w, tau=tau)
+    stop, share = oracle.online_stop(cfg, q, k, idx)
+    assert (stop <= idx["sel_cnt"]).all() and ((stop > 0) == (idx["sel_cnt"] > 0)).all()
+    N, B, S, d = w.seq_len, w.block_size, w.segment_len, w.head_dim
+    G = w.n_q_heads // w.n_kv_heads
+    nB = N // B
+    qf, kf = q.double(), k.double()
+    stopped_somewhere = False
+    for beta in range(w.batch):
+        for h in range(w.n_q_heads):
+            g = h // G
+            for b in range(nB):
+                cnt = idx["sel_cnt"][beta, h, b]
+                if cnt == 0:
+                    continue
+                s0 = (b * B // S) * S
+                lst = idx["sel_blk"][beta, h, b, :cnt]
+                pk = idx["perm_k"][beta, h]
+                vis = [[j for j in pk[c * B:(c + 1) * B] if j < s0] for c in lst]
+                best = np.zeros(cnt)
+                for i in idx["perm_q"][beta, h, b * B:(b + 1) * B]:
+                    keys = list(range(s0, i + 1)) + [j for v in vis for j in v]
+                    z = (qf[beta, h, i] @ kf[beta, g, keys].T) / math.sqrt(d)
+                    prob = torch.softmax(z, dim=0).numpy()
+                    mass = dict(zip(keys, prob))
+                    run = sum(mass[j] for j in range(s0, i + 1))
+                    for x, v in enumerate(vis):
+                        blk = sum(mass[j] for j in v)
+                        run += blk
+                        best[x] = max(best[x], blk / run)
+                np.testing.assert_allclose(share[beta, h, b, :cnt], best, rtol=1e-9, atol=1e-15)
+                below = np.nonzero(best < tau)[0]
+                want = int(below[0]) + 1 if len(below) else int(cnt)
+                assert stop[beta, h, b] == want
+                stopped_somewhere |= want < cnt
+    if tau >= 0.03:
+        assert stopped_somewhere  # the case exercises an actual stop
