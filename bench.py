@@ -498,6 +498,51 @@ def run_sweep(args):
             raise RuntimeError("device timeout")
         return row
 
+    def measure_online(w, reps=3):
+        """The measured-share early stop (labelled variant) against the same lists run in full on
+        the same path (local pass, then the permuted pass over gathered list streams), and the
+        default path with a workspace."""
+        key = (w.name, w.seed, w.seq_len, w.stripe_frac)
+        if key not in cache:
+            cache.clear()
+            cache[key] = tuple(t.to(dev) for t in gen.make_inputs(w))
+        qd, kd, vd = cache[key]
+        cfg = s2o.Config.of(w)
+        ws = s2o.alloc_prefill_workspace(cfg, dev)
+        idx = s2o.build_indices(cfg, qd, kd, ws=ws)
+        o_full, o_stop, o_ws = (torch.empty_like(qd) for _ in range(3))
+        runs = {"full_lists": lambda: s2o.attention_prefill_with_indices(cfg, qd, kd, vd, idx,
+                                                                         out=o_full),
+                "online_stop": lambda: s2o.attention_prefill_online_stop(cfg, qd, kd, vd, idx,
+                                                                         out=o_stop),
+                "default_with_workspace": lambda: s2o.attention_prefill_with_indices_ws(
+                    cfg, qd, kd, vd, idx, ws, out=o_ws)}
+        row = {"workload": w.name, "tau": w.tau, "variant": "online stop (measured share)"}
+        stop = None
+        for name, fn in runs.items():
+            r = fn()
+            if name == "online_stop":
+                stop = r[1]
+            fn()
+            e0, e1 = events()
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            row[name + "_ms"] = e0.elapsed_time(e1) / reps
+        row["listed_blocks"] = int(idx.sel_cnt.long().sum().item())
+        row["kept_blocks"] = int(stop.long().sum().item())
+        row["cut_lists"] = int((stop < idx.sel_cnt).sum().item())
+        od = torch.empty_like(qd)
+        s2o.dense_causal_prefill(cfg, qd, kd, vd, out=od)
+        torch.cuda.synchronize()
+        row["mse_vs_dense"] = {k: float(((o.float() - od.float()) ** 2).mean().item())
+                               for k, o in (("full_lists", o_full), ("online_stop", o_stop))}
+        if s2o.check_device_status(dev) != 0:
+            raise RuntimeError("device timeout")
+        return row
+
     configs = [gen.workload("llama-32k")]
     # Labelled strong-stripe workload (beside the specified ones): the permuted pass at the
     # selection density the pages report.
@@ -518,6 +563,12 @@ def run_sweep(args):
         configs = [w for w in configs if any(f"{w.name}@{w.tau}".startswith(k) for k in keep)]
     for w in configs:
         print(json.dumps({"config": measure(w)}), flush=True)
+    online = [gen.workload("llama-128k-strong", tau=t) for t in (0.005, 0.01, 0.02)]
+    online += [gen.workload("qwen-128k", tau=0.001)]
+    if args.sweep_filter:
+        online = [w for w in online if any(f"online:{w.name}@{w.tau}".startswith(k) for k in keep)]
+    for w in online:
+        print(json.dumps({"online_stop": measure_online(w)}), flush=True)
     if args.sweep_filter and "stack" not in args.sweep_filter.split(","):
         return 0
     stack = [measure(gen.layer_workload(l), reps=2, dense=(l % 8 == 7)) for l in range(32)]

@@ -137,6 +137,23 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
                                               const s2o_indices *idx, void *o,
                                               s2o_stream stream);
 
+/* Steps 3-4 with the measured-share early stop (a labelled variant of the survey's NEXT-2 row;
+ * [S2O, Summary ¶2]: blocks run from most to least important and the loop "stops once a block's
+ * score falls under a threshold τ", here the block's measured score; [BSFA, abstract]: pruning on
+ * exact block scores). Each busy query block runs its local tiles, then its listed blocks in list
+ * order; after a listed block that is not the list's last, the block's share of each row's
+ * running softmax normaliser (the block's exp-sum over the sum after it) is compared with
+ * cfg->tau, and the list stops when the share is below tau for every row of the block (that block
+ * is kept). The rows of each query block get the attention over the local window and the kept
+ * blocks. stop_cnt [batch, Hq, nB] (device int32, 16-byte aligned, owned by the caller) receives
+ * the listed blocks each query block kept (0 for empty lists). tau = 0 never stops. Uses the path
+ * without a workspace (local pass, then the permuted pass over list streams). Errors as
+ * s2o_attention_prefill_with_indices, plus S2O_ERR_INVALID_ARGUMENT for a null stop_cnt. */
+s2o_status s2o_attention_prefill_online_stop(const s2o_config *cfg, const void *q,
+                                             const void *k, const void *v,
+                                             const s2o_indices *idx, void *o, int32_t *stop_cnt,
+                                             s2o_stream stream);
+
 /* Bytes of scratch with which s2o_attention_prefill and s2o_attention_prefill_with_indices_ws run
  * the merge path and may use packed streams (see s2o_set_permuted_copy): s2o_workspace_size, a
  * 256-byte flag area, one fp32 log2-sum-exp per query row (batch · n_q_heads · N), the permuted

@@ -28,6 +28,7 @@ __all__ = [
     "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
     "prefill_workspace_size", "alloc_prefill_workspace", "attention_prefill_with_indices_ws",
     "set_permuted_copy", "layer_workspace_size", "layer_prefill", "WorkCounts", "attention_work",
+    "attention_prefill_online_stop",
 ]
 
 STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
@@ -185,6 +186,7 @@ def _load():
             "s2o_attention_prefill": [C, vp, vp, vp, vp, I, vp, sz, vp],
             "s2o_attention_prefill_with_indices": [C, vp, vp, vp, I, vp, vp],
             "s2o_attention_prefill_with_indices_ws": [C, vp, vp, vp, I, vp, vp, sz, vp],
+            "s2o_attention_prefill_online_stop": [C, vp, vp, vp, I, vp, vp, vp],
             "s2o_dense_causal_prefill": [C, vp, vp, vp, vp, vp],
             "s2o_validate_indices": [C, I, vp, sz, vp],
             "s2o_index_stats": [C, I, vp, sz, ctypes.POINTER(_Stats), vp],
@@ -371,6 +373,24 @@ def attention_prefill_with_indices_ws(cfg: Config, q, k, v, idx: Indices, ws: to
                                                          _stream(q.device)),
            "s2o_attention_prefill_with_indices_ws")
     return o
+
+
+def attention_prefill_online_stop(cfg: Config, q, k, v, idx: Indices,
+                                  out: torch.Tensor | None = None):
+    """Steps 3-4 with the measured-share early stop (labelled variant; stop threshold cfg.tau).
+    Returns (O, stop_cnt): the listed blocks each query block kept, int32 [batch, Hq, nB]."""
+    _qkv(cfg, q, k, v)
+    o = out if out is not None else torch.empty_like(q)
+    _bf16(o, q.shape, "out")
+    stop = torch.empty((cfg.batch, cfg.n_q_heads, cfg.n_blocks), dtype=torch.int32,
+                       device=q.device)
+    ci = idx._c()
+    _check(_load().s2o_attention_prefill_online_stop(ctypes.byref(cfg._c()), q.data_ptr(),
+                                                     k.data_ptr(), v.data_ptr(), ctypes.byref(ci),
+                                                     o.data_ptr(), stop.data_ptr(),
+                                                     _stream(q.device)),
+           "s2o_attention_prefill_online_stop")
+    return o, stop
 
 
 def dense_causal_prefill(cfg: Config, q, k, v, out: torch.Tensor | None = None) -> torch.Tensor:

@@ -270,6 +270,27 @@ s2o_status s2o_attention_prefill_with_indices(const s2o_config *cfg, const void 
                                     (cudaStream_t)stream));
 }
 
+s2o_status s2o_attention_prefill_online_stop(const s2o_config *cfg, const void *q,
+                                             const void *k, const void *v,
+                                             const s2o_indices *idx, void *o, int32_t *stop_cnt,
+                                             s2o_stream stream) {
+  s2o_status st = check_config(cfg);
+  if (st != S2O_OK) return st;
+  if (!q || !k || !v || !o || !stop_cnt || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(o) || !aligned16(stop_cnt) || !indices_ok(idx))
+    return S2O_ERR_INVALID_ARGUMENT;
+  const Dims d = dims_of(*cfg);
+  cudaStream_t s = (cudaStream_t)stream;
+  // Query blocks without a selected block keep none (the permuted pass writes the others).
+  if (cudaMemsetAsync(stop_cnt, 0, (size_t)d.bhq() * d.nB * sizeof(int32_t), s) != cudaSuccess)
+    return S2O_ERR_CUDA;
+  AttnArgs a{q, k, v, o, idx->perm_q, idx->perm_k, idx->sel_cnt, idx->sel_blk, idx->local_tiles,
+             false};
+  a.stop_cnt = stop_cnt;
+  a.stop_tau = cfg->tau;
+  return from_cuda(launch_attention(d, a, g_wait_limit_ns.load(), g_attention_max_ctas.load(), s));
+}
+
 s2o_status s2o_attention_prefill_with_indices_ws(const s2o_config *cfg, const void *q,
                                                  const void *k, const void *v,
                                                  const s2o_indices *idx, void *o, void *ws,

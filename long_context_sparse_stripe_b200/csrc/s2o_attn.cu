@@ -277,6 +277,9 @@ enum Bar {
   kOSel = 27,    // 2: an atom of the permuted pass's partial rows landed in the output stage
   kNumBars = 29
 };
+// Byte offset in the barrier area of the two early-stop flags (after the barriers and the TMEM
+// address).
+constexpr int kStopFlagAt = 240;
 
 // Unit sets of a launch.
 enum Mode {
@@ -316,8 +319,11 @@ struct FastDiv {
 //                local tiles, see Params::sel_only);
 //   kKindPacked  the permuted pass over packed streams from the permuted copy of K and V (see
 //                below);
-//   kKindMerge   the local pass that also merges each row with the permuted pass's partial result.
-enum Kind { kKindContig = 0, kKindList = 1, kKindPacked = 2, kKindMerge = 3 };
+//   kKindMerge   the local pass that also merges each row with the permuted pass's partial result;
+//   kKindOnline  the permuted pass over list streams with the measured-share early stop (a
+//                labelled variant): a query block's list ends after the first selected block
+//                whose share of every row's running normaliser is below τ.
+enum Kind { kKindContig = 0, kKindList = 1, kKindPacked = 2, kKindMerge = 3, kKindOnline = 4 };
 
 struct Params {
   const int32_t *perm_q, *perm_k, *sel_cnt, *sel_blk, *local_tiles;
@@ -350,6 +356,9 @@ struct Params {
   const int4 *pair_meta;
   long long chunk_cap;
   int pair_heads;
+  // Measured-share early stop (kKindOnline): the listed blocks each busy query block kept.
+  int32_t *stop_cnt;
+  float stop_tau;
 };
 
 struct Unit {
@@ -367,7 +376,7 @@ struct Unit {
 // it is the list-stream order, so that a pair is two query heads of one KV head at one block.
 template <int BN, int KIND>
 __device__ __forceinline__ Unit decode_unit(const Params &p, uint32_t u) {
-  constexpr bool PERM = KIND == kKindList || KIND == kKindPacked;
+  constexpr bool PERM = KIND == kKindList || KIND == kKindPacked || KIND == kKindOnline;
   constexpr bool PACKED = KIND == kKindPacked;
   // Unit ids are below 2^31 (the host checks): divisions by multiply-high.
   Unit r;
@@ -825,9 +834,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_kp16,
                          const __grid_constant__ CUtensorMap tm_vp16, const Params p) {
   using L = Layout<D, BN>;
-  constexpr bool PERM = KIND == kKindList || KIND == kKindPacked;
+  constexpr bool PERM = KIND == kKindList || KIND == kKindPacked || KIND == kKindOnline;
   constexpr bool PACKED = KIND == kKindPacked;
   constexpr bool MERGE = KIND == kKindMerge;
+  constexpr bool ONLINE = KIND == kKindOnline;
   constexpr int CPT = BN / kChunkRows;  // chunks per packed tile
   if (p.copy_flag != nullptr && (__ldg(p.copy_flag) & p.run_mask) != p.run_value) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -837,6 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = sbase + L::OFF_Q, sK = sbase + L::OFF_K, sV = sbase + L::OFF_V,
                  sBar = sbase + L::OFF_BAR;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_BAR + kNumBars * 8);
+  // kKindOnline: per query tile, set by its softmax group when the unit's list stops early.
+  volatile int *stop_flag = reinterpret_cast<volatile int *>(smem + L::OFF_BAR + kStopFlagAt);
   auto bar = [&](int i) { return sBar + 8u * (uint32_t)i; };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -1082,6 +1094,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool pend_last[2] = {false, false};
         uint32_t acc[2] = {0u, 0u};
         uint32_t vleft = 0;  // 2 bits per V stage: products still to issue on its tile
+        // kKindOnline: units of the current work item whose list stopped early.
+        bool done[2] = {false, false};
         // The V stage is released once every unit using the tile has issued its product.
         auto issue_pv = [&](auto xc) -> bool {
           constexpr int x = decltype(xc)::value;
@@ -1108,7 +1122,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t left = ((vleft >> (2 * vs)) & 3u) - 1u;
           vleft = (vleft & ~(3u << (2 * vs))) | ((left & 3u) << (2 * vs));
           if (left == 0) tc_commit(bar(kVEmpty + vs));
-          if (pend_last[x]) {
+          bool last = pend_last[x];
+          if (ONLINE && !last && stop_flag[x] != 0) {
+            // The softmax group stopped the unit's list at this block (its flag was written
+            // before the P arrival just waited for): this is the unit's last product, and its Q
+            // tile is free.
+            last = true;
+            done[x] = true;
+            tc_commit(bar(kQEmpty + x));
+          }
+          if (last) {
             tc_commit(bar(kOFull + x));
             acc[x] = 0u;
           }
@@ -1133,14 +1156,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto users_seq = [&](int j) -> int { return users_at<KIND>(P, j); };
         const int n_of[2] = {P.u0.lt + P.u0.cnt, P.valid1 ? P.u1.lt + P.u1.cnt : 0};
         int qk[2] = {0, 0};
+        int issued = 0;  // units that ran a product on the current stream item
+        done[0] = done[1] = false;
         // One unit's step at stream item j: its pending product goes first, or now if the unit
         // skips the next item (its V tile must leave the ring); a unit's first Q_x·Kᵀ waits for
         // its Q_x tile.
         auto step = [&](auto xc, int j, int users, int nusers, const uint64_t (&kb)[8]) -> bool {
           constexpr int x = decltype(xc)::value;
-          const bool use = (users >> x) & 1;
+          bool use = ((users >> x) & 1) && !(ONLINE && done[x]);
           if (pend[x] != kNone && (use || !((nusers >> x) & 1)) && !issue_pv(xc)) return false;
+          if (ONLINE) use = use && !done[x];  // the pending product may have ended the unit
           if (use) {
+            issued |= 1 << x;
             if (qk[x] == 0) {
               if (!mbar_wait(bar(kQFull + x), q_ph[x], lim)) return false;
               q_ph[x] ^= 1u;
@@ -1165,6 +1192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint64_t kb[8];
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) kb[kk] = kd + kOffK[kk % (D / 16)];
+          issued = 0;
           if (!step(std::integral_constant<int, 0>{}, j, users, nusers, kb) ||
               !step(std::integral_constant<int, 1>{}, j, users, nusers, kb)) {
             ok = false;
@@ -1172,7 +1200,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(kKEmpty + k_st));
           const uint32_t vs = (v_base + (uint32_t)j) & (L::VST - 1);
-          vleft = (vleft & ~(3u << (2 * vs))) | ((uint32_t)__popc(users) << (2 * vs));
+          const int eff = ONLINE ? issued : users;
+          vleft = (vleft & ~(3u << (2 * vs))) | ((uint32_t)__popc(eff) << (2 * vs));
+          if (ONLINE && eff == 0) {
+            // No unit uses this item any more (its list stopped): the V tile is released once
+            // it has landed.
+            if (!mbar_wait(bar(kVFull + vs), ((v_base + (uint32_t)j) / L::VST) & 1u, lim)) {
+              ok = false;
+              break;
+            }
+            tc_commit(bar(kVEmpty + vs));
+          }
           if (++k_st == (uint32_t)L::KST) {
             k_st = 0;
             k_ph ^= 1u;
@@ -1225,6 +1263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float m_run = -INFINITY, l_run = 0.f;
       const int n_items = u.lt + u.cnt;
+      // kKindOnline: the listed blocks this unit keeps (all, unless its list stops early); the
+      // flag is cleared before this unit's first P arrival.
+      int kept = u.cnt;
+      if (ONLINE && quad == 0 && lane == 0) stop_flag[x] = 0;
       // Keys of a selected block (for its mask) are requested before the wait for its S, the
       // block id one tile earlier.
       auto blk = [&](int n) {
@@ -1341,11 +1383,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         l_run = l_run * alpha + rs;
         m_run = PERM ? m_keep : m_use;
+        // kKindOnline: after a listed block that is not the list's last, the block's measured
+        // share of each row's running normaliser (this tile's exp-sum over the sum after it, both
+        // against the same running maximum); the list stops when it is below τ for every row of
+        // the block (a reduction over the group's 128 threads), and the flag tells the issuer
+        // before this tile's P arrival.
+        bool stop_now = false;
+        if (ONLINE && n >= u.lt && n + 1 < n_items) {
+          const bool keep = row < BN && store_row && rs / l_run >= p.stop_tau;
+          stop_now = !named_bar_or(2 + x, 128, keep);
+          if (stop_now && quad == 0 && lane == 0) stop_flag[x] = 1;
+        }
         // One arrival per warp (after the warp's tensor-memory stores): arrivals on one barrier
         // are serialised, so 128 of them would delay the product by hundreds of cycles.
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kPFull + x));
+        if (ONLINE && stop_now) {
+          kept = n - u.lt + 1;
+          break;
+        }
       }
       if (!ok) break;
       // Epilogue: O/ℓ as bf16 at the query's original row.
@@ -1355,6 +1412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++on;
       tc_fence_after();
+      if (ONLINE && quad == 0 && lane == 0) p.stop_cnt[u.qh * p.nB + u.b] = kept;
       const float inv_l = 1.f / l_run;
       uint16_t *orow = p.o + ((size_t)u.qh * p.N + i_orig) * D;
       // MERGE: the row's final result combines this pass's O/ℓ with the permuted pass's partial
@@ -1823,7 +1881,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
                      cudaStream_t st) {
   using L = Layout<D, BN>;
   static_assert(L::SMEM <= 232448, "shared memory budget");
-  static_assert(kNumBars * 8 + 4 <= (int)L::BAR_BYTES, "barrier area");
+  static_assert(kNumBars * 8 + 4 <= kStopFlagAt && kStopFlagAt + 8 <= (int)L::BAR_BYTES,
+                "barrier area");
   CUtensorMap tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp;
   const long long q_rows = d.bhq() * d.N, kv_rows = d.bhkv() * d.N;
   if (!make_map(&tq, a.q, q_rows, D, BN) || !make_map(&tqr, a.q, q_rows, D, 1) ||
@@ -1846,7 +1905,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   }
   cudaError_t e = cudaSuccess;
   for (auto fn : {s2o_attention_kernel<D, BN, kKindContig>, s2o_attention_kernel<D, BN, kKindList>,
-                  s2o_attention_kernel<D, BN, kKindPacked>, s2o_attention_kernel<D, BN, kKindMerge>})
+                  s2o_attention_kernel<D, BN, kKindPacked>, s2o_attention_kernel<D, BN, kKindMerge>,
+                  s2o_attention_kernel<D, BN, kKindOnline>})
     if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)L::SMEM)) != cudaSuccess)
       return e;
@@ -1879,6 +1939,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   p.pair_meta = a.pair_meta;
   p.chunk_cap = a.chunk_cap;
   p.pair_heads = a.copy_per_kv ? 1 : 0;
+  p.stop_cnt = a.stop_cnt;
+  p.stop_tau = a.stop_tau;
   auto launch = [&](int mode, int skip_empty, int kind) -> cudaError_t {
     p.mode = mode;
     p.skip_empty = skip_empty;
@@ -1886,7 +1948,8 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
     p.nSeg = mode == kDense ? 1 : d.nSeg;
     p.div_seg.init(p.S / BN);
     p.div_nSeg.init(p.nSeg);
-    const long long work = skip_empty && kind == kKindList ? p.n_units : p.n_items;
+    const long long work =
+        skip_empty && (kind == kKindList || kind == kKindOnline) ? p.n_units : p.n_items;
     const long long cap = max_ctas > 0 && max_ctas < sm_count() ? max_ctas : sm_count();
     const long long grid = work < cap ? work : cap;
     switch (kind) {
@@ -1900,6 +1963,10 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
         break;
       case kKindPacked:
         s2o_attention_kernel<D, BN, kKindPacked><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
+            tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
+        break;
+      case kKindOnline:
+        s2o_attention_kernel<D, BN, kKindOnline><<<(unsigned)grid, kThreads, L::SMEM, st>>>(
             tq, tqr, tk, tkr, tv, tvr, to, tkp, tvp, p);
         break;
       default:
@@ -1920,7 +1987,7 @@ cudaError_t launch_t(const Dims &d, const AttnArgs &a, uint64_t limit_ns, int ma
   auto legacy = [&]() -> cudaError_t {
     cudaError_t r = launch(kLocal, 0, kKindContig);
     if (r != cudaSuccess) return r;
-    return launch(kPermuted, 1, kKindList);
+    return launch(kPermuted, 1, a.stop_cnt != nullptr ? kKindOnline : kKindList);
   };
   if (!a.merge || a.lse == nullptr) return legacy();
   // With a workspace every path is launched and the device-side decision word lets one run (the

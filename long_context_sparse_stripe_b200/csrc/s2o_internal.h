@@ -60,6 +60,11 @@ struct AttnArgs {
   uint32_t *chunks = nullptr;     // [pairs, chunk_cap] chunk words of the packed streams
   int4 *pair_meta = nullptr;      // [pairs] tile counts {shared, unit 0 only, unit 1 only, -}
   long long chunk_cap = 0;
+  // Measured-share early stop (a labelled variant, path without a workspace only): the permuted
+  // pass stops a query block's list after the first block whose share of every row's running
+  // normaliser is below stop_tau, and writes the listed blocks each busy query block kept.
+  int32_t *stop_cnt = nullptr;
+  float stop_tau = 0.f;
 };
 cudaError_t launch_attention(const Dims &d, const AttnArgs &a, uint64_t wait_limit_ns,
                              int max_ctas, cudaStream_t st);

@@ -452,3 +452,82 @@ def test_attention_work_counts():
     assert packed.unit_tiles < 1.3 * attended
     assert packed.permuted_unit_tiles < gathered.permuted_unit_tiles
     assert packed.permuted_loaded_tiles < packed.permuted_unit_tiles
+
+
+# ----------------------------------------------------------------------------- online early stop
+
+# Full candidate lists (built at τ = 0) on GPU-supported shapes, so that later blocks carry little
+# mass and the measured-share stop cuts them: d = 64 with B = 64, and d = 128 with B = 128 and GQA.
+W_OS1 = gen.Workload("os1-d64-b64", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=2048, head_dim=64,
+                     segment_len=256, block_size=64, tau=0.0, seed=13, amp=4.0, stripe_count=60,
+                     diag=0.5)
+W_OS2 = gen.Workload("os2-d128-b128", batch=1, n_q_heads=4, n_kv_heads=2, seq_len=8192,
+                     head_dim=128, segment_len=1024, block_size=128, tau=0.0, seed=14, amp=4.0,
+                     stripe_frac=0.02, diag=0.5)
+STOP_TOL = 0.05  # relative band around τ inside which the GPU and the oracle may decide apart
+
+
+@pytest.mark.parametrize("w,tau", [(W_OS1, 0.03), (W_OS1, 0.08), (W_OS2, 0.02), (W_OS2, 0.03)],
+                         ids=["os1-0.03", "os1-0.08", "os2-0.02", "os2-0.03"])
+def test_online_stop_matches_oracle(w, tau):
+    """The measured-share stop (DEFINITION D13) on the oracle's full candidate lists: every GPU
+    stop position agrees with the oracle's shares (blocks the GPU went past have an oracle share of
+    at least τ·(1 − 5 %), the block it stopped after one below τ·(1 + 5 %)), the stops actually cut
+    lists, and the output equals the oracle's attention over the GPU's kept blocks."""
+    q, k, v = inputs(w)
+    ref = oracle.build_indices(oracle.config(w), q, k)
+    ocfg = oracle.config(w, tau=tau)
+    stop_o, share = oracle.online_stop(ocfg, q, k, ref)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w, tau=tau)
+    o, stop = s2o.attention_prefill_online_stop(cfg, qd, kd, vd, oracle_indices_on_device(ref))
+    torch.cuda.synchronize()
+    assert s2o.check_device_status() == 0
+    stop_g = stop.cpu().numpy()
+    cnt = ref["sel_cnt"]
+    assert (stop_g <= cnt).all() and ((stop_g > 0) == (cnt > 0)).all()
+    assert (stop_g < cnt).sum() > 0, "no list was cut"
+    for idx in np.argwhere(stop_g != stop_o):
+        g, c = int(stop_g[tuple(idx)]), int(cnt[tuple(idx)])
+        sh = share[tuple(idx)]
+        assert (sh[:g - 1] >= tau * (1 - STOP_TOL)).all(), (idx, g, sh[:g])
+        if g < c:
+            assert sh[g - 1] < tau * (1 + STOP_TOL), (idx, g, sh[g - 1])
+    agree = (stop_g == stop_o).mean()
+    assert agree > 0.95, f"only {agree:.3f} of the stop positions agree"
+    want, _ = oracle.attention(oracle.config(w), q, k, v, oracle.with_counts(ref, stop_g))
+    assert_close(o, want)
+
+
+def test_online_stop_tau_zero_keeps_lists_and_output():
+    """τ = 0 never stops: the kept counts are the list lengths and the output is the path
+    without a workspace, bit for bit (the same products in the same order)."""
+    w = W_A
+    q, k, v = to_dev(*inputs(w))
+    cfg = s2o.Config.of(w, tau=0.0)
+    idx = s2o.build_indices(cfg, q, k)
+    o, stop = s2o.attention_prefill_online_stop(cfg, q, k, v, idx)
+    base = s2o.attention_prefill_with_indices(cfg, q, k, v, idx)
+    torch.cuda.synchronize()
+    assert s2o.check_device_status() == 0
+    assert torch.equal(stop, idx.sel_cnt)
+    assert torch.equal(o, base)
+
+
+def test_online_stop_independent_of_grid():
+    w = W_OS1
+    q, k, v = inputs(w)
+    ref = oracle.build_indices(oracle.config(w), q, k)
+    qd, kd, vd = to_dev(q, k, v)
+    cfg = s2o.Config.of(w, tau=0.05)
+    idx = oracle_indices_on_device(ref)
+    o0, s0 = s2o.attention_prefill_online_stop(cfg, qd, kd, vd, idx)
+    try:
+        for n in (1, 3):
+            s2o.set_attention_max_ctas(n)
+            o, st = s2o.attention_prefill_online_stop(cfg, qd, kd, vd, idx)
+            torch.cuda.synchronize()
+            assert s2o.check_device_status() == 0
+            assert torch.equal(st, s0) and torch.equal(o, o0), f"grid of {n}"
+    finally:
+        s2o.set_attention_max_ctas(0)
