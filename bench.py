@@ -646,6 +646,35 @@ def run_layer(args):
     return 0
 
 
+def run_gemm(args):
+    """The decoder layer's projection GEMM alone (not the headline line): C = A·B (+ C) for one
+    shape, bf16 with fp32 accumulation, CUDA events; one JSON line."""
+    import long_context_sparse_stripe_b200 as s2o
+
+    torch.cuda.set_device(0)
+    m, n, k = (int(x) for x in args.gemm.split(","))
+    g = torch.Generator(device="cuda").manual_seed(0)
+    a = torch.randn(m, k, device="cuda", generator=g).to(torch.bfloat16)
+    b = (torch.randn(k, n, device="cuda", generator=g) / k ** 0.5).to(torch.bfloat16)
+    c = torch.empty(m, n, device="cuda", dtype=torch.bfloat16)
+    for _ in range(args.warmup):
+        s2o.gemm_bf16(a, b, c, accumulate=args.accumulate)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        s2o.gemm_bf16(a, b, c, accumulate=args.accumulate)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    tflops = 2.0 * m * n * k / (ms * 1e-3) / 1e12
+    peak = measured_peaks()[0]
+    print(json.dumps({"gemm": {"m": m, "n": n, "k": k, "accumulate": args.accumulate, "ms": ms,
+                               "tflops": tflops, "frac_of_measured_peak": tflops / peak,
+                               "status": s2o.check_device_status()}}), flush=True)
+    return 0
+
+
 def run_profile_target(args):
     """A short fixed sequence for profiler captures (not a bench line): one index build, then
     `--steps` attention calls and one dense-baseline call. Without `--ws-mode` each call is the
@@ -710,11 +739,16 @@ def main():
                     help="sweep only: comma-separated 'workload@tau' prefixes (and 'stack')")
     ap.add_argument("--layer", action="store_true",
                     help="end-to-end-shaped decoder layer, S2O vs dense attention (one JSON line)")
+    ap.add_argument("--gemm", default="",
+                    help="'M,N,K': time the decoder layer's projection GEMM alone (one JSON line)")
+    ap.add_argument("--accumulate", action="store_true", help="--gemm: C += A·B")
     ap.add_argument("--profile-target", action="store_true",
                     help="run a short fixed call sequence for profiler captures; print nothing")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "s2o":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.gemm:
+        return run_gemm(args)
     if args.profile_target:
         return run_profile_target(args)
     if args.sweep:

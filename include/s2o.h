@@ -280,8 +280,8 @@ s2o_status s2o_build_indices_static(const s2o_config *cfg, const void *q, const 
  * without trained weights this runs one Llama-3-architecture decoder layer with the S2O prefill
  * (or the dense causal baseline) as its attention: x += W_o·attn(RoPE(W_qkv·norm(x))), then
  * x += W_down·(silu(gate)·up) with [gate | up] = W_gu·norm(x). bf16 storage between the steps,
- * fp32 arithmetic; projections are cuBLAS GEMMs (bf16 in, fp32 accumulation), the rest this
- * library's kernels. Heads and sizes come from the s2o_config (hidden H = n_q_heads·head_dim). */
+ * fp32 arithmetic; projections are this library's tensor-core GEMM (s2o_gemm_bf16), the rest its
+ * other kernels. Heads and sizes come from the s2o_config (hidden H = n_q_heads·head_dim). */
 typedef struct {
   int intermediate;            /* MLP width I (multiple of 8)                                   */
   float rms_eps;               /* RMS norm epsilon (1e-5)                                       */
@@ -309,11 +309,22 @@ s2o_status s2o_layer_workspace_size(const s2o_config *cfg, const s2o_layer_confi
 /* One decoder layer in place on x [batch, N, H] bf16 (device, 16-byte aligned). The S2O path
  * builds its indices (cfg: segment_len, block_size, tau, variants) and runs the gather-attention
  * as s2o_attention_prefill does. Errors: S2O_ERR_INVALID_ARGUMENT / S2O_ERR_UNSUPPORTED for bad
- * arguments (H or I not a multiple of 8), S2O_ERR_WORKSPACE_TOO_SMALL, S2O_ERR_CUDA (a CUDA or
- * cuBLAS failure). Asynchronous on `stream`. */
+ * arguments (H or I not a multiple of 8), S2O_ERR_WORKSPACE_TOO_SMALL, S2O_ERR_CUDA (a CUDA
+ * failure). Asynchronous on `stream`. */
 s2o_status s2o_layer_prefill(const s2o_config *cfg, const s2o_layer_config *lc,
                              const s2o_layer_weights *w, void *x, void *ws, size_t ws_bytes,
                              s2o_stream stream);
+
+/* The decoder layer's projections: C[m, n] = A[m, k] · B[k, n] (+ C[m, n] when accumulate = 1),
+ * A, B and C row-major bf16 on the device (16-byte aligned, owned by the caller), the products
+ * accumulated in fp32 and the result (with the old C when accumulating) rounded to bf16 once.
+ * A tcgen05 kernel (M = 128, N = 256 tiles, TMEM accumulators, TMA loads); no counterpart on the
+ * pages beyond the model they run the attention in ([S2O, Key points]: Llama-3.1-8B).
+ * n and k must be multiples of 8 (S2O_ERR_UNSUPPORTED otherwise); any m. Every wait inside is
+ * bounded like the attention kernel's (s2o_set_wait_limit_ns, reported by
+ * s2o_check_device_status). Asynchronous on `stream`. */
+s2o_status s2o_gemm_bf16(const void *a, const void *b, void *c, int64_t m, int64_t n, int64_t k,
+                         int accumulate, s2o_stream stream);
 
 /* Diagnostic: evaluates the library's exp64 — the binary64 exponential behind the block weights of
  * the early stop (a Cody–Waite reduction by ln 2 and a degree-13 Taylor polynomial written for

@@ -28,7 +28,7 @@ __all__ = [
     "kernel_launch_count", "build_indices_static", "STATIC_WORKSPACE_BYTES",
     "prefill_workspace_size", "alloc_prefill_workspace", "attention_prefill_with_indices_ws",
     "set_permuted_copy", "layer_workspace_size", "layer_prefill", "WorkCounts", "attention_work",
-    "attention_prefill_online_stop",
+    "attention_prefill_online_stop", "gemm_bf16",
 ]
 
 STATUS = {0: "S2O_OK", 1: "S2O_ERR_INVALID_ARGUMENT", 2: "S2O_ERR_UNSUPPORTED",
@@ -193,6 +193,8 @@ def _load():
             "s2o_attention_work": [C, I, vp, sz, ctypes.POINTER(_Work), vp],
             "s2o_check_device_status": [vp],
             "s2o_exp64_eval": [vp, vp, ctypes.c_int, vp],
+            "s2o_gemm_bf16": [vp, vp, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                              ctypes.c_int, vp],
             "s2o_layer_workspace_size": [C, ctypes.POINTER(_LayerConfig), ctypes.POINTER(sz)],
             "s2o_layer_prefill": [C, ctypes.POINTER(_LayerConfig), ctypes.POINTER(_LayerWeights),
                                   vp, vp, sz, vp],
@@ -506,6 +508,25 @@ def set_attention_max_ctas(max_ctas: int) -> None:
 def check_device_status(device="cuda") -> int:
     """Synchronises and returns the library status (0 = S2O_OK, 6 = a bounded wait ran out)."""
     return _load().s2o_check_device_status(_stream(torch.device(device)))
+
+
+def gemm_bf16(a: torch.Tensor, b: torch.Tensor, c: torch.Tensor | None = None,
+              accumulate: bool = False) -> torch.Tensor:
+    """C = A·B (+ C when ``accumulate``): row-major bf16 CUDA tensors, fp32 accumulation."""
+    if a.dim() != 2 or b.dim() != 2 or a.shape[1] != b.shape[0]:
+        raise ValueError("a [m, k] and b [k, n] expected")
+    m, k = a.shape
+    n = b.shape[1]
+    _bf16(a, (m, k), "a")
+    _bf16(b, (k, n), "b")
+    if c is None:
+        if accumulate:
+            raise ValueError("accumulate needs c")
+        c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
+    _bf16(c, (m, n), "c")
+    _check(_load().s2o_gemm_bf16(a.data_ptr(), b.data_ptr(), c.data_ptr(), m, n, k,
+                                 1 if accumulate else 0, _stream(a.device)), "s2o_gemm_bf16")
+    return c
 
 
 def exp64_eval(x: torch.Tensor) -> torch.Tensor:

@@ -2,7 +2,7 @@
 
 Index kernels compile with ``--fmad=false`` (every rounding there is explicit anyway) and
 without fast-math, so the index arrays match the definition bit for bit; the attention kernel
-compiles with ``-O3``. The decoder-layer projections link cuBLAS (``-lcublas``). Used by ``__graft_entry__.build()`` and on first import of the package.
+compiles with ``-O3``. Used by ``__graft_entry__.build()`` and on first import of the package.
 """
 from __future__ import annotations
 
@@ -22,6 +22,7 @@ SOURCES = {
     "s2o_attn.cu": ["-O3"],
     "s2o_static_ws.cu": ["-O3"],
     "s2o_layer.cu": ["-O3"],
+    "s2o_gemm.cu": ["-O3"],
 }
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -58,7 +59,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         subprocess.run(cmd, check=True)
         objs.append(obj)
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcublas", "-lcudart_static",
+    subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static",
                     "-ldl", "-lrt", "-lpthread"], check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -352,9 +352,8 @@ s2o_status s2o_layer_prefill(const s2o_config *cfg, const s2o_layer_config *lc,
   const LayerWs L = layer_ws_layout(d, *lc);
   char *b = static_cast<char *>(ws);
   cudaStream_t s = (cudaStream_t)stream;
-  bool blas_ok = true;
-  cudaError_t e = launch_layer_pre(d, *lc, *w, x, b, L, s, &blas_ok);
-  if (e != cudaSuccess || !blas_ok) return S2O_ERR_CUDA;
+  cudaError_t e = launch_layer_pre(d, *lc, *w, x, b, L, g_wait_limit_ns.load(), s);
+  if (e != cudaSuccess) return S2O_ERR_CUDA;
   void *q = b + L.q, *k = b + L.k, *v = b + L.v, *o = b + L.o;
   if (lc->dense_attention) {
     AttnArgs a{q, k, v, o, nullptr, nullptr, nullptr, nullptr, nullptr, true};
@@ -367,8 +366,8 @@ s2o_status s2o_layer_prefill(const s2o_config *cfg, const s2o_layer_config *lc,
     st = s2o_attention_prefill(cfg, q, k, v, o, &idx, b + L.attn_ws, ws_bytes - L.attn_ws, stream);
     if (st != S2O_OK) return st;
   }
-  e = launch_layer_post(d, *lc, *w, x, b, L, s, &blas_ok);
-  if (e != cudaSuccess || !blas_ok) return S2O_ERR_CUDA;
+  e = launch_layer_post(d, *lc, *w, x, b, L, g_wait_limit_ns.load(), s);
+  if (e != cudaSuccess) return S2O_ERR_CUDA;
   return S2O_OK;
 }
 
@@ -430,6 +429,17 @@ s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *
 }
 
 void s2o_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+s2o_status s2o_gemm_bf16(const void *a, const void *b, void *c, int64_t m, int64_t n, int64_t k,
+                         int accumulate, s2o_stream stream) {
+  if (!a || !b || !c || !aligned16(a) || !aligned16(b) || !aligned16(c) || m <= 0 || n <= 0 ||
+      k <= 0 || (accumulate != 0 && accumulate != 1))
+    return S2O_ERR_INVALID_ARGUMENT;
+  if (n % 8 || k % 8 || m >= (1ll << 31) || n >= (1ll << 31) || k >= (1ll << 31))
+    return S2O_ERR_UNSUPPORTED;
+  return from_cuda(launch_gemm_bf16(a, b, c, m, n, k, accumulate != 0, g_wait_limit_ns.load(),
+                                    (cudaStream_t)stream));
+}
 
 s2o_status s2o_prefill_workspace_size(const s2o_config *cfg, size_t *bytes) {
   s2o_status st = check_config(cfg);
@@ -501,10 +511,11 @@ void s2o_set_attention_max_ctas(int max_ctas) {
 uint64_t s2o_kernel_launch_count(void) { return launch_count(); }
 
 s2o_status s2o_check_device_status(s2o_stream stream) {
-  unsigned int err = 0;
+  unsigned int err = 0, gerr = 0;
   cudaError_t e = read_and_clear_device_error(&err, (cudaStream_t)stream);
   if (e != cudaSuccess) return S2O_ERR_CUDA;
-  return err ? S2O_ERR_DEVICE_TIMEOUT : S2O_OK;
+  if (read_and_clear_gemm_error(&gerr, (cudaStream_t)stream) != cudaSuccess) return S2O_ERR_CUDA;
+  return err || gerr ? S2O_ERR_DEVICE_TIMEOUT : S2O_OK;
 }
 
 // Diagnostic: the library's exp64 (used for block weights) on n device doubles, so that tests

@@ -84,9 +84,14 @@ cudaError_t launch_packed_counts(const Dims &d, const int4 *pair_meta, const uin
 cudaError_t launch_busy_tiles(const Dims &d, const int32_t *sel_cnt, const int32_t *local_tiles,
                               unsigned long long *acc, cudaStream_t st);
 
+// bf16 GEMM on the tensor cores (s2o_gemm.cu): row-major C[m, n] = A[m, k]·B[k, n] (+ C when
+// `accumulate`), fp32 accumulation, one rounding to bf16; n and k multiples of 8 (16-byte rows).
+cudaError_t launch_gemm_bf16(const void *A, const void *B, void *C, long long m, long long n,
+                             long long k, bool accumulate, uint64_t limit_ns, cudaStream_t st);
+cudaError_t read_and_clear_gemm_error(unsigned int *out, cudaStream_t st);
+
 // Decoder layer (s2o_layer.cu): byte offsets of its buffers in the layer workspace (the attention's
-// own workspace starts at attn_ws), and the launches before and after the attention. A false
-// *blas_ok reports a cuBLAS failure (no later launch was made).
+// own workspace starts at attn_ws), and the launches before and after the attention.
 struct LayerWs {
   size_t h, qkv, q, k, v, o, o_rows, gu, a, freqs, cs, perm_q, perm_k, sel_cnt, sel_blk,
       local_tiles, attn_ws;
@@ -94,10 +99,10 @@ struct LayerWs {
 LayerWs layer_ws_layout(const Dims &d, const s2o_layer_config &lc);
 cudaError_t launch_layer_pre(const Dims &d, const s2o_layer_config &lc,
                              const s2o_layer_weights &w, const void *x, char *ws,
-                             const LayerWs &L, cudaStream_t st, bool *blas_ok);
+                             const LayerWs &L, uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_layer_post(const Dims &d, const s2o_layer_config &lc,
                               const s2o_layer_weights &w, void *x, char *ws, const LayerWs &L,
-                              cudaStream_t st, bool *blas_ok);
+                              uint64_t wait_limit_ns, cudaStream_t st);
 
 // Host-side count of kernel launches made by the library (all threads, all devices).
 void note_launch();

@@ -9,19 +9,17 @@
 //
 // Steps (rows = batch·N tokens, H = Hq·d):
 //   k_rmsnorm      h = bf16(g ⊙ x · (mean x² + eps)^-1/2), one warp per row
-//   GEMM           qkv = h · W_qkv                       (cuBLAS, bf16 in, fp32 accumulate)
+//   GEMM           qkv = h · W_qkv                       (tcgen05 GEMM, bf16 in, fp32 accumulate)
 //   k_rope_split   rotate q and k by the angle table, write Q/K/V head-major [b, h, N, d]
 //   attention      S2O (index build + permuted gather-attention) or dense causal
 //   k_heads_to_rows O [b, Hq, N, d] -> rows [b·N, Hq·d]
-//   GEMM           x += O_rows · W_o                     (beta = 1: the residual in the sum)
+//   GEMM           x += O_rows · W_o                     (the residual added before the rounding)
 //   k_rmsnorm      h2 = norm(x)
 //   GEMM           gu = h2 · W_gu
 //   k_silu_mul     a = bf16(silu(gate) · up)
 //   GEMM           x += a · W_down
 // The frequency table (binary64) and the angle table (cos, sin of position·f_t from binary64
 // sincos, rounded to fp32) are built per call.
-#include <cublas_v2.h>
-
 #include <cmath>
 #include <type_traits>
 
@@ -183,25 +181,6 @@ __global__ void __launch_bounds__(256)
 
 unsigned grid_for(long long n, int per) { return (unsigned)((n + per - 1) / per); }
 
-// One cuBLAS handle per host thread and device.
-cublasHandle_t blas_handle() {
-  thread_local cublasHandle_t handles[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!handles[dev] && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
-  return handles[dev];
-}
-
-// Row-major C[m, n] = A[m, k] · B[k, n] (+ C when accumulate), bf16 with fp32 accumulation: the
-// column-major product Cᵀ = Bᵀ · Aᵀ.
-bool gemm(cublasHandle_t hd, const void *A, const void *B, void *C, long long m, long long n,
-          long long k, bool accumulate) {
-  const float alpha = 1.f, beta = accumulate ? 1.f : 0.f;
-  return cublasGemmEx(hd, CUBLAS_OP_N, CUBLAS_OP_N, (int)n, (int)m, (int)k, &alpha, B, CUDA_R_16BF,
-                      (int)n, A, CUDA_R_16BF, (int)k, &beta, C, CUDA_R_16BF, (int)n,
-                      CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
-}
-
 }  // namespace
 
 namespace {
@@ -259,13 +238,8 @@ LayerWs layer_ws_layout(const Dims &d, const s2o_layer_config &lc) {
 
 cudaError_t launch_layer_pre(const Dims &d, const s2o_layer_config &lc,
                              const s2o_layer_weights &w, const void *x, char *ws,
-                             const LayerWs &L, cudaStream_t st, bool *blas_ok) {
-  *blas_ok = true;
-  cublasHandle_t hd = blas_handle();
-  if (!hd || cublasSetStream(hd, st) != CUBLAS_STATUS_SUCCESS) {
-    *blas_ok = false;
-    return cudaSuccess;
-  }
+                             const LayerWs &L, uint64_t wait_limit_ns, cudaStream_t st) {
+  cudaError_t e;
   const long long rows = (long long)d.batch * d.N, H = (long long)d.Hq * d.D;
   const long long qkvw = (long long)(d.Hq + 2 * d.Hkv) * d.D;
   uint16_t *h = reinterpret_cast<uint16_t *>(ws + L.h);
@@ -273,10 +247,9 @@ cudaError_t launch_layer_pre(const Dims &d, const s2o_layer_config &lc,
                                                static_cast<const uint16_t *>(w.attn_norm), h,
                                                (int)H, lc.rms_eps, rows);
   note_launch();
-  if (!gemm(hd, h, w.w_qkv, ws + L.qkv, rows, qkvw, H, false)) {
-    *blas_ok = false;
-    return cudaSuccess;
-  }
+  if ((e = launch_gemm_bf16(h, w.w_qkv, ws + L.qkv, rows, qkvw, H, false, wait_limit_ns, st)) !=
+      cudaSuccess)
+    return e;
   k_rope_freqs<<<1, 64, 0, st>>>(reinterpret_cast<double *>(ws + L.freqs), d.D, lc.rope_theta,
                                  lc.rope_factor, lc.rope_low_freq_factor, lc.rope_high_freq_factor,
                                  (double)lc.rope_original_context);
@@ -300,13 +273,8 @@ cudaError_t launch_layer_pre(const Dims &d, const s2o_layer_config &lc,
 
 cudaError_t launch_layer_post(const Dims &d, const s2o_layer_config &lc,
                               const s2o_layer_weights &w, void *x, char *ws, const LayerWs &L,
-                              cudaStream_t st, bool *blas_ok) {
-  *blas_ok = true;
-  cublasHandle_t hd = blas_handle();
-  if (!hd || cublasSetStream(hd, st) != CUBLAS_STATUS_SUCCESS) {
-    *blas_ok = false;
-    return cudaSuccess;
-  }
+                              uint64_t wait_limit_ns, cudaStream_t st) {
+  cudaError_t e;
   const long long rows = (long long)d.batch * d.N, H = (long long)d.Hq * d.D;
   const long long I = lc.intermediate;
   const long long pieces = rows * H / 8;
@@ -319,26 +287,23 @@ cudaError_t launch_layer_post(const Dims &d, const s2o_layer_config &lc,
         reinterpret_cast<const uint4 *>(ws + L.o), reinterpret_cast<uint4 *>(ws + L.o_rows), d.N,
         d.Hq, pieces);
   note_launch();
-  if (!gemm(hd, ws + L.o_rows, w.w_o, x, rows, H, H, true)) {
-    *blas_ok = false;
-    return cudaSuccess;
-  }
+  if ((e = launch_gemm_bf16(ws + L.o_rows, w.w_o, x, rows, H, H, true, wait_limit_ns, st)) !=
+      cudaSuccess)
+    return e;
   uint16_t *h = reinterpret_cast<uint16_t *>(ws + L.h);
   k_rmsnorm<<<grid_for(rows, 8), 256, 0, st>>>(static_cast<const uint16_t *>(x),
                                                static_cast<const uint16_t *>(w.mlp_norm), h,
                                                (int)H, lc.rms_eps, rows);
   note_launch();
-  if (!gemm(hd, h, w.w_gu, ws + L.gu, rows, 2 * I, H, false)) {
-    *blas_ok = false;
-    return cudaSuccess;
-  }
+  if ((e = launch_gemm_bf16(h, w.w_gu, ws + L.gu, rows, 2 * I, H, false, wait_limit_ns, st)) !=
+      cudaSuccess)
+    return e;
   k_silu_mul<<<(unsigned)rows, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(ws + L.gu),
                                              reinterpret_cast<uint16_t *>(ws + L.a), (int)I);
   note_launch();
-  if (!gemm(hd, ws + L.a, w.w_down, x, rows, H, I, true)) {
-    *blas_ok = false;
-    return cudaSuccess;
-  }
+  if ((e = launch_gemm_bf16(ws + L.a, w.w_down, x, rows, H, I, true, wait_limit_ns, st)) !=
+      cudaSuccess)
+    return e;
   return cudaGetLastError();
 }
 
