@@ -4,16 +4,20 @@
 //
 // C[m, n] = A[m, k] · B[k, n] (+ C[m, n] when accumulating), all row-major bf16, the sum in fp32
 // and rounded to bf16 once (the residual adds into the same rounding). One persistent CTA per SM,
-// 192 threads:
-//   warp 0      TMA producer: per K step of 64, the A tile (128 rows × 64, K-major, one 128-byte
+// 192 threads, 256 × 256 output tiles:
+//   warp 0      TMA producer: per K step of 64, the A tile (256 rows × 64, K-major, one 128-byte
 //               swizzled box) and the B tile (64 × 256, N-major: four {64, 64} boxes, one per
-//               64-column atom) into a 4-stage ring.
-//   warp 1      MMA issuer (one elected thread): four tcgen05.mma kind::f16 (M = 128, N = 256,
-//               K = 16) per stage into a TMEM accumulator of 256 fp32 columns; two accumulators
-//               alternate between tiles, so a tile's epilogue overlaps the next tile's products.
-//   warps 2-5   epilogue: the thread of TMEM lane r owns row r of the tile, reads 32 columns at a
+//               64-column atom) into a 3-stage ring.
+//   warp 1      MMA issuer (one elected thread): per stage, four tcgen05.mma kind::f16 (M = 128,
+//               N = 256, K = 16) for each 128-row half of the tile, both halves reading the same
+//               B tile, into two TMEM accumulators of 256 fp32 columns (all 512 columns). A tile's
+//               first products of a half wait until the epilogue has read that half of the previous
+//               tile.
+//   warps 2-5   epilogue: the thread of TMEM lane r owns row r of each half, reads 32 columns at a
 //               time with tcgen05.ld, adds the old C when accumulating, rounds to bf16 and stores
-//               64 bytes per row and chunk.
+//               64 bytes per row and chunk; it frees each half as soon as it has read it.
+// Per stage the two halves share the B tile: 64 KB of loads per 8.4 MFLOP (131 FLOP per byte from
+// L2), against 87 with a single 128-row half.
 // Tiles are walked in groups of 32 row tiles per column tile, so a group's A panels and the B
 // panel in use stay in L2. Every wait is bounded by %globaltimer (the same limit as the attention
 // kernel); on a timeout the kernel records it in its error word, drains its copies and products,
@@ -31,18 +35,20 @@ __device__ unsigned int g_gemm_error;
 
 namespace {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4, kThreadsG = 192, kGroupM = 32;
-constexpr uint32_t kABytes = kBM * kBK * 2;     // 16 KB: 128 rows × 128 bytes
+constexpr int kBM = 256, kHalf = 128, kBN = 256, kBK = 64, kStages = 3, kThreadsG = 192,
+              kGroupM = 16;
+constexpr uint32_t kABytes = kBM * kBK * 2;     // 32 KB: 256 rows × 128 bytes
+constexpr uint32_t kAHalf = kHalf * kBK * 2;    // 16 KB: one 128-row half
 constexpr uint32_t kBAtom = kBK * 128;          // 8 KB: 64 k-rows × 64 columns
 constexpr uint32_t kBBytes = (kBN / 64) * kBAtom;  // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kOffBar = kStages * kStageBytes;  // 192 KB of stages
 constexpr uint32_t kSmem = kOffBar + 256 + 1024;    // barriers + alignment slack
-constexpr uint32_t kTmemCols = 512;                 // two accumulators of 256 columns
+constexpr uint32_t kTmemCols = 512;                 // one accumulator of 256 columns per half
 constexpr uint64_t kDrainNs = 2000000000ull;
 
-// Barrier slots: full[4], empty[4], acc_full[2], acc_empty[2], drain.
-enum { kFull = 0, kEmpty = 4, kAccFull = 8, kAccEmpty = 10, kDrainBar = 12, kBars = 13 };
+// Barrier slots: full[3], empty[3], acc_full, acc_empty[2] (one per half), drain.
+enum { kFull = 0, kEmpty = 3, kAccFull = 6, kAccEmpty = 7, kDrainBar = 9, kBars = 10 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -199,10 +205,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
       mbar_init(bar(kFull + s), 1);
       mbar_init(bar(kEmpty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(kAccFull + b), 1);
-      mbar_init(bar(kAccEmpty + b), 4);  // one arrival per epilogue warp
-    }
+    mbar_init(bar(kAccFull), 1);
+    for (int h = 0; h < 2; ++h) mbar_init(bar(kAccEmpty + h), 4);  // one arrival per epilogue warp
     mbar_init(bar(kDrainBar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -257,18 +261,10 @@ __global__ void __launch_bounds__(kThreadsG, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, 0, 1);
+      constexpr uint32_t kIdesc = idesc_bf16(kHalf, kBN, 0, 1);
       long long it = 0;
       int tcount = 0;
       for (long long t = blockIdx.x; ok && t < g.tiles; t += gridDim.x, ++tcount) {
-        const int buf = tcount & 1;
-        // The epilogue has read this accumulator's previous tile (two tiles ago).
-        if (tcount >= 2 && !mbar_wait(bar(kAccEmpty + buf), (uint32_t)(((tcount >> 1) - 1) & 1), lim)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(buf * kBN);
         for (int ks = 0; ks < g.k_steps; ++ks, ++it) {
           const int st = (int)(it % kStages);
           if (!mbar_wait(bar(kFull + st), (uint32_t)((it / kStages) & 1), lim)) {
@@ -277,15 +273,28 @@ __global__ void __launch_bounds__(kThreadsG, 1)
           }
           tc_fence_after();
           const uint32_t a_s = sbase + st * kStageBytes, b_s = a_s + kABytes;
-          const uint64_t ad = sw128_desc(a_s, 16), bd = sw128_desc(b_s, kBAtom);
+          const uint64_t bd = sw128_desc(b_s, kBAtom);
           // K steps of 16: A advances 32 bytes inside its 128-byte rows, B 16 rows of 128 bytes.
-          const uint64_t a4[4] = {ad, ad + 2, ad + 4, ad + 6};
           const uint64_t b4[4] = {bd, bd + 128, bd + 256, bd + 384};
-          mma4(d, kIdesc, a4, b4, ks > 0 ? 1u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            // A half's first products of a tile wait until the epilogue has read that half of
+            // the previous tile.
+            if (ks == 0 && tcount > 0) {
+              if (!mbar_wait(bar(kAccEmpty + h), (uint32_t)((tcount - 1) & 1), lim)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            const uint64_t ad = sw128_desc(a_s + h * kAHalf, 16);
+            const uint64_t a4[4] = {ad, ad + 2, ad + 4, ad + 6};
+            mma4(tmem + (uint32_t)(h * kBN), kIdesc, a4, b4, ks > 0 ? 1u : 0u);
+          }
+          if (!ok) break;
           tc_commit(bar(kEmpty + st));
         }
         if (!ok) break;
-        tc_commit(bar(kAccFull + buf));
+        tc_commit(bar(kAccFull));
       }
       // Drain: every product issued above completes before TMEM is freed.
       tc_commit(bar(kDrainBar));
@@ -300,67 +309,68 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     for (long long t = blockIdx.x; ok && t < g.tiles; t += gridDim.x, ++tcount) {
       int tm, tn;
       tile_coords(g, t, tm, tn);
-      const int buf = tcount & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(kAccFull + buf), (uint32_t)((tcount >> 1) & 1), lim))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kAccFull), (uint32_t)(tcount & 1), lim))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const long long grow = (long long)tm * kBM + row;
-      const bool in_row = grow < g.m;
-      uint16_t *crow = g.c + grow * g.n + (long long)tn * kBN;
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * kBN);
+      for (int h = 0; h < 2; ++h) {
+        const long long grow = (long long)tm * kBM + h * kHalf + row;
+        const bool in_row = grow < g.m;
+        uint16_t *crow = g.c + grow * g.n + (long long)tn * kBN;
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(h * kBN);
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(taddr + c0, v);
-        const int col = tn * kBN + c0;
-        uint32_t ow[16];  // the old C values of the chunk as bf16 pairs (accumulating)
-        const bool full = in_row && col + 32 <= g.n;
-        if (g.accumulate && full) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(crow + c0);
+        for (int c0 = 0; c0 < kBN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c0, v);
+          const int col = tn * kBN + c0;
+          uint32_t ow[16];  // the old C values of the chunk as bf16 pairs (accumulating)
+          const bool full = in_row && col + 32 <= g.n;
+          if (g.accumulate && full) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(crow + c0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 o4 = src[q];
-            ow[4 * q] = o4.x;
-            ow[4 * q + 1] = o4.y;
-            ow[4 * q + 2] = o4.z;
-            ow[4 * q + 3] = o4.w;
-          }
-        }
-        tmem_wait_ld(v);
-        if (full) {
-          uint4 outv[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float lo = __uint_as_float(v[q * 8 + 2 * e]), hi = __uint_as_float(v[q * 8 + 2 * e + 1]);
-              if (g.accumulate) {
-                lo += __uint_as_float(ow[4 * q + e] << 16);
-                hi += __uint_as_float(ow[4 * q + e] & 0xffff0000u);
-              }
-              w[e] = pack_bf16(lo, hi);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 o4 = src[q];
+              ow[4 * q] = o4.x;
+              ow[4 * q + 1] = o4.y;
+              ow[4 * q + 2] = o4.z;
+              ow[4 * q + 3] = o4.w;
             }
-            outv[q] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          uint4 *dst = reinterpret_cast<uint4 *>(crow + c0);
+          tmem_wait_ld(v);
+          if (full) {
+            uint4 outv[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = outv[q];
-        } else if (in_row) {
-          // Ragged column tail: element by element.
-          for (int e = 0; e < 32 && col + e < g.n; ++e) {
-            float x = __uint_as_float(v[e]);
-            if (g.accumulate) x += __uint_as_float((uint32_t)crow[c0 + e] << 16);
-            crow[c0 + e] = (uint16_t)(pack_bf16(x, 0.f) & 0xffffu);
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float lo = __uint_as_float(v[q * 8 + 2 * e]), hi = __uint_as_float(v[q * 8 + 2 * e + 1]);
+                if (g.accumulate) {
+                  lo += __uint_as_float(ow[4 * q + e] << 16);
+                  hi += __uint_as_float(ow[4 * q + e] & 0xffff0000u);
+                }
+                w[e] = pack_bf16(lo, hi);
+              }
+              outv[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(crow + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = outv[q];
+          } else if (in_row) {
+            // Ragged column tail: element by element.
+            for (int e = 0; e < 32 && col + e < g.n; ++e) {
+              float x = __uint_as_float(v[e]);
+              if (g.accumulate) x += __uint_as_float((uint32_t)crow[c0 + e] << 16);
+              crow[c0 + e] = (uint16_t)(pack_bf16(x, 0.f) & 0xffffu);
+            }
           }
         }
+        // This warp has read its lanes of this half's accumulator: the issuer may reuse it.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kAccEmpty + h));
       }
-      // This warp has read its lanes of the accumulator: the issuer may reuse it.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kAccEmpty + buf));
     }
   }
   __syncthreads();
