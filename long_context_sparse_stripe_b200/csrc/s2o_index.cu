@@ -171,8 +171,22 @@ __global__ void __launch_bounds__(256)
   float acc = 0.f;
   for (int c0 = 0; c0 < n_chunks; c0 += kStage) {
     const int n = min(kStage, n_chunks - c0);
-    for (int x = threadIdx.x; x < n * 8; x += blockDim.x)
-      stage4[x] = __ldg(reinterpret_cast<const float4 *>(base + (size_t)(c0 + x / 8) * D) + x % 8);
+    // Eight loads in flight per thread before their stores (a load-store loop would wait for
+    // each load in turn).
+    for (int x0 = threadIdx.x; x0 < n * 8; x0 += 8 * blockDim.x) {
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int x = x0 + i * blockDim.x;
+        if (x < n * 8)
+          v[i] = __ldg(reinterpret_cast<const float4 *>(base + (size_t)(c0 + x / 8) * D) + x % 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int x = x0 + i * blockDim.x;
+        if (x < n * 8) stage4[x] = v[i];
+      }
+    }
     __syncthreads();
     if (threadIdx.x < 32) {
       int c = 0;
@@ -521,10 +535,16 @@ __global__ void __launch_bounds__(kRadixThreads)
   const int n = (int)min((long long)kRadixTile, run_len - (long long)tile * kRadixTile);
   for (int d = threadIdx.x; d < 256; d += blockDim.x) h[d] = 0;
   __syncthreads();
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const uint32_t k = score ? desc_key(__ldg(score + base + e)) : __ldg(keys + base + e);
-    atomicAdd(&h[(k >> shift) & 255u], 1);
+  // All of a thread's keys are loaded before they are counted (kRadixR loads in flight).
+  uint32_t kv[kRadixR];
+#pragma unroll
+  for (int r = 0; r < kRadixR; ++r) {
+    const int e = r * kRadixThreads + (int)threadIdx.x;
+    kv[r] = e < n ? (score ? desc_key(__ldg(score + base + e)) : __ldg(keys + base + e)) : 0u;
   }
+#pragma unroll
+  for (int r = 0; r < kRadixR; ++r)
+    if (r * kRadixThreads + (int)threadIdx.x < n) atomicAdd(&h[(kv[r] >> shift) & 255u], 1);
   __syncthreads();
   for (int d = threadIdx.x; d < 256; d += blockDim.x)
     counts[(run * 256 + d) * tiles + tile] = h[d];
