@@ -1494,8 +1494,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit();
           }
         }
-      } else if (store_row) {
-        // The whole row of O from TMEM (one wait), then 32-byte stores (full sectors).
+      } else {
+        // The whole row of O from TMEM (one wait), then 32-byte stores (full sectors). Every
+        // thread of the warp takes part in the loads (they are warp-collective); only the rows
+        // this pass writes are stored (a row of the merge path's permuted pass with no visible
+        // key is not).
         uint32_t o[D];
 #pragma unroll
         for (int c0 = 0; c0 < D / 32; ++c0)
@@ -1503,7 +1506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c0 = 0; c0 < D / 32; ++c0) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&o[c0 * 32]));
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; store_row && c < D / 16; ++c) {
           uint32_t w[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q)

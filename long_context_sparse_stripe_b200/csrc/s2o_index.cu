@@ -481,6 +481,143 @@ __global__ void __launch_bounds__(512)
   (void)n;
 }
 
+// Step 2b fused per (query head, segment), one CTA of 256 threads: rho_i = DOT(q_i, u_h) for the
+// segment's rows (also stored), their segment-local order (perm_q) and the means Qbar of the
+// ordered query blocks. The arithmetic is k_rho's, k_segment_sort's and k_block_means's step for step; fused,
+// the segment's rows come from HBM once (for rho) and the block means read them again from L2
+// right after the ordering, where three launches read Q twice. Two groups of 128 threads stage
+// chunks of 128 contiguous rows with asynchronous copies (rows padded by 16 bytes) and take one
+// row per thread; the ordering is k_segment_sort's four counting passes over R keys per thread;
+// then each warp forms the means of every eighth block of the segment.
+constexpr int kFuseThreads = 256;
+template <int D>
+constexpr size_t fused_order_smem(int R) {
+  return (size_t)(kFuseThreads / 128) * 128 * (D * 2 + 16) + D * 4 +
+         (size_t)2 * kFuseThreads * R * 4 + (size_t)(kFuseThreads / 32) * 256 * 4 + 256 * 4;
+}
+__device__ __forceinline__ void group_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+template <int D, int R>
+__global__ void __launch_bounds__(kFuseThreads, 2)
+    k_rho_order_means(const uint16_t *__restrict__ q, const float *__restrict__ u,
+                      float *__restrict__ rho, int32_t *__restrict__ perm_q,
+                      float *__restrict__ qbar, int N, int S, int B, int nB) {
+  constexpr int NT = kFuseThreads, NW = NT / 32, NG = NT / 128, RS = D * 2 + 16;
+  constexpr int CPL = D / 32;  // block-mean columns per lane (4 or 2)
+  using Vec = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
+  extern __shared__ __align__(16) unsigned char smem_f[];
+  float4 *us4 = reinterpret_cast<float4 *>(smem_f + NG * 128 * RS);  // [D/4]
+  uint32_t *skey = reinterpret_cast<uint32_t *>(us4 + D / 4);       // [NT·R]
+  uint32_t *sval = skey + NT * R;                                    // [NT·R]
+  int *hist = reinterpret_cast<int *>(sval + NT * R);                // [NW·256]
+  int *dbase = hist + NW * 256;                                      // [256]
+  const long long qh = blockIdx.y;
+  const int s0 = blockIdx.x * S;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x < D / 4)
+    us4[threadIdx.x] = reinterpret_cast<const float4 *>(u + qh * D)[threadIdx.x];
+  __syncthreads();
+  // rho: group g stages chunks g, g + NG, ... of the segment (named barrier 1 + g).
+  {
+    const int g = threadIdx.x / 128, t = threadIdx.x % 128;
+    unsigned char *stage = smem_f + g * 128 * RS;
+    const unsigned char *seg =
+        reinterpret_cast<const unsigned char *>(q + ((size_t)qh * N + s0) * D);
+    for (int c = g; c * 128 < S; c += NG) {
+      const int nrows = min(128, S - c * 128);
+      const unsigned char *src = seg + (size_t)c * 128 * D * 2;
+      for (int x = t; x < nrows * (D / 8); x += 128)
+        cp_async16(stage + (x / (D / 8)) * RS + (x % (D / 8)) * 16, src + (size_t)x * 16);
+      cp_async_wait_all();
+      group_sync(1 + g, 128);
+      if (t < nrows) {
+        uint4 v[D / 8];
+#pragma unroll
+        for (int c2 = 0; c2 < D / 8; ++c2)
+          v[c2] = *reinterpret_cast<const uint4 *>(stage + t * RS + c2 * 16);
+        const float r_i = dot_regs<D>(v, us4);
+        rho[qh * N + s0 + c * 128 + t] = r_i;  // kept in the workspace (an intermediate)
+        skey[c * 128 + t] = desc_key(r_i);
+      }
+      group_sync(1 + g, 128);  // the stage may be refilled
+    }
+  }
+  __syncthreads();
+  // perm_q: stable descending order of rho inside the segment (as k_segment_sort).
+  uint32_t key[R], val[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = warp * 32 * R + r * 32 + lane;
+    key[r] = e < S ? skey[e] : 0xffffffffu;
+    val[r] = (uint32_t)e;
+  }
+  for (int pass = 0; pass < 4; ++pass) {
+    uint32_t dig[R];
+    int dest[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) dig[r] = (key[r] >> (8 * pass)) & 255u;
+    radix_ranks<R, NW>(dig, dest, hist, dbase);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      skey[dest[r]] = key[r];
+      sval[dest[r]] = val[r];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = warp * 32 * R + r * 32 + lane;
+      key[r] = skey[e];
+      val[r] = sval[e];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = warp * 32 * R + r * 32 + lane;
+    if (e < S) perm_q[qh * N + s0 + e] = s0 + (int32_t)val[r];
+  }
+  // Qbar of the segment's ordered blocks (sval holds the order): as k_block_means, one warp per
+  // block, the rows (from L2) added in slot order.
+  const Vec *base = reinterpret_cast<const Vec *>(q + (size_t)qh * N * D) + lane;
+  for (int bl = warp; bl * B < S; bl += NW) {
+    const uint32_t *pp = sval + bl * B;
+    float acc[CPL];
+#pragma unroll
+    for (int x = 0; x < CPL; ++x) acc[x] = 0.f;
+    for (int e0 = 0; e0 < B; e0 += 32) {
+      const int my_row = s0 + (int)pp[e0 + lane];
+#pragma unroll
+      for (int h = 0; h < 32; h += 16) {
+        Vec v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int row = __shfl_sync(0xffffffffu, my_row, h + e);
+          v[e] = __ldg(base + (size_t)row * (D / CPL));
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          if constexpr (CPL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(&v[e]);
+            acc[0] = __fadd_rn(acc[0], bf16_lo(w.x));
+            acc[1] = __fadd_rn(acc[1], bf16_hi(w.x));
+            acc[2] = __fadd_rn(acc[2], bf16_lo(w.y));
+            acc[3] = __fadd_rn(acc[3], bf16_hi(w.y));
+          } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(&v[e]);
+            acc[0] = __fadd_rn(acc[0], bf16_lo(w));
+            acc[1] = __fadd_rn(acc[1], bf16_hi(w));
+          }
+        }
+      }
+    }
+    const float len = (float)B;
+    float *dst = qbar + ((size_t)qh * nB + s0 / B + bl) * D + lane * CPL;
+#pragma unroll
+    for (int x = 0; x < CPL; ++x) dst[x] = __fdiv_rn(acc[x], len);
+  }
+}
+
 // Copies the first row of each group of G rows (row_len int32, a multiple of 4, 16-byte aligned
 // rows) to the group's other G - 1 rows. Grid: (any, groups).
 __global__ void k_replicate_group_rows(int32_t *__restrict__ a, long long row_len, int G) {
@@ -1437,33 +1574,55 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   note_launch();
   // Step 2b: query scores, segment-local query ordering, query block means.
   const int qp = cfg.query_perm ? 1 : 0;
-  k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
-  note_launch();
   const dim3 seg_grid((unsigned)d.nSeg, (unsigned)bhq);
-  if (d.S <= 4096 || !qp) {
-    auto seg = [&](auto kernel, int R) -> cudaError_t {
-      const size_t smem = (size_t)2 * 512 * R * 4 + 16 * 256 * 4 + 256 * 4;
+  if (qp && d.S <= 16 * kFuseThreads) {
+    // One fused launch per (query head, segment).
+    auto fused = [&](auto kernel, int R) -> cudaError_t {
+      const size_t smem = fused_order_smem<D>(R);
       cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
       if (err != cudaSuccess) return err;
-      kernel<<<seg_grid, 512, smem, st>>>(rho, out.perm_q, d.N, d.S, qp);
+      kernel<<<seg_grid, kFuseThreads, smem, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
+                                                   d.nB);
       return cudaSuccess;
     };
-    if ((e = d.S <= 512    ? seg(k_segment_sort<1>, 1)
-             : d.S <= 1024 ? seg(k_segment_sort<2>, 2)
-             : d.S <= 2048 ? seg(k_segment_sort<4>, 4)
-                           : seg(k_segment_sort<8>, 8)) != cudaSuccess)
+    if ((e = d.S <= 256    ? fused(k_rho_order_means<D, 1>, 1)
+             : d.S <= 512  ? fused(k_rho_order_means<D, 2>, 2)
+             : d.S <= 1024 ? fused(k_rho_order_means<D, 4>, 4)
+             : d.S <= 2048 ? fused(k_rho_order_means<D, 8>, 8)
+                           : fused(k_rho_order_means<D, 16>, 16)) != cudaSuccess)
       return e;
     note_launch();
   } else {
-    // Segments longer than one CTA's sort: the multi-CTA radix sort over runs of S.
-    if ((e = radix_sort_runs(rho, rk0, rv0, rk1, rv1, rcount, nq, d.S, d.N, out.perm_q, st)) !=
-        cudaSuccess)
-      return e;
+    if (qp) {
+      k_rho<D><<<dim3((d.N + 127) / 128, (unsigned)bhq), 128, 0, st>>>(q, u, rho, d.N);
+      note_launch();
+    }
+    if (d.S <= 4096 || !qp) {
+      auto seg = [&](auto kernel, int R) -> cudaError_t {
+        const size_t smem = (size_t)2 * 512 * R * 4 + 16 * 256 * 4 + 256 * 4;
+        cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+        if (err != cudaSuccess) return err;
+        kernel<<<seg_grid, 512, smem, st>>>(rho, out.perm_q, d.N, d.S, qp);
+        return cudaSuccess;
+      };
+      if ((e = d.S <= 512    ? seg(k_segment_sort<1>, 1)
+               : d.S <= 1024 ? seg(k_segment_sort<2>, 2)
+               : d.S <= 2048 ? seg(k_segment_sort<4>, 4)
+                             : seg(k_segment_sort<8>, 8)) != cudaSuccess)
+        return e;
+      note_launch();
+    } else {
+      // Segments longer than one CTA's sort: the multi-CTA radix sort over runs of S.
+      if ((e = radix_sort_runs(rho, rk0, rv0, rk1, rv1, rcount, nq, d.S, d.N, out.perm_q, st)) !=
+          cudaSuccess)
+        return e;
+    }
+    k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
+                                                          nblk, d.Hq, d.Hkv, d.G, 0);
+    note_launch();
   }
-  k_block_means<D><<<blocks_for(nblk, 8), 256, 0, st>>>(q, out.perm_q, Qbar, d.N, d.B, d.nB,
-                                                        nblk, d.Hq, d.Hkv, d.G, 0);
-  note_launch();
   // Block scores (after the key side joins).
   if ((e = join.now()) != cudaSuccess) return e;
   const float sigma = D == 64 ? 0x1p-3f : 0x1.6a09e6p-4f;  // nearest fp32 to 1/sqrt(D)
