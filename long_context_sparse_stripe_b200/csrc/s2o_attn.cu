@@ -752,17 +752,23 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 // Fills the work list for window k0 of this CTA's share (warp 0; returns the entry count, or -1
-// past the end of the share). Without skipping, the share is the work items w = blockIdx.x +
-// k·gridDim.x, each contributing its units 2w and 2w+1 (adjacent units, which usually share
-// local tiles); with skip_empty (list streams) it is the units u = blockIdx.x + k·gridDim.x whose
-// selected list is not empty, paired in list order. Packed streams: the share is the pairs
-// w = blockIdx.x + k·gridDim.x that have a tile, each pair index at an even list position.
+// past the end of the share). Without skipping, the share is one work item per round k of
+// gridDim.x consecutive items, each contributing its units 2w and 2w+1 (adjacent units, which
+// usually share local tiles): w = k·gridDim.x + blockIdx.x, and in the local pass, in odd rounds,
+// w = k·gridDim.x + (gridDim.x − 1 − blockIdx.x). A round spans a few segments whose items repeat
+// the lengths 1..S/B, and a plain round robin with gridDim.x = 148 and 16 blocks per segment hands
+// a CTA only even or only odd block indices (units of 8 against 9 tiles on average); reversing
+// every other round gives each CTA both. With skip_empty (list streams) the share is the units
+// u = blockIdx.x + k·gridDim.x whose selected list is not empty, paired in list order. Packed
+// streams: the share is the pairs w = blockIdx.x + k·gridDim.x that have a tile, each pair index
+// at an even list position.
 template <int BN, int KIND>
 __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lane) {
   constexpr bool PACKED = KIND == kKindPacked;
   const bool by_unit = p.skip_empty && !PACKED;
   const long long span = by_unit ? kList : kList / 2;
-  const long long first = blockIdx.x + k0 * gridDim.x;
+  const bool snake = !by_unit && !PACKED && p.mode == kLocal;
+  const long long first = snake ? k0 * gridDim.x : blockIdx.x + k0 * gridDim.x;
   if (first >= (by_unit ? p.n_units : p.n_items)) return -1;
   // Whether unit u (list-stream order) has a non-empty selected list.
   auto busy = [&](long long u) -> bool {
@@ -780,7 +786,9 @@ __device__ int build_list(const Params &p, long long k0, uint32_t *list, int lan
   };
   int n = 0;
   for (long long k = k0; k < k0 + span; k += 32) {
-    const long long pos = blockIdx.x + (k + lane) * gridDim.x;
+    const long long round = k + lane;
+    const long long pos = round * gridDim.x +
+                          (snake && (round & 1) ? gridDim.x - 1 - blockIdx.x : blockIdx.x);
     if (by_unit) {
       const bool keep = busy(pos);
       const unsigned m = __ballot_sync(0xffffffffu, keep);
