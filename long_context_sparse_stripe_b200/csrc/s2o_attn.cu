@@ -22,11 +22,13 @@
 // key/value tiles: the local tiles once for both when they share them, then the two selected
 // lists interleaved. The grid is persistent (one CTA per SM); each CTA walks windows of a work
 // list that warp 0 fills between two CTA-wide barriers (the permuted pass lists only units with
-// selected blocks). When most blocks are selected, a decision kernel may have copied K and V
-// into key order (the permuted pass then loads selected blocks as tiles of the copy) and built
-// block bitmaps (bitmap streams: two consecutive blocks of one query head walk the union of
-// their selections in block order, loading a shared block once). The contiguous modes and the
-// two forms of the permuted pass are separate instantiations of the kernel.
+// selected blocks). With a workspace, a decision kernel picks the path on the device: when many
+// query blocks are busy, the permuted pass runs only the selected blocks and leaves partial rows
+// that the local pass merges (the merge path); when most blocks are selected, K and V are first
+// copied into key order, each block's rows by position, and the permuted pass streams only the
+// visible rows of a pair of units' selected blocks in 16-row chunks of the copy, a block both
+// units selected loaded once (packed streams). The contiguous modes, the forms of the permuted
+// pass and the merging local pass are separate instantiations of the kernel.
 //
 // Warp roles (384 threads):
 //   warps 0, 11 K and V producers: K (warp 0) and V (warp 11) tiles of the stream into two rings
