@@ -42,8 +42,8 @@ WORKLOAD = "llama-128k"
 # that kernel (dram__bytes_read.sum + dram__bytes_write.sum on llama-32k, scaled by the tile count
 # to llama-128k). Valid only for the kernel source it was taken on: reported as null once
 # s2o_attn.cu changes.
-ATTN_TRAFFIC = {"src_sha256_16": "75573d0d5e71199f", "workload": "llama-128k",
-                "bytes_per_launch": (405.674240e6 + 235.413504e6) * 4}
+ATTN_TRAFFIC = {"src_sha256_16": "0eeeddd21e4b9762", "workload": "llama-128k",
+                "bytes_per_launch": (403.441408e6 + 232.880128e6) * 4}
 
 
 def attention_traffic(workload):

@@ -489,21 +489,22 @@ __global__ void __launch_bounds__(512)
 // chunks of 128 contiguous rows with asynchronous copies (rows padded by 16 bytes) and take one
 // row per thread; the ordering is k_segment_sort's four counting passes over R keys per thread;
 // then each warp forms the means of every eighth block of the segment.
-constexpr int kFuseThreads = 256;
-template <int D>
+// Threads of k_rho_order_means (two CTAs per SM; 512 threads and one CTA per SM measured the same).
+constexpr int kFuseNT = 256;
+template <int D, int NT>
 constexpr size_t fused_order_smem(int R) {
-  return (size_t)(kFuseThreads / 128) * 128 * (D * 2 + 16) + D * 4 +
-         (size_t)2 * kFuseThreads * R * 4 + (size_t)(kFuseThreads / 32) * 256 * 4 + 256 * 4;
+  return (size_t)(NT / 128) * 128 * (D * 2 + 16) + D * 4 + (size_t)2 * NT * R * 4 +
+         (size_t)(NT / 32) * 256 * 4 + 256 * 4;
 }
 __device__ __forceinline__ void group_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
-template <int D, int R>
-__global__ void __launch_bounds__(kFuseThreads, 2)
+template <int D, int R, int NT>
+__global__ void __launch_bounds__(NT, NT == 256 ? 2 : 1)
     k_rho_order_means(const uint16_t *__restrict__ q, const float *__restrict__ u,
                       float *__restrict__ rho, int32_t *__restrict__ perm_q,
                       float *__restrict__ qbar, int N, int S, int B, int nB) {
-  constexpr int NT = kFuseThreads, NW = NT / 32, NG = NT / 128, RS = D * 2 + 16;
+  constexpr int NW = NT / 32, NG = NT / 128, RS = D * 2 + 16;
   constexpr int CPL = D / 32;  // block-mean columns per lane (4 or 2)
   using Vec = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
   extern __shared__ __align__(16) unsigned char smem_f[];
@@ -880,8 +881,9 @@ __global__ void __launch_bounds__(256)
 // r[qh][b][c] = DOT(Qbar_b, Kbar_c) × σ_d: a register-tiled fp32 product whose accumulators
 // each run the definition's sequential FMA chain over t = 0..D-1. A 128×128 tile per CTA, 8×8
 // accumulators per thread (paired FMAs); the operands go through shared memory transposed, 32
-// values of t at a time, and the next 32 are loaded into registers while the current ones are
-// consumed.
+// values of t at a time. Two CTAs per SM overlap one's operand loads with the other's products
+// (loading the next 32 values during the products instead measured slower: at 128 registers the
+// extra live operands spill).
 template <int D>
 __global__ void __launch_bounds__(256, 2)
     k_block_scores(const float *__restrict__ Qbar, const float *__restrict__ Kbar,
@@ -1575,22 +1577,21 @@ cudaError_t build_d(const Dims &d, const s2o_config &cfg, const uint16_t *q, con
   // Step 2b: query scores, segment-local query ordering, query block means.
   const int qp = cfg.query_perm ? 1 : 0;
   const dim3 seg_grid((unsigned)d.nSeg, (unsigned)bhq);
-  if (qp && d.S <= 16 * kFuseThreads) {
+  if (qp && d.S <= 16 * kFuseNT) {
     // One fused launch per (query head, segment).
     auto fused = [&](auto kernel, int R) -> cudaError_t {
-      const size_t smem = fused_order_smem<D>(R);
+      const size_t smem = fused_order_smem<D, kFuseNT>(R);
       cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
       if (err != cudaSuccess) return err;
-      kernel<<<seg_grid, kFuseThreads, smem, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B,
-                                                   d.nB);
+      kernel<<<seg_grid, kFuseNT, smem, st>>>(q, u, rho, out.perm_q, Qbar, d.N, d.S, d.B, d.nB);
       return cudaSuccess;
     };
-    if ((e = d.S <= 256    ? fused(k_rho_order_means<D, 1>, 1)
-             : d.S <= 512  ? fused(k_rho_order_means<D, 2>, 2)
-             : d.S <= 1024 ? fused(k_rho_order_means<D, 4>, 4)
-             : d.S <= 2048 ? fused(k_rho_order_means<D, 8>, 8)
-                           : fused(k_rho_order_means<D, 16>, 16)) != cudaSuccess)
+    if ((e = d.S <= kFuseNT       ? fused(k_rho_order_means<D, 1, kFuseNT>, 1)
+             : d.S <= 2 * kFuseNT ? fused(k_rho_order_means<D, 2, kFuseNT>, 2)
+             : d.S <= 4 * kFuseNT ? fused(k_rho_order_means<D, 4, kFuseNT>, 4)
+             : d.S <= 8 * kFuseNT ? fused(k_rho_order_means<D, 8, kFuseNT>, 8)
+                                  : fused(k_rho_order_means<D, 16, kFuseNT>, 16)) != cudaSuccess)
       return e;
     note_launch();
   } else {
