@@ -318,7 +318,8 @@ s2o_status s2o_layer_prefill(const s2o_config *cfg, const s2o_layer_config *lc,
 /* The decoder layer's projections: C[m, n] = A[m, k] · B[k, n] (+ C[m, n] when accumulate = 1),
  * A, B and C row-major bf16 on the device (16-byte aligned, owned by the caller), the products
  * accumulated in fp32 and the result (with the old C when accumulating) rounded to bf16 once.
- * A tcgen05 kernel (M = 128, N = 256 tiles, TMEM accumulators, TMA loads); no counterpart on the
+ * tcgen05 kernels (256 × 256 tiles, TMEM accumulators, TMA loads; for n and k up to 8192 on pairs
+ * of SMs, tcgen05 cta_group::2, launched as clusters of two CTAs); no counterpart on the
  * pages beyond the model they run the attention in ([S2O, Key points]: Llama-3.1-8B).
  * n and k must be multiples of 8 (S2O_ERR_UNSUPPORTED otherwise); any m. Every wait inside is
  * bounded like the attention kernel's (s2o_set_wait_limit_ns, reported by

@@ -3,8 +3,9 @@
 // S2O card's Key points: Llama-3.1-8B at 128K).
 //
 // C[m, n] = A[m, k] · B[k, n] (+ C[m, n] when accumulating), all row-major bf16, the sum in fp32
-// and rounded to bf16 once (the residual adds into the same rounding). One persistent CTA per SM,
-// 192 threads, 256 × 256 output tiles:
+// and rounded to bf16 once (the residual adds into the same rounding). Two kernels; the call takes
+// the CTA-pair kernel further below for n and k up to 8192, this one otherwise (and for a single
+// tile). One persistent CTA per SM, 192 threads, 256 × 256 output tiles:
 //   warp 0      TMA producer: per K step of 64, the A tile (256 rows × 64, K-major, one 128-byte
 //               swizzled box) and the B tile (64 × 256, N-major: four {64, 64} boxes, one per
 //               64-column atom) into a 3-stage ring.
@@ -382,6 +383,319 @@ __global__ void __launch_bounds__(kThreadsG, 1)
   }
 }
 
+// ------------------------------------------------------------------ the CTA-pair kernel
+//
+// The same product on pairs of SMs (a cluster of two CTAs, tcgen05 cta_group::2): a pair computes
+// 256 × 256 output tiles with M = 256, N = 256 products; CTA r of the pair holds rows 128r..128r+127
+// of the A tile and columns 128r..128r+127 of the B tile in its shared memory (the tensor core reads
+// both CTAs' halves), and accumulates its 128 rows × 256 columns in its own TMEM. Each CTA loads
+// 32 KB per K step of 64 (131 FLOP per byte, as the single-CTA tile), and the accumulator takes 256
+// of the 512 TMEM columns, so two alternate: the epilogue of one tile overlaps the next tile's
+// products. Roles per CTA (192 threads): warp 0 loads the CTA's halves (TMA, 128-byte swizzle,
+// no multicast) into a 6-stage ring; warp 1 of the first CTA (the leader) issues the products;
+// warps 2-5 run the epilogue of the CTA's rows. Between the two CTAs: the peer's tile loads
+// complete on the leader's stage barrier (the cta_group::2 form of the TMA load); the leader's
+// commits of a stage release and of a finished accumulator arrive on the barrier at the same
+// offset in both CTAs (the commit's cluster form; no load is multicast); every epilogue warp of
+// both CTAs releases an accumulator with a plain arrival on the leader's barrier. Every wait is
+// bounded by %globaltimer.
+constexpr int kPH = 128, kPNh = 128, kPStages = 6;
+constexpr uint32_t kPA = kPH * kBK * 2;         // 16 KB: this CTA's 128 rows of A
+constexpr uint32_t kPB = (kPNh / 64) * kBAtom;  // 16 KB: this CTA's 128 columns of B
+constexpr uint32_t kPStage = kPA + kPB;
+constexpr uint32_t kPOffBar = kPStages * kPStage;  // 192 KB of stages
+constexpr uint32_t kPSmem = kPOffBar + 256 + 1024;
+// Barrier slots: full[stages] (used on the leader), empty[stages], acc_full[2], acc_empty[2]
+// (leader), drain.
+constexpr int kPFull = 0, kPEmpty = kPStages, kPAccFull = 2 * kPStages,
+              kPAccEmpty = 2 * kPStages + 2, kPDrain = 2 * kPStages + 4, kPBars = 2 * kPStages + 5;
+static_assert(kPBars * 8 + 4 <= 256, "barrier area");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The address in CTA `rank` of the cluster of the shared-memory word at local address a.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// A wait that also orders with arrivals from the other CTA of the pair; false (recorded in the
+// error word) after limit_ns.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t a, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(&g_gemm_error, 1u);
+      return false;
+    }
+  }
+}
+// TMA tile load into this CTA's shared memory whose completion is counted on a barrier of either
+// CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *tm, int x, int y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// The same completion signalled on the barrier at this offset in both CTAs of the pair (a commit,
+// not a memory load).
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+// Four K = 16 products of one stage, M = 256 over the CTA pair; the first accumulates only if
+// `acc0` is set.
+__device__ __forceinline__ void mma4_pair(uint32_t d, uint32_t idesc, const uint64_t (&a)[4],
+                                          const uint64_t (&b)[4], uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t"
+      "setp.ne.b32 p0, %10, 0;\n\t"
+      "setp.eq.b32 p1, %0, %0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %2, %6, %1, p0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %3, %7, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %4, %8, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %5, %9, %1, p1;\n\t}\n" ::"r"(d),
+      "r"(idesc), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+      "l"(b[3]), "r"(acc0)
+      : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+__global__ void __launch_bounds__(kThreadsG, 1)
+    k_gemm_bf16_pair(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b, const GemmParams g) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem), sBar = sbase + kPOffBar;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kPOffBar + kPBars * 8);
+  auto bar = [&](int i) { return sBar + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const long long pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(bar(kPFull + s), 1);
+      mbar_init(bar(kPEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(kPAccFull + b), 1);
+      mbar_init(bar(kPAccEmpty + b), 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(bar(kPDrain), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    // Both CTAs of the pair allocate together (the same columns in each).
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = g.limit_ns;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA loads (both CTAs)
+    long long it = 0;
+    if (lane == 0) {
+      for (long long t = pair; ok && t < g.tiles; t += n_pairs) {
+        int tm, tn;
+        tile_coords(g, t, tm, tn);
+        for (int ks = 0; ks < g.k_steps; ++ks, ++it) {
+          const int st = (int)(it % kPStages);
+          if (it >= kPStages) {
+            if (!mbar_wait_cluster(bar(kPEmpty + st), (uint32_t)(((it / kPStages) - 1) & 1), lim)) {
+              ok = false;
+              break;
+            }
+          }
+          const uint32_t a_dst = sbase + st * kPStage, b_dst = a_dst + kPA;
+          const int row = tm * kBM + (int)rank * kPH, col = tn * kBN + (int)rank * kPNh;
+          if (leader) {
+            mbar_expect_tx(bar(kPFull + st), 2 * kPStage);  // both CTAs' halves
+            tma_load_2d(a_dst, &tm_a, ks * kBK, row, bar(kPFull + st));
+            for (int at = 0; at < kPNh / 64; ++at)
+              tma_load_2d(b_dst + at * kBAtom, &tm_b, col + at * 64, ks * kBK, bar(kPFull + st));
+          } else {
+            const uint32_t fb = map_to_cta(bar(kPFull + st), 0);
+            tma_load_2d_pair(a_dst, &tm_a, ks * kBK, row, fb);
+            for (int at = 0; at < kPNh / 64; ++at)
+              tma_load_2d_pair(b_dst + at * kBAtom, &tm_b, col + at * 64, ks * kBK, fb);
+          }
+        }
+      }
+      // Drain (leader): the last fill of each stage, both halves, lands before the pair exits.
+      if (leader)
+        for (int st = 0; st < kPStages; ++st) {
+          if (it <= st) continue;
+          const long long last = st + ((it - 1 - st) / kPStages) * kPStages;
+          mbar_wait_cluster(bar(kPFull + st), (uint32_t)((last / kPStages) & 1), kDrainNs);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t kIdesc = idesc_bf16(2 * kPH, kBN, 0, 1);
+      long long it = 0;
+      int tc = 0;
+      for (long long t = pair; ok && t < g.tiles; t += n_pairs, ++tc) {
+        const int b = tc & 1;
+        if (tc >= 2) {
+          if (!mbar_wait_cluster(bar(kPAccEmpty + b), (uint32_t)(((tc >> 1) - 1) & 1), lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const uint32_t d = tmem + (uint32_t)(b * kBN);
+        for (int ks = 0; ks < g.k_steps; ++ks, ++it) {
+          const int st = (int)(it % kPStages);
+          if (!mbar_wait_cluster(bar(kPFull + st), (uint32_t)((it / kPStages) & 1), lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_s = sbase + st * kPStage, b_s = a_s + kPA;
+          const uint64_t ad = sw128_desc(a_s, 16), bd = sw128_desc(b_s, kBAtom);
+          const uint64_t a4[4] = {ad, ad + 2, ad + 4, ad + 6};
+          const uint64_t b4[4] = {bd, bd + 128, bd + 256, bd + 384};
+          mma4_pair(d, kIdesc, a4, b4, ks > 0 ? 1u : 0u);
+          tc_commit_pair_both(bar(kPEmpty + st));  // frees the stage in both CTAs
+        }
+        if (!ok) break;
+        tc_commit_pair_both(bar(kPAccFull + b));  // both CTAs' epilogues
+      }
+      tc_commit_pair(bar(kPDrain));
+      mbar_wait_cluster(bar(kPDrain), 0, kDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t acc_empty_leader = map_to_cta(bar(kPAccEmpty), 0);
+    int tc = 0;
+    for (long long t = pair; ok && t < g.tiles; t += n_pairs, ++tc) {
+      const int b = tc & 1;
+      int tm, tn;
+      tile_coords(g, t, tm, tn);
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_cluster(bar(kPAccFull + b), (uint32_t)((tc >> 1) & 1), lim))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const long long grow = (long long)tm * kBM + (long long)rank * kPH + row;
+      const bool in_row = grow < g.m;
+      uint16_t *crow = g.c + grow * g.n + (long long)tn * kBN;
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * kBN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c0, v);
+        const int col = tn * kBN + c0;
+        uint32_t ow[16];
+        const bool full = in_row && col + 32 <= g.n;
+        if (g.accumulate && full) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(crow + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 o4 = src[q];
+            ow[4 * q] = o4.x;
+            ow[4 * q + 1] = o4.y;
+            ow[4 * q + 2] = o4.z;
+            ow[4 * q + 3] = o4.w;
+          }
+        }
+        tmem_wait_ld(v);
+        if (c0 + 32 == kBN) {
+          // The whole accumulator of this warp's lanes is read: release it to the issuer.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8u * (uint32_t)b);
+        }
+        if (full) {
+          uint4 outv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float lo = __uint_as_float(v[q * 8 + 2 * e]), hi = __uint_as_float(v[q * 8 + 2 * e + 1]);
+              if (g.accumulate) {
+                lo += __uint_as_float(ow[4 * q + e] << 16);
+                hi += __uint_as_float(ow[4 * q + e] & 0xffff0000u);
+              }
+              w[e] = pack_bf16(lo, hi);
+            }
+            outv[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(crow + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = outv[q];
+        } else if (in_row) {
+          for (int e = 0; e < 32 && col + e < g.n; ++e) {
+            float x = __uint_as_float(v[e]);
+            if (g.accumulate) x += __uint_as_float((uint32_t)crow[c0 + e] << 16);
+            crow[c0 + e] = (uint16_t)(pack_bf16(x, 0.f) & 0xffffu);
+          }
+        }
+      }
+    }
+  }
+  // Neither CTA leaves while the other may still signal its barriers or read its shared memory.
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static bool tried = false;
@@ -425,9 +739,7 @@ cudaError_t launch_gemm_bf16(const void *A, const void *B, void *C, long long m,
   if (m <= 0 || n <= 0 || k <= 0 || n % 8 || k % 8 || m >= (1ll << 31) || n >= (1ll << 31) ||
       k >= (1ll << 31))
     return cudaErrorInvalidValue;
-  static_assert(kSmem <= 232448, "shared memory budget");
-  CUtensorMap ta, tb;
-  if (!gemm_map(&ta, A, m, k, kBM) || !gemm_map(&tb, B, k, n, kBK)) return cudaErrorInvalidValue;
+  static_assert(kSmem <= 232448 && kPSmem <= 232448, "shared memory budget");
   GemmParams g;
   g.c = static_cast<uint16_t *>(C);
   g.m = (int)m;
@@ -439,9 +751,46 @@ cudaError_t launch_gemm_bf16(const void *A, const void *B, void *C, long long m,
   g.tiles = (long long)g.m_tiles * g.n_tiles;
   g.accumulate = accumulate ? 1 : 0;
   g.limit_ns = limit_ns;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmem);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  // The CTA pair measured faster for N and K up to 8192 (1.29-1.34 against 1.04-1.29 PFLOP/s at
+  // the decoder layer's q/k/v and output shapes); above that (N = 28672, K = 14336) its 74
+  // concurrent tiles span more row panels than L2 holds and the single-CTA kernel is faster.
+  if (n <= 8192 && k <= 8192 && g.tiles >= 2) {
+    CUtensorMap ta, tb;
+    if (!gemm_map(&ta, A, m, k, kPH) || !gemm_map(&tb, B, k, n, kBK)) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(k_gemm_bf16_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kPSmem)) != cudaSuccess)
+      return e;
+    // A persistent grid of CTA pairs: as many pairs as fit at once (one CTA per SM), at most one
+    // per tile.
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreadsG);
+    cfg.dynamicSmemBytes = kPSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)(2 * (gemm_sm_count() / 2)));
+    int max_pairs = 0;
+    if ((e = cudaOccupancyMaxActiveClusters(&max_pairs, k_gemm_bf16_pair, &cfg)) != cudaSuccess)
+      return e;
+    if (max_pairs <= 0) return cudaErrorLaunchOutOfResources;
+    const long long pairs = std::min<long long>(g.tiles, max_pairs);
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    e = cudaLaunchKernelEx(&cfg, k_gemm_bf16_pair, ta, tb, g);
+    note_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  CUtensorMap ta, tb;
+  if (!gemm_map(&ta, A, m, k, kBM) || !gemm_map(&tb, B, k, n, kBK)) return cudaErrorInvalidValue;
+  if ((e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmem)) != cudaSuccess)
+    return e;
   const long long grid = std::min<long long>(g.tiles, gemm_sm_count());
   k_gemm_bf16<<<(unsigned)grid, kThreadsG, kSmem, st>>>(ta, tb, g);
   note_launch();

@@ -1,7 +1,8 @@
 """The decoder layer's tensor-core GEMM (s2o_gemm_bf16, through the C ABI) against a plain PyTorch
 fp32 product of the same bf16 operands: C = bf16(A·B) or bf16(C + A·B), with full tiles, ragged
 edges in every dimension (m not a multiple of 128, n not of 256, k not of 64), and several tiles
-per CTA (a capped grid is not needed: 148 CTAs each take several tiles at these sizes)."""
+per CTA. Both kernels behind the call are covered: the CTA pair (n and k up to 8192, at least two
+256 × 256 tiles) and the single-CTA kernel (one tile, n above 8192, or k above 8192)."""
 import pytest
 import torch
 
@@ -18,7 +19,8 @@ def reference(a, b, c=None):
 
 
 @pytest.mark.parametrize("m,n,k", [(128, 256, 64), (256, 512, 128), (300, 520, 72),
-                                   (1000, 776, 200), (4096, 2048, 4096), (129, 8, 8)])
+                                   (1000, 776, 200), (4096, 2048, 4096), (129, 8, 8),
+                                   (520, 8200, 72), (300, 264, 8208)])
 @pytest.mark.parametrize("accumulate", [False, True])
 def test_gemm_matches_fp32_product(m, n, k, accumulate):
     g = torch.Generator(device="cuda").manual_seed(m * 7 + n * 3 + k)
