@@ -401,8 +401,10 @@ def run_s2o(args):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
                          "traffic": attention_traffic(args.workload),
-                         "kernel": "s2o_attention_kernel<128,128> (permuted pass + local pass "
-                                   "with merge)",
+                         "kernel": "s2o_attention_kernel<128,128> (" + (
+                             ("packed permuted pass + merging local pass" if work.packed else
+                              "gathered permuted pass + merging local pass") if work.merged else
+                             "local pass + permuted pass, the path without the merge") + ")",
                          "peak_source": f"{peak_kind} bf16 (burst)"},
             "e2e": {"value": whole_job_value(job_flops, 1, e2e_ms), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
