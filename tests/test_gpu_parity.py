@@ -37,6 +37,10 @@ W_F = gen.Workload("f-ragged-tiles", batch=1, n_q_heads=2, n_kv_heads=1, seq_len
 # One segment spanning the whole sequence (the local window is the causal triangle of all keys).
 W_G = gen.Workload("g-one-segment", batch=1, n_q_heads=2, n_kv_heads=2, seq_len=4096,
                    head_dim=128, segment_len=4096, block_size=128, tau=0.01, seed=12)
+# A segment that is not a whole number of 128-row chunks (320 = 2·128 + 64): the fused
+# ρ/order/Q̄ kernel stages a partial last chunk.
+W_H = gen.Workload("h-partial-chunk", batch=1, n_q_heads=2, n_kv_heads=1, seq_len=1920,
+                   head_dim=64, segment_len=320, block_size=64, tau=0.01, seed=15)
 W_TINY = gen.workload("tiny")
 
 INDEX_NAMES = ("perm_q", "perm_k", "sel_cnt", "local_tiles")
@@ -101,7 +105,7 @@ def test_exp64_bit_exact_with_oracle():
 
 @pytest.mark.parametrize("w", [
     W_TINY, W_TINY.replace(tau=0.0), W_TINY.replace(tau=0.07), W_TINY.replace(tau=0.2),
-    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E, W_F, W_G,
+    W_TINY.replace(tau=1.5), W_A, W_A.replace(query_perm=0), W_B, W_C, W_D, W_E, W_F, W_G, W_H,
     W_A.replace(shared_key_order=1), W_B.replace(shared_key_order=1),
     W_E.replace(shared_key_order=1),
     W_TINY.replace(int4_centroids=1), W_A.replace(int4_centroids=1), W_C.replace(int4_centroids=1),
@@ -132,7 +136,7 @@ def test_index_build_is_deterministic():
 # ----------------------------------------------------------------------------- attention
 
 @pytest.mark.parametrize("w", [W_TINY, W_TINY.replace(tau=0.07), W_TINY.replace(tau=1.5), W_A,
-                               W_A.replace(query_perm=0), W_C, W_D, W_F, W_G],
+                               W_A.replace(query_perm=0), W_C, W_D, W_F, W_G, W_H],
                          ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
 def test_attention_on_oracle_indices(w):
     q, k, v = inputs(w)
