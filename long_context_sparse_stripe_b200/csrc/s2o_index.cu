@@ -954,7 +954,8 @@ __global__ void __launch_bounds__(256, 2)
     const int b = b0 + tr * 8 + i;
     if (b >= nB) continue;
     float *dst = r + ((size_t)qh * nB + b) * nB + c0 + tc * 8;
-    if (c0 + tc * 8 + 8 <= nB) {
+    // 16-byte stores need 16-byte aligned rows, i.e. nB a multiple of 4 (N/B need not be).
+    if ((nB & 3) == 0 && c0 + tc * 8 + 8 <= nB) {
       reinterpret_cast<float4 *>(dst)[0] =
           make_float4(__fmul_rn(acc[i][0].x, sigma), __fmul_rn(acc[i][0].y, sigma),
                       __fmul_rn(acc[i][1].x, sigma), __fmul_rn(acc[i][1].y, sigma));
