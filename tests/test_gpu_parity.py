@@ -342,8 +342,8 @@ def _with_mode(mode, fn):
 
 
 @pytest.mark.parametrize("w", [W_A.replace(tau=0.0), W_C.replace(tau=0.0), W_D.replace(tau=0.0),
-                               W_F.replace(tau=0.0), W_A.replace(tau=0.01), W_S1, W_S2, W_S3,
-                               W_S3.replace(query_perm=0)],
+                               W_F.replace(tau=0.0), W_H.replace(tau=0.0), W_A.replace(tau=0.01),
+                               W_S1, W_S2, W_S3, W_S3.replace(query_perm=0)],
                          ids=lambda w: f"{w.name}-tau{w.tau}-qp{w.query_perm}")
 def test_merge_and_packed_paths_match_oracle(w):
     """On the oracle's indices, every form of steps 3-4 gives the oracle's output: the merge path
