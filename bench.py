@@ -339,26 +339,53 @@ def run_s2o(args):
     mse = float(((o.float() - od.float()) ** 2).mean().item())
     del od
 
-    # End to end through the public call with host buffers: pinned H2D of Q/K/V, the prefill,
-    # D2H of O, every step.
+    # End to end through the public call with host buffers: every step copies its Q/K/V from
+    # pinned host memory to the device, runs the prefill and reads O back, pipelined as a serving
+    # loop runs it: step k's inputs go up on one copy stream while step k-1 computes, and step k's
+    # output comes down on another while step k+1 computes (the two PCIe directions are
+    # independent); device inputs and outputs are double-buffered. The timed region holds every
+    # step's copies, the pipeline's fill and its drain.
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size()
+    ins = [(qd, kd, vd), tuple(torch.empty_like(t) for t in (qd, kd, vd))]
+    outs = [o, torch.empty_like(o)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    loaded, computed, read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    n_e2e = args.e2e_steps
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        s2o.attention_prefill(cfg, qd, kd, vd, out=o, idx=idx, ws=ws)
-        oh.copy_(o, non_blocking=True)
+    up.wait_stream(stream)
+    down.wait_stream(stream)
+    for step in range(n_e2e):
+        b = step % 2
+        with torch.cuda.stream(up):
+            if step >= 2:
+                up.wait_event(computed[b])  # step - 2 has finished reading these inputs
+            for dst, src in zip(ins[b], (qh, kh, vh)):
+                dst.copy_(src, non_blocking=True)
+            loaded[b].record(up)
+        stream.wait_event(loaded[b])
+        if step >= 2:
+            stream.wait_event(read[b])  # step - 2's output has been read back
+        qb, kb, vb = ins[b]
+        s2o.attention_prefill(cfg, qb, kb, vb, out=outs[b], idx=idx, ws=ws)
+        computed[b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            oh.copy_(outs[b], non_blocking=True)
+            read[b].record(down)
+    stream.wait_stream(up)
+    stream.wait_stream(down)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.e2e_steps, dev)
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / n_e2e, dev)
+    del ins, outs
     gather_ms = None
     if args.parallel == "heads" and dist is not None:
         # Assembling the whole O on every GPU, if a caller wants it: one NCCL all-gather of the
@@ -407,7 +434,10 @@ def run_s2o(args):
                              "local pass + permuted pass, the path without the merge") + ")",
                          "peak_source": f"{peak_kind} bf16 (burst)"},
             "e2e": {"value": whole_job_value(job_flops, 1, e2e_ms), "unit": UNIT,
-                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": n_e2e,
+                    "schedule": "pipelined: H2D of step k+1 and D2H of step k-1 overlap step k's "
+                                "prefill (double-buffered device inputs and outputs)"},
             "gpu_launches": launches,
             "o_all_gather_ms": gather_ms,
             "clocks": clocks.summary(),
@@ -728,7 +758,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(gen.WORKLOADS),
                     help="bench lines use the default; smaller workloads serve profiling")
     ap.add_argument("--dense-steps", type=int, default=2)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--ref-rows", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ws-mode", type=int, default=-1,
