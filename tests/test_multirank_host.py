@@ -70,3 +70,29 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
                                  ref_rows=16)
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_0(monkeypatch, capsys):
+    """The reference arm (the CPU oracle on a bounded sample) prints one JSON line with the GPU
+    arm's metric, unit and config keys, labels its extrapolation and describes its sample."""
+    import json
+
+    import bench
+    import gen
+    for var in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(var, raising=False)
+    args = types.SimpleNamespace(workload="tiny", tau=0.01, steps=1, warmup=0, gpus=1, ref_rows=16,
+                                 parallel="replica")
+    assert bench.run_reference(args) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 1
+    w = gen.workload("tiny", tau=0.01)
+    assert d["config"] == bench.workload_config("tiny", w, 1, "replica")
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
