@@ -483,9 +483,11 @@ __global__ void __launch_bounds__(512)
 
 // Step 2b fused per (query head, segment), one CTA of 256 threads: rho_i = DOT(q_i, u_h) for the
 // segment's rows (also stored), their segment-local order (perm_q) and the means Qbar of the
-// ordered query blocks. The arithmetic is k_rho's, k_segment_sort's and k_block_means's step for step; fused,
-// the segment's rows come from HBM once (for rho) and the block means read them again from L2
-// right after the ordering, where three launches read Q twice. Two groups of 128 threads stage
+// ordered query blocks. The arithmetic is k_rho's, k_segment_sort's and k_block_means's step for
+// step; fused, the segment's rows come from HBM once (for rho) and the block means read them
+// again right after the ordering, from L2 while the segment is still resident (with every SM's
+// two segments in flight at 128K tokens, about a third of those re-reads hit), where three
+// launches read Q twice and sort in between. Two groups of 128 threads stage
 // chunks of 128 contiguous rows with asynchronous copies (rows padded by 16 bytes) and take one
 // row per thread; the ordering is k_segment_sort's four counting passes over R keys per thread;
 // then each warp forms the means of every eighth block of the segment.
