@@ -92,6 +92,10 @@ def test_reference_arm_line_on_rank_0(monkeypatch, capsys):
     w = gen.workload("tiny", tau=0.01)
     assert d["config"] == bench.workload_config("tiny", w, 1, "replica")
     assert d["value"] > 0 and d["ms_per_step"] > 0
+    # A step is the sample itself; the layer's time is the labelled extrapolation of it.
+    assert d["layer_ms_extrapolated"] > 0 and "sample" in d["ms_per_step_kind"]
+    assert abs(d["value"] - w.dense_causal_flops / (d["layer_ms_extrapolated"] * 1e-3) / 1e12) \
+        <= 1e-9 * d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
