@@ -228,9 +228,10 @@ s2o_status s2o_validate_indices(const s2o_config *cfg, const s2o_indices *idx, v
 s2o_status s2o_index_stats(const s2o_config *cfg, const s2o_indices *idx, void *ws,
                            size_t ws_bytes, s2o_stats *stats, s2o_stream stream);
 
-/* Every wait inside the attention kernel (on a TMA copy, a tensor-core commit or a peer warp) is
- * bounded by this many nanoseconds of GPU time (default 2e9). When a wait runs out, the kernel
- * records it, drains its own copies and tensor-core work, frees its tensor memory and returns.
+/* Every wait inside the attention kernel and the GEMMs (on a TMA copy, a tensor-core commit, a
+ * peer warp or, in the CTA-pair GEMM, the other CTA of the pair) is bounded by this many
+ * nanoseconds of GPU time (default 2e9). When a wait runs out, the kernel records it, drains its
+ * own copies and tensor-core work, frees its tensor memory and returns.
  * Affects launches made after the call; not thread-safe against concurrent launches. */
 void s2o_set_wait_limit_ns(uint64_t ns);
 
