@@ -50,6 +50,28 @@ MUTATIONS = {
         "      for (int c = c0; c < c0 + 32 && c < nB; ++c)",
         "for (int c0 = 0; c0 < nB; c0 += nB) {\n      double part = 0.0;\n"
         "      for (int c = c0; c < c0 + nB && c < nB; ++c)"),
+    # Orderings ascending instead of descending (the shared comparator of both orderings).
+    "orderings-ascending": ("return a->key > b->key ? -1 : 1;", "return a->key < b->key ? -1 : 1;"),
+    # Selected blocks listed least important first.
+    "selection-ascending": ("if (a->p != b->p) return a->p > b->p ? -1 : 1;",
+                            "if (a->p != b->p) return a->p < b->p ? -1 : 1;"),
+    # A block whose score equals τ dropped (p > τ instead of p ≥ τ).
+    "selection-strict": ("if (ns[c] > 0 && p >= tau) {", "if (ns[c] > 0 && p > tau) {"),
+    # The query score without the mean key (rho = q·kbar_top).
+    "rho-drops-mean-key": ("u[t] = kbar_top[t] - kbar_all[t];", "u[t] = kbar_top[t];"),
+    # kbar_top pooled over the second-ranked key block instead of the top one.
+    "kbar-top-second-block": ("list_mean(K, d, perm_k, B, B, kbar_top);",
+                              "list_mean(K, d, perm_k + B, B, B, kbar_top);"),
+    # A selected block's key at the segment start let through (it is already a local key).
+    "selected-keys-le": ("if (j < s0) keys[nk++] = j;", "if (j <= s0) keys[nk++] = j;"),
+    # The segment-local query ordering never applied.
+    "query-order-skipped": (
+        "if (cfg->query_perm) qsort(tmp, (size_t)S, sizeof(keyed), cmp_keyed_desc);",
+        "if (0 && cfg->query_perm) qsort(tmp, (size_t)S, sizeof(keyed), cmp_keyed_desc);"),
+    # Query block means over original-order blocks instead of permuted ones.
+    "qbar-original-order": (
+        "list_mean(Q, d, perm_q + (size_t)b * B, B, B, Qbar + (size_t)b * d);",
+        "list_mean(Q, d, ident + (size_t)b * B, B, B, Qbar + (size_t)b * d);"),
 }
 
 # The pins that run against each mutant (all CPU, seconds each).
@@ -62,6 +84,7 @@ PIN_TESTS = [
              for w in (pins.gen.workload("tiny"), pins.SMALL_GQA)],
     lambda: [pins.test_tau_above_one_is_local_window_only(w)
              for w in (pins.gen.workload("tiny"), pins.SMALL_GQA)],
+    pins.test_threshold_is_inclusive,
     pins.test_index_arrays_are_sorted_permutations,
     pins.test_probabilities_and_selection_rule,
     pins.test_float64_rederivation_of_pooled_quantities,

@@ -221,6 +221,30 @@ def test_segment_zero_is_dense_for_any_tau():
                                    atol=1e-10)
 
 
+def test_threshold_is_inclusive():
+    """The stop keeps a block whose normalised score equals τ (p ≥ τ; "stops once a block's score
+    falls under τ", S2O card, Summary ¶2). Closed form: with every key the same vector, the key
+    scores tie and the stable ordering is the identity, so with S = 2B the first segment's keys
+    fill key blocks 0 and 1. A query block of the second segment then has exactly two candidate
+    blocks, each with B visible keys and the same centroid, so each has p = 1/2 exactly, whatever
+    the queries. At τ = 1/2 both are selected (ties by lower block id); at the next float above
+    1/2, none; query blocks of the first segment have no candidates."""
+    Bk, S, N, d = 4, 8, 16, 4
+    rng = np.random.default_rng(5)
+    q = torch.from_numpy(rng.standard_normal((1, 1, N, d), dtype=np.float32)).to(torch.bfloat16)
+    k = torch.tensor([1.0, -0.5, 0.25, 2.0]).repeat(1, 1, N, 1).to(torch.bfloat16)
+    c = dict(batch=1, n_q_heads=1, n_kv_heads=1, seq_len=N, head_dim=d, segment_len=S,
+             block_size=Bk)
+    idx = oracle.build_indices(_cfg(c, 0.5), q, k, debug=True)
+    np.testing.assert_array_equal(idx["perm_k"][0, 0], np.arange(N))
+    np.testing.assert_array_equal(idx["p"][0, 0, 2:], [[0.5, 0.5, 0.0, 0.0]] * 2)
+    np.testing.assert_array_equal(idx["sel_cnt"][0, 0], [0, 0, 2, 2])
+    np.testing.assert_array_equal(idx["sel_blk"][0, 0, 2:, :2], [[0, 1], [0, 1]])
+    above = float(np.nextafter(np.float32(0.5), np.float32(1.0)))
+    idx = oracle.build_indices(_cfg(c, above), q, k)
+    np.testing.assert_array_equal(idx["sel_cnt"][0, 0], [0, 0, 0, 0])
+
+
 # ----------------------------------------------------------------------------- invariants
 
 def test_selection_nested_in_tau_and_sparsity_monotone():
