@@ -133,6 +133,26 @@ def test_index_build_is_deterministic():
         assert torch.equal(getattr(a, name), getattr(b, name))
 
 
+@pytest.mark.parametrize("tau", [0.25, 0.125, float(np.nextafter(np.float32(0.25), np.float32(1)))],
+                         ids=["quarter", "eighth", "above-quarter"])
+def test_scores_equal_to_tau_bit_exact(tau):
+    """Block scores that equal τ exactly (the stop keeps a block with p = τ). Every key is the
+    same vector, so the key scores tie (identity key ordering) and the candidate blocks of
+    segment s (the 4s key blocks before it, 64 visible keys each) share one weight: p = 1/(4s)
+    exactly, 1/4 in segment 1 and 1/8 in segment 2. Indices bit-exact with the oracle and the
+    list lengths of the closed form."""
+    w = W_TINY.replace(tau=tau)
+    N, d = w.seq_len, w.head_dim
+    rng = np.random.default_rng(3)
+    q = torch.from_numpy(rng.standard_normal((1, 1, N, d), dtype=np.float32)).to(torch.bfloat16)
+    k = torch.tensor([1.0, -0.5, 0.25, 2.0] * (d // 4)).repeat(1, 1, N, 1).to(torch.bfloat16)
+    ref = oracle.build_indices(oracle.config(w), q, k)
+    cfg, idx, _ = gpu_indices(w, *to_dev(q, k))
+    assert_indices_equal(idx, ref, cfg.n_blocks)
+    per_segment = {0.25: [0, 4, 0, 0], 0.125: [0, 4, 8, 0]}.get(tau, [0, 0, 0, 0])
+    np.testing.assert_array_equal(ref["sel_cnt"][0, 0], np.repeat(per_segment, 4))
+
+
 # ----------------------------------------------------------------------------- attention
 
 @pytest.mark.parametrize("w", [W_TINY, W_TINY.replace(tau=0.07), W_TINY.replace(tau=1.5), W_A,
