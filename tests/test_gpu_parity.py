@@ -153,6 +153,37 @@ def test_scores_equal_to_tau_bit_exact(tau):
     np.testing.assert_array_equal(ref["sel_cnt"][0, 0], np.repeat(per_segment, 4))
 
 
+@pytest.mark.parametrize("case", ["keys", "query-row"])
+def test_non_finite_inputs_keep_valid_orderings(case):
+    """Non-finite inputs (outside the definition's domain, but the index arrays must stay valid):
+    a NaN score has the smallest sort key, so it goes after every number, ties by lower index.
+    "keys": three NaN key rows and one key with an infinite element; the mean key is NaN, so
+    every query score is NaN and the query ordering is the identity. "query-row": one NaN query
+    row; the pooled query is NaN, so every key score is NaN (identity key ordering) and the row
+    goes last in its segment. The orderings and local tiles are bit-exact with the oracle; the
+    lists (unspecified when a score is not finite) only have to be valid."""
+    w = W_TINY
+    q, k, _ = inputs(w)
+    q, k = q.clone(), k.clone()
+    N, S = w.seq_len, w.segment_len
+    if case == "keys":
+        k[0, 0, [5, 300, 777]] = float("nan")
+        k[0, 0, 901, 3] = float("inf")
+    else:
+        q[0, 0, 700] = float("nan")
+    ref = oracle.build_indices(oracle.config(w), q, k)
+    cfg, idx, ws = gpu_indices(w, *to_dev(q, k))
+    for name in ("perm_q", "perm_k", "local_tiles"):
+        np.testing.assert_array_equal(getattr(idx, name).cpu().numpy(), ref[name], err_msg=name)
+    assert s2o.validate_indices(cfg, idx, ws)
+    if case == "keys":
+        np.testing.assert_array_equal(ref["perm_k"][0, 0, -3:], [5, 300, 777])
+        np.testing.assert_array_equal(ref["perm_q"][0, 0], np.arange(N))
+    else:
+        np.testing.assert_array_equal(ref["perm_k"][0, 0], np.arange(N))
+        assert ref["perm_q"][0, 0, (700 // S + 1) * S - 1] == 700
+
+
 # ----------------------------------------------------------------------------- attention
 
 @pytest.mark.parametrize("w", [W_TINY, W_TINY.replace(tau=0.07), W_TINY.replace(tau=1.5), W_A,
