@@ -7,8 +7,10 @@ header for the passages it follows) through ctypes and builds it with gcc on fir
 Parity status per function (what pins it to something other than itself lives in
 ``tests/test_oracle_pins.py``):
 
-* ``build_indices`` — pinned by the hand-worked case in ``tests/golden/``, by invariants
-  (permutations, sortedness, nesting in τ, Σp = 1) and by float64 re-derivations.
+* ``build_indices`` — pinned by the hand-worked case in ``tests/golden/``, by the hand-derived
+  summation-order case, by a closed-form stop at p = τ (identical keys give p = 1/2 exactly), by
+  invariants (permutations, sortedness, nesting in τ, Σp = 1) and by float64 re-derivations;
+  ``tests/test_oracle_mutations.py`` checks that these pins reject planted mistakes.
 * ``attention`` — pinned by torch's causal scaled-dot-product attention at τ = 0, by per-segment
   causal attention at τ > 1, and by permutation invariance.
 * ``dense_causal`` — pinned by torch's causal scaled-dot-product attention.
