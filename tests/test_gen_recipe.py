@@ -65,7 +65,7 @@ def test_rounding_ties_go_to_even():
     lo = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8)], np.float32)
     want = torch.from_numpy(lo).to(torch.bfloat16).float().numpy()
     np.testing.assert_array_equal(want, [1.0, 1.0 + 2.0 ** -6, -1.0])
-    # gen's rounding of the same values (through a one-element slab of its own conversion path).
+    # gen's own conversion of the same values.
     got = torch.from_numpy(gen._to_bf16_bits(lo.copy()).view(np.int16)).view(torch.bfloat16)
     np.testing.assert_array_equal(got.float().numpy(), want)
 
