@@ -21,7 +21,8 @@ Parity status per function (what pins it to something other than itself lives in
   consequences (stopping never adds a block; lists stay prefixes).
 * ``layer.layer`` (the decoder layer around the attention, ``oracle/layer.py``) — pinned in
   ``tests/test_layer_oracle_pins.py`` (bf16 rounding against torch, closed-form norms, rotary
-  invariants, the frequency scaling's regimes, the silu identity, zero projections = identity).
+  invariants, the frequency scaling's regimes, the silu identity, zero projections = identity,
+  and transformers' Llama decoder layer and rotary table on the same weights).
 """
 from __future__ import annotations
 

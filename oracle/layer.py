@@ -11,8 +11,12 @@ the attention is this package's oracle (``attention`` / ``dense_causal``) on the
 
 Parity pins (``tests/test_layer_oracle_pins.py``): RMS norm of constant rows, the rotation's
 norm preservation, identity at position 0 and relative-position property, the frequency table
-against the scaling's three regimes, silu at known points, bf16 rounding against torch, and the
-whole layer with zero projections (the residual passes through unchanged).
+against the scaling's three regimes and against transformers' "llama3" rotary table, silu at
+known points, bf16 rounding against torch, the whole layer with zero projections (the residual
+passes through unchanged), and the whole layer against transformers' Llama decoder layer in
+float64 on the same weights (within a few bf16 ulps: the oracle rounds to bf16 where the GPU
+stores bf16, the library does not). ``tests/test_layer_oracle_mutations.py`` checks that these
+pins reject planted mistakes.
 """
 from __future__ import annotations
 

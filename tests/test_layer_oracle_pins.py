@@ -1,11 +1,15 @@
 """Pins of the decoder-layer oracle (``oracle/layer.py``) to facts other than itself: bf16
 rounding against torch's conversion, RMS norm on rows with a closed form, the rotary embedding's
 identity at position 0, norm preservation and relative-position property, the frequency scaling's
-regimes and continuity, the silu identity silu(z) − silu(−z) = z, and the whole layer with zero
-projections (the residual stream passes through unchanged)."""
+regimes and continuity, the silu identity silu(z) − silu(−z) = z, the whole layer with zero
+projections (the residual stream passes through unchanged), and, as a library the layer reduces
+to, transformers' Llama decoder layer and its "llama3" rotary table run on the same weights
+(test_layer_oracle_mutations.py plants mistakes in copies of the layer oracle and checks that
+these pins reject each)."""
 import math
 
 import numpy as np
+import pytest
 import torch
 
 import gen
@@ -127,3 +131,68 @@ def test_layer_inputs_are_seeded_and_thread_independent():
     # projection scale N(0, 1/fan_in), norm gains around 1
     assert abs(float(a["w_gu"].float().std()) * math.sqrt(128) - 1) < 0.05
     assert abs(float(a["attn_norm"].float().mean()) - 1) < 0.05
+
+
+# ----------------------------------------------------------------------------- against a library
+
+def _hf_layer(w, shape, wts):
+    """The same layer in transformers' own Llama implementation (float64, eager attention with a
+    causal mask), with the random weights moved into its parameter layout (x·W here, x·Wᵀ
+    there). Returns (output rows [N, H], the rotary table's inverse frequencies)."""
+    tr = pytest.importorskip("transformers")
+    from transformers.models.llama import modeling_llama as ml
+    Hq, Hkv, d, N, I = w.n_q_heads, w.n_kv_heads, w.head_dim, w.seq_len, shape.intermediate
+    H = Hq * d
+    cfg = tr.LlamaConfig(
+        hidden_size=H, num_attention_heads=Hq, num_key_value_heads=Hkv, head_dim=d,
+        intermediate_size=I, rms_norm_eps=shape.rms_eps, max_position_embeddings=131072,
+        rope_theta=shape.rope_theta, attention_bias=False, mlp_bias=False,
+        rope_scaling={"rope_type": "llama3", "factor": shape.rope_factor,
+                      "low_freq_factor": shape.rope_low_freq_factor,
+                      "high_freq_factor": shape.rope_high_freq_factor,
+                      "original_max_position_embeddings": shape.rope_original_context})
+    cfg._attn_implementation = "eager"
+    W = {k: torch.from_numpy(L.bf16_value(v)) for k, v in wts.items()}
+    layer = ml.LlamaDecoderLayer(cfg, layer_idx=0).double()
+    rot = ml.LlamaRotaryEmbedding(cfg)
+    with torch.no_grad():
+        a = layer.self_attn
+        a.q_proj.weight.copy_(W["w_qkv"][:, :Hq * d].T)
+        a.k_proj.weight.copy_(W["w_qkv"][:, Hq * d:(Hq + Hkv) * d].T)
+        a.v_proj.weight.copy_(W["w_qkv"][:, (Hq + Hkv) * d:].T)
+        a.o_proj.weight.copy_(W["w_o"].T)
+        layer.mlp.gate_proj.weight.copy_(W["w_gu"][:, :I].T)
+        layer.mlp.up_proj.weight.copy_(W["w_gu"][:, I:].T)
+        layer.mlp.down_proj.weight.copy_(W["w_down"].T)
+        layer.input_layernorm.weight.copy_(W["attn_norm"])
+        layer.post_attention_layernorm.weight.copy_(W["mlp_norm"])
+        x = W["x"].reshape(1, N, H)
+        pos = torch.arange(N)[None]
+        mask = torch.full((N, N), float("-inf"), dtype=torch.float64).triu(1)[None, None]
+        out = layer(x, attention_mask=mask, position_ids=pos, position_embeddings=rot(x, pos))
+    out = out[0] if isinstance(out, tuple) else out
+    return out.numpy().reshape(N, H), rot.inv_freq.double().numpy()
+
+
+HF_W = gen.Workload("layer-pin", 1, 2, 1, 256, 64, 128, 64, 0.0, 4)
+HF_SHAPE = SHAPE.replace(intermediate=128)
+
+
+def test_rope_frequencies_match_transformers_llama3():
+    """The frequency table against transformers' "llama3" rotary scaling (its float32 table)."""
+    _, inv = _hf_layer(HF_W, HF_SHAPE, gen.make_layer(HF_W, HF_SHAPE))
+    np.testing.assert_allclose(L.rope_frequencies(HF_W.head_dim, HF_SHAPE), inv, rtol=1e-6)
+
+
+def test_layer_matches_transformers_llama_decoder_layer():
+    """The whole layer (dense causal attention) against transformers' LlamaDecoderLayer run in
+    float64 on the same bf16 weights and input. The oracle rounds to bf16 at nine points and the
+    library at none, so the two agree to a few bf16 ulps: every element within 4 ulps of bf16 at
+    max(1, |x₂|) (2^-5 relative; measured 2 ulps) and a mean error below 0.005 (measured 0.0031).
+    A swapped operand, a wrong rotation or a dropped term moves the output by 0.4 or more."""
+    wts = gen.make_layer(HF_W, HF_SHAPE)
+    ref, _ = _hf_layer(HF_W, HF_SHAPE, wts)
+    got = L.layer(HF_W, HF_SHAPE, wts, dense=True).reshape(ref.shape)
+    err = np.abs(got - ref)
+    assert np.all(err <= 2.0 ** -5 * np.maximum(1.0, np.abs(ref))), float(err.max())
+    assert err.mean() < 0.005, float(err.mean())
