@@ -1,6 +1,6 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports every function that
 ``include/s2o.h`` declares, sizes its buffers as documented and rejects bad arguments before
-enqueueing any device work."""
+enqueueing any device work; the header compiles in a plain C99 client that links the library."""
 import ctypes
 import os
 import re
@@ -197,3 +197,45 @@ def test_attention_work_rejects_bad_arguments_before_device_work():
                                   None, None) == 1
     assert lib.s2o_attention_work(ctypes.byref(cfg._c()), None, 0x10000, small + 1,
                                   ctypes.byref(out), None) == 1
+
+
+C_CLIENT = r"""
+#include "s2o.h"
+#include <stdio.h>
+
+int main(void) {
+  s2o_config c = {1, 32, 8, 131072, 128, 2048, 128, 0.01f, 1, 0, 0};
+  size_t ws = 0, pws = 0, counts[5], bad = 0;
+  if (s2o_workspace_size(&c, &ws) != S2O_OK) return 1;
+  if (s2o_prefill_workspace_size(&c, &pws) != S2O_OK) return 2;
+  if (s2o_index_sizes(&c, counts) != S2O_OK) return 3;
+  c.head_dim = 96;
+  if (s2o_workspace_size(&c, &bad) != S2O_ERR_UNSUPPORTED) return 4;
+  printf("%zu %zu %zu %zu %zu %zu %zu %s %u\n", ws, pws, counts[0], counts[1], counts[2],
+         counts[3], counts[4], s2o_status_string(S2O_ERR_UNSUPPORTED),
+         (unsigned)S2O_STATIC_WORKSPACE_BYTES);
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C99 client (no C++, no torch) includes the header with warnings as errors, links the
+    in-tree library and makes host-only calls; it sees the sizes the binding sees."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(s2o.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                    "-L", libdir, "-l:" + os.path.basename(s2o.library_path()),
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    cfg = LLAMA_128K
+    want = [s2o.workspace_size(cfg), s2o.prefill_workspace_size(cfg), *s2o.index_sizes(cfg)]
+    assert [int(x) for x in out[:7]] == want
+    assert out[7] == "S2O_ERR_UNSUPPORTED" and int(out[8]) == s2o.STATIC_WORKSPACE_BYTES
