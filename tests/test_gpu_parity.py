@@ -525,10 +525,11 @@ STOP_TOL = 0.05  # relative band around τ inside which the GPU and the oracle m
 @pytest.mark.parametrize("w,tau", [(W_OS1, 0.03), (W_OS1, 0.08), (W_OS2, 0.02), (W_OS2, 0.03)],
                          ids=["os1-0.03", "os1-0.08", "os2-0.02", "os2-0.03"])
 def test_online_stop_matches_oracle(w, tau):
-    """The measured-share stop (DEFINITION D13) on the oracle's full candidate lists: every GPU
-    stop position agrees with the oracle's shares (blocks the GPU went past have an oracle share of
-    at least τ·(1 − 5 %), the block it stopped after one below τ·(1 + 5 %)), the stops actually cut
-    lists, and the output equals the oracle's attention over the GPU's kept blocks."""
+    """The measured-share stop (the definition's online-stop section) on the oracle's full
+    candidate lists: every GPU stop position agrees with the oracle's shares (blocks the GPU went
+    past have an oracle share of at least τ·(1 − 5 %), the block it stopped after one below
+    τ·(1 + 5 %)), the stops actually cut lists, and the output equals the oracle's attention over
+    the GPU's kept blocks."""
     q, k, v = inputs(w)
     ref = oracle.build_indices(oracle.config(w), q, k)
     ocfg = oracle.config(w, tau=tau)
