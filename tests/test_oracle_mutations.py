@@ -72,6 +72,20 @@ MUTATIONS = {
     "qbar-original-order": (
         "list_mean(Q, d, perm_q + (size_t)b * B, B, B, Qbar + (size_t)b * d);",
         "list_mean(Q, d, ident + (size_t)b * B, B, B, Qbar + (size_t)b * d);"),
+    # 4-bit centroids: codes of the key centroids without the channel's offset.
+    "int4-key-code-no-offset": ("float code = rintf((Kbar[(size_t)c * d + t] - mn) / st);",
+                                "float code = rintf(Kbar[(size_t)c * d + t] / st);"),
+    # 4-bit centroids: the integer product not scaled back by the query step.
+    "int4-query-scale-dropped": ("r[(size_t)b * nB + c] = ((float)acc * sq) * sigma;",
+                                 "r[(size_t)b * nB + c] = ((float)acc) * sigma;"),
+    # 4-bit centroids: sixteen steps over the channel's range instead of fifteen.
+    "int4-sixteen-steps": ("float st = (mx - mn) / 15.0f;", "float st = (mx - mn) / 16.0f;"),
+    # One key ordering per KV head: the pooled query of the head itself, not of its group.
+    "shared-order-own-head": ("for (int hh = g * G; hh < (g + 1) * G; ++hh) {",
+                              "for (int hh = h; hh < h + 1; ++hh) {"),
+    # One key ordering per KV head: the group's mean queries summed, not averaged.
+    "shared-order-sum-not-mean": ("for (int t = 0; t < d; ++t) qsum[t] = qsum[t] / (float)G;",
+                                  "for (int t = 0; t < d; ++t) qsum[t] = qsum[t];"),
 }
 
 # The pins that run against each mutant (all CPU, seconds each).
@@ -90,6 +104,9 @@ PIN_TESTS = [
     pins.test_float64_rederivation_of_pooled_quantities,
     pins.test_sum_order_case_chunked_means,
     pins.test_sum_order_case_normaliser_chunks,
+    pins.test_shared_key_order_variant,
+    pins.test_int4_centroid_variant,
+    pins.test_int4_scores_exact_on_grid_aligned_centroids,
     pins.test_online_stop_hand_case,
     lambda: pins.test_online_stop_against_softmax_probabilities(0.03),
 ]
@@ -116,6 +133,7 @@ def test_pins_reject_planted_mistake(tmp_path, name):
                 pin()
             except (AssertionError, ValueError):
                 caught.append(getattr(pin, "__name__", "lambda"))
+                break  # one rejection is enough
     assert caught, f"no pin caught the planted mistake {name!r}"
 
 

@@ -429,6 +429,32 @@ def test_int4_centroid_variant():
     np.testing.assert_array_equal(np.sort(v0["sel_blk"], axis=-1), np.sort(b0["sel_blk"], axis=-1))
 
 
+def test_int4_scores_exact_on_grid_aligned_centroids():
+    """Closed form of the 4-bit centroid variant: when every key centroid already lies on the
+    variant's 16-level grid and the scaled query maps to one code, the integer product gives the
+    exact centroid score σ·Q̄·(K̄ − lo)ᵀ up to float32 rounding. Keys come in 16 groups of B equal
+    rows (j/16)·e₀ and every query is e₀, so κ_j is the key's first element, each key block of the
+    ordering is one group, the centroids' first channel takes the values j/16 (lo = 0, step
+    (15/16)/15 = 1/16 exactly, codes j), the other channels are zero (code 0), and the query's one
+    non-zero scaled value takes the code 127."""
+    Bk, nB, d = 4, 16, 4
+    N = Bk * nB
+    k = np.zeros((N, d), np.float32)
+    for j in range(nB):
+        k[j * Bk:(j + 1) * Bk, 0] = j / 16
+    q = np.zeros((N, d), np.float32)
+    q[:, 0] = 1.0
+    qt, kt = (torch.from_numpy(a).to(torch.bfloat16).reshape(1, 1, N, d) for a in (q, k))
+    cfg = oracle.Config(1, 1, 1, N, d, 16, Bk, 0.01, 1, 0, 1)
+    idx = oracle.build_indices(cfg, qt, kt, debug=True)
+    Kbar, Qbar = idx["Kbar"][0, 0].astype(np.float64), idx["Qbar"][0, 0].astype(np.float64)
+    np.testing.assert_array_equal(Kbar[:, 0], (15 - np.arange(nB)) / 16)
+    np.testing.assert_array_equal(Kbar[:, 1:], 0.0)
+    np.testing.assert_array_equal(Qbar, np.tile([1.0, 0, 0, 0], (nB, 1)))
+    exact = 0.5 * Qbar[:, :1] @ Kbar[:, :1].T  # σ = 1/√4, lo = 0
+    np.testing.assert_allclose(idx["r"][0, 0], exact, rtol=1e-6, atol=0)
+
+
 # ----------------------------------------------------------------------------- summation orders
 
 SUM_ORDER = os.path.join(os.path.dirname(__file__), "golden", "sum_order_case.json")
