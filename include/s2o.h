@@ -13,9 +13,13 @@
  * ---------------------------------------
  *  - Tensors are bf16, contiguous, BHND: Q and O [batch, Hq, N, d]; K and V [batch, Hkv, N, d].
  *    Query head h reads key/value head h / (Hq/Hkv).
- *  - Every pointer except `cfg`, size outputs and `s2o_stats*` is a DEVICE pointer owned by the
- *    caller, 16-byte aligned. The library never allocates device memory: scratch comes from the
- *    caller's workspace `ws` (size from s2o_workspace_size).
+ *  - Tensor, index-array and workspace pointers are DEVICE pointers owned by the caller, 16-byte
+ *    aligned. The structs passed by pointer (s2o_config, s2o_indices, s2o_layer_config,
+ *    s2o_layer_weights) and the outputs s2o_stats, s2o_work_counts, s2o_workspace_view and the
+ *    size outputs live in HOST memory (s2o_indices, s2o_layer_weights and s2o_workspace_view hold
+ *    device pointers). The library never allocates device memory: scratch comes from the
+ *    caller's workspace `ws` (size from s2o_workspace_size), except in
+ *    s2o_build_indices_static.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Launching calls are
  *    asynchronous on it; argument errors are returned before anything is enqueued, and device
  *    faults surface at the caller's next synchronisation (CUDA convention).
