@@ -278,13 +278,17 @@ def run_s2o(args):
     ws = s2o.alloc_prefill_workspace(cfg, dev)
     stream = torch.cuda.current_stream(dev)
 
+    nvtx = torch.cuda.nvtx  # named ranges for a timeline profiler; no-ops without one
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
+        with nvtx.range("s2o index build"):
+            s2o.build_indices(cfg, qd, kd, out=idx, ws=ws)
         if ev is not None:
             ev[1].record(stream)
-        s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws, out=o)
+        with nvtx.range("s2o attention"):
+            s2o.attention_prefill_with_indices_ws(cfg, qd, kd, vd, idx, ws, out=o)
         if ev is not None:
             ev[2].record(stream)
 
