@@ -72,6 +72,16 @@ MUTATIONS = {
     "qbar-original-order": (
         "list_mean(Q, d, perm_q + (size_t)b * B, B, B, Qbar + (size_t)b * d);",
         "list_mean(Q, d, ident + (size_t)b * B, B, B, Qbar + (size_t)b * d);"),
+    # Attention logits without the 1/sqrt(d) scale.
+    "attention-no-scale": ("    z[a] = acc * inv_sqrt_d;\n    if (z[a] > m) m = z[a];",
+                           "    z[a] = acc;\n    if (z[a] > m) m = z[a];"),
+    # Attention output not divided by the softmax normaliser.
+    "attention-unnormalised": ("  for (int t = 0; t < d; ++t) out[t] /= den;", ""),
+    # Attention weights applied to the keys instead of the values.
+    "attention-values-from-keys": ("const uint16_t *vj = V + (size_t)keys[a] * d;",
+                                   "const uint16_t *vj = K + (size_t)keys[a] * d;"),
+    # Dense causal attention without the 1/sqrt(d) scale.
+    "dense-no-scale": ("        z[j] = acc * inv_sqrt_d;", "        z[j] = acc;"),
     # 4-bit centroids: codes of the key centroids without the channel's offset.
     "int4-key-code-no-offset": ("float code = rintf((Kbar[(size_t)c * d + t] - mn) / st);",
                                 "float code = rintf(Kbar[(size_t)c * d + t] / st);"),
